@@ -1,0 +1,431 @@
+"""Benchmark of the sparse-attention decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lsa|reference] [--index bf16|fp8]
+
+One step = the whole hot path over one batch: lightning-indexer scores -> top-K (+sink/window) ->
+sparse MLA gather-attention, for the 16-query decode batch over L = 131072 cached tokens
+(K = 2048, H_I = 64, d_I = 128, 128 heads, 576/512 bf16 latent).  Inputs are seeded synthetic
+tensors (lsa_synth) resident in HBM before timing; L2 is flushed (256 MB write) before every step,
+outside the per-step CUDA events.  Rank 0 prints one JSON line.
+
+N > 1 (torchrun): every rank runs an independent replica of the same decode batch (the path has no
+exchange step on one node here: replicas only), timed per rank, max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import threading
+import time
+
+import numpy as np
+import torch
+
+import lsa_synth as S
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+CONFIG = "decode128k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ------------------------------------------------------------------------------------------------
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+                if out.returncode == 0 and out.stdout.strip():
+                    self.samples.append([x.strip() for x in out.stdout.strip().split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if len(s) > 5 + i and s[5 + i] == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------------
+# the GPU arm
+# ------------------------------------------------------------------------------------------------
+
+
+class DecodeStep:
+    """Resident tensors and the three C-ABI calls of one decode step."""
+
+    def __init__(self, wl: S.Workload, index_dtype: str, device):
+        import sparse_long_context_lightning_b200 as lsa
+
+        self.lsa = lsa
+        self.wl = wl
+        self.fp8 = index_dtype == "fp8"
+        q_I, w = S.index_queries(wl, "cpu")
+        k_I = S.index_keys(wl, q_I, device)
+        self.q_I, self.w = q_I.to(device), w.to(device)
+        if self.fp8:
+            self.q_in, self.q_scale = S.quantize_e4m3_rows(self.q_I)
+            self.k_in, self.k_scale = S.quantize_e4m3_rows(k_I)
+            del k_I
+        else:
+            self.q_in, self.q_scale, self.k_in, self.k_scale = self.q_I, None, k_I, None
+        self.q_pos = wl.q_pos().to(device)
+        self.q = S.attn_queries(wl, device)
+        self.kv = S.latent_cache(wl, device)
+        B, L = wl.B, wl.L
+        self.kmax = wl.K + wl.sink + wl.window
+        self.scores = torch.empty(B, L, device=device)
+        self.idx = torch.empty(B, self.kmax, dtype=torch.int32, device=device)
+        self.cnt = torch.empty(B, dtype=torch.int32, device=device)
+        self.out = torch.empty(B, wl.H, wl.d_v, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(B, wl.H, device=device)
+        self.ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_ATTN, B, L, self.kmax, wl.H), device)
+
+    def index(self):
+        self.lsa.lsa_index_score(self.q_in, self.w, self.k_in, self.q_pos, self.scores,
+                                 q_scale=self.q_scale, k_scale=self.k_scale)
+
+    def topk(self):
+        wl = self.wl
+        self.lsa.lsa_topk_select(self.scores, wl.L, wl.K, wl.sink, wl.window, self.q_pos, self.idx, self.cnt)
+
+    def attn(self):
+        self.lsa.lsa_sparse_attn(self.q, self.kv, self.idx, self.cnt, self.wl.scale, self.out, self.lse, self.ws)
+
+
+def algorithmic_work(wl: S.Workload, counts: np.ndarray, fp8: bool):
+    """Bytes / flops each stage must touch (what the method reads and writes, nothing re-read)."""
+    B, L = wl.B, wl.L
+    vis = L  # decode: every cached key is visible
+    idx_elem = 1 if fp8 else 2
+    index_flops = 2.0 * B * wl.H_I * wl.d_I * vis
+    index_bytes = vis * wl.d_I * idx_elem + (vis * 4 if fp8 else 0) + B * vis * 4 + B * wl.H_I * (wl.d_I * idx_elem + 4)
+    topk_bytes = B * vis * 4 + B * (wl.K + wl.sink + wl.window) * 4
+    n_rows = float(counts.sum())
+    attn_bytes = n_rows * wl.d_qk * 2 + B * wl.H * wl.d_qk * 2 + B * wl.H * wl.d_v * 2 + B * wl.H * 4 + n_rows * 4
+    attn_flops = 2.0 * n_rows * wl.H * (wl.d_qk + wl.d_v)
+    return {"index": (index_flops, index_bytes), "topk": (0.0, topk_bytes), "attn": (attn_flops, attn_bytes)}
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        p = os.path.join(ROOT, "sparse_long_context_lightning_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d:
+        return None
+    if d.get("source_hash") != kernel_source_hash(d.get("sources", [])):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+STAGE_KERNEL = {"index": ("k_index_score", ["k_index_tc.cu", "k_score_simt.cu"]),
+                "topk": ("k_topk_cluster", ["k_topk.cu"]),
+                "attn": ("k_sparse_attn", ["k_attn_tc.cu", "k_attn_simt.cu"])}
+# kernels each stage launches per step (the e2e leg adds none of ours)
+LAUNCHES = {"index": 1, "topk": 1, "attn": 1}
+
+
+def run_gpu(args, rank, world, local_rank):
+    import sparse_long_context_lightning_b200 as lsa
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    wl = S.WORKLOADS[CONFIG]
+    step = DecodeStep(wl, args.index, device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    launches = dict(LAUNCHES)
+    if hasattr(lsa, "attn_launches_per_call"):
+        launches["attn"] = lsa.attn_launches_per_call()
+
+    def one_step(ev):
+        ev[0].record(stream)
+        step.index()
+        ev[1].record(stream)
+        step.topk()
+        ev[2].record(stream)
+        step.attn()
+        ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        one_step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    torch.cuda.synchronize()
+    counts = step.cnt.cpu().numpy()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0) as clk:
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()  # L2 flush, outside the step's events
+            one_step(evs[i])
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+    if world > 1:
+        torch.distributed.barrier()
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(args.steps)])  # ms
+    step_ms = float(per.sum(axis=1).mean())
+    stage_ms = per.mean(axis=0)
+
+    # e2e: host (pinned) inputs -> H2D -> the three calls -> D2H of the result, every step
+    h_q_in = step.q_in.cpu().pin_memory()
+    h_w = step.w.cpu().pin_memory()
+    h_qs = step.q_scale.cpu().pin_memory() if step.q_scale is not None else None
+    h_q = step.q.cpu().pin_memory()
+    h_qpos = step.q_pos.cpu().pin_memory()
+    h_out = torch.empty_like(step.out, device="cpu").pin_memory()
+    h_lse = torch.empty_like(step.lse, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q_in, h_w, h_q, h_qpos) + ((h_qs,) if h_qs is not None else ()))
+    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step.q_in.copy_(h_q_in, non_blocking=True)
+        step.w.copy_(h_w, non_blocking=True)
+        if h_qs is not None:
+            step.q_scale.copy_(h_qs, non_blocking=True)
+        step.q.copy_(h_q, non_blocking=True)
+        step.q_pos.copy_(h_qpos, non_blocking=True)
+        step.index()
+        step.topk()
+        step.attn()
+        h_out.copy_(step.out, non_blocking=True)
+        h_lse.copy_(step.lse, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_step = float(np.mean(e2e_ms))
+
+    # max over ranks
+    vals = torch.tensor([step_ms, e2e_step, *stage_ms.tolist()], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    step_ms, e2e_step = float(vals[0]), float(vals[1])
+    stage_ms = vals[2:].cpu().numpy()
+    if rank != 0:
+        return None
+
+    pk, pk_src = peaks()
+    work = algorithmic_work(wl, counts, step.fp8)
+    tensor_peak = pk["bf16_tflops"] * (FP8_OVER_BF16 if step.fp8 else 1.0)
+    stages = {}
+    for j, name in enumerate(("index", "topk", "attn")):
+        flops, nbytes = work[name]
+        t = stage_ms[j] * 1e-3
+        gbs = nbytes / t / 1e9
+        st = {"ms": round(float(stage_ms[j]), 5), "algorithmic_bytes": int(nbytes), "achieved_gbs": round(gbs, 1),
+              "hbm_frac": round(gbs / pk["hbm_gbs"], 4)}
+        if flops:
+            tf = flops / t / 1e12
+            st.update({"algorithmic_flops": flops, "achieved_tflops": round(tf, 2),
+                       "tensor_frac": round(tf / tensor_peak, 4)})
+        stages[name] = st
+    dom = max(stages, key=lambda k: stages[k]["ms"])
+    kname, _ = STAGE_KERNEL[dom]
+    if dom == "index":
+        roof = {"bound": "tensor", "achieved": stages[dom]["achieved_tflops"], "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": stages[dom]["tensor_frac"]}
+    else:
+        roof = {"bound": "hbm", "achieved": stages[dom]["achieved_gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": stages[dom]["hbm_frac"]}
+    roof.update({"kernel": kname, "peak_source": pk_src + (" (bf16 x2 nominal ratio)" if dom == "index" and step.fp8 else ""),
+                 "traffic": committed_traffic(kname)})
+    qps = wl.B * world / (step_ms * 1e-3)
+    n_launch = sum(launches.values()) * args.steps
+    return {
+        "metric": "sparse decode queries/s @L=128K,K=2048",
+        "value": round(qps, 1),
+        "unit": "queries/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if not step.fp8 else "e4m3-index/bf16-attn",
+        "data": "synthetic (lsa_synth, seed 0)",
+        "config": {"workload": f"{CONFIG}: B=16 decode queries, L=131072, H_I=64, d_I=128, K=2048, H=128, "
+                               f"latent 576/512 bf16", "index_dtype": args.index, "global_batch": wl.B * world,
+                   "seq_len": wl.L, "parallelism": f"replicas x{world}",
+                   "l2": "flushed (256 MB write) before every step, outside the step's CUDA events"},
+        "gather_hbm_gbs": stages["attn"]["achieved_gbs"],
+        "stages": stages,
+        "roofline": roof,
+        "e2e": {"value": round(wl.B * world / (e2e_step * 1e-3), 1), "unit": "queries/s",
+                "ms_per_step": round(e2e_step, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": n_launch,
+        "clocks": clk.summary(),
+        "wall_s_timed_region": round(wall, 4),
+    }
+
+
+# ------------------------------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline, and the --impl reference arm)
+# ------------------------------------------------------------------------------------------------
+
+
+def oracle_queries(budget_s: float, max_queries: int = 1000):
+    """Run the fp64 oracle on decode queries of the same workload until budget_s elapses.
+
+    Per query: indexer scores over all 131072 keys, top-K + union, attention over the selected
+    latent rows (gathered from the same synthetic cache).  Returns (queries, seconds, threads).
+    """
+    from oracle import lsa_oracle as O
+
+    wl = S.WORKLOADS[CONFIG]
+    q_I, w = S.index_queries(wl)
+    k_I = S.index_keys(wl, q_I)
+    kf = O.bf16_to_f64(k_I.view(torch.int16).numpy())
+    qf = O.bf16_to_f64(q_I.view(torch.int16).numpy())
+    wf = w.numpy().astype(np.float64)
+    q = S.attn_queries(wl)
+    done, t0 = 0, time.perf_counter()
+    while done < max_queries:
+        b = done % wl.B
+        sc = O.index_score(qf[b: b + 1], wf[b: b + 1], kf, np.array([wl.L - 1]))
+        sel, _, _ = O.topk_row(sc[0], wl.L - 1, wl.K, wl.sink, wl.window)
+        rows = S.latent_rows(wl, torch.as_tensor(sel))
+        O.sparse_mla_attn(O.bf16_to_f64(q[b].view(torch.int16).numpy()), O.bf16_to_f64(rows.view(torch.int16).numpy()),
+                          wl.scale)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done, dt, torch.get_num_threads()
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    # warm-up steps are untimed oracle queries; each timed step is one bounded sample (<= 2 queries)
+    for _ in range(min(args.warmup, 1)):
+        oracle_queries(0.0, 1)
+    qs, secs = 0, 0.0
+    for _ in range(args.steps):
+        n, dt, _ = oracle_queries(5.0, 2)
+        qs += n
+        secs += dt
+    v = qs / secs
+    cores = blas_threads()
+    return {"metric": "sparse decode queries/s @L=128K,K=2048", "value": round(v, 4), "unit": "queries/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (lsa_synth, seed 0)", "impl": "reference",
+            "config": {"workload": f"{CONFIG}: B=16 decode queries, L=131072, H_I=64, d_I=128, K=2048, H=128, "
+                                   f"latent 576/512 bf16", "sample": "<= 2 decode queries per step"},
+            "cpu_baseline": {"value": round(v, 4), "unit": "queries/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{qs} decode queries of the workload (full indexer over L, top-K, attention)"},
+            "e2e": {"value": round(v, 4), "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lsa", choices=["lsa", "reference"])
+    ap.add_argument("--index", default="bf16", choices=["bf16", "fp8"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    res = run_gpu(args, rank, world, local_rank)
+    if res is not None:
+        if not args.no_cpu_baseline and world == 1:
+            n, dt, _ = oracle_queries(12.0)
+            res["cpu_baseline"] = {"value": round(n / dt, 4), "unit": "queries/s", "cores": blas_threads(),
+                                   "kind": "oracle", "sample": f"{n} decode queries of the workload "
+                                                                f"(fp64 indexer over L=131072, top-K, attention)"}
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,184 @@
+/*
+ * lsa.h -- C ABI of the token-level sparse-attention hot path on B200 (sm_100a).
+ *
+ * One long-context attention layer, three stages:
+ *   1. lightning-indexer scores        lsa_index_score
+ *   2. per-query selection             lsa_topk_select   (top-K + sink/window union)
+ *                                      lsa_bucket_select (Flat buckets / 4-token micro-blocks)
+ *                                      lsa_pool_keys     (bucket representatives, cached once)
+ *   3. sparse attention over the gathered MLA latent rows   lsa_sparse_attn
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library keeps
+ *     no pointer after the call returns.  Row-major layouts; "[B, H]" means B rows of H.
+ *   - Positions are 0-based.  q_pos[b] (device int64) is the position of query b; it
+ *     sees the keys s in [0, q_pos[b]] (decode: q_pos = L - 1; causal prefill: q_pos = t).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Every
+ *     call only enqueues work on that stream: nothing synchronises with the host.
+ *   - Scratch memory ("ws") is caller-allocated device memory of at least
+ *     lsa_workspace_size(...) bytes, 256-byte aligned.  Contents need no initialisation.
+ *   - Return value: LSA_OK (0) or a negative lsa_status.  Arguments are validated
+ *     before anything is launched; a failed check launches nothing.  A launch failure
+ *     returns LSA_ERR_CUDA (the CUDA error string is kept for lsa_last_error()).
+ *     Nothing throws across this ABI.
+ *   - All calls are deterministic: the same inputs give the same bytes.
+ */
+#ifndef LSA_H_
+#define LSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LSA_OK = 0,
+  LSA_ERR_INVALID_ARG = -1,  /* a pointer, size or parameter is out of range        */
+  LSA_ERR_UNSUPPORTED = -2,  /* valid request this build does not handle (e.g. dims) */
+  LSA_ERR_WORKSPACE = -3,    /* ws is NULL, misaligned or smaller than required      */
+  LSA_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed                    */
+  LSA_ERR_DEVICE_CHECK = -5, /* a device-side check recorded a bad index              */
+  LSA_ERR_TIMEOUT = -6       /* a bounded device-side wait gave up                    */
+} lsa_status;
+
+typedef enum {
+  LSA_BF16 = 0,     /* bfloat16 elements                                            */
+  LSA_FP8_E4M3 = 1  /* OCP e4m3fn codes with one fp32 scale per row (value = code*scale) */
+} lsa_dtype;
+
+typedef enum { LSA_OP_TOPK = 1, LSA_OP_BUCKET = 2, LSA_OP_ATTN = 3 } lsa_op;
+
+/*
+ * lsa_index_score -- lightning-indexer scores.
+ *   Source: "LongCat Sparse Attention（LSA）完全拆解", section "DSA 基线：闪电索引器是怎么工作的",
+ *   equation I_{t,s} = sum_{j<H_I} w_{t,j} * ReLU(q^I_{t,j} . k^I_s): H_I index heads share one
+ *   MQA index key k^I_s, ReLU instead of softmax, FP8-capable.
+ *
+ *   scores[b*ld + s] = sum_j w[b,j] * max(0, q[b,j,:] . k[s,:])   for s <= q_pos[b]
+ *                    = -inf                                        for q_pos[b] < s < L
+ *   q_idx   [B, H_I, d_I]  bf16, or e4m3 codes with q_scale [B, H_I] fp32 (value = code*scale)
+ *   w       [B, H_I]       fp32 head weights
+ *   k_idx   [L, d_I]       bf16, or e4m3 codes with k_scale [L] fp32
+ *   q_scale, k_scale       must be NULL for LSA_BF16 and non-NULL for LSA_FP8_E4M3
+ *   scores  [B, ld]        fp32, ld >= L; entries s >= L are not touched
+ *   Supported: d_I in {32, 64, 128}; H_I in [1, 64] with H_I*d_I <= 8192 (bf16);
+ *   FP8 needs d_I multiple of 32.  q_idx/k_idx 16-byte aligned, scores 16-byte aligned,
+ *   ld a multiple of 4.  Accumulation is fp32 (products of bf16/e4m3 are exact in fp32).
+ */
+int lsa_index_score(const void* q_idx, const float* q_scale, const float* w,
+                    const void* k_idx, const float* k_scale, int dtype,
+                    int64_t B, int H_I, int d_I, int64_t L, const int64_t* q_pos,
+                    float* scores, int64_t ld, void* stream);
+
+/*
+ * lsa_topk_select -- per-query top-K, unioned with attention-sink and sliding-window positions.
+ *   Source: same page, S_t = arg topK({I_{t,s}}_{s<=t}, K) (section "DSA 基线"), and section
+ *   "机制一：流式感知索引（SI）/ 预算分解": S_t = S_sink u S_swa u S_sparse, S_sink = the first
+ *   K_sink positions, S_swa = {t-K_swa+1 .. t}, S_sparse = arg topK over s outside S_sink u S_swa.
+ *
+ *   For each query b (visible keys [0, q_pos[b]], q_pos[b] < L):
+ *     sink   = {0 .. min(sink, q_pos+1)-1}
+ *     window = {max(0, q_pos-window+1) .. q_pos} minus sink
+ *     cand   = visible positions outside sink u window
+ *     sparse = the min(K, |cand|) candidates with the largest scores; equal scores are
+ *              ordered by ascending position (exact: fp32 bit patterns are compared)
+ *   idx[b*idx_ld + i], i < count[b]: the union, ascending (sink, then sparse, then window);
+ *   idx[b*idx_ld + i] = -1 for count[b] <= i < min(idx_ld, K+sink+window).
+ *   scores [B, ld] fp32 (16-byte aligned, ld % 4 == 0); idx int32 [B, idx_ld] with
+ *   idx_ld >= K + sink + window; count int32 [B].  K >= 1, sink >= 0, window >= 0, L < 2^31.
+ *   Needs no scratch memory.
+ */
+int lsa_topk_select(const float* scores, int64_t ld, int64_t B, int64_t L, int K,
+                    int sink, int window, const int64_t* q_pos,
+                    int32_t* idx, int64_t idx_ld, int32_t* count, void* stream);
+
+/*
+ * lsa_pool_keys -- bucket / micro-block representatives (computed once per sequence, cached).
+ *   Source: "LongCat Sparse Attention（LSA）完全拆解", section "机制三：层级索引（HI）" (mean of the
+ *   sub-block's index keys, computed once and cached); lecture "从两本账看懂长上下文注意力", section
+ *   "Qwen Sparse Attention" (index keys mean-pooled in 4-token micro-blocks); "LSA 稀疏注意力會省顯存嗎",
+ *   section 二 step 2 (each bucket keeps a representative vector and its member positions).
+ *
+ *   centroids[c, :] = (1/bsz) * sum_{i<bsz} k[m(c,i), :]  in fp32, members summed in order
+ *   m(c,i) = members[c*bsz + i]   (explicit buckets; every entry in [0, L))
+ *          = c*bsz + i            (members == NULL: contiguous micro-blocks; NB <= L/bsz)
+ *   k_idx [L, d_I] bf16, or e4m3 codes with k_scale [L] (value = code*scale).
+ *   centroids [NB, d_I] fp32.  1 <= bsz <= 1024, d_I % 4 == 0.
+ */
+int lsa_pool_keys(const void* k_idx, int dtype, const float* k_scale, int64_t L, int d_I,
+                  const int32_t* members, int bsz, int64_t NB, float* centroids, void* stream);
+
+/*
+ * lsa_bucket_select -- Flat bucket or micro-block selection.
+ *   Source: "LSA 稀疏注意力會省顯存嗎", section 二 steps 2-4 (Flat compares the bucket
+ *   representatives, expands the kept buckets to member positions, adds sink and window);
+ *   lecture "从两本账看懂长上下文注意力", sections "Qwen Sparse Attention" and "尾部计数与 query 自身"
+ *   (complete micro-blocks are ranked; visible tokens of the incomplete tail block are read
+ *   directly); the representative score uses the indexer formula of lsa_index_score.
+ *
+ *   For each query b:
+ *     bscore[c] = sum_j w[b,j] * max(0, q[b,j,:] . centroids[c,:])   (fp32 centroids)
+ *     ranked    = all NB buckets (members != NULL), or the complete visible micro-blocks
+ *                 c < min(NB, (q_pos+1)/bsz) (members == NULL)
+ *     kept      = the M ranked buckets with the largest bscore (ties -> lower bucket id)
+ *     idx row   = sorted, de-duplicated union of the kept buckets' positions, the tail
+ *                 {bsz*floor((q_pos+1)/bsz) .. q_pos} (micro-block mode only), sink and
+ *                 window, restricted to [0, q_pos]; -1 padded up to idx_ld.
+ *   q_idx [B, H_I, d_I] bf16 (dtype must be LSA_BF16), w [B, H_I] fp32, centroids [NB, d_I]
+ *   fp32, members int32 [NB, bsz] or NULL.  idx int32 [B, idx_ld] with
+ *   idx_ld >= M*bsz + (bsz-1) + sink + window; count int32 [B].
+ *   1 <= M <= 1024, M*bsz + bsz + sink + window <= 8192.
+ *   ws: lsa_workspace_size(LSA_OP_BUCKET, B, NB, M, 0, 0, 0) bytes.
+ */
+int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, int dtype,
+                      int64_t B, int H_I, int d_I, const float* centroids, int64_t NB,
+                      const int32_t* members, int bsz, int M, int sink, int window, int64_t L,
+                      const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * lsa_sparse_attn -- sparse attention over the gathered MLA latent rows (absorbed MQA).
+ *   Source: "LongCat Sparse Attention（LSA）完全拆解", section "DSA 基线", u_t = Attn(h_t, {c_s |
+ *   s in S_t}) with c_s the MLA latent shared by every query head; the 1152-byte bf16 latent row
+ *   (section "瓶颈一"); "LSA 稀疏注意力會省顯存嗎", section 四 (scores q.k scaled, softmax, weighted V).
+ *
+ *   For each query b and head h, with S = {idx[b*idx_ld + i] : i < count[b]}:
+ *     z_s      = scale * q[b,h,:] . kv[s, 0:d_qk]
+ *     out[b,h] = sum_s softmax(z)_s * kv[s, 0:d_v]          (bf16, fp32 accumulation)
+ *     lse[b,h] = log sum_s exp(z_s)                          (natural log; -inf if S empty)
+ *   An empty set gives out = 0.  Entries of idx must lie in [0, L); the call does not read
+ *   idx past count[b].
+ *   q   [B, H, d_qk] bf16;  kv [L, d_qk] bf16 (row stride d_qk);  out [B, H, d_v] bf16;
+ *   lse [B, H] fp32 or NULL.  Supported: d_qk = 576, d_v = 512, H in {16, 32, 64, 128},
+ *   idx_ld >= max count, max count <= 65536.  q, kv, out 16-byte aligned.
+ *   ws: lsa_workspace_size(LSA_OP_ATTN, B, L, Kmax=idx_ld, H, 0, 0) bytes.
+ */
+int lsa_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                    const int32_t* count, int64_t B, int H, int d_qk, int d_v, float scale,
+                    void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * lsa_workspace_size -- scratch bytes a call needs (0 if none).
+ *   op = LSA_OP_TOPK:   0.
+ *   op = LSA_OP_BUCKET: (B, L=NB, K=M) -> per-query bucket scores and kept-bucket lists.
+ *   op = LSA_OP_ATTN:   (B, L, K=idx_ld, H) -> split-K partial outputs.
+ *   Returns (size_t)-1 for an unknown op or negative sizes.
+ */
+size_t lsa_workspace_size(int op, int64_t B, int64_t L, int K, int H, int sink, int window);
+
+/* lsa_strerror -- static description of a status code (never NULL). */
+const char* lsa_strerror(int status);
+
+/* lsa_last_error -- the last CUDA error message seen by this thread ("" if none). */
+const char* lsa_last_error(void);
+
+/* lsa_version -- library version string. */
+const char* lsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H_ */

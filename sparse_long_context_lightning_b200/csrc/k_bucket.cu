@@ -1,0 +1,170 @@
+// Bucket / micro-block representatives and the expansion of kept buckets to token positions.
+//
+// "LSA 稀疏注意力會省顯存嗎", section 二 steps 2-4: each bucket keeps a representative vector and its
+// member positions; Flat compares representatives, expands the kept buckets and adds sink + window.
+// "LongCat Sparse Attention（LSA）完全拆解", section "机制三：层级索引（HI）": the representative is the
+// mean of the members' index keys, computed once per sequence and cached.
+// Lecture "从两本账看懂长上下文注意力", section "Qwen Sparse Attention" / "尾部计数与 query 自身": 4-token
+// micro-blocks; the visible tokens of the incomplete tail block are added directly.
+#include "lsa_common.cuh"
+
+namespace lsa {
+namespace {
+
+// centroids[c, d] = sum_i k[m(c,i), d] / bsz, one thread per (bucket, 4 dims), members in order.
+template <int DT>
+__global__ void k_pool_keys(const void* __restrict__ kptr, const float* __restrict__ k_scale, int64_t L, int d_I,
+                            const int32_t* __restrict__ members, int bsz, int64_t NB,
+                            float* __restrict__ centroids) {
+  const int groups = d_I / 4;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t c = t / groups;
+  const int g = static_cast<int>(t % groups);
+  if (c >= NB) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = 0; i < bsz; ++i) {
+    int64_t s = members ? static_cast<int64_t>(members[c * bsz + i]) : c * bsz + i;
+    s = s < 0 ? 0 : (s >= L ? L - 1 : s);  // out-of-range members are clamped, never dereferenced
+    float4 v;
+    if (DT == LSA_BF16) {
+      const uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(kptr) + s * d_I + g * 4);
+      v.x = bf16_bits_to_f32(raw.x & 0xFFFFu);
+      v.y = bf16_bits_to_f32(raw.x >> 16);
+      v.z = bf16_bits_to_f32(raw.y & 0xFFFFu);
+      v.w = bf16_bits_to_f32(raw.y >> 16);
+    } else {
+      const uint32_t raw = *reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(kptr) + s * d_I + g * 4);
+      const float sc = k_scale[s];
+      v.x = e4m3_to_f32(raw & 0xFFu) * sc;
+      v.y = e4m3_to_f32((raw >> 8) & 0xFFu) * sc;
+      v.z = e4m3_to_f32((raw >> 16) & 0xFFu) * sc;
+      v.w = e4m3_to_f32(raw >> 24) * sc;
+    }
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  const float n = static_cast<float>(bsz);
+  acc.x /= n;
+  acc.y /= n;
+  acc.z /= n;
+  acc.w /= n;
+  reinterpret_cast<float4*>(centroids + c * d_I)[g] = acc;
+}
+
+constexpr int EX_THREADS = 1024;
+constexpr int EX_MAX = 8192;
+
+// One CTA per query: gather kept buckets' positions + tail + sink + window, bitonic sort, de-dup.
+__global__ void __launch_bounds__(EX_THREADS) k_bucket_expand(
+    const int32_t* __restrict__ kept, int64_t kept_ld, const int32_t* __restrict__ kept_count,
+    const int32_t* __restrict__ members, int bsz, int sink, int window, int tail_block,
+    const int64_t* __restrict__ q_pos, int32_t* __restrict__ idx, int64_t idx_ld,
+    int32_t* __restrict__ count, int kmax) {
+  __shared__ int32_t buf[EX_MAX];
+  __shared__ uint32_t wsum[EX_THREADS / 32];
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int qp = static_cast<int>(q_pos[b]);
+  const int nk = kept_count[b];
+  const int nmem = nk * bsz;
+  const int nsink = min(sink, qp + 1);
+  const int wlo = window > 0 ? max(0, qp - window + 1) : qp + 1;
+  const int nwin = qp + 1 - wlo;
+  const int tlo = tail_block > 0 ? ((qp + 1) / tail_block) * tail_block : qp + 1;
+  const int ntail = qp + 1 - tlo;
+  const int n = nmem + nsink + nwin + ntail;
+  int P = 1;
+  while (P < n) P <<= 1;
+  for (int i = tid; i < P; i += EX_THREADS) {
+    int v = 0x7FFFFFFF;
+    if (i < nmem) {
+      const int c = kept[static_cast<int64_t>(b) * kept_ld + i / bsz];
+      const int s = members ? members[static_cast<int64_t>(c) * bsz + (i % bsz)] : c * bsz + (i % bsz);
+      v = s <= qp ? s : 0x7FFFFFFF;
+    } else if (i < nmem + nsink) {
+      v = i - nmem;
+    } else if (i < nmem + nsink + nwin) {
+      v = wlo + (i - nmem - nsink);
+    } else if (i < n) {
+      v = tlo + (i - nmem - nsink - nwin);
+    }
+    buf[i] = v;
+  }
+  __syncthreads();
+  // bitonic sort, ascending
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < P; i += EX_THREADS) {
+        const int l = i ^ j;
+        if (l > i) {
+          const int x = buf[i], y = buf[l];
+          const bool up = (i & k) == 0;
+          if ((x > y) == up) {
+            buf[i] = y;
+            buf[l] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // de-duplicate with an ordered block scan (each thread owns a contiguous run)
+  const int per = (P + EX_THREADS - 1) / EX_THREADS;
+  const int i0 = tid * per, i1 = min(P, i0 + per);
+  uint32_t mine = 0;
+  for (int i = i0; i < i1; ++i) {
+    const int v = buf[i];
+    mine += (v != 0x7FFFFFFF) && (i == 0 || buf[i - 1] != v);
+  }
+  // exclusive scan of `mine` across the block
+  uint32_t incl = mine;
+  const int lane = tid & 31, warp = tid >> 5;
+  #pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  uint32_t wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += wsum[w];
+  uint32_t o = wbase + incl - mine;
+  int32_t* out = idx + static_cast<int64_t>(b) * idx_ld;
+  for (int i = i0; i < i1; ++i) {
+    const int v = buf[i];
+    if ((v != 0x7FFFFFFF) && (i == 0 || buf[i - 1] != v)) out[o++] = v;
+  }
+  uint32_t total = 0;
+  for (int w = 0; w < EX_THREADS / 32; ++w) total += wsum[w];
+  for (int i = static_cast<int>(total) + tid; i < kmax; i += EX_THREADS) out[i] = -1;
+  if (tid == 0) count[b] = static_cast<int32_t>(total);
+}
+
+}  // namespace
+
+int launch_pool_keys(const void* k, int dtype, const float* k_scale, int64_t L, int d_I, const int32_t* members,
+                     int bsz, int64_t NB, float* centroids, cudaStream_t s) {
+  if (NB == 0) return LSA_OK;
+  const int64_t threads = NB * (d_I / 4);
+  const int bs = 256;
+  const int64_t grid = cdiv(threads, bs);
+  if (dtype == LSA_BF16)
+    k_pool_keys<LSA_BF16><<<static_cast<unsigned>(grid), bs, 0, s>>>(k, k_scale, L, d_I, members, bsz, NB, centroids);
+  else
+    k_pool_keys<LSA_FP8_E4M3><<<static_cast<unsigned>(grid), bs, 0, s>>>(k, k_scale, L, d_I, members, bsz, NB, centroids);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_bucket_expand(const int32_t* kept, int64_t kept_ld, const int32_t* kept_count, const int32_t* members,
+                         int bsz, int sink, int window, int tail_block, const int64_t* q_pos, int64_t B,
+                         int32_t* idx, int64_t idx_ld, int32_t* count, int64_t kmax, cudaStream_t s) {
+  if (B == 0) return LSA_OK;
+  k_bucket_expand<<<static_cast<unsigned>(B), EX_THREADS, 0, s>>>(kept, kept_ld, kept_count, members, bsz, sink,
+                                                                  window, tail_block, q_pos, idx, idx_ld, count,
+                                                                  static_cast<int>(kmax));
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace lsa

@@ -1,0 +1,197 @@
+// C ABI of the library: argument validation, scratch layout, dispatch to the kernels.
+#include <cstdio>
+#include <cstring>
+
+#include "lsa_common.cuh"
+
+namespace lsa {
+
+static thread_local char g_last_error[256] = "";
+
+void set_last_error(const char* msg) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s", msg ? msg : "");
+}
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return LSA_OK;
+  set_last_error(cudaGetErrorString(e));
+  return LSA_ERR_CUDA;
+}
+
+int launch_score_simt(const void* q, const float* q_scale, const float* w, const void* k, const float* k_scale,
+                      int dtype, int64_t B, int H_I, int d_I, int64_t L, const int64_t* q_pos, float* scores,
+                      int64_t ld, cudaStream_t s);
+int launch_topk_mode(const float* scores, int64_t ld, int64_t B, int64_t L, int K, int sink, int window,
+                     const int64_t* q_pos, int mode, int div, int32_t* idx, int64_t idx_ld, int32_t* count,
+                     int64_t kmax, cudaStream_t s);
+int launch_attn_simt(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                     const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, cudaStream_t s);
+
+// Scratch layout of lsa_bucket_select: bucket scores [B, ld_nb] fp32 | kept [B, M] int32 | kept_count [B] int32
+static void bucket_ws_layout(int64_t B, int64_t NB, int M, size_t* off_kept, size_t* off_cnt, size_t* total,
+                             int64_t* ld_nb) {
+  *ld_nb = (NB + 3) / 4 * 4;
+  size_t o = align_up(static_cast<size_t>(B) * static_cast<size_t>(*ld_nb) * 4, 256);
+  *off_kept = o;
+  o = align_up(o + static_cast<size_t>(B) * static_cast<size_t>(M) * 4, 256);
+  *off_cnt = o;
+  o = align_up(o + static_cast<size_t>(B) * 4, 256);
+  *total = o;
+}
+
+}  // namespace lsa
+
+using namespace lsa;
+
+extern "C" {
+
+const char* lsa_version(void) { return "lsa-b200 0.1"; }
+
+const char* lsa_last_error(void) { return g_last_error; }
+
+const char* lsa_strerror(int status) {
+  switch (status) {
+    case LSA_OK: return "ok";
+    case LSA_ERR_INVALID_ARG: return "invalid argument";
+    case LSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case LSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case LSA_ERR_CUDA: return "CUDA error (see lsa_last_error)";
+    case LSA_ERR_DEVICE_CHECK: return "device-side check failed";
+    case LSA_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+size_t lsa_workspace_size(int op, int64_t B, int64_t L, int K, int H, int sink, int window) {
+  (void)sink;
+  (void)window;
+  if (B < 0 || L < 0 || K < 0 || H < 0) return static_cast<size_t>(-1);
+  switch (op) {
+    case LSA_OP_TOPK: return 0;
+    case LSA_OP_BUCKET: {
+      size_t ok, oc, tot;
+      int64_t ldn;
+      bucket_ws_layout(B, L, K, &ok, &oc, &tot, &ldn);
+      return tot;
+    }
+    case LSA_OP_ATTN: return sparse_attn_ws_bytes(B, K, H);
+    default: return static_cast<size_t>(-1);
+  }
+}
+
+int lsa_index_score(const void* q_idx, const float* q_scale, const float* w, const void* k_idx, const float* k_scale,
+                    int dtype, int64_t B, int H_I, int d_I, int64_t L, const int64_t* q_pos, float* scores,
+                    int64_t ld, void* stream) {
+  LSA_CHECK_ARG(B >= 0 && L >= 0 && H_I >= 1 && H_I <= 64 && ld >= L && (ld % 4) == 0);
+  LSA_CHECK_ARG(dtype == LSA_BF16 || dtype == LSA_FP8_E4M3);
+  if (B == 0 || L == 0) return LSA_OK;
+  LSA_CHECK_ARG(q_idx && w && k_idx && q_pos && scores);
+  LSA_CHECK_ARG(aligned16(q_idx) && aligned16(k_idx) && aligned16(scores));
+  LSA_CHECK_ARG(B <= 65535 * 16);
+  if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
+  if (H_I * d_I > 8192) return LSA_ERR_UNSUPPORTED;
+  if (dtype == LSA_BF16) {
+    LSA_CHECK_ARG(q_scale == nullptr && k_scale == nullptr);
+  } else {
+    LSA_CHECK_ARG(q_scale != nullptr && k_scale != nullptr);
+  }
+  return launch_index_score(q_idx, q_scale, w, k_idx, k_scale, dtype, B, H_I, d_I, L, q_pos, scores, ld,
+                            static_cast<cudaStream_t>(stream));
+}
+
+int lsa_topk_select(const float* scores, int64_t ld, int64_t B, int64_t L, int K, int sink, int window,
+                    const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count, void* stream) {
+  LSA_CHECK_ARG(B >= 0 && L >= 0 && L < (int64_t(1) << 31) && K >= 1 && sink >= 0 && window >= 0);
+  LSA_CHECK_ARG(ld >= L && (ld % 4) == 0);
+  const int64_t kmax_full = static_cast<int64_t>(K) + sink + window;
+  LSA_CHECK_ARG(idx_ld >= kmax_full);
+  if (B == 0) return LSA_OK;
+  LSA_CHECK_ARG(B <= 65535);
+  LSA_CHECK_ARG(scores && q_pos && idx && count && aligned16(scores));
+  if (L == 0) return LSA_ERR_INVALID_ARG;
+  return launch_topk_mode(scores, ld, B, L, K, sink, window, q_pos, 0, 1, idx, idx_ld, count, kmax_full,
+                          static_cast<cudaStream_t>(stream));
+}
+
+int lsa_pool_keys(const void* k_idx, int dtype, const float* k_scale, int64_t L, int d_I, const int32_t* members,
+                  int bsz, int64_t NB, float* centroids, void* stream) {
+  LSA_CHECK_ARG(L >= 0 && NB >= 0 && bsz >= 1 && bsz <= 1024 && d_I >= 4 && (d_I % 4) == 0);
+  LSA_CHECK_ARG(dtype == LSA_BF16 || dtype == LSA_FP8_E4M3);
+  if (members == nullptr) LSA_CHECK_ARG(NB <= L / bsz);
+  if (NB == 0) return LSA_OK;
+  LSA_CHECK_ARG(k_idx && centroids && aligned16(centroids));
+  if (dtype == LSA_FP8_E4M3) LSA_CHECK_ARG(k_scale != nullptr);
+  return launch_pool_keys(k_idx, dtype, k_scale, L, d_I, members, bsz, NB, centroids,
+                          static_cast<cudaStream_t>(stream));
+}
+
+int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, int dtype, int64_t B, int H_I,
+                      int d_I, const float* centroids, int64_t NB, const int32_t* members, int bsz, int M, int sink,
+                      int window, int64_t L, const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count,
+                      void* ws, size_t ws_bytes, void* stream) {
+  LSA_CHECK_ARG(B >= 0 && NB >= 1 && NB < (int64_t(1) << 31) && bsz >= 1 && M >= 1 && M <= 1024);
+  LSA_CHECK_ARG(sink >= 0 && window >= 0 && L >= 1 && H_I >= 1 && H_I <= 64);
+  LSA_CHECK_ARG(static_cast<int64_t>(M) * bsz + bsz + sink + window <= 8192);
+  const int64_t kmax_full = static_cast<int64_t>(M) * bsz + (bsz - 1) + sink + window;
+  LSA_CHECK_ARG(idx_ld >= kmax_full);
+  if (dtype != LSA_BF16 || q_scale != nullptr) return LSA_ERR_UNSUPPORTED;
+  if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
+  if (members == nullptr) LSA_CHECK_ARG(NB <= L / bsz);
+  if (B == 0) return LSA_OK;
+  LSA_CHECK_ARG(B <= 65535);
+  LSA_CHECK_ARG(q_idx && w && centroids && q_pos && idx && count && aligned16(centroids) && aligned16(q_idx));
+  size_t off_kept, off_cnt, total;
+  int64_t ldn;
+  bucket_ws_layout(B, NB, M, &off_kept, &off_cnt, &total, &ldn);
+  if (ws == nullptr || !aligned256(ws) || ws_bytes < total) return LSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  float* bscores = reinterpret_cast<float*>(base);
+  int32_t* kept = reinterpret_cast<int32_t*>(base + off_kept);
+  int32_t* kcnt = reinterpret_cast<int32_t*>(base + off_cnt);
+  int st = launch_centroid_score(q_idx, w, centroids, B, H_I, d_I, NB, bscores, ldn, s);
+  if (st != LSA_OK) return st;
+  // top-M buckets: all NB ranked (explicit members) or the complete visible micro-blocks
+  st = launch_topk_mode(bscores, ldn, B, NB, M, 0, 0, q_pos, members ? 1 : 2, bsz, kept, M, kcnt, M, s);
+  if (st != LSA_OK) return st;
+  return launch_bucket_expand(kept, M, kcnt, members, bsz, sink, window, members ? 0 : bsz, q_pos, B, idx, idx_ld,
+                              count, kmax_full, s);
+}
+
+int lsa_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                    const int32_t* count, int64_t B, int H, int d_qk, int d_v, float scale, void* out, float* lse,
+                    void* ws, size_t ws_bytes, void* stream) {
+  LSA_CHECK_ARG(B >= 0 && L >= 1 && idx_ld >= 0 && idx_ld <= 65536);
+  if (d_qk != 576 || d_v != 512) return LSA_ERR_UNSUPPORTED;
+  if (H != 16 && H != 32 && H != 64 && H != 128) return LSA_ERR_UNSUPPORTED;
+  if (B == 0) return LSA_OK;
+  LSA_CHECK_ARG(q && kv && idx && count && out);
+  LSA_CHECK_ARG(aligned16(q) && aligned16(kv) && aligned16(out));
+  LSA_CHECK_ARG(B <= 65535);
+  return launch_sparse_attn(q, kv, L, idx, idx_ld, count, B, H, scale, out, lse, ws, ws_bytes,
+                            static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace lsa {
+
+// First-version dispatch (CUDA-core kernels); the tensor-core kernels replace these below when present.
+#ifndef LSA_HAVE_TC_INDEX
+int launch_index_score(const void* q, const float* q_scale, const float* w, const void* k, const float* k_scale,
+                       int dtype, int64_t B, int H_I, int d_I, int64_t L, const int64_t* q_pos, float* scores,
+                       int64_t ld, cudaStream_t s) {
+  return launch_score_simt(q, q_scale, w, k, k_scale, dtype, B, H_I, d_I, L, q_pos, scores, ld, s);
+}
+#endif
+
+#ifndef LSA_HAVE_TC_ATTN
+size_t sparse_attn_ws_bytes(int64_t, int64_t, int) { return 0; }
+int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                       const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, void*, size_t,
+                       cudaStream_t s) {
+  return launch_attn_simt(q, kv, L, idx, idx_ld, count, B, H, scale, out, lse, s);
+}
+#endif
+
+}  // namespace lsa

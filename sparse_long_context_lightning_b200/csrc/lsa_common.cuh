@@ -1,0 +1,110 @@
+// Shared device helpers of the sm_100a library (no host-visible API here).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cooperative_groups.h>
+#include <stdint.h>
+
+#include "../../include/lsa.h"
+
+namespace cg = cooperative_groups;
+
+namespace lsa {
+
+// ---------------------------------------------------------------------------
+// host-side error plumbing
+// ---------------------------------------------------------------------------
+void set_last_error(const char* msg);
+int cuda_status(cudaError_t e);  // LSA_OK or LSA_ERR_CUDA (+ records the message)
+
+#define LSA_CHECK_ARG(cond)                  \
+  do {                                       \
+    if (!(cond)) return LSA_ERR_INVALID_ARG; \
+  } while (0)
+
+#define LSA_CUDA_TRY(expr)                           \
+  do {                                               \
+    cudaError_t e_ = (expr);                         \
+    if (e_ != cudaSuccess) return lsa::cuda_status(e_); \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+
+// bf16 bits -> fp32 (exact).
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// OCP e4m3fn code -> fp32 (exact; every e4m3 value is an fp32 value).
+__device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
+  const uint32_t sign = (c & 0x80u) << 24;
+  const uint32_t e = (c >> 3) & 0xFu;
+  const uint32_t m = c & 0x7u;
+  float v;
+  if (e == 0) {
+    v = static_cast<float>(m) * 0.001953125f;  // m/8 * 2^-6
+  } else {
+    v = __uint_as_float(((e + 120u) << 23) | (m << 20));  // (1+m/8) * 2^(e-7)
+  }
+  if ((c & 0x7Fu) == 0x7Fu) v = __uint_as_float(0x7FC00000u);
+  return __uint_as_float(__float_as_uint(v) | sign);
+}
+
+// Order-preserving map of an fp32 bit pattern to uint32: a < b (as floats, -0 < +0) <=> key(a) < key(b).
+__device__ __forceinline__ uint32_t f32_order_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace lsa
+
+// Launch helpers implemented per kernel file (called from lsa_api.cu).
+namespace lsa {
+int launch_index_score(const void* q, const float* q_scale, const float* w, const void* k,
+                       const float* k_scale, int dtype, int64_t B, int H_I, int d_I, int64_t L,
+                       const int64_t* q_pos, float* scores, int64_t ld, cudaStream_t s);
+int launch_centroid_score(const void* q, const float* w, const float* centroids, int64_t B, int H_I,
+                          int d_I, int64_t NB, float* scores, int64_t ld, cudaStream_t s);
+int launch_topk(const float* scores, int64_t ld, int64_t B, int64_t L, int K, int sink, int window,
+                const int64_t* q_pos, int64_t rank_limit_div, int32_t* idx, int64_t idx_ld, int32_t* count,
+                int64_t kmax, cudaStream_t s);
+int launch_pool_keys(const void* k, int dtype, const float* k_scale, int64_t L, int d_I,
+                     const int32_t* members, int bsz, int64_t NB, float* centroids, cudaStream_t s);
+int launch_bucket_expand(const int32_t* kept, int64_t kept_ld, const int32_t* kept_count,
+                         const int32_t* members, int bsz, int sink, int window, int tail_block,
+                         const int64_t* q_pos, int64_t B, int32_t* idx, int64_t idx_ld, int32_t* count,
+                         int64_t kmax, cudaStream_t s);
+int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                       const int32_t* count, int64_t B, int H, float scale, void* out, float* lse,
+                       void* ws, size_t ws_bytes, cudaStream_t s);
+size_t sparse_attn_ws_bytes(int64_t B, int64_t kmax, int H);
+}  // namespace lsa
