@@ -1,0 +1,314 @@
+// Lightning-indexer scores on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// "LongCat Sparse Attention（LSA）完全拆解", section "DSA 基线", equation
+//   I_{t,s} = sum_j w_{t,j} * ReLU(q^I_{t,j} . k^I_s),
+// H_I heads sharing one MQA key, ReLU instead of softmax, bf16 or FP8.
+//
+// The dense part is the contraction D[s, (b,j)] = k_s . q_{b,j}: keys are the MMA's M side (128 keys per
+// tile), the (query, head) pairs of a 256-column chunk are its N side, d_I is K.  With keys on the TMEM
+// lanes, the ReLU / weight / head-sum epilogue is a per-thread reduction over one TMEM row segment: no
+// cross-thread traffic.  Grid: (query chunk) x (key range); the 256-row query chunk stays in shared
+// memory, key tiles stream through a TMA ring.  Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer
+// (and TMEM owner), warps 2..9 = epilogue (two warpgroups, one per 128-column half of the chunk).
+// TMEM holds two 256-column fp32 accumulators so the epilogue of tile i overlaps the MMAs of tile i+1.
+#include "lsa_common.cuh"
+#include "sm100.cuh"
+
+namespace lsa {
+namespace {
+
+using namespace sm100;
+
+constexpr int IX_THREADS = 320;
+
+// Set (never cleared by the kernel) when a bounded wait of this kernel gave up.
+__device__ int g_index_tc_timeout;
+constexpr int IX_TILE_M = 128;  // keys per tile
+constexpr int IX_CHUNK_N = 256; // (query, head) columns per chunk
+
+template <bool FP8>
+struct IxCfg {
+  static constexpr int KB = FP8 ? 1 : 2;                     // 128-byte K-blocks per 128-dim row
+  static constexpr int TILE_BYTES = IX_TILE_M * 128 * KB;    // key tile
+  static constexpr int Q_BYTES = IX_CHUNK_N * 128 * KB;      // query chunk
+  static constexpr int STAGES = FP8 ? 6 : 4;
+  static constexpr int KSTEPS = 4 * KB;                      // MMA instructions per tile (32 B of K each)
+  static constexpr uint32_t IDESC = idesc_mma(IX_TILE_M, IX_CHUNK_N, FP8 ? 0u : 1u);
+  static constexpr int SMEM = 1024 + Q_BYTES + STAGES * TILE_BYTES + 2048;
+};
+
+struct IxArgs {
+  const float* w;
+  const float* q_scale;
+  const float* k_scale;
+  const int64_t* q_pos;
+  float* scores;
+  int64_t ld;
+  int L;
+  int B;
+  int H_I;
+  int n_chunks;
+  int ntiles;
+  int tiles_per_range;
+};
+
+template <bool FP8>
+__global__ void __launch_bounds__(IX_THREADS, 1)
+    k_index_score_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q, IxArgs a) {
+  using C = IxCfg<FP8>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte aligned base for the swizzled tiles
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* q_s = base;
+  unsigned char* k_s = q_s + C::Q_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(k_s + C::STAGES * C::TILE_BYTES);
+  uint64_t* full = bars;                  // [STAGES]
+  uint64_t* empty = bars + C::STAGES;     // [STAGES]
+  uint64_t* tfull = bars + 2 * C::STAGES; // [2]
+  uint64_t* tempty = tfull + 2;           // [2]
+  uint64_t* qfull = tempty + 2;           // [1]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qfull + 1);
+  float* wsm = reinterpret_cast<float*>(tmem_holder + 4);  // [256] weights of this chunk's (query, head) pairs
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chunk = blockIdx.x % a.n_chunks;
+  const int range = blockIdx.x / a.n_chunks;
+  const int t_begin = range * a.tiles_per_range;
+  const int t_end = min(a.ntiles, t_begin + a.tiles_per_range);
+  const int n_my = max(0, t_end - t_begin);
+  const int qpc = IX_CHUNK_N / a.H_I;  // queries per chunk
+  const int b0 = chunk * qpc;
+
+  if (tid == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);
+    }
+    mbar_init(qfull, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int i = tid; i < IX_CHUNK_N; i += IX_THREADS) {
+    const int b = b0 + i / a.H_I, j = i % a.H_I;
+    float v = 0.f;
+    if (b < a.B) v = a.w[static_cast<int64_t>(b) * a.H_I + j] * (a.q_scale ? a.q_scale[static_cast<int64_t>(b) * a.H_I + j] : 1.f);
+    wsm[i] = v;
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_my > 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_q);
+      mbar_expect_tx(qfull, C::Q_BYTES);
+      for (int kb = 0; kb < C::KB; ++kb)
+        tma_load_2d(q_s + kb * IX_CHUNK_N * 128, &tm_q, qfull, kb * (FP8 ? 128 : 64), chunk * IX_CHUNK_N);
+      for (int i = 0; i < n_my; ++i) {
+        const int st = i % C::STAGES;
+        const uint32_t par = ((i / C::STAGES) & 1) ^ 1;
+        if (!mbar_wait(&empty[st], par)) {
+          atomicExch(&g_index_tc_timeout, 1);
+          abort_flag = 1;
+          break;
+        }
+        mbar_expect_tx(&full[st], C::TILE_BYTES);
+        const int row = (t_begin + i) * IX_TILE_M;
+        unsigned char* dst = k_s + st * C::TILE_BYTES;
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_2d(dst + kb * IX_TILE_M * 128, &tm_k, &full[st], kb * (FP8 ? 128 : 64), row);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_my > 0) {
+      bool ok = mbar_wait(qfull, 0);
+      const uint32_t q_addr = smem_u32(q_s);
+      for (int i = 0; ok && i < n_my; ++i) {
+        const int st = i % C::STAGES;
+        const int buf = i & 1;
+        if (!mbar_wait(&full[st], (i / C::STAGES) & 1) || !mbar_wait(&tempty[buf], ((i >> 1) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(k_s + st * C::TILE_BYTES);
+        #pragma unroll
+        for (int k = 0; k < C::KSTEPS; ++k) {
+          const int kb = k >> 2, kk = k & 3;
+          const uint64_t ad = desc_sw128(k_addr + kb * IX_TILE_M * 128 + kk * 32);
+          const uint64_t bd = desc_sw128(q_addr + kb * IX_CHUNK_N * 128 + kk * 32);
+          if (FP8)
+            mma_f8(tmem + buf * IX_CHUNK_N, ad, bd, C::IDESC, k > 0);
+          else
+            mma_f16(tmem + buf * IX_CHUNK_N, ad, bd, C::IDESC, k > 0);
+        }
+        mma_commit(&empty[st]);
+        mma_commit(&tfull[buf]);
+      }
+      if (!ok) {
+        atomicExch(&g_index_tc_timeout, 1);
+        abort_flag = 1;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2..9)
+    const int ew = warp - 2;
+    const int quarter = warp & 3;        // TMEM lanes this warp may access
+    const int half = ew >> 2;            // column half of the chunk
+    const int nq_half = (IX_CHUNK_N / 2) / a.H_I;
+    for (int i = 0; i < n_my; ++i) {
+      const int buf = i & 1;
+      if (!mbar_wait(&tfull[buf], (i >> 1) & 1)) {
+        atomicExch(&g_index_tc_timeout, 1);
+        break;
+      }
+      tc_fence_after();
+      const int s = (t_begin + i) * IX_TILE_M + quarter * 32 + lane;
+      const float ks = (FP8 && s < a.L) ? a.k_scale[s] : 1.f;
+      for (int qi = 0; qi < nq_half; ++qi) {
+        const int col0 = half * (IX_CHUNK_N / 2) + qi * a.H_I;
+        float acc = 0.f;
+        for (int j0 = 0; j0 < a.H_I; j0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * IX_CHUNK_N + col0 + j0, r);
+          tmem_ld_wait();
+          const float* wv = wsm + col0 + j0;
+          #pragma unroll
+          for (int c = 0; c < 32; ++c) acc = fmaf(wv[c], fmaxf(__uint_as_float(r[c]), 0.f), acc);
+        }
+        const int b = b0 + col0 / a.H_I;
+        if (b < a.B && s < a.L) {
+          const float v = (static_cast<int64_t>(s) > a.q_pos[b]) ? -INFINITY : acc * ks;
+          a.scores[static_cast<int64_t>(b) * a.ld + s] = v;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D row-major [rows, cols] map with a (box_cols x box_rows) box and the 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* ptr, bool fp8, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  EncodeTiledFn fn = encoder();
+  if (!fn) {
+    set_last_error("cuTensorMapEncodeTiled unavailable");
+    return LSA_ERR_CUDA;
+  }
+  const int esz = fp8 ? 1 : 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * esz)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_last_error("cuTensorMapEncodeTiled failed");
+    return LSA_ERR_CUDA;
+  }
+  return LSA_OK;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <bool FP8>
+int launch_tc(const void* q, const float* q_scale, const float* w, const void* k, const float* k_scale, int64_t B,
+              int H_I, int64_t L, const int64_t* q_pos, float* scores, int64_t ld, cudaStream_t s) {
+  using C = IxCfg<FP8>;
+  CUtensorMap tk, tq;
+  const int boxc = FP8 ? 128 : 64;
+  int st = make_map(&tk, k, FP8, L, 128, boxc, IX_TILE_M);
+  if (st) return st;
+  st = make_map(&tq, q, FP8, B * H_I, 128, boxc, IX_CHUNK_N);
+  if (st) return st;
+  IxArgs a;
+  a.w = w;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.q_pos = q_pos;
+  a.scores = scores;
+  a.ld = ld;
+  a.L = static_cast<int>(L);
+  a.B = static_cast<int>(B);
+  a.H_I = H_I;
+  a.n_chunks = static_cast<int>(cdiv(B * H_I, IX_CHUNK_N));
+  a.ntiles = static_cast<int>(cdiv(L, IX_TILE_M));
+  const int sms = sm_count();
+  int ranges = a.n_chunks >= sms ? 1 : static_cast<int>(cdiv(sms, a.n_chunks));
+  if (ranges > a.ntiles) ranges = a.ntiles;
+  a.tiles_per_range = static_cast<int>(cdiv(a.ntiles, ranges));
+  ranges = static_cast<int>(cdiv(a.ntiles, a.tiles_per_range));
+  LSA_CUDA_TRY(cudaFuncSetAttribute(k_index_score_tc<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+  const int64_t grid = static_cast<int64_t>(a.n_chunks) * ranges;
+  k_index_score_tc<FP8><<<static_cast<unsigned>(grid), IX_THREADS, C::SMEM, s>>>(tk, tq, a);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+int launch_score_simt(const void* q, const float* q_scale, const float* w, const void* k, const float* k_scale,
+                      int dtype, int64_t B, int H_I, int d_I, int64_t L, const int64_t* q_pos, float* scores,
+                      int64_t ld, cudaStream_t s);
+
+// Tensor-core path for d_I = 128 with 32 or 64 heads; other shapes use the CUDA-core kernel.
+int launch_index_score(const void* q, const float* q_scale, const float* w, const void* k, const float* k_scale,
+                       int dtype, int64_t B, int H_I, int d_I, int64_t L, const int64_t* q_pos, float* scores,
+                       int64_t ld, cudaStream_t s) {
+  if (B == 0 || L == 0) return LSA_OK;
+  const bool tc = d_I == 128 && (H_I == 32 || H_I == 64) && aligned16(q) && aligned16(k) && L >= IX_TILE_M &&
+                  L < (int64_t(1) << 31);
+  if (!tc) return launch_score_simt(q, q_scale, w, k, k_scale, dtype, B, H_I, d_I, L, q_pos, scores, ld, s);
+  if (dtype == LSA_FP8_E4M3) return launch_tc<true>(q, q_scale, w, k, k_scale, B, H_I, L, q_pos, scores, ld, s);
+  return launch_tc<false>(q, q_scale, w, k, k_scale, B, H_I, L, q_pos, scores, ld, s);
+}
+
+}  // namespace lsa

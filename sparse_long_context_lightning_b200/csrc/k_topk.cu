@@ -119,8 +119,10 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     clo = 0;
     chi = a.L;
   } else {
+    // q_pos is a token position here; the candidates are the complete visible blocks
     clo = 0;
-    chi = min(a.L, (qp + 1) / a.div);
+    const int64_t nvis = qp64 < 0 ? 0 : (qp64 + 1) / a.div;
+    chi = static_cast<int>(nvis < a.L ? nvis : a.L);
   }
   const int ncand = max(0, chi - clo);
   const int K = a.K;

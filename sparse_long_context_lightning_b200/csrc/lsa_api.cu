@@ -176,15 +176,6 @@ int lsa_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx
 
 namespace lsa {
 
-// First-version dispatch (CUDA-core kernels); the tensor-core kernels replace these below when present.
-#ifndef LSA_HAVE_TC_INDEX
-int launch_index_score(const void* q, const float* q_scale, const float* w, const void* k, const float* k_scale,
-                       int dtype, int64_t B, int H_I, int d_I, int64_t L, const int64_t* q_pos, float* scores,
-                       int64_t ld, cudaStream_t s) {
-  return launch_score_simt(q, q_scale, w, k, k_scale, dtype, B, H_I, d_I, L, q_pos, scores, ld, s);
-}
-#endif
-
 #ifndef LSA_HAVE_TC_ATTN
 size_t sparse_attn_ws_bytes(int64_t, int64_t, int) { return 0; }
 int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
