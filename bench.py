@@ -173,9 +173,9 @@ def committed_traffic(kernel: str):
     return d.get("dram_bytes_per_launch")
 
 
-STAGE_KERNEL = {"index": ("k_index_score", ["k_index_tc.cu", "k_score_simt.cu"]),
+STAGE_KERNEL = {"index": ("k_index_score_tc", ["k_index_tc.cu"]),
                 "topk": ("k_topk_cluster", ["k_topk.cu"]),
-                "attn": ("k_sparse_attn", ["k_attn_tc.cu", "k_attn_simt.cu"])}
+                "attn": ("k_sparse_attn_tc", ["k_attn_tc.cu"])}
 # kernels each stage launches per step (the e2e leg adds none of ours)
 LAUNCHES = {"index": 1, "topk": 1, "attn": 1}
 
@@ -190,8 +190,7 @@ def run_gpu(args, rank, world, local_rank):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream()
     launches = dict(LAUNCHES)
-    if hasattr(lsa, "attn_launches_per_call"):
-        launches["attn"] = lsa.attn_launches_per_call()
+    launches["attn"] = 2 if lsa.lsa_workspace_size(lsa.LSA_OP_ATTN, wl.B, wl.L, step.kmax, wl.H) > 0 else 1  # + combine
 
     def one_step(ev):
         ev[0].record(stream)

@@ -1,0 +1,466 @@
+// Sparse absorbed-MQA attention over gathered MLA latent rows on tcgen05 tensor cores.
+//
+// "LongCat Sparse Attention（LSA）完全拆解", section "DSA 基线": u_t = Attn(h_t, {c_s | s in S_t}), the
+// 576-dim bf16 latent c_s shared by all 128 heads, value = its first 512 dims; section "瓶颈一": the
+// selected 1152-byte rows are scattered, so the kernel is a gather whose memory-level parallelism decides
+// the achieved bandwidth.
+//
+// B200 design.  A 128 x 512 fp32 output accumulator fills all of TMEM (128 lanes x 512 columns), leaving
+// no room for the logits, so one work unit (query b, a contiguous split of its selected rows) runs on a
+// 2-CTA cluster: CTA r owns output columns [256r, 256r+256) and latent dims D_0 = [0, 256), D_1 =
+// [256, 576).  Each CTA gathers only its own part of every selected row (512 or 640 bytes, disjoint), with
+// TMA tile::gather4 loads into 128-byte-swizzled shared memory, computes the partial logits
+// S_r = Q[:, D_r] . C[:, D_r]^T, and the two partials are exchanged through distributed shared memory
+// (remote mbarrier arrivals, no cluster-wide barrier per tile).  Both CTAs then hold the same logits,
+// run the same online softmax (lazy rescale: O is rescaled only when the running max grows by > 2^8),
+// and each accumulates P . V[:, its 256 columns] in TMEM.  The gathered tile serves both MMAs: K-major for
+// S = Q C^T and MN-major for O += P V, so no transpose is needed.  Splits of one query are merged by a
+// small combine kernel (log-sum-exp weights).
+//
+// Warp roles (192 threads): warp 0 gathers (TMA), warp 1 issues MMAs and owns TMEM, warps 2-5 run the
+// softmax (one head per thread = one TMEM lane) and the epilogue.
+#include "lsa_common.cuh"
+#include "sm100.cuh"
+
+namespace lsa {
+namespace {
+
+using namespace sm100;
+
+__device__ int g_attn_tc_timeout;  // set when a bounded wait of the kernel gave up
+
+constexpr int AT_THREADS = 192;
+constexpr int AT_T = 32;   // gathered rows per tile
+constexpr int AT_H = 128;  // heads (MMA M)
+constexpr int AT_KBQ_MAX = 5;
+constexpr int AT_STAGES = 5;
+constexpr int AT_Q_BYTES = AT_KBQ_MAX * AT_H * 128;        // 80 KB
+constexpr int AT_KB_BYTES = AT_T * 128;                    // 4 KB: one 64-dim block of a tile
+constexpr int AT_STAGE_BYTES = AT_KBQ_MAX * AT_KB_BYTES;   // 20 KB
+constexpr int AT_P_BYTES = AT_H * 128;                     // 16 KB
+constexpr int AT_SX_FLOATS = AT_T * AT_H;                  // 16 KB
+constexpr int AT_SMEM = 1024 + AT_Q_BYTES + AT_STAGES * AT_STAGE_BYTES + AT_P_BYTES + AT_SX_FLOATS * 4 + 512;
+constexpr uint32_t TM_O = 0;    // TMEM columns [0, 256): O
+constexpr uint32_t TM_S = 256;  // TMEM columns [256, 320): two S buffers of 32
+constexpr uint32_t IDESC_S = idesc_mma(128, AT_T, 1u, 0u);
+constexpr uint32_t IDESC_PV = idesc_mma(128, 256, 1u, 1u);
+constexpr float RESCALE_LOG2 = 8.f;
+
+struct AtArgs {
+  const int32_t* idx;
+  int64_t idx_ld;
+  const int32_t* count;
+  int B;
+  int L;
+  int S;  // splits per query
+  float scale_log2;
+  uint16_t* out;
+  float* lse;
+  float* ws_o;   // [B, S, 128, 512] fp32 (S > 1)
+  float* ws_ml;  // [B, S, 128, 2]   fp32 (S > 1): running max (log2 units), sum
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
+    k_sparse_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv, AtArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* q_s = base;
+  unsigned char* st_s = q_s + AT_Q_BYTES;
+  unsigned char* p_s = st_s + AT_STAGES * AT_STAGE_BYTES;
+  float* sx_s = reinterpret_cast<float*>(p_s + AT_P_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sx_s + AT_SX_FLOATS);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = kv_full + AT_STAGES;
+  uint64_t* s_full = kv_empty + AT_STAGES;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* p_full = s_empty + 2;
+  uint64_t* pv_done = p_full + 1;
+  uint64_t* sx_full = pv_done + 1;
+  uint64_t* sx_empty = sx_full + 1;
+  uint64_t* q_full = sx_empty + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(q_full + 1);
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t r = cluster_ctarank();
+  const uint32_t peer = r ^ 1u;
+  const int unit = blockIdx.x >> 1;
+  const int b = unit / a.S, split = unit % a.S;
+  const int kbq = r ? 5 : 4;
+  int n = a.count[b];
+  n = n < 0 ? 0 : (static_cast<int64_t>(n) > a.idx_ld ? static_cast<int>(a.idx_ld) : n);
+  const int rps = ((n + a.S - 1) / a.S + AT_T - 1) / AT_T * AT_T;
+  const int row0 = split * rps;
+  const int nrows = max(0, min(n, row0 + rps) - row0);
+  const int ntiles = (nrows + AT_T - 1) / AT_T;
+
+  if (tid == 0) {
+    for (int i = 0; i < AT_STAGES; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
+    mbar_init(sx_full, AT_H);   // one arrival per peer softmax thread
+    mbar_init(sx_empty, AT_H);
+    mbar_init(q_full, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's barriers are initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ gather producer
+    if (ntiles > 0) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_kv);
+        mbar_expect_tx(q_full, kbq * AT_H * 128);
+        for (int kb = 0; kb < kbq; ++kb)
+          tma_load_2d(q_s + kb * AT_H * 128, &tm_q, q_full, 256 * static_cast<int>(r) + 64 * kb, b * AT_H);
+      }
+      const int32_t* rowidx = a.idx + static_cast<int64_t>(b) * a.idx_ld + row0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int st = i % AT_STAGES;
+        const int rr = i * AT_T + lane;
+        int v = rr < nrows ? rowidx[rr] : 0;
+        v = v < 0 ? 0 : (v >= a.L ? a.L - 1 : v);
+        if (!mbar_wait(&kv_empty[st], ((i / AT_STAGES) & 1) ^ 1) || abort_flag) {
+          if (lane == 0) {
+            atomicExch(&g_attn_tc_timeout, 1);
+            abort_flag = 1;
+          }
+          break;
+        }
+        unsigned char* dst = st_s + st * AT_STAGE_BYTES;
+        if (lane == 0) mbar_expect_tx(&kv_full[st], kbq * AT_KB_BYTES);
+        #pragma unroll
+        for (int g = 0; g < AT_T / 4; ++g) {
+          const int y0 = __shfl_sync(0xffffffffu, v, 4 * g + 0);
+          const int y1 = __shfl_sync(0xffffffffu, v, 4 * g + 1);
+          const int y2 = __shfl_sync(0xffffffffu, v, 4 * g + 2);
+          const int y3 = __shfl_sync(0xffffffffu, v, 4 * g + 3);
+          if (lane == 0) {
+            for (int kb = 0; kb < kbq; ++kb)
+              tma_gather4(dst + kb * AT_KB_BYTES + g * 512, &tm_kv, &kv_full[st], 256 * static_cast<int>(r) + 64 * kb,
+                          y0, y1, y2, y3);
+          }
+        }
+        __syncwarp();
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (ntiles > 0 && lane == 0) {
+      bool ok = mbar_wait(q_full, 0);
+      const uint32_t q_addr = smem_u32(q_s);
+      const uint32_t p_addr = smem_u32(p_s);
+      for (int i = 0; ok && i <= ntiles; ++i) {
+        if (i < ntiles) {
+          const int st = i % AT_STAGES, sb = i & 1;
+          if (!mbar_wait(&kv_full[st], (i / AT_STAGES) & 1) || !mbar_wait(&s_empty[sb], ((i >> 1) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t s_addr = smem_u32(st_s + st * AT_STAGE_BYTES);
+          for (int kb = 0; kb < kbq; ++kb) {
+            #pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16(tmem + TM_S + sb * AT_T, desc_sw128(q_addr + kb * AT_H * 128 + kk * 32),
+                      desc_sw128(s_addr + kb * AT_KB_BYTES + kk * 32), IDESC_S, (kb | kk) != 0);
+          }
+          mma_commit(&s_full[sb]);
+        }
+        if (i >= 1) {
+          const int j = i - 1, stj = j % AT_STAGES;
+          if (!mbar_wait(p_full, j & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t v_addr = smem_u32(st_s + stj * AT_STAGE_BYTES);
+          #pragma unroll
+          for (int kk = 0; kk < AT_T / 16; ++kk)
+            mma_f16(tmem + TM_O, desc_sw128(p_addr + kk * 32), desc_sw128_mn(v_addr + kk * 16 * 128, AT_KB_BYTES, 1024),
+                    IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&kv_empty[stj]);
+          mma_commit(pv_done);
+        }
+      }
+      if (!ok) {
+        atomicExch(&g_attn_tc_timeout, 1);
+        abort_flag = 1;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int q4 = warp & 3;
+    const int h = q4 * 32 + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const uint32_t peer_sx = mapa(smem_u32(sx_s), peer);
+    const uint32_t peer_sx_full = mapa(smem_u32(sx_full), peer);
+    const uint32_t peer_sx_empty = mapa(smem_u32(sx_empty), peer);
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < ntiles; ++i) {
+      const int sb = i & 1;
+      const int nvalid = min(AT_T, nrows - i * AT_T);
+      if (!mbar_wait(&s_full[sb], (i >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[32];
+      tmem_ld32(trow + TM_S + sb * AT_T, sr);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[sb]);
+      // send my partial logits to the peer, then take the peer's
+      if (!mbar_wait(sx_empty, (i & 1) ^ 1)) {
+        ok = false;
+        break;
+      }
+      #pragma unroll
+      for (int c = 0; c < AT_T; ++c) st_cluster_f32(peer_sx + static_cast<uint32_t>((c * AT_H + h) * 4), __uint_as_float(sr[c]));
+      mbar_arrive_cluster(peer_sx_full);
+      if (!mbar_wait_cluster(sx_full, i & 1)) {
+        ok = false;
+        break;
+      }
+      float z[AT_T];
+      float mt = -INFINITY;
+      #pragma unroll
+      for (int c = 0; c < AT_T; ++c) {
+        const float sfull = __uint_as_float(sr[c]) + sx_s[c * AT_H + h];
+        z[c] = c < nvalid ? sfull * a.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, z[c]);
+      }
+      mbar_arrive_cluster(peer_sx_empty);
+      float alpha = 1.f;
+      bool resc = false;
+      if (i == 0) {
+        m_used = mt;
+      } else if (mt > m_used + RESCALE_LOG2) {
+        alpha = exp2f(m_used - mt);
+        m_used = mt;
+        resc = true;
+      }
+      uint32_t pk[AT_T / 2];
+      float psum = 0.f;
+      #pragma unroll
+      for (int c = 0; c < AT_T; c += 2) {
+        const __nv_bfloat162 p2 = __floats2bfloat162_rn(exp2f(z[c] - m_used), exp2f(z[c + 1] - m_used));
+        const float2 back = __bfloat1622float2(p2);
+        psum += back.x + back.y;
+        pk[c / 2] = *reinterpret_cast<const uint32_t*>(&p2);
+      }
+      l = l * alpha + psum;
+      // the previous P . V has finished: the P buffer is free and O is stable
+      if (i > 0 && !mbar_wait(pv_done, (i - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (resc) {
+        #pragma unroll 1
+        for (int k = 0; k < 8; ++k) {
+          uint32_t o[32];
+          tmem_ld32(trow + TM_O + 32 * k, o);
+          tmem_ld_wait();
+          #pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st32(trow + TM_O + 32 * k, o);
+        }
+        tmem_st_wait();
+      }
+      // P row h (32 bf16 = 64 B) into the 128-byte-swizzled K-major A tile
+      unsigned char* prow = p_s + h * 128;
+      #pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (!ok) {
+      atomicExch(&g_attn_tc_timeout, 1);
+      abort_flag = 1;
+    }
+    // ---- epilogue
+    const bool have = ok && ntiles > 0 && mbar_wait(pv_done, (ntiles - 1) & 1);
+    tc_fence_after();
+    const int64_t orow = static_cast<int64_t>(b) * AT_H + h;
+    if (a.S == 1) {
+      const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
+      uint16_t* dst = a.out + orow * 512 + 256 * r;
+      #pragma unroll 1
+      for (int k = 0; k < 8; ++k) {
+        uint32_t o[32];
+        if (have) {
+          tmem_ld32(trow + TM_O + 32 * k, o);
+          tmem_ld_wait();
+        } else {
+          #pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+        uint32_t pk[16];
+        #pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv);
+          pk[c / 2] = *reinterpret_cast<const uint32_t*>(&v);
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * k);
+        #pragma unroll
+        for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      if (r == 0 && a.lse) a.lse[orow] = (have && l > 0.f) ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
+    } else {
+      const int64_t prow_i = (static_cast<int64_t>(b) * a.S + split) * AT_H + h;
+      float* dst = a.ws_o + prow_i * 512 + 256 * r;
+      #pragma unroll 1
+      for (int k = 0; k < 8; ++k) {
+        uint32_t o[32];
+        if (have) {
+          tmem_ld32(trow + TM_O + 32 * k, o);
+          tmem_ld_wait();
+        } else {
+          #pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+        float4* d4 = reinterpret_cast<float4*>(dst + 32 * k);
+        #pragma unroll
+        for (int c = 0; c < 8; ++c)
+          d4[c] = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]), __uint_as_float(o[4 * c + 2]),
+                              __uint_as_float(o[4 * c + 3]));
+      }
+      if (r == 0) {
+        a.ws_ml[prow_i * 2 + 0] = have ? m_used : -INFINITY;
+        a.ws_ml[prow_i * 2 + 1] = have ? l : 0.f;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still touch its shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Merge the splits of one (query, head): LSE-weighted sum of the partial outputs.
+__global__ void __launch_bounds__(128) k_attn_combine(const float* __restrict__ ws_o, const float* __restrict__ ws_ml,
+                                                      int S, uint16_t* __restrict__ out, float* __restrict__ lse) {
+  const int64_t bh = blockIdx.x;  // b * 128 + h
+  const int b = static_cast<int>(bh / AT_H), h = static_cast<int>(bh % AT_H);
+  float mstar = -INFINITY;
+  for (int s = 0; s < S; ++s) {
+    const int64_t pi = (static_cast<int64_t>(b) * S + s) * AT_H + h;
+    if (ws_ml[pi * 2 + 1] > 0.f) mstar = fmaxf(mstar, ws_ml[pi * 2]);
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lsum = 0.f;
+  if (mstar != -INFINITY) {
+    for (int s = 0; s < S; ++s) {
+      const int64_t pi = (static_cast<int64_t>(b) * S + s) * AT_H + h;
+      const float ls = ws_ml[pi * 2 + 1];
+      if (!(ls > 0.f)) continue;
+      const float wgt = exp2f(ws_ml[pi * 2] - mstar);
+      lsum += wgt * ls;
+      const float4 v = reinterpret_cast<const float4*>(ws_o + pi * 512)[threadIdx.x];
+      acc.x += wgt * v.x;
+      acc.y += wgt * v.y;
+      acc.z += wgt * v.z;
+      acc.w += wgt * v.w;
+    }
+  }
+  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  uint2 pk;
+  pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+  pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+  reinterpret_cast<uint2*>(out + bh * 512)[threadIdx.x] = pk;
+  if (lse && threadIdx.x == 0) lse[bh] = lsum > 0.f ? (mstar + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
+}
+
+int splits_for(int64_t B) {
+  int64_t s = 148 / (2 * (B > 0 ? B : 1));
+  if (s < 1) s = 1;
+  if (s > 32) s = 32;
+  return static_cast<int>(s);
+}
+
+}  // namespace
+
+int make_map(CUtensorMap* m, const void* ptr, bool fp8, int64_t rows, int64_t cols, int box_cols, int box_rows);
+int launch_attn_simt(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                     const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, cudaStream_t s);
+
+size_t sparse_attn_ws_bytes(int64_t B, int64_t, int H) {
+  if (H != AT_H) return 0;
+  const int S = splits_for(B);
+  if (S == 1) return 0;
+  const size_t o = align_up(static_cast<size_t>(B) * S * AT_H * 512 * 4, 256);
+  return o + align_up(static_cast<size_t>(B) * S * AT_H * 2 * 4, 256);
+}
+
+int attn_launches_per_call(int64_t B, int H) { return (H == AT_H && splits_for(B) > 1) ? 2 : 1; }
+
+int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                       const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, void* ws,
+                       size_t ws_bytes, cudaStream_t s) {
+  if (B == 0) return LSA_OK;
+  if (H != AT_H || L >= (int64_t(1) << 31)) return launch_attn_simt(q, kv, L, idx, idx_ld, count, B, H, scale, out, lse, s);
+  const int S = splits_for(B);
+  const size_t need = sparse_attn_ws_bytes(B, idx_ld, H);
+  if (S > 1 && (ws == nullptr || !aligned256(ws) || ws_bytes < need)) return LSA_ERR_WORKSPACE;
+  CUtensorMap tq, tkv;
+  int st = make_map(&tq, q, false, B * AT_H, 576, 64, AT_H);
+  if (st) return st;
+  st = make_map(&tkv, kv, false, L, 576, 64, 1);
+  if (st) return st;
+  AtArgs a;
+  a.idx = idx;
+  a.idx_ld = idx_ld;
+  a.count = count;
+  a.B = static_cast<int>(B);
+  a.L = static_cast<int>(L);
+  a.S = S;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.ws_o = S > 1 ? static_cast<float*>(ws) : nullptr;
+  a.ws_ml = S > 1 ? reinterpret_cast<float*>(static_cast<unsigned char*>(ws) +
+                                             align_up(static_cast<size_t>(B) * S * AT_H * 512 * 4, 256))
+                  : nullptr;
+  LSA_CUDA_TRY(cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM));
+  const int64_t grid = 2 * B * S;
+  if (grid > 0x7FFFFFFF) return LSA_ERR_UNSUPPORTED;
+  k_sparse_attn_tc<<<static_cast<unsigned>(grid), AT_THREADS, AT_SMEM, s>>>(tq, tkv, a);
+  LSA_CUDA_TRY(cudaGetLastError());
+  if (S > 1) {
+    k_attn_combine<<<static_cast<unsigned>(B * AT_H), 128, 0, s>>>(a.ws_o, a.ws_ml, S, a.out, lse);
+    LSA_CUDA_TRY(cudaGetLastError());
+  }
+  return LSA_OK;
+}
+
+}  // namespace lsa

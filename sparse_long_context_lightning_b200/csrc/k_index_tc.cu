@@ -15,6 +15,10 @@
 #include "sm100.cuh"
 
 namespace lsa {
+
+int make_map(CUtensorMap* m, const void* ptr, bool fp8, int64_t rows, int64_t cols, int box_cols, int box_rows);
+int sm_count();
+
 namespace {
 
 using namespace sm100;
@@ -208,6 +212,41 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   }
 }
 
+template <bool FP8>
+int launch_tc(const void* q, const float* q_scale, const float* w, const void* k, const float* k_scale, int64_t B,
+              int H_I, int64_t L, const int64_t* q_pos, float* scores, int64_t ld, cudaStream_t s) {
+  using C = IxCfg<FP8>;
+  CUtensorMap tk, tq;
+  const int boxc = FP8 ? 128 : 64;
+  int st = make_map(&tk, k, FP8, L, 128, boxc, IX_TILE_M);
+  if (st) return st;
+  st = make_map(&tq, q, FP8, B * H_I, 128, boxc, IX_CHUNK_N);
+  if (st) return st;
+  IxArgs a;
+  a.w = w;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.q_pos = q_pos;
+  a.scores = scores;
+  a.ld = ld;
+  a.L = static_cast<int>(L);
+  a.B = static_cast<int>(B);
+  a.H_I = H_I;
+  a.n_chunks = static_cast<int>(cdiv(B * H_I, IX_CHUNK_N));
+  a.ntiles = static_cast<int>(cdiv(L, IX_TILE_M));
+  const int sms = sm_count();
+  int ranges = a.n_chunks >= sms ? 1 : static_cast<int>(cdiv(sms, a.n_chunks));
+  if (ranges > a.ntiles) ranges = a.ntiles;
+  a.tiles_per_range = static_cast<int>(cdiv(a.ntiles, ranges));
+  ranges = static_cast<int>(cdiv(a.ntiles, a.tiles_per_range));
+  LSA_CUDA_TRY(cudaFuncSetAttribute(k_index_score_tc<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+  const int64_t grid = static_cast<int64_t>(a.n_chunks) * ranges;
+  k_index_score_tc<FP8><<<static_cast<unsigned>(grid), IX_THREADS, C::SMEM, s>>>(tk, tq, a);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
 // ------------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------------
@@ -259,41 +298,6 @@ int sm_count() {
   }
   return n;
 }
-
-template <bool FP8>
-int launch_tc(const void* q, const float* q_scale, const float* w, const void* k, const float* k_scale, int64_t B,
-              int H_I, int64_t L, const int64_t* q_pos, float* scores, int64_t ld, cudaStream_t s) {
-  using C = IxCfg<FP8>;
-  CUtensorMap tk, tq;
-  const int boxc = FP8 ? 128 : 64;
-  int st = make_map(&tk, k, FP8, L, 128, boxc, IX_TILE_M);
-  if (st) return st;
-  st = make_map(&tq, q, FP8, B * H_I, 128, boxc, IX_CHUNK_N);
-  if (st) return st;
-  IxArgs a;
-  a.w = w;
-  a.q_scale = q_scale;
-  a.k_scale = k_scale;
-  a.q_pos = q_pos;
-  a.scores = scores;
-  a.ld = ld;
-  a.L = static_cast<int>(L);
-  a.B = static_cast<int>(B);
-  a.H_I = H_I;
-  a.n_chunks = static_cast<int>(cdiv(B * H_I, IX_CHUNK_N));
-  a.ntiles = static_cast<int>(cdiv(L, IX_TILE_M));
-  const int sms = sm_count();
-  int ranges = a.n_chunks >= sms ? 1 : static_cast<int>(cdiv(sms, a.n_chunks));
-  if (ranges > a.ntiles) ranges = a.ntiles;
-  a.tiles_per_range = static_cast<int>(cdiv(a.ntiles, ranges));
-  ranges = static_cast<int>(cdiv(a.ntiles, a.tiles_per_range));
-  LSA_CUDA_TRY(cudaFuncSetAttribute(k_index_score_tc<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
-  const int64_t grid = static_cast<int64_t>(a.n_chunks) * ranges;
-  k_index_score_tc<FP8><<<static_cast<unsigned>(grid), IX_THREADS, C::SMEM, s>>>(tk, tq, a);
-  return cuda_status(cudaGetLastError());
-}
-
-}  // namespace
 
 int launch_score_simt(const void* q, const float* q_scale, const float* w, const void* k, const float* k_scale,
                       int dtype, int64_t B, int H_I, int d_I, int64_t L, const int64_t* q_pos, float* scores,

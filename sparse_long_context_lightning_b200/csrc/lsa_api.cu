@@ -176,13 +176,6 @@ int lsa_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx
 
 namespace lsa {
 
-#ifndef LSA_HAVE_TC_ATTN
-size_t sparse_attn_ws_bytes(int64_t, int64_t, int) { return 0; }
-int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
-                       const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, void*, size_t,
-                       cudaStream_t s) {
-  return launch_attn_simt(q, kv, L, idx, idx_ld, count, B, H, scale, out, lse, s);
-}
-#endif
+
 
 }  // namespace lsa

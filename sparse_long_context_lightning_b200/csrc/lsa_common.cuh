@@ -107,4 +107,5 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
                        const int32_t* count, int64_t B, int H, float scale, void* out, float* lse,
                        void* ws, size_t ws_bytes, cudaStream_t s);
 size_t sparse_attn_ws_bytes(int64_t B, int64_t kmax, int H);
+int attn_launches_per_call(int64_t B, int H);
 }  // namespace lsa

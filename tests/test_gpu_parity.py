@@ -323,3 +323,32 @@ def test_pipeline_fp8_recall():
         assert attn_rel_err(out[b], ref) <= ATTN_REL
     print(f"fp8 recall mean {np.mean(rec):.4f} min {np.min(rec):.4f}")
     assert np.mean(rec) >= 0.99
+
+
+def test_sparse_attn_single_split_many_queries():
+    """Enough queries that every query runs as one split (no combine pass)."""
+    L, B, H = 30000, 80, 128
+    kv = S.normal_bf16(S.ST_KV, (L, 576), DEV)
+    q = S.normal_bf16(S.ST_Q, (B, H, 576), DEV)
+    rng = np.random.default_rng(80)
+    counts = [int(c) for c in rng.integers(1, 300, B)]
+    counts[3] = 0
+    kmax = 300
+    idx = torch.full((B, kmax), -1, dtype=torch.int32)
+    for b, c in enumerate(counts):
+        idx[b, :c] = torch.from_numpy(np.sort(rng.choice(L, size=c, replace=False)).astype(np.int32))
+    idx, cnt = idx.to(DEV), torch.tensor(counts, dtype=torch.int32, device=DEV)
+    out = torch.empty(B, H, 512, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(B, H, device=DEV)
+    ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_ATTN, B, L, kmax, H))
+    scale = 1 / math.sqrt(576)
+    lsa.lsa_sparse_attn(q, kv, idx, cnt, scale, out, lse, ws)
+    torch.cuda.synchronize()
+    for b in (0, 3, 17, 79):
+        sel = idx[b, : counts[b]].cpu().numpy()
+        ref, ref_lse = run_oracle_attention(q[b], kv, sel, scale)
+        if counts[b] == 0:
+            assert (out[b] == 0).all() and torch.isneginf(lse[b]).all()
+            continue
+        assert attn_rel_err(out[b], ref) <= ATTN_REL
+        assert np.abs(f64(lse[b]) - ref_lse).max() <= 1e-3
