@@ -107,10 +107,10 @@ class DecodeStep:
         q_I, w = S.index_queries(wl, "cpu")
         k_I = S.index_keys(wl, q_I, device)
         self.q_I, self.w = q_I.to(device), w.to(device)
+        k_I_bf16 = k_I
         if self.fp8:
             self.q_in, self.q_scale = S.quantize_e4m3_rows(self.q_I)
             self.k_in, self.k_scale = S.quantize_e4m3_rows(k_I)
-            del k_I
         else:
             self.q_in, self.q_scale, self.k_in, self.k_scale = self.q_I, None, k_I, None
         self.q_pos = wl.q_pos().to(device)
@@ -124,6 +124,13 @@ class DecodeStep:
         self.out = torch.empty(B, wl.H, wl.d_v, dtype=torch.bfloat16, device=device)
         self.lse = torch.empty(B, wl.H, device=device)
         self.ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_ATTN, B, L, self.kmax, wl.H), device)
+        if self.fp8:
+            # FP8 scan keeps the top 2K, then the exact bf16 re-rank keeps K of them
+            self.k2 = 2 * wl.K
+            self.cand = torch.empty(B, self.k2 + wl.sink + wl.window, dtype=torch.int32, device=device)
+            self.ccnt = torch.empty(B, dtype=torch.int32, device=device)
+            self.k_bf16 = k_I_bf16
+            self.ws_rf = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_REFINE, B, self.cand.shape[1], wl.K), device)
 
     def index(self):
         self.lsa.lsa_index_score(self.q_in, self.w, self.k_in, self.q_pos, self.scores,
@@ -131,7 +138,12 @@ class DecodeStep:
 
     def topk(self):
         wl = self.wl
-        self.lsa.lsa_topk_select(self.scores, wl.L, wl.K, wl.sink, wl.window, self.q_pos, self.idx, self.cnt)
+        if self.fp8:
+            self.lsa.lsa_topk_select(self.scores, wl.L, self.k2, wl.sink, wl.window, self.q_pos, self.cand, self.ccnt)
+            self.lsa.lsa_topk_refine(self.q_I, self.w, self.k_bf16, self.cand, self.ccnt, wl.K, wl.sink, wl.window,
+                                     self.q_pos, self.idx, self.cnt, self.ws_rf)
+        else:
+            self.lsa.lsa_topk_select(self.scores, wl.L, wl.K, wl.sink, wl.window, self.q_pos, self.idx, self.cnt)
 
     def attn(self):
         self.lsa.lsa_sparse_attn(self.q, self.kv, self.idx, self.cnt, self.wl.scale, self.out, self.lse, self.ws)
@@ -145,6 +157,8 @@ def algorithmic_work(wl: S.Workload, counts: np.ndarray, fp8: bool):
     index_flops = 2.0 * B * wl.H_I * wl.d_I * vis
     index_bytes = vis * wl.d_I * idx_elem + (vis * 4 if fp8 else 0) + B * vis * 4 + B * wl.H_I * (wl.d_I * idx_elem + 4)
     topk_bytes = B * vis * 4 + B * (wl.K + wl.sink + wl.window) * 4
+    if fp8:  # top-2K of the FP8 scores, then the bf16 re-rank reads 2K key rows per query
+        topk_bytes += B * 2 * wl.K * (4 + wl.d_I * 2 + 4)
     n_rows = float(counts.sum())
     attn_bytes = n_rows * wl.d_qk * 2 + B * wl.H * wl.d_qk * 2 + B * wl.H * wl.d_v * 2 + B * wl.H * 4 + n_rows * 4
     attn_flops = 2.0 * n_rows * wl.H * (wl.d_qk + wl.d_v)
@@ -190,6 +204,8 @@ def run_gpu(args, rank, world, local_rank):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream()
     launches = dict(LAUNCHES)
+    if step.fp8:
+        launches["topk"] = 4  # top-2K, re-score, top-K of the candidates, assemble
     launches["attn"] = 2 if lsa.lsa_workspace_size(lsa.LSA_OP_ATTN, wl.B, wl.L, step.kmax, wl.H) > 0 else 1  # + combine
 
     def one_step(ev):

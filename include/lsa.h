@@ -48,7 +48,7 @@ typedef enum {
   LSA_FP8_E4M3 = 1  /* OCP e4m3fn codes with one fp32 scale per row (value = code*scale) */
 } lsa_dtype;
 
-typedef enum { LSA_OP_TOPK = 1, LSA_OP_BUCKET = 2, LSA_OP_ATTN = 3 } lsa_op;
+typedef enum { LSA_OP_TOPK = 1, LSA_OP_BUCKET = 2, LSA_OP_ATTN = 3, LSA_OP_REFINE = 4 } lsa_op;
 
 /*
  * lsa_index_score -- lightning-indexer scores.
@@ -93,6 +93,27 @@ int lsa_index_score(const void* q_idx, const float* q_scale, const float* w,
 int lsa_topk_select(const float* scores, int64_t ld, int64_t B, int64_t L, int K,
                     int sink, int window, const int64_t* q_pos,
                     int32_t* idx, int64_t idx_ld, int32_t* count, void* stream);
+
+/*
+ * lsa_topk_refine -- exact re-ranking of a coarse candidate set (second stage after an FP8 pass).
+ *   Source: "LongCat Sparse Attention（LSA）完全拆解", section "机制三：层级索引（HI）": a cheap first stage
+ *   recalls candidate tokens, then the standard token-level score I_{t,s} runs on the recalled tokens
+ *   only and the final arg topK is taken there.  Here the first stage is lsa_index_score in FP8 mode
+ *   followed by lsa_topk_select with K' > K (same sink / window); this call re-scores the K' dynamic
+ *   candidates from the bf16 index queries and keys and keeps the top K of them.
+ *
+ *   cand [B, cand_ld] int32 / cand_count [B]: a row written by lsa_topk_select(..., K', sink, window)
+ *   (sink entries, then the dynamic candidates ascending, then the window entries).
+ *   For each query b: kept = the min(K, #dynamic) dynamic candidates with the largest
+ *   sum_j w[b,j] max(0, q[b,j,:] . k[s,:]) (fp32 from bf16; ties -> lower position);
+ *   idx row = sink entries, kept (ascending), window entries; -1 padded up to K + sink + window.
+ *   q_idx [B, H_I, d_I] bf16, w [B, H_I] fp32, k_idx [L, d_I] bf16; d_I in {32, 64, 128}, H_I <= 64.
+ *   idx_ld >= K + sink + window.  ws: lsa_workspace_size(LSA_OP_REFINE, B, cand_ld, K, 0, 0, 0) bytes.
+ */
+int lsa_topk_refine(const void* q_idx, const float* w, const void* k_idx, int64_t B, int H_I, int d_I,
+                    int64_t L, const int32_t* cand, int64_t cand_ld, const int32_t* cand_count, int K,
+                    int sink, int window, const int64_t* q_pos, int32_t* idx, int64_t idx_ld,
+                    int32_t* count, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * lsa_pool_keys -- bucket / micro-block representatives (computed once per sequence, cached).
@@ -164,6 +185,7 @@ int lsa_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx
  *   op = LSA_OP_TOPK:   0.
  *   op = LSA_OP_BUCKET: (B, L=NB, K=M) -> per-query bucket scores and kept-bucket lists.
  *   op = LSA_OP_ATTN:   (B, L, K=idx_ld, H) -> split-K partial outputs.
+ *   op = LSA_OP_REFINE: (B, L=cand_ld, K) -> re-ranked scores and kept lists.
  *   Returns (size_t)-1 for an unknown op or negative sizes.
  */
 size_t lsa_workspace_size(int op, int64_t B, int64_t L, int K, int H, int sink, int window);

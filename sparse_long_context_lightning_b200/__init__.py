@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "liblsa.so")
 LSA_OK = 0
 LSA_BF16 = 0
 LSA_FP8_E4M3 = 1
-LSA_OP_TOPK, LSA_OP_BUCKET, LSA_OP_ATTN = 1, 2, 3
+LSA_OP_TOPK, LSA_OP_BUCKET, LSA_OP_ATTN, LSA_OP_REFINE = 1, 2, 3, 4
 
 _STATUS = {0: "LSA_OK", -1: "LSA_ERR_INVALID_ARG", -2: "LSA_ERR_UNSUPPORTED", -3: "LSA_ERR_WORKSPACE",
            -4: "LSA_ERR_CUDA", -5: "LSA_ERR_DEVICE_CHECK", -6: "LSA_ERR_TIMEOUT"}
@@ -29,6 +29,8 @@ _P, _I64, _I32, _F32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctype
 SIGNATURES = {
     "lsa_index_score": (_I32, [_P, _P, _P, _P, _P, _I32, _I64, _I32, _I32, _I64, _P, _P, _I64, _P]),
     "lsa_topk_select": (_I32, [_P, _I64, _I64, _I64, _I32, _I32, _I32, _P, _P, _I64, _P, _P]),
+    "lsa_topk_refine": (_I32, [_P, _P, _P, _I64, _I32, _I32, _I64, _P, _I64, _P, _I32, _I32, _I32, _P, _P, _I64, _P,
+                               _P, _SZ, _P]),
     "lsa_pool_keys": (_I32, [_P, _I32, _P, _I64, _I32, _P, _I32, _I64, _P, _P]),
     "lsa_bucket_select": (_I32, [_P, _P, _P, _I32, _I64, _I32, _I32, _P, _I64, _P, _I32, _I32, _I32, _I32, _I64,
                                  _P, _P, _I64, _P, _P, _SZ, _P]),
@@ -107,6 +109,16 @@ def lsa_topk_select(scores, L, K, sink, window, q_pos, idx, count, stream=None):
     st = load_library().lsa_topk_select(_ptr(scores), scores.stride(0), scores.shape[0], L, K, sink, window,
                                         _ptr(q_pos), _ptr(idx), idx.stride(0), _ptr(count), _stream(stream))
     _check("lsa_topk_select", st)
+
+
+def lsa_topk_refine(q_idx, w, k_idx, cand, cand_count, K, sink, window, q_pos, idx, count, ws, stream=None):
+    """Re-rank the dynamic candidates of `cand` (a K' top-K row) with bf16 scores; keep the top K."""
+    B, H_I, d_I = q_idx.shape
+    st = load_library().lsa_topk_refine(_ptr(q_idx), _ptr(w), _ptr(k_idx), B, H_I, d_I, k_idx.shape[0], _ptr(cand),
+                                        cand.stride(0), _ptr(cand_count), K, sink, window, _ptr(q_pos), _ptr(idx),
+                                        idx.stride(0), _ptr(count), _ptr(ws),
+                                        0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("lsa_topk_refine", st)
 
 
 def lsa_pool_keys(k_idx, centroids, bsz, members=None, k_scale=None, stream=None):

@@ -263,9 +263,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       float psum = 0.f;
       #pragma unroll
       for (int c = 0; c < AT_T; c += 2) {
-        const __nv_bfloat162 p2 = __floats2bfloat162_rn(exp2f(z[c] - m_used), exp2f(z[c + 1] - m_used));
-        const float2 back = __bfloat1622float2(p2);
-        psum += back.x + back.y;
+        const float p0 = exp2f(z[c] - m_used), p1 = exp2f(z[c + 1] - m_used);
+        psum += p0 + p1;  // the row sum uses the fp32 probabilities (P . V uses them rounded to bf16)
+        const __nv_bfloat162 p2 = __floats2bfloat162_rn(p0, p1);
         pk[c / 2] = *reinterpret_cast<const uint32_t*>(&p2);
       }
       l = l * alpha + psum;

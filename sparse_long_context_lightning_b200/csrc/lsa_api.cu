@@ -24,6 +24,11 @@ int launch_score_simt(const void* q, const float* q_scale, const float* w, const
 int launch_topk_mode(const float* scores, int64_t ld, int64_t B, int64_t L, int K, int sink, int window,
                      const int64_t* q_pos, int mode, int div, int32_t* idx, int64_t idx_ld, int32_t* count,
                      int64_t kmax, cudaStream_t s);
+size_t refine_ws_bytes(int64_t B, int64_t cand_ld, int K);
+int launch_refine(const void* q, const float* w, const void* k, int64_t B, int H_I, int d_I, int64_t L,
+                  const int32_t* cand, int64_t cand_ld, const int32_t* cand_count, int K, int sink, int window,
+                  const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count, int64_t kmax, void* ws,
+                  cudaStream_t s);
 int launch_attn_simt(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
                      const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, cudaStream_t s);
 
@@ -75,6 +80,7 @@ size_t lsa_workspace_size(int op, int64_t B, int64_t L, int K, int H, int sink, 
       return tot;
     }
     case LSA_OP_ATTN: return sparse_attn_ws_bytes(B, K, H);
+    case LSA_OP_REFINE: return refine_ws_bytes(B, L, K);
     default: return static_cast<size_t>(-1);
   }
 }
@@ -111,6 +117,24 @@ int lsa_topk_select(const float* scores, int64_t ld, int64_t B, int64_t L, int K
   if (L == 0) return LSA_ERR_INVALID_ARG;
   return launch_topk_mode(scores, ld, B, L, K, sink, window, q_pos, 0, 1, idx, idx_ld, count, kmax_full,
                           static_cast<cudaStream_t>(stream));
+}
+
+int lsa_topk_refine(const void* q_idx, const float* w, const void* k_idx, int64_t B, int H_I, int d_I, int64_t L,
+                    const int32_t* cand, int64_t cand_ld, const int32_t* cand_count, int K, int sink, int window,
+                    const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count, void* ws, size_t ws_bytes,
+                    void* stream) {
+  LSA_CHECK_ARG(B >= 0 && L >= 1 && L < (int64_t(1) << 31) && K >= 1 && sink >= 0 && window >= 0);
+  LSA_CHECK_ARG(H_I >= 1 && H_I <= 64 && cand_ld >= 1 && cand_ld < (int64_t(1) << 31));
+  const int64_t kmax_full = static_cast<int64_t>(K) + sink + window;
+  LSA_CHECK_ARG(idx_ld >= kmax_full);
+  if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
+  if (B == 0) return LSA_OK;
+  LSA_CHECK_ARG(B <= 65535);
+  LSA_CHECK_ARG(q_idx && w && k_idx && cand && cand_count && q_pos && idx && count);
+  LSA_CHECK_ARG(aligned16(q_idx) && aligned16(k_idx));
+  if (ws == nullptr || !aligned256(ws) || ws_bytes < refine_ws_bytes(B, cand_ld, K)) return LSA_ERR_WORKSPACE;
+  return launch_refine(q_idx, w, k_idx, B, H_I, d_I, L, cand, cand_ld, cand_count, K, sink, window, q_pos, idx, idx_ld,
+                       count, kmax_full, ws, static_cast<cudaStream_t>(stream));
 }
 
 int lsa_pool_keys(const void* k_idx, int dtype, const float* k_scale, int64_t L, int d_I, const int32_t* members,

@@ -310,19 +310,76 @@ def test_pipeline_bf16(name):
 
 
 def test_pipeline_fp8_recall():
-    """FP8 index mode: top-K recall against the oracle on the bf16 inputs >= 0.99 (mean)."""
-    d, idx, cnt, q, kv, out, lse = _pipeline("decode128k", fp8=True)
-    wl = d.wl
-    ref_bf16 = d.oracle_scores_bf16()
-    rec = []
-    for b in range(d.B):
-        want, _, _ = O.topk_row(ref_bf16[b], int(d.q_pos[b]), wl.K, wl.sink, wl.window)
-        got = idx[b, : cnt[b]]
+    """FP8 index scan + exact bf16 re-rank of the top-2K: recall of the bf16 oracle's top-K >= 0.99 (mean).
+
+    Also checks that the FP8 scan alone is exact for its own inputs: its top-2K equals the oracle's
+    ranking on the e4m3-decoded values up to ties.
+    """
+    wl = S.WORKLOADS["decode128k"]
+    d = Decode(wl, fp8=True)
+    L, B = wl.L, d.B
+    scores = torch.empty(B, L, device=DEV)
+    lsa.lsa_index_score(d.q8, d.w, d.k8, d.q_pos, scores, q_scale=d.q_scale, k_scale=d.k_scale)
+    K2 = 2 * wl.K
+    cand = torch.empty(B, K2 + wl.sink + wl.window, dtype=torch.int32, device=DEV)
+    ccnt = torch.empty(B, dtype=torch.int32, device=DEV)
+    lsa.lsa_topk_select(scores, L, K2, wl.sink, wl.window, d.q_pos, cand, ccnt)
+    kmax = wl.K + wl.sink + wl.window
+    idx = torch.empty(B, kmax, dtype=torch.int32, device=DEV)
+    cnt = torch.empty(B, dtype=torch.int32, device=DEV)
+    ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_REFINE, B, cand.shape[1], wl.K))
+    lsa.lsa_topk_refine(d.q_I, d.w, d.k_I, cand, ccnt, wl.K, wl.sink, wl.window, d.q_pos, idx, cnt, ws)
+    torch.cuda.synchronize()
+    ref_fp8 = d.oracle_scores()          # oracle on the e4m3-decoded inputs
+    ref_bf16 = d.oracle_scores_bf16()    # oracle on the bf16 inputs
+    cand_h, ccnt_h = cand.cpu().numpy(), ccnt.cpu().numpy()
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    rec, raw = [], []
+    for b in range(B):
+        want8, kth8, _ = O.topk_row(ref_fp8[b], int(d.q_pos[b]), K2, wl.sink, wl.window)
+        check_index_sets(cand_h[b], int(ccnt_h[b]), want8, ref_fp8[b], kth8, cand.shape[1])
+        want, kth, _ = O.topk_row(ref_bf16[b], int(d.q_pos[b]), wl.K, wl.sink, wl.window)
+        got = idx_h[b, : cnt_h[b]]
+        assert cnt_h[b] == want.size and np.all(np.diff(got) > 0) and np.all(idx_h[b, cnt_h[b]:] == -1)
         rec.append(np.intersect1d(got, want).size / want.size)
-        ref, _ = run_oracle_attention(q[b], kv, got, wl.scale)
-        assert attn_rel_err(out[b], ref) <= ATTN_REL
-    print(f"fp8 recall mean {np.mean(rec):.4f} min {np.min(rec):.4f}")
+        w1, _, _ = O.topk_row(ref_fp8[b], int(d.q_pos[b]), wl.K, wl.sink, wl.window)
+        raw.append(np.intersect1d(w1, want).size / want.size)
+    print(f"fp8 scan + bf16 re-rank recall mean {np.mean(rec):.4f} min {np.min(rec):.4f}; "
+          f"fp8 scan alone (top-K) recall mean {np.mean(raw):.4f}")
     assert np.mean(rec) >= 0.99
+
+
+def test_topk_refine_exact_on_given_candidates():
+    """Re-rank equals the bf16 oracle's top-K restricted to the candidate set (up to ties)."""
+    wl = S.Workload("rf", L=50000, B=6, H_I=64, d_I=128, K=300, H=16, sink=4, window=64)
+    d = Decode(wl)
+    rng = np.random.default_rng(9)
+    K2 = 700
+    qp = d.q_pos.cpu().numpy()
+    cand = torch.full((wl.B, K2 + 4 + 64), -1, dtype=torch.int32)
+    counts = []
+    for b in range(wl.B):
+        nd = [K2, 10, 0, 299, 300, K2][b]
+        dyn = np.sort(rng.choice(np.arange(4, int(qp[b]) - 63), size=nd, replace=False))
+        row = np.concatenate([np.arange(4), dyn, np.arange(int(qp[b]) - 63, int(qp[b]) + 1)])
+        cand[b, : row.size] = torch.from_numpy(row.astype(np.int32))
+        counts.append(row.size)
+    cand, ccnt = cand.to(DEV), torch.tensor(counts, dtype=torch.int32, device=DEV)
+    kmax = wl.K + 4 + 64
+    idx = torch.empty(wl.B, kmax, dtype=torch.int32, device=DEV)
+    cnt = torch.empty(wl.B, dtype=torch.int32, device=DEV)
+    ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_REFINE, wl.B, cand.shape[1], wl.K))
+    lsa.lsa_topk_refine(d.q_I, d.w, d.k_I, cand, ccnt, wl.K, 4, 64, d.q_pos, idx, cnt, ws)
+    torch.cuda.synchronize()
+    ref = d.oracle_scores()
+    for b in range(wl.B):
+        row = cand[b, : counts[b]].cpu().numpy()
+        dyn = row[4: counts[b] - 64]
+        order = np.argsort(-ref[b, dyn], kind="stable")
+        take = np.sort(dyn[order[: min(wl.K, dyn.size)]])
+        kth = ref[b, take].min() if take.size else 0.0
+        want = np.concatenate([np.arange(4), take, np.arange(int(qp[b]) - 63, int(qp[b]) + 1)])
+        check_index_sets(idx[b].cpu().numpy(), int(cnt[b]), want, ref[b], kth, kmax)
 
 
 def test_sparse_attn_single_split_many_queries():
