@@ -160,6 +160,33 @@ int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, i
                       void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * lsa_bucket_select_noalloc -- lsa_bucket_select for callers that cannot allocate device memory.
+ *   The pages have no counterpart: this is a packaging variant of lsa_bucket_select.
+ *
+ *   Same arguments, layouts and results as lsa_bucket_select, minus ws / ws_bytes.  It is meant for
+ *   callers that may not call cudaMalloc (or any allocating library routine) where they select: a
+ *   plugin inside a host framework that owns every device allocation, a thread that must stay out of
+ *   the CUDA allocator, or a process with no allocation budget left.  The scratch comes from an 8 MiB
+ *   buffer compiled into the library as a __device__ array; the CUDA runtime creates it on every GPU
+ *   that loads the library, and it stays allocated there until the process exits.  The call itself
+ *   allocates nothing.
+ *   - Limit: lsa_workspace_size(LSA_OP_BUCKET, B, NB, M, 0, 0, 0) must be <= 8 MiB (8388608 bytes);
+ *     larger requests return LSA_ERR_WORKSPACE before anything is launched (lsa_last_error() gives
+ *     the sizes).  Flat selection over 156250 buckets fits up to B = 13 queries.
+ *   - Set-up: the first call on a device looks up the buffer's device address (cudaGetSymbolAddress,
+ *     with that device current) and caches it; make that first call before any stream capture.
+ *   - Sharing: every call on a device uses the same buffer, which keeps the last call's contents
+ *     (nothing in it needs clearing: each call writes what it reads).  Calls whose work overlaps on
+ *     the GPU (concurrent streams, or threads without ordering between their streams) race on it;
+ *     order them on one stream.
+ */
+int lsa_bucket_select_noalloc(const void* q_idx, const float* q_scale, const float* w, int dtype,
+                              int64_t B, int H_I, int d_I, const float* centroids, int64_t NB,
+                              const int32_t* members, int bsz, int M, int sink, int window, int64_t L,
+                              const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count,
+                              void* stream);
+
+/*
  * lsa_sparse_attn -- sparse attention over the gathered MLA latent rows (absorbed MQA).
  *   Source: "LongCat Sparse Attention（LSA）完全拆解", section "DSA 基线", u_t = Attn(h_t, {c_s |
  *   s in S_t}) with c_s the MLA latent shared by every query head; the 1152-byte bf16 latent row

@@ -34,6 +34,8 @@ SIGNATURES = {
     "lsa_pool_keys": (_I32, [_P, _I32, _P, _I64, _I32, _P, _I32, _I64, _P, _P]),
     "lsa_bucket_select": (_I32, [_P, _P, _P, _I32, _I64, _I32, _I32, _P, _I64, _P, _I32, _I32, _I32, _I32, _I64,
                                  _P, _P, _I64, _P, _P, _SZ, _P]),
+    "lsa_bucket_select_noalloc": (_I32, [_P, _P, _P, _I32, _I64, _I32, _I32, _P, _I64, _P, _I32, _I32, _I32, _I32,
+                                         _I64, _P, _P, _I64, _P, _P]),
     "lsa_sparse_attn": (_I32, [_P, _P, _I64, _P, _I64, _P, _I64, _I32, _I32, _I32, _F32, _P, _P, _P, _SZ, _P]),
     "lsa_workspace_size": (_SZ, [_I32, _I64, _I64, _I32, _I32, _I32, _I32]),
     "lsa_strerror": (ctypes.c_char_p, [_I32]),
@@ -137,6 +139,17 @@ def lsa_bucket_select(q_idx, w, centroids, members, bsz, M, sink, window, L, q_p
                                           L, _ptr(q_pos), _ptr(idx), idx.stride(0), _ptr(count), _ptr(ws),
                                           0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check("lsa_bucket_select", st)
+
+
+def lsa_bucket_select_noalloc(q_idx, w, centroids, members, bsz, M, sink, window, L, q_pos, idx, count,
+                              stream=None):
+    """lsa_bucket_select with the library's static 8 MiB scratch (for callers that cannot allocate)."""
+    B, H_I, d_I = q_idx.shape
+    st = load_library().lsa_bucket_select_noalloc(_ptr(q_idx), None, _ptr(w), _dtype_code(q_idx), B, H_I, d_I,
+                                                  _ptr(centroids), centroids.shape[0], _ptr(members), bsz, M, sink,
+                                                  window, L, _ptr(q_pos), _ptr(idx), idx.stride(0), _ptr(count),
+                                                  _stream(stream))
+    _check("lsa_bucket_select_noalloc", st)
 
 
 def lsa_sparse_attn(q, kv, idx, count, scale, out, lse=None, ws=None, stream=None):
