@@ -33,13 +33,15 @@ constexpr int AT_THREADS = 192;
 constexpr int AT_T = 32;   // gathered rows per tile
 constexpr int AT_H = 128;  // heads (MMA M)
 constexpr int AT_KBQ_MAX = 5;
-constexpr int AT_STAGES = 5;
+constexpr int AT_STAGES = 4;
 constexpr int AT_Q_BYTES = AT_KBQ_MAX * AT_H * 128;        // 80 KB
 constexpr int AT_KB_BYTES = AT_T * 128;                    // 4 KB: one 64-dim block of a tile
 constexpr int AT_STAGE_BYTES = AT_KBQ_MAX * AT_KB_BYTES;   // 20 KB
 constexpr int AT_P_BYTES = AT_H * 128;                     // 16 KB
-constexpr int AT_SX_FLOATS = AT_T * AT_H;                  // 16 KB
-constexpr int AT_SMEM = 1024 + AT_Q_BYTES + AT_STAGES * AT_STAGE_BYTES + AT_P_BYTES + AT_SX_FLOATS * 4 + 512;
+constexpr int AT_SXP = AT_T + 4;                            // padded row: 16-byte accesses are conflict-free
+constexpr int AT_SX_FLOATS = AT_H * AT_SXP;                 // 18 KB: peer's partial logits [head][row]
+constexpr uint32_t AT_SX_TX = AT_H * AT_T * 4;              // bytes the peer sends per tile
+constexpr int AT_SMEM = 1024 + AT_Q_BYTES + AT_STAGES * AT_STAGE_BYTES + AT_P_BYTES + 2 * AT_SX_FLOATS * 4 + 512;
 constexpr uint32_t TM_O = 0;    // TMEM columns [0, 256): O
 constexpr uint32_t TM_S = 256;  // TMEM columns [256, 320): two S buffers of 32
 constexpr uint32_t IDESC_S = idesc_mma(128, AT_T, 1u, 0u);
@@ -68,16 +70,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
   unsigned char* st_s = q_s + AT_Q_BYTES;
   unsigned char* p_s = st_s + AT_STAGES * AT_STAGE_BYTES;
   float* sx_s = reinterpret_cast<float*>(p_s + AT_P_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sx_s + AT_SX_FLOATS);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sx_s + 2 * AT_SX_FLOATS);  // two receive buffers
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + AT_STAGES;
   uint64_t* s_full = kv_empty + AT_STAGES;
   uint64_t* s_empty = s_full + 2;
   uint64_t* p_full = s_empty + 2;
   uint64_t* pv_done = p_full + 1;
-  uint64_t* sx_full = pv_done + 1;
-  uint64_t* sx_empty = sx_full + 1;
-  uint64_t* q_full = sx_empty + 1;
+  uint64_t* sx_full = pv_done + 1;  // [2]: the peer's partial logits of tile i landed in buffer i & 1
+  uint64_t* q_full = sx_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(q_full + 1);
   __shared__ int abort_flag;
 
@@ -105,11 +106,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     }
     mbar_init(p_full, 4);
     mbar_init(pv_done, 1);
-    mbar_init(sx_full, AT_H);   // one arrival per peer softmax thread
-    mbar_init(sx_empty, AT_H);
+    mbar_init(&sx_full[0], 1);
+    mbar_init(&sx_full[1], 1);
     mbar_init(q_full, 1);
     abort_flag = 0;
     fence_mbar_init();
+    // arm both receive buffers for their first tile: each phase completes when the peer's bytes land
+    mbar_expect_tx(&sx_full[0], AT_SX_TX);
+    mbar_expect_tx(&sx_full[1], AT_SX_TX);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
@@ -212,7 +216,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const uint32_t peer_sx = mapa(smem_u32(sx_s), peer);
     const uint32_t peer_sx_full = mapa(smem_u32(sx_full), peer);
-    const uint32_t peer_sx_empty = mapa(smem_u32(sx_empty), peer);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
@@ -229,27 +232,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[sb]);
-      // send my partial logits to the peer, then take the peer's
-      if (!mbar_wait(sx_empty, (i & 1) ^ 1)) {
+      // send my partial logits to the peer's receive buffer sb (st.async signals its mbarrier), then take the
+      // peer's.  Buffer sb is free: the peer read tile i-2 from it before it sent tile i-1, which this CTA
+      // received before getting here.
+      {
+        const uint32_t dst = peer_sx + static_cast<uint32_t>((sb * AT_SX_FLOATS + h * AT_SXP) * 4);
+        const uint32_t bar = peer_sx_full + sb * 8;
+        #pragma unroll
+        for (int c = 0; c < AT_T; c += 4)
+          st_async_v4(dst + c * 4, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), __uint_as_float(sr[c + 2]),
+                      __uint_as_float(sr[c + 3]), bar);
+      }
+      if (!mbar_wait_cluster(&sx_full[sb], (i >> 1) & 1)) {
         ok = false;
         break;
       }
+      const float4* sxrow = reinterpret_cast<const float4*>(sx_s + sb * AT_SX_FLOATS + h * AT_SXP);
+      float sp[AT_T];
       #pragma unroll
-      for (int c = 0; c < AT_T; ++c) st_cluster_f32(peer_sx + static_cast<uint32_t>((c * AT_H + h) * 4), __uint_as_float(sr[c]));
-      mbar_arrive_cluster(peer_sx_full);
-      if (!mbar_wait_cluster(sx_full, i & 1)) {
-        ok = false;
-        break;
+      for (int c = 0; c < AT_T / 4; ++c) {
+        const float4 v = sxrow[c];
+        sp[4 * c] = v.x;
+        sp[4 * c + 1] = v.y;
+        sp[4 * c + 2] = v.z;
+        sp[4 * c + 3] = v.w;
       }
+      // re-arm buffer sb for tile i+2 (before this CTA sends tile i+1, so before the peer can send i+2)
+      if (tid == 64 && i + 2 < ntiles) mbar_expect_tx(&sx_full[sb], AT_SX_TX);
       float z[AT_T];
       float mt = -INFINITY;
       #pragma unroll
       for (int c = 0; c < AT_T; ++c) {
-        const float sfull = __uint_as_float(sr[c]) + sx_s[c * AT_H + h];
+        const float sfull = __uint_as_float(sr[c]) + sp[c];
         z[c] = c < nvalid ? sfull * a.scale_log2 : -INFINITY;
         mt = fmaxf(mt, z[c]);
       }
-      mbar_arrive_cluster(peer_sx_empty);
       float alpha = 1.f;
       bool resc = false;
       if (i == 0) {

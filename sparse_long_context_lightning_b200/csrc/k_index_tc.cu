@@ -23,7 +23,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int IX_THREADS = 320;
+constexpr int IX_THREADS = 576;  // producer, MMA, 16 epilogue warps
 
 // Set (never cleared by the kernel) when a bounded wait of this kernel gave up.
 __device__ int g_index_tc_timeout;
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 8);
+      mbar_init(&tempty[i], 16);
     }
     mbar_init(qfull, 1);
     abort_flag = 0;
@@ -168,11 +168,12 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------------ epilogue (warps 2..9)
+    // ------------------------------------------------------------------ epilogue (warps 2..17)
+    // warp e handles TMEM lanes 32*(warp % 4) .. +31 (its keys) and chunk columns [64*(e/4), +64)
     const int ew = warp - 2;
-    const int quarter = warp & 3;        // TMEM lanes this warp may access
-    const int half = ew >> 2;            // column half of the chunk
-    const int nq_half = (IX_CHUNK_N / 2) / a.H_I;
+    const int quarter = warp & 3;
+    const int col0 = (ew >> 2) * 64;
+    const int nq = 64 / a.H_I;  // queries in this warp's 64 columns (1 or 2)
     for (int i = 0; i < n_my; ++i) {
       const int buf = i & 1;
       if (!mbar_wait(&tfull[buf], (i >> 1) & 1)) {
@@ -180,28 +181,32 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int s = (t_begin + i) * IX_TILE_M + quarter * 32 + lane;
-      const float ks = (FP8 && s < a.L) ? a.k_scale[s] : 1.f;
-      for (int qi = 0; qi < nq_half; ++qi) {
-        const int col0 = half * (IX_CHUNK_N / 2) + qi * a.H_I;
-        float acc = 0.f;
-        for (int j0 = 0; j0 < a.H_I; j0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * IX_CHUNK_N + col0 + j0, r);
-          tmem_ld_wait();
-          const float* wv = wsm + col0 + j0;
-          #pragma unroll
-          for (int c = 0; c < 32; ++c) acc = fmaf(wv[c], fmaxf(__uint_as_float(r[c]), 0.f), acc);
-        }
-        const int b = b0 + col0 / a.H_I;
-        if (b < a.B && s < a.L) {
-          const float v = (static_cast<int64_t>(s) > a.q_pos[b]) ? -INFINITY : acc * ks;
-          a.scores[static_cast<int64_t>(b) * a.ld + s] = v;
-        }
-      }
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * IX_CHUNK_N + col0;
+      uint32_t r0[32], r1[32];
+      tmem_ld32(taddr, r0);
+      tmem_ld32(taddr + 32, r1);
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (lane == 0) mbar_arrive(&tempty[buf]);  // the accumulator columns are in registers now
+      const int s = (t_begin + i) * IX_TILE_M + quarter * 32 + lane;
+      const float ks = (FP8 && s < a.L) ? a.k_scale[s] : 1.f;
+      const float* wv = wsm + col0;
+      float acc0 = 0.f, acc1 = 0.f;
+      #pragma unroll
+      for (int c = 0; c < 32; ++c) acc0 = fmaf(wv[c], fmaxf(__uint_as_float(r0[c]), 0.f), acc0);
+      #pragma unroll
+      for (int c = 0; c < 32; ++c) acc1 = fmaf(wv[32 + c], fmaxf(__uint_as_float(r1[c]), 0.f), acc1);
+      if (s < a.L) {
+        if (nq == 1) {
+          const int b = b0 + col0 / a.H_I;
+          if (b < a.B) a.scores[static_cast<int64_t>(b) * a.ld + s] = (s > a.q_pos[b]) ? -INFINITY : (acc0 + acc1) * ks;
+        } else {
+          const int bA = b0 + col0 / a.H_I, bB = bA + 1;
+          if (bA < a.B) a.scores[static_cast<int64_t>(bA) * a.ld + s] = (s > a.q_pos[bA]) ? -INFINITY : acc0 * ks;
+          if (bB < a.B) a.scores[static_cast<int64_t>(bB) * a.ld + s] = (s > a.q_pos[bB]) ? -INFINITY : acc1 * ks;
+        }
+      }
     }
   }
   tc_fence_before();

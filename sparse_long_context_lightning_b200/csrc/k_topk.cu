@@ -19,7 +19,7 @@
 namespace lsa {
 namespace {
 
-constexpr int TK_THREADS = 1024;
+constexpr int TK_THREADS = 512;
 constexpr int TK_WARPS = TK_THREADS / 32;
 constexpr int TK_BINS = 4096;
 constexpr int TK_CAP = 1024;
@@ -92,7 +92,7 @@ __device__ uint32_t block_sum_u32(uint32_t v, uint32_t* scratch) {
   return t;
 }
 
-__global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
+__global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
   extern __shared__ __align__(16) unsigned char dyn[];
   __shared__ TopkSmem sm;
   cg::cluster_group cluster = cg::this_cluster();
@@ -488,7 +488,7 @@ int launch_topk_mode(const float* scores, int64_t ld, int64_t B, int64_t L, int 
                      int64_t kmax, cudaStream_t s) {
   if (B == 0) return LSA_OK;
   // cluster size: smallest power of two whose chunk fits the shared-memory cache, <= 16
-  const int64_t cache_elems = 40 * 1024;  // 160 KB of fp32 scores per CTA
+  const int64_t cache_elems = 20 * 1024;  // 80 KB of fp32 scores per CTA (two CTAs per SM)
   int C = 1;
   while (C < TK_MAXC && cdiv(L, C) > cache_elems) C *= 2;
   while (C < 8 && cdiv(L, C) > 16384) C *= 2;  // spread mid-size rows over more SMs

@@ -171,6 +171,13 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t caddr, float a, float b, 
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
+// asynchronous 16-byte store into a peer CTA's shared memory that signals the peer's mbarrier
+// (complete_tx) when the bytes have landed; the mbarrier side has release semantics at cluster scope
+__device__ __forceinline__ void st_async_v4(uint32_t caddr, float a, float b, float c, float d, uint32_t cbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+               ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(cbar)
+               : "memory");
+}
 // arrive (release at cluster scope) on an mbarrier given by its shared::cluster address
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
