@@ -149,7 +149,7 @@ int lsa_pool_keys(const void* k_idx, int dtype, const float* k_scale, int64_t L,
  *                 window, restricted to [0, q_pos]; -1 padded up to idx_ld.
  *   q_idx [B, H_I, d_I] bf16 (dtype must be LSA_BF16), w [B, H_I] fp32, centroids [NB, d_I]
  *   fp32, members int32 [NB, bsz] or NULL.  idx int32 [B, idx_ld] with
- *   idx_ld >= M*bsz + (bsz-1) + sink + window; count int32 [B].
+ *   idx_ld >= M*bsz + sink + window (+ bsz-1 for the micro-block tail); count int32 [B].
  *   1 <= M <= 1024, M*bsz + bsz + sink + window <= 8192.
  *   ws: lsa_workspace_size(LSA_OP_BUCKET, B, NB, M, 0, 0, 0) bytes.
  */

@@ -20,7 +20,8 @@ namespace lsa {
 namespace {
 
 constexpr int TK_THREADS = 512;
-constexpr int TK_WARPS = TK_THREADS / 32;
+constexpr int TK_WARPS = TK_THREADS / 32;  // <= 32: per-warp arrays are reduced by one warp, lane < TK_WARPS
+static_assert(TK_WARPS <= 32, "one warp reduces the per-warp partials");
 constexpr int TK_BINS = 4096;
 constexpr int TK_CAP = 1024;
 constexpr int TK_MAXC = 16;
@@ -184,8 +185,8 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
     }
     __syncthreads();
     if (warp == 0) {
-      lo = warp_min(sm.wf0[lane]);
-      hi = warp_max(sm.wf1[lane]);
+      lo = warp_min(lane < TK_WARPS ? sm.wf0[lane] : INFINITY);
+      hi = warp_max(lane < TK_WARPS ? sm.wf1[lane] : -INFINITY);
       if (lane < C) {
         *cluster.map_shared_rank(&sm.fmin[r], lane) = lo;
         *cluster.map_shared_rank(&sm.fmax[r], lane) = hi;
@@ -367,8 +368,8 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
       }
       __syncthreads();
       if (warp == 0) {
-        lo = sm.wa[lane];
-        hi = sm.wb[lane];
+        lo = lane < TK_WARPS ? sm.wa[lane] : 0xFFFFFFFFu;
+        hi = lane < TK_WARPS ? sm.wb[lane] : 0u;
         #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
           lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
@@ -423,8 +424,8 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
   }
   __syncthreads();
   if (warp == 0) {
-    const uint32_t g = warp_sum_u32(sm.wa[lane]);
-    const uint32_t e = warp_sum_u32(sm.wb[lane]);
+    const uint32_t g = warp_sum_u32(lane < TK_WARPS ? sm.wa[lane] : 0u);
+    const uint32_t e = warp_sum_u32(lane < TK_WARPS ? sm.wb[lane] : 0u);
     if (lane < C) {
       *cluster.map_shared_rank(&sm.cgt[r], lane) = g;
       *cluster.map_shared_rank(&sm.ceq[r], lane) = e;

@@ -156,7 +156,8 @@ int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, i
   LSA_CHECK_ARG(B >= 0 && NB >= 1 && NB < (int64_t(1) << 31) && bsz >= 1 && M >= 1 && M <= 1024);
   LSA_CHECK_ARG(sink >= 0 && window >= 0 && L >= 1 && H_I >= 1 && H_I <= 64);
   LSA_CHECK_ARG(static_cast<int64_t>(M) * bsz + bsz + sink + window <= 8192);
-  const int64_t kmax_full = static_cast<int64_t>(M) * bsz + (bsz - 1) + sink + window;
+  // the incomplete tail block exists only in micro-block mode
+  const int64_t kmax_full = static_cast<int64_t>(M) * bsz + (members ? 0 : bsz - 1) + sink + window;
   LSA_CHECK_ARG(idx_ld >= kmax_full);
   if (dtype != LSA_BF16 || q_scale != nullptr) return LSA_ERR_UNSUPPORTED;
   if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
