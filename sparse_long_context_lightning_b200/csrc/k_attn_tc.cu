@@ -136,11 +136,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
           tma_load_2d(q_s + kb * AT_H * 128, &tm_q, q_full, 256 * static_cast<int>(r) + 64 * kb, b * AT_H);
       }
       const int32_t* rowidx = a.idx + static_cast<int64_t>(b) * a.idx_ld + row0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int st = i % AT_STAGES;
+      auto load_idx = [&](int i) {
         const int rr = i * AT_T + lane;
         int v = rr < nrows ? rowidx[rr] : 0;
-        v = v < 0 ? 0 : (v >= a.L ? a.L - 1 : v);
+        return v < 0 ? 0 : (v >= a.L ? a.L - 1 : v);
+      };
+      int v_next = load_idx(0);  // the next tile's row indices are fetched one tile ahead
+      for (int i = 0; i < ntiles; ++i) {
+        const int st = i % AT_STAGES;
+        const int v = v_next;
+        if (i + 1 < ntiles) v_next = load_idx(i + 1);
         if (!mbar_wait(&kv_empty[st], ((i / AT_STAGES) & 1) ^ 1) || abort_flag) {
           if (lane == 0) {
             atomicExch(&g_attn_tc_timeout, 1);
@@ -150,17 +155,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         }
         unsigned char* dst = st_s + st * AT_STAGE_BYTES;
         if (lane == 0) mbar_expect_tx(&kv_full[st], kbq * AT_KB_BYTES);
-        #pragma unroll
-        for (int g = 0; g < AT_T / 4; ++g) {
-          const int y0 = __shfl_sync(0xffffffffu, v, 4 * g + 0);
-          const int y1 = __shfl_sync(0xffffffffu, v, 4 * g + 1);
-          const int y2 = __shfl_sync(0xffffffffu, v, 4 * g + 2);
-          const int y3 = __shfl_sync(0xffffffffu, v, 4 * g + 3);
-          if (lane == 0) {
-            for (int kb = 0; kb < kbq; ++kb)
-              tma_gather4(dst + kb * AT_KB_BYTES + g * 512, &tm_kv, &kv_full[st], 256 * static_cast<int>(r) + 64 * kb,
-                          y0, y1, y2, y3);
-          }
+        __syncwarp();
+        // lane g < 8 gathers rows 4g..4g+3 of the tile (all K-blocks of this CTA's slice)
+        const int g = lane & 7;
+        const int y0 = __shfl_sync(0xffffffffu, v, 4 * g + 0);
+        const int y1 = __shfl_sync(0xffffffffu, v, 4 * g + 1);
+        const int y2 = __shfl_sync(0xffffffffu, v, 4 * g + 2);
+        const int y3 = __shfl_sync(0xffffffffu, v, 4 * g + 3);
+        if (lane < AT_T / 4) {
+          for (int kb = 0; kb < kbq; ++kb)
+            tma_gather4(dst + kb * AT_KB_BYTES + g * 512, &tm_kv, &kv_full[st], 256 * static_cast<int>(r) + 64 * kb, y0,
+                        y1, y2, y3);
         }
         __syncwarp();
       }
@@ -218,31 +223,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     const uint32_t peer_sx_full = mapa(smem_u32(sx_full), peer);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int i = 0; i < ntiles; ++i) {
-      const int sb = i & 1;
-      const int nvalid = min(AT_T, nrows - i * AT_T);
-      if (!mbar_wait(&s_full[sb], (i >> 1) & 1)) {
-        ok = false;
-        break;
-      }
+    // read S(j) from TMEM, free the buffer, and send it to the peer's receive buffer j & 1
+    auto fetch_and_send = [&](int j, uint32_t (&sr)[32]) -> bool {
+      const int sb = j & 1;
+      if (!mbar_wait(&s_full[sb], (j >> 1) & 1)) return false;
       tc_fence_after();
-      uint32_t sr[32];
       tmem_ld32(trow + TM_S + sb * AT_T, sr);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[sb]);
-      // send my partial logits to the peer's receive buffer sb (st.async signals its mbarrier), then take the
-      // peer's.  Buffer sb is free: the peer read tile i-2 from it before it sent tile i-1, which this CTA
-      // received before getting here.
-      {
-        const uint32_t dst = peer_sx + static_cast<uint32_t>((sb * AT_SX_FLOATS + h * AT_SXP) * 4);
-        const uint32_t bar = peer_sx_full + sb * 8;
-        #pragma unroll
-        for (int c = 0; c < AT_T; c += 4)
-          st_async_v4(dst + c * 4, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), __uint_as_float(sr[c + 2]),
-                      __uint_as_float(sr[c + 3]), bar);
-      }
+      const uint32_t dst = peer_sx + static_cast<uint32_t>((sb * AT_SX_FLOATS + h * AT_SXP) * 4);
+      const uint32_t bar = peer_sx_full + sb * 8;
+      #pragma unroll
+      for (int c = 0; c < AT_T; c += 4)
+        st_async_v4(dst + c * 4, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), __uint_as_float(sr[c + 2]),
+                    __uint_as_float(sr[c + 3]), bar);
+      return true;
+    };
+    uint32_t sr[32];
+    if (ntiles > 0) ok = fetch_and_send(0, sr);
+    for (int i = 0; ok && i < ntiles; ++i) {
+      const int sb = i & 1;
+      const int nvalid = min(AT_T, nrows - i * AT_T);
+      // the peer's partial logits of tile i.  Its receive buffer for tile i+1 is free: the peer read tile
+      // i-1 from it before sending tile i, which has arrived.
       if (!mbar_wait_cluster(&sx_full[sb], (i >> 1) & 1)) {
         ok = false;
         break;
@@ -259,6 +264,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       }
       // re-arm buffer sb for tile i+2 (before this CTA sends tile i+1, so before the peer can send i+2)
       if (tid == 64 && i + 2 < ntiles) mbar_expect_tx(&sx_full[sb], AT_SX_TX);
+      uint32_t sr_next[32];
+      if (i + 1 < ntiles && !fetch_and_send(i + 1, sr_next)) {
+        ok = false;
+        break;
+      }
       float z[AT_T];
       float mt = -INFINITY;
       #pragma unroll
@@ -315,6 +325,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
+      #pragma unroll
+      for (int c = 0; c < 32; ++c) sr[c] = sr_next[c];
     }
     if (!ok) {
       atomicExch(&g_attn_tc_timeout, 1);

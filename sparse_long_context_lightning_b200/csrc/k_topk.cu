@@ -15,6 +15,7 @@
 // the selected positions in ascending order.  All cross-CTA synchronisation is the hardware
 // cluster barrier: no spin-waits, no global atomics, no scratch memory.
 #include "lsa_common.cuh"
+#include "sm100.cuh"
 
 namespace lsa {
 namespace {
@@ -67,6 +68,7 @@ struct TopkSmem {
   // broadcast slots (written by the CTA that decides)
   uint32_t b_bin, b_above, b_count;
   uint32_t b_T, b_need_eq;
+  uint64_t load_bar;
 };
 
 struct Row {
@@ -153,12 +155,26 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
   const float* grow = a.scores + static_cast<int64_t>(b) * a.ld;
   Row row;
   if (a.cached) {
+    // one bulk asynchronous copy of the aligned part of the chunk, the last < 4 scores by plain loads
     float* cache = reinterpret_cast<float*>(dyn);
     const int lend = min(c1, chi);
     const int nvec = max(0, (lend - c0) / 4);
-    const float4* g4 = reinterpret_cast<const float4*>(grow + c0);
-    for (int i = tid; i < nvec; i += TK_THREADS) reinterpret_cast<float4*>(cache)[i] = __ldcs(g4 + i);
+    if (tid == 0) {
+      sm100::mbar_init(&sm.load_bar, 1);
+      sm100::fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+      if (nvec > 0) {
+        sm100::mbar_expect_tx(&sm.load_bar, static_cast<uint32_t>(nvec) * 16u);
+        sm100::bulk_load(cache, grow + c0, static_cast<uint32_t>(nvec) * 16u, &sm.load_bar);
+      } else {
+        sm100::mbar_arrive(&sm.load_bar);
+      }
+    }
     for (int s = c0 + nvec * 4 + tid; s < lend; s += TK_THREADS) cache[s - c0] = grow[s];
+    // bounded wait (the copy is in bounds by construction); on give-up the row is left as the copy made it
+    sm100::mbar_wait(&sm.load_bar, 0);
     row.src = cache;
     row.base = c0;
     __syncthreads();

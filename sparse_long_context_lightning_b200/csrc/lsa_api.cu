@@ -179,8 +179,9 @@ int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, i
   // top-M buckets: all NB ranked (explicit members) or the complete visible micro-blocks
   st = launch_topk_mode(bscores, ldn, B, NB, M, 0, 0, q_pos, members ? 1 : 2, bsz, kept, M, kcnt, M, s);
   if (st != LSA_OK) return st;
+  // rows are -1 padded up to idx_ld
   return launch_bucket_expand(kept, M, kcnt, members, bsz, sink, window, members ? 0 : bsz, q_pos, B, idx, idx_ld,
-                              count, kmax_full, s);
+                              count, idx_ld, s);
 }
 
 int lsa_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
