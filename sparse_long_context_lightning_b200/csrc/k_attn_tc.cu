@@ -136,16 +136,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
           tma_load_2d(q_s + kb * AT_H * 128, &tm_q, q_full, 256 * static_cast<int>(r) + 64 * kb, b * AT_H);
       }
       const int32_t* rowidx = a.idx + static_cast<int64_t>(b) * a.idx_ld + row0;
-      auto load_idx = [&](int i) {
+      // raw row indices are loaded two tiles ahead and only clamped when used, so the loads stay in
+      // flight while the producer waits for a free stage
+      auto load_idx = [&](int i) -> int {
         const int rr = i * AT_T + lane;
-        int v = rr < nrows ? rowidx[rr] : 0;
-        return v < 0 ? 0 : (v >= a.L ? a.L - 1 : v);
+        return rr < nrows ? rowidx[rr] : 0;
       };
-      int v_next = load_idx(0);  // the next tile's row indices are fetched one tile ahead
+      int v_a = load_idx(0);
+      int v_b = ntiles > 1 ? load_idx(1) : 0;
       for (int i = 0; i < ntiles; ++i) {
         const int st = i % AT_STAGES;
-        const int v = v_next;
-        if (i + 1 < ntiles) v_next = load_idx(i + 1);
+        const int v_raw = v_a;
+        v_a = v_b;
+        if (i + 2 < ntiles) v_b = load_idx(i + 2);
         if (!mbar_wait(&kv_empty[st], ((i / AT_STAGES) & 1) ^ 1) || abort_flag) {
           if (lane == 0) {
             atomicExch(&g_attn_tc_timeout, 1);
@@ -158,6 +161,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         __syncwarp();
         // lane g < 8 gathers rows 4g..4g+3 of the tile (all K-blocks of this CTA's slice)
         const int g = lane & 7;
+        const int v = v_raw < 0 ? 0 : (v_raw >= a.L ? a.L - 1 : v_raw);
         const int y0 = __shfl_sync(0xffffffffu, v, 4 * g + 0);
         const int y1 = __shfl_sync(0xffffffffu, v, 4 * g + 1);
         const int y2 = __shfl_sync(0xffffffffu, v, 4 * g + 2);
