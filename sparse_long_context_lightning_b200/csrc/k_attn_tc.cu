@@ -38,10 +38,10 @@ constexpr int AT_Q_BYTES = AT_KBQ_MAX * AT_H * 128;        // 80 KB
 constexpr int AT_KB_BYTES = AT_T * 128;                    // 4 KB: one 64-dim block of a tile
 constexpr int AT_STAGE_BYTES = AT_KBQ_MAX * AT_KB_BYTES;   // 20 KB
 constexpr int AT_P_BYTES = AT_H * 128;                     // 16 KB
-constexpr int AT_SXP = AT_T + 4;                            // padded row: 16-byte accesses are conflict-free
-constexpr int AT_SX_FLOATS = AT_H * AT_SXP;                 // 18 KB: peer's partial logits [head][row]
+constexpr int AT_SX_FLOATS = AT_H * AT_T;                   // 16 KB: partial logits [head][row], 16-byte chunks
+                                                            // of a row swizzled by (head & 7)
 constexpr uint32_t AT_SX_TX = AT_H * AT_T * 4;              // bytes the peer sends per tile
-constexpr int AT_SMEM = 1024 + AT_Q_BYTES + AT_STAGES * AT_STAGE_BYTES + AT_P_BYTES + 2 * AT_SX_FLOATS * 4 + 512;
+constexpr int AT_SMEM = 1024 + AT_Q_BYTES + AT_STAGES * AT_STAGE_BYTES + AT_P_BYTES + 3 * AT_SX_FLOATS * 4 + 512;
 constexpr uint32_t TM_O = 0;    // TMEM columns [0, 256): O
 constexpr uint32_t TM_S = 256;  // TMEM columns [256, 320): two S buffers of 32
 constexpr uint32_t IDESC_S = idesc_mma(128, AT_T, 1u, 0u);
@@ -70,7 +70,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
   unsigned char* st_s = q_s + AT_Q_BYTES;
   unsigned char* p_s = st_s + AT_STAGES * AT_STAGE_BYTES;
   float* sx_s = reinterpret_cast<float*>(p_s + AT_P_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sx_s + 2 * AT_SX_FLOATS);  // two receive buffers
+  float* sx_out = sx_s + 2 * AT_SX_FLOATS;  // staging of this CTA's partial logits for the bulk copy
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sx_out + AT_SX_FLOATS);  // after two receive buffers + staging
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + AT_STAGES;
   uint64_t* s_full = kv_empty + AT_STAGES;
@@ -176,42 +177,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
+    // S = Q C^T runs two tiles ahead of O += P V, so the softmax never waits for its next logits
     if (ntiles > 0 && lane == 0) {
       bool ok = mbar_wait(q_full, 0);
       const uint32_t q_addr = smem_u32(q_s);
       const uint32_t p_addr = smem_u32(p_s);
-      for (int i = 0; ok && i <= ntiles; ++i) {
-        if (i < ntiles) {
-          const int st = i % AT_STAGES, sb = i & 1;
-          if (!mbar_wait(&kv_full[st], (i / AT_STAGES) & 1) || !mbar_wait(&s_empty[sb], ((i >> 1) & 1) ^ 1)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t s_addr = smem_u32(st_s + st * AT_STAGE_BYTES);
-          for (int kb = 0; kb < kbq; ++kb) {
-            #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16(tmem + TM_S + sb * AT_T, desc_sw128(q_addr + kb * AT_H * 128 + kk * 32),
-                      desc_sw128(s_addr + kb * AT_KB_BYTES + kk * 32), IDESC_S, (kb | kk) != 0);
-          }
-          mma_commit(&s_full[sb]);
-        }
-        if (i >= 1) {
-          const int j = i - 1, stj = j % AT_STAGES;
-          if (!mbar_wait(p_full, j & 1)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(st_s + stj * AT_STAGE_BYTES);
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % AT_STAGES, sb = j & 1;
+        if (!mbar_wait(&kv_full[st], (j / AT_STAGES) & 1) || !mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1)) return false;
+        tc_fence_after();
+        const uint32_t s_addr = smem_u32(st_s + st * AT_STAGE_BYTES);
+        for (int kb = 0; kb < kbq; ++kb) {
           #pragma unroll
-          for (int kk = 0; kk < AT_T / 16; ++kk)
-            mma_f16(tmem + TM_O, desc_sw128(p_addr + kk * 32), desc_sw128_mn(v_addr + kk * 16 * 128, AT_KB_BYTES, 1024),
-                    IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&kv_empty[stj]);
-          mma_commit(pv_done);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem + TM_S + sb * AT_T, desc_sw128(q_addr + kb * AT_H * 128 + kk * 32),
+                    desc_sw128(s_addr + kb * AT_KB_BYTES + kk * 32), IDESC_S, (kb | kk) != 0);
         }
+        mma_commit(&s_full[sb]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int stj = j % AT_STAGES;
+        if (!mbar_wait(p_full, j & 1)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(st_s + stj * AT_STAGE_BYTES);
+        #pragma unroll
+        for (int kk = 0; kk < AT_T / 16; ++kk)
+          mma_f16(tmem + TM_O, desc_sw128(p_addr + kk * 32), desc_sw128_mn(v_addr + kk * 16 * 128, AT_KB_BYTES, 1024),
+                  IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&kv_empty[stj]);
+        mma_commit(pv_done);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      if (ok && ntiles > 1) ok = issue_s(1);
+      for (int i = 0; ok && i < ntiles; ++i) {
+        if (i + 2 < ntiles && !issue_s(i + 2)) ok = false;
+        if (ok && !issue_pv(i)) ok = false;
       }
       if (!ok) {
         atomicExch(&g_attn_tc_timeout, 1);
@@ -227,7 +229,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     const uint32_t peer_sx_full = mapa(smem_u32(sx_full), peer);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    // read S(j) from TMEM, free the buffer, and send it to the peer's receive buffer j & 1
+    // read S(j) from TMEM, free the buffer, stage this warp's 32 rows in shared memory and send them to the
+    // peer's receive buffer j & 1 as one 4 KB bulk copy per warp (all four complete on the peer's mbarrier)
     auto fetch_and_send = [&](int j, uint32_t (&sr)[32]) -> bool {
       const int sb = j & 1;
       if (!mbar_wait(&s_full[sb], (j >> 1) & 1)) return false;
@@ -235,14 +238,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       tmem_ld32(trow + TM_S + sb * AT_T, sr);
       tmem_ld_wait();
       tc_fence_before();
+      // this warp's staging rows are free once its previous bulk copy has read them
+      if (lane == 0) bulk_wait_read0();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[sb]);
-      const uint32_t dst = peer_sx + static_cast<uint32_t>((sb * AT_SX_FLOATS + h * AT_SXP) * 4);
-      const uint32_t bar = peer_sx_full + sb * 8;
+      float4* row = reinterpret_cast<float4*>(sx_out + h * AT_T);
       #pragma unroll
-      for (int c = 0; c < AT_T; c += 4)
-        st_async_v4(dst + c * 4, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), __uint_as_float(sr[c + 2]),
-                    __uint_as_float(sr[c + 3]), bar);
+      for (int c = 0; c < AT_T / 4; ++c)
+        row[c ^ (h & 7)] = make_float4(__uint_as_float(sr[4 * c]), __uint_as_float(sr[4 * c + 1]),
+                                       __uint_as_float(sr[4 * c + 2]), __uint_as_float(sr[4 * c + 3]));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t off = static_cast<uint32_t>((sb * AT_SX_FLOATS + q4 * 32 * AT_T) * 4);
+        bulk_store_peer(peer_sx + off, sx_out + q4 * 32 * AT_T, 32 * AT_T * 4, peer_sx_full + sb * 8);
+        bulk_commit();
+      }
       return true;
     };
     uint32_t sr[32];
@@ -256,11 +267,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         ok = false;
         break;
       }
-      const float4* sxrow = reinterpret_cast<const float4*>(sx_s + sb * AT_SX_FLOATS + h * AT_SXP);
+      const float4* sxrow = reinterpret_cast<const float4*>(sx_s + sb * AT_SX_FLOATS + h * AT_T);
       float sp[AT_T];
       #pragma unroll
       for (int c = 0; c < AT_T / 4; ++c) {
-        const float4 v = sxrow[c];
+        const float4 v = sxrow[c ^ (h & 7)];
         sp[4 * c] = v.x;
         sp[4 * c + 1] = v.y;
         sp[4 * c + 2] = v.z;
@@ -337,6 +348,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       abort_flag = 1;
     }
     // ---- epilogue
+    if (lane == 0) bulk_wait_read0();  // this warp's last outgoing copy has read its staging rows
     const bool have = ok && ntiles > 0 && mbar_wait(pv_done, (ntiles - 1) & 1);
     tc_fence_after();
     const int64_t orow = static_cast<int64_t>(b) * AT_H + h;

@@ -75,6 +75,20 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// bulk copy own shared memory -> a peer CTA's shared memory, completing on the peer's mbarrier
+// (caddr_dst / caddr_bar are shared::cluster addresses from mapa)
+__device__ __forceinline__ void bulk_store_peer(uint32_t caddr_dst, const void* src, uint32_t bytes, uint32_t caddr_bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(caddr_dst), "r"(smem_u32(src)), "r"(bytes), "r"(caddr_bar)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until the source reads of every committed bulk copy of this thread are done
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------------------------------------
 // tcgen05
 // ---------------------------------------------------------------------------------------------
