@@ -47,6 +47,7 @@ constexpr uint32_t TM_S = 256;  // TMEM columns [256, 320): two S buffers of 32
 constexpr uint32_t IDESC_S = idesc_mma(128, AT_T, 1u, 0u);
 constexpr uint32_t IDESC_PV = idesc_mma(128, 256, 1u, 1u);
 constexpr float RESCALE_LOG2 = 8.f;
+constexpr int AT_PF = 4;  // tiles between the L2 prefetch of a tile's rows and their gather into shared memory
 
 struct AtArgs {
   const int32_t* idx;
@@ -143,6 +144,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         const int rr = i * AT_T + lane;
         return rr < nrows ? rowidx[rr] : 0;
       };
+      auto clamp_row = [&](int v) { return v < 0 ? 0 : (v >= a.L ? a.L - 1 : v); };
+      // L2 prefetch of the rows of tile j (lanes 0..7: one 4-row group each, every K-block of the slice)
+      auto prefetch_tile = [&](int j, int v_raw) {
+        const int v = clamp_row(v_raw);
+        const int g = lane & 7;
+        const int y0 = __shfl_sync(0xffffffffu, v, 4 * g + 0);
+        const int y1 = __shfl_sync(0xffffffffu, v, 4 * g + 1);
+        const int y2 = __shfl_sync(0xffffffffu, v, 4 * g + 2);
+        const int y3 = __shfl_sync(0xffffffffu, v, 4 * g + 3);
+        if (lane < AT_T / 4)
+          for (int kb = 0; kb < kbq; ++kb) tma_prefetch_gather4(&tm_kv, 256 * static_cast<int>(r) + 64 * kb, y0, y1, y2, y3);
+        (void)j;
+      };
+      // the first AT_PF tiles are prefetched up front; afterwards tile i + AT_PF is prefetched when tile i is
+      // gathered (its indices were loaded two iterations earlier)
+      for (int j = 0; j < min(AT_PF, ntiles); ++j) prefetch_tile(j, load_idx(j));
+      int p_a = AT_PF < ntiles ? load_idx(AT_PF) : 0;
+      int p_b = AT_PF + 1 < ntiles ? load_idx(AT_PF + 1) : 0;
       int v_a = load_idx(0);
       int v_b = ntiles > 1 ? load_idx(1) : 0;
       for (int i = 0; i < ntiles; ++i) {
@@ -150,6 +169,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         const int v_raw = v_a;
         v_a = v_b;
         if (i + 2 < ntiles) v_b = load_idx(i + 2);
+        if (i + AT_PF < ntiles) prefetch_tile(i + AT_PF, p_a);
+        p_a = p_b;
+        if (i + AT_PF + 2 < ntiles) p_b = load_idx(i + AT_PF + 2);
         if (!mbar_wait(&kv_empty[st], ((i / AT_STAGES) & 1) ^ 1) || abort_flag) {
           if (lane == 0) {
             atomicExch(&g_attn_tc_timeout, 1);
@@ -162,7 +184,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         __syncwarp();
         // lane g < 8 gathers rows 4g..4g+3 of the tile (all K-blocks of this CTA's slice)
         const int g = lane & 7;
-        const int v = v_raw < 0 ? 0 : (v_raw >= a.L ? a.L - 1 : v_raw);
+        const int v = clamp_row(v_raw);
         const int y0 = __shfl_sync(0xffffffffu, v, 4 * g + 0);
         const int y1 = __shfl_sync(0xffffffffu, v, 4 * g + 1);
         const int y2 = __shfl_sync(0xffffffffu, v, 4 * g + 2);

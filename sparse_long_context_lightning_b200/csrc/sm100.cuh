@@ -247,6 +247,13 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// L2 prefetch of the same 4-row gather (no shared memory, no completion)
+__device__ __forceinline__ void tma_prefetch_gather4(const CUtensorMap* m, int x, int y0, int y1, int y2, int y3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile::gather4 [%0, {%1, %2, %3, %4, %5}];"
+               ::"l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+               : "memory");
+}
+
 // 32 lanes x 32 columns store to TMEM (inverse of tmem_ld32)
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
