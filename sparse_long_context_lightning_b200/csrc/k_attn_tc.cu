@@ -9,16 +9,17 @@
 // no room for the logits, so one work unit (query b, a contiguous split of its selected rows) runs on a
 // 2-CTA cluster: CTA r owns output columns [256r, 256r+256) and latent dims D_0 = [0, 256), D_1 =
 // [256, 576).  Each CTA gathers only its own part of every selected row (512 or 640 bytes, disjoint), with
-// TMA tile::gather4 loads into 128-byte-swizzled shared memory, computes the partial logits
+// 16-byte cp.async copies from four gather warps into 128-byte-swizzled shared memory (many rows in flight
+// per SM; a TMA gather4 per 4 rows x 128 bytes issued too slowly here), computes the partial logits
 // S_r = Q[:, D_r] . C[:, D_r]^T, and the two partials are exchanged through distributed shared memory
-// (remote mbarrier arrivals, no cluster-wide barrier per tile).  Both CTAs then hold the same logits,
+// (one bulk shared-to-shared copy per warp and tile, completing on the peer's mbarrier).  Both CTAs then hold the same logits,
 // run the same online softmax (lazy rescale: O is rescaled only when the running max grows by > 2^8),
 // and each accumulates P . V[:, its 256 columns] in TMEM.  The gathered tile serves both MMAs: K-major for
 // S = Q C^T and MN-major for O += P V, so no transpose is needed.  Splits of one query are merged by a
 // small combine kernel (log-sum-exp weights).
 //
-// Warp roles (192 threads): warp 0 gathers (TMA), warp 1 issues MMAs and owns TMEM, warps 2-5 run the
-// softmax (one head per thread = one TMEM lane) and the epilogue.
+// Warp roles (288 threads): warps 0-3 gather, warp 4 issues MMAs (S two tiles ahead of P.V) and owns TMEM,
+// warps 5-8 run the softmax (one head per thread = one TMEM lane) and the epilogue.
 #include "lsa_common.cuh"
 #include "sm100.cuh"
 
@@ -29,7 +30,10 @@ using namespace sm100;
 
 __device__ int g_attn_tc_timeout;  // set when a bounded wait of the kernel gave up
 
-constexpr int AT_THREADS = 192;
+constexpr int AT_THREADS = 288;  // 4 gather warps, 1 MMA warp, 4 softmax warps
+constexpr int AT_GATHER_WARPS = 4;
+constexpr int AT_MMA_WARP = 4;
+constexpr int AT_SM_TID0 = 160;  // first softmax thread
 constexpr int AT_T = 32;   // gathered rows per tile
 constexpr int AT_H = 128;  // heads (MMA M)
 constexpr int AT_KBQ_MAX = 5;
@@ -47,9 +51,9 @@ constexpr uint32_t TM_S = 256;  // TMEM columns [256, 320): two S buffers of 32
 constexpr uint32_t IDESC_S = idesc_mma(128, AT_T, 1u, 0u);
 constexpr uint32_t IDESC_PV = idesc_mma(128, 256, 1u, 1u);
 constexpr float RESCALE_LOG2 = 8.f;
-constexpr int AT_PF = 4;  // tiles between the L2 prefetch of a tile's rows and their gather into shared memory
 
 struct AtArgs {
+  const uint16_t* kv;  // latent cache [L, 576] bf16
   const int32_t* idx;
   int64_t idx_ld;
   const int32_t* count;
@@ -64,7 +68,7 @@ struct AtArgs {
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
-    k_sparse_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv, AtArgs a) {
+    k_sparse_attn_tc(const __grid_constant__ CUtensorMap tm_q, AtArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* q_s = base;
@@ -99,7 +103,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
 
   if (tid == 0) {
     for (int i = 0; i < AT_STAGES; ++i) {
-      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_full[i], AT_GATHER_WARPS * 32);  // one cp.async arrival per gather thread
       mbar_init(&kv_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -117,7 +121,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     mbar_expect_tx(&sx_full[0], AT_SX_TX);
     mbar_expect_tx(&sx_full[1], AT_SX_TX);
   }
-  if (warp == 1) {
+  if (warp == AT_MMA_WARP) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
@@ -127,41 +131,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ gather producer
+  if (warp < AT_GATHER_WARPS) {
+    // ------------------------------------------------------------------ gather producers
+    // Warp w copies rows 8w..8w+7 of every tile: 16-byte cp.async chunks of this CTA's slice of each row,
+    // placed in the 128-byte-swizzled K-major layout (chunk c of row t at (c ^ (t & 7)) * 16 in its K-block).
     if (ntiles > 0) {
-      if (lane == 0) {
+      if (tid == 0) {
         tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_kv);
         mbar_expect_tx(q_full, kbq * AT_H * 128);
         for (int kb = 0; kb < kbq; ++kb)
           tma_load_2d(q_s + kb * AT_H * 128, &tm_q, q_full, 256 * static_cast<int>(r) + 64 * kb, b * AT_H);
       }
       const int32_t* rowidx = a.idx + static_cast<int64_t>(b) * a.idx_ld + row0;
-      // raw row indices are loaded two tiles ahead and only clamped when used, so the loads stay in
-      // flight while the producer waits for a free stage
+      const uint16_t* kvr = a.kv + 256 * r;  // this CTA's slice starts at latent dim 256 r
+      const int cpr = kbq * 8;              // 16-byte chunks per row
+      // raw row indices (lane l < 8: row 8w + l) are loaded two tiles ahead and clamped at use
       auto load_idx = [&](int i) -> int {
-        const int rr = i * AT_T + lane;
+        const int rr = i * AT_T + warp * 8 + (lane & 7);
         return rr < nrows ? rowidx[rr] : 0;
       };
-      auto clamp_row = [&](int v) { return v < 0 ? 0 : (v >= a.L ? a.L - 1 : v); };
-      // L2 prefetch of the rows of tile j (lanes 0..7: one 4-row group each, every K-block of the slice)
-      auto prefetch_tile = [&](int j, int v_raw) {
-        const int v = clamp_row(v_raw);
-        const int g = lane & 7;
-        const int y0 = __shfl_sync(0xffffffffu, v, 4 * g + 0);
-        const int y1 = __shfl_sync(0xffffffffu, v, 4 * g + 1);
-        const int y2 = __shfl_sync(0xffffffffu, v, 4 * g + 2);
-        const int y3 = __shfl_sync(0xffffffffu, v, 4 * g + 3);
-        if (lane < AT_T / 4)
-          for (int kb = 0; kb < kbq; ++kb) tma_prefetch_gather4(&tm_kv, 256 * static_cast<int>(r) + 64 * kb, y0, y1, y2, y3);
-        (void)j;
-      };
-      // the first AT_PF tiles are prefetched up front; afterwards tile i + AT_PF is prefetched when tile i is
-      // gathered (its indices were loaded two iterations earlier)
-      for (int j = 0; j < min(AT_PF, ntiles); ++j) prefetch_tile(j, load_idx(j));
-      int p_a = AT_PF < ntiles ? load_idx(AT_PF) : 0;
-      int p_b = AT_PF + 1 < ntiles ? load_idx(AT_PF + 1) : 0;
       int v_a = load_idx(0);
       int v_b = ntiles > 1 ? load_idx(1) : 0;
       for (int i = 0; i < ntiles; ++i) {
@@ -169,9 +157,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         const int v_raw = v_a;
         v_a = v_b;
         if (i + 2 < ntiles) v_b = load_idx(i + 2);
-        if (i + AT_PF < ntiles) prefetch_tile(i + AT_PF, p_a);
-        p_a = p_b;
-        if (i + AT_PF + 2 < ntiles) p_b = load_idx(i + AT_PF + 2);
         if (!mbar_wait(&kv_empty[st], ((i / AT_STAGES) & 1) ^ 1) || abort_flag) {
           if (lane == 0) {
             atomicExch(&g_attn_tc_timeout, 1);
@@ -179,25 +164,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
           }
           break;
         }
+        const int v = v_raw < 0 ? 0 : (v_raw >= a.L ? a.L - 1 : v_raw);
         unsigned char* dst = st_s + st * AT_STAGE_BYTES;
-        if (lane == 0) mbar_expect_tx(&kv_full[st], kbq * AT_KB_BYTES);
-        __syncwarp();
-        // lane g < 8 gathers rows 4g..4g+3 of the tile (all K-blocks of this CTA's slice)
-        const int g = lane & 7;
-        const int v = clamp_row(v_raw);
-        const int y0 = __shfl_sync(0xffffffffu, v, 4 * g + 0);
-        const int y1 = __shfl_sync(0xffffffffu, v, 4 * g + 1);
-        const int y2 = __shfl_sync(0xffffffffu, v, 4 * g + 2);
-        const int y3 = __shfl_sync(0xffffffffu, v, 4 * g + 3);
-        if (lane < AT_T / 4) {
-          for (int kb = 0; kb < kbq; ++kb)
-            tma_gather4(dst + kb * AT_KB_BYTES + g * 512, &tm_kv, &kv_full[st], 256 * static_cast<int>(r) + 64 * kb, y0,
-                        y1, y2, y3);
+        for (int q = lane; q < 8 * cpr; q += 32) {
+          const int rr = q / cpr, c = q - rr * cpr;
+          const int row_in_tile = warp * 8 + rr;
+          const int srow = __shfl_sync(0xffffffffu, v, rr);  // every lane takes part: rr < 8
+          const int kb = c >> 3, c8 = c & 7;
+          cp_async16(dst + kb * AT_KB_BYTES + row_in_tile * 128 + ((c8 ^ (row_in_tile & 7)) << 4),
+                     kvr + static_cast<int64_t>(srow) * 576 + c * 8);
         }
-        __syncwarp();
+        cp_async_arrive_noinc(&kv_full[st]);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == AT_MMA_WARP) {
     // ------------------------------------------------------------------ MMA issuer
     // S = Q C^T runs two tiles ahead of O += P V, so the softmax never waits for its next logits
     if (ntiles > 0 && lane == 0) {
@@ -207,6 +187,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       auto issue_s = [&](int j) -> bool {
         const int st = j % AT_STAGES, sb = j & 1;
         if (!mbar_wait(&kv_full[st], (j / AT_STAGES) & 1) || !mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1)) return false;
+        fence_proxy_async_smem();  // the cp.async (generic proxy) writes are read by the tensor cores
         tc_fence_after();
         const uint32_t s_addr = smem_u32(st_s + st * AT_STAGE_BYTES);
         for (int kb = 0; kb < kbq; ++kb) {
@@ -300,7 +281,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         sp[4 * c + 3] = v.w;
       }
       // re-arm buffer sb for tile i+2 (before this CTA sends tile i+1, so before the peer can send i+2)
-      if (tid == 64 && i + 2 < ntiles) mbar_expect_tx(&sx_full[sb], AT_SX_TX);
+      if (tid == AT_SM_TID0 && i + 2 < ntiles) mbar_expect_tx(&sx_full[sb], AT_SX_TX);
       uint32_t sr_next[32];
       if (i + 1 < ntiles && !fetch_and_send(i + 1, sr_next)) {
         ok = false;
@@ -426,7 +407,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // no CTA leaves while its peer may still touch its shared memory
-  if (warp == 1) {
+  if (warp == AT_MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -499,12 +480,11 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   const int S = splits_for(B);
   const size_t need = sparse_attn_ws_bytes(B, idx_ld, H);
   if (S > 1 && (ws == nullptr || !aligned256(ws) || ws_bytes < need)) return LSA_ERR_WORKSPACE;
-  CUtensorMap tq, tkv;
-  int st = make_map(&tq, q, false, B * AT_H, 576, 64, AT_H);
-  if (st) return st;
-  st = make_map(&tkv, kv, false, L, 576, 64, 1);
+  CUtensorMap tq;
+  const int st = make_map(&tq, q, false, B * AT_H, 576, 64, AT_H);
   if (st) return st;
   AtArgs a;
+  a.kv = static_cast<const uint16_t*>(kv);
   a.idx = idx;
   a.idx_ld = idx_ld;
   a.count = count;
@@ -521,7 +501,7 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   LSA_CUDA_TRY(cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM));
   const int64_t grid = 2 * B * S;
   if (grid > 0x7FFFFFFF) return LSA_ERR_UNSUPPORTED;
-  k_sparse_attn_tc<<<static_cast<unsigned>(grid), AT_THREADS, AT_SMEM, s>>>(tq, tkv, a);
+  k_sparse_attn_tc<<<static_cast<unsigned>(grid), AT_THREADS, AT_SMEM, s>>>(tq, a);
   LSA_CUDA_TRY(cudaGetLastError());
   if (S > 1) {
     k_attn_combine<<<static_cast<unsigned>(B * AT_H), 128, 0, s>>>(a.ws_o, a.ws_ml, S, a.out, lse);

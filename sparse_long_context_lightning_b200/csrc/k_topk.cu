@@ -337,8 +337,8 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
       cluster.sync();
       if (r == 0) {
         const uint32_t n = min(sm.ncoll, static_cast<uint32_t>(TK_CAP));
-        if (tid < static_cast<int>(n)) {
-          const uint32_t k = sm.coll_key[tid], p = sm.coll_pos[tid];
+        for (uint32_t t = tid; t < n; t += TK_THREADS) {
+          const uint32_t k = sm.coll_key[t], p = sm.coll_pos[t];
           uint32_t gt = 0, eqlow = 0;
           for (uint32_t j = 0; j < n; ++j) {
             const uint32_t kj = sm.coll_key[j];
@@ -453,44 +453,31 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
     gt_before += sm.cgt[c];
     eq_before += sm.ceq[c];
   }
-  // exclusive eq prefix of my warp inside the CTA
-  uint32_t eq_wbefore = 0;
-  for (int w = 0; w < warp; ++w) eq_wbefore += sm.wb[w];
-  // pass 2: selected count per warp
-  uint32_t sel_w = 0;
-  {
-    uint32_t run_eq = eq_before + eq_wbefore;
-    for (int s0 = w0; s0 < w1; s0 += 32) {
-      const int s = s0 + lane;
-      uint32_t k = 0;
-      if (s < w1) k = f32_order_key(row.val(s));
-      const uint32_t eqm = __ballot_sync(0xffffffffu, s < w1 && k == T);
-      const uint32_t er = run_eq + __popc(eqm & lanemask_lt());
-      const bool sel = s < w1 && (k > T || (k == T && er < need_eq));
-      sel_w += __popc(__ballot_sync(0xffffffffu, sel));
-      run_eq += __popc(eqm);
-    }
+  // exclusive gt / eq prefixes of my warp inside the CTA
+  uint32_t gt_wbefore = 0, eq_wbefore = 0;
+  for (int w = 0; w < warp; ++w) {
+    gt_wbefore += sm.wa[w];
+    eq_wbefore += sm.wb[w];
   }
-  __syncthreads();
-  if (lane == 0) sm.wc[warp] = sel_w;
-  __syncthreads();
-  uint32_t sel_wbefore = 0;
-  for (int w = 0; w < warp; ++w) sel_wbefore += sm.wc[w];
-  const uint32_t sel_before = gt_before + min(eq_before, need_eq);
+  // a selected element's output slot = nsink + (#greater before it) + min(#equal before it, need_eq)
   {
+    uint32_t run_gt = gt_before + gt_wbefore;
     uint32_t run_eq = eq_before + eq_wbefore;
-    uint32_t run_sel = static_cast<uint32_t>(nsink) + sel_before + sel_wbefore;
+    const uint32_t lim = static_cast<uint32_t>(nsink + nsel);
     for (int s0 = w0; s0 < w1; s0 += 32) {
       const int s = s0 + lane;
       uint32_t k = 0;
       if (s < w1) k = f32_order_key(row.val(s));
-      const uint32_t eqm = __ballot_sync(0xffffffffu, s < w1 && k == T);
-      const uint32_t er = run_eq + __popc(eqm & lanemask_lt());
-      const bool sel = s < w1 && (k > T || (k == T && er < need_eq));
-      const uint32_t selm = __ballot_sync(0xffffffffu, sel);
-      const uint32_t o = run_sel + __popc(selm & lanemask_lt());
-      if (sel && o < static_cast<uint32_t>(nsink + nsel)) out[o] = s;  // bounded even if T were wrong
-      run_sel += __popc(selm);
+      const bool is_gt = s < w1 && k > T;
+      const bool is_eq = s < w1 && k == T;
+      const uint32_t gtm = __ballot_sync(0xffffffffu, is_gt);
+      const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
+      const uint32_t lt = lanemask_lt();
+      const uint32_t eq_before_me = run_eq + __popc(eqm & lt);
+      const bool sel = is_gt || (is_eq && eq_before_me < need_eq);
+      const uint32_t o = static_cast<uint32_t>(nsink) + run_gt + __popc(gtm & lt) + min(eq_before_me, need_eq);
+      if (sel && o < lim) out[o] = s;  // bounded even if T were wrong
+      run_gt += __popc(gtm);
       run_eq += __popc(eqm);
     }
   }
