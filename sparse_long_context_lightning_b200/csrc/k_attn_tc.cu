@@ -157,7 +157,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         const int v_raw = v_a;
         v_a = v_b;
         if (i + 2 < ntiles) v_b = load_idx(i + 2);
-        if (!mbar_wait(&kv_empty[st], ((i / AT_STAGES) & 1) ^ 1) || abort_flag) {
+        if (!mbar_spin(&kv_empty[st], ((i / AT_STAGES) & 1) ^ 1) || abort_flag) {
           if (lane == 0) {
             atomicExch(&g_attn_tc_timeout, 1);
             abort_flag = 1;
@@ -181,12 +181,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     // ------------------------------------------------------------------ MMA issuer
     // S = Q C^T runs two tiles ahead of O += P V, so the softmax never waits for its next logits
     if (ntiles > 0 && lane == 0) {
-      bool ok = mbar_wait(q_full, 0);
+      bool ok = mbar_spin(q_full, 0);
       const uint32_t q_addr = smem_u32(q_s);
       const uint32_t p_addr = smem_u32(p_s);
       auto issue_s = [&](int j) -> bool {
         const int st = j % AT_STAGES, sb = j & 1;
-        if (!mbar_wait(&kv_full[st], (j / AT_STAGES) & 1) || !mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1)) return false;
+        if (!mbar_spin(&kv_full[st], (j / AT_STAGES) & 1) || !mbar_spin(&s_empty[sb], ((j >> 1) & 1) ^ 1)) return false;
         fence_proxy_async_smem();  // the cp.async (generic proxy) writes are read by the tensor cores
         tc_fence_after();
         const uint32_t s_addr = smem_u32(st_s + st * AT_STAGE_BYTES);
@@ -201,7 +201,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       };
       auto issue_pv = [&](int j) -> bool {
         const int stj = j % AT_STAGES;
-        if (!mbar_wait(p_full, j & 1)) return false;
+        if (!mbar_spin(p_full, j & 1)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(st_s + stj * AT_STAGE_BYTES);
         #pragma unroll
@@ -236,7 +236,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     // peer's receive buffer j & 1 as one 4 KB bulk copy per warp (all four complete on the peer's mbarrier)
     auto fetch_and_send = [&](int j, uint32_t (&sr)[32]) -> bool {
       const int sb = j & 1;
-      if (!mbar_wait(&s_full[sb], (j >> 1) & 1)) return false;
+      if (!mbar_spin(&s_full[sb], (j >> 1) & 1)) return false;
       tc_fence_after();
       tmem_ld32(trow + TM_S + sb * AT_T, sr);
       tmem_ld_wait();
@@ -315,7 +315,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       }
       l = l * alpha + psum;
       // the previous P . V has finished: the P buffer is free and O is stable
-      if (i > 0 && !mbar_wait(pv_done, (i - 1) & 1)) {
+      if (i > 0 && !mbar_spin(pv_done, (i - 1) & 1)) {
         ok = false;
         break;
       }
@@ -352,7 +352,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     }
     // ---- epilogue
     if (lane == 0) bulk_wait_read0();  // this warp's last outgoing copy has read its staging rows
-    const bool have = ok && ntiles > 0 && mbar_wait(pv_done, (ntiles - 1) & 1);
+    const bool have = ok && ntiles > 0 && mbar_spin(pv_done, (ntiles - 1) & 1);
     tc_fence_after();
     const int64_t orow = static_cast<int64_t>(b) * AT_H + h;
     if (a.S == 1) {

@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
   // ---- level 0 range: min / max of the candidates (non-finite values clamp into the end bins)
   {
     float lo = INFINITY, hi = -INFINITY;
+    #pragma unroll 4
     for (int s = a0 + tid; s < a1; s += TK_THREADS) {
       const float x = row.val(s);
       if (isfinite(x)) {
@@ -228,6 +229,7 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
     // ---- histogram of this level ------------------------------------------------------
     for (int i = tid; i < TK_BINS; i += TK_THREADS) sm.hist[i] = 0;
     __syncthreads();
+    #pragma unroll 4
     for (int s = a0 + tid; s < a1; s += TK_THREADS) {
       const float x = row.val(s);
       int bin;
@@ -314,6 +316,7 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
       uint32_t* rn = cluster.map_shared_rank(&sm.ncoll, 0);
       uint32_t* rk = cluster.map_shared_rank(&sm.coll_key[0], 0);
       uint32_t* rp = cluster.map_shared_rank(&sm.coll_pos[0], 0);
+      #pragma unroll 4
       for (int s = a0 + tid; s < a1; s += TK_THREADS) {
         const float x = row.val(s);
         const uint32_t k = f32_order_key(x);
@@ -423,16 +426,23 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
 
   // ---- ordered compaction: selected = key > T, or key == T among the first need_eq of them ----
   const int n = max(0, a1 - a0);
-  const int per_w = ((n + TK_WARPS - 1) / TK_WARPS + 31) & ~31;
+  const int per_w = ((n + TK_WARPS - 1) / TK_WARPS + 127) & ~127;  // multiple of 128: 4 chunks per pass
   const int w0 = a0 + warp * per_w;
   const int w1 = min(a1, w0 + per_w);
   uint32_t gt_w = 0, eq_w = 0;
-  for (int s0 = w0; s0 < w1; s0 += 32) {
-    const int s = s0 + lane;
-    uint32_t k = 0;
-    if (s < w1) k = f32_order_key(row.val(s));
-    gt_w += __popc(__ballot_sync(0xffffffffu, s < w1 && k > T));
-    eq_w += __popc(__ballot_sync(0xffffffffu, s < w1 && k == T));
+  for (int s0 = w0; s0 < w1; s0 += 128) {
+    uint32_t k[4];
+    #pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int s = s0 + 32 * u + lane;
+      k[u] = s < w1 ? f32_order_key(row.val(s)) : 0u;
+    }
+    #pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const bool in = s0 + 32 * u + lane < w1;
+      gt_w += __popc(__ballot_sync(0xffffffffu, in && k[u] > T));
+      eq_w += __popc(__ballot_sync(0xffffffffu, in && k[u] == T));
+    }
   }
   if (lane == 0) {
     sm.wa[warp] = gt_w;
@@ -464,10 +474,17 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
     uint32_t run_gt = gt_before + gt_wbefore;
     uint32_t run_eq = eq_before + eq_wbefore;
     const uint32_t lim = static_cast<uint32_t>(nsink + nsel);
-    for (int s0 = w0; s0 < w1; s0 += 32) {
-      const int s = s0 + lane;
-      uint32_t k = 0;
-      if (s < w1) k = f32_order_key(row.val(s));
+    for (int s00 = w0; s00 < w1; s00 += 128) {
+     uint32_t kk[4];
+     #pragma unroll
+     for (int u = 0; u < 4; ++u) {
+       const int s = s00 + 32 * u + lane;
+       kk[u] = s < w1 ? f32_order_key(row.val(s)) : 0u;
+     }
+     #pragma unroll
+     for (int u = 0; u < 4; ++u) {
+      const int s = s00 + 32 * u + lane;
+      const uint32_t k = kk[u];
       const bool is_gt = s < w1 && k > T;
       const bool is_eq = s < w1 && k == T;
       const uint32_t gtm = __ballot_sync(0xffffffffu, is_gt);
@@ -479,6 +496,7 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
       if (sel && o < lim) out[o] = s;  // bounded even if T were wrong
       run_gt += __popc(gtm);
       run_eq += __popc(eqm);
+     }
     }
   }
   // keep this CTA's shared memory alive until every remote access of the cluster is done
