@@ -4,28 +4,33 @@
 // section "机制一：流式感知索引（SI）/ 预算分解": the sink and the window are fixed, the top-K runs
 // over the positions outside them, and the three sets are unioned.
 //
-// Design (B200): one thread-block cluster of C CTAs (C <= 16) per score row.  Each CTA owns a
-// contiguous chunk of the row and, when it fits, keeps it in shared memory, so HBM is read once.
-// The threshold is found by histogram refinement:
-//   level 0  4096 linear value bins over [min, max] of the row's candidates,
-//   level 1+ 4096-way radix digits of the order-preserving uint32 key inside the boundary bin,
-// each level's per-CTA histograms summed across the cluster through distributed shared memory
-// (DSMEM), until the boundary bin holds <= 1024 elements.  Those are gathered into CTA 0's shared
-// memory and ranked exactly (score descending, position ascending).  A final ordered pass writes
-// the selected positions in ascending order.  All cross-CTA synchronisation is the hardware
-// cluster barrier: no spin-waits, no global atomics, no scratch memory.
+// Design (B200): one thread-block cluster of C CTAs (C <= 16) per score row, two CTAs per SM.  Each CTA
+// owns a contiguous chunk of the row and, when it fits (<= 16384 scores), keeps it in shared memory (one
+// bulk asynchronous copy), so HBM is read once.  The threshold is found by refining the order-preserving
+// uint32 key: level 0 histograms 256 bins over the candidates' key range, each further level one 8-bit
+// digit inside the boundary bin.  Per-CTA histograms are all-gathered through distributed shared memory
+// (DSMEM), so every CTA finds the boundary bin itself (one cluster barrier per level).  When the
+// boundary bin holds <= 1024 elements, its keys are all-gathered too and every CTA finishes the
+// refinement locally; the tie shares and every CTA's output offset follow from the gathered counts, so
+// the ordered write pass needs no further communication.  Common case: three cluster barriers.  Each
+// CTA runs this code once, so the passes are short rolled loops (a small instruction footprint) rather
+// than unrolled code.  All synchronisation is the hardware cluster barrier: no spin-waits on memory, no
+// global atomics, no scratch memory.
+#include <mutex>
+
 #include "lsa_common.cuh"
 #include "sm100.cuh"
 
 namespace lsa {
 namespace {
 
-constexpr int TK_THREADS = 512;
+constexpr int TK_THREADS = 1024;
 constexpr int TK_WARPS = TK_THREADS / 32;  // <= 32: per-warp arrays are reduced by one warp, lane < TK_WARPS
 static_assert(TK_WARPS <= 32, "one warp reduces the per-warp partials");
-constexpr int TK_BINS = 4096;
-constexpr int TK_CAP = 1024;
-constexpr int TK_MAXC = 16;
+constexpr int TK_BINS = 256;   // one 8-bit digit of the order key per refinement level
+constexpr int TK_CAP = 1024;   // boundary-bin size that is all-gathered and finished locally
+constexpr int TK_MAXC = 16;    // cluster size limit (non-portable above 8)
+constexpr int TK_CACHE = 24576;  // scores per CTA kept in shared memory (96 KB)
 
 enum { MODE_TOKEN = 0, MODE_ALL = 1, MODE_BLOCKS = 2 };
 
@@ -44,38 +49,31 @@ struct TopkArgs {
   int32_t* count;
   int kmax;
   int chunk;   // positions per CTA (multiple of 4)
-  int cached;  // chunk kept in dynamic shared memory
+  int cached;  // chunk <= TK_CACHE: kept in dynamic shared memory
 };
 
+// Dynamic shared memory: hall[2][C][TK_BINS] (every CTA's histogram of a level, all-gathered, double
+// buffered by level parity), then the cached chunk (scores, converted in place to order keys).
 struct TopkSmem {
-  uint32_t hist[TK_BINS];
-  uint32_t hred[TK_BINS];
-  uint32_t coll_key[TK_CAP];
-  uint32_t coll_pos[TK_CAP];
-  uint32_t ncoll;
-  uint32_t stot[TK_MAXC];
-  float fmin[TK_MAXC];
-  float fmax[TK_MAXC];
-  uint32_t kmin[TK_MAXC];
-  uint32_t kmax[TK_MAXC];
-  uint32_t cgt[TK_MAXC];
-  uint32_t ceq[TK_MAXC];
-  uint32_t wa[TK_WARPS];
-  uint32_t wb[TK_WARPS];
-  uint32_t wc[TK_WARPS];
-  float wf0[TK_WARPS];
-  float wf1[TK_WARPS];
-  // broadcast slots (written by the CTA that decides)
-  uint32_t b_bin, b_above, b_count;
-  uint32_t b_T, b_need_eq;
+  uint32_t h[TK_BINS];     // this CTA's histogram of a level / the local refinement histogram
+  uint32_t tot[TK_BINS];   // cluster-wide histogram of a level
+  uint32_t cand[TK_CAP];   // boundary-bin keys; CTA c's at [segoff[c], segoff[c] + segcnt[c])
+  uint8_t cand_w[TK_CAP];  // warp of each of this CTA's own boundary-bin elements (local slot order)
+  uint32_t kmin[TK_MAXC], kmax[TK_MAXC];
+  uint32_t above[TK_MAXC];  // CTA c's elements above the boundary bins of all levels
+  uint32_t segoff[TK_MAXC], segcnt[TK_MAXC];
+  uint32_t gtb[TK_MAXC], eqb[TK_MAXC];  // CTA c's boundary elements with key > T / key == T
+  uint32_t wa[TK_WARPS], wb[TK_WARPS];
+  uint32_t wgt[TK_WARPS], weq[TK_WARPS];  // this CTA's elements with key > T / key == T, per warp
+  uint32_t ccount;
+  uint32_t sel_bin, sel_above, sel_count;
   uint64_t load_bar;
 };
 
-struct Row {
-  const float* src;  // element s of the row is src[s - base]
-  int base;
-  __device__ __forceinline__ float val(int s) const { return src[s - base]; }
-};
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
@@ -83,27 +81,18 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
-// Block-wide sum of one uint32 per thread; every thread gets the total.
-__device__ uint32_t block_sum_u32(uint32_t v, uint32_t* scratch) {
-  v = warp_sum_u32(v);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __syncthreads();
-  if (lane == 0) scratch[warp] = v;
-  __syncthreads();
-  uint32_t t = lane < TK_WARPS ? scratch[lane] : 0u;
-  t = warp_sum_u32(t);
-  return t;
-}
+// Keys of valid elements are >= 1 (key 0, a negative-NaN pattern, is merged into key 1); key 0 marks a
+// position outside this CTA's candidate range, so it is never counted or selected.
+__device__ __forceinline__ uint32_t valid_key(float x) { return max(f32_order_key(x), 1u); }
+__device__ __forceinline__ bool key_finite(uint32_t k) { return k > 0x007FFFFFu && k < 0xFF800000u; }
 
-__global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
-  extern __shared__ __align__(16) unsigned char dyn[];
-  __shared__ TopkSmem sm;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int C = static_cast<int>(cluster.num_blocks());
-  const int r = static_cast<int>(cluster.block_rank());
-  const int b = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
+// The candidate range of row b, the fixed (sink / window) entries, the padding and the count.  CTA rank 0
+// writes everything but the top-K part of the row.
+struct RowSetup {
+  int nsink, clo, chi, ncand, nsel;
+  int32_t* out;
+};
+__device__ __forceinline__ RowSetup row_setup(const TopkArgs& a, int b, int r, int tid) {
   const int64_t qp64 = a.q_pos[b];
   const int qp = static_cast<int>(qp64 < 0 ? -1 : (qp64 >= a.L ? a.L - 1 : qp64));
   int nsink = 0, clo = 0, chi = 0, wlo = 0, whi = 0;  // window = [wlo, whi)
@@ -127,38 +116,153 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
     const int64_t nvis = qp64 < 0 ? 0 : (qp64 + 1) / a.div;
     chi = static_cast<int>(nvis < a.L ? nvis : a.L);
   }
-  const int ncand = max(0, chi - clo);
-  const int K = a.K;
-  int32_t* out = a.idx + static_cast<int64_t>(b) * a.idx_ld;
+  RowSetup rs;
+  rs.nsink = nsink;
+  rs.clo = clo;
+  rs.chi = chi;
+  rs.ncand = max(0, chi - clo);
+  rs.nsel = a.K > 0 ? min(a.K, rs.ncand) : 0;
+  rs.out = a.idx + static_cast<int64_t>(b) * a.idx_ld;
   const int nwin = whi - wlo;
-  const int nsel = min(K, ncand);
-  const int total = nsink + nsel + nwin;
-
-  // rank 0 writes the fixed positions, the padding and the count
+  const int total = nsink + rs.nsel + nwin;
   if (r == 0) {
-    for (int i = tid; i < nsink; i += TK_THREADS) out[i] = i;
-    for (int i = tid; i < nwin; i += TK_THREADS) out[nsink + nsel + i] = wlo + i;
-    for (int i = total + tid; i < a.kmax; i += TK_THREADS) out[i] = -1;
+    for (int i = tid; i < nsink; i += TK_THREADS) rs.out[i] = i;
+    for (int i = tid; i < nwin; i += TK_THREADS) rs.out[nsink + rs.nsel + i] = wlo + i;
+    for (int i = total + tid; i < a.kmax; i += TK_THREADS) rs.out[i] = -1;
     if (tid == 0) a.count[b] = total;
   }
+  return rs;
+}
 
+// This CTA's view of its chunk: groups of 4 consecutive positions starting at c0.  Group g holds
+// positions c0 + 4g .. c0 + 4g + 3; an element is valid when its position is in [a0, a1).
+struct Chunk {
+  const float* grow;  // the score row in global memory
+  const uint4* keys;  // the chunk's order keys in shared memory (0 = invalid), or nullptr
+  int c0, a0, a1;
+  __device__ __forceinline__ uint4 from_scores(int g, float4 v) const {
+    const int s0 = c0 + 4 * g;
+    uint4 k;
+    if (s0 >= a0 && s0 + 4 <= a1) {
+      k.x = valid_key(v.x);
+      k.y = valid_key(v.y);
+      k.z = valid_key(v.z);
+      k.w = valid_key(v.w);
+    } else {
+      k.x = (s0 >= a0 && s0 < a1) ? valid_key(v.x) : 0u;
+      k.y = (s0 + 1 >= a0 && s0 + 1 < a1) ? valid_key(v.y) : 0u;
+      k.z = (s0 + 2 >= a0 && s0 + 2 < a1) ? valid_key(v.z) : 0u;
+      k.w = (s0 + 3 >= a0 && s0 + 3 < a1) ? valid_key(v.w) : 0u;
+    }
+    return k;
+  }
+  __device__ __forceinline__ uint4 load(int g) const {
+    if (keys) return keys[g];
+    const int s0 = c0 + 4 * g;
+    float4 v;
+    v.x = (s0 >= a0 && s0 < a1) ? __ldg(grow + s0) : 0.f;
+    v.y = (s0 + 1 >= a0 && s0 + 1 < a1) ? __ldg(grow + s0 + 1) : 0.f;
+    v.z = (s0 + 2 >= a0 && s0 + 2 < a1) ? __ldg(grow + s0 + 2) : 0.f;
+    v.w = (s0 + 3 >= a0 && s0 + 3 < a1) ? __ldg(grow + s0 + 3) : 0.f;
+    return from_scores(g, v);
+  }
+};
+
+// Boundary bin of hist[] (bins ascend with the key): the bin holding the need-th largest element.
+// Warp 0 only; lane l scans bins [8l, 8l + 8).  Writes sel_bin / sel_above / sel_count.
+__device__ __forceinline__ void find_boundary(TopkSmem& sm, const uint32_t* hist, uint32_t need, int lane) {
+  const uint4 v0 = reinterpret_cast<const uint4*>(hist)[2 * lane];
+  const uint4 v1 = reinterpret_cast<const uint4*>(hist)[2 * lane + 1];
+  const uint32_t t[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  uint32_t lsum = 0;
+  #pragma unroll
+  for (int j = 0; j < 8; ++j) lsum += t[j];
+  uint32_t suf = lsum;  // inclusive suffix sum over lanes (higher lanes hold higher bins)
+  #pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += v;
+  }
+  uint32_t acc = suf - lsum;  // elements in bins above this lane's range
+  if (acc < need && acc + lsum >= need) {
+    for (int j = 7; j >= 0; --j) {
+      if (acc + t[j] >= need) {
+        sm.sel_bin = static_cast<uint32_t>(lane * 8 + j);
+        sm.sel_above = acc;
+        sm.sel_count = t[j];
+        break;
+      }
+      acc += t[j];
+    }
+  }
+}
+
+// Level geometry over [klo, khi]: 256 bins of width 2^shift.
+__device__ __forceinline__ int level_shift(uint32_t klo, uint32_t khi) {
+  const uint32_t span = khi - klo;
+  const int bits = span ? 32 - __clz(span) : 0;
+  return bits > 8 ? bits - 8 : 0;
+}
+// Key range [nlo, nhi] of bin `bin` of a level over [klo, khi].
+__device__ __forceinline__ void bin_range(uint32_t klo, uint32_t khi, int shift, uint32_t bin, uint32_t& nlo,
+                                          uint32_t& nhi) {
+  nlo = klo + (bin << shift);
+  const uint64_t hi64 = static_cast<uint64_t>(nlo) + ((uint64_t(1) << shift) - 1);
+  nhi = static_cast<uint32_t>(hi64 < khi ? hi64 : khi);
+}
+
+// Warp-exclusive prefix and warp total of a per-lane count in [0, 7], from three ballots.
+__device__ __forceinline__ uint32_t ballot_prefix(uint32_t v, uint32_t lt, uint32_t& total) {
+  const uint32_t b0 = __ballot_sync(0xffffffffu, v & 1u);
+  const uint32_t b1 = __ballot_sync(0xffffffffu, v & 2u);
+  const uint32_t b2 = __ballot_sync(0xffffffffu, v & 4u);
+  total = __popc(b0) + 2u * __popc(b1) + 4u * __popc(b2);
+  return __popc(b0 & lt) + 2u * __popc(b1 & lt) + 4u * __popc(b2 & lt);
+}
+
+__global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
+  extern __shared__ __align__(16) unsigned char dyn[];
+  __shared__ __align__(16) TopkSmem sm;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int r = static_cast<int>(cluster.block_rank());
+  const int b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  cluster_arrive_relaxed();  // the matching wait comes before the first DSMEM access
+  uint32_t* hall = reinterpret_cast<uint32_t*>(dyn);  // [2][C][TK_BINS]
+
+  const RowSetup rs = row_setup(a, b, r, tid);
+  const int K = a.K;
   const int c0 = r * a.chunk;
   const int c1 = min(a.L, c0 + a.chunk);
-  const int a0 = max(c0, clo), a1 = min(c1, chi);  // my candidates
-
-  if (ncand <= K) {  // every candidate is selected (row-uniform branch: no cluster sync)
-    for (int s = a0 + tid; s < a1; s += TK_THREADS) out[nsink + (s - clo)] = s;
+  const int a0 = max(c0, rs.clo), a1 = min(c1, rs.chi);  // my candidates
+  if (rs.ncand <= K || K <= 0) {  // every candidate, or none, is selected (row-uniform branch)
+    if (K > 0)
+      for (int s = a0 + tid; s < a1; s += TK_THREADS) rs.out[rs.nsink + (s - rs.clo)] = s;
+    cluster_wait();
     return;
   }
+  if (tid < TK_MAXC) sm.above[tid] = 0;
+  if (tid < TK_WARPS) {
+    sm.wgt[tid] = 0;
+    sm.weq[tid] = 0;
+  }
 
-  // ---- stage the chunk -------------------------------------------------------------
-  const float* grow = a.scores + static_cast<int64_t>(b) * a.ld;
-  Row row;
+  // ---- stage the chunk ----
+  Chunk ch;
+  ch.grow = a.scores + static_cast<int64_t>(b) * a.ld;
+  ch.keys = nullptr;
+  ch.c0 = c0;
+  ch.a0 = a0;
+  ch.a1 = a1;
+  const int ng = a1 > a0 ? (a1 - c0 + 3) / 4 : 0;  // groups [g_lo, ng) hold my candidates
+  const int g_lo = a1 > a0 ? (a0 - c0) / 4 : 0;
+  float4* cache = reinterpret_cast<float4*>(dyn + static_cast<size_t>(2 * C * TK_BINS) * 4);
   if (a.cached) {
-    // one bulk asynchronous copy of the aligned part of the chunk, the last < 4 scores by plain loads
-    float* cache = reinterpret_cast<float*>(dyn);
-    const int lend = min(c1, chi);
-    const int nvec = max(0, (lend - c0) / 4);
+    float* cf = reinterpret_cast<float*>(cache);
+    const int lend = min(c1, rs.chi);
+    const bool aligned = (reinterpret_cast<uintptr_t>(ch.grow + c0) & 15u) == 0;
+    const int nvec = aligned ? max(0, (lend - c0) / 4) : 0;
     if (tid == 0) {
       sm100::mbar_init(&sm.load_bar, 1);
       sm100::fence_mbar_init();
@@ -167,340 +271,322 @@ __global__ void __launch_bounds__(TK_THREADS, 2) k_topk_cluster(TopkArgs a) {
     if (tid == 0) {
       if (nvec > 0) {
         sm100::mbar_expect_tx(&sm.load_bar, static_cast<uint32_t>(nvec) * 16u);
-        sm100::bulk_load(cache, grow + c0, static_cast<uint32_t>(nvec) * 16u, &sm.load_bar);
+        sm100::bulk_load(cf, ch.grow + c0, static_cast<uint32_t>(nvec) * 16u, &sm.load_bar);
       } else {
         sm100::mbar_arrive(&sm.load_bar);
       }
     }
-    for (int s = c0 + nvec * 4 + tid; s < lend; s += TK_THREADS) cache[s - c0] = grow[s];
-    // bounded wait (the copy is in bounds by construction); on give-up the row is left as the copy made it
+    // the unaligned rest (or the whole chunk when the row is not 16-byte aligned) by plain loads
+    for (int s = c0 + nvec * 4 + tid; s < 4 * ng + c0; s += TK_THREADS) cf[s - c0] = s < lend ? ch.grow[s] : 0.f;
+    // bounded wait (the copy is in bounds by construction)
     sm100::mbar_wait(&sm.load_bar, 0);
-    row.src = cache;
-    row.base = c0;
     __syncthreads();
-  } else {
-    row.src = grow;
-    row.base = 0;
   }
+  // warp w walks groups [gw0, gw1); lane l takes every 32nd group from gw0 + l
+  const int per_w = (ng - g_lo + TK_WARPS - 1) / TK_WARPS;
+  const int gw0 = g_lo + warp * per_w;
+  const int gw1 = min(ng, gw0 + per_w);
 
-  // ---- level 0 range: min / max of the candidates (non-finite values clamp into the end bins)
+  // ---- order keys (in place, when cached) and the finite key range of the candidates ----
   {
-    float lo = INFINITY, hi = -INFINITY;
-    #pragma unroll 4
-    for (int s = a0 + tid; s < a1; s += TK_THREADS) {
-      const float x = row.val(s);
-      if (isfinite(x)) {
-        lo = fminf(lo, x);
-        hi = fmaxf(hi, x);
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (int g = gw0 + lane; g < gw1; g += 32) {
+      uint4 k;
+      if (a.cached) {
+        k = ch.from_scores(g, cache[g]);
+        reinterpret_cast<uint4*>(cache)[g] = k;
+      } else {
+        k = ch.load(g);
       }
+      if (key_finite(k.x)) { lo = min(lo, k.x); hi = max(hi, k.x); }
+      if (key_finite(k.y)) { lo = min(lo, k.y); hi = max(hi, k.y); }
+      if (key_finite(k.z)) { lo = min(lo, k.z); hi = max(hi, k.z); }
+      if (key_finite(k.w)) { lo = min(lo, k.w); hi = max(hi, k.w); }
     }
-    lo = warp_min(lo);
-    hi = warp_max(hi);
+    if (a.cached) ch.keys = reinterpret_cast<const uint4*>(cache);  // each thread reads back only its own groups
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
     if (lane == 0) {
-      sm.wf0[warp] = lo;
-      sm.wf1[warp] = hi;
+      sm.wa[warp] = lo;
+      sm.wb[warp] = hi;
     }
     __syncthreads();
     if (warp == 0) {
-      lo = warp_min(lane < TK_WARPS ? sm.wf0[lane] : INFINITY);
-      hi = warp_max(lane < TK_WARPS ? sm.wf1[lane] : -INFINITY);
-      if (lane < C) {
-        *cluster.map_shared_rank(&sm.fmin[r], lane) = lo;
-        *cluster.map_shared_rank(&sm.fmax[r], lane) = hi;
-      }
-    }
-    cluster.sync();
-  }
-  float gmin = INFINITY, gmax = -INFINITY;
-  for (int c = 0; c < C; ++c) {
-    gmin = fminf(gmin, sm.fmin[c]);
-    gmax = fmaxf(gmax, sm.fmax[c]);
-  }
-  if (!(gmin <= gmax)) gmin = gmax = 0.f;  // no finite candidate at all
-  const float inv = gmax > gmin ? static_cast<float>(TK_BINS) / (gmax - gmin) : 0.f;
-
-  uint32_t need = static_cast<uint32_t>(K);
-  uint32_t klo = 0, khi = 0xFFFFFFFFu;
-  int shift = 0;
-  bool resolved = false;  // threshold key known without collection (all remaining keys equal)
-  uint32_t T = 0, need_eq = 0;
-
-  for (int level = 0; level < 5; ++level) {
-    // ---- histogram of this level ------------------------------------------------------
-    for (int i = tid; i < TK_BINS; i += TK_THREADS) sm.hist[i] = 0;
-    __syncthreads();
-    #pragma unroll 4
-    for (int s = a0 + tid; s < a1; s += TK_THREADS) {
-      const float x = row.val(s);
-      int bin;
-      if (level == 0) {
-        const float t = (x - gmin) * inv;
-        bin = t >= static_cast<float>(TK_BINS - 1) ? TK_BINS - 1 : (t > 0.f ? static_cast<int>(t) : 0);
-        if (x != x) bin = TK_BINS - 1;
-      } else {
-        const uint32_t k = f32_order_key(x);
-        if (k < klo || k > khi) continue;
-        bin = static_cast<int>((k - klo) >> shift);
-      }
-      atomicAdd(&sm.hist[bin], 1u);
-    }
-    cluster.sync();
-    // ---- sum my slice of bins across the cluster ----------------------------------------
-    const int per = TK_BINS / C;
-    const int blo = r * per;
-    uint32_t mysum = 0;
-    for (int i = tid; i < per; i += TK_THREADS) {
-      uint32_t t = 0;
-      for (int c = 0; c < C; ++c) t += *cluster.map_shared_rank(&sm.hist[blo + i], c);
-      sm.hred[i] = t;
-      mysum += t;
-    }
-    mysum = block_sum_u32(mysum, sm.wa);
-    if (tid < C) *cluster.map_shared_rank(&sm.stot[r], tid) = mysum;
-    cluster.sync();
-    // ---- the CTA whose slice holds the boundary picks the bin and broadcasts it -------------
-    uint32_t above = 0;
-    int bslice = 0;
-    for (int c = C - 1; c >= 0; --c) {
-      if (above + sm.stot[c] >= need) {
-        bslice = c;
-        break;
-      }
-      above += sm.stot[c];
-    }
-    if (r == bslice && warp == 0) {
-      // scan my slice from the top: lane l owns bins [l*per/32, (l+1)*per/32)
-      const int pl = per / 32;
-      uint32_t lsum = 0;
-      for (int i = 0; i < pl; ++i) lsum += sm.hred[lane * pl + i];
-      // inclusive suffix sums over lanes (higher lanes hold higher bins)
-      uint32_t suf = lsum;
-      #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
-        if (lane + o < 32) suf += v;
-      }
-      const uint32_t above_lane = above + suf - lsum;  // bins above my lane's range
-      const bool mine = above_lane < need && above_lane + lsum >= need;
-      if (mine) {
-        uint32_t acc = above_lane;
-        for (int i = pl - 1; i >= 0; --i) {
-          const uint32_t h = sm.hred[lane * pl + i];
-          if (acc + h >= need) {
-            for (int c = 0; c < C; ++c) {
-              *cluster.map_shared_rank(&sm.b_bin, c) = static_cast<uint32_t>(blo + lane * pl + i);
-              *cluster.map_shared_rank(&sm.b_above, c) = acc;
-              *cluster.map_shared_rank(&sm.b_count, c) = h;
-            }
-            break;
-          }
-          acc += h;
-        }
-      }
-    }
-    cluster.sync();
-    const uint32_t bstar = sm.b_bin;
-    need -= sm.b_above;
-    const uint32_t bcount = sm.b_count;
-
-    if (level > 0 && shift == 0) {  // the bin is a single key value: pure tie
-      T = klo + bstar;
-      need_eq = need;
-      resolved = true;
-      break;
-    }
-    if (bcount <= static_cast<uint32_t>(TK_CAP)) {
-      // ---- gather the boundary bin into CTA 0 and rank it exactly ----------------------------
-      if (r == 0 && tid == 0) sm.ncoll = 0;
-      cluster.sync();
-      uint32_t* rn = cluster.map_shared_rank(&sm.ncoll, 0);
-      uint32_t* rk = cluster.map_shared_rank(&sm.coll_key[0], 0);
-      uint32_t* rp = cluster.map_shared_rank(&sm.coll_pos[0], 0);
-      #pragma unroll 4
-      for (int s = a0 + tid; s < a1; s += TK_THREADS) {
-        const float x = row.val(s);
-        const uint32_t k = f32_order_key(x);
-        bool in;
-        if (level == 0) {
-          const float t = (x - gmin) * inv;
-          int bin = t >= static_cast<float>(TK_BINS - 1) ? TK_BINS - 1 : (t > 0.f ? static_cast<int>(t) : 0);
-          if (x != x) bin = TK_BINS - 1;
-          in = bin == static_cast<int>(bstar);
-        } else {
-          in = k >= klo && k <= khi && ((k - klo) >> shift) == bstar;
-        }
-        if (in) {
-          const uint32_t slot = atomicAdd(rn, 1u);
-          if (slot < static_cast<uint32_t>(TK_CAP)) {
-            rk[slot] = k;
-            rp[slot] = static_cast<uint32_t>(s);
-          }
-        }
-      }
-      cluster.sync();
-      if (r == 0) {
-        const uint32_t n = min(sm.ncoll, static_cast<uint32_t>(TK_CAP));
-        for (uint32_t t = tid; t < n; t += TK_THREADS) {
-          const uint32_t k = sm.coll_key[t], p = sm.coll_pos[t];
-          uint32_t gt = 0, eqlow = 0;
-          for (uint32_t j = 0; j < n; ++j) {
-            const uint32_t kj = sm.coll_key[j];
-            gt += kj > k;
-            eqlow += (kj == k) & (sm.coll_pos[j] < p);
-          }
-          if (gt + eqlow == need - 1) {
-            for (int c = 0; c < C; ++c) {
-              *cluster.map_shared_rank(&sm.b_T, c) = k;
-              *cluster.map_shared_rank(&sm.b_need_eq, c) = need - gt;
-            }
-          }
-        }
-      }
-      cluster.sync();
-      T = sm.b_T;
-      need_eq = sm.b_need_eq;
-      resolved = true;
-      break;
-    }
-    // ---- refine: next level is a radix digit inside the boundary bin's key range ------------
-    if (level == 0) {
-      uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-      for (int s = a0 + tid; s < a1; s += TK_THREADS) {
-        const float x = row.val(s);
-        const float t = (x - gmin) * inv;
-        int bin = t >= static_cast<float>(TK_BINS - 1) ? TK_BINS - 1 : (t > 0.f ? static_cast<int>(t) : 0);
-        if (x != x) bin = TK_BINS - 1;
-        if (bin == static_cast<int>(bstar)) {
-          const uint32_t k = f32_order_key(x);
-          lo = min(lo, k);
-          hi = max(hi, k);
-        }
-      }
+      lo = lane < TK_WARPS ? sm.wa[lane] : 0xFFFFFFFFu;
+      hi = lane < TK_WARPS ? sm.wb[lane] : 0u;
       #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
         hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
       }
-      if (lane == 0) {
-        sm.wa[warp] = lo;
-        sm.wb[warp] = hi;
+    }
+    cluster_wait();  // every CTA of the cluster has started: DSMEM is addressable
+    if (warp == 0 && lane < C) {
+      *cluster.map_shared_rank(&sm.kmin[r], lane) = lo;
+      *cluster.map_shared_rank(&sm.kmax[r], lane) = hi;
+    }
+    cluster.sync();
+  }
+  uint32_t klo = 0xFFFFFFFFu, khi = 0u;
+  for (int c = 0; c < C; ++c) {
+    klo = min(klo, sm.kmin[c]);
+    khi = max(khi, sm.kmax[c]);
+  }
+  if (klo > khi) klo = khi = 0x80000000u;  // no finite candidate: every key is clamped into one bin
+
+  // ---- cluster-level refinement: each level histograms one 8-bit digit of (key - klo) in [klo, khi] ----
+  // Level 0 covers every valid key: keys outside the finite range are clamped to it, so the first bin's
+  // range extends down to key 1 and the last occupied bin's range up to 0xFFFFFFFF.
+  uint32_t need = static_cast<uint32_t>(K);
+  uint32_t T = 0, need_eq = 0;
+  bool gathered = false;
+  for (int level = 0; level < 8; ++level) {
+    const int shift = level_shift(klo, khi);
+    const uint32_t bmax = (khi - klo) >> shift;  // last occupied bin, <= 255
+    uint32_t* hl = hall + (level & 1) * C * TK_BINS;
+    if (tid < TK_BINS) sm.h[tid] = 0;
+    __syncthreads();
+    for (int g = gw0 + lane; g < gw1; g += 32) {
+      const uint4 k4 = ch.load(g);
+      const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
+      #pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (level == 0) {
+          if (k[e]) atomicAdd(&sm.h[(min(max(k[e], klo), khi) - klo) >> shift], 1u);
+        } else if (k[e] >= klo && k[e] <= khi) {
+          atomicAdd(&sm.h[(k[e] - klo) >> shift], 1u);
+        }
       }
+    }
+    __syncthreads();
+    for (int i = tid; i < TK_BINS * C; i += TK_THREADS) {
+      const int c = i / TK_BINS, bin = i - c * TK_BINS;
+      *cluster.map_shared_rank(hl + r * TK_BINS + bin, c) = sm.h[bin];
+    }
+    cluster.sync();
+    if (tid < TK_BINS) {
+      uint32_t v = 0;
+      for (int c = 0; c < C; ++c) v += hl[c * TK_BINS + tid];
+      sm.tot[tid] = v;
+    }
+    __syncthreads();
+    if (warp == 0) find_boundary(sm, sm.tot, need, lane);
+    __syncthreads();
+    const uint32_t bstar = sm.sel_bin, bcount = sm.sel_count;
+    need -= sm.sel_above;
+    if (warp < C) {  // CTA `warp`'s elements above the boundary bin
+      uint32_t v = 0;
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t bin = static_cast<uint32_t>(lane * 8 + j);
+        v += bin > bstar ? hl[warp * TK_BINS + bin] : 0u;
+      }
+      v = warp_sum_u32(v);
+      if (lane == 0) sm.above[warp] += v;
+    }
+    uint32_t nlo, nhi;
+    bin_range(klo, khi, shift, bstar, nlo, nhi);
+    if (level == 0 && bstar == 0) nlo = 1u;  // valid keys are >= 1
+    if (level == 0 && bstar == bmax) nhi = 0xFFFFFFFFu;
+    const bool tie = nlo == nhi;  // the boundary bin is one key value
+    const bool gather = !tie && bcount <= static_cast<uint32_t>(TK_CAP);
+    if (!tie && !gather) {
+      klo = nlo;
+      khi = nhi;
+      continue;
+    }
+    // ---- final level: per-warp counts above the bin; the bin's elements gathered (or, for a one-key
+    // bin, counted as ties) ----
+    if (gather) {
+      if (tid < C) {
+        uint32_t o = 0;
+        for (int c = 0; c < tid; ++c) o += hl[c * TK_BINS + bstar];
+        sm.segoff[tid] = o;
+        sm.segcnt[tid] = hl[tid * TK_BINS + bstar];
+      }
+      if (tid == 0) sm.ccount = 0;
       __syncthreads();
-      if (warp == 0) {
-        lo = lane < TK_WARPS ? sm.wa[lane] : 0xFFFFFFFFu;
-        hi = lane < TK_WARPS ? sm.wb[lane] : 0u;
-        #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-          hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-        }
-        if (lane < C) {
-          *cluster.map_shared_rank(&sm.kmin[r], lane) = lo;
-          *cluster.map_shared_rank(&sm.kmax[r], lane) = hi;
+    }
+    const uint32_t off = gather ? sm.segoff[r] : 0u;
+    uint32_t nab = 0, nin = 0;
+    for (int g = gw0 + lane; g < gw1; g += 32) {
+      const uint4 k4 = ch.load(g);
+      const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
+      #pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        nab += k[e] > nhi;
+        if (k[e] >= nlo && k[e] <= nhi) {
+          if (gather) {
+            const uint32_t slot = atomicAdd(&sm.ccount, 1u);
+            sm.cand[off + slot] = k[e];
+            sm.cand_w[slot] = static_cast<uint8_t>(warp);
+          } else {
+            ++nin;
+          }
         }
       }
-      cluster.sync();
-      klo = 0xFFFFFFFFu;
-      khi = 0u;
-      for (int c = 0; c < C; ++c) {
-        klo = min(klo, sm.kmin[c]);
-        khi = max(khi, sm.kmax[c]);
+    }
+    nab = warp_sum_u32(nab);
+    nin = warp_sum_u32(nin);
+    if (lane == 0) {
+      sm.wgt[warp] = nab;  // gathered elements above T are added after the local refinement
+      sm.weq[warp] = nin;
+    }
+    if (tie) {
+      T = nlo;
+      need_eq = need;
+      if (tid < C) {
+        sm.gtb[tid] = 0;
+        sm.eqb[tid] = hl[tid * TK_BINS + bstar];
       }
     } else {
-      const uint32_t nlo = klo + (bstar << shift);
-      const uint64_t nhi = static_cast<uint64_t>(nlo) + ((1ull << shift) - 1ull);
+      __syncthreads();
+      const uint32_t mine = sm.segcnt[r];
+      for (uint32_t i = tid; i < mine * static_cast<uint32_t>(C); i += TK_THREADS) {
+        const uint32_t c = i / mine, j = off + (i - c * mine);
+        if (static_cast<int>(c) != r) *cluster.map_shared_rank(&sm.cand[j], static_cast<int>(c)) = sm.cand[j];
+      }
+      cluster.sync();  // last cluster barrier of this path: no DSMEM access after it
       klo = nlo;
-      khi = static_cast<uint32_t>(nhi < khi ? nhi : khi);
+      khi = nhi;
+      gathered = true;
     }
-    if (klo == khi) {
-      T = klo;
-      need_eq = need;
-      resolved = true;
-      break;
-    }
-    const uint32_t span = khi - klo;
-    const int bits = 32 - __clz(span);
-    shift = bits > 12 ? bits - 12 : 0;
+    break;
   }
-  (void)resolved;
 
-  // ---- ordered compaction: selected = key > T, or key == T among the first need_eq of them ----
-  const int n = max(0, a1 - a0);
-  const int per_w = ((n + TK_WARPS - 1) / TK_WARPS + 127) & ~127;  // multiple of 128: 4 chunks per pass
-  const int w0 = a0 + warp * per_w;
-  const int w1 = min(a1, w0 + per_w);
-  uint32_t gt_w = 0, eq_w = 0;
-  for (int s0 = w0; s0 < w1; s0 += 128) {
-    uint32_t k[4];
-    #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int s = s0 + 32 * u + lane;
-      k[u] = s < w1 ? f32_order_key(row.val(s)) : 0u;
+  if (gathered) {
+    // ---- local refinement of the gathered boundary bin (every CTA redundantly, no communication) ----
+    const uint32_t n = sm.sel_count;
+    for (int lv = 0; lv < 6; ++lv) {
+      const int shift = level_shift(klo, khi);
+      __syncthreads();  // sel_* and h are rewritten below
+      if (tid < TK_BINS) sm.h[tid] = 0;
+      __syncthreads();
+      for (uint32_t j = tid; j < n; j += TK_THREADS) {
+        const uint32_t k = sm.cand[j];
+        if (k >= klo && k <= khi) atomicAdd(&sm.h[(k - klo) >> shift], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) find_boundary(sm, sm.h, need, lane);
+      __syncthreads();
+      need -= sm.sel_above;
+      uint32_t nlo, nhi;
+      bin_range(klo, khi, shift, sm.sel_bin, nlo, nhi);
+      klo = nlo;
+      khi = nhi;
+      if (nlo == nhi) break;  // reached at shift 0 at the latest
     }
-    #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const bool in = s0 + 32 * u + lane < w1;
-      gt_w += __popc(__ballot_sync(0xffffffffu, in && k[u] > T));
-      eq_w += __popc(__ballot_sync(0xffffffffu, in && k[u] == T));
+    T = klo;
+    need_eq = need;
+    if (warp < C) {  // CTA `warp`'s boundary elements above / at T
+      const uint32_t o = sm.segoff[warp], m = sm.segcnt[warp];
+      uint32_t g = 0, e = 0;
+      for (uint32_t j = lane; j < m; j += 32) {
+        const uint32_t k = sm.cand[o + j];
+        g += k > T;
+        e += k == T;
+      }
+      g = warp_sum_u32(g);
+      e = warp_sum_u32(e);
+      if (lane == 0) {
+        sm.gtb[warp] = g;
+        sm.eqb[warp] = e;
+      }
     }
-  }
-  if (lane == 0) {
-    sm.wa[warp] = gt_w;
-    sm.wb[warp] = eq_w;
+    // my own boundary elements, attributed to the warps that hold them
+    const uint32_t off = sm.segoff[r], mine = sm.segcnt[r];
+    for (uint32_t j = tid; j < mine; j += TK_THREADS) {
+      const uint32_t k = sm.cand[off + j];
+      if (k > T) atomicAdd(&sm.wgt[sm.cand_w[j]], 1u);
+      if (k == T) atomicAdd(&sm.weq[sm.cand_w[j]], 1u);
+    }
   }
   __syncthreads();
-  if (warp == 0) {
-    const uint32_t g = warp_sum_u32(lane < TK_WARPS ? sm.wa[lane] : 0u);
-    const uint32_t e = warp_sum_u32(lane < TK_WARPS ? sm.wb[lane] : 0u);
-    if (lane < C) {
-      *cluster.map_shared_rank(&sm.cgt[r], lane) = g;
-      *cluster.map_shared_rank(&sm.ceq[r], lane) = e;
+
+  // ---- this CTA's output offset and its share of the ties (ties go to the lowest positions) ----
+  uint32_t base = static_cast<uint32_t>(rs.nsink), eq_seen = 0, take = 0;
+  for (int c = 0; c <= r; ++c) {
+    const uint32_t tk = min(need_eq - min(eq_seen, need_eq), sm.eqb[c]);
+    if (c == r) {
+      take = tk;
+    } else {
+      base += sm.above[c] + sm.gtb[c] + tk;
     }
+    eq_seen += sm.eqb[c];
   }
-  cluster.sync();
-  uint32_t gt_before = 0, eq_before = 0;
-  for (int c = 0; c < r; ++c) {
-    gt_before += sm.cgt[c];
-    eq_before += sm.ceq[c];
-  }
-  // exclusive gt / eq prefixes of my warp inside the CTA
-  uint32_t gt_wbefore = 0, eq_wbefore = 0;
+  uint32_t gt_run = 0, eq_run = 0;  // this CTA's elements > T / == T in the warps before mine
   for (int w = 0; w < warp; ++w) {
-    gt_wbefore += sm.wa[w];
-    eq_wbefore += sm.wb[w];
+    gt_run += sm.wgt[w];
+    eq_run += sm.weq[w];
   }
-  // a selected element's output slot = nsink + (#greater before it) + min(#equal before it, need_eq)
-  {
-    uint32_t run_gt = gt_before + gt_wbefore;
-    uint32_t run_eq = eq_before + eq_wbefore;
-    const uint32_t lim = static_cast<uint32_t>(nsink + nsel);
-    for (int s00 = w0; s00 < w1; s00 += 128) {
-     uint32_t kk[4];
-     #pragma unroll
-     for (int u = 0; u < 4; ++u) {
-       const int s = s00 + 32 * u + lane;
-       kk[u] = s < w1 ? f32_order_key(row.val(s)) : 0u;
-     }
-     #pragma unroll
-     for (int u = 0; u < 4; ++u) {
-      const int s = s00 + 32 * u + lane;
-      const uint32_t k = kk[u];
-      const bool is_gt = s < w1 && k > T;
-      const bool is_eq = s < w1 && k == T;
-      const uint32_t gtm = __ballot_sync(0xffffffffu, is_gt);
-      const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
-      const uint32_t lt = lanemask_lt();
-      const uint32_t eq_before_me = run_eq + __popc(eqm & lt);
-      const bool sel = is_gt || (is_eq && eq_before_me < need_eq);
-      const uint32_t o = static_cast<uint32_t>(nsink) + run_gt + __popc(gtm & lt) + min(eq_before_me, need_eq);
-      if (sel && o < lim) out[o] = s;  // bounded even if T were wrong
-      run_gt += __popc(gtm);
-      run_eq += __popc(eqm);
-     }
+
+  // ---- ordered write: a selected element's slot = base + (#gt before it) + min(#eq before it, take) ----
+  const uint32_t lim = static_cast<uint32_t>(rs.nsink + rs.nsel);
+  const uint32_t lt = lanemask_lt();
+  for (int g0 = gw0; g0 < gw1; g0 += 32) {
+    const int g = g0 + lane;
+    uint4 k4 = make_uint4(0u, 0u, 0u, 0u);
+    if (g < gw1) k4 = ch.load(g);
+    const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
+    uint32_t ngt = 0, neq = 0;
+    #pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      ngt += k[e] > T;
+      neq += k[e] == T;
     }
+    uint32_t gtot, etot = 0, epre = 0;
+    const uint32_t gpre = ballot_prefix(ngt, lt, gtot);
+    if (__any_sync(0xffffffffu, neq != 0)) epre = ballot_prefix(neq, lt, etot);
+    if (ngt | neq) {
+      uint32_t gb = gt_run + gpre, eb = eq_run + epre;
+      const int s0 = c0 + 4 * g;
+      #pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool gt = k[e] > T, eq = k[e] == T;
+        if (gt || (eq && eb < take)) {
+          const uint32_t o = base + gb + min(eb, take);
+          if (o < lim) rs.out[o] = s0 + e;  // bounded even if the counts were inconsistent
+        }
+        gb += gt;
+        eb += eq;
+      }
+    }
+    gt_run += gtot;
+    eq_run += etot;
   }
-  // keep this CTA's shared memory alive until every remote access of the cluster is done
-  cluster.sync();
+}
+
+// Clusters of C CTAs (one CTA per SM) that can be resident at once on the current device.
+int resident_clusters(int C) {
+  static std::mutex mu;
+  static int table[64][TK_MAXC + 1];
+  static bool done[64][TK_MAXC + 1];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev][C]) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, 1, 1);
+    cfg.blockDim = dim3(TK_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = 120 * 1024;  // more than half an SM's shared memory: one CTA per SM
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_topk_cluster, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = 1;
+    }
+    table[dev][C] = n;
+    done[dev][C] = true;
+  }
+  return table[dev][C];
 }
 
 }  // namespace
@@ -509,13 +595,25 @@ int launch_topk_mode(const float* scores, int64_t ld, int64_t B, int64_t L, int 
                      const int64_t* q_pos, int mode, int div, int32_t* idx, int64_t idx_ld, int32_t* count,
                      int64_t kmax, cudaStream_t s) {
   if (B == 0) return LSA_OK;
-  // cluster size: smallest power of two whose chunk fits the shared-memory cache, <= 16
-  const int64_t cache_elems = 20 * 1024;  // 80 KB of fp32 scores per CTA (two CTAs per SM)
-  int C = 1;
-  while (C < TK_MAXC && cdiv(L, C) > cache_elems) C *= 2;
-  while (C < 8 && cdiv(L, C) > 16384) C *= 2;  // spread mid-size rows over more SMs
+  LSA_CUDA_TRY(cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    2 * TK_MAXC * TK_BINS * 4 + TK_CACHE * 4));
+  LSA_CUDA_TRY(cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+  // Cluster size: among the sizes whose chunk fits the shared-memory cache, the one with the least work
+  // on the busiest SM -- (chunk + a fixed per-CTA cost) x the number of cluster waves the batch needs.
+  // Rows too long for any cluster's cache are streamed from global memory by clusters of 16.
+  int C = TK_MAXC;
+  double best = -1.0;
+  for (int c = 1; c <= TK_MAXC; ++c) {
+    const int64_t chunk = (cdiv(L, c) + 3) / 4 * 4;
+    if (chunk > TK_CACHE) continue;
+    const double waves = static_cast<double>(cdiv(B, resident_clusters(c)));
+    const double cost = (static_cast<double>(chunk) + 2048.0) * waves;
+    if (best < 0.0 || cost < best) {
+      best = cost;
+      C = c;
+    }
+  }
   int64_t chunk = (cdiv(L, C) + 3) / 4 * 4;
-  const int cached = chunk <= cache_elems ? 1 : 0;
   if (chunk == 0) chunk = 4;
   TopkArgs a;
   a.scores = scores;
@@ -532,11 +630,9 @@ int launch_topk_mode(const float* scores, int64_t ld, int64_t B, int64_t L, int 
   a.count = count;
   a.kmax = static_cast<int>(kmax);
   a.chunk = static_cast<int>(chunk);
-  a.cached = cached;
-  const size_t dyn = cached ? static_cast<size_t>(chunk) * 4 : 0;
-  LSA_CUDA_TRY(cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(cache_elems * 4)));
-  LSA_CUDA_TRY(cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+  a.cached = chunk <= TK_CACHE ? 1 : 0;
+  // all-gathered histograms (two levels' worth), then the cached chunk
+  const size_t dyn = static_cast<size_t>(2 * C * TK_BINS) * 4 + (a.cached ? static_cast<size_t>(chunk) * 4 : 0);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, static_cast<unsigned>(B), 1);
   cfg.blockDim = dim3(TK_THREADS, 1, 1);
