@@ -122,7 +122,7 @@ int launch_attn_simt(const void* q, const void* kv, int64_t L, const int32_t* id
                      const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, cudaStream_t s) {
   if (B == 0) return LSA_OK;
   const size_t smem = AS_HG * AS_DQK * 4 + AS_TILE * AS_STRIDE * 2 + AS_HG * AS_TILE * 4 + 3 * AS_HG * 4;
-  LSA_CUDA_TRY(cudaFuncSetAttribute(k_attn_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+  LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_attn_simt), static_cast<int>(smem)));
   const dim3 grid(static_cast<unsigned>(H / AS_HG), static_cast<unsigned>(B));
   k_attn_simt<<<grid, AS_THREADS, smem, s>>>(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(kv), L, idx,
                                             idx_ld, count, H, scale, static_cast<uint16_t*>(out), lse);

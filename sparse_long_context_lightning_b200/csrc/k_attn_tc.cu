@@ -498,7 +498,7 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   a.ws_ml = S > 1 ? reinterpret_cast<float*>(static_cast<unsigned char*>(ws) +
                                              align_up(static_cast<size_t>(B) * S * AT_H * 512 * 4, 256))
                   : nullptr;
-  LSA_CUDA_TRY(cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM));
+  LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_sparse_attn_tc), AT_SMEM));
   const int64_t grid = 2 * B * S;
   if (grid > 0x7FFFFFFF) return LSA_ERR_UNSUPPORTED;
   k_sparse_attn_tc<<<static_cast<unsigned>(grid), AT_THREADS, AT_SMEM, s>>>(tq, a);

@@ -244,7 +244,7 @@ int launch_tc(const void* q, const float* q_scale, const float* w, const void* k
   if (ranges > a.ntiles) ranges = a.ntiles;
   a.tiles_per_range = static_cast<int>(cdiv(a.ntiles, ranges));
   ranges = static_cast<int>(cdiv(a.ntiles, a.tiles_per_range));
-  LSA_CUDA_TRY(cudaFuncSetAttribute(k_index_score_tc<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+  LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_index_score_tc<FP8>), C::SMEM));
   const int64_t grid = static_cast<int64_t>(a.n_chunks) * ranges;
   k_index_score_tc<FP8><<<static_cast<unsigned>(grid), IX_THREADS, C::SMEM, s>>>(tk, tq, a);
   return cuda_status(cudaGetLastError());

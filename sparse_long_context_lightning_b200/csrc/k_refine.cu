@@ -160,7 +160,7 @@ int launch_refine(const void* q, const float* w, const void* k, int64_t B, int H
                                                    rs, out_ld, ndyn_m1);
       break;
     case 128:
-      LSA_CUDA_TRY(cudaFuncSetAttribute(k_rescore<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
+      LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_rescore<128>), 64 * 1024));
       k_rescore<128><<<grid, RF_THREADS, smem, s>>>(qq, w, kk, H_I, L, cand, cand_ld, cand_count, q_pos, sink,
                                                     window, rs, out_ld, ndyn_m1);
       break;

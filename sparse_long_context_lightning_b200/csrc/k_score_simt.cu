@@ -113,15 +113,15 @@ int launch_kt(const void* q, int q_fp8, const float* q_scale, const float* w, co
   const size_t smem = static_cast<size_t>(H_I) * d_I * 4 + static_cast<size_t>(H_I) * 4;
   switch (d_I) {
     case 32:
-      LSA_CUDA_TRY(cudaFuncSetAttribute(k_score_simt<KT, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
+      LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_score_simt<KT, 32>), 64 * 1024));
       k_score_simt<KT, 32><<<grid, SC_THREADS, smem, st>>>(q, q_fp8, q_scale, w, k, k_scale, H_I, L, B, q_pos, out, ld);
       break;
     case 64:
-      LSA_CUDA_TRY(cudaFuncSetAttribute(k_score_simt<KT, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
+      LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_score_simt<KT, 64>), 64 * 1024));
       k_score_simt<KT, 64><<<grid, SC_THREADS, smem, st>>>(q, q_fp8, q_scale, w, k, k_scale, H_I, L, B, q_pos, out, ld);
       break;
     case 128:
-      LSA_CUDA_TRY(cudaFuncSetAttribute(k_score_simt<KT, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
+      LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_score_simt<KT, 128>), 64 * 1024));
       k_score_simt<KT, 128><<<grid, SC_THREADS, smem, st>>>(q, q_fp8, q_scale, w, k, k_scale, H_I, L, B, q_pos, out, ld);
       break;
     default:

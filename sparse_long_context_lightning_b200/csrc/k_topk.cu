@@ -31,6 +31,7 @@ constexpr int TK_BINS = 256;   // one 8-bit digit of the order key per refinemen
 constexpr int TK_CAP = 1024;   // boundary-bin size that is all-gathered and finished locally
 constexpr int TK_MAXC = 16;    // cluster size limit (non-portable above 8)
 constexpr int TK_CACHE = 24576;  // scores per CTA kept in shared memory (96 KB)
+constexpr int TK_PIECES = 4;     // the chunk arrives in this many bulk copies; each warp waits for its own
 
 enum { MODE_TOKEN = 0, MODE_ALL = 1, MODE_BLOCKS = 2 };
 
@@ -67,7 +68,8 @@ struct TopkSmem {
   uint32_t wgt[TK_WARPS], weq[TK_WARPS];  // this CTA's elements with key > T / key == T, per warp
   uint32_t ccount;
   uint32_t sel_bin, sel_above, sel_count;
-  uint64_t load_bar;
+  uint32_t res_T, res_need_eq;
+  uint64_t load_bar[TK_PIECES];  // one per piece of the chunk's bulk copy
 };
 
 __device__ __forceinline__ void cluster_arrive_relaxed() {
@@ -156,15 +158,19 @@ struct Chunk {
     }
     return k;
   }
-  __device__ __forceinline__ uint4 load(int g) const {
-    if (keys) return keys[g];
+  // the group's scores straight from global memory (0 outside [a0, a1))
+  __device__ __forceinline__ float4 gload(int g) const {
     const int s0 = c0 + 4 * g;
     float4 v;
     v.x = (s0 >= a0 && s0 < a1) ? __ldg(grow + s0) : 0.f;
     v.y = (s0 + 1 >= a0 && s0 + 1 < a1) ? __ldg(grow + s0 + 1) : 0.f;
     v.z = (s0 + 2 >= a0 && s0 + 2 < a1) ? __ldg(grow + s0 + 2) : 0.f;
     v.w = (s0 + 3 >= a0 && s0 + 3 < a1) ? __ldg(grow + s0 + 3) : 0.f;
-    return from_scores(g, v);
+    return v;
+  }
+  __device__ __forceinline__ uint4 load(int g) const {
+    if (keys) return keys[g];
+    return from_scores(g, gload(g));
   }
 };
 
@@ -258,56 +264,87 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
   const int ng = a1 > a0 ? (a1 - c0 + 3) / 4 : 0;  // groups [g_lo, ng) hold my candidates
   const int g_lo = a1 > a0 ? (a0 - c0) / 4 : 0;
   float4* cache = reinterpret_cast<float4*>(dyn + static_cast<size_t>(2 * C * TK_BINS) * 4);
-  if (a.cached) {
-    float* cf = reinterpret_cast<float*>(cache);
-    const int lend = min(c1, rs.chi);
-    const bool aligned = (reinterpret_cast<uintptr_t>(ch.grow + c0) & 15u) == 0;
-    const int nvec = aligned ? max(0, (lend - c0) / 4) : 0;
-    if (tid == 0) {
-      sm100::mbar_init(&sm.load_bar, 1);
-      sm100::fence_mbar_init();
-    }
-    __syncthreads();
-    if (tid == 0) {
-      if (nvec > 0) {
-        sm100::mbar_expect_tx(&sm.load_bar, static_cast<uint32_t>(nvec) * 16u);
-        sm100::bulk_load(cf, ch.grow + c0, static_cast<uint32_t>(nvec) * 16u, &sm.load_bar);
-      } else {
-        sm100::mbar_arrive(&sm.load_bar);
-      }
-    }
-    // the unaligned rest (or the whole chunk when the row is not 16-byte aligned) by plain loads
-    for (int s = c0 + nvec * 4 + tid; s < 4 * ng + c0; s += TK_THREADS) cf[s - c0] = s < lend ? ch.grow[s] : 0.f;
-    // bounded wait (the copy is in bounds by construction)
-    sm100::mbar_wait(&sm.load_bar, 0);
-    __syncthreads();
-  }
   // warp w walks groups [gw0, gw1); lane l takes every 32nd group from gw0 + l
   const int per_w = (ng - g_lo + TK_WARPS - 1) / TK_WARPS;
   const int gw0 = g_lo + warp * per_w;
   const int gw1 = min(ng, gw0 + per_w);
+  // Cached rows: groups [g_lo, nvec) arrive in TK_PIECES bulk copies of pg groups (16-byte aligned rows
+  // only); the rest -- a ragged last group, or every group of an unaligned row -- is read from global
+  // memory by the thread that converts it.  Each warp waits for the pieces its groups lie in, so every
+  // copy is waited for before the CTA can exit.
+  int nvec = 0, pg = 1;
+  if (a.cached) {
+    const bool aligned = (reinterpret_cast<uintptr_t>(ch.grow + c0) & 15u) == 0;
+    nvec = (aligned && ng > g_lo) ? (a1 - c0) / 4 : 0;
+    const int npv = max(0, nvec - g_lo);
+    pg = max(1, (npv + TK_PIECES - 1) / TK_PIECES);
+    if (tid == 0) {
+      for (int p = 0; p < TK_PIECES; ++p) sm100::mbar_init(&sm.load_bar[p], 1);
+      sm100::fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+      for (int p = 0; p < TK_PIECES; ++p) {
+        const int p0 = g_lo + p * pg, p1 = min(nvec, p0 + pg);
+        if (p1 > p0) {
+          sm100::mbar_expect_tx(&sm.load_bar[p], static_cast<uint32_t>(p1 - p0) * 16u);
+          sm100::bulk_load(cache + p0, ch.grow + c0 + 4 * p0, static_cast<uint32_t>(p1 - p0) * 16u, &sm.load_bar[p]);
+        } else {
+          sm100::mbar_arrive(&sm.load_bar[p]);
+        }
+      }
+    }
+    if (gw1 > gw0 && gw0 < nvec) {
+      // bounded waits (the copies are in bounds by construction)
+      const int plast = (min(gw1, nvec) - 1 - g_lo) / pg;
+      for (int p = (gw0 - g_lo) / pg; p <= plast; ++p) sm100::mbar_wait(&sm.load_bar[p], 0);
+    }
+  }
 
   // ---- order keys (in place, when cached) and the finite key range of the candidates ----
   {
-    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    uint32_t lo1 = 0xFFFFFFFFu, hi = 0u;  // lo1 = min(key) - 1 over valid keys (invalid: 0 - 1 = max)
     for (int g = gw0 + lane; g < gw1; g += 32) {
       uint4 k;
       if (a.cached) {
-        k = ch.from_scores(g, cache[g]);
+        k = ch.from_scores(g, g < nvec ? cache[g] : ch.gload(g));
         reinterpret_cast<uint4*>(cache)[g] = k;
       } else {
         k = ch.load(g);
       }
-      if (key_finite(k.x)) { lo = min(lo, k.x); hi = max(hi, k.x); }
-      if (key_finite(k.y)) { lo = min(lo, k.y); hi = max(hi, k.y); }
-      if (key_finite(k.z)) { lo = min(lo, k.z); hi = max(hi, k.z); }
-      if (key_finite(k.w)) { lo = min(lo, k.w); hi = max(hi, k.w); }
+      lo1 = min(min(lo1, k.x - 1u), min(k.y - 1u, min(k.z - 1u, k.w - 1u)));
+      hi = max(max(hi, k.x), max(k.y, max(k.z, k.w)));
     }
     if (a.cached) ch.keys = reinterpret_cast<const uint4*>(cache);  // each thread reads back only its own groups
+    uint32_t lo = lo1 + 1u;  // 0 when this thread saw no valid key
     #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      lo1 = min(lo1, __shfl_xor_sync(0xffffffffu, lo1, o));
       hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    lo = lo1 + 1u;
+    if (hi != 0u && (!key_finite(lo) || !key_finite(hi))) {
+      // non-finite scores in this warp's range (rare): redo the warp's range over finite keys only
+      lo = 0xFFFFFFFFu;
+      hi = 0u;
+      for (int g = gw0 + lane; g < gw1; g += 32) {
+        const uint4 k4 = ch.load(g);
+        const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (key_finite(k[e])) {
+            lo = min(lo, k[e]);
+            hi = max(hi, k[e]);
+          }
+        }
+      }
+      #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      }
+    } else if (hi == 0u) {
+      lo = 0xFFFFFFFFu;  // no valid key in this warp's range
     }
     if (lane == 0) {
       sm.wa[warp] = lo;
@@ -457,29 +494,38 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
   }
 
   if (gathered) {
-    // ---- local refinement of the gathered boundary bin (every CTA redundantly, no communication) ----
-    const uint32_t n = sm.sel_count;
-    for (int lv = 0; lv < 6; ++lv) {
-      const int shift = level_shift(klo, khi);
-      __syncthreads();  // sel_* and h are rewritten below
-      if (tid < TK_BINS) sm.h[tid] = 0;
-      __syncthreads();
-      for (uint32_t j = tid; j < n; j += TK_THREADS) {
-        const uint32_t k = sm.cand[j];
-        if (k >= klo && k <= khi) atomicAdd(&sm.h[(k - klo) >> shift], 1u);
+    // ---- local refinement of the gathered boundary bin: warp 0 of every CTA, redundantly, with no
+    // block or cluster barrier between levels ----
+    if (warp == 0) {
+      const uint32_t n = sm.sel_count;
+      for (int lv = 0; lv < 6; ++lv) {
+        const int shift = level_shift(klo, khi);
+        reinterpret_cast<uint4*>(sm.h)[2 * lane] = make_uint4(0u, 0u, 0u, 0u);
+        reinterpret_cast<uint4*>(sm.h)[2 * lane + 1] = make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
+        for (uint32_t j = lane; j < n; j += 32) {
+          const uint32_t k = sm.cand[j];
+          if (k >= klo && k <= khi) atomicAdd(&sm.h[(k - klo) >> shift], 1u);
+        }
+        __syncwarp();
+        find_boundary(sm, sm.h, need, lane);
+        __syncwarp();
+        need -= sm.sel_above;
+        uint32_t nlo, nhi;
+        bin_range(klo, khi, shift, sm.sel_bin, nlo, nhi);
+        klo = nlo;
+        khi = nhi;
+        __syncwarp();  // every lane has read sel_* and h before the next level rewrites them
+        if (nlo == nhi) break;  // reached at shift 0 at the latest
       }
-      __syncthreads();
-      if (warp == 0) find_boundary(sm, sm.h, need, lane);
-      __syncthreads();
-      need -= sm.sel_above;
-      uint32_t nlo, nhi;
-      bin_range(klo, khi, shift, sm.sel_bin, nlo, nhi);
-      klo = nlo;
-      khi = nhi;
-      if (nlo == nhi) break;  // reached at shift 0 at the latest
+      if (lane == 0) {
+        sm.res_T = klo;
+        sm.res_need_eq = need;
+      }
     }
-    T = klo;
-    need_eq = need;
+    __syncthreads();
+    T = sm.res_T;
+    need_eq = sm.res_need_eq;
     if (warp < C) {  // CTA `warp`'s boundary elements above / at T
       const uint32_t o = sm.segoff[warp], m = sm.segcnt[warp];
       uint32_t g = 0, e = 0;
@@ -539,7 +585,19 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     uint32_t gtot, etot = 0, epre = 0;
     const uint32_t gpre = ballot_prefix(ngt, lt, gtot);
     if (__any_sync(0xffffffffu, neq != 0)) epre = ballot_prefix(neq, lt, etot);
-    if (ngt | neq) {
+    if (etot == 0u) {  // no ties in this step of the warp (the common case): gt elements only
+      if (ngt) {
+        uint32_t o = base + gt_run + gpre + min(eq_run, take);
+        const int s0 = c0 + 4 * g;
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (k[e] > T) {
+            if (o < lim) rs.out[o] = s0 + e;  // bounded even if the counts were inconsistent
+            ++o;
+          }
+        }
+      }
+    } else if (ngt | neq) {
       uint32_t gb = gt_run + gpre, eb = eq_run + epre;
       const int s0 = c0 + 4 * g;
       #pragma unroll
@@ -547,7 +605,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
         const bool gt = k[e] > T, eq = k[e] == T;
         if (gt || (eq && eb < take)) {
           const uint32_t o = base + gb + min(eb, take);
-          if (o < lim) rs.out[o] = s0 + e;  // bounded even if the counts were inconsistent
+          if (o < lim) rs.out[o] = s0 + e;
         }
         gb += gt;
         eb += eq;
@@ -595,9 +653,20 @@ int launch_topk_mode(const float* scores, int64_t ld, int64_t B, int64_t L, int 
                      const int64_t* q_pos, int mode, int div, int32_t* idx, int64_t idx_ld, int32_t* count,
                      int64_t kmax, cudaStream_t s) {
   if (B == 0) return LSA_OK;
-  LSA_CUDA_TRY(cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    2 * TK_MAXC * TK_BINS * 4 + TK_CACHE * 4));
-  LSA_CUDA_TRY(cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+  {
+    // the kernel's attributes, once per device (host calls stay off the launch path)
+    static std::mutex mu;
+    static bool set[64];
+    int dev = 0;
+    LSA_CUDA_TRY(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64 || !set[dev]) {
+      LSA_CUDA_TRY(cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        2 * TK_MAXC * TK_BINS * 4 + TK_CACHE * 4));
+      LSA_CUDA_TRY(cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+      if (dev >= 0 && dev < 64) set[dev] = true;
+    }
+  }
   // Cluster size: among the sizes whose chunk fits the shared-memory cache, the one with the least work
   // on the busiest SM -- (chunk + a fixed per-CTA cost) x the number of cluster waves the batch needs.
   // Rows too long for any cluster's cache are streamed from global memory by clusters of 16.

@@ -6,6 +6,9 @@
 #include <cooperative_groups.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <vector>
+
 #include "../../include/lsa.h"
 
 namespace cg = cooperative_groups;
@@ -28,6 +31,27 @@ int cuda_status(cudaError_t e);  // LSA_OK or LSA_ERR_CUDA (+ records the messag
     cudaError_t e_ = (expr);                         \
     if (e_ != cudaSuccess) return lsa::cuda_status(e_); \
   } while (0)
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device): the attribute outlives
+// the launch, so later launches skip the host call.
+inline cudaError_t func_smem_once(const void* f, int bytes) {
+  struct Entry {
+    const void* f;
+    int dev;
+    int bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& x : done)
+    if (x.f == f && x.dev == dev && x.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.push_back(Entry{f, dev, bytes});
+  return e;
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
