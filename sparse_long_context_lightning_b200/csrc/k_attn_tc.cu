@@ -5,21 +5,25 @@
 // selected 1152-byte rows are scattered, so the kernel is a gather whose memory-level parallelism decides
 // the achieved bandwidth.
 //
-// B200 design.  A 128 x 512 fp32 output accumulator fills all of TMEM (128 lanes x 512 columns), leaving
-// no room for the logits, so one work unit (query b, a contiguous split of its selected rows) runs on a
-// 2-CTA cluster: CTA r owns output columns [256r, 256r+256) and latent dims D_0 = [0, 256), D_1 =
-// [256, 576).  Each CTA gathers only its own part of every selected row (512 or 640 bytes, disjoint), with
-// 16-byte cp.async copies from four gather warps into 128-byte-swizzled shared memory (many rows in flight
-// per SM; a TMA gather4 per 4 rows x 128 bytes issued too slowly here), computes the partial logits
-// S_r = Q[:, D_r] . C[:, D_r]^T, and the two partials are exchanged through distributed shared memory
-// (one bulk shared-to-shared copy per warp and tile, completing on the peer's mbarrier).  Both CTAs then hold the same logits,
-// run the same online softmax (lazy rescale: O is rescaled only when the running max grows by > 2^8),
-// and each accumulates P . V[:, its 256 columns] in TMEM.  The gathered tile serves both MMAs: K-major for
-// S = Q C^T and MN-major for O += P V, so no transpose is needed.  Splits of one query are merged by a
-// small combine kernel (log-sum-exp weights).
+// B200 design.  A 128 x 512 fp32 output accumulator would fill all of TMEM (128 lanes x 512 columns), so
+// the value dims are split over two CTAs: CTA (unit, r) owns output columns [256r, 256r + 256) of one
+// work unit (query b, a contiguous split of its selected rows).  The two CTAs are independent -- no
+// cluster, no per-tile communication: each gathers the full 1152-byte rows of its tiles (the pair reads
+// the same rows at about the same time, so the second read is served by L2) and computes the complete
+// logits S = Q C^T itself.  Duplicating the logits MMA costs less than exchanging partial logits between
+// CTAs, whose DSMEM latency made every tile wait.
 //
-// Warp roles (288 threads): warps 0-3 gather, warp 4 issues MMAs (S two tiles ahead of P.V) and owns TMEM,
-// warps 5-8 run the softmax (one head per thread = one TMEM lane) and the epilogue.
+// TMEM (512 columns): O [0, 256), two S buffers [256, 320), and Q's dims [0, 384) as the A operand of the
+// logits MMA [320, 512) (two bf16 per column).  Q's dims [384, 576) stay in shared memory (48 KB).  The
+// gathered tile (32 rows x 9 K-blocks of 64 dims, 128-byte swizzled) serves both MMAs: K-major for
+// S = Q C^T and MN-major (its first 512 dims) for O += P V, so no transpose is needed.  Online softmax with
+// lazy rescale (O is rescaled only when the running max grows by > 2^8).  Splits of one query are merged
+// by a small combine kernel (log-sum-exp weights).
+//
+// Warp roles (288 threads): warps 0-3 gather (16-byte cp.async copies, many rows in flight per SM; a TMA
+// gather4 per 4 rows x 128 bytes issued too slowly here), warp 4 issues the MMAs (S two tiles ahead of
+// P.V) and owns TMEM, warps 5-8 load Q into TMEM, then run the softmax (one head per thread = one TMEM
+// lane) and the epilogue.
 #include "lsa_common.cuh"
 #include "sm100.cuh"
 
@@ -30,29 +34,33 @@ using namespace sm100;
 
 __device__ int g_attn_tc_timeout;  // set when a bounded wait of the kernel gave up
 
-constexpr int AT_THREADS = 288;  // 4 gather warps, 1 MMA warp, 4 softmax warps
+constexpr int AT_THREADS = 352;  // 4 gather warps, 4 softmax warps, 3 MMA-issuing warps
 constexpr int AT_GATHER_WARPS = 4;
-constexpr int AT_MMA_WARP = 4;
-constexpr int AT_SM_TID0 = 160;  // first softmax thread
-constexpr int AT_T = 32;   // gathered rows per tile
-constexpr int AT_H = 128;  // heads (MMA M)
-constexpr int AT_KBQ_MAX = 5;
+constexpr int AT_MMA_WARP = 4;   // logits of even tiles; owns TMEM
+constexpr int AT_MMA_WARP2 = 9;  // logits of odd tiles
+constexpr int AT_PV_WARP = 10;   // O += P V
+constexpr int AT_T = 32;         // gathered rows per tile
+constexpr int AT_H = 128;        // heads (MMA M)
+constexpr int AT_KB = 9;         // 64-dim K-blocks of a 576-dim row
+constexpr int AT_KB_TQ = 6;      // Q K-blocks held in TMEM (dims [0, 384))
+constexpr int AT_KB_SQ = AT_KB - AT_KB_TQ;  // Q K-blocks in shared memory (dims [384, 576))
 constexpr int AT_STAGES = 4;
-constexpr int AT_Q_BYTES = AT_KBQ_MAX * AT_H * 128;        // 80 KB
+constexpr int AT_QS_BYTES = AT_KB_SQ * AT_H * 128;         // 48 KB
 constexpr int AT_KB_BYTES = AT_T * 128;                    // 4 KB: one 64-dim block of a tile
-constexpr int AT_STAGE_BYTES = AT_KBQ_MAX * AT_KB_BYTES;   // 20 KB
-constexpr int AT_P_BYTES = AT_H * 128;                     // 16 KB
-constexpr int AT_SX_FLOATS = AT_H * AT_T;                   // 16 KB: partial logits [head][row], 16-byte chunks
-                                                            // of a row swizzled by (head & 7)
-constexpr uint32_t AT_SX_TX = AT_H * AT_T * 4;              // bytes the peer sends per tile
-constexpr int AT_SMEM = 1024 + AT_Q_BYTES + AT_STAGES * AT_STAGE_BYTES + AT_P_BYTES + 3 * AT_SX_FLOATS * 4 + 512;
+constexpr int AT_STAGE_BYTES = AT_KB * AT_KB_BYTES;        // 36 KB
+constexpr int AT_P_BYTES = AT_H * 128;                     // 16 KB (32 bf16 per head used)
+constexpr int AT_SMEM = 1024 + AT_QS_BYTES + AT_STAGES * AT_STAGE_BYTES + AT_P_BYTES + 512;
 constexpr uint32_t TM_O = 0;    // TMEM columns [0, 256): O
 constexpr uint32_t TM_S = 256;  // TMEM columns [256, 320): two S buffers of 32
+constexpr uint32_t TM_Q = 320;  // TMEM columns [320, 512): Q dims [0, 384), two bf16 per column
 constexpr uint32_t IDESC_S = idesc_mma(128, AT_T, 1u, 0u);
 constexpr uint32_t IDESC_PV = idesc_mma(128, 256, 1u, 1u);
 constexpr float RESCALE_LOG2 = 8.f;
+static_assert(TM_Q + AT_KB_TQ * 32 == 512, "TMEM columns");
+static_assert(AT_SMEM <= 232448, "shared memory");
 
 struct AtArgs {
+  const uint16_t* q;   // absorbed queries [B, 128, 576] bf16
   const uint16_t* kv;  // latent cache [L, 576] bf16
   const int32_t* idx;
   int64_t idx_ld;
@@ -67,33 +75,29 @@ struct AtArgs {
   float* ws_ml;  // [B, S, 128, 2]   fp32 (S > 1): running max (log2 units), sum
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
+__global__ void __launch_bounds__(AT_THREADS, 1)
     k_sparse_attn_tc(const __grid_constant__ CUtensorMap tm_q, AtArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* q_s = base;
-  unsigned char* st_s = q_s + AT_Q_BYTES;
+  unsigned char* st_s = q_s + AT_QS_BYTES;
   unsigned char* p_s = st_s + AT_STAGES * AT_STAGE_BYTES;
-  float* sx_s = reinterpret_cast<float*>(p_s + AT_P_BYTES);
-  float* sx_out = sx_s + 2 * AT_SX_FLOATS;  // staging of this CTA's partial logits for the bulk copy
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sx_out + AT_SX_FLOATS);  // after two receive buffers + staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + AT_P_BYTES);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + AT_STAGES;
   uint64_t* s_full = kv_empty + AT_STAGES;
   uint64_t* s_empty = s_full + 2;
   uint64_t* p_full = s_empty + 2;
   uint64_t* pv_done = p_full + 1;
-  uint64_t* sx_full = pv_done + 1;  // [2]: the peer's partial logits of tile i landed in buffer i & 1
-  uint64_t* q_full = sx_full + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(q_full + 1);
+  uint64_t* q_full = pv_done + 1;   // Q's shared-memory K-blocks landed (TMA)
+  uint64_t* qt_full = q_full + 1;   // Q's TMEM part written by the softmax warps
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qt_full + 1);
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t r = cluster_ctarank();
-  const uint32_t peer = r ^ 1u;
-  const int unit = blockIdx.x >> 1;
+  const int r = static_cast<int>(blockIdx.x & 1u);  // value half
+  const int unit = static_cast<int>(blockIdx.x >> 1);
   const int b = unit / a.S, split = unit % a.S;
-  const int kbq = r ? 5 : 4;
   int n = a.count[b];
   n = n < 0 ? 0 : (static_cast<int64_t>(n) > a.idx_ld ? static_cast<int>(a.idx_ld) : n);
   const int rps = ((n + a.S - 1) / a.S + AT_T - 1) / AT_T * AT_T;
@@ -108,18 +112,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
+      mbar_init(&s_empty[i], 4);  // the four softmax warps have read the buffer
     }
     mbar_init(p_full, 4);
     mbar_init(pv_done, 1);
-    mbar_init(&sx_full[0], 1);
-    mbar_init(&sx_full[1], 1);
     mbar_init(q_full, 1);
+    mbar_init(qt_full, 4);
     abort_flag = 0;
     fence_mbar_init();
-    // arm both receive buffers for their first tile: each phase completes when the peer's bytes land
-    mbar_expect_tx(&sx_full[0], AT_SX_TX);
-    mbar_expect_tx(&sx_full[1], AT_SX_TX);
   }
   if (warp == AT_MMA_WARP) {
     tmem_alloc(tmem_holder, 512);
@@ -127,24 +127,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync_all();  // the peer's barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
   if (warp < AT_GATHER_WARPS) {
     // ------------------------------------------------------------------ gather producers
-    // Warp w copies rows 8w..8w+7 of every tile: 16-byte cp.async chunks of this CTA's slice of each row,
-    // placed in the 128-byte-swizzled K-major layout (chunk c of row t at (c ^ (t & 7)) * 16 in its K-block).
+    // Warp w copies rows 8w..8w+7 of every tile: 72 16-byte cp.async chunks per row, placed in the
+    // 128-byte-swizzled K-major layout (chunk c of row t at (c & 7 ^ t & 7) * 16 in K-block c / 8).
     if (ntiles > 0) {
       if (tid == 0) {
         tma_prefetch_desc(&tm_q);
-        mbar_expect_tx(q_full, kbq * AT_H * 128);
-        for (int kb = 0; kb < kbq; ++kb)
-          tma_load_2d(q_s + kb * AT_H * 128, &tm_q, q_full, 256 * static_cast<int>(r) + 64 * kb, b * AT_H);
+        mbar_expect_tx(q_full, AT_KB_SQ * AT_H * 128);
+        for (int kb = 0; kb < AT_KB_SQ; ++kb)
+          tma_load_2d(q_s + kb * AT_H * 128, &tm_q, q_full, 64 * (AT_KB_TQ + kb), b * AT_H);
       }
       const int32_t* rowidx = a.idx + static_cast<int64_t>(b) * a.idx_ld + row0;
-      const uint16_t* kvr = a.kv + 256 * r;  // this CTA's slice starts at latent dim 256 r
-      const int cpr = kbq * 8;              // 16-byte chunks per row
+      constexpr int CPR = AT_KB * 8;  // 16-byte chunks per row
       // raw row indices (lane l < 8: row 8w + l) are loaded two tiles ahead and clamped at use
       auto load_idx = [&](int i) -> int {
         const int rr = i * AT_T + warp * 8 + (lane & 7);
@@ -166,57 +164,81 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         }
         const int v = v_raw < 0 ? 0 : (v_raw >= a.L ? a.L - 1 : v_raw);
         unsigned char* dst = st_s + st * AT_STAGE_BYTES;
-        for (int q = lane; q < 8 * cpr; q += 32) {
-          const int rr = q / cpr, c = q - rr * cpr;
+        #pragma unroll 2
+        for (int q = lane; q < 8 * CPR; q += 32) {
+          const int rr = q / CPR, c = q - rr * CPR;
           const int row_in_tile = warp * 8 + rr;
           const int srow = __shfl_sync(0xffffffffu, v, rr);  // every lane takes part: rr < 8
           const int kb = c >> 3, c8 = c & 7;
           cp_async16(dst + kb * AT_KB_BYTES + row_in_tile * 128 + ((c8 ^ (row_in_tile & 7)) << 4),
-                     kvr + static_cast<int64_t>(srow) * 576 + c * 8);
+                     a.kv + static_cast<int64_t>(srow) * 576 + c * 8);
         }
         cp_async_arrive_noinc(&kv_full[st]);
       }
     }
-  } else if (warp == AT_MMA_WARP) {
-    // ------------------------------------------------------------------ MMA issuer
-    // S = Q C^T runs two tiles ahead of O += P V, so the softmax never waits for its next logits
-    if (ntiles > 0 && lane == 0) {
-      bool ok = mbar_spin(q_full, 0);
-      const uint32_t q_addr = smem_u32(q_s);
-      const uint32_t p_addr = smem_u32(p_s);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % AT_STAGES, sb = j & 1;
-        if (!mbar_spin(&kv_full[st], (j / AT_STAGES) & 1) || !mbar_spin(&s_empty[sb], ((j >> 1) & 1) ^ 1)) return false;
+  } else if (warp == AT_MMA_WARP || warp == AT_MMA_WARP2) {
+    // ------------------------------------------------------------------ logits MMAs
+    // One thread issues about one tcgen05.mma per 30 ns, so the logits MMAs (36 per tile) are split over
+    // two issuing warps by tile parity, each with its own S buffer; S runs up to two tiles ahead of P.V.
+    const int sb = warp == AT_MMA_WARP ? 0 : 1;
+    if (ntiles > sb && lane == 0) {
+      bool ok = mbar_spin(q_full, 0) && mbar_spin(qt_full, 0);
+      tc_fence_after();
+      const uint64_t qdesc = desc_sw128(smem_u32(q_s));
+      const uint32_t d = tmem + TM_S + sb * AT_T;
+      for (int j = sb; ok && j < ntiles; j += 2) {
+        const int st = j % AT_STAGES;
+        if (!mbar_spin(&kv_full[st], (j / AT_STAGES) & 1) || !mbar_spin(&s_empty[sb], ((j >> 1) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
         fence_proxy_async_smem();  // the cp.async (generic proxy) writes are read by the tensor cores
         tc_fence_after();
-        const uint32_t s_addr = smem_u32(st_s + st * AT_STAGE_BYTES);
-        for (int kb = 0; kb < kbq; ++kb) {
+        const uint64_t sdesc = desc_sw128(smem_u32(st_s + st * AT_STAGE_BYTES));
+        // dims [0, 384): A = Q from TMEM (8 columns per K = 16 step); descriptors advance in 16-byte units
+        #pragma unroll
+        for (int kb = 0; kb < AT_KB_TQ; ++kb) {
           #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f16(tmem + TM_S + sb * AT_T, desc_sw128(q_addr + kb * AT_H * 128 + kk * 32),
-                    desc_sw128(s_addr + kb * AT_KB_BYTES + kk * 32), IDESC_S, (kb | kk) != 0);
+            mma_f16_ta(d, tmem + TM_Q + kb * 32 + kk * 8, sdesc + ((kb * AT_KB_BYTES + kk * 32) >> 4), IDESC_S,
+                       (kb | kk) != 0);
+        }
+        // dims [384, 576): A = Q from shared memory
+        #pragma unroll
+        for (int kb = 0; kb < AT_KB_SQ; ++kb) {
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(d, qdesc + ((kb * AT_H * 128 + kk * 32) >> 4),
+                    sdesc + (((AT_KB_TQ + kb) * AT_KB_BYTES + kk * 32) >> 4), IDESC_S, 1u);
         }
         mma_commit(&s_full[sb]);
-        return true;
-      };
-      auto issue_pv = [&](int j) -> bool {
+      }
+      if (!ok) {
+        atomicExch(&g_attn_tc_timeout, 1);
+        abort_flag = 1;
+      }
+    }
+  } else if (warp == AT_PV_WARP) {
+    // ------------------------------------------------------------------ O += P V
+    if (ntiles > 0 && lane == 0) {
+      bool ok = true;
+      const uint64_t pdesc = desc_sw128(smem_u32(p_s));
+      for (int j = 0; ok && j < ntiles; ++j) {
         const int stj = j % AT_STAGES;
-        if (!mbar_spin(p_full, j & 1)) return false;
+        // P(j) written means the softmax has read S(j): the logits MMAs of tile j are complete
+        if (!mbar_spin(p_full, j & 1)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(st_s + stj * AT_STAGE_BYTES);
+        // V = this CTA's value columns [256r, 256r + 256) = K-blocks 4r .. 4r + 3 of the tile, read MN-major
+        const uint32_t v_addr = smem_u32(st_s + stj * AT_STAGE_BYTES + 4 * r * AT_KB_BYTES);
         #pragma unroll
         for (int kk = 0; kk < AT_T / 16; ++kk)
-          mma_f16(tmem + TM_O, desc_sw128(p_addr + kk * 32), desc_sw128_mn(v_addr + kk * 16 * 128, AT_KB_BYTES, 1024),
+          mma_f16(tmem + TM_O, pdesc + ((kk * 32) >> 4), desc_sw128_mn(v_addr + kk * 16 * 128, AT_KB_BYTES, 1024),
                   IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&kv_empty[stj]);
         mma_commit(pv_done);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      if (ok && ntiles > 1) ok = issue_s(1);
-      for (int i = 0; ok && i < ntiles; ++i) {
-        if (i + 2 < ntiles && !issue_s(i + 2)) ok = false;
-        if (ok && !issue_pv(i)) ok = false;
       }
       if (!ok) {
         atomicExch(&g_attn_tc_timeout, 1);
@@ -224,75 +246,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------------ softmax + epilogue
+    // ------------------------------------------------------------------ Q into TMEM, softmax + epilogue
     const int q4 = warp & 3;
     const int h = q4 * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const uint32_t peer_sx = mapa(smem_u32(sx_s), peer);
-    const uint32_t peer_sx_full = mapa(smem_u32(sx_full), peer);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    // read S(j) from TMEM, free the buffer, stage this warp's 32 rows in shared memory and send them to the
-    // peer's receive buffer j & 1 as one 4 KB bulk copy per warp (all four complete on the peer's mbarrier)
-    auto fetch_and_send = [&](int j, uint32_t (&sr)[32]) -> bool {
-      const int sb = j & 1;
-      if (!mbar_spin(&s_full[sb], (j >> 1) & 1)) return false;
+    if (ntiles > 0) {
+      // Q row h, dims [0, 384) -> TMEM lane h, columns TM_Q + 32 kb + j hold dims 64 kb + 2j, 64 kb + 2j + 1
+      const uint4* qrow = reinterpret_cast<const uint4*>(a.q + (static_cast<int64_t>(b) * AT_H + h) * 576);
+      #pragma unroll 1
+      for (int kb = 0; kb < AT_KB_TQ; ++kb) {
+        uint32_t v[32];
+        #pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 x = __ldg(qrow + kb * 8 + c);
+          v[4 * c] = x.x;
+          v[4 * c + 1] = x.y;
+          v[4 * c + 2] = x.z;
+          v[4 * c + 3] = x.w;
+        }
+        tmem_st32(trow + TM_Q + 32 * kb, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qt_full);
+    }
+    for (int i = 0; ok && i < ntiles; ++i) {
+      const int sb = i & 1;
+      const int nvalid = min(AT_T, nrows - i * AT_T);
+      uint32_t sr[32];
+      if (!mbar_spin(&s_full[sb], (i >> 1) & 1)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       tmem_ld32(trow + TM_S + sb * AT_T, sr);
       tmem_ld_wait();
       tc_fence_before();
-      // this warp's staging rows are free once its previous bulk copy has read them
-      if (lane == 0) bulk_wait_read0();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[sb]);
-      float4* row = reinterpret_cast<float4*>(sx_out + h * AT_T);
-      #pragma unroll
-      for (int c = 0; c < AT_T / 4; ++c)
-        row[c ^ (h & 7)] = make_float4(__uint_as_float(sr[4 * c]), __uint_as_float(sr[4 * c + 1]),
-                                       __uint_as_float(sr[4 * c + 2]), __uint_as_float(sr[4 * c + 3]));
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        const uint32_t off = static_cast<uint32_t>((sb * AT_SX_FLOATS + q4 * 32 * AT_T) * 4);
-        bulk_store_peer(peer_sx + off, sx_out + q4 * 32 * AT_T, 32 * AT_T * 4, peer_sx_full + sb * 8);
-        bulk_commit();
-      }
-      return true;
-    };
-    uint32_t sr[32];
-    if (ntiles > 0) ok = fetch_and_send(0, sr);
-    for (int i = 0; ok && i < ntiles; ++i) {
-      const int sb = i & 1;
-      const int nvalid = min(AT_T, nrows - i * AT_T);
-      // the peer's partial logits of tile i.  Its receive buffer for tile i+1 is free: the peer read tile
-      // i-1 from it before sending tile i, which has arrived.
-      if (!mbar_wait_cluster(&sx_full[sb], (i >> 1) & 1)) {
-        ok = false;
-        break;
-      }
-      const float4* sxrow = reinterpret_cast<const float4*>(sx_s + sb * AT_SX_FLOATS + h * AT_T);
-      float sp[AT_T];
-      #pragma unroll
-      for (int c = 0; c < AT_T / 4; ++c) {
-        const float4 v = sxrow[c ^ (h & 7)];
-        sp[4 * c] = v.x;
-        sp[4 * c + 1] = v.y;
-        sp[4 * c + 2] = v.z;
-        sp[4 * c + 3] = v.w;
-      }
-      // re-arm buffer sb for tile i+2 (before this CTA sends tile i+1, so before the peer can send i+2)
-      if (tid == AT_SM_TID0 && i + 2 < ntiles) mbar_expect_tx(&sx_full[sb], AT_SX_TX);
-      uint32_t sr_next[32];
-      if (i + 1 < ntiles && !fetch_and_send(i + 1, sr_next)) {
-        ok = false;
-        break;
-      }
       float z[AT_T];
       float mt = -INFINITY;
       #pragma unroll
       for (int c = 0; c < AT_T; ++c) {
-        const float sfull = __uint_as_float(sr[c]) + sp[c];
-        z[c] = c < nvalid ? sfull * a.scale_log2 : -INFINITY;
+        z[c] = c < nvalid ? __uint_as_float(sr[c]) * a.scale_log2 : -INFINITY;
         mt = fmaxf(mt, z[c]);
       }
       float alpha = 1.f;
@@ -343,15 +342,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      #pragma unroll
-      for (int c = 0; c < 32; ++c) sr[c] = sr_next[c];
     }
     if (!ok) {
       atomicExch(&g_attn_tc_timeout, 1);
       abort_flag = 1;
     }
     // ---- epilogue
-    if (lane == 0) bulk_wait_read0();  // this warp's last outgoing copy has read its staging rows
     const bool have = ok && ntiles > 0 && mbar_spin(pv_done, (ntiles - 1) & 1);
     tc_fence_after();
     const int64_t orow = static_cast<int64_t>(b) * AT_H + h;
@@ -406,7 +402,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync_all();  // no CTA leaves while its peer may still touch its shared memory
   if (warp == AT_MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -483,7 +478,9 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   CUtensorMap tq;
   const int st = make_map(&tq, q, false, B * AT_H, 576, 64, AT_H);
   if (st) return st;
+  if (!aligned16(q)) return LSA_ERR_INVALID_ARG;
   AtArgs a;
+  a.q = static_cast<const uint16_t*>(q);
   a.kv = static_cast<const uint16_t*>(kv);
   a.idx = idx;
   a.idx_ld = idx_ld;
