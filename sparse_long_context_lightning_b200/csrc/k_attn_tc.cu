@@ -288,30 +288,34 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[sb]);
       float z[AT_T];
-      float mt = -INFINITY;
       #pragma unroll
-      for (int c = 0; c < AT_T; ++c) {
-        z[c] = c < nvalid ? __uint_as_float(sr[c]) * a.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, z[c]);
-      }
+      for (int c = 0; c < AT_T; ++c) z[c] = c < nvalid ? __uint_as_float(sr[c]) * a.scale_log2 : -INFINITY;
+      // row max and sum as trees of 8 independent chains (one warp per scheduler: latency, not issue, bound)
+      float m8[8];
+      #pragma unroll
+      for (int j = 0; j < 8; ++j) m8[j] = z[j];
+      #pragma unroll
+      for (int c = 8; c < AT_T; ++c) m8[c & 7] = fmaxf(m8[c & 7], z[c]);
+      const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       float alpha = 1.f;
       bool resc = false;
       if (i == 0) {
         m_used = mt;
       } else if (mt > m_used + RESCALE_LOG2) {
-        alpha = exp2f(m_used - mt);
+        alpha = ex2_approx(m_used - mt);
         m_used = mt;
         resc = true;
       }
       uint32_t pk[AT_T / 2];
-      float psum = 0.f;
+      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       #pragma unroll
       for (int c = 0; c < AT_T; c += 2) {
-        const float p0 = exp2f(z[c] - m_used), p1 = exp2f(z[c + 1] - m_used);
-        psum += p0 + p1;  // the row sum uses the fp32 probabilities (P . V uses them rounded to bf16)
+        const float p0 = ex2_approx(z[c] - m_used), p1 = ex2_approx(z[c + 1] - m_used);
+        s8[(c >> 1) & 7] += p0 + p1;  // the row sum uses the fp32 probabilities (P . V uses them rounded to bf16)
         const __nv_bfloat162 p2 = __floats2bfloat162_rn(p0, p1);
         pk[c / 2] = *reinterpret_cast<const uint32_t*>(&p2);
       }
+      const float psum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
       l = l * alpha + psum;
       // the previous P . V has finished: the P buffer is free and O is stable
       if (i > 0 && !mbar_spin(pv_done, (i - 1) & 1)) {

@@ -151,6 +151,13 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_
       : "memory");
 }
 // kind::f8f6f4 (e4m3 x e4m3 -> f32)
+// 2^x by the hardware approximation (ex2.approx.ftz.f32: relative error about 2^-22; 2^-inf = +0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // A operand from tensor memory: M rows on the M lanes, two 16-bit K elements per 32-bit column (the lower
 // K index in the low half), so one K = 16 step reads 8 columns starting at `a_tmem`.
 __device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
