@@ -10,6 +10,9 @@ outside the per-step CUDA events.  Rank 0 prints one JSON line.
 
 N > 1 (torchrun): every rank runs an independent replica of the same decode batch (the path has no
 exchange step on one node here: replicas only), timed per rank, max over ranks.
+
+At N = 1 the line also carries "prefill_chunk": the latency of one causal prefill chunk (8192 queries,
+FP8 scan + bf16 re-rank, K = 2048 + sink 4 + window 128) with its per-stage times (--no-prefill skips it).
 """
 
 from __future__ import annotations
@@ -194,6 +197,41 @@ STAGE_KERNEL = {"index": ("k_index_score_tc", ["k_index_tc.cu"]),
 LAUNCHES = {"index": 1, "topk": 1, "attn": 1}
 
 
+def prefill_chunk(device, l2_flush, iters: int = 3):
+    """Latency of one causal prefill chunk: 8192 queries at positions 122880..131071 over L = 131072, FP8
+    scan + exact bf16 re-rank to K = 2048, sink 4 + window 128, attention over the selected rows.
+    Inputs resident in HBM; L2 flushed before each iteration, outside the events."""
+    wl = S.WORKLOADS["prefill"]
+    step = DecodeStep(wl, "fp8", device)
+    stream = torch.cuda.current_stream()
+
+    def once(ev):
+        ev[0].record(stream)
+        step.index()
+        ev[1].record(stream)
+        step.topk()
+        ev[2].record(stream)
+        step.attn()
+        ev[3].record(stream)
+
+    l2_flush()
+    once([torch.cuda.Event(enable_timing=True) for _ in range(4)])  # warm-up
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(iters)]
+    for i in range(iters):
+        l2_flush()
+        once(evs[i])
+    torch.cuda.synchronize()
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(iters)])
+    ms = float(per.sum(axis=1).mean())
+    st = per.mean(axis=0)
+    del step
+    torch.cuda.empty_cache()
+    return {"workload": "prefill: 8192 causal queries (q_pos 122880..131071), L=131072, FP8 scan + bf16 re-rank, "
+                        "K=2048 + sink 4 + window 128, H=128", "ms": round(ms, 3),
+            "stages_ms": {"index": round(float(st[0]), 3), "topk": round(float(st[1]), 3), "attn": round(float(st[2]), 3)},
+            "queries_per_s": round(wl.B / (ms * 1e-3), 1), "iterations": iters}
+
+
 def run_gpu(args, rank, world, local_rank):
     import sparse_long_context_lightning_b200 as lsa
 
@@ -290,6 +328,7 @@ def run_gpu(args, rank, world, local_rank):
     stage_ms = vals[2:].cpu().numpy()
     if rank != 0:
         return None
+    prefill = None if (args.no_prefill or world > 1) else prefill_chunk(device, l2_flush)
 
     pk, pk_src = peaks()
     work = algorithmic_work(wl, counts, step.fp8)
@@ -343,6 +382,7 @@ def run_gpu(args, rank, world, local_rank):
         "gpu_launches": n_launch,
         "clocks": clk.summary(),
         "wall_s_timed_region": round(wall, 4),
+        "prefill_chunk": prefill,
     }
 
 
@@ -421,6 +461,7 @@ def main():
     ap.add_argument("--impl", default="lsa", choices=["lsa", "reference"])
     ap.add_argument("--index", default="bf16", choices=["bf16", "fp8"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-chunk latency measurement")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
