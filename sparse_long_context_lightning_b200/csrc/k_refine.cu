@@ -7,6 +7,7 @@
 // pass with top-K' (K' > K), and the second stage re-scores those K' positions from the bf16 index
 // queries and keys, so the kept set matches the full-precision ranking.
 #include "lsa_common.cuh"
+#include "sm100.cuh"
 
 namespace lsa {
 
@@ -89,6 +90,192 @@ __global__ void __launch_bounds__(RF_THREADS) k_rescore(const uint16_t* __restri
   out[static_cast<int64_t>(b) * out_ld + j] = acc;
 }
 
+// Tensor-core re-score for d_I = 128 and H_I in {32, 64}: the same I(q_b, k_s) as k_rescore, computed as
+// D[cand, head] = K_cand . Q_b^T on tcgen05 (candidates = M, 128 per tile, on the TMEM lanes; heads = N;
+// d_I = 128 = K, 8 MMAs of K = 16), with the ReLU / weight / head sum in the epilogue (one candidate per
+// thread).  The candidates' key rows (256 B each) are gathered with 16-byte cp.async copies into the
+// 128-byte-swizzled K-major layout; three stages, two TMEM accumulators.  CTA (split, b) handles the
+// tiles split, split + nsplit, ... of query b.
+constexpr int RT_THREADS = 288;  // warps 0-3 gather, warp 4 MMA (TMEM owner), warps 5-8 epilogue
+constexpr int RT_STAGES = 3;
+constexpr int RT_TILE = 128;
+constexpr int RT_KB_BYTES = RT_TILE * 128;       // 16 KB: 64 dims of a tile
+constexpr int RT_STAGE_BYTES = 2 * RT_KB_BYTES;  // 32 KB
+constexpr int RT_Q_BYTES = 64 * 256;             // up to 64 heads x 128 dims bf16
+constexpr int RT_SMEM = 1024 + RT_Q_BYTES + RT_STAGES * RT_STAGE_BYTES + 256;
+
+__device__ int g_rescore_tc_timeout;
+
+__global__ void __launch_bounds__(RT_THREADS, 2)
+    k_rescore_tc(const uint16_t* __restrict__ q, const float* __restrict__ w, const uint16_t* __restrict__ k, int H_I,
+                 int64_t L, const int32_t* __restrict__ cand, int64_t cand_ld, const int32_t* __restrict__ cand_count,
+                 const int64_t* __restrict__ q_pos, int sink, int window, float* __restrict__ out, int64_t out_ld,
+                 int64_t* __restrict__ ndyn_m1) {
+  using namespace sm100;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* q_s = base;
+  unsigned char* st_s = q_s + RT_Q_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(st_s + RT_STAGES * RT_STAGE_BYTES);
+  uint64_t* kv_full = bars;                    // [RT_STAGES]
+  uint64_t* kv_empty = kv_full + RT_STAGES;    // [RT_STAGES]
+  uint64_t* acc_full = kv_empty + RT_STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;          // [2]
+  uint64_t* q_ready = acc_empty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(q_ready + 1);
+  __shared__ float w_s[64];
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.y, split = blockIdx.x, nsplit = gridDim.x;
+  const Fixed f = fixed_of(q_pos[b], sink, window);
+  const int n = min(static_cast<int64_t>(cand_count[b]), cand_ld);
+  const int ndyn = max(0, n - f.nsink - (f.whi - f.wlo));
+  if (split == 0 && tid == 0) ndyn_m1[b] = static_cast<int64_t>(ndyn) - 1;
+  const int ntiles_all = static_cast<int>((out_ld + RT_TILE - 1) / RT_TILE);
+  const int ntiles_act = (ndyn + RT_TILE - 1) / RT_TILE;
+  // this CTA's active tiles: split, split + nsplit, ... below ntiles_act
+  const int nmine = split < ntiles_act ? (ntiles_act - split + nsplit - 1) / nsplit : 0;
+  const int32_t* crow = cand + static_cast<int64_t>(b) * cand_ld + f.nsink;
+  float* orow = out + static_cast<int64_t>(b) * out_ld;
+
+  if (tid == 0) {
+    for (int i = 0; i < RT_STAGES; ++i) {
+      mbar_init(&kv_full[i], 128);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_init(q_ready, 4);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_holder, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp < 4) {
+    // ---- gather: warp w copies rows 32w..32w+31 of a tile, 16 chunks of 16 B per row
+    bool ok = true;
+    for (int i = 0; ok && i < nmine; ++i) {
+      const int t = split + i * nsplit, st = i % RT_STAGES;
+      const int j = t * RT_TILE + warp * 32 + lane;
+      int64_t s = j < ndyn ? crow[j] : 0;
+      s = s < 0 ? 0 : (s >= L ? L - 1 : s);
+      if (!mbar_spin(&kv_empty[st], ((i / RT_STAGES) & 1) ^ 1) || abort_flag) {
+        ok = false;
+        break;
+      }
+      unsigned char* dst = st_s + st * RT_STAGE_BYTES;
+      #pragma unroll 4
+      for (int q16 = lane; q16 < 32 * 16; q16 += 32) {
+        const int rr = q16 >> 4, c = q16 & 15;  // row of the warp's 32, 16-byte chunk of the row
+        const int row = warp * 32 + rr;
+        const int64_t srow = __shfl_sync(0xffffffffu, s, rr);
+        const int kb = c >> 3, c8 = c & 7;
+        cp_async16(dst + kb * RT_KB_BYTES + row * 128 + ((c8 ^ (row & 7)) << 4), k + srow * 128 + c * 8);
+      }
+      cp_async_arrive_noinc(&kv_full[st]);
+    }
+    if (!ok && lane == 0) {
+      atomicExch(&g_rescore_tc_timeout, 1);
+      abort_flag = 1;
+    }
+  } else if (warp == 4) {
+    // ---- MMA: D (128 candidates x H_I) = K_tile . Q^T, into accumulator i & 1
+    if (lane == 0 && nmine > 0) {
+      bool ok = mbar_spin(q_ready, 0);
+      const uint32_t idesc = idesc_mma(128, H_I, 1u, 0u);
+      const uint64_t qdesc = desc_sw128(smem_u32(q_s));
+      for (int i = 0; ok && i < nmine; ++i) {
+        const int st = i % RT_STAGES, ab = i & 1;
+        if (!mbar_spin(&kv_full[st], (i / RT_STAGES) & 1) || !mbar_spin(&acc_empty[ab], ((i >> 1) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint64_t kdesc = desc_sw128(smem_u32(st_s + st * RT_STAGE_BYTES));
+        #pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem + ab * 64, kdesc + ((kb * RT_KB_BYTES + kk * 32) >> 4),
+                    qdesc + ((kb * H_I * 128 + kk * 32) >> 4), idesc, (kb | kk) != 0);
+        }
+        mma_commit(&kv_empty[st]);
+        mma_commit(&acc_full[ab]);
+      }
+      if (!ok) {
+        atomicExch(&g_rescore_tc_timeout, 1);
+        abort_flag = 1;
+      }
+    }
+  } else {
+    // ---- epilogue warps: Q (H_I x 128, swizzled B tile) and the weights first, then one candidate per thread
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;  // candidate row of the tile = TMEM lane
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int et = tid - 160;
+    bool ok = true;
+    if (nmine > 0) {
+      for (int x = et; x < H_I * 16; x += 128) {
+        const int h = x >> 4, c = x & 15, kb = c >> 3, c8 = c & 7;
+        const uint4 v = *reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * H_I + h) * 128 + c * 8);
+        *reinterpret_cast<uint4*>(q_s + kb * H_I * 128 + h * 128 + ((c8 ^ (h & 7)) << 4)) = v;
+      }
+      for (int x = et; x < H_I; x += 128) w_s[x] = w[static_cast<int64_t>(b) * H_I + x];
+      fence_proxy_async_smem();  // generic stores read by the tensor cores
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+      ok = mbar_spin(q_ready, 0);  // the weights of every epilogue warp are visible
+    }
+    for (int i = 0; ok && i < nmine; ++i) {
+      const int t = split + i * nsplit, ab = i & 1;
+      if (!mbar_spin(&acc_full[ab], (i >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float acc = 0.f;
+      for (int c0 = 0; c0 < H_I; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(trow + ab * 64 + c0, v);
+        tmem_ld_wait();
+        #pragma unroll
+        for (int c = 0; c < 32; ++c) acc = fmaf(w_s[c0 + c], fmaxf(__uint_as_float(v[c]), 0.f), acc);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      const int j = t * RT_TILE + row;
+      if (j < out_ld) orow[j] = j < ndyn ? acc : -INFINITY;
+    }
+    if (!ok) {
+      atomicExch(&g_rescore_tc_timeout, 1);
+      abort_flag = 1;
+    }
+    // tiles of this CTA past the dynamic candidates: -inf
+    for (int t = split + nmine * nsplit; t < ntiles_all; t += nsplit) {
+      const int j = t * RT_TILE + row;
+      if (j < out_ld) orow[j] = -INFINITY;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // idx row = sink entries, then the kept dynamic candidates (ascending), then the window entries.
 __global__ void __launch_bounds__(256) k_refine_assemble(const int32_t* __restrict__ cand, int64_t cand_ld,
                                                          const int32_t* __restrict__ cand_count,
@@ -150,7 +337,16 @@ int launch_refine(const void* q, const float* w, const void* k, int64_t B, int H
   const size_t smem = static_cast<size_t>(H_I) * d_I * 4 + static_cast<size_t>(H_I) * 4;
   const uint16_t* qq = static_cast<const uint16_t*>(q);
   const uint16_t* kk = static_cast<const uint16_t*>(k);
-  switch (d_I) {
+  if (d_I == 128 && (H_I == 32 || H_I == 64) && B <= 65535) {
+    // tensor cores; tiles of a query spread over up to ~2 waves of CTAs when the batch is small
+    const int64_t tiles = cdiv(out_ld, RT_TILE);
+    int64_t nsplit = (2 * 148 + B - 1) / B;
+    if (nsplit > tiles) nsplit = tiles;
+    if (nsplit < 1) nsplit = 1;
+    LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_rescore_tc), RT_SMEM));
+    k_rescore_tc<<<dim3(static_cast<unsigned>(nsplit), static_cast<unsigned>(B)), RT_THREADS, RT_SMEM, s>>>(
+        qq, w, kk, H_I, L, cand, cand_ld, cand_count, q_pos, sink, window, rs, out_ld, ndyn_m1);
+  } else switch (d_I) {
     case 32:
       k_rescore<32><<<grid, RF_THREADS, smem, s>>>(qq, w, kk, H_I, L, cand, cand_ld, cand_count, q_pos, sink, window,
                                                    rs, out_ld, ndyn_m1);

@@ -300,6 +300,13 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// L2 prefetch of `bytes` (a multiple of 16) contiguous global bytes from a 16-byte aligned address; no shared
+// memory, no completion to wait for
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
+}
+
 // L2 prefetch of the same 4-row gather (no shared memory, no completion)
 __device__ __forceinline__ void tma_prefetch_gather4(const CUtensorMap* m, int x, int y0, int y1, int y2, int y3) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile::gather4 [%0, {%1, %2, %3, %4, %5}];"
