@@ -34,11 +34,13 @@ using namespace sm100;
 
 __device__ int g_attn_tc_timeout;  // set when a bounded wait of the kernel gave up
 
-constexpr int AT_THREADS = 352;  // 4 gather warps, 4 softmax warps, 3 MMA-issuing warps
-constexpr int AT_GATHER_WARPS = 4;
-constexpr int AT_MMA_WARP = 4;   // logits of even tiles; owns TMEM
-constexpr int AT_MMA_WARP2 = 9;  // logits of odd tiles
-constexpr int AT_PV_WARP = 10;   // O += P V
+constexpr int AT_THREADS = 736;  // 16 gather warps, 3 MMA-issuing warps, 4 softmax warps
+// A warp's 16-byte cp.async copies are issue-latency bound (one CTA reaches ~18 GB/s with 4 gather warps,
+// ~36 GB/s with 16, measured), so the gather runs on 16 warps, two rows of each tile per warp.
+constexpr int AT_GATHER_WARPS = 16;
+constexpr int AT_MMA_WARP = 16;   // logits of even tiles; owns TMEM
+constexpr int AT_MMA_WARP2 = 17;  // logits of odd tiles
+constexpr int AT_PV_WARP = 18;    // O += P V; warps 19-22: softmax (warp % 4 = the TMEM lane quarter)
 constexpr int AT_T = 32;         // gathered rows per tile
 constexpr int AT_H = 128;        // heads (MMA M)
 constexpr int AT_KB = 9;         // 64-dim K-blocks of a 576-dim row
@@ -132,7 +134,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 
   if (warp < AT_GATHER_WARPS) {
     // ------------------------------------------------------------------ gather producers
-    // Warp w copies rows 8w..8w+7 of every tile: 72 16-byte cp.async chunks per row, placed in the
+    // Warp w copies rows 2w, 2w + 1 of every tile: 72 16-byte cp.async chunks per row, placed in the
     // 128-byte-swizzled K-major layout (chunk c of row t at (c & 7 ^ t & 7) * 16 in K-block c / 8).
     if (ntiles > 0) {
       if (tid == 0) {
@@ -143,9 +145,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       }
       const int32_t* rowidx = a.idx + static_cast<int64_t>(b) * a.idx_ld + row0;
       constexpr int CPR = AT_KB * 8;  // 16-byte chunks per row
-      // raw row indices (lane l < 8: row 8w + l) are loaded two tiles ahead and clamped at use
+      // raw row indices (lane l < 2: row 2w + l) are loaded two tiles ahead and clamped at use
       auto load_idx = [&](int i) -> int {
-        const int rr = i * AT_T + warp * 8 + (lane & 7);
+        const int rr = i * AT_T + warp * 2 + (lane & 1);
         return rr < nrows ? rowidx[rr] : 0;
       };
       int v_a = load_idx(0);
@@ -164,14 +166,17 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         }
         const int v = v_raw < 0 ? 0 : (v_raw >= a.L ? a.L - 1 : v_raw);
         unsigned char* dst = st_s + st * AT_STAGE_BYTES;
-        #pragma unroll 2
-        for (int q = lane; q < 8 * CPR; q += 32) {
-          const int rr = q / CPR, c = q - rr * CPR;
-          const int row_in_tile = warp * 8 + rr;
-          const int srow = __shfl_sync(0xffffffffu, v, rr);  // every lane takes part: rr < 8
-          const int kb = c >> 3, c8 = c & 7;
-          cp_async16(dst + kb * AT_KB_BYTES + row_in_tile * 128 + ((c8 ^ (row_in_tile & 7)) << 4),
-                     a.kv + static_cast<int64_t>(srow) * 576 + c * 8);
+        #pragma unroll
+        for (int k = 0; k < (2 * CPR + 31) / 32; ++k) {
+          const int q = lane + 32 * k;
+          const int rr = q >= CPR ? 1 : 0, c = q - rr * CPR;
+          const int row_in_tile = warp * 2 + rr;
+          const int srow = __shfl_sync(0xffffffffu, v, rr);  // every lane takes part
+          if (q < 2 * CPR) {
+            const int kb = c >> 3, c8 = c & 7;
+            cp_async16(dst + kb * AT_KB_BYTES + row_in_tile * 128 + ((c8 ^ (row_in_tile & 7)) << 4),
+                       a.kv + static_cast<int64_t>(srow) * 576 + c * 8);
+          }
         }
         cp_async_arrive_noinc(&kv_full[st]);
       }
