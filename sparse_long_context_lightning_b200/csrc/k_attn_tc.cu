@@ -92,8 +92,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   uint64_t* p_full = s_empty + 2;
   uint64_t* pv_done = p_full + 1;
   uint64_t* q_full = pv_done + 1;   // Q's shared-memory K-blocks landed (TMA)
-  uint64_t* qt_full = q_full + 1;   // Q's TMEM part written by the softmax warps
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qt_full + 1);
+  uint64_t* qt_full = q_full + 1;   // Q's TMEM part written by the softmax warps (stages 1-3 free again)
+  uint64_t* qst_full = qt_full + 1; // Q's TMEM part landed in stages 1-3 (TMA staging)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qst_full + 1);
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -120,6 +121,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     mbar_init(pv_done, 1);
     mbar_init(q_full, 1);
     mbar_init(qt_full, 4);
+    mbar_init(qst_full, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -142,6 +144,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         mbar_expect_tx(q_full, AT_KB_SQ * AT_H * 128);
         for (int kb = 0; kb < AT_KB_SQ; ++kb)
           tma_load_2d(q_s + kb * AT_H * 128, &tm_q, q_full, 64 * (AT_KB_TQ + kb), b * AT_H);
+        // Q dims [0, 384) are staged in stages 1-3 (free until the softmax warps have moved them into TMEM)
+        mbar_expect_tx(qst_full, AT_KB_TQ * AT_H * 128);
+        for (int kb = 0; kb < AT_KB_TQ; ++kb)
+          tma_load_2d(st_s + AT_STAGE_BYTES + kb * AT_H * 128, &tm_q, qst_full, 64 * kb, b * AT_H);
       }
       const int32_t* rowidx = a.idx + static_cast<int64_t>(b) * a.idx_ld + row0;
       constexpr int CPR = AT_KB * 8;  // 16-byte chunks per row
@@ -157,7 +163,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         const int v_raw = v_a;
         v_a = v_b;
         if (i + 2 < ntiles) v_b = load_idx(i + 2);
-        if (!mbar_spin(&kv_empty[st], ((i / AT_STAGES) & 1) ^ 1) || abort_flag) {
+        // stages 1-3 hold the Q staging until the softmax warps have copied it into TMEM
+        const bool staged_ok = !(i >= 1 && i < AT_STAGES) || mbar_spin(qt_full, 0);
+        if (!staged_ok || !mbar_spin(&kv_empty[st], ((i / AT_STAGES) & 1) ^ 1) || abort_flag) {
           if (lane == 0) {
             atomicExch(&g_attn_tc_timeout, 1);
             abort_flag = 1;
@@ -258,14 +266,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     if (ntiles > 0) {
-      // Q row h, dims [0, 384) -> TMEM lane h, columns TM_Q + 32 kb + j hold dims 64 kb + 2j, 64 kb + 2j + 1
-      const uint4* qrow = reinterpret_cast<const uint4*>(a.q + (static_cast<int64_t>(b) * AT_H + h) * 576);
+      // Q row h, dims [0, 384) -> TMEM lane h, columns TM_Q + 32 kb + j hold dims 64 kb + 2j, 64 kb + 2j + 1;
+      // read from the TMA staging (128-byte swizzle: chunk c of row h at ((c ^ h) & 7) * 16)
+      if (!mbar_spin(qst_full, 0)) ok = false;
       #pragma unroll 1
       for (int kb = 0; kb < AT_KB_TQ; ++kb) {
+        const unsigned char* src = st_s + AT_STAGE_BYTES + kb * AT_H * 128 + h * 128;
         uint32_t v[32];
         #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const uint4 x = __ldg(qrow + kb * 8 + c);
+          const uint4 x = *reinterpret_cast<const uint4*>(src + ((c ^ (h & 7)) << 4));
           v[4 * c] = x.x;
           v[4 * c + 1] = x.y;
           v[4 * c + 2] = x.z;
