@@ -47,6 +47,7 @@ constexpr int AT_KB = 9;         // 64-dim K-blocks of a 576-dim row
 constexpr int AT_KB_TQ = 6;      // Q K-blocks held in TMEM (dims [0, 384))
 constexpr int AT_KB_SQ = AT_KB - AT_KB_TQ;  // Q K-blocks in shared memory (dims [384, 576))
 constexpr int AT_STAGES = 4;
+constexpr int AT_O_PITCH = 1040;  // epilogue staging: 1 KB of O per head row + 16 B (rows in different banks)
 constexpr int AT_QS_BYTES = AT_KB_SQ * AT_H * 128;         // 48 KB
 constexpr int AT_KB_BYTES = AT_T * 128;                    // 4 KB: one 64-dim block of a tile
 constexpr int AT_STAGE_BYTES = AT_KB * AT_KB_BYTES;        // 36 KB
@@ -60,6 +61,7 @@ constexpr uint32_t IDESC_PV = idesc_mma(128, 256, 1u, 1u);
 constexpr float RESCALE_LOG2 = 8.f;
 static_assert(TM_Q + AT_KB_TQ * 32 == 512, "TMEM columns");
 static_assert(AT_SMEM <= 232448, "shared memory");
+static_assert(AT_H * AT_O_PITCH <= AT_STAGES * AT_STAGE_BYTES, "epilogue staging fits the stages");
 
 struct AtArgs {
   const uint16_t* q;   // absorbed queries [B, 128, 576] bf16
@@ -370,9 +372,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     const bool have = ok && ntiles > 0 && mbar_spin(pv_done, (ntiles - 1) & 1);
     tc_fence_after();
     const int64_t orow = static_cast<int64_t>(b) * AT_H + h;
+    // O (row h = this thread's TMEM lane) is staged in the stage memory -- free once the last P.V completed --
+    // with a padded row pitch (no bank conflicts), then written with one bulk copy per row
+    unsigned char* srow = st_s + h * AT_O_PITCH;
     if (a.S == 1) {
       const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
-      uint16_t* dst = a.out + orow * 512 + 256 * r;
       #pragma unroll 1
       for (int k = 0; k < 8; ++k) {
         uint32_t o[32];
@@ -389,14 +393,15 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv);
           pk[c / 2] = *reinterpret_cast<const uint32_t*>(&v);
         }
-        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * k);
+        uint4* d4 = reinterpret_cast<uint4*>(srow + 64 * k);
         #pragma unroll
         for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
+      fence_proxy_async_smem();
+      bulk_store_global(a.out + orow * 512 + 256 * r, srow, 512);
       if (r == 0 && a.lse) a.lse[orow] = (have && l > 0.f) ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
     } else {
       const int64_t prow_i = (static_cast<int64_t>(b) * a.S + split) * AT_H + h;
-      float* dst = a.ws_o + prow_i * 512 + 256 * r;
       #pragma unroll 1
       for (int k = 0; k < 8; ++k) {
         uint32_t o[32];
@@ -407,17 +412,21 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] = 0u;
         }
-        float4* d4 = reinterpret_cast<float4*>(dst + 32 * k);
+        float4* d4 = reinterpret_cast<float4*>(srow + 128 * k);
         #pragma unroll
         for (int c = 0; c < 8; ++c)
           d4[c] = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]), __uint_as_float(o[4 * c + 2]),
                               __uint_as_float(o[4 * c + 3]));
       }
+      fence_proxy_async_smem();
+      bulk_store_global(a.ws_o + prow_i * 512 + 256 * r, srow, 1024);
       if (r == 0) {
         a.ws_ml[prow_i * 2 + 0] = have ? m_used : -INFINITY;
         a.ws_ml[prow_i * 2 + 1] = have ? l : 0.f;
       }
     }
+    bulk_commit();
+    bulk_wait_read0();  // the staging rows are read before the CTA can exit
   }
   tc_fence_before();
   __syncthreads();

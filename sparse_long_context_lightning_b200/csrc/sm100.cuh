@@ -116,6 +116,13 @@ __device__ __forceinline__ void bulk_store_peer(uint32_t caddr_dst, const void* 
                ::"r"(caddr_dst), "r"(smem_u32(src)), "r"(bytes), "r"(caddr_bar)
                : "memory");
 }
+// bulk copy shared (this CTA) -> global, `bytes` a multiple of 16, both addresses 16-byte aligned; complete
+// with bulk_commit + bulk_wait_read0 before the shared source is reused
+__device__ __forceinline__ void bulk_store_global(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // wait until the source reads of every committed bulk copy of this thread are done
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
