@@ -436,30 +436,55 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   }
 }
 
-// Merge the splits of one (query, head): LSE-weighted sum of the partial outputs.
+// Merge the splits of one (query, head): LSE-weighted sum of the partial outputs.  Every load is issued before
+// any is used (one L2 round trip) for up to 8 splits; more splits fall back to a second pass.
+constexpr int CB_MAXS = 8;
 __global__ void __launch_bounds__(128) k_attn_combine(const float* __restrict__ ws_o, const float* __restrict__ ws_ml,
                                                       int S, uint16_t* __restrict__ out, float* __restrict__ lse) {
   const int64_t bh = blockIdx.x;  // b * 128 + h
   const int b = static_cast<int>(bh / AT_H), h = static_cast<int>(bh % AT_H);
+  const int64_t p0 = static_cast<int64_t>(b) * S * AT_H + h;  // partial of split s: p0 + s * AT_H
+  float2 ml[CB_MAXS];
+  float4 v[CB_MAXS];
+  #pragma unroll
+  for (int sp = 0; sp < CB_MAXS; ++sp) {
+    if (sp < S) {
+      ml[sp] = reinterpret_cast<const float2*>(ws_ml)[p0 + sp * AT_H];
+      v[sp] = reinterpret_cast<const float4*>(ws_o + (p0 + sp * AT_H) * 512)[threadIdx.x];
+    }
+  }
   float mstar = -INFINITY;
-  for (int s = 0; s < S; ++s) {
-    const int64_t pi = (static_cast<int64_t>(b) * S + s) * AT_H + h;
-    if (ws_ml[pi * 2 + 1] > 0.f) mstar = fmaxf(mstar, ws_ml[pi * 2]);
+  #pragma unroll
+  for (int sp = 0; sp < CB_MAXS; ++sp)
+    if (sp < S && ml[sp].y > 0.f) mstar = fmaxf(mstar, ml[sp].x);
+  for (int sp = CB_MAXS; sp < S; ++sp) {
+    const float2 m = reinterpret_cast<const float2*>(ws_ml)[p0 + sp * AT_H];
+    if (m.y > 0.f) mstar = fmaxf(mstar, m.x);
   }
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float lsum = 0.f;
   if (mstar != -INFINITY) {
-    for (int s = 0; s < S; ++s) {
-      const int64_t pi = (static_cast<int64_t>(b) * S + s) * AT_H + h;
-      const float ls = ws_ml[pi * 2 + 1];
-      if (!(ls > 0.f)) continue;
-      const float wgt = exp2f(ws_ml[pi * 2] - mstar);
-      lsum += wgt * ls;
-      const float4 v = reinterpret_cast<const float4*>(ws_o + pi * 512)[threadIdx.x];
-      acc.x += wgt * v.x;
-      acc.y += wgt * v.y;
-      acc.z += wgt * v.z;
-      acc.w += wgt * v.w;
+    #pragma unroll
+    for (int sp = 0; sp < CB_MAXS; ++sp) {
+      if (sp < S && ml[sp].y > 0.f) {
+        const float wgt = exp2f(ml[sp].x - mstar);
+        lsum += wgt * ml[sp].y;
+        acc.x += wgt * v[sp].x;
+        acc.y += wgt * v[sp].y;
+        acc.z += wgt * v[sp].z;
+        acc.w += wgt * v[sp].w;
+      }
+    }
+    for (int sp = CB_MAXS; sp < S; ++sp) {
+      const float2 m = reinterpret_cast<const float2*>(ws_ml)[p0 + sp * AT_H];
+      if (!(m.y > 0.f)) continue;
+      const float wgt = exp2f(m.x - mstar);
+      const float4 x = reinterpret_cast<const float4*>(ws_o + (p0 + sp * AT_H) * 512)[threadIdx.x];
+      lsum += wgt * m.y;
+      acc.x += wgt * x.x;
+      acc.y += wgt * x.y;
+      acc.z += wgt * x.z;
+      acc.w += wgt * x.w;
     }
   }
   const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
