@@ -81,6 +81,9 @@ struct AtArgs {
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
     k_sparse_attn_tc(const __grid_constant__ CUtensorMap tm_q, AtArgs a) {
+  // every global access of this kernel comes after the previous kernel of the stream has completed
+  sm100::pdl_wait();
+  sm100::pdl_launch_dependents();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* q_s = base;
@@ -441,6 +444,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 constexpr int CB_MAXS = 8;
 __global__ void __launch_bounds__(128) k_attn_combine(const float* __restrict__ ws_o, const float* __restrict__ ws_ml,
                                                       int S, uint16_t* __restrict__ out, float* __restrict__ lse) {
+  // every global access of this kernel comes after the previous kernel of the stream has completed
+  sm100::pdl_wait();
+  sm100::pdl_launch_dependents();
   const int64_t bh = blockIdx.x;  // b * 128 + h
   const int b = static_cast<int>(bh / AT_H), h = static_cast<int>(bh % AT_H);
   const int64_t p0 = static_cast<int64_t>(b) * S * AT_H + h;  // partial of split s: p0 + s * AT_H
@@ -551,11 +557,10 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_sparse_attn_tc), AT_SMEM));
   const int64_t grid = 2 * B * S;
   if (grid > 0x7FFFFFFF) return LSA_ERR_UNSUPPORTED;
-  k_sparse_attn_tc<<<static_cast<unsigned>(grid), AT_THREADS, AT_SMEM, s>>>(tq, a);
-  LSA_CUDA_TRY(cudaGetLastError());
+  LSA_CUDA_TRY(launch_pdl(k_sparse_attn_tc, dim3(static_cast<unsigned>(grid)), dim3(AT_THREADS), AT_SMEM, s, 0u, tq, a));
   if (S > 1) {
-    k_attn_combine<<<static_cast<unsigned>(B * AT_H), 128, 0, s>>>(a.ws_o, a.ws_ml, S, a.out, lse);
-    LSA_CUDA_TRY(cudaGetLastError());
+    LSA_CUDA_TRY(launch_pdl(k_attn_combine, dim3(static_cast<unsigned>(B * AT_H)), dim3(128), 0, s, 0u,
+                            static_cast<const float*>(a.ws_o), static_cast<const float*>(a.ws_ml), S, a.out, lse));
   }
   return LSA_OK;
 }

@@ -59,6 +59,9 @@ struct IxArgs {
 template <bool FP8>
 __global__ void __launch_bounds__(IX_THREADS, 1)
     k_index_score_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q, IxArgs a) {
+  // every global access of this kernel comes after the previous kernel of the stream has completed
+  sm100::pdl_wait();
+  sm100::pdl_launch_dependents();
   using C = IxCfg<FP8>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 1024-byte aligned base for the swizzled tiles
@@ -246,8 +249,8 @@ int launch_tc(const void* q, const float* q_scale, const float* w, const void* k
   ranges = static_cast<int>(cdiv(a.ntiles, a.tiles_per_range));
   LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_index_score_tc<FP8>), C::SMEM));
   const int64_t grid = static_cast<int64_t>(a.n_chunks) * ranges;
-  k_index_score_tc<FP8><<<static_cast<unsigned>(grid), IX_THREADS, C::SMEM, s>>>(tk, tq, a);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch_pdl(k_index_score_tc<FP8>, dim3(static_cast<unsigned>(grid)), dim3(IX_THREADS), C::SMEM, s, 0u,
+                                tk, tq, a));
 }
 
 }  // namespace

@@ -227,6 +227,9 @@ __device__ __forceinline__ uint32_t ballot_prefix(uint32_t v, uint32_t lt, uint3
 }
 
 __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
+  // every global access of this kernel comes after the previous kernel of the stream has completed
+  sm100::pdl_wait();
+  sm100::pdl_launch_dependents();
   extern __shared__ __align__(16) unsigned char dyn[];
   __shared__ __align__(16) TopkSmem sm;
   cg::cluster_group cluster = cg::this_cluster();
@@ -702,19 +705,8 @@ int launch_topk_mode(const float* scores, int64_t ld, int64_t B, int64_t L, int 
   a.cached = chunk <= TK_CACHE ? 1 : 0;
   // all-gathered histograms (two levels' worth), then the cached chunk
   const size_t dyn = static_cast<size_t>(2 * C * TK_BINS) * 4 + (a.cached ? static_cast<size_t>(chunk) * 4 : 0);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(C, static_cast<unsigned>(B), 1);
-  cfg.blockDim = dim3(TK_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = dyn;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  LSA_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_topk_cluster, a));
+  LSA_CUDA_TRY(launch_pdl(k_topk_cluster, dim3(C, static_cast<unsigned>(B), 1), dim3(TK_THREADS), dyn, s,
+                          static_cast<unsigned>(C), a));
   return LSA_OK;
 }
 

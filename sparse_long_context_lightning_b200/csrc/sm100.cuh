@@ -130,6 +130,13 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic-serialization attribute may start
+// while the previous kernel of the stream is still running; pdl_wait() blocks until that kernel has completed
+// and its memory is visible (a no-op without the attribute).  pdl_launch_dependents() lets the next kernel's
+// launch begin once every CTA of this grid has executed it (or exited).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------------------------
 // tcgen05
 // ---------------------------------------------------------------------------------------------
