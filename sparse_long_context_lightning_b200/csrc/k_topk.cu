@@ -68,7 +68,6 @@ struct TopkSmem {
   uint32_t wgt[TK_WARPS], weq[TK_WARPS];  // this CTA's elements with key > T / key == T, per warp
   uint32_t ccount;
   uint32_t sel_bin, sel_above, sel_count;
-  uint32_t res_T, res_need_eq;
   uint64_t load_bar[TK_PIECES];  // one per piece of the chunk's bulk copy
 };
 
@@ -482,6 +481,10 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
         sm.eqb[tid] = hl[tid * TK_BINS + bstar];
       }
     } else {
+      if (tid < TK_BINS) {  // both local refinement histograms start empty
+        sm.h[tid] = 0;
+        sm.tot[tid] = 0;
+      }
       __syncthreads();
       const uint32_t mine = sm.segcnt[r];
       for (uint32_t i = tid; i < mine * static_cast<uint32_t>(C); i += TK_THREADS) {
@@ -497,38 +500,33 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
   }
 
   if (gathered) {
-    // ---- local refinement of the gathered boundary bin: warp 0 of every CTA, redundantly, with no
-    // block or cluster barrier between levels ----
-    if (warp == 0) {
-      const uint32_t n = sm.sel_count;
-      for (int lv = 0; lv < 6; ++lv) {
-        const int shift = level_shift(klo, khi);
-        reinterpret_cast<uint4*>(sm.h)[2 * lane] = make_uint4(0u, 0u, 0u, 0u);
-        reinterpret_cast<uint4*>(sm.h)[2 * lane + 1] = make_uint4(0u, 0u, 0u, 0u);
-        __syncwarp();
-        for (uint32_t j = lane; j < n; j += 32) {
-          const uint32_t k = sm.cand[j];
-          if (k >= klo && k <= khi) atomicAdd(&sm.h[(k - klo) >> shift], 1u);
-        }
-        __syncwarp();
-        find_boundary(sm, sm.h, need, lane);
-        __syncwarp();
-        need -= sm.sel_above;
-        uint32_t nlo, nhi;
-        bin_range(klo, khi, shift, sm.sel_bin, nlo, nhi);
-        klo = nlo;
-        khi = nhi;
-        __syncwarp();  // every lane has read sel_* and h before the next level rewrites them
-        if (nlo == nhi) break;  // reached at shift 0 at the latest
+    // ---- local refinement of the gathered boundary bin, redundantly in every CTA: one key per thread
+    // (the bin holds <= TK_CAP == TK_THREADS keys); the two histograms alternate by level, so the one
+    // for the next level is cleared while warp 0 scans this one: two block barriers per level ----
+    static_assert(TK_CAP <= TK_THREADS, "one gathered key per thread");
+    const uint32_t n = sm.sel_count;
+    const uint32_t key = static_cast<uint32_t>(tid) < n ? sm.cand[tid] : 0u;
+    for (int lv = 0; lv < 6; ++lv) {
+      const int shift = level_shift(klo, khi);
+      uint32_t* hcur = (lv & 1) ? sm.tot : sm.h;
+      uint32_t* hnext = (lv & 1) ? sm.h : sm.tot;
+      if (static_cast<uint32_t>(tid) < n && key >= klo && key <= khi) atomicAdd(&hcur[(key - klo) >> shift], 1u);
+      __syncthreads();
+      if (warp == 0) {
+        find_boundary(sm, hcur, need, lane);
+      } else if (tid < TK_BINS + 32) {
+        hnext[tid - 32] = 0u;  // scanned by the previous level, which ended at a barrier
       }
-      if (lane == 0) {
-        sm.res_T = klo;
-        sm.res_need_eq = need;
-      }
+      __syncthreads();
+      need -= sm.sel_above;
+      uint32_t nlo, nhi;
+      bin_range(klo, khi, shift, sm.sel_bin, nlo, nhi);
+      klo = nlo;
+      khi = nhi;
+      if (nlo == nhi) break;  // reached at shift 0 at the latest
     }
-    __syncthreads();
-    T = sm.res_T;
-    need_eq = sm.res_need_eq;
+    T = klo;
+    need_eq = need;
     if (warp < C) {  // CTA `warp`'s boundary elements above / at T
       const uint32_t o = sm.segoff[warp], m = sm.segcnt[warp];
       uint32_t g = 0, e = 0;
