@@ -56,6 +56,44 @@ struct IxArgs {
   int tiles_per_range;
 };
 
+// acc0 = sum_c w[c] ReLU(r0[c]), acc1 = sum_c w[32 + c] ReLU(r1[c]).  The 64 weights are the same for every
+// lane (a broadcast): read as 16 float4 so that the epilogue's shared-memory reads (one wavefront per load
+// instruction) stay small next to the tensor cores' operand reads from the same shared memory.
+__device__ __forceinline__ void relu_weighted_sum64(const float* w, const uint32_t (&r0)[32], const uint32_t (&r1)[32],
+                                                    float& acc0, float& acc1) {
+  const float4* w4 = reinterpret_cast<const float4*>(w);
+  acc0 = 0.f;
+  acc1 = 0.f;
+  #pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float4 v = w4[c];
+    acc0 = fmaf(v.x, fmaxf(__uint_as_float(r0[4 * c]), 0.f), acc0);
+    acc0 = fmaf(v.y, fmaxf(__uint_as_float(r0[4 * c + 1]), 0.f), acc0);
+    acc0 = fmaf(v.z, fmaxf(__uint_as_float(r0[4 * c + 2]), 0.f), acc0);
+    acc0 = fmaf(v.w, fmaxf(__uint_as_float(r0[4 * c + 3]), 0.f), acc0);
+  }
+  #pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float4 v = w4[8 + c];
+    acc1 = fmaf(v.x, fmaxf(__uint_as_float(r1[4 * c]), 0.f), acc1);
+    acc1 = fmaf(v.y, fmaxf(__uint_as_float(r1[4 * c + 1]), 0.f), acc1);
+    acc1 = fmaf(v.z, fmaxf(__uint_as_float(r1[4 * c + 2]), 0.f), acc1);
+    acc1 = fmaf(v.w, fmaxf(__uint_as_float(r1[4 * c + 3]), 0.f), acc1);
+  }
+}
+
+// The chunk's 256 (query, head) weights (times the FP8 query scales) into shared memory, by the 512 epilogue
+// threads (e = 0..511), which then synchronise among themselves (named barrier 1).
+__device__ __forceinline__ void load_weights(float* wsm, const IxArgs& a, int b0, int e) {
+  if (e < IX_CHUNK_N) {
+    const int b = b0 + e / a.H_I, j = e % a.H_I;
+    float v = 0.f;
+    if (b < a.B) v = a.w[static_cast<int64_t>(b) * a.H_I + j] * (a.q_scale ? a.q_scale[static_cast<int64_t>(b) * a.H_I + j] : 1.f);
+    wsm[e] = v;
+  }
+  named_bar_sync(1, IX_THREADS - 64);
+}
+
 template <bool FP8>
 __global__ void __launch_bounds__(IX_THREADS, 1)
     k_index_score_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q, IxArgs a) {
@@ -75,7 +113,8 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   uint64_t* tempty = tfull + 2;           // [2]
   uint64_t* qfull = tempty + 2;           // [1]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qfull + 1);
-  float* wsm = reinterpret_cast<float*>(tmem_holder + 4);  // [256] weights of this chunk's (query, head) pairs
+  // [256] weights of this chunk's (query, head) pairs, 16-byte aligned: the epilogue reads them as float4
+  float* wsm = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(bars) + 256);
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -99,12 +138,6 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     mbar_init(qfull, 1);
     abort_flag = 0;
     fence_mbar_init();
-  }
-  for (int i = tid; i < IX_CHUNK_N; i += IX_THREADS) {
-    const int b = b0 + i / a.H_I, j = i % a.H_I;
-    float v = 0.f;
-    if (b < a.B) v = a.w[static_cast<int64_t>(b) * a.H_I + j] * (a.q_scale ? a.q_scale[static_cast<int64_t>(b) * a.H_I + j] : 1.f);
-    wsm[i] = v;
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
@@ -142,7 +175,10 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_my > 0) {
       bool ok = mbar_wait(qfull, 0);
-      const uint32_t q_addr = smem_u32(q_s);
+      // descriptors of the first K step; a step's are these plus its byte offset / 16 (the start-address
+      // field holds shared addresses < 256 KB, so the addition never carries out of it)
+      const uint64_t q_desc = desc_sw128(smem_u32(q_s));
+      const uint64_t k_desc = desc_sw128(smem_u32(k_s));
       for (int i = 0; ok && i < n_my; ++i) {
         const int st = i % C::STAGES;
         const int buf = i & 1;
@@ -151,12 +187,12 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(k_s + st * C::TILE_BYTES);
+        const uint64_t kd = k_desc + static_cast<uint64_t>((st * C::TILE_BYTES) >> 4);
         #pragma unroll
         for (int k = 0; k < C::KSTEPS; ++k) {
           const int kb = k >> 2, kk = k & 3;
-          const uint64_t ad = desc_sw128(k_addr + kb * IX_TILE_M * 128 + kk * 32);
-          const uint64_t bd = desc_sw128(q_addr + kb * IX_CHUNK_N * 128 + kk * 32);
+          const uint64_t ad = kd + static_cast<uint64_t>((kb * IX_TILE_M * 128 + kk * 32) >> 4);
+          const uint64_t bd = q_desc + static_cast<uint64_t>((kb * IX_CHUNK_N * 128 + kk * 32) >> 4);
           if (FP8)
             mma_f8(tmem + buf * IX_CHUNK_N, ad, bd, C::IDESC, k > 0);
           else
@@ -173,6 +209,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..17)
     // warp e handles TMEM lanes 32*(warp % 4) .. +31 (its keys) and chunk columns [64*(e/4), +64)
+    load_weights(wsm, a, b0, tid - 64);  // off the producer's critical path: needed at the first tfull
     const int ew = warp - 2;
     const int quarter = warp & 3;
     const int col0 = (ew >> 2) * 64;
@@ -194,12 +231,8 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       if (lane == 0) mbar_arrive(&tempty[buf]);  // the accumulator columns are in registers now
       const int s = (t_begin + i) * IX_TILE_M + quarter * 32 + lane;
       const float ks = (FP8 && s < a.L) ? a.k_scale[s] : 1.f;
-      const float* wv = wsm + col0;
-      float acc0 = 0.f, acc1 = 0.f;
-      #pragma unroll
-      for (int c = 0; c < 32; ++c) acc0 = fmaf(wv[c], fmaxf(__uint_as_float(r0[c]), 0.f), acc0);
-      #pragma unroll
-      for (int c = 0; c < 32; ++c) acc1 = fmaf(wv[32 + c], fmaxf(__uint_as_float(r1[c]), 0.f), acc1);
+      float acc0, acc1;
+      relu_weighted_sum64(wsm + col0, r0, r1, acc0, acc1);
       if (s < a.L) {
         if (nq == 1) {
           const int b = b0 + col0 / a.H_I;
@@ -319,7 +352,8 @@ int launch_index_score(const void* q, const float* q_scale, const float* w, cons
   const bool tc = d_I == 128 && (H_I == 32 || H_I == 64) && aligned16(q) && aligned16(k) && L >= IX_TILE_M &&
                   L < (int64_t(1) << 31);
   if (!tc) return launch_score_simt(q, q_scale, w, k, k_scale, dtype, B, H_I, d_I, L, q_pos, scores, ld, s);
-  if (dtype == LSA_FP8_E4M3) return launch_tc<true>(q, q_scale, w, k, k_scale, B, H_I, L, q_pos, scores, ld, s);
+  const bool fp8 = dtype == LSA_FP8_E4M3;
+  if (fp8) return launch_tc<true>(q, q_scale, w, k, k_scale, B, H_I, L, q_pos, scores, ld, s);
   return launch_tc<false>(q, q_scale, w, k, k_scale, B, H_I, L, q_pos, scores, ld, s);
 }
 

@@ -266,7 +266,9 @@ __device__ __forceinline__ void st_async_v4(uint32_t caddr, float a, float b, fl
                ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(cbar)
                : "memory");
 }
-// arrive (release at cluster scope) on an mbarrier given by its shared::cluster address
+// arrive (release at cluster scope) on an mbarrier given by its shared::cluster address.  The release orders
+// every earlier memory access of the thread, global stores included, at cluster scope: it waits for them
+// (~0.8 us after a tile's global stores).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
 }
