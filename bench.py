@@ -11,6 +11,10 @@ outside the per-step CUDA events.  Rank 0 prints one JSON line.
 N > 1 (torchrun): every rank runs an independent replica of the same decode batch (the path has no
 exchange step on one node here: replicas only), timed per rank, max over ranks.
 
+"e2e" is the same step through the C-ABI with host buffers: every step copies its inputs from pinned host
+memory, runs the three calls and copies the output back.  The sequence is captured once as a CUDA graph and
+replayed per step (the form a serving loop uses); "eager_ms_per_step" is the same sequence issued call by call.
+
 At N = 1 the line also carries "prefill_chunk": the latency of one causal prefill chunk (8192 queries,
 FP8 scan + bf16 re-rank, K = 2048 + sink 4 + window 128) with its per-stage times (--no-prefill skips it).
 """
@@ -23,6 +27,7 @@ import json
 import math
 import os
 import subprocess
+import sys
 import threading
 import time
 
@@ -297,11 +302,7 @@ def run_gpu(args, rank, world, local_rank):
     h_lse = torch.empty_like(step.lse, device="cpu").pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (h_q_in, h_w, h_q, h_qpos, h_qs, h_qI) if t is not None)
     d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        l2_flush()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+    def e2e_body():
         step.q_in.copy_(h_q_in, non_blocking=True)
         step.w.copy_(h_w, non_blocking=True)
         if h_qs is not None:
@@ -314,11 +315,34 @@ def run_gpu(args, rank, world, local_rank):
         step.attn()
         h_out.copy_(step.out, non_blocking=True)
         h_lse.copy_(step.lse, non_blocking=True)
-        e1.record(stream)
-        e1.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(e0.elapsed_time(e1))
-    e2e_step = float(np.mean(e2e_ms))
+
+    def e2e_time(run):
+        ms = []
+        for i in range(args.warmup + args.steps):
+            l2_flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            run()
+            e1.record(stream)
+            e1.synchronize()
+            if i >= args.warmup:
+                ms.append(e0.elapsed_time(e1))
+        return float(np.mean(ms))
+
+    # eagerly (one host call per copy and per C-ABI call), then the same sequence captured once as a CUDA graph
+    # and replayed: the serving form, where the host launches a step with one call
+    e2e_eager = e2e_time(e2e_body)
+    e2e_mode = "cuda-graph"
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            e2e_body()
+        torch.cuda.synchronize()
+        e2e_step = e2e_time(graph.replay)
+    except Exception as exc:  # capture unsupported here: report the eager figure
+        print(f"[bench] CUDA-graph capture of the e2e step failed ({exc}); reporting the eager e2e", file=sys.stderr)
+        graph, e2e_mode, e2e_step = None, "eager", e2e_eager
+    del graph
 
     # max over ranks
     vals = torch.tensor([step_ms, e2e_step, *stage_ms.tolist()], dtype=torch.float64, device=device)
@@ -378,7 +402,8 @@ def run_gpu(args, rank, world, local_rank):
         "stages": stages,
         "roofline": roof,
         "e2e": {"value": round(wl.B * world / (e2e_step * 1e-3), 1), "unit": "queries/s",
-                "ms_per_step": round(e2e_step, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+                "ms_per_step": round(e2e_step, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "mode": e2e_mode, "eager_ms_per_step": round(e2e_eager, 5)},
         "gpu_launches": n_launch,
         "clocks": clk.summary(),
         "wall_s_timed_region": round(wall, 4),
