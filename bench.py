@@ -15,7 +15,8 @@ exchange step on one node here: replicas only), timed per rank, max over ranks.
 memory, runs the three calls and copies the output back.  The sequence is captured once as a CUDA graph and
 replayed per step (the form a serving loop uses); "eager_ms_per_step" is the same sequence issued call by call.
 
-At N = 1 the line also carries "prefill_chunk": the latency of one causal prefill chunk (8192 queries,
+At N = 1 the line also carries "long_context": per-stage times of the 1M-token decode (FP8 token path and
+micro-block selection) and of the 10M-token Flat bucket workload (--no-configs skips them), and "prefill_chunk": the latency of one causal prefill chunk (8192 queries,
 FP8 scan + bf16 re-rank, K = 2048 + sink 4 + window 128) with its per-stage times (--no-prefill skips it).
 """
 
@@ -237,6 +238,128 @@ def prefill_chunk(device, l2_flush, iters: int = 3):
             "queries_per_s": round(wl.B / (ms * 1e-3), 1), "iterations": iters}
 
 
+class BucketStep:
+    """Representative (bucket / micro-block) selection then attention: the C-ABI calls of one step of the
+    micro-block (4-token blocks, top-512 + tail) or Flat (64-member buckets, top-32) variant.  The
+    representatives are built once before timing (the untimed precompute)."""
+
+    def __init__(self, wl: S.Workload, device):
+        import sparse_long_context_lightning_b200 as lsa
+
+        self.lsa, self.wl = lsa, wl
+        q_I, w = S.index_queries(wl, "cpu")
+        k_I = S.index_keys(wl, q_I, device)
+        self.q_I, self.w = q_I.to(device), w.to(device)
+        self.members = S.bucket_members(wl, device) if wl.mode == "flat" else None
+        nb = self.members.shape[0] if self.members is not None else wl.L // wl.bsz
+        self.cen = torch.empty(nb, wl.d_I, device=device)
+        lsa.lsa_pool_keys(k_I, self.cen, wl.bsz, members=self.members)
+        del k_I
+        self.q_pos = wl.q_pos().to(device)
+        self.idx = torch.empty(wl.B, wl.kmax, dtype=torch.int32, device=device)
+        self.cnt = torch.empty(wl.B, dtype=torch.int32, device=device)
+        self.ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_BUCKET, wl.B, nb, wl.M), device)
+        self.q = S.attn_queries(wl, device)
+        self.kv = S.latent_cache(wl, device)
+        self.out = torch.empty(wl.B, wl.H, wl.d_v, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(wl.B, wl.H, device=device)
+        self.ws_a = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_ATTN, wl.B, wl.L, wl.kmax, wl.H), device)
+        self.nb = nb
+
+    def select(self):
+        wl = self.wl
+        self.lsa.lsa_bucket_select(self.q_I, self.w, self.cen, self.members, wl.bsz, wl.M, wl.sink, wl.window, wl.L,
+                                   self.q_pos, self.idx, self.cnt, self.ws)
+
+    def attn(self):
+        self.lsa.lsa_sparse_attn(self.q, self.kv, self.idx, self.cnt, self.wl.scale, self.out, self.lse, self.ws_a)
+
+
+def _time_stages(stages, l2_flush, iters):
+    """Mean CUDA-event time (ms) of each callable in `stages`, run in order, L2 flushed before each pass."""
+    stream = torch.cuda.current_stream()
+    n = len(stages)
+
+    def once(ev):
+        ev[0].record(stream)
+        for j, f in enumerate(stages):
+            f()
+            ev[j + 1].record(stream)
+
+    for _ in range(3):
+        l2_flush()
+        once([torch.cuda.Event(enable_timing=True) for _ in range(n + 1)])
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(iters)]
+    for i in range(iters):
+        l2_flush()
+        once(evs[i])
+    torch.cuda.synchronize()
+    return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n)] for i in range(iters)]).mean(axis=0)
+
+
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1965 MHz (clocks.max.sm)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def _stage(ms, nbytes, flops=None, peak_tflops=None, pipe="tensor"):
+    hbm = peaks()[0]["hbm_gbs"]
+    d = {"ms": round(float(ms), 5), "algorithmic_bytes": int(nbytes),
+         "achieved_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)}
+    if flops:
+        d["algorithmic_flops"] = float(flops)
+        d["achieved_tflops"] = round(flops / (ms * 1e-3) / 1e12, 2)
+        d[f"{pipe}_frac"] = round(flops / (ms * 1e-3) / 1e12 / peak_tflops, 4)
+    return d
+
+
+def long_context_configs(device, l2_flush, iters: int = 10):
+    """Per-stage times of the long-context workloads (one GPU, inputs resident, L2 flushed before each pass):
+    1M-token decode with the FP8 token path, 1M-token decode with micro-block selection, and the 10M-token
+    Flat bucket workload.  Each stage's fraction is against the measured HBM copy peak (and, for the indexer,
+    the FP8 tensor peak = measured bf16 x 2)."""
+    res = {}
+    bf16 = peaks()[0]["bf16_tflops"]
+    # 1M tokens, FP8 scan -> top-2K -> exact bf16 re-rank -> attention
+    wl = S.WORKLOADS["decode1m"]
+    step = DecodeStep(wl, "fp8", device)
+    st = _time_stages([step.index, step.topk, step.attn], l2_flush, iters)
+    rows = float(step.cnt.sum().item())
+    B, L = wl.B, wl.L
+    ix_bytes = L * wl.d_I + L * 4 + B * L * 4 + B * wl.H_I * wl.d_I + B * wl.H_I * 8
+    ix_flops = 2.0 * B * wl.H_I * wl.d_I * L
+    tk_bytes = B * L * 4 + B * 2 * wl.K * (wl.d_I * 2 + 4) + B * step.kmax * 4
+    at_bytes = rows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
+    res["decode1m_fp8"] = {
+        "workload": "B=4 decode queries, L=1048576, e4m3 indexer (H_I=64, d_I=128), top-4096 + exact bf16 re-rank "
+                    "to K=2048, sink 4 + window 128, H=128",
+        "stages": {"index": _stage(st[0], ix_bytes, ix_flops, FP8_OVER_BF16 * bf16), "topk_rerank": _stage(st[1], tk_bytes),
+                   "attn": _stage(st[2], at_bytes)},
+        "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
+    del step
+    torch.cuda.empty_cache()
+    for name in ("decode1m_mb", "flat10m"):
+        wl = S.WORKLOADS[name]
+        bstep = BucketStep(wl, device)
+        st = _time_stages([bstep.select, bstep.attn], l2_flush, iters)
+        B = wl.B
+        rows = float(bstep.cnt.sum().item())
+        sel_bytes = bstep.nb * wl.d_I * 4 + B * bstep.nb * 4 + B * wl.kmax * 4 + \
+            (B * wl.M * wl.bsz * 4 if wl.mode == "flat" else 0)
+        sel_flops = 2.0 * B * wl.H_I * wl.d_I * bstep.nb
+        at_bytes = rows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
+        desc = ("B=4 decode queries, L=1048576, 4-token mean-pooled blocks (fp32), top-512 blocks + tail + sink 4 + "
+                "window 128, H=128" if name == "decode1m_mb" else
+                "B=8 decode queries, L=10000000, 156250 Flat buckets of 64 (fp32 representatives), top-32 buckets + "
+                "sink 4 + window 512, H=128, 11.5 GB latent cache")
+        res[name] = {"workload": desc,
+                     "stages": {"bucket_select": _stage(st[0], sel_bytes, sel_flops, FP32_ALU_TFLOPS, "fp32_alu"),
+                                "attn": _stage(st[1], at_bytes)},
+                     "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
+        del bstep
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_gpu(args, rank, world, local_rank):
     import sparse_long_context_lightning_b200 as lsa
 
@@ -353,6 +476,7 @@ def run_gpu(args, rank, world, local_rank):
     if rank != 0:
         return None
     prefill = None if (args.no_prefill or world > 1) else prefill_chunk(device, l2_flush)
+    long_ctx = None if (args.no_configs or world > 1) else long_context_configs(device, l2_flush)
 
     pk, pk_src = peaks()
     work = algorithmic_work(wl, counts, step.fp8)
@@ -408,6 +532,7 @@ def run_gpu(args, rank, world, local_rank):
         "clocks": clk.summary(),
         "wall_s_timed_region": round(wall, 4),
         "prefill_chunk": prefill,
+        "long_context": long_ctx,
     }
 
 
@@ -487,6 +612,8 @@ def main():
     ap.add_argument("--index", default="bf16", choices=["bf16", "fp8"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-chunk latency measurement")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the long-context workloads (1M-token FP8 / micro-block decode, 10M-token Flat)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

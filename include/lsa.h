@@ -48,7 +48,13 @@ typedef enum {
   LSA_FP8_E4M3 = 1  /* OCP e4m3fn codes with one fp32 scale per row (value = code*scale) */
 } lsa_dtype;
 
-typedef enum { LSA_OP_TOPK = 1, LSA_OP_BUCKET = 2, LSA_OP_ATTN = 3, LSA_OP_REFINE = 4 } lsa_op;
+typedef enum {
+  LSA_OP_TOPK = 1,
+  LSA_OP_BUCKET = 2,
+  LSA_OP_ATTN = 3,
+  LSA_OP_REFINE = 4,
+  LSA_OP_BUCKET_MIN = 5 /* the smaller lsa_bucket_select workspace: CUDA-core representative scoring */
+} lsa_op;
 
 /*
  * lsa_index_score -- lightning-indexer scores.
@@ -151,7 +157,13 @@ int lsa_pool_keys(const void* k_idx, int dtype, const float* k_scale, int64_t L,
  *   fp32, members int32 [NB, bsz] or NULL.  idx int32 [B, idx_ld] with
  *   idx_ld >= M*bsz + sink + window (+ bsz-1 for the micro-block tail); count int32 [B].
  *   1 <= M <= 1024, M*bsz + bsz + sink + window <= 8192.
- *   ws: lsa_workspace_size(LSA_OP_BUCKET, B, NB, M, 0, 0, 0) bytes.
+ *   ws: lsa_workspace_size(LSA_OP_BUCKET, B, NB, M, 0, 0, 0) bytes; at least
+ *   lsa_workspace_size(LSA_OP_BUCKET_MIN, B, NB, M, 0, 0, 0) bytes (else LSA_ERR_WORKSPACE).
+ *   Scoring: with the full workspace and d_I = 128, H_I in {32, 64}, NB >= 128 the representatives are
+ *   scored on the tensor cores from their exact three-part bf16 split (written into the workspace each
+ *   call: every product with the bf16 query is exact, the sums are fp32); otherwise on the CUDA cores
+ *   (fp32).  Both are fp32-accurate; they can keep different buckets only where two representatives'
+ *   scores lie within fp32 rounding of the M-th.
  */
 int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, int dtype,
                       int64_t B, int H_I, int d_I, const float* centroids, int64_t NB,
@@ -163,14 +175,15 @@ int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, i
  * lsa_bucket_select_noalloc -- lsa_bucket_select for callers that cannot allocate device memory.
  *   The pages have no counterpart: this is a packaging variant of lsa_bucket_select.
  *
- *   Same arguments, layouts and results as lsa_bucket_select, minus ws / ws_bytes.  It is meant for
+ *   Same arguments, layouts and results as lsa_bucket_select given the smaller workspace
+ *   (LSA_OP_BUCKET_MIN: CUDA-core scoring), minus ws / ws_bytes.  It is meant for
  *   callers that may not call cudaMalloc (or any allocating library routine) where they select: a
  *   plugin inside a host framework that owns every device allocation, a thread that must stay out of
  *   the CUDA allocator, or a process with no allocation budget left.  The scratch comes from an 8 MiB
  *   buffer compiled into the library as a __device__ array; the CUDA runtime creates it on every GPU
  *   that loads the library, and it stays allocated there until the process exits.  The call itself
  *   allocates nothing.
- *   - Limit: lsa_workspace_size(LSA_OP_BUCKET, B, NB, M, 0, 0, 0) must be <= 8 MiB (8388608 bytes);
+ *   - Limit: lsa_workspace_size(LSA_OP_BUCKET_MIN, B, NB, M, 0, 0, 0) must be <= 8 MiB (8388608 bytes);
  *     larger requests return LSA_ERR_WORKSPACE before anything is launched (lsa_last_error() gives
  *     the sizes).  Flat selection over 156250 buckets fits up to B = 13 queries.
  *   - Set-up: the first call on a device looks up the buffer's device address (cudaGetSymbolAddress,
@@ -210,7 +223,9 @@ int lsa_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx
 /*
  * lsa_workspace_size -- scratch bytes a call needs (0 if none).
  *   op = LSA_OP_TOPK:   0.
- *   op = LSA_OP_BUCKET: (B, L=NB, K=M) -> per-query bucket scores and kept-bucket lists.
+ *   op = LSA_OP_BUCKET: (B, L=NB, K=M) -> per-query bucket scores and kept-bucket lists, plus the
+ *                       representatives' bf16 split for tensor-core scoring (NB * 768 bytes).
+ *   op = LSA_OP_BUCKET_MIN: the same without the split (CUDA-core scoring).
  *   op = LSA_OP_ATTN:   (B, L, K=idx_ld, H) -> split-K partial outputs.
  *   op = LSA_OP_REFINE: (B, L=cand_ld, K) -> re-ranked scores and kept lists.
  *   Returns (size_t)-1 for an unknown op or negative sizes.

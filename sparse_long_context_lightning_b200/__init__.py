@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "liblsa.so")
 LSA_OK = 0
 LSA_BF16 = 0
 LSA_FP8_E4M3 = 1
-LSA_OP_TOPK, LSA_OP_BUCKET, LSA_OP_ATTN, LSA_OP_REFINE = 1, 2, 3, 4
+LSA_OP_TOPK, LSA_OP_BUCKET, LSA_OP_ATTN, LSA_OP_REFINE, LSA_OP_BUCKET_MIN = 1, 2, 3, 4, 5
 
 _STATUS = {0: "LSA_OK", -1: "LSA_ERR_INVALID_ARG", -2: "LSA_ERR_UNSUPPORTED", -3: "LSA_ERR_WORKSPACE",
            -4: "LSA_ERR_CUDA", -5: "LSA_ERR_DEVICE_CHECK", -6: "LSA_ERR_TIMEOUT"}

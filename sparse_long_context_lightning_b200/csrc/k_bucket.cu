@@ -8,7 +8,12 @@
 // micro-blocks; the visible tokens of the incomplete tail block are added directly.
 #include "lsa_common.cuh"
 
+#include <algorithm>
+
 namespace lsa {
+
+int sm_count();
+
 namespace {
 
 // centroids[c, d] = sum_i k[m(c,i), d] / bsz, one thread per (bucket, 4 dims), members in order.
@@ -142,6 +147,31 @@ __global__ void __launch_bounds__(EX_THREADS) k_bucket_expand(
   if (tid == 0) count[b] = static_cast<int32_t>(total);
 }
 
+// out[p * n + i] (p = 0, 1, 2): bf16 parts of x[i] with x[i] = part0 + part1 + part2 exactly.  Each part is
+// the round-to-nearest bf16 of what the earlier parts leave; the remainders are exact fp32 differences and
+// shrink by 8 significand bits per part, so the third part holds the last 8 of fp32's 24 bits exactly.
+__global__ void k_split_bf16x3(const float4* __restrict__ x, int64_t n4, uint2* __restrict__ out) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = x[i];
+    const float e[4] = {v.x, v.y, v.z, v.w};
+    uint32_t part[3][4];
+    #pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float r = e[c];
+      #pragma unroll
+      for (int p = 0; p < 3; ++p) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(r);
+        part[p][c] = static_cast<uint32_t>(__bfloat16_as_ushort(h));
+        r -= __bfloat162float(h);
+      }
+    }
+    #pragma unroll
+    for (int p = 0; p < 3; ++p)
+      out[p * n4 + i] = make_uint2(part[p][0] | (part[p][1] << 16), part[p][2] | (part[p][3] << 16));
+  }
+}
+
 }  // namespace
 
 int launch_pool_keys(const void* k, int dtype, const float* k_scale, int64_t L, int d_I, const int32_t* members,
@@ -154,6 +184,17 @@ int launch_pool_keys(const void* k, int dtype, const float* k_scale, int64_t L, 
     k_pool_keys<LSA_BF16><<<static_cast<unsigned>(grid), bs, 0, s>>>(k, k_scale, L, d_I, members, bsz, NB, centroids);
   else
     k_pool_keys<LSA_FP8_E4M3><<<static_cast<unsigned>(grid), bs, 0, s>>>(k, k_scale, L, d_I, members, bsz, NB, centroids);
+  return cuda_status(cudaGetLastError());
+}
+
+// fp32 [n] (n % 4 == 0, 16-byte aligned) -> bf16 [3, n]
+int launch_split_bf16x3(const float* x, int64_t n, void* out, cudaStream_t s) {
+  if (n == 0) return LSA_OK;
+  const int64_t n4 = n / 4;
+  const int threads = 256;
+  const int64_t blocks = std::min<int64_t>(cdiv(n4, threads), static_cast<int64_t>(sm_count()) * 8);
+  k_split_bf16x3<<<static_cast<unsigned>(blocks), threads, 0, s>>>(reinterpret_cast<const float4*>(x), n4,
+                                                                   static_cast<uint2*>(out));
   return cuda_status(cudaGetLastError());
 }
 

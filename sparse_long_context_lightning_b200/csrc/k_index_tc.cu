@@ -54,6 +54,7 @@ struct IxArgs {
   int n_chunks;
   int ntiles;
   int tiles_per_range;
+  int split_rows;  // SPLITS > 1: rows between the key matrices that are summed (the exact bf16 split parts)
 };
 
 // acc0 = sum_c w[c] ReLU(r0[c]), acc1 = sum_c w[32 + c] ReLU(r1[c]).  The 64 weights are the same for every
@@ -94,9 +95,13 @@ __device__ __forceinline__ void load_weights(float* wsm, const IxArgs& a, int b0
   named_bar_sync(1, IX_THREADS - 64);
 }
 
-template <bool FP8>
+// SPLITS > 1 (bf16 only): each key is the sum of SPLITS bf16 rows, split_rows apart in the key matrix (the
+// exact three-part bf16 split of an fp32 key): a tile's accumulator takes SPLITS consecutive key stages
+// before its epilogue.  q_pos == nullptr: no causal mask.
+template <bool FP8, int SPLITS>
 __global__ void __launch_bounds__(IX_THREADS, 1)
     k_index_score_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q, IxArgs a) {
+  static_assert(SPLITS == 1 || !FP8, "split keys are bf16");
   // every global access of this kernel comes after the previous kernel of the stream has completed
   sm100::pdl_wait();
   sm100::pdl_launch_dependents();
@@ -156,16 +161,16 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       mbar_expect_tx(qfull, C::Q_BYTES);
       for (int kb = 0; kb < C::KB; ++kb)
         tma_load_2d(q_s + kb * IX_CHUNK_N * 128, &tm_q, qfull, kb * (FP8 ? 128 : 64), chunk * IX_CHUNK_N);
-      for (int i = 0; i < n_my; ++i) {
-        const int st = i % C::STAGES;
-        const uint32_t par = ((i / C::STAGES) & 1) ^ 1;
+      for (int j = 0; j < n_my * SPLITS; ++j) {  // stage j: tile j / SPLITS, split part j % SPLITS
+        const int st = j % C::STAGES;
+        const uint32_t par = ((j / C::STAGES) & 1) ^ 1;
         if (!mbar_wait(&empty[st], par)) {
           atomicExch(&g_index_tc_timeout, 1);
           abort_flag = 1;
           break;
         }
         mbar_expect_tx(&full[st], C::TILE_BYTES);
-        const int row = (t_begin + i) * IX_TILE_M;
+        const int row = (t_begin + j / SPLITS) * IX_TILE_M + (j % SPLITS) * a.split_rows;
         unsigned char* dst = k_s + st * C::TILE_BYTES;
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_2d(dst + kb * IX_TILE_M * 128, &tm_k, &full[st], kb * (FP8 ? 128 : 64), row);
@@ -180,25 +185,34 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       const uint64_t q_desc = desc_sw128(smem_u32(q_s));
       const uint64_t k_desc = desc_sw128(smem_u32(k_s));
       for (int i = 0; ok && i < n_my; ++i) {
-        const int st = i % C::STAGES;
         const int buf = i & 1;
-        if (!mbar_wait(&full[st], (i / C::STAGES) & 1) || !mbar_wait(&tempty[buf], ((i >> 1) & 1) ^ 1)) {
+        if (!mbar_wait(&tempty[buf], ((i >> 1) & 1) ^ 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        const uint64_t kd = k_desc + static_cast<uint64_t>((st * C::TILE_BYTES) >> 4);
-        #pragma unroll
-        for (int k = 0; k < C::KSTEPS; ++k) {
-          const int kb = k >> 2, kk = k & 3;
-          const uint64_t ad = kd + static_cast<uint64_t>((kb * IX_TILE_M * 128 + kk * 32) >> 4);
-          const uint64_t bd = q_desc + static_cast<uint64_t>((kb * IX_CHUNK_N * 128 + kk * 32) >> 4);
-          if (FP8)
-            mma_f8(tmem + buf * IX_CHUNK_N, ad, bd, C::IDESC, k > 0);
-          else
-            mma_f16(tmem + buf * IX_CHUNK_N, ad, bd, C::IDESC, k > 0);
+        #pragma unroll 1
+        for (int p = 0; p < SPLITS; ++p) {
+          const int j = i * SPLITS + p;
+          const int st = j % C::STAGES;
+          if (!mbar_wait(&full[st], (j / C::STAGES) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t kd = k_desc + static_cast<uint64_t>((st * C::TILE_BYTES) >> 4);
+          #pragma unroll
+          for (int k = 0; k < C::KSTEPS; ++k) {
+            const int kb = k >> 2, kk = k & 3;
+            const uint64_t ad = kd + static_cast<uint64_t>((kb * IX_TILE_M * 128 + kk * 32) >> 4);
+            const uint64_t bd = q_desc + static_cast<uint64_t>((kb * IX_CHUNK_N * 128 + kk * 32) >> 4);
+            if (FP8)
+              mma_f8(tmem + buf * IX_CHUNK_N, ad, bd, C::IDESC, (p | k) != 0);
+            else
+              mma_f16(tmem + buf * IX_CHUNK_N, ad, bd, C::IDESC, (p | k) != 0);
+          }
+          mma_commit(&empty[st]);
         }
-        mma_commit(&empty[st]);
+        if (!ok) break;
         mma_commit(&tfull[buf]);
       }
       if (!ok) {
@@ -236,11 +250,11 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       if (s < a.L) {
         if (nq == 1) {
           const int b = b0 + col0 / a.H_I;
-          if (b < a.B) a.scores[static_cast<int64_t>(b) * a.ld + s] = (s > a.q_pos[b]) ? -INFINITY : (acc0 + acc1) * ks;
+          if (b < a.B) a.scores[static_cast<int64_t>(b) * a.ld + s] = (a.q_pos && s > a.q_pos[b]) ? -INFINITY : (acc0 + acc1) * ks;
         } else {
           const int bA = b0 + col0 / a.H_I, bB = bA + 1;
-          if (bA < a.B) a.scores[static_cast<int64_t>(bA) * a.ld + s] = (s > a.q_pos[bA]) ? -INFINITY : acc0 * ks;
-          if (bB < a.B) a.scores[static_cast<int64_t>(bB) * a.ld + s] = (s > a.q_pos[bB]) ? -INFINITY : acc1 * ks;
+          if (bA < a.B) a.scores[static_cast<int64_t>(bA) * a.ld + s] = (a.q_pos && s > a.q_pos[bA]) ? -INFINITY : acc0 * ks;
+          if (bB < a.B) a.scores[static_cast<int64_t>(bB) * a.ld + s] = (a.q_pos && s > a.q_pos[bB]) ? -INFINITY : acc1 * ks;
         }
       }
     }
@@ -253,13 +267,13 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   }
 }
 
-template <bool FP8>
+template <bool FP8, int SPLITS>
 int launch_tc(const void* q, const float* q_scale, const float* w, const void* k, const float* k_scale, int64_t B,
               int H_I, int64_t L, const int64_t* q_pos, float* scores, int64_t ld, cudaStream_t s) {
   using C = IxCfg<FP8>;
   CUtensorMap tk, tq;
   const int boxc = FP8 ? 128 : 64;
-  int st = make_map(&tk, k, FP8, L, 128, boxc, IX_TILE_M);
+  int st = make_map(&tk, k, FP8, L * SPLITS, 128, boxc, IX_TILE_M);
   if (st) return st;
   st = make_map(&tq, q, FP8, B * H_I, 128, boxc, IX_CHUNK_N);
   if (st) return st;
@@ -279,10 +293,11 @@ int launch_tc(const void* q, const float* q_scale, const float* w, const void* k
   int ranges = a.n_chunks >= sms ? 1 : static_cast<int>(cdiv(sms, a.n_chunks));
   if (ranges > a.ntiles) ranges = a.ntiles;
   a.tiles_per_range = static_cast<int>(cdiv(a.ntiles, ranges));
+  a.split_rows = static_cast<int>(L);
   ranges = static_cast<int>(cdiv(a.ntiles, a.tiles_per_range));
-  LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_index_score_tc<FP8>), C::SMEM));
+  LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_index_score_tc<FP8, SPLITS>), C::SMEM));
   const int64_t grid = static_cast<int64_t>(a.n_chunks) * ranges;
-  return cuda_status(launch_pdl(k_index_score_tc<FP8>, dim3(static_cast<unsigned>(grid)), dim3(IX_THREADS), C::SMEM, s, 0u,
+  return cuda_status(launch_pdl(k_index_score_tc<FP8, SPLITS>, dim3(static_cast<unsigned>(grid)), dim3(IX_THREADS), C::SMEM, s, 0u,
                                 tk, tq, a));
 }
 
@@ -353,8 +368,18 @@ int launch_index_score(const void* q, const float* q_scale, const float* w, cons
                   L < (int64_t(1) << 31);
   if (!tc) return launch_score_simt(q, q_scale, w, k, k_scale, dtype, B, H_I, d_I, L, q_pos, scores, ld, s);
   const bool fp8 = dtype == LSA_FP8_E4M3;
-  if (fp8) return launch_tc<true>(q, q_scale, w, k, k_scale, B, H_I, L, q_pos, scores, ld, s);
-  return launch_tc<false>(q, q_scale, w, k, k_scale, B, H_I, L, q_pos, scores, ld, s);
+  if (fp8) return launch_tc<true, 1>(q, q_scale, w, k, k_scale, B, H_I, L, q_pos, scores, ld, s);
+  return launch_tc<false, 1>(q, q_scale, w, k, k_scale, B, H_I, L, q_pos, scores, ld, s);
+}
+
+// Representative scores on the tensor cores: key n = split[n] + split[NB + n] + split[2 NB + n], the exact
+// three-part bf16 split of an fp32 representative, so every product with a bf16 query is exact and only
+// the fp32 accumulation rounds (as on the CUDA cores).  No causal mask.  Shapes: d_I = 128, H_I in {32, 64},
+// NB >= 128; the caller checks them.
+int launch_centroid_score_tc(const void* q, const float* w, const void* split, int64_t B, int H_I, int64_t NB,
+                             float* scores, int64_t ld, cudaStream_t s) {
+  if (B == 0 || NB == 0) return LSA_OK;
+  return launch_tc<false, 3>(q, nullptr, w, split, nullptr, B, H_I, NB, nullptr, scores, ld, s);
 }
 
 }  // namespace lsa

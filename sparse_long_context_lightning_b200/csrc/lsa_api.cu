@@ -33,15 +33,27 @@ int launch_attn_simt(const void* q, const void* kv, int64_t L, const int32_t* id
                      const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, cudaStream_t s);
 
 // Scratch layout of lsa_bucket_select: bucket scores [B, ld_nb] fp32 | kept [B, M] int32 | kept_count [B] int32
-static void bucket_ws_layout(int64_t B, int64_t NB, int M, size_t* off_kept, size_t* off_cnt, size_t* total,
-                             int64_t* ld_nb) {
+// | (tensor-core scoring) the representatives' exact three-part bf16 split [3, NB, 128] bf16.  Without the last
+// part (a smaller workspace) the representatives are scored on the CUDA cores.
+static void bucket_ws_layout(int64_t B, int64_t NB, int M, size_t* off_kept, size_t* off_cnt, size_t* off_split,
+                             size_t* total_min, size_t* total, int64_t* ld_nb) {
   *ld_nb = (NB + 3) / 4 * 4;
   size_t o = align_up(static_cast<size_t>(B) * static_cast<size_t>(*ld_nb) * 4, 256);
   *off_kept = o;
   o = align_up(o + static_cast<size_t>(B) * static_cast<size_t>(M) * 4, 256);
   *off_cnt = o;
   o = align_up(o + static_cast<size_t>(B) * 4, 256);
-  *total = o;
+  *total_min = o;
+  *off_split = o;
+  *total = align_up(o + static_cast<size_t>(NB) * 128 * 2 * 3, 256);
+}
+
+// the workspace without the split part (CUDA-core scoring)
+size_t bucket_ws_min_bytes(int64_t B, int64_t NB, int M) {
+  size_t a, b, c, mn, tot;
+  int64_t ld;
+  bucket_ws_layout(B, NB, M, &a, &b, &c, &mn, &tot, &ld);
+  return mn;
 }
 
 }  // namespace lsa
@@ -74,11 +86,12 @@ size_t lsa_workspace_size(int op, int64_t B, int64_t L, int K, int H, int sink, 
   switch (op) {
     case LSA_OP_TOPK: return 0;
     case LSA_OP_BUCKET: {
-      size_t ok, oc, tot;
+      size_t ok, oc, osp, mn, tot;
       int64_t ldn;
-      bucket_ws_layout(B, L, K, &ok, &oc, &tot, &ldn);
+      bucket_ws_layout(B, L, K, &ok, &oc, &osp, &mn, &tot, &ldn);
       return tot;
     }
+    case LSA_OP_BUCKET_MIN: return bucket_ws_min_bytes(B, L, K);
     case LSA_OP_ATTN: return sparse_attn_ws_bytes(B, K, H);
     case LSA_OP_REFINE: return refine_ws_bytes(B, L, K);
     default: return static_cast<size_t>(-1);
@@ -165,16 +178,25 @@ int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, i
   if (B == 0) return LSA_OK;
   LSA_CHECK_ARG(B <= 65535);
   LSA_CHECK_ARG(q_idx && w && centroids && q_pos && idx && count && aligned16(centroids) && aligned16(q_idx));
-  size_t off_kept, off_cnt, total;
+  size_t off_kept, off_cnt, off_split, total_min, total;
   int64_t ldn;
-  bucket_ws_layout(B, NB, M, &off_kept, &off_cnt, &total, &ldn);
-  if (ws == nullptr || !aligned256(ws) || ws_bytes < total) return LSA_ERR_WORKSPACE;
+  bucket_ws_layout(B, NB, M, &off_kept, &off_cnt, &off_split, &total_min, &total, &ldn);
+  if (ws == nullptr || !aligned256(ws) || ws_bytes < total_min) return LSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned char* base = static_cast<unsigned char*>(ws);
   float* bscores = reinterpret_cast<float*>(base);
   int32_t* kept = reinterpret_cast<int32_t*>(base + off_kept);
   int32_t* kcnt = reinterpret_cast<int32_t*>(base + off_cnt);
-  int st = launch_centroid_score(q_idx, w, centroids, B, H_I, d_I, NB, bscores, ldn, s);
+  // tensor cores when the workspace holds the split and the shape is the tensor-core indexer's
+  const bool tc = ws_bytes >= total && d_I == 128 && (H_I == 32 || H_I == 64) && NB >= 128 && NB < (int64_t(1) << 29);
+  int st;
+  if (tc) {
+    void* split = base + off_split;
+    st = launch_split_bf16x3(centroids, NB * 128, split, s);
+    if (st == LSA_OK) st = launch_centroid_score_tc(q_idx, w, split, B, H_I, NB, bscores, ldn, s);
+  } else {
+    st = launch_centroid_score(q_idx, w, centroids, B, H_I, d_I, NB, bscores, ldn, s);
+  }
   if (st != LSA_OK) return st;
   // top-M buckets: all NB ranked (explicit members) or the complete visible micro-blocks
   st = launch_topk_mode(bscores, ldn, B, NB, M, 0, 0, q_pos, members ? 1 : 2, bsz, kept, M, kcnt, M, s);

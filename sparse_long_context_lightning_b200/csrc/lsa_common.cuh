@@ -146,6 +146,10 @@ int launch_index_score(const void* q, const float* q_scale, const float* w, cons
                        const int64_t* q_pos, float* scores, int64_t ld, cudaStream_t s);
 int launch_centroid_score(const void* q, const float* w, const float* centroids, int64_t B, int H_I,
                           int d_I, int64_t NB, float* scores, int64_t ld, cudaStream_t s);
+int launch_split_bf16x3(const float* x, int64_t n, void* out, cudaStream_t s);
+int launch_centroid_score_tc(const void* q, const float* w, const void* split, int64_t B, int H_I, int64_t NB,
+                             float* scores, int64_t ld, cudaStream_t s);
+size_t bucket_ws_min_bytes(int64_t B, int64_t NB, int M);
 int launch_topk(const float* scores, int64_t ld, int64_t B, int64_t L, int K, int sink, int window,
                 const int64_t* q_pos, int64_t rank_limit_div, int32_t* idx, int64_t idx_ld, int32_t* count,
                 int64_t kmax, cudaStream_t s);

@@ -57,7 +57,9 @@ int lsa_bucket_select_noalloc(const void* q_idx, const float* q_scale, const flo
                               int d_I, const float* centroids, int64_t NB, const int32_t* members, int bsz, int M,
                               int sink, int window, int64_t L, const int64_t* q_pos, int32_t* idx, int64_t idx_ld,
                               int32_t* count, void* stream) {
-  const size_t need = lsa_workspace_size(LSA_OP_BUCKET, B, NB, M, 0, 0, 0);
+  // the static buffer serves the CUDA-core scoring (no room reserved for the tensor-core path's split copy of
+  // the representatives)
+  const size_t need = lsa_workspace_size(LSA_OP_BUCKET_MIN, B, NB, M, 0, 0, 0);
   if (need == static_cast<size_t>(-1)) return LSA_ERR_INVALID_ARG;
   if (need > lsa::kNoAllocScratchBytes) {
     char msg[160];

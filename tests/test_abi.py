@@ -44,8 +44,11 @@ def test_status_strings(lib):
 
 def test_workspace_sizes(lib):
     assert lib.lsa_workspace_size(lsa.LSA_OP_TOPK, 16, 131072, 2048, 0, 0, 0) == 0
-    nb = lib.lsa_workspace_size(lsa.LSA_OP_BUCKET, 8, 156250, 32, 0, 0, 0)
+    nb = lib.lsa_workspace_size(lsa.LSA_OP_BUCKET_MIN, 8, 156250, 32, 0, 0, 0)
     assert nb >= 8 * 156250 * 4 + 8 * 32 * 4 + 8 * 4 and nb % 256 == 0
+    # the full workspace adds the representatives' three-part bf16 split (3 x 156250 x 128 x 2 bytes)
+    full = lib.lsa_workspace_size(lsa.LSA_OP_BUCKET, 8, 156250, 32, 0, 0, 0)
+    assert full >= nb + 3 * 156250 * 128 * 2 and full % 256 == 0
     assert lib.lsa_workspace_size(99, 1, 1, 1, 1, 0, 0) == ctypes.c_size_t(-1).value
     assert lib.lsa_workspace_size(lsa.LSA_OP_ATTN, -1, 1, 1, 1, 0, 0) == ctypes.c_size_t(-1).value
 

@@ -42,7 +42,8 @@ def test_noalloc_matches_allocating_entry_point(flat):
     q_I, w, cen, members, qp, kmax, nb = _case(L, B, M, bsz, sink, window, flat)
     ref_idx = torch.empty(B, kmax, dtype=torch.int32, device=DEV)
     ref_cnt = torch.empty(B, dtype=torch.int32, device=DEV)
-    ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_BUCKET, B, nb, M))
+    # the static scratch has the smaller workspace's layout: CUDA-core scoring, as here
+    ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_BUCKET_MIN, B, nb, M))
     lsa.lsa_bucket_select(q_I, w, cen, members, bsz, M, sink, window, L, qp, ref_idx, ref_cnt, ws)
     for _ in range(2):  # two calls in a row share the static scratch
         idx = torch.full((B, kmax), 99, dtype=torch.int32, device=DEV)
