@@ -62,70 +62,100 @@ constexpr int EX_THREADS = 1024;
 constexpr int EX_MAX = 8192;
 
 // One CTA per query: gather kept buckets' positions + tail + sink + window, bitonic sort, de-dup.
+// E elements per thread (P = 1024 E slots, blocked: thread t holds slots [E t, E t + E)); the sorting
+// network's compare-exchange stages run in registers (partner in the same thread), by warp shuffles
+// (partner in the same warp) or through shared memory (two block barriers per stage) by partner distance.
+template <int E>
 __global__ void __launch_bounds__(EX_THREADS) k_bucket_expand(
     const int32_t* __restrict__ kept, int64_t kept_ld, const int32_t* __restrict__ kept_count,
     const int32_t* __restrict__ members, int bsz, int sink, int window, int tail_block,
     const int64_t* __restrict__ q_pos, int32_t* __restrict__ idx, int64_t idx_ld,
     int32_t* __restrict__ count, int kmax) {
-  __shared__ int32_t buf[EX_MAX];
+  constexpr int P = EX_THREADS * E;
+  __shared__ int32_t buf[P];
   __shared__ uint32_t wsum[EX_THREADS / 32];
   const int b = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int qp = static_cast<int>(q_pos[b]);
-  const int nk = kept_count[b];
+  const int nk = min(kept_count[b], static_cast<int>(kept_ld));
   const int nmem = nk * bsz;
   const int nsink = min(sink, qp + 1);
   const int wlo = window > 0 ? max(0, qp - window + 1) : qp + 1;
   const int nwin = qp + 1 - wlo;
   const int tlo = tail_block > 0 ? ((qp + 1) / tail_block) * tail_block : qp + 1;
   const int ntail = qp + 1 - tlo;
-  const int n = nmem + nsink + nwin + ntail;
-  int P = 1;
-  while (P < n) P <<= 1;
-  for (int i = tid; i < P; i += EX_THREADS) {
-    int v = 0x7FFFFFFF;
+  const int n = min(nmem + nsink + nwin + ntail, P);  // the host sizes P for the largest n
+  int v[E];
+  #pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = tid * E + e;
+    int x = 0x7FFFFFFF;
     if (i < nmem) {
       const int c = kept[static_cast<int64_t>(b) * kept_ld + i / bsz];
       const int s = members ? members[static_cast<int64_t>(c) * bsz + (i % bsz)] : c * bsz + (i % bsz);
-      v = s <= qp ? s : 0x7FFFFFFF;
+      x = s <= qp ? s : 0x7FFFFFFF;
     } else if (i < nmem + nsink) {
-      v = i - nmem;
+      x = i - nmem;
     } else if (i < nmem + nsink + nwin) {
-      v = wlo + (i - nmem - nsink);
+      x = wlo + (i - nmem - nsink);
     } else if (i < n) {
-      v = tlo + (i - nmem - nsink - nwin);
+      x = tlo + (i - nmem - nsink - nwin);
     }
-    buf[i] = v;
+    v[e] = x;
   }
-  __syncthreads();
-  // bitonic sort, ascending
+  // bitonic sort, ascending: slot i meets slot i ^ j; the lower slot keeps the min when (i & k) == 0
   for (int k = 2; k <= P; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < P; i += EX_THREADS) {
-        const int l = i ^ j;
-        if (l > i) {
-          const int x = buf[i], y = buf[l];
-          const bool up = (i & k) == 0;
-          if ((x > y) == up) {
-            buf[i] = y;
-            buf[l] = x;
+      if (j < E) {
+        #pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int f = e ^ j;
+          if (f > e) {
+            const int i = tid * E + e;
+            const bool asc = (i & k) == 0;
+            const int x = v[e], y = v[f];
+            if ((x > y) == asc) {
+              v[e] = y;
+              v[f] = x;
+            }
           }
         }
+      } else if (j < 32 * E) {
+        const int tj = j / E;  // partner thread distance, < 32
+        #pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = tid * E + e;
+          const int y = __shfl_xor_sync(0xffffffffu, v[e], tj);
+          const bool keep_min = ((i & j) == 0) == ((i & k) == 0);
+          v[e] = keep_min ? min(v[e], y) : max(v[e], y);
+        }
+      } else {
+        #pragma unroll
+        for (int e = 0; e < E; ++e) buf[tid * E + e] = v[e];
+        __syncthreads();
+        #pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = tid * E + e;
+          const int y = buf[i ^ j];
+          const bool keep_min = ((i & j) == 0) == ((i & k) == 0);
+          v[e] = keep_min ? min(v[e], y) : max(v[e], y);
+        }
+        __syncthreads();
       }
-      __syncthreads();
     }
   }
-  // de-duplicate with an ordered block scan (each thread owns a contiguous run)
-  const int per = (P + EX_THREADS - 1) / EX_THREADS;
-  const int i0 = tid * per, i1 = min(P, i0 + per);
+  // de-duplicate: a slot is kept if it is valid and differs from the slot before it
+  const int prev_last = __shfl_up_sync(0xffffffffu, v[E - 1], 1);
+  buf[tid] = v[E - 1];  // for lane 0: the last slot of the previous warp's last thread
+  __syncthreads();
+  int before = tid == 0 ? -1 : (lane == 0 ? buf[tid - 1] : prev_last);
   uint32_t mine = 0;
-  for (int i = i0; i < i1; ++i) {
-    const int v = buf[i];
-    mine += (v != 0x7FFFFFFF) && (i == 0 || buf[i - 1] != v);
+  #pragma unroll
+  for (int e = 0; e < E; ++e) {
+    mine += (v[e] != 0x7FFFFFFF) && (v[e] != before);
+    before = v[e];
   }
-  // exclusive scan of `mine` across the block
   uint32_t incl = mine;
-  const int lane = tid & 31, warp = tid >> 5;
   #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
@@ -133,18 +163,22 @@ __global__ void __launch_bounds__(EX_THREADS) k_bucket_expand(
   }
   if (lane == 31) wsum[warp] = incl;
   __syncthreads();
-  uint32_t wbase = 0;
-  for (int w = 0; w < warp; ++w) wbase += wsum[w];
+  uint32_t wbase = 0, total = 0;
+  for (int w = 0; w < EX_THREADS / 32; ++w) {
+    const uint32_t x = wsum[w];
+    wbase += w < warp ? x : 0u;
+    total += x;
+  }
   uint32_t o = wbase + incl - mine;
   int32_t* out = idx + static_cast<int64_t>(b) * idx_ld;
-  for (int i = i0; i < i1; ++i) {
-    const int v = buf[i];
-    if ((v != 0x7FFFFFFF) && (i == 0 || buf[i - 1] != v)) out[o++] = v;
+  before = tid == 0 ? -1 : (lane == 0 ? buf[tid - 1] : prev_last);
+  #pragma unroll
+  for (int e = 0; e < E; ++e) {
+    if ((v[e] != 0x7FFFFFFF) && (v[e] != before) && o < static_cast<uint32_t>(kmax)) out[o++] = v[e];
+    before = v[e];
   }
-  uint32_t total = 0;
-  for (int w = 0; w < EX_THREADS / 32; ++w) total += wsum[w];
   for (int i = static_cast<int>(total) + tid; i < kmax; i += EX_THREADS) out[i] = -1;
-  if (tid == 0) count[b] = static_cast<int32_t>(total);
+  if (tid == 0) count[b] = static_cast<int32_t>(min(total, static_cast<uint32_t>(kmax)));
 }
 
 // out[p * n + i] (p = 0, 1, 2): bf16 parts of x[i] with x[i] = part0 + part1 + part2 exactly.  Each part is
@@ -202,9 +236,23 @@ int launch_bucket_expand(const int32_t* kept, int64_t kept_ld, const int32_t* ke
                          int bsz, int sink, int window, int tail_block, const int64_t* q_pos, int64_t B,
                          int32_t* idx, int64_t idx_ld, int32_t* count, int64_t kmax, cudaStream_t s) {
   if (B == 0) return LSA_OK;
-  k_bucket_expand<<<static_cast<unsigned>(B), EX_THREADS, 0, s>>>(kept, kept_ld, kept_count, members, bsz, sink,
-                                                                  window, tail_block, q_pos, idx, idx_ld, count,
-                                                                  static_cast<int>(kmax));
+  // slots for the largest union: every kept bucket's members + sink + window + tail
+  const int64_t nmax = kept_ld * bsz + sink + window + (tail_block > 0 ? tail_block - 1 : 0);
+  if (nmax > EX_MAX) return LSA_ERR_INVALID_ARG;
+  const dim3 grid(static_cast<unsigned>(B)), block(EX_THREADS);
+  const int km = static_cast<int>(kmax);
+  if (nmax <= 1024)
+    k_bucket_expand<1><<<grid, block, 0, s>>>(kept, kept_ld, kept_count, members, bsz, sink, window, tail_block, q_pos,
+                                              idx, idx_ld, count, km);
+  else if (nmax <= 2048)
+    k_bucket_expand<2><<<grid, block, 0, s>>>(kept, kept_ld, kept_count, members, bsz, sink, window, tail_block, q_pos,
+                                              idx, idx_ld, count, km);
+  else if (nmax <= 4096)
+    k_bucket_expand<4><<<grid, block, 0, s>>>(kept, kept_ld, kept_count, members, bsz, sink, window, tail_block, q_pos,
+                                              idx, idx_ld, count, km);
+  else
+    k_bucket_expand<8><<<grid, block, 0, s>>>(kept, kept_ld, kept_count, members, bsz, sink, window, tail_block, q_pos,
+                                              idx, idx_ld, count, km);
   return cuda_status(cudaGetLastError());
 }
 
