@@ -241,7 +241,7 @@ def prefill_chunk(device, l2_flush, iters: int = 3):
 class BucketStep:
     """Representative (bucket / micro-block) selection then attention: the C-ABI calls of one step of the
     micro-block (4-token blocks, top-512 + tail) or Flat (64-member buckets, top-32) variant.  The
-    representatives are built once before timing (the untimed precompute)."""
+    representatives and their bf16 split are built once before timing (the untimed precompute)."""
 
     def __init__(self, wl: S.Workload, device):
         import sparse_long_context_lightning_b200 as lsa
@@ -255,10 +255,13 @@ class BucketStep:
         self.cen = torch.empty(nb, wl.d_I, device=device)
         lsa.lsa_pool_keys(k_I, self.cen, wl.bsz, members=self.members)
         del k_I
+        # cached beside the representatives: their exact bf16 split for the tensor-core scoring
+        self.split = torch.empty(3, nb, wl.d_I, dtype=torch.bfloat16, device=device)
+        lsa.lsa_split_representatives(self.cen, self.split)
         self.q_pos = wl.q_pos().to(device)
         self.idx = torch.empty(wl.B, wl.kmax, dtype=torch.int32, device=device)
         self.cnt = torch.empty(wl.B, dtype=torch.int32, device=device)
-        self.ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_BUCKET, wl.B, nb, wl.M), device)
+        self.ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_BUCKET_MIN, wl.B, nb, wl.M), device)
         self.q = S.attn_queries(wl, device)
         self.kv = S.latent_cache(wl, device)
         self.out = torch.empty(wl.B, wl.H, wl.d_v, dtype=torch.bfloat16, device=device)
@@ -268,8 +271,8 @@ class BucketStep:
 
     def select(self):
         wl = self.wl
-        self.lsa.lsa_bucket_select(self.q_I, self.w, self.cen, self.members, wl.bsz, wl.M, wl.sink, wl.window, wl.L,
-                                   self.q_pos, self.idx, self.cnt, self.ws)
+        self.lsa.lsa_bucket_select_split(self.q_I, self.w, self.split, self.members, wl.bsz, wl.M, wl.sink, wl.window,
+                                         wl.L, self.q_pos, self.idx, self.cnt, self.ws)
 
     def attn(self):
         self.lsa.lsa_sparse_attn(self.q, self.kv, self.idx, self.cnt, self.wl.scale, self.out, self.lse, self.ws_a)
@@ -295,10 +298,6 @@ def _time_stages(stages, l2_flush, iters):
         once(evs[i])
     torch.cuda.synchronize()
     return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n)] for i in range(iters)]).mean(axis=0)
-
-
-# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1965 MHz (clocks.max.sm)
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def _stage(ms, nbytes, flops=None, peak_tflops=None, pipe="tensor"):
@@ -343,16 +342,18 @@ def long_context_configs(device, l2_flush, iters: int = 10):
         st = _time_stages([bstep.select, bstep.attn], l2_flush, iters)
         B = wl.B
         rows = float(bstep.cnt.sum().item())
-        sel_bytes = bstep.nb * wl.d_I * 4 + B * bstep.nb * 4 + B * wl.kmax * 4 + \
+        sel_bytes = bstep.nb * wl.d_I * 6 + B * bstep.nb * 4 + B * wl.kmax * 4 + \
             (B * wl.M * wl.bsz * 4 if wl.mode == "flat" else 0)
         sel_flops = 2.0 * B * wl.H_I * wl.d_I * bstep.nb
         at_bytes = rows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
-        desc = ("B=4 decode queries, L=1048576, 4-token mean-pooled blocks (fp32), top-512 blocks + tail + sink 4 + "
-                "window 128, H=128" if name == "decode1m_mb" else
-                "B=8 decode queries, L=10000000, 156250 Flat buckets of 64 (fp32 representatives), top-32 buckets + "
-                "sink 4 + window 512, H=128, 11.5 GB latent cache")
+        desc = ("B=4 decode queries, L=1048576, 4-token mean-pooled blocks (fp32, scored from their cached exact "
+                "3 x bf16 split on tensor cores), top-512 blocks + tail + sink 4 + window 128, H=128"
+                if name == "decode1m_mb" else
+                "B=8 decode queries, L=10000000, 156250 Flat buckets of 64 (fp32 representatives scored from their "
+                "cached exact 3 x bf16 split on tensor cores), top-32 buckets + sink 4 + window 512, H=128, "
+                "11.5 GB latent cache")
         res[name] = {"workload": desc,
-                     "stages": {"bucket_select": _stage(st[0], sel_bytes, sel_flops, FP32_ALU_TFLOPS, "fp32_alu"),
+                     "stages": {"bucket_select": _stage(st[0], sel_bytes, 3 * sel_flops, bf16),
                                 "attn": _stage(st[1], at_bytes)},
                      "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
         del bstep

@@ -172,6 +172,33 @@ int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, i
                       void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * lsa_split_representatives -- the exact three-part bf16 split of fp32 representatives, for
+ *   lsa_bucket_select_split: computed once with the representatives (lsa_pool_keys) and cached beside
+ *   them.  Not on the pages: a layout of the pages' representative for the tensor cores.
+ *
+ *   split[p*NB*d_I + c*d_I + d], p = 0, 1, 2, are bf16 with
+ *     centroids[c*d_I + d] = split0 + split1 + split2   exactly
+ *   (each part is the round-to-nearest bf16 of what the earlier parts leave; 8 + 8 + 8 significand bits).
+ *   centroids [NB, d_I] fp32, split bf16 [3, NB, d_I] (6*NB*d_I bytes); both 16-byte aligned; d_I % 4 == 0.
+ *   Values must not exceed the largest bf16 (about 3.39e38) in magnitude (means of bf16 keys never do);
+ *   larger ones make the first part infinite.
+ */
+int lsa_split_representatives(const float* centroids, int64_t NB, int d_I, void* split, void* stream);
+
+/*
+ * lsa_bucket_select_split -- lsa_bucket_select with the representatives given as their cached split
+ *   (lsa_split_representatives), so no per-call conversion.  Same selection rule, arguments and results
+ *   as lsa_bucket_select with its full workspace (tensor-core scoring), with `split` in place of
+ *   `centroids` (and no q_scale / dtype: q_idx is bf16).  Shapes: d_I = 128, H_I in {32, 64}, NB >= 128
+ *   (others: LSA_ERR_UNSUPPORTED).
+ *   ws: lsa_workspace_size(LSA_OP_BUCKET_MIN, B, NB, M, 0, 0, 0) bytes.
+ */
+int lsa_bucket_select_split(const void* q_idx, const float* w, int64_t B, int H_I, int d_I, const void* split,
+                            int64_t NB, const int32_t* members, int bsz, int M, int sink, int window, int64_t L,
+                            const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/*
  * lsa_bucket_select_noalloc -- lsa_bucket_select for callers that cannot allocate device memory.
  *   The pages have no counterpart: this is a packaging variant of lsa_bucket_select.
  *

@@ -36,6 +36,9 @@ SIGNATURES = {
                                  _P, _P, _I64, _P, _P, _SZ, _P]),
     "lsa_bucket_select_noalloc": (_I32, [_P, _P, _P, _I32, _I64, _I32, _I32, _P, _I64, _P, _I32, _I32, _I32, _I32,
                                          _I64, _P, _P, _I64, _P, _P]),
+    "lsa_split_representatives": (_I32, [_P, _I64, _I32, _P, _P]),
+    "lsa_bucket_select_split": (_I32, [_P, _P, _I64, _I32, _I32, _P, _I64, _P, _I32, _I32, _I32, _I32, _I64, _P, _P,
+                                       _I64, _P, _P, _SZ, _P]),
     "lsa_sparse_attn": (_I32, [_P, _P, _I64, _P, _I64, _P, _I64, _I32, _I32, _I32, _F32, _P, _P, _P, _SZ, _P]),
     "lsa_workspace_size": (_SZ, [_I32, _I64, _I64, _I32, _I32, _I32, _I32]),
     "lsa_strerror": (ctypes.c_char_p, [_I32]),
@@ -139,6 +142,23 @@ def lsa_bucket_select(q_idx, w, centroids, members, bsz, M, sink, window, L, q_p
                                           L, _ptr(q_pos), _ptr(idx), idx.stride(0), _ptr(count), _ptr(ws),
                                           0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check("lsa_bucket_select", st)
+
+
+def lsa_split_representatives(centroids, split, stream=None):
+    """split[p] (bf16 [3, NB, d_I]): centroids == split[0] + split[1] + split[2] exactly."""
+    NB, d_I = centroids.shape
+    st = load_library().lsa_split_representatives(_ptr(centroids), NB, d_I, _ptr(split), _stream(stream))
+    _check("lsa_split_representatives", st)
+
+
+def lsa_bucket_select_split(q_idx, w, split, members, bsz, M, sink, window, L, q_pos, idx, count, ws, stream=None):
+    """lsa_bucket_select from the representatives' cached bf16 split (lsa_split_representatives)."""
+    B, H_I, d_I = q_idx.shape
+    st = load_library().lsa_bucket_select_split(_ptr(q_idx), _ptr(w), B, H_I, d_I, _ptr(split), split.shape[1],
+                                                _ptr(members), bsz, M, sink, window, L, _ptr(q_pos), _ptr(idx),
+                                                idx.stride(0), _ptr(count), _ptr(ws),
+                                                0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("lsa_bucket_select_split", st)
 
 
 def lsa_bucket_select_noalloc(q_idx, w, centroids, members, bsz, M, sink, window, L, q_pos, idx, count,

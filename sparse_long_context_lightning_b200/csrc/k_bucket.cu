@@ -85,15 +85,25 @@ __global__ void __launch_bounds__(EX_THREADS) k_bucket_expand(
   const int tlo = tail_block > 0 ? ((qp + 1) / tail_block) * tail_block : qp + 1;
   const int ntail = qp + 1 - tlo;
   const int n = min(nmem + nsink + nwin + ntail, P);  // the host sizes P for the largest n
+  // kept buckets, then their members: E independent loads per round trip
+  int c[E], m[E];
+  #pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = tid * E + e;
+    c[e] = i < nmem ? kept[static_cast<int64_t>(b) * kept_ld + i / bsz] : 0;
+  }
+  #pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = tid * E + e;
+    m[e] = (i < nmem && members) ? members[static_cast<int64_t>(c[e]) * bsz + (i % bsz)] : c[e] * bsz + (i % bsz);
+  }
   int v[E];
   #pragma unroll
   for (int e = 0; e < E; ++e) {
     const int i = tid * E + e;
     int x = 0x7FFFFFFF;
     if (i < nmem) {
-      const int c = kept[static_cast<int64_t>(b) * kept_ld + i / bsz];
-      const int s = members ? members[static_cast<int64_t>(c) * bsz + (i % bsz)] : c * bsz + (i % bsz);
-      x = s <= qp ? s : 0x7FFFFFFF;
+      x = m[e] <= qp ? m[e] : 0x7FFFFFFF;
     } else if (i < nmem + nsink) {
       x = i - nmem;
     } else if (i < nmem + nsink + nwin) {

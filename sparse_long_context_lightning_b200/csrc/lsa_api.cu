@@ -162,10 +162,16 @@ int lsa_pool_keys(const void* k_idx, int dtype, const float* k_scale, int64_t L,
                           static_cast<cudaStream_t>(stream));
 }
 
-int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, int dtype, int64_t B, int H_I,
-                      int d_I, const float* centroids, int64_t NB, const int32_t* members, int bsz, int M, int sink,
-                      int window, int64_t L, const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count,
-                      void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace lsa {
+// The selection of lsa_bucket_select / lsa_bucket_select_split: representatives as fp32 `centroids` or as
+// their cached bf16 split (`split_given`, then centroids == nullptr).
+static int bucket_select_impl(const void* q_idx, const float* q_scale, const float* w, int dtype, int64_t B, int H_I,
+                              int d_I, const float* centroids, const void* split_given, int64_t NB,
+                              const int32_t* members, int bsz, int M, int sink, int window, int64_t L,
+                              const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count, void* ws,
+                              size_t ws_bytes, void* stream) {
   LSA_CHECK_ARG(B >= 0 && NB >= 1 && NB < (int64_t(1) << 31) && bsz >= 1 && M >= 1 && M <= 1024);
   LSA_CHECK_ARG(sink >= 0 && window >= 0 && L >= 1 && H_I >= 1 && H_I <= 64);
   LSA_CHECK_ARG(static_cast<int64_t>(M) * bsz + bsz + sink + window <= 8192);
@@ -174,10 +180,14 @@ int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, i
   LSA_CHECK_ARG(idx_ld >= kmax_full);
   if (dtype != LSA_BF16 || q_scale != nullptr) return LSA_ERR_UNSUPPORTED;
   if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
+  // the shapes the tensor-core scoring tiles
+  const bool tc_shape = d_I == 128 && (H_I == 32 || H_I == 64) && NB >= 128 && NB < (int64_t(1) << 29);
+  if (split_given && !tc_shape) return LSA_ERR_UNSUPPORTED;
   if (members == nullptr) LSA_CHECK_ARG(NB <= L / bsz);
   if (B == 0) return LSA_OK;
   LSA_CHECK_ARG(B <= 65535);
-  LSA_CHECK_ARG(q_idx && w && centroids && q_pos && idx && count && aligned16(centroids) && aligned16(q_idx));
+  LSA_CHECK_ARG(q_idx && w && (centroids || split_given) && q_pos && idx && count && aligned16(q_idx));
+  LSA_CHECK_ARG(centroids ? aligned16(centroids) : aligned16(split_given));
   size_t off_kept, off_cnt, off_split, total_min, total;
   int64_t ldn;
   bucket_ws_layout(B, NB, M, &off_kept, &off_cnt, &off_split, &total_min, &total, &ldn);
@@ -187,10 +197,11 @@ int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, i
   float* bscores = reinterpret_cast<float*>(base);
   int32_t* kept = reinterpret_cast<int32_t*>(base + off_kept);
   int32_t* kcnt = reinterpret_cast<int32_t*>(base + off_cnt);
-  // tensor cores when the workspace holds the split and the shape is the tensor-core indexer's
-  const bool tc = ws_bytes >= total && d_I == 128 && (H_I == 32 || H_I == 64) && NB >= 128 && NB < (int64_t(1) << 29);
   int st;
-  if (tc) {
+  if (split_given) {
+    st = launch_centroid_score_tc(q_idx, w, split_given, B, H_I, NB, bscores, ldn, s);
+  } else if (tc_shape && ws_bytes >= total) {
+    // tensor cores when the workspace holds the split
     void* split = base + off_split;
     st = launch_split_bf16x3(centroids, NB * 128, split, s);
     if (st == LSA_OK) st = launch_centroid_score_tc(q_idx, w, split, B, H_I, NB, bscores, ldn, s);
@@ -204,6 +215,34 @@ int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, i
   // rows are -1 padded up to idx_ld
   return launch_bucket_expand(kept, M, kcnt, members, bsz, sink, window, members ? 0 : bsz, q_pos, B, idx, idx_ld,
                               count, idx_ld, s);
+}
+}  // namespace lsa
+
+extern "C" {
+
+int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, int dtype, int64_t B, int H_I,
+                      int d_I, const float* centroids, int64_t NB, const int32_t* members, int bsz, int M, int sink,
+                      int window, int64_t L, const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count,
+                      void* ws, size_t ws_bytes, void* stream) {
+  if (centroids == nullptr && B > 0) return LSA_ERR_INVALID_ARG;
+  return bucket_select_impl(q_idx, q_scale, w, dtype, B, H_I, d_I, centroids, nullptr, NB, members, bsz, M, sink,
+                            window, L, q_pos, idx, idx_ld, count, ws, ws_bytes, stream);
+}
+
+int lsa_bucket_select_split(const void* q_idx, const float* w, int64_t B, int H_I, int d_I, const void* split,
+                            int64_t NB, const int32_t* members, int bsz, int M, int sink, int window, int64_t L,
+                            const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count, void* ws,
+                            size_t ws_bytes, void* stream) {
+  if (split == nullptr && B > 0) return LSA_ERR_INVALID_ARG;
+  return bucket_select_impl(q_idx, nullptr, w, LSA_BF16, B, H_I, d_I, nullptr, split, NB, members, bsz, M, sink,
+                            window, L, q_pos, idx, idx_ld, count, ws, ws_bytes, stream);
+}
+
+int lsa_split_representatives(const float* centroids, int64_t NB, int d_I, void* split, void* stream) {
+  LSA_CHECK_ARG(NB >= 0 && d_I >= 4 && (d_I % 4) == 0);
+  if (NB == 0) return LSA_OK;
+  LSA_CHECK_ARG(centroids && split && aligned16(centroids) && aligned16(split));
+  return launch_split_bf16x3(centroids, NB * d_I, split, static_cast<cudaStream_t>(stream));
 }
 
 int lsa_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,

@@ -171,7 +171,9 @@ def test_pool_keys(fp8):
 # --------------------------------------------------------------------------------------------
 
 
-def _bucket_case(L, B, M, bsz, sink, window, flat, tie_check=True):
+def _bucket_case(L, B, M, bsz, sink, window, flat, tie_check=True, path="full"):
+    """path: "full" workspace (tensor-core scoring of the split representatives where the shape allows),
+    "min" workspace (CUDA-core scoring), or "split" (lsa_bucket_select_split from a cached split)."""
     wl = S.Workload("bk", L=L, B=B, H_I=64, d_I=128, K=M * bsz, H=16, sink=sink, window=window,
                     mode="flat" if flat else "microblock", bsz=bsz, M=M)
     q_I, w = S.index_queries(wl)
@@ -190,8 +192,16 @@ def _bucket_case(L, B, M, bsz, sink, window, flat, tie_check=True):
     kmax = M * bsz + (bsz - 1) + sink + window
     idx = torch.full((B, kmax), 777, dtype=torch.int32, device=DEV)
     cnt = torch.empty(B, dtype=torch.int32, device=DEV)
-    ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_BUCKET, B, nb, M))
-    lsa.lsa_bucket_select(q_I.to(DEV), w.to(DEV), cen, members, bsz, M, sink, window, L, qp.to(DEV), idx, cnt, ws)
+    if path == "split":
+        split = torch.empty(3, nb, 128, dtype=torch.bfloat16, device=DEV)
+        lsa.lsa_split_representatives(cen, split)
+        ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_BUCKET_MIN, B, nb, M))
+        lsa.lsa_bucket_select_split(q_I.to(DEV), w.to(DEV), split, members, bsz, M, sink, window, L, qp.to(DEV), idx,
+                                    cnt, ws)
+    else:
+        op = lsa.LSA_OP_BUCKET if path == "full" else lsa.LSA_OP_BUCKET_MIN
+        ws = lsa.workspace(lsa.lsa_workspace_size(op, B, nb, M))
+        lsa.lsa_bucket_select(q_I.to(DEV), w.to(DEV), cen, members, bsz, M, sink, window, L, qp.to(DEV), idx, cnt, ws)
     torch.cuda.synchronize()
     kf = f64(k)
     mem_np = members.cpu().numpy() if flat else None
@@ -223,8 +233,31 @@ def test_microblock_select(tail):
     _bucket_case(L=4 * 16384 + tail, B=4, M=512, bsz=4, sink=4, window=128, flat=False)
 
 
-def test_flat_bucket_select():
-    _bucket_case(L=64 * 10000, B=8, M=32, bsz=64, sink=4, window=512, flat=True)
+@pytest.mark.parametrize("path", ["full", "min", "split"])
+def test_flat_bucket_select(path):
+    _bucket_case(L=64 * 10000, B=8, M=32, bsz=64, sink=4, window=512, flat=True, path=path)
+
+
+@pytest.mark.parametrize("path", ["min", "split"])
+def test_microblock_select_paths(path):
+    _bucket_case(L=4 * 16384 + 3, B=4, M=512, bsz=4, sink=4, window=128, flat=False, path=path)
+
+
+def test_split_representatives_exact():
+    """The three bf16 parts sum exactly (in fp64) to the fp32 representative, across magnitudes and signs."""
+    g = torch.Generator().manual_seed(5)
+    mant = torch.rand(4096, 128, generator=g) * 2 - 1
+    expo = torch.randint(-40, 40, (4096, 128), generator=g).float()
+    cen = (mant * torch.pow(2.0, expo)).float()
+    # up to the largest bf16 (about 3.39e38); fp32 values beyond it overflow the first part
+    cen[0, :8] = torch.tensor([0.0, -0.0, 1.0, -1.0, 3.0e38, -3.0e38, 1.17549435e-38, 2.0 ** -100])
+    cen_d = cen.to(DEV)
+    split = torch.empty(3, 4096, 128, dtype=torch.bfloat16, device=DEV)
+    lsa.lsa_split_representatives(cen_d, split)
+    parts = split.float().double().cpu()
+    assert torch.equal(parts.sum(0), cen.double())
+    # each part is the bf16 rounding of what the earlier parts leave
+    assert torch.equal(split[0].float().cpu(), cen.bfloat16().float())
 
 
 def test_microblock_small_rows():
