@@ -139,6 +139,7 @@ __device__ __forceinline__ RowSetup row_setup(const TopkArgs& a, int b, int r, i
 // positions c0 + 4g .. c0 + 4g + 3; an element is valid when its position is in [a0, a1).
 struct Chunk {
   const float* grow;  // the score row in global memory
+  bool vec;           // grow + c0 is 16-byte aligned
   const uint4* keys;  // the chunk's order keys in shared memory (0 = invalid), or nullptr
   int c0, a0, a1;
   __device__ __forceinline__ uint4 from_scores(int g, float4 v) const {
@@ -160,6 +161,8 @@ struct Chunk {
   // the group's scores straight from global memory (0 outside [a0, a1))
   __device__ __forceinline__ float4 gload(int g) const {
     const int s0 = c0 + 4 * g;
+    // whole group in range of a 16-byte aligned row: one 16-byte load (chunks start at multiples of 4)
+    if (vec && s0 >= a0 && s0 + 4 <= a1) return __ldg(reinterpret_cast<const float4*>(grow + s0));
     float4 v;
     v.x = (s0 >= a0 && s0 < a1) ? __ldg(grow + s0) : 0.f;
     v.y = (s0 + 1 >= a0 && s0 + 1 < a1) ? __ldg(grow + s0 + 1) : 0.f;
@@ -260,6 +263,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
   Chunk ch;
   ch.grow = a.scores + static_cast<int64_t>(b) * a.ld;
   ch.keys = nullptr;
+  ch.vec = (reinterpret_cast<uintptr_t>(ch.grow + c0) & 15u) == 0;
   ch.c0 = c0;
   ch.a0 = a0;
   ch.a1 = a1;
@@ -668,14 +672,15 @@ int launch_topk_mode(const float* scores, int64_t ld, int64_t B, int64_t L, int 
       if (dev >= 0 && dev < 64) set[dev] = true;
     }
   }
-  // Cluster size: among the sizes whose chunk fits the shared-memory cache, the one with the least work
-  // on the busiest SM -- (chunk + a fixed per-CTA cost) x the number of cluster waves the batch needs.
-  // Rows too long for any cluster's cache are streamed from global memory by clusters of 16.
+  // Cluster size: the one with the least work on the busiest SM -- (chunk + a fixed per-CTA cost) x the
+  // number of cluster waves the batch needs.  A chunk larger than the shared-memory cache is streamed from
+  // global memory (L2) on every pass; measured per element that costs about what the cached passes do,
+  // while smaller clusters save the barriers, so many rows (a prefill chunk: 8192 x 131072) run one CTA
+  // per row (5.9 ms against 7.8 ms for 6-CTA clusters) and a few long rows use large clusters.
   int C = TK_MAXC;
   double best = -1.0;
   for (int c = 1; c <= TK_MAXC; ++c) {
     const int64_t chunk = (cdiv(L, c) + 3) / 4 * 4;
-    if (chunk > TK_CACHE) continue;
     const double waves = static_cast<double>(cdiv(B, resident_clusters(c)));
     const double cost = (static_cast<double>(chunk) + 2048.0) * waves;
     if (best < 0.0 || cost < best) {
