@@ -32,6 +32,7 @@ constexpr int TK_CAP = 1024;   // boundary-bin size that is all-gathered and fin
 constexpr int TK_MAXC = 16;    // cluster size limit (non-portable above 8)
 constexpr int TK_CACHE = 24576;  // scores per CTA kept in shared memory (96 KB)
 constexpr int TK_PIECES = 4;     // the chunk arrives in this many bulk copies; each warp waits for its own
+constexpr int TK_UNROLL = 4;     // groups per lane whose loads are in flight together in a pass
 
 enum { MODE_TOKEN = 0, MODE_ALL = 1, MODE_BLOCKS = 2 };
 
@@ -174,7 +175,47 @@ struct Chunk {
     if (keys) return keys[g];
     return from_scores(g, gload(g));
   }
+  // groups g0 + 32u (u < TK_UNROLL) of one lane, all loads issued before any is used (a streamed chunk
+  // comes from L2: one load in flight per thread would leave the pass latency-bound); 0 keys past gend
+  __device__ __forceinline__ void load_batch(int g0, int gend, uint4 (&k)[TK_UNROLL]) const {
+    if (keys) {
+      #pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int g = g0 + 32 * u;
+        k[u] = g < gend ? keys[g] : make_uint4(0u, 0u, 0u, 0u);
+      }
+    } else {
+      float4 v[TK_UNROLL];
+      #pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int g = g0 + 32 * u;
+        v[u] = g < gend ? gload(g) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      #pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int g = g0 + 32 * u;
+        k[u] = g < gend ? from_scores(g, v[u]) : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  }
 };
+
+// f(keys of group g) for this lane's groups gw0 + lane, +32, ... < gw1: one at a time from the shared-memory
+// cache, or TK_UNROLL at a time (loads in flight together) when the chunk is streamed from global memory.
+template <bool STREAMED, class F>
+__device__ __forceinline__ void for_groups(const Chunk& ch, int gw0, int gw1, int lane, F&& f) {
+  if (!STREAMED) {
+    for (int g = gw0 + lane; g < gw1; g += 32) f(ch.keys[g]);
+  } else {
+    for (int g0 = gw0 + lane; g0 < gw1; g0 += 32 * TK_UNROLL) {
+      uint4 kb[TK_UNROLL];
+      ch.load_batch(g0, gw1, kb);
+      #pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u)
+        if (g0 + 32 * u < gw1) f(kb[u]);
+    }
+  }
+}
 
 // Boundary bin of hist[] (bins ascend with the key): the bin holding the need-th largest element.
 // Warp 0 only; lane l scans bins [8l, 8l + 8).  Writes sel_bin / sel_above / sel_count.
@@ -228,6 +269,10 @@ __device__ __forceinline__ uint32_t ballot_prefix(uint32_t v, uint32_t lt, uint3
   return __popc(b0 & lt) + 2u * __popc(b1 & lt) + 4u * __popc(b2 & lt);
 }
 
+// STREAMED: the chunk exceeds the shared-memory cache (a.cached == 0) and every pass reads it from global
+// memory; otherwise it is cached (a.cached == 1).  Two instantiations keep the cached passes' code free of the
+// streamed ones' load batching.
+template <bool STREAMED>
 __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
   // every global access of this kernel comes after the previous kernel of the stream has completed
   sm100::pdl_wait();
@@ -310,16 +355,18 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
   // ---- order keys (in place, when cached) and the finite key range of the candidates ----
   {
     uint32_t lo1 = 0xFFFFFFFFu, hi = 0u;  // lo1 = min(key) - 1 over valid keys (invalid: 0 - 1 = max)
-    for (int g = gw0 + lane; g < gw1; g += 32) {
-      uint4 k;
-      if (a.cached) {
-        k = ch.from_scores(g, g < nvec ? cache[g] : ch.gload(g));
+    if (a.cached) {
+      for (int g = gw0 + lane; g < gw1; g += 32) {
+        const uint4 k = ch.from_scores(g, g < nvec ? cache[g] : ch.gload(g));
         reinterpret_cast<uint4*>(cache)[g] = k;
-      } else {
-        k = ch.load(g);
+        lo1 = min(min(lo1, k.x - 1u), min(k.y - 1u, min(k.z - 1u, k.w - 1u)));
+        hi = max(max(hi, k.x), max(k.y, max(k.z, k.w)));
       }
-      lo1 = min(min(lo1, k.x - 1u), min(k.y - 1u, min(k.z - 1u, k.w - 1u)));
-      hi = max(max(hi, k.x), max(k.y, max(k.z, k.w)));
+    } else {
+      for_groups<STREAMED>(ch, gw0, gw1, lane, [&](const uint4 k) {
+        lo1 = min(min(lo1, k.x - 1u), min(k.y - 1u, min(k.z - 1u, k.w - 1u)));
+        hi = max(max(hi, k.x), max(k.y, max(k.z, k.w)));
+      });
     }
     if (a.cached) ch.keys = reinterpret_cast<const uint4*>(cache);  // each thread reads back only its own groups
     uint32_t lo = lo1 + 1u;  // 0 when this thread saw no valid key
@@ -392,8 +439,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     uint32_t* hl = hall + (level & 1) * C * TK_BINS;
     if (tid < TK_BINS) sm.h[tid] = 0;
     __syncthreads();
-    for (int g = gw0 + lane; g < gw1; g += 32) {
-      const uint4 k4 = ch.load(g);
+    for_groups<STREAMED>(ch, gw0, gw1, lane, [&](const uint4 k4) {
       const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
       #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -403,7 +449,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
           atomicAdd(&sm.h[(k[e] - klo) >> shift], 1u);
         }
       }
-    }
+    });
     __syncthreads();
     for (int i = tid; i < TK_BINS * C; i += TK_THREADS) {
       const int c = i / TK_BINS, bin = i - c * TK_BINS;
@@ -454,8 +500,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     }
     const uint32_t off = gather ? sm.segoff[r] : 0u;
     uint32_t nab = 0, nin = 0;
-    for (int g = gw0 + lane; g < gw1; g += 32) {
-      const uint4 k4 = ch.load(g);
+    for_groups<STREAMED>(ch, gw0, gw1, lane, [&](const uint4 k4) {
       const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
       #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -470,7 +515,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
           }
         }
       }
-    }
+    });
     nab = warp_sum_u32(nab);
     nin = warp_sum_u32(nin);
     if (lane == 0) {
@@ -576,10 +621,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
   // ---- ordered write: a selected element's slot = base + (#gt before it) + min(#eq before it, take) ----
   const uint32_t lim = static_cast<uint32_t>(rs.nsink + rs.nsel);
   const uint32_t lt = lanemask_lt();
-  for (int g0 = gw0; g0 < gw1; g0 += 32) {
-    const int g = g0 + lane;
-    uint4 k4 = make_uint4(0u, 0u, 0u, 0u);
-    if (g < gw1) k4 = ch.load(g);
+  // one warp-wide step: groups g = (step base) + lane, warp-uniform control flow (ballots)
+  auto step = [&](const int g, const uint4 k4) {
     const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
     uint32_t ngt = 0, neq = 0;
     #pragma unroll
@@ -618,9 +661,22 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     }
     gt_run += gtot;
     eq_run += etot;
+  };
+  if (!STREAMED) {
+    for (int g0 = gw0; g0 < gw1; g0 += 32) {
+      const int g = g0 + lane;
+      step(g, g < gw1 ? ch.keys[g] : make_uint4(0u, 0u, 0u, 0u));
+    }
+  } else {
+    for (int gb0 = gw0; gb0 < gw1; gb0 += 32 * TK_UNROLL) {
+      uint4 kb[TK_UNROLL];
+      ch.load_batch(gb0 + lane, gw1, kb);  // 0 keys past the end, as in every step
+      #pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u)  // steps of 32 groups, in order
+        if (gb0 + 32 * u < gw1) step(gb0 + 32 * u + lane, kb[u]);
+    }
   }
 }
-
 // Clusters of C CTAs (one CTA per SM) that can be resident at once on the current device.
 int resident_clusters(int C) {
   static std::mutex mu;
@@ -642,7 +698,7 @@ int resident_clusters(int C) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, k_topk_cluster, &cfg) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, k_topk_cluster<false>, &cfg) != cudaSuccess || n < 1) {
       cudaGetLastError();
       n = 1;
     }
@@ -666,9 +722,12 @@ int launch_topk_mode(const float* scores, int64_t ld, int64_t B, int64_t L, int 
     LSA_CUDA_TRY(cudaGetDevice(&dev));
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= 64 || !set[dev]) {
-      LSA_CUDA_TRY(cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        2 * TK_MAXC * TK_BINS * 4 + TK_CACHE * 4));
-      LSA_CUDA_TRY(cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+      for (const void* f : {reinterpret_cast<const void*>(k_topk_cluster<false>),
+                            reinterpret_cast<const void*>(k_topk_cluster<true>)}) {
+        LSA_CUDA_TRY(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          2 * TK_MAXC * TK_BINS * 4 + TK_CACHE * 4));
+        LSA_CUDA_TRY(cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+      }
       if (dev >= 0 && dev < 64) set[dev] = true;
     }
   }
@@ -708,8 +767,8 @@ int launch_topk_mode(const float* scores, int64_t ld, int64_t B, int64_t L, int 
   a.cached = chunk <= TK_CACHE ? 1 : 0;
   // all-gathered histograms (two levels' worth), then the cached chunk
   const size_t dyn = static_cast<size_t>(2 * C * TK_BINS) * 4 + (a.cached ? static_cast<size_t>(chunk) * 4 : 0);
-  LSA_CUDA_TRY(launch_pdl(k_topk_cluster, dim3(C, static_cast<unsigned>(B), 1), dim3(TK_THREADS), dyn, s,
-                          static_cast<unsigned>(C), a));
+  LSA_CUDA_TRY(launch_pdl(a.cached ? k_topk_cluster<false> : k_topk_cluster<true>,
+                          dim3(C, static_cast<unsigned>(B), 1), dim3(TK_THREADS), dyn, s, static_cast<unsigned>(C), a));
   return LSA_OK;
 }
 
