@@ -22,12 +22,14 @@ primitives (matmul, stable sort, exp, log) as steps and no blocking or fusion:
                       expands to positions, adds sink and window); lecture §"Qwen Sparse
                       Attention" and §"尾部计数与 query 自身" (complete micro-blocks are ranked,
                       visible tokens of the incomplete tail block are read directly).
+* ``hi_select_row``   LongCat page §"机制三：层级索引（HI）": page scores from the sub-blocks' mean
+                      keys, top-M pages, then the token score and arg topK on the recalled tokens.
 * ``softmax_attention`` / ``sparse_mla_attn``
                       LongCat page §"DSA 基线", u_t = Attn(h_t, {c_s | s in S_t}) in the absorbed
                       MQA form (one latent c_s shared by all heads; value = first 512 dims);
                       "LSA 稀疏注意力會省顯存嗎" §四 (score q.k/sqrt(d), softmax, weighted V).
 
-Readings where the pages are silent (also listed in the design doc):
+Readings where the pages are silent:
   positions are 0-based; the window includes the query position itself; K counts
   only the dynamic part; ties at the K-th score go to the lower position / bucket
   id; fewer candidates than K means all are taken; an empty set gives output 0 and
@@ -192,6 +194,60 @@ def bucket_select_row(bscore_row: np.ndarray, q_pos: int, M: int, sink: int, win
     sel = np.unique(np.concatenate([s_sink, pos, tail, s_swa]))
     sel = sel[(sel >= 0) & (sel <= q_pos)]
     return sel.astype(np.int64), mth, int(nrank)
+
+
+# ---------------------------------------------------------------------------
+# HI: two-stage (page -> token) selection
+# ---------------------------------------------------------------------------
+
+
+def hi_select_row(q_I_b: np.ndarray, w_b: np.ndarray, k_I: np.ndarray, q_pos: int, P: int, Bsub: int, M: int,
+                  K: int, sink: int, window: int):
+    """One query of the hierarchical index: (sorted positions, K-th token score, M-th page score, recalled).
+
+    LongCat page §"机制三：层级索引（HI）".  Stage one: the sequence is cut into pages of P tokens and
+    sub-blocks of Bsub tokens; each sub-block n keeps the mean of its index keys; the page score is
+    I_page(p) = sum_j w_j sum_{n in page p} ReLU(q_j . kmean_n); the M best pages among p <= q_pos/P
+    (0-based: pages that start at or before the query) are recalled (stable sort on descending score:
+    ties -> lower page id).  Stage two: the token score I_{t,s} (the indexer formula) on the recalled
+    tokens only, and the same sink / window union and arg topK as ``topk_row`` over them.
+
+    Readings: a page's score sums its complete sub-blocks that are entirely visible (end <= q_pos);
+    the visible tokens of the sub-block holding q_pos that is not entirely visible, i.e.
+    {Bsub*floor((q_pos+1)/Bsub) .. q_pos}, have no mean key and join the recalled tokens directly (as
+    the micro-block tail).  Recalled tokens are clipped to [0, q_pos].
+    """
+    q_pos = int(q_pos)
+    k_I = np.asarray(k_I, dtype=np.float64)
+    L = k_I.shape[0]
+    # stage one: sub-block means and their indexer scores, summed per page
+    nvis = min(L // Bsub, (q_pos + 1) // Bsub)  # complete sub-blocks entirely visible
+    kmean = pool_keys(k_I, block=Bsub)[:nvis]
+    sub = bucket_scores(np.asarray(q_I_b, np.float64)[None], np.asarray(w_b, np.float64)[None], kmean)[0]
+    per_page = P // Bsub
+    npages = q_pos // P + 1
+    page = np.zeros(npages)
+    for p in range(npages):
+        page[p] = sub[p * per_page: min((p + 1) * per_page, nvis)].sum()
+    order = np.argsort(-page, kind="stable")
+    chosen = order[: min(M, npages)]
+    mth_page = float(page[chosen[-1]]) if chosen.size else -np.inf
+    recalled = (chosen[:, None] * P + np.arange(P)[None, :]).reshape(-1)
+    tail = np.arange(((q_pos + 1) // Bsub) * Bsub, q_pos + 1)
+    recalled = np.union1d(recalled, tail).astype(np.int64)
+    recalled = recalled[recalled <= q_pos]
+    # stage two: token scores on the recalled tokens, sink / window union, arg topK
+    scores = index_score(np.asarray(q_I_b)[None], np.asarray(w_b)[None], k_I[recalled],
+                         np.array([len(recalled) - 1]))[0]
+    s_sink, s_swa = fixed_positions(q_pos, sink, window)
+    fixed = np.union1d(s_sink, s_swa)
+    keep = ~np.isin(recalled, fixed)
+    cand, cand_sc = recalled[keep], scores[keep]
+    order = np.argsort(-cand_sc, kind="stable")
+    take = cand[order[: min(K, cand.size)]]
+    kth = float(cand_sc[order[min(K, cand.size) - 1]]) if cand.size else -np.inf
+    sel = np.union1d(np.union1d(s_sink, take), s_swa)
+    return sel.astype(np.int64), kth, mth_page, recalled
 
 
 # ---------------------------------------------------------------------------

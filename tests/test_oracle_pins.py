@@ -331,3 +331,79 @@ def test_attention_shift_invariance_of_logits():
     o2, lse2 = O.softmax_attention(qb, big, kv[:, :3], 1.0)
     np.testing.assert_allclose(o1, o2, rtol=1e-10)
     np.testing.assert_allclose(lse2 - lse1, 1000.0, rtol=1e-12)
+
+
+# --------------------------------------------------------------------------------------------
+# HI two-stage selection (LongCat page, section on hierarchical indexing)
+# --------------------------------------------------------------------------------------------
+
+
+def _hi_inputs(seed, L, H=4, d=16):
+    rng = np.random.default_rng(seed)
+    return rng.normal(size=(H, d)), rng.uniform(0.1, 1.0, size=H) * rng.choice([-1.0, 1.0], size=H), \
+        rng.normal(size=(L, d))
+
+
+@pytest.mark.parametrize("L,q_pos", [(300, 299), (300, 170), (257, 256)])
+def test_hi_equals_flat_when_every_page_is_recalled(L, q_pos):
+    """M * P >= L: stage one recalls every visible token, so HI is the flat token top-K."""
+    q, w, k = _hi_inputs(1, L)
+    sel, kth, _, recalled = O.hi_select_row(q, w, k, q_pos, P=32, Bsub=8, M=64, K=20, sink=2, window=8)
+    assert np.array_equal(recalled, np.arange(q_pos + 1))
+    flat = O.index_score(q[None], w[None], k, np.array([q_pos]))[0]
+    want, want_kth, _ = O.topk_row(flat, q_pos, 20, 2, 8)
+    assert np.array_equal(sel, want) and kth == want_kth
+
+
+def test_hi_pages_of_one_subblock_are_the_microblock_ranking():
+    """P == Bsub: a page is one sub-block, so stage one is the micro-block ranking (tail rule included)."""
+    q, w, k = _hi_inputs(2, 203)
+    q_pos = 202
+    _, _, mth, recalled = O.hi_select_row(q, w, k, q_pos, P=4, Bsub=4, M=7, K=5, sink=0, window=0)
+    reps = O.pool_keys(k, block=4)
+    bs = O.bucket_scores(q[None], w[None], reps)[0]
+    want, want_mth, _ = O.bucket_select_row(bs, q_pos, 7, 0, 0, block=4)
+    assert np.array_equal(recalled, want) and mth == want_mth
+
+
+def test_hi_brute_force_tiny():
+    """Loops over the definition, written independently of the oracle's array code."""
+    L, P, Bs, M, K, sink, window, q_pos = 50, 8, 4, 2, 5, 1, 3, 45
+    q, w, k = _hi_inputs(3, L, H=3, d=5)
+
+    def tok(s):
+        return sum(w[j] * max(0.0, sum(q[j][d] * k[s][d] for d in range(5))) for j in range(3))
+
+    def mean_key(n):
+        return [sum(k[n * Bs + i][d] for i in range(Bs)) / Bs for d in range(5)]
+
+    page_score = {}
+    for p in range(q_pos // P + 1):
+        tot = 0.0
+        for n in range(p * P // Bs, (p + 1) * P // Bs):
+            if n * Bs + Bs - 1 <= q_pos:  # entirely visible complete sub-block
+                km = mean_key(n)
+                tot += sum(w[j] * max(0.0, sum(q[j][d] * km[d] for d in range(5))) for j in range(3))
+        page_score[p] = tot
+    pages = sorted(page_score, key=lambda p: (-page_score[p], p))[:M]
+    recalled = {p * P + i for p in pages for i in range(P)} | set(range((q_pos + 1) // Bs * Bs, q_pos + 1))
+    recalled = sorted(s for s in recalled if s <= q_pos)
+    fixed = set(range(min(sink, q_pos + 1))) | set(range(q_pos - window + 1, q_pos + 1))
+    cand = [s for s in recalled if s not in fixed]
+    take = sorted(cand, key=lambda s: (-tok(s), s))[:K]
+    want = sorted(fixed | set(take))
+    sel, _, _, rec = O.hi_select_row(q, w, k, q_pos, P, Bs, M, K, sink, window)
+    assert rec.tolist() == recalled
+    assert sel.tolist() == want
+
+
+def test_hi_is_causal():
+    """Keys after the query position change neither stage."""
+    q, w, k = _hi_inputs(4, 400)
+    q_pos = 233
+    a = O.hi_select_row(q, w, k, q_pos, P=16, Bsub=8, M=5, K=12, sink=2, window=4)
+    k2 = k.copy()
+    k2[q_pos + 1:] = np.random.default_rng(9).normal(size=k2[q_pos + 1:].shape) * 10
+    b = O.hi_select_row(q, w, k2, q_pos, P=16, Bsub=8, M=5, K=12, sink=2, window=4)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[3], b[3]) and a[2] == b[2]
+    assert a[3].max() <= q_pos
