@@ -199,6 +199,38 @@ int lsa_bucket_select_split(const void* q_idx, const float* w, int64_t B, int H_
                             void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * lsa_hi_select -- hierarchical (two-stage) selection: pages, then tokens.
+ *   Source: "LongCat Sparse Attention（LSA）完全拆解", section "机制三：层级索引（HI）": pages of P tokens,
+ *   sub-blocks of Bsub tokens with cached mean index keys; page score
+ *     I_page(b, p) = sum_j w[b,j] sum_{n in page p} max(0, q[b,j,:] . kmean_n);
+ *   the M best pages are recalled; the token score I(b, s) (lsa_index_score's formula) then runs on the
+ *   recalled tokens only, with lsa_topk_select's sink / window union and arg topK over them.
+ *
+ *   For each query b (q_pos[b] < L):
+ *     ranked pages = p with p*P <= q_pos[b]; a page's score sums its complete sub-blocks that end at or
+ *                    before q_pos[b] (fp32 sums of fp32-accurate sub-block scores); ties -> lower page
+ *     recalled     = tokens of the min(M, #ranked) best pages, plus the visible tokens
+ *                    {Bsub*floor((q_pos+1)/Bsub) .. q_pos} of the sub-block holding q_pos when that
+ *                    sub-block is not entirely visible (it has no mean key), clipped to [0, q_pos]
+ *     idx row      = sink, the min(K, #recalled outside sink u window) recalled tokens with the largest
+ *                    I(b, s) (fp32 from bf16; ties -> lower position), window; ascending; -1 padded up to
+ *                    K + sink + window (lsa_topk_select's row layout).
+ *   q_idx [B, H_I, 128] bf16, w [B, H_I] fp32, k_idx [L, 128] bf16 (the token keys), sub_split = the exact
+ *   bf16 split (lsa_split_representatives) of the sub-block means lsa_pool_keys(k_idx, Bsub) gives:
+ *   bf16 [3, floor(L/Bsub), 128].  H_I in {32, 64}; floor(L/Bsub) >= 128 (else LSA_ERR_UNSUPPORTED).
+ *   P % Bsub == 0, 1 <= M <= 1024.  idx int32 [B, idx_ld], idx_ld >= K + sink + window; count int32 [B].
+ *   ws: lsa_hi_workspace_size(B, L, P, Bsub, M, K, sink, window) bytes.
+ *   With M*P >= L every visible token is recalled and the result is lsa_index_score + lsa_topk_select's.
+ */
+int lsa_hi_select(const void* q_idx, const float* w, const void* k_idx, int64_t B, int H_I, int d_I,
+                  int64_t L, const void* sub_split, int P, int Bsub, int M, int K, int sink, int window,
+                  const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count,
+                  void* ws, size_t ws_bytes, void* stream);
+
+/* lsa_hi_workspace_size -- scratch bytes of lsa_hi_select; (size_t)-1 for invalid sizes. */
+size_t lsa_hi_workspace_size(int64_t B, int64_t L, int P, int Bsub, int M, int K, int sink, int window);
+
+/*
  * lsa_bucket_select_noalloc -- lsa_bucket_select for callers that cannot allocate device memory.
  *   The pages have no counterpart: this is a packaging variant of lsa_bucket_select.
  *

@@ -39,6 +39,9 @@ SIGNATURES = {
     "lsa_split_representatives": (_I32, [_P, _I64, _I32, _P, _P]),
     "lsa_bucket_select_split": (_I32, [_P, _P, _I64, _I32, _I32, _P, _I64, _P, _I32, _I32, _I32, _I32, _I64, _P, _P,
                                        _I64, _P, _P, _SZ, _P]),
+    "lsa_hi_select": (_I32, [_P, _P, _P, _I64, _I32, _I32, _I64, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P, _I64,
+                             _P, _P, _SZ, _P]),
+    "lsa_hi_workspace_size": (_SZ, [_I64, _I64, _I32, _I32, _I32, _I32, _I32, _I32]),
     "lsa_sparse_attn": (_I32, [_P, _P, _I64, _P, _I64, _P, _I64, _I32, _I32, _I32, _F32, _P, _P, _P, _SZ, _P]),
     "lsa_workspace_size": (_SZ, [_I32, _I64, _I64, _I32, _I32, _I32, _I32]),
     "lsa_strerror": (ctypes.c_char_p, [_I32]),
@@ -159,6 +162,20 @@ def lsa_bucket_select_split(q_idx, w, split, members, bsz, M, sink, window, L, q
                                                 idx.stride(0), _ptr(count), _ptr(ws),
                                                 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check("lsa_bucket_select_split", st)
+
+
+def lsa_hi_workspace_size(B, L, P, Bsub, M, K, sink, window):
+    return load_library().lsa_hi_workspace_size(B, L, P, Bsub, M, K, sink, window)
+
+
+def lsa_hi_select(q_idx, w, k_idx, sub_split, P, Bsub, M, K, sink, window, q_pos, idx, count, ws, stream=None):
+    """Two-stage selection: top-M pages from the sub-block means' split, then token top-K on their tokens."""
+    B, H_I, d_I = q_idx.shape
+    L = k_idx.shape[0]
+    st = load_library().lsa_hi_select(_ptr(q_idx), _ptr(w), _ptr(k_idx), B, H_I, d_I, L, _ptr(sub_split), P, Bsub, M,
+                                      K, sink, window, _ptr(q_pos), _ptr(idx), idx.stride(0), _ptr(count), _ptr(ws),
+                                      0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("lsa_hi_select", st)
 
 
 def lsa_bucket_select_noalloc(q_idx, w, centroids, members, bsz, M, sink, window, L, q_pos, idx, count,

@@ -56,6 +56,36 @@ size_t bucket_ws_min_bytes(int64_t B, int64_t NB, int M) {
   return mn;
 }
 
+// Scratch layout of lsa_hi_select: sub-block scores [B, ld_sub] fp32 | page scores [B, ld_pg] fp32 |
+// kept pages [B, M] int32 | kept count [B] | candidate rows [B, cand_ld] int32 | candidate count [B] |
+// the re-rank's own scratch.
+struct HiLayout {
+  int64_t nsub, npages, ld_sub, ld_pg, cand_ld;
+  size_t o_page, o_kept, o_kcnt, o_cand, o_ccnt, o_ref, total;
+};
+static HiLayout hi_ws_layout(int64_t B, int64_t L, int P, int Bsub, int M, int K, int sink, int window) {
+  HiLayout h;
+  h.nsub = L / Bsub;
+  h.npages = cdiv(L, P);
+  h.ld_sub = (h.nsub + 3) / 4 * 4;
+  h.ld_pg = (h.npages + 3) / 4 * 4;
+  h.cand_ld = static_cast<int64_t>(M) * P + (Bsub - 1) + sink + window;
+  size_t o = align_up(static_cast<size_t>(B) * h.ld_sub * 4, 256);
+  h.o_page = o;
+  o = align_up(o + static_cast<size_t>(B) * h.ld_pg * 4, 256);
+  h.o_kept = o;
+  o = align_up(o + static_cast<size_t>(B) * M * 4, 256);
+  h.o_kcnt = o;
+  o = align_up(o + static_cast<size_t>(B) * 4, 256);
+  h.o_cand = o;
+  o = align_up(o + static_cast<size_t>(B) * h.cand_ld * 4, 256);
+  h.o_ccnt = o;
+  o = align_up(o + static_cast<size_t>(B) * 4, 256);
+  h.o_ref = o;
+  h.total = o + refine_ws_bytes(B, h.cand_ld, K);
+  return h;
+}
+
 }  // namespace lsa
 
 using namespace lsa;
@@ -243,6 +273,48 @@ int lsa_split_representatives(const float* centroids, int64_t NB, int d_I, void*
   if (NB == 0) return LSA_OK;
   LSA_CHECK_ARG(centroids && split && aligned16(centroids) && aligned16(split));
   return launch_split_bf16x3(centroids, NB * d_I, split, static_cast<cudaStream_t>(stream));
+}
+
+size_t lsa_hi_workspace_size(int64_t B, int64_t L, int P, int Bsub, int M, int K, int sink, int window) {
+  if (B < 0 || L < 1 || P < 1 || Bsub < 1 || P % Bsub != 0 || M < 1 || K < 1 || sink < 0 || window < 0)
+    return static_cast<size_t>(-1);
+  return hi_ws_layout(B, L, P, Bsub, M, K, sink, window).total;
+}
+
+int lsa_hi_select(const void* q_idx, const float* w, const void* k_idx, int64_t B, int H_I, int d_I, int64_t L,
+                  const void* sub_split, int P, int Bsub, int M, int K, int sink, int window, const int64_t* q_pos,
+                  int32_t* idx, int64_t idx_ld, int32_t* count, void* ws, size_t ws_bytes, void* stream) {
+  LSA_CHECK_ARG(B >= 0 && L >= 1 && L < (int64_t(1) << 31) && K >= 1 && sink >= 0 && window >= 0);
+  LSA_CHECK_ARG(Bsub >= 1 && P >= Bsub && P % Bsub == 0 && P <= 65536 && M >= 1 && M <= 1024);
+  LSA_CHECK_ARG(static_cast<int64_t>(M) * P + Bsub + sink + window < (int64_t(1) << 31));
+  LSA_CHECK_ARG(idx_ld >= static_cast<int64_t>(K) + sink + window);
+  // the sub-block scoring is the tensor-core representative scoring
+  if (d_I != 128 || (H_I != 32 && H_I != 64) || L / Bsub < 128 || L / Bsub >= (int64_t(1) << 29))
+    return LSA_ERR_UNSUPPORTED;
+  if (B == 0) return LSA_OK;
+  LSA_CHECK_ARG(B <= 65535);
+  LSA_CHECK_ARG(q_idx && w && k_idx && sub_split && q_pos && idx && count);
+  LSA_CHECK_ARG(aligned16(q_idx) && aligned16(k_idx) && aligned16(sub_split));
+  const HiLayout h = hi_ws_layout(B, L, P, Bsub, M, K, sink, window);
+  if (ws == nullptr || !aligned256(ws) || ws_bytes < h.total) return LSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  float* sub = reinterpret_cast<float*>(base);
+  float* page = reinterpret_cast<float*>(base + h.o_page);
+  int32_t* kept = reinterpret_cast<int32_t*>(base + h.o_kept);
+  int32_t* kcnt = reinterpret_cast<int32_t*>(base + h.o_kcnt);
+  int32_t* cand = reinterpret_cast<int32_t*>(base + h.o_cand);
+  int32_t* ccnt = reinterpret_cast<int32_t*>(base + h.o_ccnt);
+  // stage one: sub-block scores, page sums, the top-M pages (every page ranked; pages past q_pos are -inf)
+  int st = launch_centroid_score_tc(q_idx, w, sub_split, B, H_I, h.nsub, sub, h.ld_sub, s);
+  if (st == LSA_OK) st = launch_page_sum(sub, h.ld_sub, h.nsub, P, Bsub, h.npages, B, q_pos, page, h.ld_pg, s);
+  if (st == LSA_OK) st = launch_topk_mode(page, h.ld_pg, B, h.npages, M, 0, 0, q_pos, 1, 1, kept, M, kcnt, M, s);
+  // the recalled tokens as a candidate row, then stage two: the token score and top-K on them
+  if (st == LSA_OK) st = launch_page_expand(kept, M, kcnt, P, Bsub, sink, window, q_pos, B, cand, h.cand_ld, ccnt, s);
+  if (st == LSA_OK)
+    st = launch_refine(q_idx, w, k_idx, B, H_I, d_I, L, cand, h.cand_ld, ccnt, K, sink, window, q_pos, idx, idx_ld,
+                       count, static_cast<int64_t>(K) + sink + window, base + h.o_ref, s);
+  return st;
 }
 
 int lsa_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,

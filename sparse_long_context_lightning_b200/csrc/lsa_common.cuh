@@ -150,6 +150,11 @@ int launch_split_bf16x3(const float* x, int64_t n, void* out, cudaStream_t s);
 int launch_centroid_score_tc(const void* q, const float* w, const void* split, int64_t B, int H_I, int64_t NB,
                              float* scores, int64_t ld, cudaStream_t s);
 size_t bucket_ws_min_bytes(int64_t B, int64_t NB, int M);
+int launch_page_sum(const float* sub, int64_t sub_ld, int64_t nsub, int P, int Bsub, int64_t npages, int64_t B,
+                    const int64_t* q_pos, float* page, int64_t page_ld, cudaStream_t s);
+int launch_page_expand(const int32_t* kept, int64_t kept_ld, const int32_t* kcnt, int P, int Bsub, int sink,
+                       int window, const int64_t* q_pos, int64_t B, int32_t* cand, int64_t cand_ld,
+                       int32_t* ccount, cudaStream_t s);
 int launch_topk(const float* scores, int64_t ld, int64_t B, int64_t L, int K, int sink, int window,
                 const int64_t* q_pos, int64_t rank_limit_div, int32_t* idx, int64_t idx_ld, int32_t* count,
                 int64_t kmax, cudaStream_t s);

@@ -442,3 +442,72 @@ def test_sparse_attn_single_split_many_queries():
             continue
         assert attn_rel_err(out[b], ref) <= ATTN_REL
         assert np.abs(f64(lse[b]) - ref_lse).max() <= 1e-3
+
+
+# --------------------------------------------------------------------------------------------
+# HI two-stage selection
+# --------------------------------------------------------------------------------------------
+
+
+def _hi_run(wl, q_pos, P, Bsub, M):
+    q_I, w = S.index_queries(wl)
+    k = S.index_keys(wl, q_I, DEV)
+    nsub = wl.L // Bsub
+    means = torch.empty(nsub, 128, device=DEV)
+    lsa.lsa_pool_keys(k, means, Bsub)
+    split = torch.empty(3, nsub, 128, dtype=torch.bfloat16, device=DEV)
+    lsa.lsa_split_representatives(means, split)
+    kmax = wl.K + wl.sink + wl.window
+    idx = torch.full((wl.B, kmax), 777, dtype=torch.int32, device=DEV)
+    cnt = torch.empty(wl.B, dtype=torch.int32, device=DEV)
+    ws = lsa.workspace(lsa.lsa_hi_workspace_size(wl.B, wl.L, P, Bsub, M, wl.K, wl.sink, wl.window))
+    qp = torch.as_tensor(q_pos, dtype=torch.int64, device=DEV)
+    lsa.lsa_hi_select(q_I.to(DEV), w.to(DEV), k, split, P, Bsub, M, wl.K, wl.sink, wl.window, qp, idx, cnt, ws)
+    torch.cuda.synchronize()
+    return q_I, w, k, idx.cpu().numpy(), cnt.cpu().numpy()
+
+
+@pytest.mark.parametrize("L,M", [(65536 + 37, 32), (40000, 64)])
+def test_hi_select(L, M):
+    """Against the oracle: the same set, except tokens whose score ties the K-th within 1e-5 (a page
+    ranked differently at the M-th place would put tokens of other pages in the set and fail here)."""
+    P, Bsub = 128, 8
+    wl = S.Workload("hi", L=L, B=4, H_I=64, d_I=128, K=512, H=16, sink=4, window=128, needles="cos06",
+                    n_needles=L // 100)
+    q_pos = [L - 1, L - 501, 30003, 2047]
+    q_I, w, k, idx_h, cnt_h = _hi_run(wl, q_pos, P, Bsub, M)
+    qf, wf, kf = f64(q_I), f64(w), f64(k)
+    for b in range(wl.B):
+        want, kth, mth, recalled = O.hi_select_row(qf[b], wf[b], kf, q_pos[b], P, Bsub, M, wl.K, wl.sink, wl.window)
+        got = idx_h[b, : cnt_h[b]]
+        assert np.all(np.diff(got) > 0) and np.all(idx_h[b, cnt_h[b]:] == -1)
+        assert got.max() <= q_pos[b]
+        if np.array_equal(got, want):
+            continue
+        tok = O.index_score(qf[b][None], wf[b][None], kf[np.setxor1d(got, want)], np.array([L]))[0]
+        assert np.all(np.abs(tok - kth) <= 1e-5 * abs(kth)), (b, np.setxor1d(got, want)[:8])
+
+
+def test_hi_every_page_recalled_is_the_flat_selection():
+    """M * P >= L: every visible token is recalled, so the result is the flat indexer + top-K's (up to
+    ties of the K-th score within 1e-5, the two paths rounding the fp32 sums differently)."""
+    P, Bsub, L = 128, 8, 32768 + 200
+    wl = S.Workload("hi2", L=L, B=2, H_I=64, d_I=128, K=1024, H=16, sink=4, window=128, needles="cos06",
+                    n_needles=300)
+    q_pos = [L - 1, 20000]
+    q_I, w, k, idx_h, cnt_h = _hi_run(wl, q_pos, P, Bsub, M=(L + P - 1) // P)
+    scores = torch.empty(wl.B, (L + 3) // 4 * 4, device=DEV)
+    qp = torch.as_tensor(q_pos, dtype=torch.int64, device=DEV)
+    lsa.lsa_index_score(q_I.to(DEV), w.to(DEV), k, qp, scores)
+    kmax = wl.K + wl.sink + wl.window
+    idx = torch.empty(wl.B, kmax, dtype=torch.int32, device=DEV)
+    cnt = torch.empty(wl.B, dtype=torch.int32, device=DEV)
+    lsa.lsa_topk_select(scores, L, wl.K, wl.sink, wl.window, qp, idx, cnt)
+    flat_h, fcnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    sc = scores.cpu().numpy()
+    for b in range(wl.B):
+        got, ref = idx_h[b, : cnt_h[b]], flat_h[b, : fcnt[b]]
+        diff = np.setxor1d(got, ref)
+        if diff.size:
+            kth = np.sort(sc[b, np.setdiff1d(ref, np.union1d(np.arange(4), np.arange(q_pos[b] - 127, q_pos[b] + 1)))])[0]
+            assert np.all(np.abs(sc[b, diff] - kth) <= 1e-5 * abs(kth)), (b, diff[:8])
