@@ -278,6 +278,55 @@ class BucketStep:
         self.lsa.lsa_sparse_attn(self.q, self.kv, self.idx, self.cnt, self.wl.scale, self.out, self.lse, self.ws_a)
 
 
+class HiStep:
+    """Hierarchical selection (pages of 128 tokens, 8-token sub-blocks, top-1024 pages, token top-K on the
+    recalled tokens) beside the flat bf16 indexer + top-K over the same keys, then attention.  The sub-block
+    means and their bf16 split are built once before timing (the untimed precompute)."""
+
+    P, BSUB, M = 128, 8, 1024
+
+    def __init__(self, wl: S.Workload, device):
+        import sparse_long_context_lightning_b200 as lsa
+
+        self.lsa, self.wl = lsa, wl
+        q_I, w = S.index_queries(wl, "cpu")
+        self.k = S.index_keys(wl, q_I, device)
+        self.q_I, self.w = q_I.to(device), w.to(device)
+        nsub = wl.L // self.BSUB
+        means = torch.empty(nsub, wl.d_I, device=device)
+        lsa.lsa_pool_keys(self.k, means, self.BSUB)
+        self.split = torch.empty(3, nsub, wl.d_I, dtype=torch.bfloat16, device=device)
+        lsa.lsa_split_representatives(means, self.split)
+        del means
+        self.q_pos = wl.q_pos().to(device)
+        kmax = wl.K + wl.sink + wl.window
+        self.idx = torch.empty(wl.B, kmax, dtype=torch.int32, device=device)
+        self.cnt = torch.empty(wl.B, dtype=torch.int32, device=device)
+        self.ws = lsa.workspace(lsa.lsa_hi_workspace_size(wl.B, wl.L, self.P, self.BSUB, self.M, wl.K, wl.sink,
+                                                          wl.window), device)
+        self.scores = torch.empty(wl.B, wl.L, device=device)
+        self.fidx = torch.empty_like(self.idx)
+        self.fcnt = torch.empty_like(self.cnt)
+        self.q = S.attn_queries(wl, device)
+        self.kv = S.latent_cache(wl, device)
+        self.out = torch.empty(wl.B, wl.H, wl.d_v, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(wl.B, wl.H, device=device)
+        self.ws_a = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_ATTN, wl.B, wl.L, kmax, wl.H), device)
+
+    def hi(self):
+        wl = self.wl
+        self.lsa.lsa_hi_select(self.q_I, self.w, self.k, self.split, self.P, self.BSUB, self.M, wl.K, wl.sink,
+                               wl.window, self.q_pos, self.idx, self.cnt, self.ws)
+
+    def flat(self):
+        wl = self.wl
+        self.lsa.lsa_index_score(self.q_I, self.w, self.k, self.q_pos, self.scores)
+        self.lsa.lsa_topk_select(self.scores, wl.L, wl.K, wl.sink, wl.window, self.q_pos, self.fidx, self.fcnt)
+
+    def attn(self):
+        self.lsa.lsa_sparse_attn(self.q, self.kv, self.idx, self.cnt, self.wl.scale, self.out, self.lse, self.ws_a)
+
+
 def _time_stages(stages, l2_flush, iters):
     """Mean CUDA-event time (ms) of each callable in `stages`, run in order, L2 flushed before each pass."""
     stream = torch.cuda.current_stream()
@@ -335,6 +384,26 @@ def long_context_configs(device, l2_flush, iters: int = 10):
                    "attn": _stage(st[2], at_bytes)},
         "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
     del step
+    torch.cuda.empty_cache()
+    # 1M tokens, hierarchical selection (bf16) against the flat bf16 indexer + top-K on the same keys
+    wl = S.WORKLOADS["decode1m"]
+    hstep = HiStep(wl, device)
+    st = _time_stages([hstep.hi, hstep.attn, hstep.flat], l2_flush, iters)
+    B, L = wl.B, wl.L
+    recalled = HiStep.M * HiStep.P
+    sub_flops = 3 * 2.0 * B * wl.H_I * wl.d_I * (L // HiStep.BSUB)
+    tok_flops = 2.0 * B * wl.H_I * wl.d_I * recalled
+    hi_bytes = (L // HiStep.BSUB) * wl.d_I * 6 + B * recalled * (wl.d_I * 2 + 8)
+    hrows = float(hstep.cnt.sum().item())
+    h_at_bytes = hrows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
+    res["decode1m_hi"] = {
+        "workload": "B=4 decode queries, L=1048576, bf16 indexer keys; pages of 128 tokens, 8-token sub-block means "
+                    "(cached bf16 split), top-1024 pages (131072 recalled tokens), exact token top-2048 on them, "
+                    "sink 4 + window 128, H=128",
+        "stages": {"hi_select": _stage(st[0], hi_bytes, sub_flops + tok_flops, bf16), "attn": _stage(st[1], h_at_bytes)},
+        "flat_select_ms": round(float(st[2]), 5),
+        "ms": round(float(st[0] + st[1]), 5), "queries_per_s": round(B / (float(st[0] + st[1]) * 1e-3), 1)}
+    del hstep
     torch.cuda.empty_cache()
     for name in ("decode1m_mb", "flat10m"):
         wl = S.WORKLOADS[name]
