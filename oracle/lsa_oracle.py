@@ -24,6 +24,8 @@ primitives (matmul, stable sort, exp, log) as steps and no blocking or fusion:
                       visible tokens of the incomplete tail block are read directly).
 * ``hi_select_row``   LongCat page §"机制三：层级索引（HI）": page scores from the sub-blocks' mean
                       keys, top-M pages, then the token score and arg topK on the recalled tokens.
+* ``lse_merge``       LongCat page §"训练与 kernel：混合稀疏注意力算子（HFA）": partial attentions merged by
+                      online-softmax (log-sum-exp) rescaling.
 * ``softmax_attention`` / ``sparse_mla_attn``
                       LongCat page §"DSA 基线", u_t = Attn(h_t, {c_s | s in S_t}) in the absorbed
                       MQA form (one latent c_s shared by all heads; value = first 512 dims);
@@ -280,6 +282,29 @@ def sparse_mla_attn(q: np.ndarray, kv_rows: np.ndarray, scale: float, d_v: int =
     """Absorbed-MQA form: each gathered latent row c_s [d_qk] is the key, its first d_v dims the value."""
     kv_rows = np.asarray(kv_rows, dtype=np.float64)
     return softmax_attention(q, kv_rows, kv_rows[:, :d_v], scale)
+
+
+def lse_merge(parts):
+    """Online-softmax merge of partial attentions over disjoint key sets: [(o_i [H, d_v], lse_i [H])] ->
+    (o, lse) of the attention over their union.
+
+    LongCat page §"训练与 kernel：混合稀疏注意力算子（HFA）": the sparse and sliding-window operators' partial
+    outputs are combined by rescaling with their log-sum-exp statistics.  With m = max_i lse_i:
+    o = sum_i exp(lse_i - m) o_i / sum_i exp(lse_i - m), lse = m + log sum_i exp(lse_i - m); parts with
+    lse = -inf (empty key sets) carry no weight.
+    """
+    os_ = [np.asarray(o, dtype=np.float64) for o, _ in parts]
+    ls = np.stack([np.asarray(l, dtype=np.float64) for _, l in parts])  # [n, H]
+    m = ls.max(axis=0)
+    out = np.zeros_like(os_[0])
+    lse = np.full(ls.shape[1], -np.inf)
+    ok = np.isfinite(m)
+    if ok.any():
+        wts = np.where(np.isfinite(ls[:, ok]), np.exp(ls[:, ok] - m[ok]), 0.0)  # [n, H']
+        den = wts.sum(axis=0)
+        out[ok] = sum(wts[i][:, None] * os_[i][ok] for i in range(len(os_))) / den[:, None]
+        lse[ok] = m[ok] + np.log(den)
+    return out, lse
 
 
 # ---------------------------------------------------------------------------

@@ -407,3 +407,26 @@ def test_hi_is_causal():
     b = O.hi_select_row(q, w, k2, q_pos, P=16, Bsub=8, M=5, K=12, sink=2, window=4)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[3], b[3]) and a[2] == b[2]
     assert a[3].max() <= q_pos
+
+
+# --------------------------------------------------------------------------------------------
+# HFA: LSE merge of partial attentions
+# --------------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("cuts", [[5], [1, 7], [0, 3, 3, 12]])
+def test_lse_merge_equals_attention_over_the_union(cuts):
+    """Merging the attentions of a partition (empty parts included) is the attention over the whole set."""
+    rng = np.random.default_rng(11)
+    q, kv = rng.normal(size=(6, 24)), rng.normal(size=(12, 24))
+    bounds = [0] + cuts + [12]
+    parts = [O.softmax_attention(q, kv[a:b], kv[a:b, :10], 0.3) for a, b in zip(bounds[:-1], bounds[1:])]
+    o, lse = O.lse_merge(parts)
+    ref_o, ref_lse = O.softmax_attention(q, kv, kv[:, :10], 0.3)
+    np.testing.assert_allclose(o, ref_o, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_lse_merge_of_empty_parts_is_empty():
+    o, lse = O.lse_merge([(np.zeros((3, 4)), np.full(3, -np.inf))] * 2)
+    assert np.all(o == 0) and np.all(lse == -np.inf)
