@@ -53,7 +53,8 @@ typedef enum {
   LSA_OP_BUCKET = 2,
   LSA_OP_ATTN = 3,
   LSA_OP_REFINE = 4,
-  LSA_OP_BUCKET_MIN = 5 /* the smaller lsa_bucket_select workspace: CUDA-core representative scoring */
+  LSA_OP_BUCKET_MIN = 5, /* the smaller lsa_bucket_select workspace: CUDA-core representative scoring */
+  LSA_OP_HYBRID_ATTN = 6
 } lsa_op;
 
 /*
@@ -280,12 +281,33 @@ int lsa_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx
                     void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * lsa_hybrid_attn -- lsa_sparse_attn over a selection row split into its two parts, run concurrently.
+ *   Source: "LongCat Sparse Attention（LSA）完全拆解", section "训练与 kernel：混合稀疏注意力算子（HFA）": the
+ *   core attention is split into a sparse-gather operator over S_sparse and a sliding-window operator over
+ *   the contiguous positions, dispatched on separate non-blocking streams and merged by online-softmax
+ *   (log-sum-exp) rescaling -- mathematically one attention over the union.
+ *
+ *   idx / count: rows in lsa_topk_select's layout (sink entries, then the sparse entries, then the window
+ *   entries, for the same sink / window / q_pos).  The fixed part (sink {0..} and window {..q_pos}) is read
+ *   as contiguous positions; the sparse part from the row.  out / lse: as lsa_sparse_attn over the whole row
+ *   (equal up to fp32 rounding of the merge).  The fixed part runs on a library-owned second stream (created
+ *   on the first call on a device: make that call before any stream capture), forked from and joined back
+ *   into `stream` with events.  H other than 128: one pass over the union on `stream`.
+ *   ws: lsa_workspace_size(LSA_OP_HYBRID_ATTN, B, L, idx_ld, H, sink, window) bytes.
+ */
+int lsa_hybrid_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                    const int32_t* count, int64_t B, int H, int d_qk, int d_v, int sink, int window,
+                    const int64_t* q_pos, float scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/*
  * lsa_workspace_size -- scratch bytes a call needs (0 if none).
  *   op = LSA_OP_TOPK:   0.
  *   op = LSA_OP_BUCKET: (B, L=NB, K=M) -> per-query bucket scores and kept-bucket lists, plus the
  *                       representatives' bf16 split for tensor-core scoring (NB * 768 bytes).
  *   op = LSA_OP_BUCKET_MIN: the same without the split (CUDA-core scoring).
  *   op = LSA_OP_ATTN:   (B, L, K=idx_ld, H) -> split-K partial outputs.
+ *   op = LSA_OP_HYBRID_ATTN: (B, L, K=idx_ld, H, sink, window) -> both branches' partials and index rows.
  *   op = LSA_OP_REFINE: (B, L=cand_ld, K) -> re-ranked scores and kept lists.
  *   Returns (size_t)-1 for an unknown op or negative sizes.
  */

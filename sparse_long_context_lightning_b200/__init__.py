@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "liblsa.so")
 LSA_OK = 0
 LSA_BF16 = 0
 LSA_FP8_E4M3 = 1
-LSA_OP_TOPK, LSA_OP_BUCKET, LSA_OP_ATTN, LSA_OP_REFINE, LSA_OP_BUCKET_MIN = 1, 2, 3, 4, 5
+LSA_OP_TOPK, LSA_OP_BUCKET, LSA_OP_ATTN, LSA_OP_REFINE, LSA_OP_BUCKET_MIN, LSA_OP_HYBRID_ATTN = 1, 2, 3, 4, 5, 6
 
 _STATUS = {0: "LSA_OK", -1: "LSA_ERR_INVALID_ARG", -2: "LSA_ERR_UNSUPPORTED", -3: "LSA_ERR_WORKSPACE",
            -4: "LSA_ERR_CUDA", -5: "LSA_ERR_DEVICE_CHECK", -6: "LSA_ERR_TIMEOUT"}
@@ -42,6 +42,8 @@ SIGNATURES = {
     "lsa_hi_select": (_I32, [_P, _P, _P, _I64, _I32, _I32, _I64, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P, _I64,
                              _P, _P, _SZ, _P]),
     "lsa_hi_workspace_size": (_SZ, [_I64, _I64, _I32, _I32, _I32, _I32, _I32, _I32]),
+    "lsa_hybrid_attn": (_I32, [_P, _P, _I64, _P, _I64, _P, _I64, _I32, _I32, _I32, _I32, _I32, _P, _F32, _P, _P, _P,
+                               _SZ, _P]),
     "lsa_sparse_attn": (_I32, [_P, _P, _I64, _P, _I64, _P, _I64, _I32, _I32, _I32, _F32, _P, _P, _P, _SZ, _P]),
     "lsa_workspace_size": (_SZ, [_I32, _I64, _I64, _I32, _I32, _I32, _I32]),
     "lsa_strerror": (ctypes.c_char_p, [_I32]),
@@ -197,6 +199,17 @@ def lsa_sparse_attn(q, kv, idx, count, scale, out, lse=None, ws=None, stream=Non
                                         d_qk, d_v, float(scale), _ptr(out), _ptr(lse), _ptr(ws),
                                         0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check("lsa_sparse_attn", st)
+
+
+def lsa_hybrid_attn(q, kv, idx, count, sink, window, q_pos, scale, out, lse=None, ws=None, stream=None):
+    """lsa_sparse_attn over sink | sparse | window rows, the fixed part on a second stream, merged by LSE."""
+    B, H, d_qk = q.shape
+    d_v = out.shape[-1]
+    st = load_library().lsa_hybrid_attn(_ptr(q), _ptr(kv), kv.shape[0], _ptr(idx), idx.stride(0), _ptr(count), B, H,
+                                        d_qk, d_v, sink, window, _ptr(q_pos), float(scale), _ptr(out), _ptr(lse),
+                                        _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                        _stream(stream))
+    _check("lsa_hybrid_attn", st)
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:

@@ -71,7 +71,9 @@ struct AtArgs {
   const int32_t* count;
   int B;
   int L;
-  int S;  // splits per query
+  int S;        // splits per query of this launch
+  int S_total;  // partial slots per query in ws_o / ws_ml (this launch fills [slot0, slot0 + S)); 1 = no partials
+  int slot0;
   float scale_log2;
   uint16_t* out;
   float* lse;
@@ -378,7 +380,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     // O (row h = this thread's TMEM lane) is staged in the stage memory -- free once the last P.V completed --
     // with a padded row pitch (no bank conflicts), then written with one bulk copy per row
     unsigned char* srow = st_s + h * AT_O_PITCH;
-    if (a.S == 1) {
+    if (a.S_total == 1) {
       const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
       #pragma unroll 1
       for (int k = 0; k < 8; ++k) {
@@ -404,7 +406,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       bulk_store_global(a.out + orow * 512 + 256 * r, srow, 512);
       if (r == 0 && a.lse) a.lse[orow] = (have && l > 0.f) ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
     } else {
-      const int64_t prow_i = (static_cast<int64_t>(b) * a.S + split) * AT_H + h;
+      const int64_t prow_i = (static_cast<int64_t>(b) * a.S_total + a.slot0 + split) * AT_H + h;
       #pragma unroll 1
       for (int k = 0; k < 8; ++k) {
         uint32_t o[32];
@@ -503,6 +505,31 @@ __global__ void __launch_bounds__(128) k_attn_combine(const float* __restrict__ 
   if (lse && threadIdx.x == 0) lse[bh] = lsum > 0.f ? (mstar + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
 }
 
+// The hybrid operator's two index sets from a selection row (sink | sparse | window, lsa_topk_select's layout):
+// the sparse entries, and the fixed (sink + window) entries -- contiguous position ranges.
+__global__ void __launch_bounds__(256) k_hfa_split(const int32_t* __restrict__ idx, int64_t idx_ld,
+                                                   const int32_t* __restrict__ count, int sink, int window,
+                                                   const int64_t* __restrict__ q_pos, int32_t* __restrict__ sp,
+                                                   int32_t* __restrict__ sp_cnt, int32_t* __restrict__ fx,
+                                                   int64_t fx_ld, int32_t* __restrict__ fx_cnt) {
+  const int b = blockIdx.x;
+  const int qp = static_cast<int>(q_pos[b]);
+  const int nsink = min(sink, qp + 1);
+  const int wlo = window > 0 ? max(qp - window + 1, nsink) : qp + 1;
+  const int nwin = qp + 1 - wlo;
+  int n = count[b];
+  n = n < 0 ? 0 : (static_cast<int64_t>(n) > idx_ld ? static_cast<int>(idx_ld) : n);
+  const int ndyn = max(0, n - nsink - nwin);
+  const int32_t* row = idx + static_cast<int64_t>(b) * idx_ld;
+  for (int i = threadIdx.x; i < ndyn; i += 256) sp[static_cast<int64_t>(b) * idx_ld + i] = row[nsink + i];
+  for (int i = threadIdx.x; i < nsink + nwin; i += 256)
+    fx[static_cast<int64_t>(b) * fx_ld + i] = i < nsink ? i : wlo + (i - nsink);
+  if (threadIdx.x == 0) {
+    sp_cnt[b] = ndyn;
+    fx_cnt[b] = nsink + nwin;
+  }
+}
+
 int splits_for(int64_t B) {
   int64_t s = 148 / (2 * (B > 0 ? B : 1));
   if (s < 1) s = 1;
@@ -547,6 +574,8 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   a.B = static_cast<int>(B);
   a.L = static_cast<int>(L);
   a.S = S;
+  a.S_total = S;
+  a.slot0 = 0;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
@@ -562,6 +591,121 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
     LSA_CUDA_TRY(launch_pdl(k_attn_combine, dim3(static_cast<unsigned>(B * AT_H)), dim3(128), 0, s, 0u,
                             static_cast<const float*>(a.ws_o), static_cast<const float*>(a.ws_ml), S, a.out, lse));
   }
+  return LSA_OK;
+}
+
+// Hybrid (sparse + contiguous) operator: workspace = partials of S + 1 slots (the sparse branch's S splits and
+// the fixed branch's one) | ml of those | sparse rows [B, idx_ld] | fixed rows [B, sink + window] | two counts.
+struct HfaLayout {
+  int S;
+  size_t o_ml, o_sp, o_fx, o_spc, o_fxc, total;
+};
+static HfaLayout hfa_layout(int64_t B, int64_t idx_ld, int sink, int window) {
+  HfaLayout h;
+  h.S = splits_for(B);
+  const int St = h.S + 1;
+  size_t o = align_up(static_cast<size_t>(B) * St * AT_H * 512 * 4, 256);
+  h.o_ml = o;
+  o = align_up(o + static_cast<size_t>(B) * St * AT_H * 2 * 4, 256);
+  h.o_sp = o;
+  o = align_up(o + static_cast<size_t>(B) * idx_ld * 4, 256);
+  h.o_fx = o;
+  o = align_up(o + static_cast<size_t>(B) * (sink + window) * 4, 256);
+  h.o_spc = o;
+  o = align_up(o + static_cast<size_t>(B) * 4, 256);
+  h.o_fxc = o;
+  h.total = align_up(o + static_cast<size_t>(B) * 4, 256);
+  return h;
+}
+
+size_t hybrid_attn_ws_bytes(int64_t B, int64_t idx_ld, int H, int sink, int window) {
+  if (H != AT_H) return 0;
+  return hfa_layout(B, idx_ld, sink, window).total;
+}
+
+// a second, non-blocking stream and fork / join events per device (created on first use)
+static int side_stream(cudaStream_t* side, cudaEvent_t* fork, cudaEvent_t* join) {
+  static std::mutex mu;
+  static cudaStream_t st[64];
+  static cudaEvent_t ef[64], ej[64];
+  int dev = 0;
+  LSA_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return LSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!st[dev]) {
+    LSA_CUDA_TRY(cudaStreamCreateWithFlags(&st[dev], cudaStreamNonBlocking));
+    LSA_CUDA_TRY(cudaEventCreateWithFlags(&ef[dev], cudaEventDisableTiming));
+    LSA_CUDA_TRY(cudaEventCreateWithFlags(&ej[dev], cudaEventDisableTiming));
+  }
+  *side = st[dev];
+  *fork = ef[dev];
+  *join = ej[dev];
+  return LSA_OK;
+}
+
+int launch_hybrid_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                       const int32_t* count, int64_t B, int H, int sink, int window, const int64_t* q_pos,
+                       float scale, void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t s) {
+  if (B == 0) return LSA_OK;
+  // other head counts: one pass over the union (the same result, computed at once)
+  if (H != AT_H || L >= (int64_t(1) << 31)) return launch_attn_simt(q, kv, L, idx, idx_ld, count, B, H, scale, out, lse, s);
+  const HfaLayout h = hfa_layout(B, idx_ld, sink, window);
+  if (ws == nullptr || !aligned256(ws) || ws_bytes < h.total) return LSA_ERR_WORKSPACE;
+  if (!aligned16(q)) return LSA_ERR_INVALID_ARG;
+  CUtensorMap tq;
+  const int st = make_map(&tq, q, false, B * AT_H, 576, 64, AT_H);
+  if (st) return st;
+  cudaStream_t side;
+  cudaEvent_t ev_fork, ev_join;
+  const int ss = side_stream(&side, &ev_fork, &ev_join);
+  if (ss) return ss;
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  int32_t* sp = reinterpret_cast<int32_t*>(base + h.o_sp);
+  int32_t* fx = reinterpret_cast<int32_t*>(base + h.o_fx);
+  int32_t* spc = reinterpret_cast<int32_t*>(base + h.o_spc);
+  int32_t* fxc = reinterpret_cast<int32_t*>(base + h.o_fxc);
+  const int64_t fx_ld = sink + window;
+  k_hfa_split<<<static_cast<unsigned>(B), 256, 0, s>>>(idx, idx_ld, count, sink, window, q_pos, sp, spc, fx,
+                                                       fx_ld > 0 ? fx_ld : 1, fxc);
+  LSA_CUDA_TRY(cudaGetLastError());
+  AtArgs a;
+  a.q = static_cast<const uint16_t*>(q);
+  a.kv = static_cast<const uint16_t*>(kv);
+  a.B = static_cast<int>(B);
+  a.L = static_cast<int>(L);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.S_total = h.S + 1;
+  a.ws_o = reinterpret_cast<float*>(base);
+  a.ws_ml = reinterpret_cast<float*>(base + h.o_ml);
+  LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_sparse_attn_tc), AT_SMEM));
+  // fixed branch (sink + window, contiguous) on the side stream: slot S, one split
+  LSA_CUDA_TRY(cudaEventRecord(ev_fork, s));
+  LSA_CUDA_TRY(cudaStreamWaitEvent(side, ev_fork, 0));
+  AtArgs af = a;
+  af.idx = fx;
+  af.idx_ld = fx_ld > 0 ? fx_ld : 1;
+  af.count = fxc;
+  af.S = 1;
+  af.slot0 = h.S;
+  // a plain launch: its inputs arrive through the fork event, not from the side stream's previous kernel
+  k_sparse_attn_tc<<<static_cast<unsigned>(2 * B), AT_THREADS, AT_SMEM, side>>>(tq, af);
+  LSA_CUDA_TRY(cudaGetLastError());
+  LSA_CUDA_TRY(cudaEventRecord(ev_join, side));
+  // sparse branch on the caller's stream: slots [0, S)
+  AtArgs as = a;
+  as.idx = sp;
+  as.idx_ld = idx_ld;
+  as.count = spc;
+  as.S = h.S;
+  as.slot0 = 0;
+  LSA_CUDA_TRY(launch_pdl(k_sparse_attn_tc, dim3(static_cast<unsigned>(2 * B * h.S)), dim3(AT_THREADS), AT_SMEM, s, 0u,
+                          tq, as));
+  // merge: the online-softmax (LSE) combination of all S + 1 partials
+  LSA_CUDA_TRY(cudaStreamWaitEvent(s, ev_join, 0));
+  LSA_CUDA_TRY(launch_pdl(k_attn_combine, dim3(static_cast<unsigned>(B * AT_H)), dim3(128), 0, s, 0u,
+                          static_cast<const float*>(a.ws_o), static_cast<const float*>(a.ws_ml), h.S + 1, a.out, lse));
   return LSA_OK;
 }
 

@@ -123,6 +123,7 @@ size_t lsa_workspace_size(int op, int64_t B, int64_t L, int K, int H, int sink, 
     }
     case LSA_OP_BUCKET_MIN: return bucket_ws_min_bytes(B, L, K);
     case LSA_OP_ATTN: return sparse_attn_ws_bytes(B, K, H);
+    case LSA_OP_HYBRID_ATTN: return hybrid_attn_ws_bytes(B, K, H, sink, window);
     case LSA_OP_REFINE: return refine_ws_bytes(B, L, K);
     default: return static_cast<size_t>(-1);
   }
@@ -273,6 +274,22 @@ int lsa_split_representatives(const float* centroids, int64_t NB, int d_I, void*
   if (NB == 0) return LSA_OK;
   LSA_CHECK_ARG(centroids && split && aligned16(centroids) && aligned16(split));
   return launch_split_bf16x3(centroids, NB * d_I, split, static_cast<cudaStream_t>(stream));
+}
+
+int lsa_hybrid_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                    const int32_t* count, int64_t B, int H, int d_qk, int d_v, int sink, int window,
+                    const int64_t* q_pos, float scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                    void* stream) {
+  LSA_CHECK_ARG(B >= 0 && L >= 1 && idx_ld >= 0 && idx_ld <= 65536 && sink >= 0 && window >= 0);
+  LSA_CHECK_ARG(static_cast<int64_t>(sink) + window <= 65536);
+  if (d_qk != 576 || d_v != 512) return LSA_ERR_UNSUPPORTED;
+  if (H != 16 && H != 32 && H != 64 && H != 128) return LSA_ERR_UNSUPPORTED;
+  if (B == 0) return LSA_OK;
+  LSA_CHECK_ARG(q && kv && idx && count && q_pos && out);
+  LSA_CHECK_ARG(aligned16(q) && aligned16(kv) && aligned16(out));
+  LSA_CHECK_ARG(B <= 65535);
+  return launch_hybrid_attn(q, kv, L, idx, idx_ld, count, B, H, sink, window, q_pos, scale, out, lse, ws, ws_bytes,
+                            static_cast<cudaStream_t>(stream));
 }
 
 size_t lsa_hi_workspace_size(int64_t B, int64_t L, int P, int Bsub, int M, int K, int sink, int window) {

@@ -164,6 +164,10 @@ int launch_bucket_expand(const int32_t* kept, int64_t kept_ld, const int32_t* ke
                          const int32_t* members, int bsz, int sink, int window, int tail_block,
                          const int64_t* q_pos, int64_t B, int32_t* idx, int64_t idx_ld, int32_t* count,
                          int64_t kmax, cudaStream_t s);
+int launch_hybrid_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                       const int32_t* count, int64_t B, int H, int sink, int window, const int64_t* q_pos,
+                       float scale, void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t s);
+size_t hybrid_attn_ws_bytes(int64_t B, int64_t idx_ld, int H, int sink, int window);
 int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
                        const int32_t* count, int64_t B, int H, float scale, void* out, float* lse,
                        void* ws, size_t ws_bytes, cudaStream_t s);

@@ -511,3 +511,51 @@ def test_hi_every_page_recalled_is_the_flat_selection():
         if diff.size:
             kth = np.sort(sc[b, np.setdiff1d(ref, np.union1d(np.arange(4), np.arange(q_pos[b] - 127, q_pos[b] + 1)))])[0]
             assert np.all(np.abs(sc[b, diff] - kth) <= 1e-5 * abs(kth)), (b, diff[:8])
+
+
+# --------------------------------------------------------------------------------------------
+# HFA: sparse and contiguous branches on two streams, merged by LSE
+# --------------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("H,sink,window", [(128, 4, 128), (128, 0, 0), (128, 16, 1024), (16, 4, 128)])
+def test_hybrid_attn(H, sink, window):
+    """Against the oracle's merge of the two branches (and the attention over the union it equals), and
+    against the single-pass kernel on the same rows."""
+    L, B, K = 40000 + 5, 5, 700
+    q_pos = [L - 1, L - 1, 30000, 900, 10]
+    wl = S.Workload("hfa", L=L, B=B, H_I=64, d_I=128, K=K, H=H, sink=sink, window=window, needles="cos06",
+                    n_needles=400)
+    d = Decode(wl, q_pos=torch.tensor(q_pos, dtype=torch.int64))
+    scores = torch.empty(B, L + 3, device=DEV)
+    lsa.lsa_index_score(d.q_I, d.w, d.k_I, d.q_pos, scores)
+    kmax = K + sink + window
+    idx = torch.empty(B, kmax, dtype=torch.int32, device=DEV)
+    cnt = torch.empty(B, dtype=torch.int32, device=DEV)
+    lsa.lsa_topk_select(scores, L, K, sink, window, d.q_pos, idx, cnt)
+    kv = S.normal_bf16(S.ST_KV, (L, 576), DEV)
+    q = S.normal_bf16(S.ST_Q, (B, H, 576), DEV)
+    scale = 1 / math.sqrt(576)
+    out = torch.empty(B, H, 512, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(B, H, device=DEV)
+    ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_HYBRID_ATTN, B, L, kmax, H, sink, window))
+    lsa.lsa_hybrid_attn(q, kv, idx, cnt, sink, window, d.q_pos, scale, out, lse, ws)
+    out1 = torch.empty_like(out)
+    lse1 = torch.empty_like(lse)
+    lsa.lsa_sparse_attn(q, kv, idx, cnt, scale, out1, lse1, lsa.workspace(lsa.lsa_workspace_size(
+        lsa.LSA_OP_ATTN, B, L, kmax, H)))
+    torch.cuda.synchronize()
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(B):
+        row = idx_h[b, : cnt_h[b]]
+        s_sink, s_swa = O.fixed_positions(q_pos[b], sink, window)
+        fixed = np.union1d(s_sink, s_swa)
+        sparse = np.setdiff1d(row, fixed)
+        assert np.array_equal(np.union1d(sparse, fixed), row)
+        merged = O.lse_merge([run_oracle_attention(q[b], kv, sparse, scale),
+                              run_oracle_attention(q[b], kv, fixed, scale)])
+        ref, ref_lse = run_oracle_attention(q[b], kv, row, scale)
+        np.testing.assert_allclose(merged[0], ref, rtol=1e-9, atol=1e-12)
+        assert attn_rel_err(out[b], merged[0]) <= ATTN_REL
+        assert np.abs(f64(lse[b]) - merged[1]).max() <= 1e-3
+        assert attn_rel_err(out[b], f64(out1[b])) <= ATTN_REL
