@@ -405,6 +405,29 @@ def long_context_configs(device, l2_flush, iters: int = 10):
         "ms": round(float(st[0] + st[1]), 5), "queries_per_s": round(B / (float(st[0] + st[1]) * 1e-3), 1)}
     del hstep
     torch.cuda.empty_cache()
+    # the pages' fixed / dynamic split (sink 16 + window 1024 + 1024 sparse) at 128K: the attention as one
+    # gather pass over the row and as the hybrid operator (contiguous part on a second stream, LSE merge)
+    wl = S.Workload("decode128k_si", L=131072, B=16, H_I=64, d_I=128, K=1024, H=128, sink=16, window=1024,
+                    needles="cos06", n_needles=1310)
+    step = DecodeStep(wl, "bf16", device)
+    step.index()
+    step.topk()
+    ws_h = step.lsa.workspace(step.lsa.lsa_workspace_size(step.lsa.LSA_OP_HYBRID_ATTN, wl.B, wl.L, step.kmax, wl.H,
+                                                          wl.sink, wl.window), device)
+
+    def hybrid():
+        step.lsa.lsa_hybrid_attn(step.q, step.kv, step.idx, step.cnt, wl.sink, wl.window, step.q_pos, wl.scale,
+                                 step.out, step.lse, ws_h)
+
+    st = _time_stages([step.attn, hybrid], l2_flush, iters)
+    rows = float(step.cnt.sum().item())
+    at_bytes = rows * (wl.d_qk * 2 + 4) + wl.B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
+    res["decode128k_hfa"] = {
+        "workload": "B=16 decode queries, L=131072, sink 16 + window 1024 + top-1024 sparse (the pages' 1:1 fixed / "
+                    "dynamic budget), H=128",
+        "stages": {"attn_single_pass": _stage(st[0], at_bytes), "attn_hybrid": _stage(st[1], at_bytes)}}
+    del step, ws_h
+    torch.cuda.empty_cache()
     for name in ("decode1m_mb", "flat10m"):
         wl = S.WORKLOADS[name]
         bstep = BucketStep(wl, device)

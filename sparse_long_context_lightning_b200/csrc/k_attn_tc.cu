@@ -79,10 +79,12 @@ struct AtArgs {
   float* lse;
   float* ws_o;   // [B, S, 128, 512] fp32 (S > 1)
   float* ws_ml;  // [B, S, 128, 2]   fp32 (S > 1): running max (log2 units), sum
+  int contig;    // rows ascending and unique by construction (the hybrid operator's sink + window rows): a tile
+                 // whose rows are consecutive positions is one TMA tile load instead of a row gather
 };
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
-    k_sparse_attn_tc(const __grid_constant__ CUtensorMap tm_q, AtArgs a) {
+    k_sparse_attn_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv, AtArgs a) {
   // every global access of this kernel comes after the previous kernel of the stream has completed
   sm100::pdl_wait();
   sm100::pdl_launch_dependents();
@@ -163,13 +165,26 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         const int rr = i * AT_T + warp * 2 + (lane & 1);
         return rr < nrows ? rowidx[rr] : 0;
       };
+      // contiguous rows: the tile's first position when its rows are consecutive positions, else -1 (the
+      // rows are ascending and unique, so first and last decide); loaded two tiles ahead as well
+      auto tile_start = [&](int i) -> int {
+        if (!a.contig) return -1;
+        const int m = min(AT_T, nrows - i * AT_T);
+        const int f = rowidx[i * AT_T], l = rowidx[i * AT_T + m - 1];
+        return (f >= 0 && l < a.L && l - f == m - 1) ? f : -1;
+      };
       int v_a = load_idx(0);
       int v_b = ntiles > 1 ? load_idx(1) : 0;
+      int c_a = tile_start(0);
+      int c_b = ntiles > 1 ? tile_start(1) : -1;
       for (int i = 0; i < ntiles; ++i) {
         const int st = i % AT_STAGES;
         const int v_raw = v_a;
         v_a = v_b;
         if (i + 2 < ntiles) v_b = load_idx(i + 2);
+        const int c_now = c_a;
+        c_a = c_b;
+        if (i + 2 < ntiles) c_b = tile_start(i + 2);
         // stages 1-3 hold the Q staging until the softmax warps have copied it into TMEM
         const bool staged_ok = !(i >= 1 && i < AT_STAGES) || mbar_spin(qt_full, 0);
         if (!staged_ok || !mbar_spin(&kv_empty[st], ((i / AT_STAGES) & 1) ^ 1) || abort_flag) {
@@ -179,8 +194,17 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           }
           break;
         }
-        const int v = v_raw < 0 ? 0 : (v_raw >= a.L ? a.L - 1 : v_raw);
         unsigned char* dst = st_s + st * AT_STAGE_BYTES;
+        if (c_now >= 0) {  // consecutive rows: nine 32-row TMA boxes in the same swizzled layout
+          if (tid == 0) {
+            mbar_expect_tx(&kv_full[st], AT_STAGE_BYTES);
+            for (int kb = 0; kb < AT_KB; ++kb) tma_load_2d(dst + kb * AT_KB_BYTES, &tm_kv, &kv_full[st], 64 * kb, c_now);
+          } else {
+            mbar_arrive(&kv_full[st]);
+          }
+          continue;
+        }
+        const int v = v_raw < 0 ? 0 : (v_raw >= a.L ? a.L - 1 : v_raw);
         #pragma unroll
         for (int k = 0; k < (2 * CPR + 31) / 32; ++k) {
           const int q = lane + 32 * k;
@@ -561,11 +585,14 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   const int S = splits_for(B);
   const size_t need = sparse_attn_ws_bytes(B, idx_ld, H);
   if (S > 1 && (ws == nullptr || !aligned256(ws) || ws_bytes < need)) return LSA_ERR_WORKSPACE;
-  CUtensorMap tq;
-  const int st = make_map(&tq, q, false, B * AT_H, 576, 64, AT_H);
+  CUtensorMap tq, tkv;
+  int st = make_map(&tq, q, false, B * AT_H, 576, 64, AT_H);
+  if (st) return st;
+  st = make_map(&tkv, kv, false, L, 576, 64, AT_T);
   if (st) return st;
   if (!aligned16(q)) return LSA_ERR_INVALID_ARG;
   AtArgs a;
+  a.contig = 0;
   a.q = static_cast<const uint16_t*>(q);
   a.kv = static_cast<const uint16_t*>(kv);
   a.idx = idx;
@@ -586,7 +613,8 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_sparse_attn_tc), AT_SMEM));
   const int64_t grid = 2 * B * S;
   if (grid > 0x7FFFFFFF) return LSA_ERR_UNSUPPORTED;
-  LSA_CUDA_TRY(launch_pdl(k_sparse_attn_tc, dim3(static_cast<unsigned>(grid)), dim3(AT_THREADS), AT_SMEM, s, 0u, tq, a));
+  LSA_CUDA_TRY(launch_pdl(k_sparse_attn_tc, dim3(static_cast<unsigned>(grid)), dim3(AT_THREADS), AT_SMEM, s, 0u, tq, tkv,
+                          a));
   if (S > 1) {
     LSA_CUDA_TRY(launch_pdl(k_attn_combine, dim3(static_cast<unsigned>(B * AT_H)), dim3(128), 0, s, 0u,
                             static_cast<const float*>(a.ws_o), static_cast<const float*>(a.ws_ml), S, a.out, lse));
@@ -594,16 +622,21 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   return LSA_OK;
 }
 
-// Hybrid (sparse + contiguous) operator: workspace = partials of S + 1 slots (the sparse branch's S splits and
-// the fixed branch's one) | ml of those | sparse rows [B, idx_ld] | fixed rows [B, sink + window] | two counts.
+// Hybrid (sparse + contiguous) operator: workspace = partials of S_sp + S_fix slots (the two branches' splits)
+// | ml of those | sparse rows [B, idx_ld] | fixed rows [B, sink + window] | two counts.
 struct HfaLayout {
-  int S;
+  int S_sp, S_fix;  // splits of the sparse and the fixed branch (the SMs shared by their row budgets)
   size_t o_ml, o_sp, o_fx, o_spc, o_fxc, total;
 };
 static HfaLayout hfa_layout(int64_t B, int64_t idx_ld, int sink, int window) {
   HfaLayout h;
-  h.S = splits_for(B);
-  const int St = h.S + 1;
+  const int S = splits_for(B);
+  const int64_t fixed = static_cast<int64_t>(sink) + window;
+  const int64_t sparse = max(int64_t(0), idx_ld - fixed);
+  h.S_fix = fixed + sparse > 0 ? static_cast<int>((S * fixed + (fixed + sparse) / 2) / (fixed + sparse)) : 0;
+  h.S_fix = min(max(h.S_fix, 1), max(S - 1, 1));
+  h.S_sp = max(S - h.S_fix, 1);
+  const int St = h.S_sp + h.S_fix;
   size_t o = align_up(static_cast<size_t>(B) * St * AT_H * 512 * 4, 256);
   h.o_ml = o;
   o = align_up(o + static_cast<size_t>(B) * St * AT_H * 2 * 4, 256);
@@ -652,8 +685,10 @@ int launch_hybrid_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   const HfaLayout h = hfa_layout(B, idx_ld, sink, window);
   if (ws == nullptr || !aligned256(ws) || ws_bytes < h.total) return LSA_ERR_WORKSPACE;
   if (!aligned16(q)) return LSA_ERR_INVALID_ARG;
-  CUtensorMap tq;
-  const int st = make_map(&tq, q, false, B * AT_H, 576, 64, AT_H);
+  CUtensorMap tq, tkv;
+  int st = make_map(&tq, q, false, B * AT_H, 576, 64, AT_H);
+  if (st) return st;
+  st = make_map(&tkv, kv, false, L, 576, 64, AT_T);
   if (st) return st;
   cudaStream_t side;
   cudaEvent_t ev_fork, ev_join;
@@ -676,36 +711,39 @@ int launch_hybrid_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
-  a.S_total = h.S + 1;
+  a.S_total = h.S_sp + h.S_fix;
   a.ws_o = reinterpret_cast<float*>(base);
   a.ws_ml = reinterpret_cast<float*>(base + h.o_ml);
   LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_sparse_attn_tc), AT_SMEM));
-  // fixed branch (sink + window, contiguous) on the side stream: slot S, one split
+  // fixed branch (sink + window, contiguous: TMA tile loads) on the side stream: slots [S_sp, S_sp + S_fix)
   LSA_CUDA_TRY(cudaEventRecord(ev_fork, s));
   LSA_CUDA_TRY(cudaStreamWaitEvent(side, ev_fork, 0));
   AtArgs af = a;
   af.idx = fx;
   af.idx_ld = fx_ld > 0 ? fx_ld : 1;
   af.count = fxc;
-  af.S = 1;
-  af.slot0 = h.S;
+  af.S = h.S_fix;
+  af.slot0 = h.S_sp;
+  af.contig = 1;
   // a plain launch: its inputs arrive through the fork event, not from the side stream's previous kernel
-  k_sparse_attn_tc<<<static_cast<unsigned>(2 * B), AT_THREADS, AT_SMEM, side>>>(tq, af);
+  k_sparse_attn_tc<<<static_cast<unsigned>(2 * B * h.S_fix), AT_THREADS, AT_SMEM, side>>>(tq, tkv, af);
   LSA_CUDA_TRY(cudaGetLastError());
   LSA_CUDA_TRY(cudaEventRecord(ev_join, side));
-  // sparse branch on the caller's stream: slots [0, S)
+  // sparse branch (row gathers) on the caller's stream: slots [0, S_sp)
   AtArgs as = a;
   as.idx = sp;
   as.idx_ld = idx_ld;
   as.count = spc;
-  as.S = h.S;
+  as.S = h.S_sp;
   as.slot0 = 0;
-  LSA_CUDA_TRY(launch_pdl(k_sparse_attn_tc, dim3(static_cast<unsigned>(2 * B * h.S)), dim3(AT_THREADS), AT_SMEM, s, 0u,
-                          tq, as));
+  as.contig = 0;
+  LSA_CUDA_TRY(launch_pdl(k_sparse_attn_tc, dim3(static_cast<unsigned>(2 * B * h.S_sp)), dim3(AT_THREADS), AT_SMEM, s,
+                          0u, tq, tkv, as));
   // merge: the online-softmax (LSE) combination of all S + 1 partials
   LSA_CUDA_TRY(cudaStreamWaitEvent(s, ev_join, 0));
   LSA_CUDA_TRY(launch_pdl(k_attn_combine, dim3(static_cast<unsigned>(B * AT_H)), dim3(128), 0, s, 0u,
-                          static_cast<const float*>(a.ws_o), static_cast<const float*>(a.ws_ml), h.S + 1, a.out, lse));
+                          static_cast<const float*>(a.ws_o), static_cast<const float*>(a.ws_ml), h.S_sp + h.S_fix, a.out,
+                          lse));
   return LSA_OK;
 }
 
