@@ -453,6 +453,18 @@ def long_context_configs(device, l2_flush, iters: int = 10):
     return res
 
 
+def max_over_ranks(vals: torch.Tensor, world: int) -> torch.Tensor:
+    """Element-wise max over the ranks (the slowest rank's times); identity for one process."""
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    return vals
+
+
+def job_rate(per_rank_units: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the units every rank processed, over the slowest rank's time."""
+    return per_rank_units * world / (ms * 1e-3)
+
+
 def run_gpu(args, rank, world, local_rank):
     import sparse_long_context_lightning_b200 as lsa
 
@@ -569,9 +581,8 @@ def run_gpu(args, rank, world, local_rank):
     del graph
 
     # max over ranks
-    vals = torch.tensor([step_ms, e2e_step, *stage_ms.tolist()], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    vals = max_over_ranks(torch.tensor([step_ms, e2e_step, *stage_ms.tolist()], dtype=torch.float64, device=device),
+                          world)
     step_ms, e2e_step = float(vals[0]), float(vals[1])
     stage_ms = vals[2:].cpu().numpy()
     if rank != 0:
@@ -604,7 +615,7 @@ def run_gpu(args, rank, world, local_rank):
                 "frac": stages[dom]["hbm_frac"]}
     roof.update({"kernel": kname, "peak_source": pk_src + (" (bf16 x2 nominal ratio)" if dom == "index" and step.fp8 else ""),
                  "traffic": committed_traffic(kname)})
-    qps = wl.B * world / (step_ms * 1e-3)
+    qps = job_rate(wl.B, world, step_ms)
     n_launch = sum(launches.values()) * args.steps
     return {
         "metric": "sparse decode queries/s @L=128K,K=2048",
@@ -626,7 +637,7 @@ def run_gpu(args, rank, world, local_rank):
         "gather_hbm_gbs": stages["attn"]["achieved_gbs"],
         "stages": stages,
         "roofline": roof,
-        "e2e": {"value": round(wl.B * world / (e2e_step * 1e-3), 1), "unit": "queries/s",
+        "e2e": {"value": round(job_rate(wl.B, world, e2e_step), 1), "unit": "queries/s",
                 "ms_per_step": round(e2e_step, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "mode": e2e_mode, "eager_ms_per_step": round(e2e_eager, 5)},
         "gpu_launches": n_launch,
@@ -680,7 +691,8 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def run_reference(args, rank):
+def run_reference(args, rank, world=1):
+    """The oracle on the host cores; under torchrun only rank 0 runs it (the others return None at once)."""
     if rank != 0:
         return None
     # warm-up steps are untimed oracle queries; each timed step is one bounded sample (<= 2 queries)
@@ -694,7 +706,7 @@ def run_reference(args, rank):
     v = qs / secs
     cores = blas_threads()
     return {"metric": "sparse decode queries/s @L=128K,K=2048", "value": round(v, 4), "unit": "queries/s",
-            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 2),
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (lsa_synth, seed 0)", "impl": "reference",
             "config": {"workload": f"{CONFIG}: B=16 decode queries, L=131072, H_I=64, d_I=128, K=2048, H=128, "
@@ -723,7 +735,7 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
-        res = run_reference(args, rank)
+        res = run_reference(args, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
         return
