@@ -24,6 +24,8 @@ primitives (matmul, stable sort, exp, log) as steps and no blocking or fusion:
                       visible tokens of the incomplete tail block are read directly).
 * ``hi_select_row``   LongCat page §"机制三：层级索引（HI）": page scores from the sub-blocks' mean
                       keys, top-M pages, then the token score and arg topK on the recalled tokens.
+* ``msa_select_row``  lecture "从两本账看懂长上下文注意力", §"MiniMax Sparse Attention": block score = max of
+                      its tokens' index scores, per-group top-k blocks, the local block always kept.
 * ``lse_merge``       LongCat page §"训练与 kernel：混合稀疏注意力算子（HFA）": partial attentions merged by
                       online-softmax (log-sum-exp) rescaling.
 * ``softmax_attention`` / ``sparse_mla_attn``
@@ -250,6 +252,42 @@ def hi_select_row(q_I_b: np.ndarray, w_b: np.ndarray, k_I: np.ndarray, q_pos: in
     kth = float(cand_sc[order[min(K, cand.size) - 1]]) if cand.size else -np.inf
     sel = np.union1d(np.union1d(s_sink, take), s_swa)
     return sel.astype(np.int64), kth, mth_page, recalled
+
+
+# ---------------------------------------------------------------------------
+# MSA: group-wise block selection
+# ---------------------------------------------------------------------------
+
+
+def msa_select_row(q_I_b: np.ndarray, w_b: np.ndarray, k_I: np.ndarray, q_pos: int, G: int, block: int, KB: int):
+    """One query of group-wise block selection: per group g, (sorted positions, KB-th block score).
+
+    Lecture "从两本账看懂长上下文注意力", section "MiniMax Sparse Attention": the index branch scores tokens,
+    a block's score is the max of its tokens' scores, each GQA group picks its own top-k blocks (its query
+    heads share them) and the current local block is always kept.
+
+    Readings: group g's token score is the indexer formula over its own index heads
+    j in [g*H_I/G, (g+1)*H_I/G); the ranked blocks are those entirely before the local block (the block
+    holding q_pos), i.e. c < q_pos // block; the top-KB of them (stable sort on descending score: ties ->
+    lower block) plus the local block's visible tokens {block*(q_pos//block) .. q_pos} form the group's set.
+    """
+    q_pos = int(q_pos)
+    H = q_I_b.shape[0]
+    hg = H // G
+    lb = q_pos // block
+    out = []
+    for g in range(G):
+        sl = slice(g * hg, (g + 1) * hg)
+        sc = index_score(np.asarray(q_I_b)[None, sl], np.asarray(w_b)[None, sl], np.asarray(k_I)[: lb * block],
+                         np.array([lb * block - 1]))[0] if lb > 0 else np.zeros(0)
+        bscore = sc.reshape(lb, block).max(axis=1) if lb > 0 else np.zeros(0)
+        order = np.argsort(-bscore, kind="stable")
+        chosen = order[: min(KB, lb)]
+        kth = float(bscore[chosen[-1]]) if chosen.size else -np.inf
+        pos = (chosen[:, None] * block + np.arange(block)[None, :]).reshape(-1)
+        pos = np.union1d(pos, np.arange(lb * block, q_pos + 1)).astype(np.int64)
+        out.append((pos, kth))
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -430,3 +430,46 @@ def test_lse_merge_equals_attention_over_the_union(cuts):
 def test_lse_merge_of_empty_parts_is_empty():
     o, lse = O.lse_merge([(np.zeros((3, 4)), np.full(3, -np.inf))] * 2)
     assert np.all(o == 0) and np.all(lse == -np.inf)
+
+
+# --------------------------------------------------------------------------------------------
+# MSA group-wise block selection
+# --------------------------------------------------------------------------------------------
+
+
+def test_msa_one_group_is_block_topk_of_max_pooled_scores():
+    """G = 1: the block ranking of max-pooled flat token scores, by a loop-level brute force."""
+    rng = np.random.default_rng(21)
+    q, w, k = rng.normal(size=(4, 8)), rng.uniform(0.1, 1, size=4), rng.normal(size=(200, 8))
+    q_pos, block, KB = 171, 16, 3
+    (pos, kth), = O.msa_select_row(q, w, k, q_pos, G=1, block=block, KB=KB)
+
+    def tok(s):
+        return sum(w[j] * max(0.0, float(q[j] @ k[s])) for j in range(4))
+
+    lb = q_pos // block
+    bs = {c: max(tok(s) for s in range(c * block, c * block + block)) for c in range(lb)}
+    keep = sorted(bs, key=lambda c: (-bs[c], c))[:KB]
+    want = sorted({c * block + i for c in keep for i in range(block)} | set(range(lb * block, q_pos + 1)))
+    assert pos.tolist() == want and kth == pytest.approx(bs[keep[-1]], rel=1e-12)
+
+
+def test_msa_groups_use_their_own_index_heads():
+    """Group g's selection depends only on index heads of group g (the others are scrambled freely)."""
+    rng = np.random.default_rng(22)
+    q, w, k = rng.normal(size=(8, 8)), rng.uniform(0.1, 1, size=8), rng.normal(size=(300, 8))
+    a = O.msa_select_row(q, w, k, 299, G=4, block=16, KB=4)
+    q2, w2 = q.copy(), w.copy()
+    q2[2:], w2[2:] = rng.normal(size=(6, 8)), rng.uniform(0.1, 1, size=6)  # heads of groups 1..3 only
+    b = O.msa_select_row(q2, w2, k, 299, G=4, block=16, KB=4)
+    assert np.array_equal(a[0][0], b[0][0]) and a[0][1] == b[0][1]
+    single = O.msa_select_row(q[0:2], w[0:2], k, 299, G=1, block=16, KB=4)[0]
+    assert np.array_equal(a[0][0], single[0])
+
+
+def test_msa_local_block_only_near_the_start():
+    """No complete block before the query: only the local block's visible tokens."""
+    rng = np.random.default_rng(23)
+    q, w, k = rng.normal(size=(2, 4)), rng.uniform(size=2), rng.normal(size=(40, 4))
+    (pos, kth), = O.msa_select_row(q, w, k, 9, G=1, block=16, KB=2)
+    assert pos.tolist() == list(range(10)) and kth == -np.inf
