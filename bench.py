@@ -327,6 +327,38 @@ class HiStep:
         self.lsa.lsa_sparse_attn(self.q, self.kv, self.idx, self.cnt, self.wl.scale, self.out, self.lse, self.ws_a)
 
 
+class MsaStep:
+    """Group-wise block selection (G groups of the 64 index heads, each keeping its top-KB 128-token blocks by
+    max-pooled token score plus the local block) and each query-head group's attention over its own blocks."""
+
+    def __init__(self, wl: S.Workload, device, G: int, KB: int):
+        import sparse_long_context_lightning_b200 as lsa
+
+        self.lsa, self.wl, self.G, self.KB = lsa, wl, G, KB
+        q_I, w = S.index_queries(wl, "cpu")
+        self.k = S.index_keys(wl, q_I, device)
+        self.q_I, self.w = q_I.to(device), w.to(device)
+        self.q_pos = wl.q_pos().to(device)
+        ld = (G * KB + 1) * 128
+        self.idx = torch.empty(wl.B, ld, dtype=torch.int32, device=device)
+        self.gmask = torch.empty(wl.B, ld, dtype=torch.uint8, device=device)
+        self.cnt = torch.empty(wl.B, dtype=torch.int32, device=device)
+        self.ws = lsa.workspace(lsa.lsa_msa_workspace_size(wl.B, wl.L, G, KB), device)
+        self.q = S.attn_queries(wl, device)
+        self.kv = S.latent_cache(wl, device)
+        self.out = torch.empty(wl.B, wl.H, wl.d_v, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(wl.B, wl.H, device=device)
+        self.ws_a = lsa.workspace(lsa.lsa_msa_attn_workspace_size(wl.B, ld, G), device)
+
+    def select(self):
+        self.lsa.lsa_msa_select(self.q_I, self.w, self.k, self.G, self.KB, self.q_pos, self.idx, self.gmask,
+                                self.cnt, self.ws)
+
+    def attn(self):
+        self.lsa.lsa_msa_attn(self.q, self.kv, self.idx, self.gmask, self.cnt, self.G, self.wl.scale, self.out,
+                              self.lse, self.ws_a)
+
+
 def _time_stages(stages, l2_flush, iters):
     """Mean CUDA-event time (ms) of each callable in `stages`, run in order, L2 flushed before each pass."""
     stream = torch.cuda.current_stream()
@@ -427,6 +459,28 @@ def long_context_configs(device, l2_flush, iters: int = 10):
                     "dynamic budget), H=128",
         "stages": {"attn_single_pass": _stage(st[0], at_bytes), "attn_hybrid": _stage(st[1], at_bytes)}}
     del step, ws_h
+    torch.cuda.empty_cache()
+    # group-wise block selection at 128K: 8 groups, each its top-16 blocks of 128 (2048 tokens per group) + the
+    # local block; the attention stage reads each group's rows for its 16 query heads
+    wl = S.WORKLOADS["decode128k"]
+    mstep = MsaStep(wl, device, G=8, KB=16)
+    st = _time_stages([mstep.select, mstep.attn], l2_flush, iters)
+    B, L = wl.B, wl.L
+    nblk = L // 128
+    sel_bytes = L * wl.d_I * 2 + B * 8 * nblk * 4 + B * mstep.idx.shape[1] * 5
+    sel_flops = 2.0 * B * wl.H_I * wl.d_I * L
+    rows = float(mstep.cnt.sum().item())
+    gm = mstep.gmask.cpu().numpy()
+    grp_rows = float(sum(int(((gm[b, : int(c)] >> g) & 1).sum()) for b, c in enumerate(mstep.cnt.cpu().tolist())
+                         for g in range(8)))
+    at_bytes = rows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
+    res["decode128k_msa"] = {
+        "workload": "B=16 decode queries, L=131072, bf16 indexer (H_I=64 as 8 groups of 8 heads), top-16 blocks of "
+                    "128 per group + the local block, H=128 (8 groups of 16 query heads)",
+        "stages": {"msa_select": _stage(st[0], sel_bytes, sel_flops, bf16), "attn": _stage(st[1], at_bytes)},
+        "union_rows_per_query": round(rows / B, 1), "group_rows_per_query": round(grp_rows / B, 1),
+        "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
+    del mstep
     torch.cuda.empty_cache()
     for name in ("decode1m_mb", "flat10m"):
         wl = S.WORKLOADS[name]

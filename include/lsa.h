@@ -232,6 +232,47 @@ int lsa_hi_select(const void* q_idx, const float* w, const void* k_idx, int64_t 
 size_t lsa_hi_workspace_size(int64_t B, int64_t L, int P, int Bsub, int M, int K, int sink, int window);
 
 /*
+ * lsa_msa_select -- group-wise block selection.
+ *   Source: lecture "从两本账看懂长上下文注意力", section "MiniMax Sparse Attention": the index branch scores
+ *   tokens, a block's score is the max of its tokens' scores, each GQA group picks its own top-k blocks (the
+ *   group's query heads share them) and the current local block is always kept.
+ *
+ *   Blocks of 128 tokens.  For each query b and group g (index heads [g*64/G, (g+1)*64/G)):
+ *     token score  = sum_{j in g} w[b,j] max(0, q[b,j,:] . k[s,:])           (fp32 from bf16)
+ *     block score  = max over the block's tokens (blocks before the local block, lb = q_pos[b] / 128)
+ *     kept(b, g)   = the min(KB, lb) blocks with the largest block score (ties -> lower block), plus lb
+ *   idx row b: the tokens of the union of kept(b, g) over g, ascending (the local block up to q_pos[b]);
+ *   gmask[b*idx_ld + i]: bit g set when group g kept the block of idx[b*idx_ld + i]; count[b] entries.
+ *   q_idx [B, 64, 128] bf16, w [B, 64] fp32, k_idx [L, 128] bf16; G in {1, 2, 4, 8}; G*KB + 1 <= 1024;
+ *   L >= 128.  idx int32 / gmask uint8 [B, idx_ld], idx_ld >= (G*KB + 1) * 128.
+ *   ws: lsa_msa_workspace_size(B, L, G, KB) bytes.  The block scores come from the indexer's tensor-core
+ *   kernel with a grouped block-max epilogue (no token scores are written).
+ */
+int lsa_msa_select(const void* q_idx, const float* w, const void* k_idx, int64_t B, int H_I, int d_I,
+                   int64_t L, int G, int KB, const int64_t* q_pos, int32_t* idx, uint8_t* gmask,
+                   int64_t idx_ld, int32_t* count, void* ws, size_t ws_bytes, void* stream);
+
+/* lsa_msa_workspace_size -- scratch bytes of lsa_msa_select; (size_t)-1 for invalid sizes. */
+size_t lsa_msa_workspace_size(int64_t B, int64_t L, int G, int KB);
+
+/*
+ * lsa_msa_attn -- attention over a group-wise selection: each head attends to its own group's rows.
+ *   Source: the same section (a group's query heads share its blocks).
+ *   out[b,h] / lse[b,h] = lsa_sparse_attn's attention of head h (group g = h / (128 / G)) over the entries of
+ *   idx[b, :count[b]] whose gmask has bit g.  Each group's rows are compacted first (k_msa_group_rows), then
+ *   the (query, group) pairs run as B*G queries of 128 / G heads (q, out and lse viewed accordingly).  Head
+ *   groups of fewer than 128 heads run on the CUDA-core attention kernel; the tensor-core "KV-outer" form
+ *   (each KV tile loaded once for every group that kept it) is not built.
+ *   H = 128, G in {1, 2, 4, 8}.  ws: lsa_msa_attn_workspace_size(B, idx_ld, G) bytes.
+ */
+int lsa_msa_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, const uint8_t* gmask,
+                 int64_t idx_ld, const int32_t* count, int64_t B, int H, int d_qk, int d_v, int G,
+                 float scale, void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* lsa_msa_attn_workspace_size -- scratch bytes of lsa_msa_attn; (size_t)-1 for invalid sizes. */
+size_t lsa_msa_attn_workspace_size(int64_t B, int64_t idx_ld, int G);
+
+/*
  * lsa_bucket_select_noalloc -- lsa_bucket_select for callers that cannot allocate device memory.
  *   The pages have no counterpart: this is a packaging variant of lsa_bucket_select.
  *

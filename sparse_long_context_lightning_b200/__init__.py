@@ -44,6 +44,10 @@ SIGNATURES = {
     "lsa_hi_workspace_size": (_SZ, [_I64, _I64, _I32, _I32, _I32, _I32, _I32, _I32]),
     "lsa_hybrid_attn": (_I32, [_P, _P, _I64, _P, _I64, _P, _I64, _I32, _I32, _I32, _I32, _I32, _P, _F32, _P, _P, _P,
                                _SZ, _P]),
+    "lsa_msa_select": (_I32, [_P, _P, _P, _I64, _I32, _I32, _I64, _I32, _I32, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
+    "lsa_msa_workspace_size": (_SZ, [_I64, _I64, _I32, _I32]),
+    "lsa_msa_attn_workspace_size": (_SZ, [_I64, _I64, _I32]),
+    "lsa_msa_attn": (_I32, [_P, _P, _I64, _P, _P, _I64, _P, _I64, _I32, _I32, _I32, _I32, _F32, _P, _P, _P, _SZ, _P]),
     "lsa_sparse_attn": (_I32, [_P, _P, _I64, _P, _I64, _P, _I64, _I32, _I32, _I32, _F32, _P, _P, _P, _SZ, _P]),
     "lsa_workspace_size": (_SZ, [_I32, _I64, _I64, _I32, _I32, _I32, _I32]),
     "lsa_strerror": (ctypes.c_char_p, [_I32]),
@@ -210,6 +214,33 @@ def lsa_hybrid_attn(q, kv, idx, count, sink, window, q_pos, scale, out, lse=None
                                         _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                         _stream(stream))
     _check("lsa_hybrid_attn", st)
+
+
+def lsa_msa_workspace_size(B, L, G, KB):
+    return load_library().lsa_msa_workspace_size(B, L, G, KB)
+
+
+def lsa_msa_select(q_idx, w, k_idx, G, KB, q_pos, idx, gmask, count, ws, stream=None):
+    """Group-wise block selection: per group of index heads, top-KB 128-token blocks by max-pooled score."""
+    B, H_I, d_I = q_idx.shape
+    st = load_library().lsa_msa_select(_ptr(q_idx), _ptr(w), _ptr(k_idx), B, H_I, d_I, k_idx.shape[0], G, KB,
+                                       _ptr(q_pos), _ptr(idx), _ptr(gmask), idx.stride(0), _ptr(count), _ptr(ws),
+                                       0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("lsa_msa_select", st)
+
+
+def lsa_msa_attn_workspace_size(B, idx_ld, G):
+    return load_library().lsa_msa_attn_workspace_size(B, idx_ld, G)
+
+
+def lsa_msa_attn(q, kv, idx, gmask, count, G, scale, out, lse=None, ws=None, stream=None):
+    """Attention over a group-wise selection: head h attends to the rows its group kept."""
+    B, H, d_qk = q.shape
+    d_v = out.shape[-1]
+    st = load_library().lsa_msa_attn(_ptr(q), _ptr(kv), kv.shape[0], _ptr(idx), _ptr(gmask), idx.stride(0),
+                                     _ptr(count), B, H, d_qk, d_v, G, float(scale), _ptr(out), _ptr(lse), _ptr(ws),
+                                     0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("lsa_msa_attn", st)
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:

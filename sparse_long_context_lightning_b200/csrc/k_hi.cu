@@ -101,6 +101,124 @@ __global__ void __launch_bounds__(PE_THREADS) k_page_expand(const int32_t* __res
   if (tid == 0) ccount[b] = nsink + ndyn + nwin;
 }
 
+// Group-wise block selection, per query b (one CTA): the entries are every group's kept blocks
+// (kept[(b G + g) kept_ld + j], j < kcnt) and the local block (all groups); the distinct blocks, ascending,
+// expand to their tokens (the local block up to q_pos), each token carrying the bit mask of the groups that
+// chose its block.  Blocks before the local one are complete and entirely visible.
+__global__ void __launch_bounds__(PE_THREADS) k_msa_expand(const int32_t* __restrict__ kept, int64_t kept_ld,
+                                                           const int32_t* __restrict__ kcnt, int G, int block,
+                                                           const int64_t* __restrict__ q_pos,
+                                                           int32_t* __restrict__ idx, uint8_t* __restrict__ gmask,
+                                                           int64_t idx_ld, int32_t* __restrict__ count) {
+  __shared__ int32_t ent_blk[PE_THREADS];
+  __shared__ uint32_t ent_bit[PE_THREADS];
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int qp = static_cast<int>(q_pos[b]);
+  const int lb = qp / block;
+  // entries: group g's kept blocks at [g kept_ld, g kept_ld + kcnt), the local block last
+  const int n_ent = G * static_cast<int>(kept_ld) + 1;
+  for (int e = tid; e < n_ent; e += PE_THREADS) {
+    int blk = -1;
+    uint32_t bit = 0u;
+    if (e == n_ent - 1) {
+      blk = lb;
+      bit = (1u << G) - 1u;
+    } else {
+      const int g = e / static_cast<int>(kept_ld), j = e % static_cast<int>(kept_ld);
+      if (j < kcnt[b * G + g]) {
+        blk = kept[(static_cast<int64_t>(b) * G + g) * kept_ld + j];
+        bit = 1u << g;
+      }
+    }
+    ent_blk[e] = blk;
+    ent_bit[e] = bit;
+  }
+  __syncthreads();
+  // a distinct block is written by its first entry: mask = OR over its entries, rank = distinct blocks below
+  int nd = 0;  // distinct blocks in total (every thread counts: uniform)
+  for (int e = 0; e < n_ent; ++e) {
+    const int x = ent_blk[e];
+    bool first = x >= 0;
+    for (int f = 0; first && f < e; ++f) first = ent_blk[f] != x;
+    nd += first;
+  }
+  int32_t* row = idx + static_cast<int64_t>(b) * idx_ld;
+  uint8_t* mrow = gmask + static_cast<int64_t>(b) * idx_ld;
+  for (int e = tid; e < n_ent; e += PE_THREADS) {
+    const int x = ent_blk[e];
+    if (x < 0) continue;
+    bool first = true;
+    uint32_t mask = 0u;
+    int rank = 0;
+    for (int f = 0; f < n_ent; ++f) {
+      const int y = ent_blk[f];
+      if (y == x) {
+        mask |= ent_bit[f];
+        if (f < e) first = false;
+      }
+    }
+    if (!first) continue;
+    for (int f = 0; f < n_ent; ++f) {  // distinct blocks below x
+      const int y = ent_blk[f];
+      if (y >= 0 && y < x) {
+        bool fy = true;
+        for (int f2 = 0; fy && f2 < f; ++f2) fy = ent_blk[f2] != y;
+        rank += fy;
+      }
+    }
+    // every block below the local one is complete: the offset is rank * block
+    const int lo = x * block, hi = min(x * block + block, qp + 1);
+    for (int t = lo; t < hi; ++t) {
+      row[rank * block + (t - lo)] = t;
+      mrow[rank * block + (t - lo)] = static_cast<uint8_t>(mask);
+    }
+  }
+  if (tid == 0) count[b] = (nd - 1) * block + (qp + 1 - lb * block);
+}
+
+// out[b G + g] = q_pos[b] + delta (the per-(query, group) positions of group-wise selection)
+__global__ void k_shift_qpos(const int64_t* __restrict__ q_pos, int64_t n, int G, int64_t delta,
+                             int64_t* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = q_pos[i / G] + delta;
+}
+
+// Each group's own rows out of a group-wise selection: grows[(b G + g) idx_ld + i] = the i-th entry of
+// idx[b, :count[b]] whose gmask has bit g (ascending, as in the union row); gcount[b G + g] of them.  One
+// CTA per (query, group): an ordered block scan of the bit.
+__global__ void __launch_bounds__(PS_THREADS) k_msa_group_rows(const int32_t* __restrict__ idx,
+                                                               const uint8_t* __restrict__ gmask, int64_t idx_ld,
+                                                               const int32_t* __restrict__ count, int G,
+                                                               int32_t* __restrict__ grows,
+                                                               int32_t* __restrict__ gcount) {
+  __shared__ uint32_t wsum[PS_THREADS / 32];
+  const int bg = blockIdx.x;
+  const int b = bg / G, g = bg % G;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = min(static_cast<int64_t>(max(count[b], 0)), idx_ld);
+  const int32_t* row = idx + static_cast<int64_t>(b) * idx_ld;
+  const uint8_t* mrow = gmask + static_cast<int64_t>(b) * idx_ld;
+  int32_t* out = grows + static_cast<int64_t>(bg) * idx_ld;
+  uint32_t base = 0;
+  for (int i0 = 0; i0 < n; i0 += PS_THREADS) {
+    const int i = i0 + tid;
+    const bool mine = i < n && ((mrow[i] >> g) & 1u);
+    const uint32_t bal = __ballot_sync(0xffffffffu, mine);
+    if (lane == 0) wsum[warp] = __popc(bal);
+    __syncthreads();
+    uint32_t before = 0, total = 0;
+    for (int w = 0; w < PS_THREADS / 32; ++w) {
+      before += w < warp ? wsum[w] : 0u;
+      total += wsum[w];
+    }
+    if (mine) out[base + before + __popc(bal & ((1u << lane) - 1u))] = row[i];
+    base += total;
+    __syncthreads();  // wsum is rewritten by the next step
+  }
+  if (tid == 0) gcount[bg] = static_cast<int32_t>(base);
+}
+
 }  // namespace
 
 int launch_page_sum(const float* sub, int64_t sub_ld, int64_t nsub, int P, int Bsub, int64_t npages, int64_t B,
@@ -118,6 +236,30 @@ int launch_page_expand(const int32_t* kept, int64_t kept_ld, const int32_t* kcnt
   if (kept_ld > PE_THREADS) return LSA_ERR_INVALID_ARG;
   k_page_expand<<<static_cast<unsigned>(B), PE_THREADS, 0, s>>>(kept, kept_ld, kcnt, P, Bsub, sink, window, q_pos,
                                                                 cand, cand_ld, ccount);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_msa_expand(const int32_t* kept, int64_t kept_ld, const int32_t* kcnt, int G, int block,
+                      const int64_t* q_pos, int64_t B, int32_t* idx, uint8_t* gmask, int64_t idx_ld, int32_t* count,
+                      cudaStream_t s) {
+  if (B == 0) return LSA_OK;
+  if (G * kept_ld + 1 > PE_THREADS) return LSA_ERR_INVALID_ARG;
+  k_msa_expand<<<static_cast<unsigned>(B), PE_THREADS, 0, s>>>(kept, kept_ld, kcnt, G, block, q_pos, idx, gmask,
+                                                               idx_ld, count);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_shift_qpos(const int64_t* q_pos, int64_t B, int G, int64_t delta, int64_t* out, cudaStream_t s) {
+  const int64_t n = B * G;
+  if (n == 0) return LSA_OK;
+  k_shift_qpos<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, s>>>(q_pos, n, G, delta, out);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_msa_group_rows(const int32_t* idx, const uint8_t* gmask, int64_t idx_ld, const int32_t* count, int64_t B,
+                          int G, int32_t* grows, int32_t* gcount, cudaStream_t s) {
+  if (B == 0) return LSA_OK;
+  k_msa_group_rows<<<static_cast<unsigned>(B * G), PS_THREADS, 0, s>>>(idx, gmask, idx_ld, count, G, grows, gcount);
   return cuda_status(cudaGetLastError());
 }
 

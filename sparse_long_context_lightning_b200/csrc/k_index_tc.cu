@@ -83,6 +83,53 @@ __device__ __forceinline__ void relu_weighted_sum64(const float* w, const uint32
   }
 }
 
+// order-preserving map of floats onto unsigned keys (0 lies below every float) and back
+__device__ __forceinline__ uint32_t float_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Grouped block maxima of one tile for one warp (32 keys x the 64 heads of query b): the G group sums of each
+// key, their max over the warp's keys, then over the tile's four lane quarters through shared memory -- the
+// quarter that contributes last writes the G block scores and clears the slot (its next user is four tiles
+// later, which no warp reaches before every warp has finished this tile).
+template <int G>
+__device__ __forceinline__ void block_max_epilogue(const IxArgs& a, const float* w, const uint32_t (&r0)[32],
+                                                   const uint32_t (&r1)[32], int s, int b, int tile, int lane,
+                                                   uint32_t* mx, uint32_t* cnt) {
+  constexpr int GW = 64 / G;  // heads per group
+  float acc[G];
+  #pragma unroll
+  for (int g = 0; g < G; ++g) acc[g] = 0.f;
+  #pragma unroll
+  for (int c = 0; c < 32; ++c) acc[c / GW] = fmaf(w[c], fmaxf(__uint_as_float(r0[c]), 0.f), acc[c / GW]);
+  #pragma unroll
+  for (int c = 0; c < 32; ++c)
+    acc[(32 + c) / GW] = fmaf(w[32 + c], fmaxf(__uint_as_float(r1[c]), 0.f), acc[(32 + c) / GW]);
+  const bool valid = b < a.B && s < a.L && s <= a.q_pos[b];
+  #pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float v = valid ? acc[g] : -INFINITY;
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) atomicMax(&mx[g], float_key(v));
+  }
+  if (lane == 0) {
+    __threadfence_block();
+    if (atomicAdd(cnt, 1u) == 3u) {
+      #pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const uint32_t k = atomicExch(&mx[g], 0u);
+        if (b < a.B) a.scores[(static_cast<int64_t>(b) * G + g) * a.ld + tile] = key_float(k);
+      }
+      atomicExch(cnt, 0u);
+    }
+  }
+}
+
 // The chunk's 256 (query, head) weights (times the FP8 query scales) into shared memory, by the 512 epilogue
 // threads (e = 0..511), which then synchronise among themselves (named barrier 1).
 __device__ __forceinline__ void load_weights(float* wsm, const IxArgs& a, int b0, int e) {
@@ -98,10 +145,15 @@ __device__ __forceinline__ void load_weights(float* wsm, const IxArgs& a, int b0
 // SPLITS > 1 (bf16 only): each key is the sum of SPLITS bf16 rows, split_rows apart in the key matrix (the
 // exact three-part bf16 split of an fp32 key): a tile's accumulator takes SPLITS consecutive key stages
 // before its epilogue.  q_pos == nullptr: no causal mask.
-template <bool FP8, int SPLITS>
+// G > 0 (bf16, H_I = 64): grouped block maxima instead of token scores -- for each query b, group g of index
+// heads [8g', ...) (64 / G heads each) and 128-key tile t, scores[(b G + g) ld + t] = the max over the tile's keys
+// s <= q_pos[b] of sum_{j in g} w_j ReLU(q_j . k_s) (-inf when none): the block scores of group-wise block
+// selection, without writing token scores.
+template <bool FP8, int SPLITS, int G>
 __global__ void __launch_bounds__(IX_THREADS, 1)
     k_index_score_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q, IxArgs a) {
   static_assert(SPLITS == 1 || !FP8, "split keys are bf16");
+  static_assert(G == 0 || (!FP8 && SPLITS == 1 && 64 % G == 0), "grouped block maxima: bf16 keys, H_I = 64");
   // every global access of this kernel comes after the previous kernel of the stream has completed
   sm100::pdl_wait();
   sm100::pdl_launch_dependents();
@@ -120,6 +172,10 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qfull + 1);
   // [256] weights of this chunk's (query, head) pairs, 16-byte aligned: the epilogue reads them as float4
   float* wsm = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(bars) + 256);
+  // G > 0: running block maxima (order keys) per [tile mod 4][column group][group] and the number of lane
+  // quarters that have contributed per [tile mod 4][column group]
+  uint32_t* gmax = reinterpret_cast<uint32_t*>(wsm + IX_CHUNK_N);
+  uint32_t* gcnt = gmax + 4 * 4 * 8;
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -223,6 +279,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..17)
     // warp e handles TMEM lanes 32*(warp % 4) .. +31 (its keys) and chunk columns [64*(e/4), +64)
+    if (G > 0 && tid - 64 < 4 * 4 * 8 + 16) gmax[tid - 64] = 0u;  // cleared before the epilogue barrier
     load_weights(wsm, a, b0, tid - 64);  // off the producer's critical path: needed at the first tfull
     const int ew = warp - 2;
     const int quarter = warp & 3;
@@ -244,6 +301,11 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);  // the accumulator columns are in registers now
       const int s = (t_begin + i) * IX_TILE_M + quarter * 32 + lane;
+      if constexpr (G > 0) {
+        block_max_epilogue<G>(a, wsm + col0, r0, r1, s, b0 + (col0 >> 6), t_begin + i, lane,
+                              gmax + ((i & 3) * 4 + (ew >> 2)) * 8, gcnt + (i & 3) * 4 + (ew >> 2));
+        continue;
+      }
       const float ks = (FP8 && s < a.L) ? a.k_scale[s] : 1.f;
       float acc0, acc1;
       relu_weighted_sum64(wsm + col0, r0, r1, acc0, acc1);
@@ -267,7 +329,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   }
 }
 
-template <bool FP8, int SPLITS>
+template <bool FP8, int SPLITS, int G = 0>
 int launch_tc(const void* q, const float* q_scale, const float* w, const void* k, const float* k_scale, int64_t B,
               int H_I, int64_t L, const int64_t* q_pos, float* scores, int64_t ld, cudaStream_t s) {
   using C = IxCfg<FP8>;
@@ -295,9 +357,10 @@ int launch_tc(const void* q, const float* q_scale, const float* w, const void* k
   a.tiles_per_range = static_cast<int>(cdiv(a.ntiles, ranges));
   a.split_rows = static_cast<int>(L);
   ranges = static_cast<int>(cdiv(a.ntiles, a.tiles_per_range));
-  LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_index_score_tc<FP8, SPLITS>), C::SMEM));
+  LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_index_score_tc<FP8, SPLITS, G>), C::SMEM));
   const int64_t grid = static_cast<int64_t>(a.n_chunks) * ranges;
-  return cuda_status(launch_pdl(k_index_score_tc<FP8, SPLITS>, dim3(static_cast<unsigned>(grid)), dim3(IX_THREADS), C::SMEM, s, 0u,
+  return cuda_status(launch_pdl(k_index_score_tc<FP8, SPLITS, G>, dim3(static_cast<unsigned>(grid)), dim3(IX_THREADS),
+                                C::SMEM, s, 0u,
                                 tk, tq, a));
 }
 
@@ -370,6 +433,20 @@ int launch_index_score(const void* q, const float* q_scale, const float* w, cons
   const bool fp8 = dtype == LSA_FP8_E4M3;
   if (fp8) return launch_tc<true, 1>(q, q_scale, w, k, k_scale, B, H_I, L, q_pos, scores, ld, s);
   return launch_tc<false, 1>(q, q_scale, w, k, k_scale, B, H_I, L, q_pos, scores, ld, s);
+}
+
+// Grouped block maxima (group-wise block selection): scores[(b G + g) ld + t] for 128-key tiles t; bf16,
+// d_I = 128, H_I = 64, G in {1, 2, 4, 8}; the caller checks the shapes.
+int launch_block_max_tc(const void* q, const float* w, const void* k, int64_t B, int64_t L, int G,
+                        const int64_t* q_pos, float* scores, int64_t ld, cudaStream_t s) {
+  if (B == 0 || L == 0) return LSA_OK;
+  switch (G) {
+    case 1: return launch_tc<false, 1, 1>(q, nullptr, w, k, nullptr, B, 64, L, q_pos, scores, ld, s);
+    case 2: return launch_tc<false, 1, 2>(q, nullptr, w, k, nullptr, B, 64, L, q_pos, scores, ld, s);
+    case 4: return launch_tc<false, 1, 4>(q, nullptr, w, k, nullptr, B, 64, L, q_pos, scores, ld, s);
+    case 8: return launch_tc<false, 1, 8>(q, nullptr, w, k, nullptr, B, 64, L, q_pos, scores, ld, s);
+    default: return LSA_ERR_UNSUPPORTED;
+  }
 }
 
 // Representative scores on the tensor cores: key n = split[n] + split[NB + n] + split[2 NB + n], the exact

@@ -86,6 +86,26 @@ static HiLayout hi_ws_layout(int64_t B, int64_t L, int P, int Bsub, int M, int K
   return h;
 }
 
+// Scratch layout of lsa_msa_select: block scores [B G, ld_nb] fp32 | per-(query, group) positions [B G] int64 |
+// kept blocks [B G, KB] int32 | kept count [B G] int32.
+struct MsaLayout {
+  int64_t nb, ld_nb;
+  size_t o_qp, o_kept, o_kcnt, total;
+};
+static MsaLayout msa_ws_layout(int64_t B, int64_t L, int G, int KB) {
+  MsaLayout m;
+  m.nb = cdiv(L, 128);
+  m.ld_nb = (m.nb + 3) / 4 * 4;
+  size_t o = align_up(static_cast<size_t>(B) * G * m.ld_nb * 4, 256);
+  m.o_qp = o;
+  o = align_up(o + static_cast<size_t>(B) * G * 8, 256);
+  m.o_kept = o;
+  o = align_up(o + static_cast<size_t>(B) * G * KB * 4, 256);
+  m.o_kcnt = o;
+  m.total = align_up(o + static_cast<size_t>(B) * G * 4, 256);
+  return m;
+}
+
 }  // namespace lsa
 
 using namespace lsa;
@@ -290,6 +310,68 @@ int lsa_hybrid_attn(const void* q, const void* kv, int64_t L, const int32_t* idx
   LSA_CHECK_ARG(B <= 65535);
   return launch_hybrid_attn(q, kv, L, idx, idx_ld, count, B, H, sink, window, q_pos, scale, out, lse, ws, ws_bytes,
                             static_cast<cudaStream_t>(stream));
+}
+
+size_t lsa_msa_workspace_size(int64_t B, int64_t L, int G, int KB) {
+  if (B < 0 || L < 1 || G < 1 || KB < 1) return static_cast<size_t>(-1);
+  return msa_ws_layout(B, L, G, KB).total;
+}
+
+int lsa_msa_select(const void* q_idx, const float* w, const void* k_idx, int64_t B, int H_I, int d_I, int64_t L,
+                   int G, int KB, const int64_t* q_pos, int32_t* idx, uint8_t* gmask, int64_t idx_ld,
+                   int32_t* count, void* ws, size_t ws_bytes, void* stream) {
+  LSA_CHECK_ARG(B >= 0 && L >= 1 && L < (int64_t(1) << 31) && KB >= 1 && G >= 1);
+  if (d_I != 128 || H_I != 64 || (G != 1 && G != 2 && G != 4 && G != 8) || L < 128) return LSA_ERR_UNSUPPORTED;
+  LSA_CHECK_ARG(static_cast<int64_t>(G) * KB + 1 <= 1024);
+  LSA_CHECK_ARG(idx_ld >= (static_cast<int64_t>(G) * KB + 1) * 128);
+  if (B == 0) return LSA_OK;
+  LSA_CHECK_ARG(B <= 65535 / G);
+  LSA_CHECK_ARG(q_idx && w && k_idx && q_pos && idx && gmask && count && aligned16(q_idx) && aligned16(k_idx));
+  const MsaLayout m = msa_ws_layout(B, L, G, KB);
+  if (ws == nullptr || !aligned256(ws) || ws_bytes < m.total) return LSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  float* bs = reinterpret_cast<float*>(base);
+  int64_t* qp1 = reinterpret_cast<int64_t*>(base + m.o_qp);
+  int32_t* kept = reinterpret_cast<int32_t*>(base + m.o_kept);
+  int32_t* kcnt = reinterpret_cast<int32_t*>(base + m.o_kcnt);
+  // block scores per (query, group), fused into the indexer's epilogue; then per (query, group) the top-KB of
+  // the blocks before the local one (MODE_BLOCKS ranks c < (pos + 1) / 128 with pos = q_pos - 1)
+  int st = launch_block_max_tc(q_idx, w, k_idx, B, L, G, q_pos, bs, m.ld_nb, s);
+  if (st == LSA_OK) st = launch_shift_qpos(q_pos, B, G, -1, qp1, s);
+  if (st == LSA_OK) st = launch_topk_mode(bs, m.ld_nb, B * G, m.nb, KB, 0, 0, qp1, 2, 128, kept, KB, kcnt, KB, s);
+  if (st == LSA_OK) st = launch_msa_expand(kept, KB, kcnt, G, 128, q_pos, B, idx, gmask, idx_ld, count, s);
+  return st;
+}
+
+size_t lsa_msa_attn_workspace_size(int64_t B, int64_t idx_ld, int G) {
+  if (B < 0 || idx_ld < 0 || G < 1) return static_cast<size_t>(-1);
+  const size_t rows = align_up(static_cast<size_t>(B) * G * idx_ld * 4, 256);
+  return rows + align_up(static_cast<size_t>(B) * G * 4, 256) + sparse_attn_ws_bytes(B * G, idx_ld, 128 / G);
+}
+
+int lsa_msa_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, const uint8_t* gmask, int64_t idx_ld,
+                 const int32_t* count, int64_t B, int H, int d_qk, int d_v, int G, float scale, void* out, float* lse,
+                 void* ws, size_t ws_bytes, void* stream) {
+  LSA_CHECK_ARG(B >= 0 && L >= 1 && idx_ld >= 0 && idx_ld <= 65536);
+  if (d_qk != 576 || d_v != 512 || H != 128 || (G != 1 && G != 2 && G != 4 && G != 8)) return LSA_ERR_UNSUPPORTED;
+  if (B == 0) return LSA_OK;
+  LSA_CHECK_ARG(q && kv && idx && gmask && count && out);
+  LSA_CHECK_ARG(aligned16(q) && aligned16(kv) && aligned16(out) && B * G <= 65535);
+  if (ws == nullptr || !aligned256(ws) || ws_bytes < lsa_msa_attn_workspace_size(B, idx_ld, G)) return LSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  int32_t* grows = reinterpret_cast<int32_t*>(base);
+  const size_t o_cnt = align_up(static_cast<size_t>(B) * G * idx_ld * 4, 256);
+  int32_t* gcnt = reinterpret_cast<int32_t*>(base + o_cnt);
+  const size_t o_att = o_cnt + align_up(static_cast<size_t>(B) * G * 4, 256);
+  // each group's rows, then the attention of the (query, group) pairs: q / out / lse viewed as [B G, 128 / G, ...]
+  // (a group's heads are contiguous)
+  int st = launch_msa_group_rows(idx, gmask, idx_ld, count, B, G, grows, gcnt, s);
+  if (st == LSA_OK)
+    st = launch_sparse_attn(q, kv, L, grows, idx_ld, gcnt, B * G, 128 / G, scale, out, lse, base + o_att,
+                            ws_bytes - o_att, s);
+  return st;
 }
 
 size_t lsa_hi_workspace_size(int64_t B, int64_t L, int P, int Bsub, int M, int K, int sink, int window) {

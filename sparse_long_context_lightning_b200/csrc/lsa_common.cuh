@@ -171,6 +171,14 @@ size_t hybrid_attn_ws_bytes(int64_t B, int64_t idx_ld, int H, int sink, int wind
 int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
                        const int32_t* count, int64_t B, int H, float scale, void* out, float* lse,
                        void* ws, size_t ws_bytes, cudaStream_t s);
+int launch_msa_group_rows(const int32_t* idx, const uint8_t* gmask, int64_t idx_ld, const int32_t* count, int64_t B,
+                          int G, int32_t* grows, int32_t* gcount, cudaStream_t s);
+int launch_block_max_tc(const void* q, const float* w, const void* k, int64_t B, int64_t L, int G,
+                        const int64_t* q_pos, float* scores, int64_t ld, cudaStream_t s);
+int launch_msa_expand(const int32_t* kept, int64_t kept_ld, const int32_t* kcnt, int G, int block,
+                      const int64_t* q_pos, int64_t B, int32_t* idx, uint8_t* gmask, int64_t idx_ld, int32_t* count,
+                      cudaStream_t s);
+int launch_shift_qpos(const int64_t* q_pos, int64_t B, int G, int64_t delta, int64_t* out, cudaStream_t s);
 size_t sparse_attn_ws_bytes(int64_t B, int64_t kmax, int H);
 int attn_launches_per_call(int64_t B, int H);
 }  // namespace lsa

@@ -559,3 +559,72 @@ def test_hybrid_attn(H, sink, window):
         assert attn_rel_err(out[b], merged[0]) <= ATTN_REL
         assert np.abs(f64(lse[b]) - merged[1]).max() <= 1e-3
         assert attn_rel_err(out[b], f64(out1[b])) <= ATTN_REL
+
+
+# --------------------------------------------------------------------------------------------
+# MSA: group-wise block selection and the attention over it
+# --------------------------------------------------------------------------------------------
+
+
+def _msa_case(L, B, G, KB, q_pos):
+    wl = S.Workload("msa", L=L, B=B, H_I=64, d_I=128, K=KB * 128, H=128, needles="cos06", n_needles=L // 100)
+    q_I, w = S.index_queries(wl)
+    k = S.index_keys(wl, q_I, DEV)
+    ld = (G * KB + 1) * 128
+    idx = torch.full((B, ld), -7, dtype=torch.int32, device=DEV)
+    gm = torch.zeros(B, ld, dtype=torch.uint8, device=DEV)
+    cnt = torch.empty(B, dtype=torch.int32, device=DEV)
+    ws = lsa.workspace(lsa.lsa_msa_workspace_size(B, L, G, KB))
+    qp = torch.as_tensor(q_pos, dtype=torch.int64, device=DEV)
+    lsa.lsa_msa_select(q_I.to(DEV), w.to(DEV), k, G, KB, qp, idx, gm, cnt, ws)
+    torch.cuda.synchronize()
+    return q_I, w, k, qp, idx, gm, cnt
+
+
+@pytest.mark.parametrize("G,KB", [(8, 16), (1, 8), (4, 5)])
+def test_msa_select(G, KB):
+    """Each group's set (the union row's entries with its bit) against the oracle; blocks may differ only where
+    their score ties the KB-th within 1e-5."""
+    L, B = 40000 + 77, 4
+    q_pos = [L - 1, 20000, 127, 300]
+    q_I, w, k, _, idx, gm, cnt = _msa_case(L, B, G, KB, q_pos)
+    qf, wf, kf = f64(q_I), f64(w), f64(k)
+    idx_h, gm_h, cnt_h = idx.cpu().numpy(), gm.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(B):
+        row, m = idx_h[b, : cnt_h[b]], gm_h[b, : cnt_h[b]]
+        assert np.all(np.diff(row) > 0) and row.max() == q_pos[b]
+        want = O.msa_select_row(qf[b], wf[b], kf, q_pos[b], G, 128, KB)
+        for g in range(G):
+            got = row[(m >> g) & 1 == 1]
+            ref, kth = want[g]
+            if np.array_equal(got, ref):
+                continue
+            hg = 64 // G
+            for blk in np.unique(np.setxor1d(got, ref) // 128):
+                sc = O.index_score(qf[b][None, g * hg:(g + 1) * hg], wf[b][None, g * hg:(g + 1) * hg],
+                                   kf[blk * 128:(blk + 1) * 128], np.array([127]))[0].max()
+                assert abs(sc - kth) <= 1e-5 * abs(kth), (b, g, blk)
+
+
+def test_msa_attn():
+    """Head h attends to its group's rows only: against the oracle attention per head over those rows."""
+    L, B, G, KB = 40000 + 77, 3, 8, 16
+    q_pos = [L - 1, 20000, 5000]
+    _, _, _, _, idx, gm, cnt = _msa_case(L, B, G, KB, q_pos)
+    kv = S.normal_bf16(S.ST_KV, (L, 576), DEV)
+    q = S.normal_bf16(S.ST_Q, (B, 128, 576), DEV)
+    scale = 1 / math.sqrt(576)
+    out = torch.empty(B, 128, 512, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(B, 128, device=DEV)
+    ws = lsa.workspace(lsa.lsa_msa_attn_workspace_size(B, idx.shape[1], G))
+    lsa.lsa_msa_attn(q, kv, idx, gm, cnt, G, scale, out, lse, ws)
+    torch.cuda.synchronize()
+    idx_h, gm_h, cnt_h = idx.cpu().numpy(), gm.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(B):
+        row, m = idx_h[b, : cnt_h[b]], gm_h[b, : cnt_h[b]]
+        for g in range(G):
+            sel = row[(m >> g) & 1 == 1]
+            heads = slice(g * 16, (g + 1) * 16)
+            ref, ref_lse = run_oracle_attention(q[b, heads], kv, sel, scale)
+            assert attn_rel_err(out[b, heads], ref) <= ATTN_REL, (b, g)
+            assert np.abs(f64(lse[b, heads]) - ref_lse).max() <= 1e-3
