@@ -15,9 +15,11 @@ exchange step on one node here: replicas only), timed per rank, max over ranks.
 memory, runs the three calls and copies the output back.  The sequence is captured once as a CUDA graph and
 replayed per step (the form a serving loop uses); "eager_ms_per_step" is the same sequence issued call by call.
 
-At N = 1 the line also carries "long_context": per-stage times of the 1M-token decode (FP8 token path and
-micro-block selection) and of the 10M-token Flat bucket workload (--no-configs skips them), and "prefill_chunk": the latency of one causal prefill chunk (8192 queries,
-FP8 scan + bf16 re-rank, K = 2048 + sink 4 + window 128) with its per-stage times (--no-prefill skips it).
+At N = 1 the line also carries "long_context": per-stage times of the 1M-token decode (FP8 token path,
+hierarchical selection, micro-block selection), of the hybrid attention and the group-wise block selection at
+128K, and of the 10M-token Flat bucket workload (--no-configs skips them), and "prefill_chunk": the latency of one
+causal prefill chunk (8192 queries, FP8 scan + bf16 re-rank, K = 2048 + sink 4 + window 128) with its per-stage
+times (--no-prefill skips it).
 """
 
 from __future__ import annotations

@@ -260,9 +260,9 @@ size_t lsa_msa_workspace_size(int64_t B, int64_t L, int G, int KB);
  *   Source: the same section (a group's query heads share its blocks).
  *   out[b,h] / lse[b,h] = lsa_sparse_attn's attention of head h (group g = h / (128 / G)) over the entries of
  *   idx[b, :count[b]] whose gmask has bit g.  Each group's rows are compacted first (k_msa_group_rows), then
- *   the (query, group) pairs run as B*G queries of 128 / G heads (q, out and lse viewed accordingly).  Head
- *   groups of fewer than 128 heads run on the CUDA-core attention kernel; the tensor-core "KV-outer" form
- *   (each KV tile loaded once for every group that kept it) is not built.
+ *   each (query, group) pair runs the tensor-core attention as one 128-head query whose first 128 / G rows are
+ *   the group's heads and whose other rows are zero (outputs dropped).  The "KV-outer" form (each KV tile
+ *   loaded once for every group that kept it) is not built.
  *   H = 128, G in {1, 2, 4, 8}.  ws: lsa_msa_attn_workspace_size(B, idx_ld, G) bytes.
  */
 int lsa_msa_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, const uint8_t* gmask,

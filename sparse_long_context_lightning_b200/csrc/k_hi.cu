@@ -11,10 +11,14 @@
 #include "lsa_common.cuh"
 
 namespace lsa {
+
+int sm_count();
+
 namespace {
 
 constexpr int PS_THREADS = 256;
 constexpr int PE_THREADS = 1024;
+constexpr int GR_THREADS = 1024;
 
 // page[b, p] = sum of the scores of page p's complete sub-blocks that end at or before q_pos (sequential
 // fp32 sum, ascending sub-block), for pages that start at or before q_pos; -inf for the others.
@@ -102,79 +106,83 @@ __global__ void __launch_bounds__(PE_THREADS) k_page_expand(const int32_t* __res
 }
 
 // Group-wise block selection, per query b (one CTA): the entries are every group's kept blocks
-// (kept[(b G + g) kept_ld + j], j < kcnt) and the local block (all groups); the distinct blocks, ascending,
-// expand to their tokens (the local block up to q_pos), each token carrying the bit mask of the groups that
-// chose its block.  Blocks before the local one are complete and entirely visible.
+// (kept[(b G + g) kept_ld + j], j < kcnt) and the local block (all groups), keyed (block << 8 | group bit).  The
+// keys are sorted (bitonic, in shared memory); the first key of each block's run is its head, the run's bits
+// OR to the block's group mask, and an ordered scan of the heads gives each distinct block its rank.  The
+// blocks, ascending, then expand to their tokens with coalesced writes: every block below the local one is
+// complete and entirely visible (offset rank * block), the local block is the last and ends at q_pos.
 __global__ void __launch_bounds__(PE_THREADS) k_msa_expand(const int32_t* __restrict__ kept, int64_t kept_ld,
                                                            const int32_t* __restrict__ kcnt, int G, int block,
                                                            const int64_t* __restrict__ q_pos,
                                                            int32_t* __restrict__ idx, uint8_t* __restrict__ gmask,
                                                            int64_t idx_ld, int32_t* __restrict__ count) {
-  __shared__ int32_t ent_blk[PE_THREADS];
-  __shared__ uint32_t ent_bit[PE_THREADS];
+  constexpr uint64_t PAD = ~0ull;
+  __shared__ uint64_t key[PE_THREADS];
+  __shared__ int32_t dblk[PE_THREADS];
+  __shared__ uint8_t dmask[PE_THREADS];
+  __shared__ uint32_t wsum[PE_THREADS / 32];
   const int b = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int qp = static_cast<int>(q_pos[b]);
   const int lb = qp / block;
-  // entries: group g's kept blocks at [g kept_ld, g kept_ld + kcnt), the local block last
-  const int n_ent = G * static_cast<int>(kept_ld) + 1;
-  for (int e = tid; e < n_ent; e += PE_THREADS) {
-    int blk = -1;
-    uint32_t bit = 0u;
-    if (e == n_ent - 1) {
-      blk = lb;
-      bit = (1u << G) - 1u;
-    } else {
-      const int g = e / static_cast<int>(kept_ld), j = e % static_cast<int>(kept_ld);
-      if (j < kcnt[b * G + g]) {
-        blk = kept[(static_cast<int64_t>(b) * G + g) * kept_ld + j];
-        bit = 1u << g;
-      }
+  const int kl = static_cast<int>(kept_ld);
+  const int n_ent = G * kl + 1;  // <= PE_THREADS (checked by the launcher)
+  int np = 32;
+  while (np < n_ent) np <<= 1;
+  if (tid < np) {
+    uint64_t k = PAD;
+    if (tid == n_ent - 1) {
+      k = (static_cast<uint64_t>(lb) << 8) | ((1u << G) - 1u);
+    } else if (tid < n_ent - 1) {
+      const int g = tid / kl, j = tid % kl;
+      if (j < kcnt[b * G + g])
+        k = (static_cast<uint64_t>(kept[(static_cast<int64_t>(b) * G + g) * kept_ld + j]) << 8) | (1u << g);
     }
-    ent_blk[e] = blk;
-    ent_bit[e] = bit;
+    key[tid] = k;
   }
   __syncthreads();
-  // a distinct block is written by its first entry: mask = OR over its entries, rank = distinct blocks below
-  int nd = 0;  // distinct blocks in total (every thread counts: uniform)
-  for (int e = 0; e < n_ent; ++e) {
-    const int x = ent_blk[e];
-    bool first = x >= 0;
-    for (int f = 0; first && f < e; ++f) first = ent_blk[f] != x;
-    nd += first;
+  for (int size = 2; size <= np; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const int p = tid ^ stride;
+      if (tid < np && p > tid) {
+        const uint64_t x = key[tid], y = key[p];
+        if ((x > y) == ((tid & size) == 0)) {
+          key[tid] = y;
+          key[p] = x;
+        }
+      }
+      __syncthreads();
+    }
   }
+  const uint64_t kt = tid < np ? key[tid] : PAD;
+  const uint64_t blk = kt >> 8;
+  const bool head = kt != PAD && (tid == 0 || (key[tid - 1] >> 8) != blk);
+  uint32_t mask = 0u;
+  if (head)  // a run holds at most one entry per group plus the local block's
+    for (int p = tid; p < np && key[p] != PAD && (key[p] >> 8) == blk; ++p) mask |= static_cast<uint32_t>(key[p] & 0xFFu);
+  const uint32_t bal = __ballot_sync(0xffffffffu, head);
+  if (lane == 0) wsum[warp] = __popc(bal);
+  __syncthreads();
+  int before = 0, nd = 0;
+  for (int w = 0; w < PE_THREADS / 32; ++w) {
+    before += w < warp ? static_cast<int>(wsum[w]) : 0;
+    nd += static_cast<int>(wsum[w]);
+  }
+  if (head) {
+    const int rank = before + __popc(bal & ((1u << lane) - 1u));
+    dblk[rank] = static_cast<int32_t>(blk);
+    dmask[rank] = static_cast<uint8_t>(mask);
+  }
+  __syncthreads();
+  const int total = (nd - 1) * block + (qp + 1 - lb * block);
   int32_t* row = idx + static_cast<int64_t>(b) * idx_ld;
   uint8_t* mrow = gmask + static_cast<int64_t>(b) * idx_ld;
-  for (int e = tid; e < n_ent; e += PE_THREADS) {
-    const int x = ent_blk[e];
-    if (x < 0) continue;
-    bool first = true;
-    uint32_t mask = 0u;
-    int rank = 0;
-    for (int f = 0; f < n_ent; ++f) {
-      const int y = ent_blk[f];
-      if (y == x) {
-        mask |= ent_bit[f];
-        if (f < e) first = false;
-      }
-    }
-    if (!first) continue;
-    for (int f = 0; f < n_ent; ++f) {  // distinct blocks below x
-      const int y = ent_blk[f];
-      if (y >= 0 && y < x) {
-        bool fy = true;
-        for (int f2 = 0; fy && f2 < f; ++f2) fy = ent_blk[f2] != y;
-        rank += fy;
-      }
-    }
-    // every block below the local one is complete: the offset is rank * block
-    const int lo = x * block, hi = min(x * block + block, qp + 1);
-    for (int t = lo; t < hi; ++t) {
-      row[rank * block + (t - lo)] = t;
-      mrow[rank * block + (t - lo)] = static_cast<uint8_t>(mask);
-    }
+  for (int t = tid; t < total; t += PE_THREADS) {
+    const int r = t / block;
+    row[t] = dblk[r] * block + (t - r * block);
+    mrow[t] = dmask[r];
   }
-  if (tid == 0) count[b] = (nd - 1) * block + (qp + 1 - lb * block);
+  if (tid == 0) count[b] = total;
 }
 
 // out[b G + g] = q_pos[b] + delta (the per-(query, group) positions of group-wise selection)
@@ -187,12 +195,12 @@ __global__ void k_shift_qpos(const int64_t* __restrict__ q_pos, int64_t n, int G
 // Each group's own rows out of a group-wise selection: grows[(b G + g) idx_ld + i] = the i-th entry of
 // idx[b, :count[b]] whose gmask has bit g (ascending, as in the union row); gcount[b G + g] of them.  One
 // CTA per (query, group): an ordered block scan of the bit.
-__global__ void __launch_bounds__(PS_THREADS) k_msa_group_rows(const int32_t* __restrict__ idx,
+__global__ void __launch_bounds__(GR_THREADS) k_msa_group_rows(const int32_t* __restrict__ idx,
                                                                const uint8_t* __restrict__ gmask, int64_t idx_ld,
                                                                const int32_t* __restrict__ count, int G,
                                                                int32_t* __restrict__ grows,
                                                                int32_t* __restrict__ gcount) {
-  __shared__ uint32_t wsum[PS_THREADS / 32];
+  __shared__ uint32_t wsum[GR_THREADS / 32];
   const int bg = blockIdx.x;
   const int b = bg / G, g = bg % G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -201,14 +209,14 @@ __global__ void __launch_bounds__(PS_THREADS) k_msa_group_rows(const int32_t* __
   const uint8_t* mrow = gmask + static_cast<int64_t>(b) * idx_ld;
   int32_t* out = grows + static_cast<int64_t>(bg) * idx_ld;
   uint32_t base = 0;
-  for (int i0 = 0; i0 < n; i0 += PS_THREADS) {
+  for (int i0 = 0; i0 < n; i0 += GR_THREADS) {
     const int i = i0 + tid;
     const bool mine = i < n && ((mrow[i] >> g) & 1u);
     const uint32_t bal = __ballot_sync(0xffffffffu, mine);
     if (lane == 0) wsum[warp] = __popc(bal);
     __syncthreads();
     uint32_t before = 0, total = 0;
-    for (int w = 0; w < PS_THREADS / 32; ++w) {
+    for (int w = 0; w < GR_THREADS / 32; ++w) {
       before += w < warp ? wsum[w] : 0u;
       total += wsum[w];
     }
@@ -217,6 +225,41 @@ __global__ void __launch_bounds__(PS_THREADS) k_msa_group_rows(const int32_t* __
     __syncthreads();  // wsum is rewritten by the next step
   }
   if (tid == 0) gcount[bg] = static_cast<int32_t>(base);
+}
+
+// Per-group attention queries: qg[b G + g] is a 128-head query whose rows h < 128 / G are head g 128 / G + h
+// of q[b] and whose other rows are 0 (their outputs are dropped).  16-byte units: a 576-wide bf16 row is 72.
+__global__ void k_msa_pad_q(const uint4* __restrict__ q, int G, int64_t n_bg, uint4* __restrict__ qg) {
+  const int64_t total = n_bg * 128 * 72;
+  const int hg = 128 / G;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / 72;
+    const int c = static_cast<int>(i % 72);
+    const int64_t bg = r / 128;
+    const int h = static_cast<int>(r % 128);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (h < hg) v = q[((bg / G) * 128 + (bg % G) * hg + h) * 72 + c];
+    qg[i] = v;
+  }
+}
+
+// The real rows back: out[b, h] = outg[b G + h / (128 / G), h mod (128 / G)] (512-wide bf16 rows: 64 units),
+// lse likewise when given.
+__global__ void k_msa_unpad(const uint4* __restrict__ outg, const float* __restrict__ lseg, int G, int64_t B,
+                            uint4* __restrict__ out, float* __restrict__ lse) {
+  const int64_t total = B * 128 * 64;
+  const int hg = 128 / G;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / 64;
+    const int c = static_cast<int>(i % 64);
+    const int64_t b = r / 128;
+    const int h = static_cast<int>(r % 128);
+    const int64_t src = (b * G + h / hg) * 128 + h % hg;
+    out[i] = outg[src * 64 + c];
+    if (lse != nullptr && c == 0) lse[r] = lseg[src];
+  }
 }
 
 }  // namespace
@@ -259,7 +302,21 @@ int launch_shift_qpos(const int64_t* q_pos, int64_t B, int G, int64_t delta, int
 int launch_msa_group_rows(const int32_t* idx, const uint8_t* gmask, int64_t idx_ld, const int32_t* count, int64_t B,
                           int G, int32_t* grows, int32_t* gcount, cudaStream_t s) {
   if (B == 0) return LSA_OK;
-  k_msa_group_rows<<<static_cast<unsigned>(B * G), PS_THREADS, 0, s>>>(idx, gmask, idx_ld, count, G, grows, gcount);
+  k_msa_group_rows<<<static_cast<unsigned>(B * G), GR_THREADS, 0, s>>>(idx, gmask, idx_ld, count, G, grows, gcount);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_msa_pad_q(const void* q, int G, int64_t B, void* qg, cudaStream_t s) {
+  if (B == 0) return LSA_OK;
+  k_msa_pad_q<<<static_cast<unsigned>(sm_count() * 4), 256, 0, s>>>(static_cast<const uint4*>(q), G, B * G,
+                                                                    static_cast<uint4*>(qg));
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_msa_unpad(const void* outg, const float* lseg, int G, int64_t B, void* out, float* lse, cudaStream_t s) {
+  if (B == 0) return LSA_OK;
+  k_msa_unpad<<<static_cast<unsigned>(sm_count() * 4), 256, 0, s>>>(static_cast<const uint4*>(outg), lseg, G, B,
+                                                                    static_cast<uint4*>(out), lse);
   return cuda_status(cudaGetLastError());
 }
 

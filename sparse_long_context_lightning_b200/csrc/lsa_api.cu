@@ -344,10 +344,31 @@ int lsa_msa_select(const void* q_idx, const float* w, const void* k_idx, int64_t
   return st;
 }
 
+struct MsaAttnLayout {
+  size_t o_cnt, o_q, o_out, o_lse, o_att, total;
+};
+static MsaAttnLayout msa_attn_layout(int64_t B, int64_t idx_ld, int G) {
+  MsaAttnLayout m;
+  const size_t bg = static_cast<size_t>(B) * G;
+  m.o_cnt = align_up(bg * idx_ld * 4, 256);
+  size_t o = m.o_cnt + align_up(bg * 4, 256);
+  m.o_q = m.o_out = m.o_lse = o;
+  if (G > 1) {  // the padded 128-head queries, their outputs and lse
+    m.o_q = o;
+    o += align_up(bg * 128 * 576 * 2, 256);
+    m.o_out = o;
+    o += align_up(bg * 128 * 512 * 2, 256);
+    m.o_lse = o;
+    o += align_up(bg * 128 * 4, 256);
+  }
+  m.o_att = o;
+  m.total = o + sparse_attn_ws_bytes(static_cast<int64_t>(bg), idx_ld, 128);
+  return m;
+}
+
 size_t lsa_msa_attn_workspace_size(int64_t B, int64_t idx_ld, int G) {
   if (B < 0 || idx_ld < 0 || G < 1) return static_cast<size_t>(-1);
-  const size_t rows = align_up(static_cast<size_t>(B) * G * idx_ld * 4, 256);
-  return rows + align_up(static_cast<size_t>(B) * G * 4, 256) + sparse_attn_ws_bytes(B * G, idx_ld, 128 / G);
+  return msa_attn_layout(B, idx_ld, G).total;
 }
 
 int lsa_msa_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, const uint8_t* gmask, int64_t idx_ld,
@@ -358,19 +379,29 @@ int lsa_msa_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, c
   if (B == 0) return LSA_OK;
   LSA_CHECK_ARG(q && kv && idx && gmask && count && out);
   LSA_CHECK_ARG(aligned16(q) && aligned16(kv) && aligned16(out) && B * G <= 65535);
-  if (ws == nullptr || !aligned256(ws) || ws_bytes < lsa_msa_attn_workspace_size(B, idx_ld, G)) return LSA_ERR_WORKSPACE;
+  const MsaAttnLayout m = msa_attn_layout(B, idx_ld, G);
+  if (ws == nullptr || !aligned256(ws) || ws_bytes < m.total) return LSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned char* base = static_cast<unsigned char*>(ws);
   int32_t* grows = reinterpret_cast<int32_t*>(base);
-  const size_t o_cnt = align_up(static_cast<size_t>(B) * G * idx_ld * 4, 256);
-  int32_t* gcnt = reinterpret_cast<int32_t*>(base + o_cnt);
-  const size_t o_att = o_cnt + align_up(static_cast<size_t>(B) * G * 4, 256);
-  // each group's rows, then the attention of the (query, group) pairs: q / out / lse viewed as [B G, 128 / G, ...]
-  // (a group's heads are contiguous)
+  int32_t* gcnt = reinterpret_cast<int32_t*>(base + m.o_cnt);
+  // each group's rows; then one 128-head attention per (query, group) on the tensor cores, the group's heads in
+  // the first 128 / G rows of a zero-padded query (G = 1: the query itself)
   int st = launch_msa_group_rows(idx, gmask, idx_ld, count, B, G, grows, gcnt, s);
+  if (G == 1) {
+    if (st == LSA_OK)
+      st = launch_sparse_attn(q, kv, L, grows, idx_ld, gcnt, B, 128, scale, out, lse, base + m.o_att,
+                              ws_bytes - m.o_att, s);
+    return st;
+  }
+  void* qg = base + m.o_q;
+  void* outg = base + m.o_out;
+  float* lseg = reinterpret_cast<float*>(base + m.o_lse);
+  if (st == LSA_OK) st = launch_msa_pad_q(q, G, B, qg, s);
   if (st == LSA_OK)
-    st = launch_sparse_attn(q, kv, L, grows, idx_ld, gcnt, B * G, 128 / G, scale, out, lse, base + o_att,
-                            ws_bytes - o_att, s);
+    st = launch_sparse_attn(qg, kv, L, grows, idx_ld, gcnt, B * G, 128, scale, outg, lseg, base + m.o_att,
+                            ws_bytes - m.o_att, s);
+  if (st == LSA_OK) st = launch_msa_unpad(outg, lseg, G, B, out, lse, s);
   return st;
 }
 

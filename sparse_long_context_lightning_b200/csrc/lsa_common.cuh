@@ -171,6 +171,8 @@ size_t hybrid_attn_ws_bytes(int64_t B, int64_t idx_ld, int H, int sink, int wind
 int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
                        const int32_t* count, int64_t B, int H, float scale, void* out, float* lse,
                        void* ws, size_t ws_bytes, cudaStream_t s);
+int launch_msa_pad_q(const void* q, int G, int64_t B, void* qg, cudaStream_t s);
+int launch_msa_unpad(const void* outg, const float* lseg, int G, int64_t B, void* out, float* lse, cudaStream_t s);
 int launch_msa_group_rows(const int32_t* idx, const uint8_t* gmask, int64_t idx_ld, const int32_t* count, int64_t B,
                           int G, int32_t* grows, int32_t* gcount, cudaStream_t s);
 int launch_block_max_tc(const void* q, const float* w, const void* k, int64_t B, int64_t L, int G,
