@@ -26,6 +26,12 @@ primitives (matmul, stable sort, exp, log) as steps and no blocking or fusion:
                       keys, top-M pages, then the token score and arg topK on the recalled tokens.
 * ``msa_select_row``  lecture "从两本账看懂长上下文注意力", §"MiniMax Sparse Attention": block score = max of
                       its tokens' index scores, per-group top-k blocks, the local block always kept.
+* ``tree_select_row`` "LSA 稀疏注意力會省顯存嗎", §二 step 3 (the Tree version searches level by level,
+                      keeping candidates at each level); "超长上下文LSA注意力技术开源", §"Qwen LSA注意力优化原理与
+                      核心创新" (keys clustered into a tree; the query scans only cluster centres, then picks
+                      buckets).  Two levels over the Flat buckets; parity unpinned beyond the pins in the tests
+                      (full beam = Flat, one child per parent = Flat, a hand-built case where a parent's mean
+                      hides its best child).
 * ``lse_merge``       LongCat page §"训练与 kernel：混合稀疏注意力算子（HFA）": partial attentions merged by
                       online-softmax (log-sum-exp) rescaling.
 * ``softmax_attention`` / ``sparse_mla_attn``
@@ -288,6 +294,55 @@ def msa_select_row(q_I_b: np.ndarray, w_b: np.ndarray, k_I: np.ndarray, q_pos: i
         pos = np.union1d(pos, np.arange(lb * block, q_pos + 1)).astype(np.int64)
         out.append((pos, kth))
     return out
+
+
+# ---------------------------------------------------------------------------
+# D-LSA Tree: level-by-level search over cluster centres, then the Flat buckets
+# ---------------------------------------------------------------------------
+
+
+def tree_parents(reps: np.ndarray, F: int) -> np.ndarray:
+    """Level-2 centres: parent p is the plain mean of the representatives of buckets [p*F, min((p+1)*F, NB)).
+
+    The pages give no rule for building the tree; grouping F consecutive bucket ids under one parent, with the
+    parent's centre the mean of its children's centres, is the plainest reading (a clusterer that emits its
+    buckets in cluster order gives exactly this layout)."""
+    reps = np.asarray(reps, dtype=np.float64)
+    nb = reps.shape[0]
+    return np.stack([reps[p * F: min((p + 1) * F, nb)].mean(axis=0) for p in range(-(-nb // F))])
+
+
+def tree_select_row(q_I_b: np.ndarray, w_b: np.ndarray, reps: np.ndarray, members: np.ndarray, F: int, M2: int,
+                    M: int, q_pos: int, sink: int, window: int):
+    """One query of the two-level tree search: (sorted positions, M-th candidate bucket score, M2-th parent score).
+
+    Level 2: every parent centre is scored with the indexer formula and the M2 best parents are kept (stable
+    sort on descending score: ties -> lower parent id).  Level 1: the kept parents' children (ascending bucket
+    id) are the candidates; they are scored the same way and the M best are kept (ties -> lower bucket id).
+    The kept buckets expand to their members, with sink and window, clipped to [0, q_pos], as in Flat mode.
+    """
+    q_pos = int(q_pos)
+    reps = np.asarray(reps, dtype=np.float64)
+    nb = reps.shape[0]
+    q = np.asarray(q_I_b)[None]
+    w = np.asarray(w_b)[None]
+    parents = tree_parents(reps, F)
+    ps = bucket_scores(q, w, parents)[0]
+    porder = np.argsort(-ps, kind="stable")
+    n2 = min(M2, parents.shape[0])
+    kept_parents = np.sort(porder[:n2])
+    m2th = float(ps[porder[n2 - 1]])
+    cand = np.concatenate([np.arange(p * F, min((p + 1) * F, nb)) for p in kept_parents]).astype(np.int64)
+    cs = bucket_scores(q, w, reps[cand])[0]
+    corder = np.argsort(-cs, kind="stable")
+    n1 = min(M, cand.size)
+    chosen = cand[corder[:n1]]
+    mth = float(cs[corder[n1 - 1]])
+    pos = np.asarray(members, dtype=np.int64)[chosen].reshape(-1)
+    s_sink, s_swa = fixed_positions(q_pos, sink, window)
+    sel = np.unique(np.concatenate([s_sink, pos, s_swa]))
+    sel = sel[(sel >= 0) & (sel <= q_pos)]
+    return sel.astype(np.int64), mth, m2th
 
 
 # ---------------------------------------------------------------------------

@@ -473,3 +473,78 @@ def test_msa_local_block_only_near_the_start():
     q, w, k = rng.normal(size=(2, 4)), rng.uniform(size=2), rng.normal(size=(40, 4))
     (pos, kth), = O.msa_select_row(q, w, k, 9, G=1, block=16, KB=2)
     assert pos.tolist() == list(range(10)) and kth == -np.inf
+
+
+# --------------------------------------------------------------------------
+# D-LSA Tree: two-level search
+# --------------------------------------------------------------------------
+
+
+def test_tree_parents_are_child_means_with_ragged_last():
+    """Parent p = mean of buckets [pF, min((p+1)F, NB)): NB = 5, F = 2 -> means of (0,1), (2,3) and (4) alone."""
+    reps = np.array([[1.0, 0.0], [3.0, 2.0], [5.0, -1.0], [7.0, 1.0], [-4.0, 9.0]])
+    par = O.tree_parents(reps, 2)
+    assert par.tolist() == [[2.0, 1.0], [6.0, 0.0], [-4.0, 9.0]]
+
+
+def _tree_case(seed=3, NB=37, bsz=5, d=8, H=3):
+    rng = np.random.default_rng(seed)
+    L = NB * bsz
+    members = rng.permutation(L).reshape(NB, bsz)
+    reps = rng.standard_normal((NB, d))
+    q = rng.standard_normal((H, d))
+    w = rng.uniform(0.0, 1.0, H)
+    return L, members, reps, q, w
+
+
+def test_tree_full_beam_is_flat():
+    """Keeping every parent makes every bucket a candidate: the search is the Flat search."""
+    L, members, reps, q, w = _tree_case()
+    flat_scores = O.bucket_scores(q[None], w[None], reps)[0]
+    for F in (1, 4, 6, 37):
+        NP = -(-37 // F)
+        for M in (1, 5, 11):
+            sel, mth, _ = O.tree_select_row(q, w, reps, members, F, NP, M, L - 1, 2, 3)
+            want, want_mth, _ = O.bucket_select_row(flat_scores, L - 1, M, 2, 3, members=members)
+            assert np.array_equal(sel, want) and mth == want_mth, (F, M)
+
+
+def test_tree_one_child_per_parent_is_flat():
+    """F = 1: the parents are the buckets, the M2 >= M best of them hold the M best buckets."""
+    L, members, reps, q, w = _tree_case(seed=5)
+    flat_scores = O.bucket_scores(q[None], w[None], reps)[0]
+    for M, M2 in ((3, 3), (3, 10), (7, 8)):
+        sel, _, _ = O.tree_select_row(q, w, reps, members, 1, M2, M, L - 1, 0, 0)
+        want, _, _ = O.bucket_select_row(flat_scores, L - 1, M, 0, 0, members=members)
+        assert np.array_equal(sel, want), (M, M2)
+
+
+def test_tree_parent_mean_hides_best_child():
+    """A bucket whose centre is average can hide a strong member (the LSA page warns of exactly this); here a
+    parent's mean hides its best child, so the narrow beam misses what Flat keeps.
+
+    q = (1, 0), one head, w = 1.  Buckets 0, 1 (parent 0): centres (10, 0), (-10, 0) -> parent (0, 0), score 0.
+    Buckets 2, 3 (parent 1): centres (1, 0), (2, 0) -> parent (1.5, 0), score 1.5.  M2 = 1 keeps parent 1; of its
+    children bucket 3 (score 2) beats bucket 2 (score 1).  Flat keeps bucket 0 (score 10)."""
+    reps = np.array([[10.0, 0.0], [-10.0, 0.0], [1.0, 0.0], [2.0, 0.0]])
+    members = np.array([[0, 1], [2, 3], [4, 5], [6, 7]])
+    q, w = np.array([[1.0, 0.0]]), np.array([1.0])
+    sel, mth, m2th = O.tree_select_row(q, w, reps, members, 2, 1, 1, 7, 0, 0)
+    assert sel.tolist() == [6, 7] and mth == 2.0 and m2th == 1.5
+    sel2, _, _ = O.tree_select_row(q, w, reps, members, 2, 2, 1, 7, 0, 0)
+    assert sel2.tolist() == [0, 1]
+    # ties at level 1 go to the lower bucket id: equal children under the kept parent
+    reps_t = np.array([[10.0, 0.0], [-10.0, 0.0], [2.0, 0.0], [2.0, 0.0]])
+    sel3, _, _ = O.tree_select_row(q, w, reps_t, members, 2, 1, 1, 7, 0, 0)
+    assert sel3.tolist() == [4, 5]
+
+
+def test_tree_union_clip_and_short_candidate_list():
+    """Fewer candidates than M: all are kept; members past q_pos are dropped; sink and window join."""
+    reps = np.array([[1.0], [2.0], [3.0], [4.0], [5.0]])
+    members = np.array([[0, 9], [1, 8], [2, 7], [3, 6], [4, 5]])
+    q, w = np.array([[1.0]]), np.array([1.0])
+    # F = 2: parents (1.5), (3.5), (5); M2 = 1 keeps parent 2 (bucket 4 alone); M = 3 > 1 candidate
+    sel, mth, m2th = O.tree_select_row(q, w, reps, members, 2, 1, 3, 6, 1, 2)
+    assert m2th == 5.0 and mth == 5.0
+    assert sel.tolist() == [0, 4, 5, 6]
