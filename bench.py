@@ -504,6 +504,37 @@ def long_context_configs(device, l2_flush, iters: int = 10):
                      "stages": {"bucket_select": _stage(st[0], sel_bytes, 3 * sel_flops, bf16),
                                 "attn": _stage(st[1], at_bytes)},
                      "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
+        if name == "flat10m":
+            # the Tree form over the same buckets: parents of 64 consecutive buckets, top-64 parents, then the
+            # top-32 of their 4096 children; timed beside Flat, with the share of Flat's positions it keeps
+            F, M2 = 64, 64
+            lsa_ = bstep.lsa
+            NP = -(-bstep.nb // F)
+            par = torch.empty(NP, wl.d_I, device=device)
+            lsa_.lsa_tree_parents(bstep.cen, F, par)
+            t_idx, t_cnt = torch.empty_like(bstep.idx), torch.empty_like(bstep.cnt)
+            ws_t = lsa_.workspace(lsa_.lsa_tree_workspace_size(B, NP, F, M2, wl.M), device)
+
+            def tree():
+                lsa_.lsa_tree_select(bstep.q_I, bstep.w, bstep.cen, par, F, bstep.members, M2, wl.M, wl.sink,
+                                     wl.window, wl.L, bstep.q_pos, t_idx, t_cnt, ws_t)
+
+            st_t = _time_stages([tree], l2_flush, iters)
+            bstep.select()
+            tree()
+            torch.cuda.synchronize()
+            fi, fc, ti, tc = bstep.idx.cpu(), bstep.cnt.cpu(), t_idx.cpu(), t_cnt.cpu()
+            kept = [len(np.intersect1d(fi[b, : fc[b]].numpy(), ti[b, : tc[b]].numpy())) / max(int(fc[b]), 1)
+                    for b in range(B)]
+            t_bytes = NP * wl.d_I * 4 + B * M2 * F * (wl.d_I * 4 + 8) + B * wl.kmax * 4
+            t_flops = 2.0 * B * wl.H_I * wl.d_I * (NP + M2 * F)
+            res["flat10m_tree"] = {
+                "workload": "flat10m's buckets as a two-level tree: 2442 parents of 64 consecutive buckets (mean "
+                            "centres), top-64 parents, top-32 of their 4096 children, + sink 4 + window 512",
+                "stages": {"tree_select": _stage(st_t[0], t_bytes)}, "tree_select_flops": t_flops,
+                "flat_select_ms": round(float(st[0]), 5),
+                "share_of_flat_positions_kept": round(float(np.mean(kept)), 4)}
+            del par, t_idx, t_cnt, ws_t
         del bstep
         torch.cuda.empty_cache()
     return res

@@ -173,6 +173,41 @@ int lsa_bucket_select(const void* q_idx, const float* q_scale, const float* w, i
                       void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * lsa_tree_parents -- the level-2 centres of the tree search (untimed precompute, beside the bucket centres).
+ *   Source: "超长上下文LSA注意力技术开源", section "Qwen LSA注意力优化原理与核心创新" (keys clustered into a
+ *   tree of cluster centres).  The pages give no construction; the reading here: parent p covers buckets
+ *   [p*F, min((p+1)*F, NB)) and its centre is their centres' plain mean,
+ *     parents[p, d] = (sum_{c in p} centroids[c, d], summed in order) / (number of children)   (fp32)
+ *   centroids [NB, d_I] fp32, parents [ceil(NB/F), d_I] fp32.  1 <= d_I <= 128, F >= 1.
+ */
+int lsa_tree_parents(const float* centroids, int64_t NB, int d_I, int F, float* parents, void* stream);
+
+/*
+ * lsa_tree_select -- two-level tree search over the Flat buckets (the Tree form of lsa_bucket_select).
+ *   Source: "LSA 稀疏注意力會省顯存嗎", section 二 step 3 (the Tree version searches level by level, keeping
+ *   candidates at each level); the same page's step 4 and lsa_bucket_select for the expansion.
+ *
+ *   For each query b (scores: the indexer formula on a centre, fp32, as lsa_bucket_select):
+ *     level 2   kept parents  = the M2 parents with the largest score (ties -> lower parent id)
+ *     level 1   candidates    = the kept parents' children, in ascending bucket id
+ *               kept buckets  = the M candidates with the largest score (ties -> lower bucket id)
+ *     idx row   = sorted, de-duplicated union of the kept buckets' members, sink and window, restricted to
+ *                 [0, q_pos]; -1 padded up to idx_ld.  count[b] entries.
+ *   With M2 >= NP every bucket is a candidate and the result is lsa_bucket_select's (Flat).
+ *   q_idx [B, H_I, d_I] bf16, w [B, H_I] fp32, centroids [NB, d_I] fp32, parents [NP, d_I] fp32 from
+ *   lsa_tree_parents (NP = ceil(NB/F)), members int32 [NB, bsz].  d_I in {32, 64, 128}, H_I <= 64,
+ *   1 <= M2, M <= 1024; M*bsz + sink + window <= min(8192, idx_ld).
+ *   ws: lsa_tree_workspace_size(B, NP, F, M2, M) bytes.
+ */
+int lsa_tree_select(const void* q_idx, const float* w, int64_t B, int H_I, int d_I, const float* centroids,
+                    int64_t NB, const float* parents, int64_t NP, int F, const int32_t* members, int bsz, int M2,
+                    int M, int sink, int window, int64_t L, const int64_t* q_pos, int32_t* idx, int64_t idx_ld,
+                    int32_t* count, void* ws, size_t ws_bytes, void* stream);
+
+/* lsa_tree_workspace_size -- scratch bytes of lsa_tree_select; (size_t)-1 for invalid sizes. */
+size_t lsa_tree_workspace_size(int64_t B, int64_t NP, int F, int M2, int M);
+
+/*
  * lsa_split_representatives -- the exact three-part bf16 split of fp32 representatives, for
  *   lsa_bucket_select_split: computed once with the representatives (lsa_pool_keys) and cached beside
  *   them.  Not on the pages: a layout of the pages' representative for the tensor cores.

@@ -44,6 +44,10 @@ SIGNATURES = {
     "lsa_hi_workspace_size": (_SZ, [_I64, _I64, _I32, _I32, _I32, _I32, _I32, _I32]),
     "lsa_hybrid_attn": (_I32, [_P, _P, _I64, _P, _I64, _P, _I64, _I32, _I32, _I32, _I32, _I32, _P, _F32, _P, _P, _P,
                                _SZ, _P]),
+    "lsa_tree_parents": (_I32, [_P, _I64, _I32, _I32, _P, _P]),
+    "lsa_tree_workspace_size": (_SZ, [_I64, _I64, _I32, _I32, _I32]),
+    "lsa_tree_select": (_I32, [_P, _P, _I64, _I32, _I32, _P, _I64, _P, _I64, _I32, _P, _I32, _I32, _I32, _I32, _I32,
+                               _I64, _P, _P, _I64, _P, _P, _SZ, _P]),
     "lsa_msa_select": (_I32, [_P, _P, _P, _I64, _I32, _I32, _I64, _I32, _I32, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "lsa_msa_workspace_size": (_SZ, [_I64, _I64, _I32, _I32]),
     "lsa_msa_attn_workspace_size": (_SZ, [_I64, _I64, _I32]),
@@ -168,6 +172,29 @@ def lsa_bucket_select_split(q_idx, w, split, members, bsz, M, sink, window, L, q
                                                 idx.stride(0), _ptr(count), _ptr(ws),
                                                 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check("lsa_bucket_select_split", st)
+
+
+def lsa_tree_parents(centroids, F, parents, stream=None):
+    """Level-2 centres of the tree search: parent p = mean of the centres of buckets [pF, min((p+1)F, NB))."""
+    NB, d_I = centroids.shape
+    st = load_library().lsa_tree_parents(_ptr(centroids), NB, d_I, F, _ptr(parents), _stream(stream))
+    _check("lsa_tree_parents", st)
+
+
+def lsa_tree_workspace_size(B, NP, F, M2, M):
+    return load_library().lsa_tree_workspace_size(B, NP, F, M2, M)
+
+
+def lsa_tree_select(q_idx, w, centroids, parents, F, members, M2, M, sink, window, L, q_pos, idx, count, ws,
+                    stream=None):
+    """Two-level tree search: top-M2 parents, then the top-M of their children, expanded as Flat buckets."""
+    B, H_I, d_I = q_idx.shape
+    NB, bsz = members.shape
+    st = load_library().lsa_tree_select(_ptr(q_idx), _ptr(w), B, H_I, d_I, _ptr(centroids), NB, _ptr(parents),
+                                        parents.shape[0], F, _ptr(members), bsz, M2, M, sink, window, L,
+                                        _ptr(q_pos), _ptr(idx), idx.stride(0), _ptr(count), _ptr(ws),
+                                        0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("lsa_tree_select", st)
 
 
 def lsa_hi_workspace_size(B, L, P, Bsub, M, K, sink, window):

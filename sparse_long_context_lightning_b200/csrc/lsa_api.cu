@@ -106,6 +106,41 @@ static MsaLayout msa_ws_layout(int64_t B, int64_t L, int G, int KB) {
   return m;
 }
 
+// Scratch layout of lsa_tree_select: parent scores [B, ldp] fp32 | kept parents [B, M2] | count [B] |
+// candidate scores [B, ldc] fp32 | candidate buckets [B, ldc] int32 | selected slots [B, M] | count [B] |
+// kept buckets [B, M] | count [B] | the parents' split [3, NP, 128] bf16.
+struct TreeLayout {
+  int64_t ldp, n_cand, ldc;
+  size_t o_kp, o_kpc, o_cs, o_cid, o_pos, o_posc, o_kb, o_kbc, o_split, total;
+};
+static TreeLayout tree_ws_layout(int64_t B, int64_t NP, int F, int M2, int M) {
+  TreeLayout t;
+  t.ldp = (NP + 3) / 4 * 4;
+  t.n_cand = static_cast<int64_t>(M2) * F;
+  t.ldc = (t.n_cand + 3) / 4 * 4;
+  const size_t b = static_cast<size_t>(B);
+  size_t o = align_up(b * t.ldp * 4, 256);
+  t.o_kp = o;
+  o = align_up(o + b * M2 * 4, 256);
+  t.o_kpc = o;
+  o = align_up(o + b * 4, 256);
+  t.o_cs = o;
+  o = align_up(o + b * t.ldc * 4, 256);
+  t.o_cid = o;
+  o = align_up(o + b * t.ldc * 4, 256);
+  t.o_pos = o;
+  o = align_up(o + b * M * 4, 256);
+  t.o_posc = o;
+  o = align_up(o + b * 4, 256);
+  t.o_kb = o;
+  o = align_up(o + b * M * 4, 256);
+  t.o_kbc = o;
+  o = align_up(o + b * 4, 256);
+  t.o_split = o;  // the parents' exact three-part bf16 split (tensor-core scoring of level 2)
+  t.total = align_up(o + static_cast<size_t>(NP) * 128 * 2 * 3, 256);
+  return t;
+}
+
 }  // namespace lsa
 
 using namespace lsa;
@@ -341,6 +376,68 @@ int lsa_msa_select(const void* q_idx, const float* w, const void* k_idx, int64_t
   if (st == LSA_OK) st = launch_shift_qpos(q_pos, B, G, -1, qp1, s);
   if (st == LSA_OK) st = launch_topk_mode(bs, m.ld_nb, B * G, m.nb, KB, 0, 0, qp1, 2, 128, kept, KB, kcnt, KB, s);
   if (st == LSA_OK) st = launch_msa_expand(kept, KB, kcnt, G, 128, q_pos, B, idx, gmask, idx_ld, count, s);
+  return st;
+}
+
+int lsa_tree_parents(const float* centroids, int64_t NB, int d_I, int F, float* parents, void* stream) {
+  LSA_CHECK_ARG(NB >= 0 && d_I >= 1 && d_I <= 128 && F >= 1);
+  if (NB == 0) return LSA_OK;
+  LSA_CHECK_ARG(centroids && parents);
+  return launch_tree_parents(centroids, NB, d_I, F, parents, static_cast<cudaStream_t>(stream));
+}
+
+size_t lsa_tree_workspace_size(int64_t B, int64_t NP, int F, int M2, int M) {
+  if (B < 0 || NP < 0 || F < 1 || M2 < 1 || M < 1) return static_cast<size_t>(-1);
+  return tree_ws_layout(B, NP, F, M2, M).total;
+}
+
+int lsa_tree_select(const void* q_idx, const float* w, int64_t B, int H_I, int d_I, const float* centroids,
+                    int64_t NB, const float* parents, int64_t NP, int F, const int32_t* members, int bsz, int M2,
+                    int M, int sink, int window, int64_t L, const int64_t* q_pos, int32_t* idx, int64_t idx_ld,
+                    int32_t* count, void* ws, size_t ws_bytes, void* stream) {
+  LSA_CHECK_ARG(B >= 0 && NB >= 1 && NB < (int64_t(1) << 31) && F >= 1 && NP == cdiv(NB, F) && bsz >= 1);
+  LSA_CHECK_ARG(M2 >= 1 && M2 <= 1024 && M >= 1 && M <= 1024 && static_cast<int64_t>(M2) * F < (int64_t(1) << 30));
+  LSA_CHECK_ARG(sink >= 0 && window >= 0 && L >= 1 && H_I >= 1 && H_I <= 64);
+  LSA_CHECK_ARG(static_cast<int64_t>(M) * bsz + sink + window <= 8192);
+  LSA_CHECK_ARG(idx_ld >= static_cast<int64_t>(M) * bsz + sink + window);
+  if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
+  if (B == 0) return LSA_OK;
+  LSA_CHECK_ARG(B <= 65535);
+  LSA_CHECK_ARG(q_idx && w && centroids && parents && members && q_pos && idx && count);
+  LSA_CHECK_ARG(aligned16(q_idx) && aligned16(centroids) && aligned16(parents));
+  const TreeLayout t = tree_ws_layout(B, NP, F, M2, M);
+  if (ws == nullptr || !aligned256(ws) || ws_bytes < t.total) return LSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  float* pscore = reinterpret_cast<float*>(base);
+  int32_t* kp = reinterpret_cast<int32_t*>(base + t.o_kp);
+  int32_t* kpc = reinterpret_cast<int32_t*>(base + t.o_kpc);
+  float* cscore = reinterpret_cast<float*>(base + t.o_cs);
+  int32_t* cid = reinterpret_cast<int32_t*>(base + t.o_cid);
+  int32_t* kpos = reinterpret_cast<int32_t*>(base + t.o_pos);
+  int32_t* kposc = reinterpret_cast<int32_t*>(base + t.o_posc);
+  int32_t* kb = reinterpret_cast<int32_t*>(base + t.o_kb);
+  int32_t* kbc = reinterpret_cast<int32_t*>(base + t.o_kbc);
+  // level 2: every parent centre scored -- on the tensor cores from the parents' exact bf16 split where the
+  // shape tiles (fp32-accurate, as the Flat path), else on the CUDA cores -- and the M2 best kept
+  int st;
+  if (d_I == 128 && (H_I == 32 || H_I == 64) && NP >= 128 && NP < (int64_t(1) << 29)) {
+    void* split = base + t.o_split;
+    st = launch_split_bf16x3(parents, NP * 128, split, s);
+    if (st == LSA_OK) st = launch_centroid_score_tc(q_idx, w, split, B, H_I, NP, pscore, t.ldp, s);
+  } else {
+    st = launch_centroid_score(q_idx, w, parents, B, H_I, d_I, NP, pscore, t.ldp, s);
+  }
+  if (st == LSA_OK) st = launch_topk_mode(pscore, t.ldp, B, NP, M2, 0, 0, q_pos, 1, 1, kp, M2, kpc, M2, s);
+  // level 1: the kept parents' children, scored by gather; the M best candidate slots
+  if (st == LSA_OK)
+    st = launch_tree_child_score(q_idx, w, B, H_I, d_I, centroids, NB, F, kp, M2, kpc, t.n_cand, cscore, cid, t.ldc,
+                                 s);
+  if (st == LSA_OK) st = launch_topk_mode(cscore, t.ldc, B, t.n_cand, M, 0, 0, q_pos, 1, 1, kpos, M, kposc, M, s);
+  if (st == LSA_OK) st = launch_tree_map(kpos, M, kposc, cid, t.ldc, t.n_cand, B, kb, M, kbc, s);
+  // the kept buckets' members, sink and window (Flat expansion)
+  if (st == LSA_OK)
+    st = launch_bucket_expand(kb, M, kbc, members, bsz, sink, window, 0, q_pos, B, idx, idx_ld, count, idx_ld, s);
   return st;
 }
 

@@ -243,6 +243,80 @@ def test_microblock_select_paths(path):
     _bucket_case(L=4 * 16384 + 3, B=4, M=512, bsz=4, sink=4, window=128, flat=False, path=path)
 
 
+def _tree_run(L, B, bsz, F, M2, M, sink, window, q_pos=None):
+    """lsa_tree_select against the oracle's two-level search on the fp64 pooled keys.  Returns the GPU rows."""
+    wl = S.Workload("tr", L=L, B=B, H_I=64, d_I=128, K=M * bsz, H=16, sink=sink, window=window, mode="flat",
+                    bsz=bsz, M=M)
+    q_I, w = S.index_queries(wl)
+    k = S.normal_bf16(S.ST_KI, (L, 128), DEV)
+    members = S.bucket_members(wl).to(DEV)
+    nb = members.shape[0]
+    cen = torch.empty(nb, 128, device=DEV)
+    lsa.lsa_pool_keys(k, cen, bsz, members=members)
+    NP = -(-nb // F)
+    par = torch.empty(NP, 128, device=DEV)
+    lsa.lsa_tree_parents(cen, F, par)
+    qp = torch.full((B,), L - 1, dtype=torch.int64) if q_pos is None else torch.as_tensor(q_pos, dtype=torch.int64)
+    kmax = M * bsz + sink + window
+    idx = torch.full((B, kmax), 777, dtype=torch.int32, device=DEV)
+    cnt = torch.empty(B, dtype=torch.int32, device=DEV)
+    ws = lsa.workspace(lsa.lsa_tree_workspace_size(B, NP, F, M2, M))
+    lsa.lsa_tree_select(q_I.to(DEV), w.to(DEV), cen, par, F, members, M2, M, sink, window, L, qp.to(DEV), idx, cnt,
+                        ws)
+    torch.cuda.synchronize()
+    # the parents themselves: fp32 means of the fp32 centres
+    np.testing.assert_allclose(f64(par), O.tree_parents(f64(cen), F), rtol=1e-5, atol=1e-5)
+    mem_np = members.cpu().numpy()
+    reps = O.pool_keys(f64(k), mem_np)
+    parents = O.tree_parents(reps, F)
+    qf, wf = f64(q_I), f64(w)
+    bs = O.bucket_scores(qf, wf, reps)
+    ps = O.bucket_scores(qf, wf, parents)
+    owner = np.empty(L, np.int64)
+    owner[mem_np.reshape(-1)] = np.repeat(np.arange(nb), bsz)
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(B):
+        want, mth, m2th = O.tree_select_row(qf[b], wf[b], reps, mem_np, F, M2, M, int(qp[b]), sink, window)
+        got = idx_h[b, : cnt_h[b]]
+        assert np.all(np.diff(got) > 0) and np.all(idx_h[b, cnt_h[b]:] == -1)
+        if np.array_equal(got, want):
+            continue
+        # only where a bucket ties the M-th candidate, or its parent ties the M2-th parent, within fp32 rounding
+        for c in np.unique(owner[np.setxor1d(got, want)]):
+            near_child = abs(bs[b, c] - mth) <= 1e-5 * abs(mth)
+            near_parent = abs(ps[b, c // F] - m2th) <= 1e-5 * abs(m2th)
+            assert near_child or near_parent, (b, c, bs[b, c], mth, ps[b, c // F], m2th)
+    return idx_h, cnt_h
+
+
+@pytest.mark.parametrize("F,M2,M", [(64, 16, 32), (10, 1000, 32), (1, 40, 32), (100, 1, 100)])
+def test_tree_select(F, M2, M):
+    """Two-level search over 10000 Flat buckets of 64 (ragged last parent for F = 64; F = 10 with M2 = NP is
+    the full beam; F = 1 ranks the buckets themselves; F = 100, M2 = 1 has exactly M candidates)."""
+    L, B = 64 * 10000, 6
+    _tree_run(L, B, 64, F, M2, M, 4, 512, q_pos=[L - 1, L - 1, L // 2, 70000, L - 1, 4000])
+
+
+def test_tree_full_beam_matches_flat():
+    """M2 >= NP: the tree search keeps what lsa_bucket_select (CUDA-core scoring) keeps."""
+    L, B, bsz, M = 64 * 4000, 4, 64, 16
+    idx_t, cnt_t = _tree_run(L, B, bsz, 16, 250, M, 4, 128)
+    wl = S.Workload("tr", L=L, B=B, H_I=64, d_I=128, K=M * bsz, H=16, sink=4, window=128, mode="flat", bsz=bsz, M=M)
+    q_I, w = S.index_queries(wl)
+    k = S.normal_bf16(S.ST_KI, (L, 128), DEV)
+    members = S.bucket_members(wl).to(DEV)
+    cen = torch.empty(members.shape[0], 128, device=DEV)
+    lsa.lsa_pool_keys(k, cen, bsz, members=members)
+    idx = torch.full((B, M * bsz + 4 + 128), 777, dtype=torch.int32, device=DEV)
+    cnt = torch.empty(B, dtype=torch.int32, device=DEV)
+    ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_BUCKET_MIN, B, members.shape[0], M))
+    qp = torch.full((B,), L - 1, dtype=torch.int64, device=DEV)
+    lsa.lsa_bucket_select(q_I.to(DEV), w.to(DEV), cen, members, bsz, M, 4, 128, L, qp, idx, cnt, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(cnt.cpu().numpy(), cnt_t)
+    assert np.array_equal(idx.cpu().numpy(), idx_t)
+
+
 def test_split_representatives_exact():
     """The three bf16 parts sum exactly (in fp64) to the fp32 representative, across magnitudes and signs."""
     g = torch.Generator().manual_seed(5)
