@@ -2,11 +2,21 @@
  * lsa.h -- C ABI of the token-level sparse-attention hot path on B200 (sm_100a).
  *
  * One long-context attention layer, three stages:
- *   1. lightning-indexer scores        lsa_index_score
+ *   1. lightning-indexer scores        lsa_index_score   (bf16 or FP8-e4m3 keys)
  *   2. per-query selection             lsa_topk_select   (top-K + sink/window union)
- *                                      lsa_bucket_select (Flat buckets / 4-token micro-blocks)
- *                                      lsa_pool_keys     (bucket representatives, cached once)
- *   3. sparse attention over the gathered MLA latent rows   lsa_sparse_attn
+ *                                      lsa_topk_refine   (FP8 scan's top-2K re-ranked exactly in bf16)
+ *                                      lsa_bucket_select, lsa_bucket_select_split, lsa_bucket_select_noalloc
+ *                                                        (Flat buckets / 4-token micro-blocks)
+ *                                      lsa_tree_select   (two-level tree search over the Flat buckets)
+ *                                      lsa_hi_select     (pages, then tokens: hierarchical index)
+ *                                      lsa_msa_select    (group-wise 128-token blocks)
+ *      precompute, cached once:        lsa_pool_keys, lsa_split_representatives, lsa_tree_parents
+ *   3. sparse attention over the gathered MLA latent rows
+ *                                      lsa_sparse_attn   (one pass over the selected rows)
+ *                                      lsa_hybrid_attn   (sink + window and sparse rows on two streams,
+ *                                                         merged by log-sum-exp)
+ *                                      lsa_msa_attn      (each head group over its own blocks)
+ *   Scratch sizes: lsa_workspace_size and the per-call *_workspace_size functions.
  *
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library keeps

@@ -83,3 +83,54 @@ def test_argument_checks_launch_nothing(lib):
     # empty batches are a no-op
     assert lib.lsa_topk_select(fake, 4096, 0, 4096, 8, 0, 0, fake, fake, 8, fake, None) == 0
     assert lib.lsa_sparse_attn(fake, fake, 10, fake, 8, fake, 0, 16, 576, 512, 1.0, fake, None, None, 0, None) == 0
+
+
+def test_selection_workspace_sizes(lib):
+    """Host-side size arithmetic of the tree, MSA and HI scratch (no device involved)."""
+    bad = ctypes.c_size_t(-1).value
+    # tree: at least the parent scores, both candidate rows and the parents' bf16 split
+    t = lib.lsa_tree_workspace_size(8, 2442, 64, 64, 32)
+    assert t % 256 == 0 and t >= 8 * 2444 * 4 + 2 * 8 * 4096 * 4 + 3 * 2442 * 128 * 2
+    assert lib.lsa_tree_workspace_size(8, 2442, 0, 64, 32) == bad
+    assert lib.lsa_tree_workspace_size(-1, 2442, 64, 64, 32) == bad
+    # MSA selection: block scores for every (query, group)
+    m = lib.lsa_msa_workspace_size(16, 131072, 8, 16)
+    assert m % 256 == 0 and m >= 16 * 8 * 1024 * 4
+    # MSA attention: per-group rows plus the padded 128-head queries and outputs when G > 1
+    a8 = lib.lsa_msa_attn_workspace_size(16, 129 * 128, 8)
+    a1 = lib.lsa_msa_attn_workspace_size(16, 129 * 128, 1)
+    assert a8 >= 16 * 8 * 129 * 128 * 4 + 16 * 8 * 128 * (576 + 512) * 2 and a1 < a8
+    assert lib.lsa_msa_attn_workspace_size(16, 128, 0) == bad
+    assert lib.lsa_hi_workspace_size(4, 1 << 20, 128, 8, 1024, 2048, 4, 128) > 0
+
+
+def test_selection_argument_checks_launch_nothing(lib):
+    P = ctypes.c_void_p
+    fake = P(0x1000)  # never dereferenced: every call below fails validation first
+    # tree: NP must be ceil(NB / F)
+    assert lib.lsa_tree_select(fake, fake, 1, 64, 128, fake, 1000, fake, 99, 10, fake, 64, 8, 4, 0, 0, 64000, fake,
+                               fake, 256, fake, fake, 1 << 20, None) == -1
+    # tree: M2 above 1024
+    assert lib.lsa_tree_select(fake, fake, 1, 64, 128, fake, 1000, fake, 100, 10, fake, 64, 2000, 4, 0, 0, 64000,
+                               fake, fake, 256, fake, fake, 1 << 20, None) == -1
+    # tree: unsupported d_I
+    assert lib.lsa_tree_select(fake, fake, 1, 64, 48, fake, 1000, fake, 100, 10, fake, 64, 8, 4, 0, 0, 64000, fake,
+                               fake, 256, fake, fake, 1 << 20, None) == -2
+    # tree: workspace missing
+    assert lib.lsa_tree_select(fake, fake, 1, 64, 128, fake, 1000, fake, 100, 10, fake, 64, 8, 4, 0, 0, 64000, fake,
+                               fake, 256, fake, None, 0, None) == -3
+    # tree parents: F = 0
+    assert lib.lsa_tree_parents(fake, 1000, 128, 0, fake, None) == -1
+    # MSA selection: G = 3, and idx_ld too small for G*KB + 1 blocks
+    assert lib.lsa_msa_select(fake, fake, fake, 1, 64, 128, 4096, 3, 4, fake, fake, fake, 1 << 16, fake, fake,
+                              1 << 20, None) == -2
+    assert lib.lsa_msa_select(fake, fake, fake, 1, 64, 128, 4096, 8, 4, fake, fake, fake, 128, fake, fake, 1 << 20,
+                              None) == -1
+    # MSA attention: G = 3; workspace missing
+    assert lib.lsa_msa_attn(fake, fake, 4096, fake, fake, 1024, fake, 1, 128, 576, 512, 3, 1.0, fake, None, fake,
+                            1 << 20, None) == -2
+    assert lib.lsa_msa_attn(fake, fake, 4096, fake, fake, 1024, fake, 1, 128, 576, 512, 8, 1.0, fake, None, None, 0,
+                            None) == -3
+    # empty batches are a no-op
+    assert lib.lsa_tree_select(fake, fake, 0, 64, 128, fake, 1000, fake, 100, 10, fake, 64, 8, 4, 0, 0, 64000, fake,
+                               fake, 256, fake, None, 0, None) == 0
