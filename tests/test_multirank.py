@@ -62,3 +62,21 @@ def test_reference_arm_runs_on_rank_zero_only():
         steps, warmup = 1, 3
 
     assert bench.run_reference(Args(), rank=1, world=2) is None
+
+
+@pytest.mark.timeout(300)
+def test_reference_arm_line_on_rank_zero():
+    """The oracle arm's JSON line carries the contract keys, with its own value repeated in cpu_baseline and e2e."""
+    import bench
+
+    class Args:
+        steps, warmup = 1, 3
+
+    res = bench.run_reference(Args(), rank=0, world=1)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in res, key
+    assert res["impl"] == "reference" and res["value"] > 0 and res["steps"] == 1
+    assert res["cpu_baseline"]["value"] == res["value"] and res["cpu_baseline"]["kind"] == "oracle"
+    assert res["e2e"]["value"] == res["value"] and res["e2e"]["h2d_bytes_per_step"] == 0
+    assert res["metric"] == "sparse decode queries/s @L=128K,K=2048"
