@@ -408,6 +408,17 @@ const char* lsa_last_error(void);
 /* lsa_version -- library version string. */
 const char* lsa_version(void);
 
+/*
+ * lsa_device_status -- whether a tensor-core kernel gave up a bounded wait.
+ *   Every wait of the tensor-core kernels (indexer, re-rank re-score, attention) on an mbarrier is bounded
+ *   (2 s of globaltimer); a wait that runs out sets a device flag, the kernel tears down (its TMEM freed) and
+ *   its outputs for that launch are not valid.  This call synchronises `stream`, then reads and clears the
+ *   flags: LSA_ERR_TIMEOUT if any was set since the previous call (lsa_last_error names the kernels),
+ *   LSA_ERR_CUDA if the stream or the flag read failed, else LSA_OK.  Not part of the hot path (it blocks the
+ *   host); meant for a serving loop's periodic health check.
+ */
+int lsa_device_status(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -54,6 +54,7 @@ SIGNATURES = {
     "lsa_msa_attn": (_I32, [_P, _P, _I64, _P, _P, _I64, _P, _I64, _I32, _I32, _I32, _I32, _F32, _P, _P, _P, _SZ, _P]),
     "lsa_sparse_attn": (_I32, [_P, _P, _I64, _P, _I64, _P, _I64, _I32, _I32, _I32, _F32, _P, _P, _P, _SZ, _P]),
     "lsa_workspace_size": (_SZ, [_I32, _I64, _I64, _I32, _I32, _I32, _I32]),
+    "lsa_device_status": (_I32, [_P]),
     "lsa_strerror": (ctypes.c_char_p, [_I32]),
     "lsa_last_error": (ctypes.c_char_p, []),
     "lsa_version": (ctypes.c_char_p, []),
@@ -172,6 +173,11 @@ def lsa_bucket_select_split(q_idx, w, split, members, bsz, M, sink, window, L, q
                                                 idx.stride(0), _ptr(count), _ptr(ws),
                                                 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check("lsa_bucket_select_split", st)
+
+
+def lsa_device_status(stream=None):
+    """Synchronise the stream and raise if a tensor-core kernel gave up a bounded wait since the last check."""
+    _check("lsa_device_status", load_library().lsa_device_status(_stream(stream)))
 
 
 def lsa_tree_parents(centroids, F, parents, stream=None):

@@ -747,4 +747,15 @@ int launch_hybrid_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   return LSA_OK;
 }
 
+// The kernel's give-up flag, read and cleared (1: a bounded wait gave up since the last call; -1: CUDA error)
+int take_attn_timeout() {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_attn_tc_timeout, sizeof(int)) != cudaSuccess) return -1;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_attn_tc_timeout, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
+}
+
 }  // namespace lsa

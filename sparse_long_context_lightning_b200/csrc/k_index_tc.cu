@@ -459,4 +459,15 @@ int launch_centroid_score_tc(const void* q, const float* w, const void* split, i
   return launch_tc<false, 3>(q, nullptr, w, split, nullptr, B, H_I, NB, nullptr, scores, ld, s);
 }
 
+// The kernel's give-up flag, read and cleared (1: a bounded wait gave up since the last call; -1: CUDA error)
+int take_index_timeout() {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_index_tc_timeout, sizeof(int)) != cudaSuccess) return -1;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_index_tc_timeout, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
+}
+
 }  // namespace lsa

@@ -372,4 +372,15 @@ int launch_refine(const void* q, const float* w, const void* k, int64_t B, int H
   return cuda_status(cudaGetLastError());
 }
 
+// The kernel's give-up flag, read and cleared (1: a bounded wait gave up since the last call; -1: CUDA error)
+int take_rescore_timeout() {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_rescore_tc_timeout, sizeof(int)) != cudaSuccess) return -1;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_rescore_tc_timeout, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
+}
+
 }  // namespace lsa

@@ -149,6 +149,21 @@ extern "C" {
 
 const char* lsa_version(void) { return "lsa-b200 0.1"; }
 
+int lsa_device_status(void* stream) {
+  const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_status(e);
+  const int ix = take_index_timeout(), at = take_attn_timeout(), rs = take_rescore_timeout();
+  if (ix < 0 || at < 0 || rs < 0) return cuda_status(cudaGetLastError());
+  if (ix || at || rs) {
+    char msg[128];
+    std::snprintf(msg, sizeof(msg), "bounded wait gave up in:%s%s%s", ix ? " k_index_score_tc" : "",
+                  at ? " k_sparse_attn_tc" : "", rs ? " k_rescore_tc" : "");
+    set_last_error(msg);
+    return LSA_ERR_TIMEOUT;
+  }
+  return LSA_OK;
+}
+
 const char* lsa_last_error(void) { return g_last_error; }
 
 const char* lsa_strerror(int status) {

@@ -171,6 +171,9 @@ size_t hybrid_attn_ws_bytes(int64_t B, int64_t idx_ld, int H, int sink, int wind
 int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
                        const int32_t* count, int64_t B, int H, float scale, void* out, float* lse,
                        void* ws, size_t ws_bytes, cudaStream_t s);
+int take_index_timeout();
+int take_attn_timeout();
+int take_rescore_timeout();
 int launch_tree_parents(const float* reps, int64_t NB, int d_I, int F, float* parents, cudaStream_t s);
 int launch_tree_child_score(const void* q, const float* w, int64_t B, int H_I, int d_I, const float* reps, int64_t NB,
                             int F, const int32_t* kp, int64_t kp_ld, const int32_t* kpc, int64_t n_cand,
