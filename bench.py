@@ -740,11 +740,12 @@ def run_gpu(args, rank, world, local_rank):
 # ------------------------------------------------------------------------------------------------
 
 
-def oracle_queries(budget_s: float, max_queries: int = 1000):
+def oracle_queries(budget_s: float, max_queries: int = 1000, stages: dict | None = None):
     """Run the fp64 oracle on decode queries of the same workload until budget_s elapses.
 
     Per query: indexer scores over all 131072 keys, top-K + union, attention over the selected
-    latent rows (gathered from the same synthetic cache).  Returns (queries, seconds, threads).
+    latent rows (gathered from the same synthetic cache).  Returns (queries, seconds, threads); when
+    ``stages`` is given it receives each stage's seconds summed over the queries.
     """
     from oracle import lsa_oracle as O
 
@@ -756,17 +757,27 @@ def oracle_queries(budget_s: float, max_queries: int = 1000):
     wf = w.numpy().astype(np.float64)
     q = S.attn_queries(wl)
     done, t0 = 0, time.perf_counter()
+    acc = {"index": 0.0, "topk": 0.0, "attn": 0.0}
     while done < max_queries:
         b = done % wl.B
+        ta = time.perf_counter()
         sc = O.index_score(qf[b: b + 1], wf[b: b + 1], kf, np.array([wl.L - 1]))
+        tb = time.perf_counter()
         sel, _, _ = O.topk_row(sc[0], wl.L - 1, wl.K, wl.sink, wl.window)
+        tc = time.perf_counter()
         rows = S.latent_rows(wl, torch.as_tensor(sel))
         O.sparse_mla_attn(O.bf16_to_f64(q[b].view(torch.int16).numpy()), O.bf16_to_f64(rows.view(torch.int16).numpy()),
                           wl.scale)
+        td = time.perf_counter()
+        acc["index"] += tb - ta
+        acc["topk"] += tc - tb
+        acc["attn"] += td - tc
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
+    if stages is not None:
+        stages.update(acc)
     return done, dt, torch.get_num_threads()
 
 
@@ -835,10 +846,12 @@ def main():
     res = run_gpu(args, rank, world, local_rank)
     if res is not None:
         if not args.no_cpu_baseline and world == 1:
-            n, dt, _ = oracle_queries(12.0)
+            st = {}
+            n, dt, _ = oracle_queries(12.0, stages=st)
             res["cpu_baseline"] = {"value": round(n / dt, 4), "unit": "queries/s", "cores": blas_threads(),
                                    "kind": "oracle", "sample": f"{n} decode queries of the workload "
-                                                                f"(fp64 indexer over L=131072, top-K, attention)"}
+                                                                f"(fp64 indexer over L=131072, top-K, attention)",
+                                   "stage_queries_per_s": {k: round(n / v, 3) for k, v in st.items() if v > 0}}
         print(json.dumps(res), flush=True)
     if world > 1:
         torch.distributed.barrier()
