@@ -475,6 +475,25 @@ def test_msa_local_block_only_near_the_start():
     assert pos.tolist() == list(range(10)) and kth == -np.inf
 
 
+def test_msa_block_ties_go_to_the_lower_block_and_max_not_sum():
+    """One head, w = 1, q = (1,), blocks of 2: a token's score is max(0, k), a block's the max of its tokens'.
+
+    Tokens 0..7 hold k = (3, 0 | 1, 1 | 3, -5 | 0, 0), blocks 0..3 score 3, 1, 3, 0; the query sits at 9 (local
+    block 4).  KB = 1 keeps block 0 (tied with block 2: the lower block wins); KB = 2 keeps blocks 0 and 2.  With
+    block 1 raised to (2, 2) its max (2) is still below 3 while its ReLU sum (4) would beat blocks 0 and 2 (3
+    each): the max, not a sum, decides."""
+    q, w = np.array([[1.0]]), np.array([1.0])
+    k = np.array([[3.0], [0.0], [1.0], [1.0], [3.0], [-5.0], [0.0], [0.0], [2.0], [7.0]])
+    (pos1, kth1), = O.msa_select_row(q, w, k, 9, G=1, block=2, KB=1)
+    assert pos1.tolist() == [0, 1, 8, 9] and kth1 == 3.0
+    (pos2, kth2), = O.msa_select_row(q, w, k, 9, G=1, block=2, KB=2)
+    assert pos2.tolist() == [0, 1, 4, 5, 8, 9] and kth2 == 3.0
+    k2 = k.copy()
+    k2[2:4] = 2.0
+    (pos3, _), = O.msa_select_row(q, w, k2, 9, G=1, block=2, KB=2)
+    assert pos3.tolist() == [0, 1, 4, 5, 8, 9]
+
+
 # --------------------------------------------------------------------------
 # D-LSA Tree: two-level search
 # --------------------------------------------------------------------------
