@@ -308,7 +308,10 @@ size_t lsa_msa_workspace_size(int64_t B, int64_t L, int G, int KB);
  *   each (query, group) pair runs the tensor-core attention as one 128-head query whose first 128 / G rows are
  *   the group's heads and whose other rows are zero (outputs dropped).  The "KV-outer" form (each KV tile
  *   loaded once for every group that kept it) is not built.
- *   H = 128, G in {1, 2, 4, 8}.  ws: lsa_msa_attn_workspace_size(B, idx_ld, G) bytes.
+ *   q [B, 128, 576] bf16, kv [L, 576] bf16 (value = first 512 dims), idx / gmask / count as lsa_msa_select
+ *   writes them (idx_ld <= 65536), out [B, 128, 512] bf16, lse [B, 128] fp32 or NULL; all 16-byte aligned.
+ *   H = 128, d_qk = 576, d_v = 512, G in {1, 2, 4, 8}, B*G <= 65535.
+ *   ws: lsa_msa_attn_workspace_size(B, idx_ld, G) bytes.
  */
 int lsa_msa_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, const uint8_t* gmask,
                  int64_t idx_ld, const int32_t* count, int64_t B, int H, int d_qk, int d_v, int G,
