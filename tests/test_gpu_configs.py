@@ -5,7 +5,6 @@ and last) of the 8192-query causal prefill chunk.  The 10M-token Flat workload k
 cache on the device; the oracle rebuilds every representative from the member keys in fp64.
 """
 
-import math
 
 import numpy as np
 import pytest
@@ -15,7 +14,7 @@ import lsa_synth as S
 import sparse_long_context_lightning_b200 as lsa
 from oracle import lsa_oracle as O
 
-from gpu_common import ATTN_REL, Decode, attn_rel_err, check_index_sets, dequant_rows, f64, run_oracle_attention
+from gpu_common import ATTN_REL, Decode, attn_rel_err, f64, run_oracle_attention
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
