@@ -336,7 +336,12 @@ size_t lsa_msa_attn_workspace_size(int64_t B, int64_t idx_ld, int G);
  *     larger requests return LSA_ERR_WORKSPACE before anything is launched (lsa_last_error() gives
  *     the sizes).  Flat selection over 156250 buckets fits up to B = 13 queries.
  *   - Set-up: the first call on a device looks up the buffer's device address (cudaGetSymbolAddress,
- *     with that device current) and caches it; make that first call before any stream capture.
+ *     with that device current) and caches it; make that first call before any stream capture.  Under
+ *     lazy module loading (the CUDA 12 default) that lookup also loads the library's module on the
+ *     device, which is when the runtime creates the 8 MiB buffer: a caller that must not see any
+ *     allocation at selection time makes one warm-up call beforehand.  Later calls allocate nothing.
+ *     The cached address belongs to the device's primary context; after cudaDeviceReset on that
+ *     device, calling this entry point there again is not supported.
  *   - Sharing: every call on a device uses the same buffer, which keeps the last call's contents
  *     (nothing in it needs clearing: each call writes what it reads).  Calls whose work overlaps on
  *     the GPU (concurrent streams, or threads without ordering between their streams) race on it;

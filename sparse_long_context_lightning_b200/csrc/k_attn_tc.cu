@@ -299,7 +299,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     if (ntiles > 0) {
       // Q row h, dims [0, 384) -> TMEM lane h, columns TM_Q + 32 kb + j hold dims 64 kb + 2j, 64 kb + 2j + 1;
       // read from the TMA staging (128-byte swizzle: chunk c of row h at ((c ^ h) & 7) * 16)
-      if (!mbar_spin(qst_full, 0)) ok = false;
+      // every wait of these warps is decided warp-wide: the TMEM loads and stores that follow are warp-collective
+      // (.sync.aligned) and must be executed by all 32 lanes or by none
+      if (!__all_sync(0xffffffffu, mbar_spin(qst_full, 0))) ok = false;
       #pragma unroll 1
       for (int kb = 0; kb < AT_KB_TQ; ++kb) {
         const unsigned char* src = st_s + AT_STAGE_BYTES + kb * AT_H * 128 + h * 128;
@@ -323,7 +325,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       const int sb = i & 1;
       const int nvalid = min(AT_T, nrows - i * AT_T);
       uint32_t sr[32];
-      if (!mbar_spin(&s_full[sb], (i >> 1) & 1)) {
+      if (!__all_sync(0xffffffffu, mbar_spin(&s_full[sb], (i >> 1) & 1))) {
         ok = false;
         break;
       }
@@ -364,12 +366,14 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       const float psum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
       l = l * alpha + psum;
       // the previous P . V has finished: the P buffer is free and O is stable
-      if (i > 0 && !mbar_spin(pv_done, (i - 1) & 1)) {
+      if (i > 0 && !__all_sync(0xffffffffu, mbar_spin(pv_done, (i - 1) & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      if (resc) {
+      // a warp rescales its O rows when any of its heads' running max grew (alpha = 1 for the other lanes): the
+      // TMEM loads / stores are warp-collective, so the branch must not depend on the lane
+      if (__any_sync(0xffffffffu, resc)) {
         #pragma unroll 1
         for (int k = 0; k < 8; ++k) {
           uint32_t o[32];
@@ -398,7 +402,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       abort_flag = 1;
     }
     // ---- epilogue
-    const bool have = ok && ntiles > 0 && mbar_spin(pv_done, (ntiles - 1) & 1);
+    const bool have = __all_sync(0xffffffffu, ok && ntiles > 0 && mbar_spin(pv_done, (ntiles - 1) & 1));
     tc_fence_after();
     const int64_t orow = static_cast<int64_t>(b) * AT_H + h;
     // O (row h = this thread's TMEM lane) is staged in the stage memory -- free once the last P.V completed --

@@ -287,8 +287,10 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     const int nq = 64 / a.H_I;  // queries in this warp's 64 columns (1 or 2)
     for (int i = 0; i < n_my; ++i) {
       const int buf = i & 1;
-      if (!mbar_wait(&tfull[buf], (i >> 1) & 1)) {
+      // decided warp-wide: the TMEM loads below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (i >> 1) & 1))) {
         atomicExch(&g_index_tc_timeout, 1);
+        abort_flag = 1;
         break;
       }
       tc_fence_after();

@@ -235,11 +235,12 @@ __global__ void __launch_bounds__(RT_THREADS, 2)
       fence_proxy_async_smem();  // generic stores read by the tensor cores
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
-      ok = mbar_spin(q_ready, 0);  // the weights of every epilogue warp are visible
+      ok = __all_sync(0xffffffffu, mbar_spin(q_ready, 0));  // the weights of every epilogue warp are visible
     }
     for (int i = 0; ok && i < nmine; ++i) {
       const int t = split + i * nsplit, ab = i & 1;
-      if (!mbar_spin(&acc_full[ab], (i >> 1) & 1)) {
+      // decided warp-wide: the TMEM loads below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_spin(&acc_full[ab], (i >> 1) & 1))) {
         ok = false;
         break;
       }

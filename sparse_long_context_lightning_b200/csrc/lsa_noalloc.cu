@@ -24,7 +24,11 @@ std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_bucket_scratch on the current device.  The name is only a host-side stand-in:
-// the address must come from the runtime, once per device, with that device current.
+// the address must come from the runtime, once per device, with that device current.  With lazy module
+// loading (the CUDA 12 default) this lookup is also what loads the library's module on the device, so
+// the first call on a device is the one that creates the 8 MiB buffer there.  The cached address
+// belongs to the device's primary context: after cudaDeviceReset on that device it is stale, and
+// calling this entry point on that device again is not supported.
 int scratch_for_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -75,9 +79,12 @@ int lsa_bucket_select_noalloc(const void* q_idx, const float* q_scale, const flo
   const int st = lsa::scratch_for_current_device(&scratch);
   if (st != LSA_OK) return st;
   // Nothing in this scratch has to start at zero: every byte the selection reads is written first
-  // within the same call.
+  // within the same call.  The size passed on is the smaller workspace's, not the whole buffer: given
+  // more, lsa_bucket_select would take its tensor-core branch (which stores a split copy of the
+  // representatives) for the shapes where that copy fits, and this entry point promises the CUDA-core
+  // scoring for every shape.
   return lsa_bucket_select(q_idx, q_scale, w, dtype, B, H_I, d_I, centroids, NB, members, bsz, M, sink, window, L,
-                           q_pos, idx, idx_ld, count, scratch, lsa::kNoAllocScratchBytes, stream);
+                           q_pos, idx, idx_ld, count, scratch, need, stream);
 }
 
 }  // extern "C"

@@ -7,11 +7,14 @@ scratch: index sets are integer results, so they must match exactly, on two call
 is collected last so that a run stopping at the first failure has already run every other test.
 """
 
+import numpy as np
 import pytest
 import torch
 
 import lsa_synth as S
 import sparse_long_context_lightning_b200 as lsa
+from oracle import lsa_oracle as O
+from gpu_common import TIE_REL, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -33,12 +36,20 @@ def _case(L, B, M, bsz, sink, window, flat):
     return q_I, w, cen, members, qp, kmax, nb
 
 
-@pytest.mark.parametrize("flat", [True, False])
-def test_noalloc_matches_allocating_entry_point(flat):
-    if flat:
-        L, B, M, bsz, sink, window = 64 * 20000, 8, 32, 64, 4, 512
-    else:
-        L, B, M, bsz, sink, window = 4 * 16384 + 3, 4, 512, 4, 4, 128
+# (flat, L, B, M, bsz, sink, window).  The small cases (2048 and 4096 representatives) are shapes where the
+# whole static buffer would also hold the tensor-core path's split copy of the representatives; the entry
+# point must still score on the CUDA cores, as the smaller workspace does.
+CASES = {
+    "flat-20000": (True, 64 * 20000, 8, 32, 64, 4, 512),
+    "micro-16384": (False, 4 * 16384 + 3, 4, 512, 4, 4, 128),
+    "flat-2048": (True, 64 * 2048, 4, 32, 64, 4, 512),
+    "micro-4096": (False, 4 * 4096 + 2, 3, 64, 4, 4, 128),
+}
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_noalloc_matches_allocating_entry_point(case):
+    flat, L, B, M, bsz, sink, window = CASES[case]
     q_I, w, cen, members, qp, kmax, nb = _case(L, B, M, bsz, sink, window, flat)
     ref_idx = torch.empty(B, kmax, dtype=torch.int32, device=DEV)
     ref_cnt = torch.empty(B, dtype=torch.int32, device=DEV)
@@ -68,3 +79,48 @@ def test_noalloc_rejects_requests_beyond_the_static_buffer():
         lsa.lsa_bucket_select_noalloc(q_I, w, cen, members, 64, M, 4, 512, NB * 64, qp, idx, cnt)
     assert e.value.status == -3  # LSA_ERR_WORKSPACE
     assert b"static buffer" in lsa.load_library().lsa_last_error()
+
+
+@pytest.mark.parametrize("case", ["flat-2048", "micro-4096"])
+def test_noalloc_small_tables_match_the_oracle(case):
+    """With few representatives the result is also the oracle's selection (ties at the M-th score aside)."""
+    flat, L, B, M, bsz, sink, window = CASES[case]
+    q_I, w, cen, members, qp, kmax, nb = _case(L, B, M, bsz, sink, window, flat)
+    idx = torch.full((B, kmax), 99, dtype=torch.int32, device=DEV)
+    cnt = torch.full((B,), -7, dtype=torch.int32, device=DEV)
+    lsa.lsa_bucket_select_noalloc(q_I, w, cen, members, bsz, M, sink, window, L, qp, idx, cnt)
+    torch.cuda.synchronize()
+    k = S.normal_bf16(S.ST_KI, (L, 128), "cpu")
+    mem_np = members.cpu().numpy() if flat else None
+    reps = O.pool_keys(f64(k), mem_np) if flat else O.pool_keys(f64(k), block=bsz)
+    bs = O.bucket_scores(f64(q_I.cpu()), f64(w.cpu()), reps)
+    owner = {}
+    if flat:
+        for c, row in enumerate(mem_np):
+            for x in row:
+                owner[int(x)] = c
+    idx_h, cnt_h, qp_h = idx.cpu().numpy(), cnt.cpu().numpy(), qp.cpu().numpy()
+    for b in range(B):
+        want, mth, _ = O.bucket_select_row(bs[b], int(qp_h[b]), M, sink, window, members=mem_np,
+                                           block=None if flat else bsz)
+        got = idx_h[b, : cnt_h[b]]
+        assert np.all(np.diff(got) > 0) and np.all(idx_h[b, cnt_h[b]:] == -1)
+        for x in np.setxor1d(got, want).tolist():
+            c = owner[x] if flat else x // bsz
+            assert abs(bs[b, c] - mth) <= TIE_REL * abs(mth), (b, x, bs[b, c], mth)
+
+
+def test_noalloc_second_call_allocates_nothing():
+    """After a first call on the device (which may load the module and with it the static buffer), a
+    further call leaves the device's free memory unchanged."""
+    flat, L, B, M, bsz, sink, window = CASES["flat-2048"]
+    q_I, w, cen, members, qp, kmax, nb = _case(L, B, M, bsz, sink, window, flat)
+    idx = torch.empty(B, kmax, dtype=torch.int32, device=DEV)
+    cnt = torch.empty(B, dtype=torch.int32, device=DEV)
+    lsa.lsa_bucket_select_noalloc(q_I, w, cen, members, bsz, M, sink, window, L, qp, idx, cnt)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    lsa.lsa_bucket_select_noalloc(q_I, w, cen, members, bsz, M, sink, window, L, qp, idx, cnt)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
