@@ -417,15 +417,29 @@ const char* lsa_last_error(void);
 const char* lsa_version(void);
 
 /*
- * lsa_device_status -- whether a tensor-core kernel gave up a bounded wait.
+ * lsa_device_status -- whether a kernel gave up a bounded wait or failed a device-side check.
  *   Every wait of the tensor-core kernels (indexer, re-rank re-score, attention) on an mbarrier is bounded
- *   (2 s of globaltimer); a wait that runs out sets a device flag, the kernel tears down (its TMEM freed) and
- *   its outputs for that launch are not valid.  This call synchronises `stream`, then reads and clears the
- *   flags: LSA_ERR_TIMEOUT if any was set since the previous call (lsa_last_error names the kernels),
+ *   (2 s of globaltimer); a wait that runs out sets a device flag, the kernel's other roles stop at their next
+ *   wait, the issuing threads wait (bounded) for the copies and MMAs they started, TMEM is freed and the
+ *   outputs of that launch are not valid.  The decode attention kernel also checks every selected index
+ *   against [0, L): an index outside it is clamped (the access stays in bounds) and flagged.
+ *   This call synchronises `stream`, then reads and clears the flags: LSA_ERR_TIMEOUT if a wait gave up since
+ *   the previous call, else LSA_ERR_DEVICE_CHECK if an index check failed (lsa_last_error names the kernel),
  *   LSA_ERR_CUDA if the stream or the flag read failed, else LSA_OK.  Not part of the hot path (it blocks the
  *   host); meant for a serving loop's periodic health check.
  */
 int lsa_device_status(void* stream);
+
+/*
+ * lsa_selftest_wait -- exercises the bounded-wait give-up path that lsa_device_status reports.
+ *   The pages have no counterpart: this is a health check of the library's failure reporting.
+ *   Launches one thread that waits on an mbarrier nothing ever completes, for at most limit_ns nanoseconds
+ *   of globaltimer (1 <= limit_ns <= 10^9); the wait runs out, the kernel records the give-up in the same
+ *   way as the tensor-core kernels and returns.  No copy, MMA or TMEM is involved, so nothing is left in
+ *   flight.  The next lsa_device_status on `stream` returns LSA_ERR_TIMEOUT naming "k_selftest_wait", and
+ *   the one after it LSA_OK.  Returns LSA_ERR_INVALID_ARG for a limit outside the range.
+ */
+int lsa_selftest_wait(uint64_t limit_ns, void* stream);
 
 #ifdef __cplusplus
 }

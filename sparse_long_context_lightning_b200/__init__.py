@@ -55,6 +55,7 @@ SIGNATURES = {
     "lsa_sparse_attn": (_I32, [_P, _P, _I64, _P, _I64, _P, _I64, _I32, _I32, _I32, _F32, _P, _P, _P, _SZ, _P]),
     "lsa_workspace_size": (_SZ, [_I32, _I64, _I64, _I32, _I32, _I32, _I32]),
     "lsa_device_status": (_I32, [_P]),
+    "lsa_selftest_wait": (_I32, [ctypes.c_uint64, _P]),
     "lsa_strerror": (ctypes.c_char_p, [_I32]),
     "lsa_last_error": (ctypes.c_char_p, []),
     "lsa_version": (ctypes.c_char_p, []),
@@ -98,7 +99,7 @@ def _stream(stream):
 def _check(fn: str, st: int):
     if st != LSA_OK:
         lib = load_library()
-        raise LsaError(fn, st, lib.lsa_last_error().decode() if st == -4 else "")
+        raise LsaError(fn, st, lib.lsa_last_error().decode() if st in (-4, -5, -6) else "")
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -176,8 +177,14 @@ def lsa_bucket_select_split(q_idx, w, split, members, bsz, M, sink, window, L, q
 
 
 def lsa_device_status(stream=None):
-    """Synchronise the stream and raise if a tensor-core kernel gave up a bounded wait since the last check."""
+    """Synchronise the stream and raise if a kernel gave up a bounded wait (LSA_ERR_TIMEOUT) or failed a
+    device-side index check (LSA_ERR_DEVICE_CHECK) since the last check."""
     _check("lsa_device_status", load_library().lsa_device_status(_stream(stream)))
+
+
+def lsa_selftest_wait(limit_ns, stream=None):
+    """Launch a kernel whose bounded wait on an mbarrier nothing completes runs out after limit_ns."""
+    _check("lsa_selftest_wait", load_library().lsa_selftest_wait(int(limit_ns), _stream(stream)))
 
 
 def lsa_tree_parents(centroids, F, parents, stream=None):

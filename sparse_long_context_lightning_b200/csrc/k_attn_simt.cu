@@ -8,6 +8,8 @@
 namespace lsa {
 namespace {
 
+__device__ int g_attn_simt_check;  // set when a selected index was outside [0, L) (the row was clamped)
+
 constexpr int AS_THREADS = 256;
 constexpr int AS_HG = 16;
 constexpr int AS_TILE = 32;
@@ -48,6 +50,7 @@ __global__ void __launch_bounds__(AS_THREADS) k_attn_simt(const uint16_t* __rest
     for (int i = tid; i < nt * (AS_DQK / 8); i += AS_THREADS) {
       const int r = i / (AS_DQK / 8), c = i % (AS_DQK / 8);
       int64_t s = rowidx[t0 + r];
+      if (s < 0 || s >= L) atomicExch(&g_attn_simt_check, 1);  // clamped below: the access stays in bounds
       s = s < 0 ? 0 : (s >= L ? L - 1 : s);
       const uint4 v = *reinterpret_cast<const uint4*>(kv + s * AS_DQK + c * 8);
       uint32_t* dst = reinterpret_cast<uint32_t*>(kvs + r * AS_STRIDE + c * 8);
@@ -127,6 +130,16 @@ int launch_attn_simt(const void* q, const void* kv, int64_t L, const int32_t* id
   k_attn_simt<<<grid, AS_THREADS, smem, s>>>(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(kv), L, idx,
                                             idx_ld, count, H, scale, static_cast<uint16_t*>(out), lse);
   return cuda_status(cudaGetLastError());
+}
+
+// The index-range flag, read and cleared (1: an index outside [0, L) was clamped since the last call; -1: CUDA
+// error).
+int take_attn_simt_check() {
+  int c = 0;
+  if (cudaMemcpyFromSymbol(&c, g_attn_simt_check, sizeof(int)) != cudaSuccess) return -1;
+  const int zero = 0;
+  if (c != 0 && cudaMemcpyToSymbol(g_attn_simt_check, &zero, sizeof(int)) != cudaSuccess) return -1;
+  return c;
 }
 
 }  // namespace lsa

@@ -33,6 +33,7 @@ namespace {
 using namespace sm100;
 
 __device__ int g_attn_tc_timeout;  // set when a bounded wait of the kernel gave up
+__device__ int g_attn_tc_check;    // set when a selected index was outside [0, L) (the row was clamped)
 
 constexpr int AT_THREADS = 736;  // 16 gather warps, 3 MMA-issuing warps, 4 softmax warps
 // A warp's 16-byte cp.async copies are issue-latency bound (one CTA reaches ~18 GB/s with 4 gather warps,
@@ -204,6 +205,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           }
           continue;
         }
+        if (lane < 2 && i * AT_T + warp * 2 + lane < nrows && (v_raw < 0 || v_raw >= a.L))
+          atomicExch(&g_attn_tc_check, 1);
         const int v = v_raw < 0 ? 0 : (v_raw >= a.L ? a.L - 1 : v_raw);
         #pragma unroll
         for (int k = 0; k < (2 * CPR + 31) / 32; ++k) {
@@ -571,24 +574,47 @@ int make_map(CUtensorMap* m, const void* ptr, bool fp8, int64_t rows, int64_t co
 int launch_attn_simt(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
                      const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, cudaStream_t s);
 
-size_t sparse_attn_ws_bytes(int64_t B, int64_t, int H) {
+int attn2_units(int64_t B, int64_t idx_ld);
+int launch_sparse_attn_2p(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
+                          const int32_t* count, int64_t B, float scale, void* out, float* lse, void* ws, int S,
+                          cudaStream_t s);
+
+// Partial slots per query of lsa_sparse_attn with 128 heads: the two-pass kernel's work units when the batch
+// fits one wave of it (decode batches), else the value-half kernel's splits.
+static int attn_slots(int64_t B, int64_t idx_ld) {
+  const int s2 = attn2_units(B, idx_ld);
+  return s2 > 0 ? s2 : splits_for(B);
+}
+
+size_t sparse_attn_ws_bytes(int64_t B, int64_t idx_ld, int H) {
   if (H != AT_H) return 0;
-  const int S = splits_for(B);
+  const int S = attn_slots(B, idx_ld);
   if (S == 1) return 0;
   const size_t o = align_up(static_cast<size_t>(B) * S * AT_H * 512 * 4, 256);
   return o + align_up(static_cast<size_t>(B) * S * AT_H * 2 * 4, 256);
 }
 
-int attn_launches_per_call(int64_t B, int H) { return (H == AT_H && splits_for(B) > 1) ? 2 : 1; }
+int attn_launches_per_call(int64_t B, int64_t idx_ld, int H) { return (H == AT_H && attn_slots(B, idx_ld) > 1) ? 2 : 1; }
+
+int launch_attn_combine(const float* ws_o, const float* ws_ml, int S, int64_t B, void* out, float* lse,
+                        cudaStream_t s) {
+  LSA_CUDA_TRY(launch_pdl(k_attn_combine, dim3(static_cast<unsigned>(B * AT_H)), dim3(128), 0, s, 0u, ws_o, ws_ml, S,
+                          static_cast<uint16_t*>(out), lse));
+  return LSA_OK;
+}
 
 int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
                        const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, void* ws,
                        size_t ws_bytes, cudaStream_t s) {
   if (B == 0) return LSA_OK;
   if (H != AT_H || L >= (int64_t(1) << 31)) return launch_attn_simt(q, kv, L, idx, idx_ld, count, B, H, scale, out, lse, s);
-  const int S = splits_for(B);
+  const int S2 = attn2_units(B, idx_ld);
+  const int S = S2 > 0 ? S2 : splits_for(B);
   const size_t need = sparse_attn_ws_bytes(B, idx_ld, H);
   if (S > 1 && (ws == nullptr || !aligned256(ws) || ws_bytes < need)) return LSA_ERR_WORKSPACE;
+  if (!aligned16(q)) return LSA_ERR_INVALID_ARG;
+  // decode batches: one SM per (query, row range), rows read once, logits computed once
+  if (S2 > 0) return launch_sparse_attn_2p(q, kv, L, idx, idx_ld, count, B, scale, out, lse, ws, S2, s);
   CUtensorMap tq, tkv;
   int st = make_map(&tq, q, false, B * AT_H, 576, 64, AT_H);
   if (st) return st;
@@ -751,14 +777,16 @@ int launch_hybrid_attn(const void* q, const void* kv, int64_t L, const int32_t* 
   return LSA_OK;
 }
 
-// The kernel's give-up flag, read and cleared (1: a bounded wait gave up since the last call; -1: CUDA error)
-int take_attn_timeout() {
-  int v = 0;
+// The kernel's give-up flag, read and cleared (1: a bounded wait gave up since the last call; -1: CUDA error);
+// *check receives (and clears) the index-range flag.
+int take_attn_timeout(int* check) {
+  int v = 0, c = 0;
   if (cudaMemcpyFromSymbol(&v, g_attn_tc_timeout, sizeof(int)) != cudaSuccess) return -1;
-  if (v != 0) {
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(g_attn_tc_timeout, &zero, sizeof(int)) != cudaSuccess) return -1;
-  }
+  if (cudaMemcpyFromSymbol(&c, g_attn_tc_check, sizeof(int)) != cudaSuccess) return -1;
+  const int zero = 0;
+  if (v != 0 && cudaMemcpyToSymbol(g_attn_tc_timeout, &zero, sizeof(int)) != cudaSuccess) return -1;
+  if (c != 0 && cudaMemcpyToSymbol(g_attn_tc_check, &zero, sizeof(int)) != cudaSuccess) return -1;
+  *check = c;
   return v;
 }
 

@@ -3,6 +3,7 @@
 #include <cstring>
 
 #include "lsa_common.cuh"
+#include "sm100.cuh"
 
 namespace lsa {
 
@@ -141,25 +142,63 @@ static TreeLayout tree_ws_layout(int64_t B, int64_t NP, int F, int M2, int M) {
   return t;
 }
 
+// Self-test of the give-up path: one thread waits on an mbarrier that nothing completes, with a short limit.
+__device__ int g_selftest_timeout;
+__global__ void k_selftest_wait(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  sm100::mbar_init(&bar, 1);
+  sm100::fence_mbar_init();
+  // phase 0 of `bar` never completes: the bounded wait runs out after limit_ns
+  if (!sm100::mbar_wait(&bar, 0, limit_ns)) atomicExch(&g_selftest_timeout, 1);
+}
+
+static int take_selftest_timeout() {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_selftest_timeout, sizeof(int)) != cudaSuccess) return -1;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_selftest_timeout, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
+}
+
 }  // namespace lsa
 
 using namespace lsa;
 
 extern "C" {
 
-const char* lsa_version(void) { return "lsa-b200 0.1"; }
+const char* lsa_version(void) { return "lsa-b200 0.2"; }
+
+int lsa_selftest_wait(uint64_t limit_ns, void* stream) {
+  LSA_CHECK_ARG(limit_ns >= 1 && limit_ns <= 1000000000ull);
+  k_selftest_wait<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  LSA_CUDA_TRY(cudaGetLastError());
+  return LSA_OK;
+}
 
 int lsa_device_status(void* stream) {
   const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_status(e);
-  const int ix = take_index_timeout(), at = take_attn_timeout(), rs = take_rescore_timeout();
-  if (ix < 0 || at < 0 || rs < 0) return cuda_status(cudaGetLastError());
-  if (ix || at || rs) {
-    char msg[128];
-    std::snprintf(msg, sizeof(msg), "bounded wait gave up in:%s%s%s", ix ? " k_index_score_tc" : "",
-                  at ? " k_sparse_attn_tc" : "", rs ? " k_rescore_tc" : "");
+  int a2_check = 0, at_check = 0;
+  const int ix = take_index_timeout(), at = take_attn_timeout(&at_check), rs = take_rescore_timeout();
+  const int a2 = take_attn2_flags(&a2_check), stw = take_selftest_timeout(), sm_check = take_attn_simt_check();
+  if (ix < 0 || at < 0 || rs < 0 || a2 < 0 || stw < 0 || sm_check < 0) return cuda_status(cudaGetLastError());
+  if (ix || at || rs || a2 || stw) {
+    char msg[192];
+    std::snprintf(msg, sizeof(msg), "bounded wait gave up in:%s%s%s%s%s", ix ? " k_index_score_tc" : "",
+                  at ? " k_sparse_attn_tc" : "", rs ? " k_rescore_tc" : "", a2 ? " k_sparse_attn_2p" : "",
+                  stw ? " k_selftest_wait" : "");
     set_last_error(msg);
     return LSA_ERR_TIMEOUT;
+  }
+  if (a2_check || at_check || sm_check) {
+    char msg[192];
+    std::snprintf(msg, sizeof(msg), "device check failed (a selected index outside [0, L); the row was clamped) in:%s%s%s",
+                  a2_check ? " k_sparse_attn_2p" : "", at_check ? " k_sparse_attn_tc" : "",
+                  sm_check ? " k_attn_simt" : "");
+    set_last_error(msg);
+    return LSA_ERR_DEVICE_CHECK;
   }
   return LSA_OK;
 }

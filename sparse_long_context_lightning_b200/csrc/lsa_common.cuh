@@ -172,7 +172,8 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
                        const int32_t* count, int64_t B, int H, float scale, void* out, float* lse,
                        void* ws, size_t ws_bytes, cudaStream_t s);
 int take_index_timeout();
-int take_attn_timeout();
+int take_attn_timeout(int* check);
+int take_attn_simt_check();
 int take_rescore_timeout();
 int launch_tree_parents(const float* reps, int64_t NB, int d_I, int F, float* parents, cudaStream_t s);
 int launch_tree_child_score(const void* q, const float* w, int64_t B, int H_I, int d_I, const float* reps, int64_t NB,
@@ -191,5 +192,6 @@ int launch_msa_expand(const int32_t* kept, int64_t kept_ld, const int32_t* kcnt,
                       cudaStream_t s);
 int launch_shift_qpos(const int64_t* q_pos, int64_t B, int G, int64_t delta, int64_t* out, cudaStream_t s);
 size_t sparse_attn_ws_bytes(int64_t B, int64_t kmax, int H);
-int attn_launches_per_call(int64_t B, int H);
+int attn_launches_per_call(int64_t B, int64_t idx_ld, int H);
+int take_attn2_flags(int* check);
 }  // namespace lsa

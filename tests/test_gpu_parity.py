@@ -489,6 +489,66 @@ def test_topk_refine_exact_on_given_candidates():
         check_index_sets(idx[b].cpu().numpy(), int(cnt[b]), want, ref[b], kth, kmax)
 
 
+def _attn_case(q, kv, idx, cnt, scale, check_rows):
+    B, H = q.shape[0], q.shape[1]
+    kmax = idx.shape[1]
+    out = torch.empty(B, H, 512, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(B, H, device=DEV)
+    ws = lsa.workspace(lsa.lsa_workspace_size(lsa.LSA_OP_ATTN, B, kv.shape[0], kmax, H))
+    lsa.lsa_sparse_attn(q, kv, idx, cnt, scale, out, lse, ws)
+    lsa.lsa_device_status()
+    counts = cnt.cpu().tolist()
+    for b in check_rows:
+        sel = idx[b, : counts[b]].cpu().numpy()
+        ref, ref_lse = run_oracle_attention(q[b], kv, sel, scale)
+        if counts[b] == 0:
+            assert (out[b] == 0).all() and torch.isneginf(lse[b]).all()
+            continue
+        assert attn_rel_err(out[b], ref) <= ATTN_REL, b
+        assert np.abs(f64(lse[b]) - ref_lse).max() <= 1e-3, b
+
+
+def test_sparse_attn_decode_units():
+    """The decode batch shape (16 queries, rows of up to 2048): units of up to 8 tiles of 32 rows, ragged
+    counts (full, one short of a tile, a single row, none) and every query checked."""
+    L, B, H = 40000, 16, 128
+    kv = S.normal_bf16(S.ST_KV, (L, 576), DEV)
+    q = S.normal_bf16(S.ST_Q, (B, H, 576), DEV)
+    counts = [2048, 2047, 2017, 1, 0, 256, 255, 33, 32, 31, 1500, 2048, 2048, 1999, 64, 2000]
+    kmax = 2048
+    rng = np.random.default_rng(16)
+    idx = torch.full((B, kmax), -1, dtype=torch.int32)
+    for b, c in enumerate(counts):
+        idx[b, :c] = torch.from_numpy(np.sort(rng.choice(L, size=c, replace=False)).astype(np.int32))
+    _attn_case(q, kv, idx.to(DEV), torch.tensor(counts, dtype=torch.int32, device=DEV), 1 / math.sqrt(576),
+               range(B))
+
+
+def test_sparse_attn_rescales_within_a_unit():
+    """Logits that grow along each unit's rows by several 2^8 steps for some heads and shrink for others: the
+    running softmax reference moves tile by tile for part of a warp's heads (the lazy rescale of O), and the
+    second value half must replay those rescales exactly."""
+    L, B, H = 32768, 16, 128
+    g = torch.Generator().manual_seed(7)
+    u = torch.randn(576, generator=g, dtype=torch.float64)
+    u /= u.norm()
+    # t(s) ramps 0 -> 500 over each eighth of the cache, so a unit (an eighth of a query's sorted rows) sees it
+    # grow by ~60 per tile: z grows by ~3.7 (q_h . u) in log2 units per tile
+    s = torch.arange(L, dtype=torch.float64)
+    t = 500.0 * ((8.0 * s / L) % 1.0)
+    noise = S.normal_bf16(S.ST_KV, (L, 576), "cpu").double()
+    kv = (t[:, None] * u[None, :] + noise).to(torch.bfloat16).to(DEV)
+    q = S.normal_bf16(S.ST_Q, (B, H, 576), DEV)
+    kmax = 2048
+    rng = np.random.default_rng(17)
+    idx = torch.stack([torch.from_numpy(np.sort(rng.choice(L, size=kmax, replace=False)).astype(np.int32))
+                       for _ in range(B)])
+    counts = [kmax] * B
+    counts[5] = 1111
+    _attn_case(q, kv, idx.to(DEV), torch.tensor(counts, dtype=torch.int32, device=DEV), 1 / math.sqrt(576),
+               range(B))
+
+
 def test_sparse_attn_single_split_many_queries():
     """Enough queries that every query runs as one split (no combine pass)."""
     L, B, H = 30000, 80, 128
