@@ -41,7 +41,8 @@ import lsa_synth as S
 ROOT = os.path.dirname(os.path.abspath(__file__))
 CONFIG = "decode128k"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s), used only when no FP8 measurement is committed
+FP8_PEAK_FILE = os.path.join(ROOT, "profiles", "fp8_peak.json")
 
 
 def peaks():
@@ -50,6 +51,69 @@ def peaks():
         d = json.load(open(p))
         return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def fp8_peak():
+    """(e4m3 dense TFLOP/s burst, sustained, source): the committed measurement of this machine's B200s
+    (`python bench.py --measure-tensor-peaks`), else the bf16 peak x the nominal ratio."""
+    if os.path.exists(FP8_PEAK_FILE):
+        d = json.load(open(FP8_PEAK_FILE))
+        return float(d["fp8_e4m3_tflops"]), float(d["fp8_e4m3_tflops_sustained"]), "measured (profiles/fp8_peak.json)"
+    pk, src = peaks()
+    return pk["bf16_tflops"] * FP8_OVER_BF16, pk["bf16_tflops_sustained"] * FP8_OVER_BF16, src + " bf16 x2 (nominal)"
+
+
+def measure_tensor_peaks(device, seconds: float = 4.0):
+    """Dense GEMM throughput of this GPU with the library GEMMs: torch._scaled_mm e4m3 x e4m3 -> bf16 and
+    torch.matmul bf16, 8192^3 (2 N^3 flops each).  Burst = best of 10 single launches (CUDA events); sustained =
+    back-to-back launches for `seconds`, with the SM clock sampled meanwhile.  No clock or power setting is
+    touched."""
+    n = 8192
+    torch.manual_seed(0)
+    a16 = torch.randn(n, n, device=device, dtype=torch.bfloat16)
+    b16 = torch.randn(n, n, device=device, dtype=torch.bfloat16)
+    a8 = a16.to(torch.float8_e4m3fn)
+    b8 = b16.to(torch.float8_e4m3fn).t().contiguous().t()  # column-major, as _scaled_mm wants
+    one = torch.ones((), device=device, dtype=torch.float32)
+    ops = {"fp8_e4m3": lambda: torch._scaled_mm(a8, b8, scale_a=one, scale_b=one, out_dtype=torch.bfloat16),
+           "bf16": lambda: torch.matmul(a16, b16)}
+    flops = 2.0 * n ** 3
+    res = {}
+    for name, f in ops.items():
+        for _ in range(5):
+            f()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        with ClockSampler(device.index or 0) as clk:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps, t0 = 0, time.perf_counter()
+            e0.record()
+            while time.perf_counter() - t0 < seconds:
+                for _ in range(20):
+                    f()
+                reps += 20
+                torch.cuda.synchronize()
+            e1.record()
+            e1.synchronize()
+            ms = e0.elapsed_time(e1)
+        res[name] = {"burst_tflops": round(flops / (best * 1e-3) / 1e12, 1),
+                     "sustained_tflops": round(flops * reps / (ms * 1e-3) / 1e12, 1), "clocks": clk.summary()}
+    return {"fp8_e4m3_tflops": res["fp8_e4m3"]["burst_tflops"],
+            "fp8_e4m3_tflops_sustained": res["fp8_e4m3"]["sustained_tflops"],
+            "bf16_tflops_same_run": res["bf16"]["burst_tflops"],
+            "bf16_tflops_sustained_same_run": res["bf16"]["sustained_tflops"],
+            "clocks": {k: v["clocks"] for k, v in res.items()},
+            "gpu": torch.cuda.get_device_name(device),
+            "how": "torch._scaled_mm(e4m3 [8192,8192] x e4m3 [8192,8192] col-major, unit scales, bf16 out) and "
+                   "torch.matmul bf16 8192^3, 2*N^3 flops: best of 10 CUDA-event launches (burst) and back-to-back "
+                   f"launches for {seconds:.0f} s (sustained)"}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -204,6 +268,48 @@ STAGE_KERNEL = {"index": ("k_index_score_tc", ["k_index_tc.cu"]),
 LAUNCHES = {"index": 1, "topk": 1, "attn": 1}
 
 
+def dynamic_recall(idx_a, cnt_a, idx_b, cnt_b, q_pos, sink: int, window: int):
+    """Mean and min over rows of |A_dyn & B_dyn| / |B_dyn|, the sink and window positions left out (B is the
+    reference selection)."""
+    ia, ca, ib, cb, qp = (t.cpu().numpy() for t in (idx_a, cnt_a, idx_b, cnt_b, q_pos))
+    rec = []
+    for r in range(ia.shape[0]):
+        lo = max(int(qp[r]) - window + 1, 0) if window > 0 else int(qp[r]) + 1
+        a, b = ia[r, : ca[r]], ib[r, : cb[r]]
+        a = a[(a >= sink) & (a < lo)]
+        b = b[(b >= sink) & (b < lo)]
+        rec.append(np.intersect1d(a, b).size / max(b.size, 1))
+    return {"mean": round(float(np.mean(rec)), 5), "min": round(float(np.min(rec)), 5), "rows": len(rec)}
+
+
+def fp8_decode(device, l2_flush, bf16_step, iters: int = 10):
+    """The decode step with the FP8 indexer (e4m3 scan -> top-2K -> exact bf16 re-rank -> K): per-stage times, the
+    scan's fraction of the measured e4m3 peak, and the recall of its selection against the bf16 path's (which the
+    parity tests pin to the exact top-K up to ties), on the dynamic part."""
+    wl = bf16_step.wl
+    step = DecodeStep(wl, "fp8", device)
+    st = _time_stages([step.index, step.topk, step.attn], l2_flush, iters)
+    step.index()
+    step.topk()
+    bf16_step.index()
+    bf16_step.topk()
+    torch.cuda.synchronize()
+    counts = step.cnt.cpu().numpy()
+    work = algorithmic_work(wl, counts, True)
+    p8, _, p8_src = fp8_peak()
+    res = {"workload": f"{CONFIG} with the e4m3 indexer (per-row scales), top-2K + exact bf16 re-rank to K",
+           "stages": {"index": _stage(st[0], work["index"][1], work["index"][0], p8),
+                      "topk_rerank": _stage(st[1], work["topk"][1]),
+                      "attn": _stage(st[2], work["attn"][1], work["attn"][0], peaks()[0]["bf16_tflops"])},
+           "ms_per_step": round(float(st.sum()), 5), "queries_per_s": round(wl.B / (float(st.sum()) * 1e-3), 1),
+           "fp8_peak_tflops": p8, "fp8_peak_source": p8_src,
+           "recall_vs_bf16_selection": dynamic_recall(step.idx, step.cnt, bf16_step.idx, bf16_step.cnt, step.q_pos,
+                                                      wl.sink, wl.window)}
+    del step
+    torch.cuda.empty_cache()
+    return res
+
+
 def prefill_chunk(device, l2_flush, iters: int = 3):
     """Latency of one causal prefill chunk: 8192 queries at positions 122880..131071 over L = 131072, FP8
     scan + exact bf16 re-rank to K = 2048, sink 4 + window 128, attention over the selected rows.
@@ -231,11 +337,25 @@ def prefill_chunk(device, l2_flush, iters: int = 3):
     per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(iters)])
     ms = float(per.sum(axis=1).mean())
     st = per.mean(axis=0)
-    del step
+    # the FP8 scan's rate against the measured e4m3 peak: 2 H_I d_I flops per visible (query, key) pair
+    pairs = float(sum(int(p) + 1 for p in wl.q_pos().tolist()))
+    scan_flops = 2.0 * wl.H_I * wl.d_I * pairs
+    p8, _, p8_src = fp8_peak()
+    # recall of the FP8 selection against the bf16 path's on every row (bf16 scores into the same buffer)
+    idx8, cnt8 = step.idx.clone(), step.cnt.clone()
+    step.lsa.lsa_index_score(step.q_I, step.w, step.k_bf16, step.q_pos, step.scores)
+    step.lsa.lsa_topk_select(step.scores, wl.L, wl.K, wl.sink, wl.window, step.q_pos, step.idx, step.cnt)
+    torch.cuda.synchronize()
+    rec = dynamic_recall(idx8, cnt8, step.idx, step.cnt, step.q_pos, wl.sink, wl.window)
+    del step, idx8, cnt8
     torch.cuda.empty_cache()
     return {"workload": "prefill: 8192 causal queries (q_pos 122880..131071), L=131072, FP8 scan + bf16 re-rank, "
                         "K=2048 + sink 4 + window 128, H=128", "ms": round(ms, 3),
             "stages_ms": {"index": round(float(st[0]), 3), "topk": round(float(st[1]), 3), "attn": round(float(st[2]), 3)},
+            "index_scan": {"algorithmic_flops": scan_flops, "achieved_tflops": round(scan_flops / (st[0] * 1e-3) / 1e12, 1),
+                           "tensor_frac": round(scan_flops / (st[0] * 1e-3) / 1e12 / p8, 4), "peak_tflops": p8,
+                           "peak_source": p8_src},
+            "recall_vs_bf16_selection": rec,
             "queries_per_s": round(wl.B / (ms * 1e-3), 1), "iterations": iters}
 
 
@@ -413,7 +533,7 @@ def long_context_configs(device, l2_flush, iters: int = 10):
     res["decode1m_fp8"] = {
         "workload": "B=4 decode queries, L=1048576, e4m3 indexer (H_I=64, d_I=128), top-4096 + exact bf16 re-rank "
                     "to K=2048, sink 4 + window 128, H=128",
-        "stages": {"index": _stage(st[0], ix_bytes, ix_flops, FP8_OVER_BF16 * bf16), "topk_rerank": _stage(st[1], tk_bytes),
+        "stages": {"index": _stage(st[0], ix_bytes, ix_flops, fp8_peak()[0]), "topk_rerank": _stage(st[1], tk_bytes),
                    "attn": _stage(st[2], at_bytes)},
         "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
     del step
@@ -573,18 +693,23 @@ def run_gpu(args, rank, world, local_rank):
         launches["topk"] = 4  # top-2K, re-score, top-K of the candidates, assemble
     launches["attn"] = 2 if lsa.lsa_workspace_size(lsa.LSA_OP_ATTN, wl.B, wl.L, step.kmax, wl.H) > 0 else 1  # + combine
 
-    def one_step(ev):
+    def one_step(ev, stage_events: bool):
+        # the timed steps record events only around the whole step, so consecutive kernels overlap their
+        # launches (programmatic dependent launch) as in a serving loop; the stage breakdown comes from a
+        # second pass of the same steps with an event between the stages
         ev[0].record(stream)
         step.index()
-        ev[1].record(stream)
+        if stage_events:
+            ev[1].record(stream)
         step.topk()
-        ev[2].record(stream)
+        if stage_events:
+            ev[2].record(stream)
         step.attn()
         ev[3].record(stream)
 
     for _ in range(args.warmup):
         l2_flush()
-        one_step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+        one_step([torch.cuda.Event(enable_timing=True) for _ in range(4)], True)
     torch.cuda.synchronize()
     counts = step.cnt.cpu().numpy()
 
@@ -596,14 +721,21 @@ def run_gpu(args, rank, world, local_rank):
         t0 = time.perf_counter()
         for i in range(args.steps):
             l2_flush()  # outside the step's events
-            one_step(evs[i])
+            one_step(evs[i], False)
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
     if world > 1:
         torch.distributed.barrier()
-    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(args.steps)])  # ms
-    step_ms = float(per.sum(axis=1).mean())
+    step_ms = float(np.mean([evs[i][0].elapsed_time(evs[i][3]) for i in range(args.steps)]))
+    # stage breakdown (not the headline): the same steps with events between the stages
+    evs_st = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        l2_flush()
+        one_step(evs_st[i], True)
+    torch.cuda.synchronize()
+    per = np.array([[evs_st[i][j].elapsed_time(evs_st[i][j + 1]) for j in range(3)] for i in range(args.steps)])
     stage_ms = per.mean(axis=0)
+    stage_sum_ms = float(per.sum(axis=1).mean())
 
     # e2e: host (pinned) inputs -> H2D -> the three calls -> D2H of the result, every step
     h_q_in = step.q_in.cpu().pin_memory()
@@ -667,18 +799,19 @@ def run_gpu(args, rank, world, local_rank):
     del graph
 
     # max over ranks
-    vals = max_over_ranks(torch.tensor([step_ms, e2e_step, *stage_ms.tolist()], dtype=torch.float64, device=device),
-                          world)
-    step_ms, e2e_step = float(vals[0]), float(vals[1])
-    stage_ms = vals[2:].cpu().numpy()
+    vals = max_over_ranks(torch.tensor([step_ms, e2e_step, stage_sum_ms, *stage_ms.tolist()], dtype=torch.float64,
+                                       device=device), world)
+    step_ms, e2e_step, stage_sum_ms = float(vals[0]), float(vals[1]), float(vals[2])
+    stage_ms = vals[3:].cpu().numpy()
     if rank != 0:
         return None
     prefill = None if (args.no_prefill or world > 1) else prefill_chunk(device, l2_flush)
+    fp8_line = None if (args.no_configs or world > 1 or step.fp8) else fp8_decode(device, l2_flush, step)
     long_ctx = None if (args.no_configs or world > 1) else long_context_configs(device, l2_flush)
 
     pk, pk_src = peaks()
     work = algorithmic_work(wl, counts, step.fp8)
-    tensor_peak = pk["bf16_tflops"] * (FP8_OVER_BF16 if step.fp8 else 1.0)
+    tensor_peak = fp8_peak()[0] if step.fp8 else pk["bf16_tflops"]
     stages = {}
     for j, name in enumerate(("index", "topk", "attn")):
         flops, nbytes = work[name]
@@ -699,7 +832,7 @@ def run_gpu(args, rank, world, local_rank):
     else:
         roof = {"bound": "hbm", "achieved": stages[dom]["achieved_gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": stages[dom]["hbm_frac"]}
-    roof.update({"kernel": kname, "peak_source": pk_src + (" (bf16 x2 nominal ratio)" if dom == "index" and step.fp8 else ""),
+    roof.update({"kernel": kname, "peak_source": fp8_peak()[2] if (dom == "index" and step.fp8) else pk_src,
                  "traffic": committed_traffic(kname)})
     qps = job_rate(wl.B, world, step_ms)
     n_launch = sum(launches.values()) * args.steps
@@ -722,6 +855,10 @@ def run_gpu(args, rank, world, local_rank):
                    "l2": "flushed before every step (256 MB write + 256 MB read), outside the step's CUDA events"},
         "gather_hbm_gbs": stages["attn"]["achieved_gbs"],
         "stages": stages,
+        "stages_sum_ms": round(stage_sum_ms, 5),
+        "stages_note": "per-stage times from a second pass of the same steps with CUDA events between the stages "
+                       "(those events also stop the stages' launches from overlapping); ms_per_step is timed with "
+                       "events around each whole step only",
         "roofline": roof,
         "e2e": {"value": round(job_rate(wl.B, world, e2e_step), 1), "unit": "queries/s",
                 "ms_per_step": round(e2e_step, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
@@ -729,6 +866,7 @@ def run_gpu(args, rank, world, local_rank):
         "gpu_launches": n_launch,
         "clocks": clk.summary(),
         "wall_s_timed_region": round(wall, 4),
+        "fp8_decode": fp8_line,
         "prefill_chunk": prefill,
         "long_context": long_ctx,
     }
@@ -780,6 +918,86 @@ def oracle_queries(budget_s: float, max_queries: int = 1000, stages: dict | None
     return done, dt, torch.get_num_threads()
 
 
+def _oracle_pipeline(wl, O, q_I, w, kf, rows, q_pos_of):
+    """Oracle time per stage over query rows `rows`: indexer scores over the visible keys, top-K with the sink /
+    window union, attention over the selected latent rows.  Returns (rows done, {stage: seconds})."""
+    qf = O.bf16_to_f64(q_I.view(torch.int16).numpy())
+    wf = w.numpy().astype(np.float64)
+    acc = {"index": 0.0, "topk": 0.0, "attn": 0.0}
+    for b in rows:
+        qp = int(q_pos_of(b))
+        ta = time.perf_counter()
+        sc = O.index_score(qf[b: b + 1], wf[b: b + 1], kf[: qp + 1], np.array([qp]))
+        tb = time.perf_counter()
+        sel, _, _ = O.topk_row(sc[0], qp, wl.K, wl.sink, wl.window)
+        tc = time.perf_counter()
+        qa = S.normal_bf16_rows(S.ST_Q, torch.arange(b * wl.H, (b + 1) * wl.H), wl.d_qk)
+        kv = S.latent_rows(wl, torch.as_tensor(sel))
+        O.sparse_mla_attn(O.bf16_to_f64(qa.view(torch.int16).numpy()), O.bf16_to_f64(kv.view(torch.int16).numpy()),
+                          wl.scale)
+        td = time.perf_counter()
+        acc["index"] += tb - ta
+        acc["topk"] += tc - tb
+        acc["attn"] += td - tc
+    return len(rows), acc
+
+
+def oracle_configs():
+    """The oracle on the other workloads, each on a bounded sample, as rows (queries) per second per stage.
+    Input generation and the untimed precompute (representatives) are outside the timed stages."""
+    from oracle import lsa_oracle as O
+
+    def rates(n, acc):
+        tot = sum(acc.values())
+        return {"queries_per_s": round(n / tot, 4), "queries": n,
+                "stage_queries_per_s": {k: round(n / v, 3) for k, v in acc.items() if v > 0}}
+
+    res = {}
+    wl = S.WORKLOADS["tiny"]
+    q_I, w = S.index_queries(wl)
+    kf = O.bf16_to_f64(S.index_keys(wl, q_I).view(torch.int16).numpy())
+    n, acc = _oracle_pipeline(wl, O, q_I, w, kf, [0] * 20, lambda b: wl.L - 1)
+    res["tiny"] = dict(rates(n, acc), sample="the one decode query, 20 times")
+    wl = S.WORKLOADS["decode1m"]
+    q_I, w = S.index_queries(wl)
+    kf = O.bf16_to_f64(S.index_keys(wl, q_I).view(torch.int16).numpy())
+    n, acc = _oracle_pipeline(wl, O, q_I, w, kf, [0], lambda b: wl.L - 1)
+    res["decode1m"] = dict(rates(n, acc), sample="1 of the 4 decode queries (bf16 indexer over all 1048576 keys)")
+    del kf
+    wl = S.WORKLOADS["prefill"]
+    q_I, w = S.index_queries(wl)
+    kf = O.bf16_to_f64(S.index_keys(wl, q_I).view(torch.int16).numpy())
+    qpos = wl.q_pos()
+    n, acc = _oracle_pipeline(wl, O, q_I, w, kf, [0, wl.B // 2, wl.B - 1], lambda b: int(qpos[b]))
+    res["prefill"] = dict(rates(n, acc), sample="3 of the 8192 causal query rows (first, middle, last), bf16 indexer")
+    del kf
+    # flat10m: the oracle's Flat selection and attention for one query over a table of the first 1/16 of the
+    # buckets (their representatives built from their member keys beforehand, like the cached GPU table)
+    wl = S.WORKLOADS["flat10m"]
+    q_I, w = S.index_queries(wl)
+    mem = S.bucket_members(wl)
+    nb = mem.shape[0] // 16
+    msub = mem[:nb]
+    keys = S.index_key_rows(wl, q_I, msub.reshape(-1).long())
+    reps = O.pool_keys(O.bf16_to_f64(keys.view(torch.int16).numpy()).reshape(-1, wl.d_I),
+                       np.arange(nb * wl.bsz).reshape(nb, wl.bsz))
+    qf = O.bf16_to_f64(q_I.view(torch.int16).numpy())
+    wf = w.numpy().astype(np.float64)
+    ta = time.perf_counter()
+    bs = O.bucket_scores(qf[:1], wf[:1], reps)
+    sel, _, _ = O.bucket_select_row(bs[0], wl.L - 1, wl.M, wl.sink, wl.window, members=msub.numpy())
+    tb = time.perf_counter()
+    qa = S.normal_bf16_rows(S.ST_Q, torch.arange(0, wl.H), wl.d_qk)
+    kv = S.latent_rows(wl, torch.as_tensor(sel))
+    O.sparse_mla_attn(O.bf16_to_f64(qa.view(torch.int16).numpy()), O.bf16_to_f64(kv.view(torch.int16).numpy()),
+                      wl.scale)
+    tc = time.perf_counter()
+    res["flat10m"] = {"sample": f"1 decode query; bucket table = the first {nb} of {mem.shape[0]} buckets",
+                      "buckets_scored_and_selected_per_s": round(nb / (tb - ta), 1),
+                      "attention_queries_per_s": round(1.0 / (tc - tb), 3), "attention_rows": int(len(sel))}
+    return res
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -824,8 +1042,13 @@ def main():
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-chunk latency measurement")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the long-context workloads (1M-token FP8 / micro-block decode, 10M-token Flat)")
+    ap.add_argument("--measure-tensor-peaks", action="store_true",
+                    help="measure the dense e4m3 and bf16 GEMM peaks of this GPU, print them as JSON and exit")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.measure_tensor_peaks:
+        print(json.dumps(measure_tensor_peaks(torch.device("cuda", 0))), flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -850,7 +1073,8 @@ def main():
             res["cpu_baseline"] = {"value": round(n / dt, 4), "unit": "queries/s", "cores": blas_threads(),
                                    "kind": "oracle", "sample": f"{n} decode queries of the workload "
                                                                 f"(fp64 indexer over L=131072, top-K, attention)",
-                                   "stage_queries_per_s": {k: round(n / v, 3) for k, v in st.items() if v > 0}}
+                                   "stage_queries_per_s": {k: round(n / v, 3) for k, v in st.items() if v > 0},
+                                   "other_workloads": oracle_configs() if not args.no_configs else None}
         print(json.dumps(res), flush=True)
     if world > 1:
         torch.distributed.barrier()

@@ -8,19 +8,21 @@
 // the units of a decode batch fill the SMs once (one CTA per SM).  Each unit's rows are read once from HBM and
 // its logits are computed once, for all 128 heads:
 //   pass 1  gathers whole rows (16-byte cp.async into the 128-byte-swizzled K-major tile), computes the logits
-//           S = Q C^T on the tensor cores (Q dims [0, 384) as the A operand in TMEM, dims [384, 576) in shared
-//           memory), runs the online softmax, keeps P (bf16) of every tile in shared memory and accumulates
-//           O[:, 0:256) += P V[:, 0:256);
-//   pass 2  gathers only value dims [256, 512) of the same rows again (512 bytes per row, mostly served by L2)
-//           and accumulates O[:, 256:512) += P V[:, 256:512) from the kept P, into the TMEM columns that held S
-//           and Q in pass 1, replaying pass 1's (rare) rescales of the running softmax reference.
-// A 128 x 512 fp32 accumulator is all of TMEM, so the two value halves cannot both live beside Q and S; the
-// second half costs a 512-byte L2 read per row instead of a second CTA that would gather the full rows and
-// recompute the logits.  Units of one query are merged by the combine kernel (log-sum-exp weights).
+//           S = Q C^T on the tensor cores with all of Q (576 dims = 288 columns) as the A operand in TMEM, and
+//           runs the online softmax; P (bf16) of every tile is kept in shared memory.  A stage is released as
+//           soon as its logits MMAs complete, and four warps issue the logits (one tile each, four S buffers),
+//           so four row tiles are in flight;
+//   pass 2  gathers value dims [0, 512) of the same rows again (1 KB per row, mostly served by L2) and
+//           accumulates O = P V for both value halves (all 512 TMEM columns), replaying pass 1's (rare)
+//           rescales of the running softmax reference.
+// A 128 x 512 fp32 accumulator is all of TMEM, so O cannot live beside Q and S: the value dims cost a second
+// (L2) read per row instead of a second CTA that would gather the full rows and recompute the logits.  Units of
+// one query are merged by the combine kernel (log-sum-exp weights).
 //
-// Warp roles (736 threads): warps 0-15 gather (two rows of each tile per warp), 16 and 17 issue the logits
-// MMAs of even / odd tiles (16 owns TMEM), 18 issues the P.V MMAs of both passes, 19-22 move Q into TMEM,
-// run the softmax (one head per thread = one TMEM lane) and write the output.
+// Warp roles (768 threads): warps 0-15 gather (two rows of each tile per warp), 16-19 issue the logits MMAs of
+// tiles j = warp - 16 (mod 4) (16 owns TMEM; 19 also issues pass 2's P.V MMAs), 20-23 move Q into TMEM and run
+// the softmax (one head per thread = one TMEM lane).  The output is written by the twenty gather and softmax
+// warps (five per TMEM lane quarter).
 #include <algorithm>
 
 #include "lsa_common.cuh"
@@ -34,40 +36,38 @@ using namespace sm100;
 __device__ int g_attn2_timeout;  // a bounded wait of the kernel gave up
 __device__ int g_attn2_check;    // a selected index was outside [0, L) (the row was clamped)
 
-constexpr int A2_THREADS = 736;
+constexpr int A2_THREADS = 768;
 constexpr int A2_GATHER_WARPS = 16;
-constexpr int A2_MMA_WARP = 16;   // logits of even tiles; owns TMEM
-constexpr int A2_MMA_WARP2 = 17;  // logits of odd tiles
-constexpr int A2_PV_WARP = 18;    // O += P V (both passes); warps 19-22: softmax and epilogue
+constexpr int A2_LOGIT_WARP0 = 16;  // warps 16-19 issue the logits; 16 owns TMEM
+constexpr int A2_PV_WARP = 19;      // also issues pass 2's P.V
+constexpr int A2_SOFTMAX_WARP0 = 20;  // warps 20-23
 constexpr int A2_T = 32;          // rows per tile
 constexpr int A2_H = 128;         // heads (MMA M)
 constexpr int A2_KB = 9;          // 64-dim K-blocks of a 576-dim row
-constexpr int A2_KB_TQ = 6;       // Q K-blocks held in TMEM (dims [0, 384))
-constexpr int A2_KB_SQ = 3;       // Q K-blocks in shared memory (dims [384, 576))
 constexpr int A2_MAXT = 8;        // tiles per work unit (P of every tile is kept)
-constexpr int A2_STAGES = 3;
-constexpr int A2_O_PITCH = 1040;  // epilogue staging: 1 KB per head row + 16 B (rows in different banks)
-constexpr int A2_QS_BYTES = A2_KB_SQ * A2_H * 128;          // 48 KB
+constexpr int A2_STAGES = 4;      // = the number of logits-issuing warps: tile j uses stage j % 4
+constexpr int A2_QSLOTS = 4;      // Q K-blocks staged at a time (in the P area) on their way into TMEM
 constexpr int A2_KB_BYTES = A2_T * 128;                     // 4 KB: one 64-dim block of a tile
 constexpr int A2_STAGE_BYTES = A2_KB * A2_KB_BYTES;         // 36 KB
+constexpr int A2_QKB_BYTES = A2_H * 128;                    // 16 KB: one 64-dim block of Q
 constexpr int A2_P_BYTES = (A2_MAXT / 2) * A2_H * 128;      // 64 KB: two tiles' P per 128-byte head row
 constexpr int A2_M_BYTES = A2_MAXT * A2_H * 4;              // running softmax reference after each tile
 constexpr int A2_IDX_BYTES = A2_MAXT * A2_T * 4;            // the unit's row indices (pass 2 re-reads them)
+constexpr int A2_FIN_BYTES = A2_H * 4 * 2;                  // final sum and reference per head (epilogue)
 constexpr int A2_BAR_BYTES = 512;
-constexpr int A2_SMEM =
-    1024 + A2_QS_BYTES + A2_STAGES * A2_STAGE_BYTES + A2_P_BYTES + A2_M_BYTES + A2_IDX_BYTES + A2_BAR_BYTES;
-constexpr uint32_t TM_O0 = 0;    // O value dims [0, 256)
-constexpr uint32_t TM_S = 256;   // pass 1: two S buffers of 32 columns
-constexpr uint32_t TM_Q = 320;   // pass 1: Q dims [0, 384), two bf16 per column
+constexpr int A2_SMEM = 1024 + A2_STAGES * A2_STAGE_BYTES + A2_P_BYTES + A2_M_BYTES + A2_IDX_BYTES + A2_FIN_BYTES +
+                        A2_BAR_BYTES;
+constexpr uint32_t TM_S = 0;     // pass 1: four S buffers of 32 columns [0, 128)
+constexpr uint32_t TM_Q = 224;   // pass 1: Q dims [0, 576), two bf16 per column [224, 512)
+constexpr uint32_t TM_O0 = 0;    // pass 2: O value dims [0, 256)
 constexpr uint32_t TM_O1 = 256;  // pass 2: O value dims [256, 512)
 constexpr uint32_t IDESC_S = idesc_mma(128, A2_T, 1u, 0u);
 constexpr uint32_t IDESC_PV = idesc_mma(128, 256, 1u, 1u);
 constexpr float RESCALE_LOG2 = 8.f;
 constexpr uint64_t WAIT_NS = 2000000000ull;
-static_assert(TM_Q + A2_KB_TQ * 32 == 512, "TMEM columns");
+static_assert(TM_Q + A2_KB * 32 == 512 && TM_S + A2_STAGES * A2_T <= TM_Q, "TMEM columns");
 static_assert(A2_SMEM <= 232448, "shared memory");
-static_assert(A2_KB_TQ * A2_H * 128 <= A2_STAGE_BYTES + A2_P_BYTES, "Q staging fits stage 2 + the P area");
-static_assert(A2_H * A2_O_PITCH <= A2_QS_BYTES + A2_STAGES * A2_STAGE_BYTES, "epilogue staging fits");
+static_assert(A2_QSLOTS * A2_QKB_BYTES <= A2_P_BYTES, "Q staging slots fit the P area");
 
 struct A2Args {
   const uint16_t* q;   // absorbed queries [B, 128, 576] bf16
@@ -109,6 +109,20 @@ __device__ __forceinline__ void drain_mmas(uint64_t* bar) {
   (void)mbar_spin(bar, 0, WAIT_NS);
 }
 
+// O rows of this thread's TMEM lane scaled by alpha (both value halves), warp-collective.
+__device__ __forceinline__ void rescale_o(uint32_t trow, float alpha) {
+  #pragma unroll 1
+  for (int k = 0; k < 16; ++k) {
+    uint32_t o[32];
+    tmem_ld32(trow + 32 * k, o);
+    tmem_ld_wait();
+    #pragma unroll
+    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+    tmem_st32(trow + 32 * k, o);
+  }
+  tmem_st_wait();
+}
+
 __global__ void __launch_bounds__(A2_THREADS, 1)
     k_sparse_attn_2p(const __grid_constant__ CUtensorMap tm_q, A2Args a) {
   // every global access of this kernel comes after the previous kernel of the stream has completed
@@ -116,68 +130,81 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   pdl_launch_dependents();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* q_s = base;
-  unsigned char* st_s = q_s + A2_QS_BYTES;
-  unsigned char* p_s = st_s + A2_STAGES * A2_STAGE_BYTES;
+  unsigned char* st_s = base;
+  unsigned char* p_s = st_s + A2_STAGES * A2_STAGE_BYTES;  // P of every tile; Q staging slots before that
   float* m_s = reinterpret_cast<float*>(p_s + A2_P_BYTES);
   int* idx_s = reinterpret_cast<int*>(m_s + A2_MAXT * A2_H);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(idx_s + A2_MAXT * A2_T);
-  uint64_t* kv_full = bars;                // [3] the gather of a ring tile landed (512 cp.async arrivals)
-  uint64_t* kv_empty = kv_full + 3;        // [3] the P.V that read the ring tile completed
-  uint64_t* s_full = kv_empty + 3;         // [2] logits of a tile complete
-  uint64_t* s_empty = s_full + 2;          // [2] the softmax warps have read the S buffer
-  uint64_t* p_full = s_empty + 2;          // [8] P of tile j written (pass 1 rescale of O0 done)
-  uint64_t* pv_done = p_full + A2_MAXT;    // [8] pass-1 P.V of tile j complete
-  uint64_t* pv1_done = pv_done + A2_MAXT;  // [8] pass-2 P.V of tile j complete
-  uint64_t* resc_done = pv1_done + A2_MAXT;  // pass 2: the softmax warps rescaled O1 (one phase per event)
-  uint64_t* q_full = resc_done + 1;        // Q's shared-memory K-blocks landed (TMA)
-  uint64_t* qst_full = q_full + 1;         // Q's TMEM part landed in the staging area (TMA)
-  uint64_t* qt_full = qst_full + 1;        // Q's TMEM part written by the four softmax warps
-  uint64_t* drain = qt_full + 1;           // [3] per issuing thread, used only after a give-up
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 3);
+  float* fin_s = reinterpret_cast<float*>(idx_s + A2_MAXT * A2_T);  // [128] final sums, [128] final references
+  uint64_t* bars = reinterpret_cast<uint64_t*>(fin_s + 2 * A2_H);
+  uint64_t* kv_full = bars;                     // [4] a ring tile's gather landed (512 cp.async arrivals)
+  uint64_t* kv_empty = kv_full + A2_STAGES;     // [4] the MMAs that read the ring tile completed
+  uint64_t* s_full = kv_empty + A2_STAGES;      // [4] logits of a tile complete
+  uint64_t* s_empty = s_full + A2_STAGES;       // [4] the softmax warps have read the S buffer
+  uint64_t* p_full = s_empty + A2_STAGES;       // [8] P of tile j written
+  uint64_t* pv_done = p_full + A2_MAXT;         // [8] pass-2 P.V of tile j complete
+  uint64_t* resc_done = pv_done + A2_MAXT;      // pass 2: the softmax warps rescaled O (one phase per event)
+  uint64_t* q_slot = resc_done + 1;             // [4] a Q K-block landed in its staging slot (TMA)
+  uint64_t* qt_full = q_slot + A2_QSLOTS;       // all of Q written into TMEM by the four softmax warps
+  uint64_t* drain = qt_full + 1;                // [4] per issuing thread, used only after a give-up
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  int* resc_any = reinterpret_cast<int*>(tmem_holder + 2);  // [8] some head rescaled O at tile j (pass 1)
+  int* resc_any = reinterpret_cast<int*>(tmem_holder + 2);  // [8] some head's reference moved at tile j
+  int* have_s = resc_any + A2_MAXT;                         // the softmax warps completed both passes
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = static_cast<int>(blockIdx.x / static_cast<unsigned>(a.S));
   const int unit = static_cast<int>(blockIdx.x % static_cast<unsigned>(a.S));
+  // units split the row range by idx_ld (not by count), so the index loads need not wait for the count
+  const int T_ld = static_cast<int>((a.idx_ld + A2_T - 1) / A2_T);
+  const int t0 = static_cast<int>(static_cast<int64_t>(unit) * T_ld / a.S);
+  const int t1 = static_cast<int>(static_cast<int64_t>(unit + 1) * T_ld / a.S);
+  const int row0 = t0 * A2_T;
+  const int32_t* rowidx = a.idx + static_cast<int64_t>(b) * a.idx_ld + row0;
+  const int rows_ld = static_cast<int>(min(static_cast<int64_t>(t1 * A2_T), a.idx_ld)) - row0;  // readable entries
+  // gather warps: the raw indices of their rows of the first two tiles, loaded beside the count
+  const int my_row = (warp & 15) * 2 + (lane & 1);
+  int v_a = 0, v_b = 0;
+  if (warp < A2_GATHER_WARPS) {
+    if (my_row < rows_ld) v_a = rowidx[my_row];
+    if (A2_T + my_row < rows_ld) v_b = rowidx[A2_T + my_row];
+  }
   int n = a.count[b];
   n = n < 0 ? 0 : (static_cast<int64_t>(n) > a.idx_ld ? static_cast<int>(a.idx_ld) : n);
-  const int T = (n + A2_T - 1) / A2_T;
-  const int t0 = static_cast<int>(static_cast<int64_t>(unit) * T / a.S);
-  const int t1 = static_cast<int>(static_cast<int64_t>(unit + 1) * T / a.S);
-  int ntiles = t1 - t0;
+  const int nrows = max(0, min(n, t1 * A2_T) - row0);
+  int ntiles = (nrows + A2_T - 1) / A2_T;
   if (ntiles > A2_MAXT) {  // the host sizes S so that this never happens
     if (tid == 0) atomicExch(&g_attn2_check, 1);
     ntiles = 0;
   }
-  const int row0 = t0 * A2_T;
-  const int nrows = ntiles > 0 ? min(n, t1 * A2_T) - row0 : 0;
 
   if (tid == 0) {
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < A2_STAGES; ++i) {
       mbar_init(&kv_full[i], A2_GATHER_WARPS * 32);
       mbar_init(&kv_empty[i], 1);
-      mbar_init(&drain[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 4);
+      mbar_init(&drain[i], 1);
+      mbar_init(&q_slot[i], 1);
     }
     for (int i = 0; i < A2_MAXT; ++i) {
       mbar_init(&p_full[i], 4);
       mbar_init(&pv_done[i], 1);
-      mbar_init(&pv1_done[i], 1);
       resc_any[i] = 0;
     }
     mbar_init(resc_done, 4);
-    mbar_init(q_full, 1);
-    mbar_init(qst_full, 1);
     mbar_init(qt_full, 4);
     *abort_flag = 0;
+    *have_s = 0;
     fence_mbar_init();
+    if (ntiles > 0) {  // Q's first four K-blocks into the staging slots (the softmax warps fetch the rest)
+      tma_prefetch_desc(&tm_q);
+      for (int kb = 0; kb < A2_QSLOTS; ++kb) {
+        mbar_expect_tx(&q_slot[kb], A2_QKB_BYTES);
+        tma_load_2d(p_s + kb * A2_QKB_BYTES, &tm_q, &q_slot[kb], 64 * kb, b * A2_H);
+      }
+    }
   }
-  if (warp == A2_MMA_WARP) {
+  if (warp == A2_LOGIT_WARP0) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
@@ -185,220 +212,165 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);  // this warp's TMEM lane quarter
+  const int h = (warp & 3) * 32 + lane;                                          // = its head in the epilogue
 
   if (warp < A2_GATHER_WARPS) {
     // ------------------------------------------------------------------ gather
     // Ring tile i < ntiles: whole rows of pass-1 tile i (72 16-byte chunks per row); i >= ntiles: value dims
-    // [256, 512) of pass-2 tile i - ntiles (chunks 32..63).  Warp w copies rows 2w, 2w + 1 of each tile, chunk c
+    // [0, 512) of pass-2 tile i - ntiles (chunks 0..63).  Warp w copies rows 2w, 2w + 1 of each tile, chunk c
     // of row t at K-block c / 8, byte ((c & 7) ^ (t & 7)) * 16 of the row's 128-byte line (128-byte swizzle).
     if (ntiles > 0) {
-      if (tid == 0) {
-        tma_prefetch_desc(&tm_q);
-        mbar_expect_tx(q_full, A2_KB_SQ * A2_H * 128);
-        for (int kb = 0; kb < A2_KB_SQ; ++kb)
-          tma_load_2d(q_s + kb * A2_H * 128, &tm_q, q_full, 64 * (A2_KB_TQ + kb), b * A2_H);
-        // Q dims [0, 384) are staged in stage 2 and the P area until the softmax warps move them into TMEM
-        mbar_expect_tx(qst_full, A2_KB_TQ * A2_H * 128);
-        for (int kb = 0; kb < A2_KB_TQ; ++kb)
-          tma_load_2d(st_s + 2 * A2_STAGE_BYTES + kb * A2_H * 128, &tm_q, qst_full, 64 * kb, b * A2_H);
-      }
-      const int32_t* rowidx = a.idx + static_cast<int64_t>(b) * a.idx_ld + row0;
-      const int my_row = warp * 2 + (lane & 1);  // lanes 0 and 1 hold the indices of the warp's two rows
-      auto load_idx = [&](int i) -> int {
-        const int rr = i * A2_T + my_row;
-        return rr < nrows ? rowidx[rr] : 0;
-      };
-      int v_a = load_idx(0);
-      int v_b = ntiles > 1 ? load_idx(1) : 0;
       const int nring = 2 * ntiles;
       for (int i = 0; i < nring; ++i) {
         const int st = i % A2_STAGES;
         int v;
         if (i < ntiles) {
+          const int rr = i * A2_T + my_row;
           const int v_raw = v_a;
           v_a = v_b;
-          if (i + 2 < ntiles) v_b = load_idx(i + 2);
+          if (i + 2 < ntiles && (i + 2) * A2_T + my_row < rows_ld) v_b = rowidx[(i + 2) * A2_T + my_row];
           const bool in_range = v_raw >= 0 && v_raw < a.L;
-          if (lane < 2 && i * A2_T + my_row < nrows && !in_range) atomicExch(&g_attn2_check, 1);
-          v = in_range ? v_raw : (v_raw < 0 ? 0 : a.L - 1);
-          if (lane < 2) idx_s[i * A2_T + my_row] = v;  // read back by the same lane in pass 2
+          if (lane < 2 && rr < nrows && !in_range) atomicExch(&g_attn2_check, 1);
+          v = (rr < nrows && in_range) ? v_raw : (rr < nrows && v_raw >= a.L ? a.L - 1 : 0);
+          if (lane < 2) idx_s[rr] = v;  // read back by the same lane in pass 2
         } else {
           v = idx_s[(i - ntiles) * A2_T + my_row];
         }
-        // stage 2 holds the Q staging until the softmax warps have moved it into TMEM
-        bool ok = i != 2 || wait_ab(qt_full, 0, abort_flag);
-        ok = ok && wait_ab(&kv_empty[st], ((i / A2_STAGES) & 1) ^ 1, abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
+        if (!__all_sync(0xffffffffu, wait_ab(&kv_empty[st], ((i / A2_STAGES) & 1) ^ 1, abort_flag))) {
           if (lane == 0) give_up(abort_flag);
           break;
         }
         unsigned char* dst = st_s + st * A2_STAGE_BYTES;
-        if (i < ntiles) {
-          #pragma unroll
-          for (int k = 0; k < (2 * 72 + 31) / 32; ++k) {
-            const int q = lane + 32 * k;
-            const int rr = q >= 72 ? 1 : 0, c = q - rr * 72;
-            const int t = warp * 2 + rr;
-            const int srow = __shfl_sync(0xffffffffu, v, rr);
-            if (q < 2 * 72)
-              cp_async16(dst + (c >> 3) * A2_KB_BYTES + t * 128 + (((c & 7) ^ (t & 7)) << 4),
-                         a.kv + static_cast<int64_t>(srow) * 576 + c * 8);
-          }
-        } else {
-          #pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            const int c = 32 + lane;
-            const int t = warp * 2 + rr;
-            const int srow = __shfl_sync(0xffffffffu, v, rr);
+        const int nch = i < ntiles ? 72 : 64;  // chunks per row
+        #pragma unroll
+        for (int k = 0; k < (2 * 72 + 31) / 32; ++k) {
+          const int q = lane + 32 * k;
+          const int rr = q >= nch ? 1 : 0, c = q - rr * nch;
+          const int t = warp * 2 + rr;
+          const int srow = __shfl_sync(0xffffffffu, v, rr);
+          if (q < 2 * nch)
             cp_async16(dst + (c >> 3) * A2_KB_BYTES + t * 128 + (((c & 7) ^ (t & 7)) << 4),
                        a.kv + static_cast<int64_t>(srow) * 576 + c * 8);
-          }
         }
         cp_async_arrive_noinc(&kv_full[st]);
       }
       asm volatile("cp.async.wait_all;" ::: "memory");
-      if (tid == 0) {  // the Q loads have landed before the CTA can exit (they always complete)
-        (void)mbar_spin(q_full, 0, WAIT_NS);
-        (void)mbar_spin(qst_full, 0, WAIT_NS);
-      }
     }
-  } else if (warp == A2_MMA_WARP || warp == A2_MMA_WARP2) {
-    // ------------------------------------------------------------------ logits MMAs (pass 1)
-    // One thread issues about one tcgen05.mma per 30 ns, so the 36 logits MMAs of a tile are issued by two
-    // warps by tile parity, each into its own S buffer.
-    const int sb = warp == A2_MMA_WARP ? 0 : 1;
-    if (ntiles > sb && lane == 0) {
-      bool ok = wait_ab(q_full, 0, abort_flag) && wait_ab(qt_full, 0, abort_flag);
-      bool issued = false;
-      tc_fence_after();
-      const uint64_t qdesc = desc_sw128(smem_u32(q_s));
-      const uint32_t d = tmem + TM_S + sb * A2_T;
-      for (int j = sb; ok && j < ntiles; j += 2) {
-        const int st = j % A2_STAGES;
-        if (!wait_ab(&kv_full[st], (j / A2_STAGES) & 1, abort_flag) ||
-            !wait_ab(&s_empty[sb], ((j >> 1) & 1) ^ 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        fence_proxy_async_smem();  // the cp.async (generic proxy) writes are read by the tensor cores
-        tc_fence_after();
-        const uint64_t sdesc = desc_sw128(smem_u32(st_s + st * A2_STAGE_BYTES));
-        #pragma unroll
-        for (int kb = 0; kb < A2_KB_TQ; ++kb) {
-          #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16_ta(d, tmem + TM_Q + kb * 32 + kk * 8, sdesc + ((kb * A2_KB_BYTES + kk * 32) >> 4), IDESC_S,
-                       (kb | kk) != 0);
-        }
-        #pragma unroll
-        for (int kb = 0; kb < A2_KB_SQ; ++kb) {
-          #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16(d, qdesc + ((kb * A2_H * 128 + kk * 32) >> 4),
-                    sdesc + (((A2_KB_TQ + kb) * A2_KB_BYTES + kk * 32) >> 4), IDESC_S, 1u);
-        }
-        mma_commit(&s_full[sb]);
-        issued = true;
-      }
-      if (!ok) {
-        give_up(abort_flag);
-        if (issued) drain_mmas(&drain[sb]);
-      }
-    }
-  } else if (warp == A2_PV_WARP) {
-    // ------------------------------------------------------------------ O += P V (both passes)
-    if (ntiles > 0 && lane == 0) {
+  } else if (warp < A2_SOFTMAX_WARP0) {
+    // ------------------------------------------------------------------ logits MMAs (pass 1), P.V (pass 2)
+    // One thread issues about one tcgen05.mma per 30-50 ns, so tile j's 36 logits MMAs are issued by warp
+    // 16 + j % 4 into S buffer j % 4 from stage j % 4: four tiles' logits are in flight at once.
+    const int lw = warp - A2_LOGIT_WARP0;
+    if (lane == 0 && ntiles > 0) {
       bool ok = true, issued = false;
-      // pass 1: O0 += P_j V_j[:, 0:256)
-      for (int j = 0; ok && j < ntiles; ++j) {
-        if (!wait_ab(&p_full[j], 0, abort_flag)) {
-          ok = false;
-          break;
-        }
+      if (ntiles > lw) {
+        ok = wait_ab(qt_full, 0, abort_flag);
         tc_fence_after();
-        const int st = j % A2_STAGES;
-        const uint64_t pdesc = desc_sw128(smem_u32(p_s + (j >> 1) * A2_H * 128)) + (((j & 1) * 64) >> 4);
-        const uint32_t v_addr = smem_u32(st_s + st * A2_STAGE_BYTES);
-        #pragma unroll
-        for (int kk = 0; kk < A2_T / 16; ++kk)
-          mma_f16(tmem + TM_O0, pdesc + ((kk * 32) >> 4), desc_sw128_mn(v_addr + kk * 16 * 128, A2_KB_BYTES, 1024),
-                  IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&kv_empty[st]);
-        mma_commit(&pv_done[j]);
-        issued = true;
-      }
-      // pass 2: O1 += P_j V_j[:, 256:512), into the columns of S and Q (every logits MMA has completed and the
-      // last S was read: p_full of the last tile was observed above)
-      int events = 0;
-      for (int j = 0; ok && j < ntiles; ++j) {
-        const int i = ntiles + j, st = i % A2_STAGES;
-        if (!wait_ab(&kv_full[st], (i / A2_STAGES) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        if (j > 0 && resc_any[j]) {  // replay pass 1's rescale at this tile on O1
-          if (!wait_ab(resc_done, events & 1, abort_flag)) {
+        const uint32_t d = tmem + TM_S + lw * A2_T;
+        const uint64_t sdesc = desc_sw128(smem_u32(st_s + lw * A2_STAGE_BYTES));
+        for (int j = lw; ok && j < ntiles; j += A2_STAGES) {
+          const int use = j / A2_STAGES;
+          if (!wait_ab(&kv_full[lw], use & 1, abort_flag) || !wait_ab(&s_empty[lw], (use & 1) ^ 1, abort_flag)) {
             ok = false;
             break;
           }
-          ++events;
+          fence_proxy_async_smem();  // the cp.async (generic proxy) writes are read by the tensor cores
+          tc_fence_after();
+          #pragma unroll
+          for (int kb = 0; kb < A2_KB; ++kb) {
+            #pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ta(d, tmem + TM_Q + kb * 32 + kk * 8, sdesc + ((kb * A2_KB_BYTES + kk * 32) >> 4), IDESC_S,
+                         (kb | kk) != 0);
+          }
+          mma_commit(&kv_empty[lw]);  // the stage is free once the logits have read it
+          mma_commit(&s_full[lw]);
+          issued = true;
         }
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const uint64_t pdesc = desc_sw128(smem_u32(p_s + (j >> 1) * A2_H * 128)) + (((j & 1) * 64) >> 4);
-        const uint32_t v_addr = smem_u32(st_s + st * A2_STAGE_BYTES + 4 * A2_KB_BYTES);
-        #pragma unroll
-        for (int kk = 0; kk < A2_T / 16; ++kk)
-          mma_f16(tmem + TM_O1, pdesc + ((kk * 32) >> 4), desc_sw128_mn(v_addr + kk * 16 * 128, A2_KB_BYTES, 1024),
-                  IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&kv_empty[st]);
-        mma_commit(&pv1_done[j]);
+      }
+      if (ok && warp == A2_PV_WARP) {
+        // pass 2: O[:, 0:256) += P_j V_j[:, 0:256), O[:, 256:512) += P_j V_j[:, 256:512), into the columns of S
+        // and Q (every logits MMA has completed and the last S was read: p_full of the last tile)
+        int events = 0;
+        ok = wait_ab(&p_full[ntiles - 1], 0, abort_flag);
+        for (int j = 0; ok && j < ntiles; ++j) {
+          const int i = ntiles + j, st = i % A2_STAGES;
+          if (!wait_ab(&kv_full[st], (i / A2_STAGES) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (j > 0 && resc_any[j]) {  // replay pass 1's rescale at this tile on O
+            if (!wait_ab(resc_done, events & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            ++events;
+          }
+          fence_proxy_async_smem();
+          tc_fence_after();
+          const uint64_t pdesc = desc_sw128(smem_u32(p_s + (j >> 1) * A2_H * 128)) + (((j & 1) * 64) >> 4);
+          const uint32_t v_addr = smem_u32(st_s + st * A2_STAGE_BYTES);
+          #pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            #pragma unroll
+            for (int kk = 0; kk < A2_T / 16; ++kk)
+              mma_f16(tmem + (half ? TM_O1 : TM_O0), pdesc + ((kk * 32) >> 4),
+                      desc_sw128_mn(v_addr + half * 4 * A2_KB_BYTES + kk * 16 * 128, A2_KB_BYTES, 1024), IDESC_PV,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&kv_empty[st]);
+          mma_commit(&pv_done[j]);
+          issued = true;
+        }
       }
       if (!ok) {
         give_up(abort_flag);
-        if (issued) drain_mmas(&drain[2]);
+        if (issued) drain_mmas(&drain[lw]);
       }
     }
   } else {
-    // ------------------------------------------------------------------ Q into TMEM, softmax, epilogue
-    const int q4 = warp & 3;
-    const int h = q4 * 32 + lane;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    // ------------------------------------------------------------------ Q into TMEM, softmax (pass 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     if (ntiles > 0) {
-      // Q row h, dims [0, 384) -> TMEM lane h, columns TM_Q + 32 kb + j hold dims 64 kb + 2j, 64 kb + 2j + 1
-      // (read from the TMA staging: chunk c of row h at ((c ^ h) & 7) * 16).  Every wait here is decided
-      // warp-wide: the TMEM loads and stores are warp-collective.
-      ok = __all_sync(0xffffffffu, wait_ab(qst_full, 0, abort_flag));
-      if (ok) {
-        #pragma unroll 1
-        for (int kb = 0; kb < A2_KB_TQ; ++kb) {
-          const unsigned char* src = st_s + 2 * A2_STAGE_BYTES + kb * A2_H * 128 + h * 128;
-          uint32_t v[32];
-          #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 x = *reinterpret_cast<const uint4*>(src + ((c ^ (h & 7)) << 4));
-            v[4 * c] = x.x;
-            v[4 * c + 1] = x.y;
-            v[4 * c + 2] = x.z;
-            v[4 * c + 3] = x.w;
-          }
-          tmem_st32(trow + TM_Q + 32 * kb, v);
+      // Q row h, 64-dim block kb -> TMEM lane h, columns TM_Q + 32 kb + j hold dims 64 kb + 2j, 64 kb + 2j + 1,
+      // read from the TMA staging slot kb % 4 (chunk c of row h at ((c ^ h) & 7) * 16).  This loop always runs
+      // to the end (it has no break, so every Q load it waits for is issued and has landed before the CTA can
+      // exit, and the four warps meet at every named barrier); its waits are on TMA loads, which always complete,
+      // and are bounded all the same.  Every wait is decided warp-wide: the TMEM stores are warp-collective.
+      #pragma unroll 1
+      for (int kb = 0; kb < A2_KB; ++kb) {
+        const int slot = kb % A2_QSLOTS;
+        if (!__all_sync(0xffffffffu, mbar_spin(&q_slot[slot], (kb / A2_QSLOTS) & 1, WAIT_NS))) ok = false;
+        const unsigned char* src = p_s + slot * A2_QKB_BYTES + h * 128;
+        uint32_t v[32];
+        #pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 x = *reinterpret_cast<const uint4*>(src + ((c ^ (h & 7)) << 4));
+          v[4 * c] = x.x;
+          v[4 * c + 1] = x.y;
+          v[4 * c + 2] = x.z;
+          v[4 * c + 3] = x.w;
         }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(qt_full);
-        // the P area doubles as Q staging: all four warps have read it before any P is written
-        ok = __all_sync(0xffffffffu, wait_ab(qt_full, 0, abort_flag));
+        if (ok) tmem_st32(trow + TM_Q + 32 * kb, v);
+        named_bar_sync(1, 128);  // the four softmax warps have read the slot
+        if (warp == A2_SOFTMAX_WARP0 && lane == 0 && kb + A2_QSLOTS < A2_KB) {
+          mbar_expect_tx(&q_slot[slot], A2_QKB_BYTES);
+          tma_load_2d(p_s + slot * A2_QKB_BYTES, &tm_q, &q_slot[slot], 64 * (kb + A2_QSLOTS), b * A2_H);
+        }
       }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qt_full);
+      // the P area doubles as Q staging: all four warps are past it before any P is written
+      ok = ok && __all_sync(0xffffffffu, wait_ab(qt_full, 0, abort_flag));
     }
-    // ---- pass 1: softmax of each tile's logits, P kept per tile
     for (int i = 0; ok && i < ntiles; ++i) {
-      const int sb = i & 1;
+      const int sb = i % A2_STAGES;
       const int nvalid = min(A2_T, nrows - i * A2_T);
-      if (!__all_sync(0xffffffffu, wait_ab(&s_full[sb], (i >> 1) & 1, abort_flag))) {
+      if (!__all_sync(0xffffffffu, wait_ab(&s_full[sb], (i / A2_STAGES) & 1, abort_flag))) {
         ok = false;
         break;
       }
@@ -428,6 +400,7 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         resc = true;
       }
       m_s[i * A2_H + h] = m_used;
+      if (__any_sync(0xffffffffu, resc) && lane == 0) resc_any[i] = 1;
       uint32_t pk[A2_T / 2];
       float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       #pragma unroll
@@ -438,26 +411,6 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         pk[c / 2] = *reinterpret_cast<const uint32_t*>(&p2);
       }
       l = l * alpha + ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-      if (__any_sync(0xffffffffu, resc)) {
-        // the warp rescales its O0 rows (alpha = 1 for heads whose reference did not move) once the previous
-        // tile's P.V has completed; pass 2 replays it on O1
-        if (lane == 0) resc_any[i] = 1;
-        if (!__all_sync(0xffffffffu, wait_ab(&pv_done[i - 1], 0, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        #pragma unroll 1
-        for (int k = 0; k < 8; ++k) {
-          uint32_t o[32];
-          tmem_ld32(trow + TM_O0 + 32 * k, o);
-          tmem_ld_wait();
-          #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          tmem_st32(trow + TM_O0 + 32 * k, o);
-        }
-        tmem_st_wait();
-      }
       // P row h of tile i (32 bf16 = 64 B) -> K elements [32 (i & 1), +32) of head row h in P block i / 2
       unsigned char* prow = p_s + (i >> 1) * A2_H * 128 + h * 128;
       #pragma unroll
@@ -466,102 +419,86 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         *reinterpret_cast<uint4*>(prow + ((((i & 1) * 4 + c) ^ (h & 7)) << 4)) = v;
       }
       fence_proxy_async_smem();
-      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[i]);
     }
     if (!ok) give_up(abort_flag);
-    // ---- pass 2: the rescales of pass 1, replayed on O1 (every warp takes part; alpha = 1 where nothing moved)
+    // ---- pass 2: the rescales of pass 1, replayed on O (every warp takes part; alpha = 1 where nothing moved)
     named_bar_sync(1, 128);  // resc_any and m_s of every softmax warp are visible
     for (int j = 1; ok && j < ntiles; ++j) {
       if (!resc_any[j]) continue;
-      if (!__all_sync(0xffffffffu, wait_ab(&pv1_done[j - 1], 0, abort_flag))) {
+      if (!__all_sync(0xffffffffu, wait_ab(&pv_done[j - 1], 0, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float alpha = ex2_approx(m_s[(j - 1) * A2_H + h] - m_s[j * A2_H + h]);
-      #pragma unroll 1
-      for (int k = 0; k < 8; ++k) {
-        uint32_t o[32];
-        tmem_ld32(trow + TM_O1 + 32 * k, o);
-        tmem_ld_wait();
-        #pragma unroll
-        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-        tmem_st32(trow + TM_O1 + 32 * k, o);
-      }
-      tmem_st_wait();
+      rescale_o(trow, ex2_approx(m_s[(j - 1) * A2_H + h] - m_s[j * A2_H + h]));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(resc_done);
     }
     if (!ok) give_up(abort_flag);
-    // ---- epilogue: O row h of both value halves (rows staged in the Q / stage memory, free once the last
-    // pass-2 P.V completed; one bulk copy per row)
-    const bool have =
-        __all_sync(0xffffffffu, ok && ntiles > 0 && wait_ab(&pv1_done[ntiles > 0 ? ntiles - 1 : 0], 0, abort_flag));
-    tc_fence_after();
+    const bool have = __all_sync(0xffffffffu, ok && ntiles > 0 && wait_ab(&pv_done[ntiles > 0 ? ntiles - 1 : 0], 0, abort_flag));
+    fin_s[h] = l;
+    fin_s[A2_H + h] = m_used;
+    if (have && lane == 0) atomicAdd(have_s, 1);
     const int64_t orow = static_cast<int64_t>(b) * A2_H + h;
-    unsigned char* srow = q_s + h * A2_O_PITCH;
     if (a.S == 1) {
-      const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
-      #pragma unroll 1
-      for (int k = 0; k < 16; ++k) {  // 16 x 32 columns: O0 then O1
-        uint32_t o[32];
-        if (have) {
-          tmem_ld32(trow + (k < 8 ? TM_O0 + 32 * k : TM_O1 + 32 * (k - 8)), o);
-          tmem_ld_wait();
-        } else {
-          #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = 0u;
-        }
-        uint32_t pk[16];
-        #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv);
-          pk[c / 2] = *reinterpret_cast<const uint32_t*>(&v);
-        }
-        uint4* d4 = reinterpret_cast<uint4*>(srow + 64 * k);
-        #pragma unroll
-        for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
-      bulk_store_global(a.out + orow * 512, srow, 1024);
-      bulk_commit();
       if (a.lse) a.lse[orow] = (have && l > 0.f) ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
     } else {
       const int64_t prow_i = (static_cast<int64_t>(b) * a.S + unit) * A2_H + h;
-      #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        if (half == 1) bulk_wait_read0();  // this row's staging is free again
-        #pragma unroll 1
-        for (int k = 0; k < 8; ++k) {
-          uint32_t o[32];
-          if (have) {
-            tmem_ld32(trow + (half == 0 ? TM_O0 : TM_O1) + 32 * k, o);
-            tmem_ld_wait();
-          } else {
-            #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = 0u;
-          }
-          float4* d4 = reinterpret_cast<float4*>(srow + 128 * k);
-          #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            d4[c] = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]), __uint_as_float(o[4 * c + 2]),
-                                __uint_as_float(o[4 * c + 3]));
-        }
-        fence_proxy_async_smem();
-        bulk_store_global(a.ws_o + prow_i * 512 + 256 * half, srow, 1024);
-        bulk_commit();
-      }
       a.ws_ml[prow_i * 2 + 0] = have ? m_used : -INFINITY;
       a.ws_ml[prow_i * 2 + 1] = have ? l : 0.f;
     }
-    bulk_wait_read0();  // the staging rows are read before the CTA can exit
+  }
+  // ------------------------------------------------------------------ output (gather and softmax warps)
+  // Five warps per TMEM lane quarter (four gather warps, one softmax warp) write O's 16 column chunks of 32
+  // (value dims 32c .. 32c + 31) straight from TMEM: the output row normalised to bf16 (one unit per query),
+  // else the fp32 partial.
+  if (warp < A2_GATHER_WARPS || warp >= A2_SOFTMAX_WARP0) {
+    named_bar_sync(2, (A2_GATHER_WARPS + 4) * 32);  // fin_s, have_s
+    const bool have = *reinterpret_cast<volatile int*>(have_s) == 4;
+    const int rank = warp < A2_GATHER_WARPS ? warp / 4 : 4;  // this warp's place among its quarter's five
+    const float l = fin_s[h];
+    tc_fence_after();
+    const int64_t orow = static_cast<int64_t>(b) * A2_H + h;
+    #pragma unroll 1
+    for (int c = rank; c < 16; c += 5) {
+      uint32_t o[32];
+      if (have) {
+        tmem_ld32(trow + 32 * c, o);  // chunks 0-7: O0 columns, 8-15: O1 columns (TM_O1 = TM_O0 + 256)
+        tmem_ld_wait();
+      } else {
+        #pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] = 0u;
+      }
+      if (a.S == 1) {
+        const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
+        uint4* d4 = reinterpret_cast<uint4*>(a.out + orow * 512 + 32 * c);
+        #pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t pk[4];
+          #pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[8 * k + 2 * e]) * inv,
+                                                           __uint_as_float(o[8 * k + 2 * e + 1]) * inv);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&v);
+          }
+          d4[k] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      } else {
+        const int64_t prow_i = (static_cast<int64_t>(b) * a.S + unit) * A2_H + h;
+        float4* d4 = reinterpret_cast<float4*>(a.ws_o + prow_i * 512 + 32 * c);
+        #pragma unroll
+        for (int k = 0; k < 8; ++k)
+          d4[k] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]), __uint_as_float(o[4 * k + 2]),
+                              __uint_as_float(o[4 * k + 3]));
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == A2_MMA_WARP) {
+  if (warp == A2_LOGIT_WARP0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
