@@ -23,6 +23,8 @@
 // tiles j = warp - 16 (mod 4) (16 owns TMEM; 19 also issues pass 2's P.V MMAs), 20-23 move Q into TMEM and run
 // the softmax (one head per thread = one TMEM lane).  The output is written by the twenty gather and softmax
 // warps (five per TMEM lane quarter).
+#include <cuda_fp16.h>
+
 #include <algorithm>
 
 #include "lsa_common.cuh"
@@ -46,7 +48,7 @@ constexpr int A2_H = 128;         // heads (MMA M)
 constexpr int A2_KB = 9;          // 64-dim K-blocks of a 576-dim row
 constexpr int A2_MAXT = 8;        // tiles per work unit (P of every tile is kept)
 constexpr int A2_STAGES = 4;      // = the number of logits-issuing warps: tile j uses stage j % 4
-constexpr int A2_QSLOTS = 4;      // Q K-blocks staged at a time (in the P area) on their way into TMEM
+constexpr int A2_QSLOTS = 9;      // Q's 64-dim blocks, all staged at once (stages 1-3 and the P area)
 constexpr int A2_KB_BYTES = A2_T * 128;                     // 4 KB: one 64-dim block of a tile
 constexpr int A2_STAGE_BYTES = A2_KB * A2_KB_BYTES;         // 36 KB
 constexpr int A2_QKB_BYTES = A2_H * 128;                    // 16 KB: one 64-dim block of Q
@@ -67,7 +69,9 @@ constexpr float RESCALE_LOG2 = 8.f;
 constexpr uint64_t WAIT_NS = 2000000000ull;
 static_assert(TM_Q + A2_KB * 32 == 512 && TM_S + A2_STAGES * A2_T <= TM_Q, "TMEM columns");
 static_assert(A2_SMEM <= 232448, "shared memory");
-static_assert(A2_QSLOTS * A2_QKB_BYTES <= A2_P_BYTES, "Q staging slots fit the P area");
+static_assert(A2_STAGE_BYTES + A2_QSLOTS * A2_QKB_BYTES <= A2_STAGES * A2_STAGE_BYTES + A2_P_BYTES,
+              "Q staging fits stages 1-3 and the P area");
+static_assert(20 * 4096 <= A2_STAGES * A2_STAGE_BYTES, "epilogue staging: 4 KB per output warp in the stages");
 
 struct A2Args {
   const uint16_t* q;   // absorbed queries [B, 128, 576] bf16
@@ -80,8 +84,8 @@ struct A2Args {
   float scale_log2;
   uint16_t* out;
   float* lse;
-  float* ws_o;   // [B, S, 128, 512] fp32 (S > 1)
-  float* ws_ml;  // [B, S, 128, 2]   fp32 (S > 1): softmax reference (log2 units), sum
+  __half* ws_o;  // [B, S, 128, 512] fp16 (S > 1): unit u's O, unnormalised, times 2^-e (e per row)
+  float* ws_ml;  // [B, S, 128, 2]   fp32 (S > 1): softmax reference + e (log2 units), sum times 2^-e
 };
 
 // Bounded wait that also returns false once another role of the CTA has given up.
@@ -125,9 +129,9 @@ __device__ __forceinline__ void rescale_o(uint32_t trow, float alpha) {
 
 __global__ void __launch_bounds__(A2_THREADS, 1)
     k_sparse_attn_2p(const __grid_constant__ CUtensorMap tm_q, A2Args a) {
-  // every global access of this kernel comes after the previous kernel of the stream has completed
-  pdl_wait();
-  pdl_launch_dependents();
+  // Q, the barriers and TMEM are set up while the previous kernel of the stream may still run (programmatic
+  // dependent launch): Q is an input the pipeline's previous kernels do not write; every other global access
+  // (indices, counts, cache, outputs) comes after pdl_wait()
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* st_s = base;
@@ -143,9 +147,10 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   uint64_t* p_full = s_empty + A2_STAGES;       // [8] P of tile j written
   uint64_t* pv_done = p_full + A2_MAXT;         // [8] pass-2 P.V of tile j complete
   uint64_t* resc_done = pv_done + A2_MAXT;      // pass 2: the softmax warps rescaled O (one phase per event)
-  uint64_t* q_slot = resc_done + 1;             // [4] a Q K-block landed in its staging slot (TMA)
+  uint64_t* q_slot = resc_done + 1;             // [9] Q's 64-dim block kb landed in its staging slot (TMA)
   uint64_t* qt_full = q_slot + A2_QSLOTS;       // all of Q written into TMEM by the four softmax warps
   uint64_t* drain = qt_full + 1;                // [4] per issuing thread, used only after a give-up
+  unsigned char* q_st = st_s + A2_STAGE_BYTES;  // Q staging: block kb at q_st + kb * 16 KB
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* resc_any = reinterpret_cast<int*>(tmem_holder + 2);  // [8] some head's reference moved at tile j
@@ -154,6 +159,39 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = static_cast<int>(blockIdx.x / static_cast<unsigned>(a.S));
   const int unit = static_cast<int>(blockIdx.x % static_cast<unsigned>(a.S));
+  if (tid == 0) {
+    for (int i = 0; i < A2_STAGES; ++i) {
+      mbar_init(&kv_full[i], A2_GATHER_WARPS * 32);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
+      mbar_init(&drain[i], 1);
+    }
+    for (int i = 0; i < A2_QSLOTS; ++i) mbar_init(&q_slot[i], 1);
+    for (int i = 0; i < A2_MAXT; ++i) {
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+      resc_any[i] = 0;
+    }
+    mbar_init(resc_done, 4);
+    mbar_init(qt_full, 4);
+    *abort_flag = 0;
+    *have_s = 0;
+    fence_mbar_init();
+    // all of Q into the staging slots at once, before the count is known (an empty unit waits for these loads
+    // before it exits)
+    tma_prefetch_desc(&tm_q);
+    for (int kb = 0; kb < A2_QSLOTS; ++kb) {
+      mbar_expect_tx(&q_slot[kb], A2_QKB_BYTES);
+      tma_load_2d(q_st + kb * A2_QKB_BYTES, &tm_q, &q_slot[kb], 64 * kb, b * A2_H);
+    }
+  }
+  if (warp == A2_LOGIT_WARP0) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  pdl_wait();
+  pdl_launch_dependents();
   // units split the row range by idx_ld (not by count), so the index loads need not wait for the count
   const int T_ld = static_cast<int>((a.idx_ld + A2_T - 1) / A2_T);
   const int t0 = static_cast<int>(static_cast<int64_t>(unit) * T_ld / a.S);
@@ -175,38 +213,6 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   if (ntiles > A2_MAXT) {  // the host sizes S so that this never happens
     if (tid == 0) atomicExch(&g_attn2_check, 1);
     ntiles = 0;
-  }
-
-  if (tid == 0) {
-    for (int i = 0; i < A2_STAGES; ++i) {
-      mbar_init(&kv_full[i], A2_GATHER_WARPS * 32);
-      mbar_init(&kv_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
-      mbar_init(&drain[i], 1);
-      mbar_init(&q_slot[i], 1);
-    }
-    for (int i = 0; i < A2_MAXT; ++i) {
-      mbar_init(&p_full[i], 4);
-      mbar_init(&pv_done[i], 1);
-      resc_any[i] = 0;
-    }
-    mbar_init(resc_done, 4);
-    mbar_init(qt_full, 4);
-    *abort_flag = 0;
-    *have_s = 0;
-    fence_mbar_init();
-    if (ntiles > 0) {  // Q's first four K-blocks into the staging slots (the softmax warps fetch the rest)
-      tma_prefetch_desc(&tm_q);
-      for (int kb = 0; kb < A2_QSLOTS; ++kb) {
-        mbar_expect_tx(&q_slot[kb], A2_QKB_BYTES);
-        tma_load_2d(p_s + kb * A2_QKB_BYTES, &tm_q, &q_slot[kb], 64 * kb, b * A2_H);
-      }
-    }
-  }
-  if (warp == A2_LOGIT_WARP0) {
-    tmem_alloc(tmem_holder, 512);
-    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
@@ -237,7 +243,10 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         } else {
           v = idx_s[(i - ntiles) * A2_T + my_row];
         }
-        if (!__all_sync(0xffffffffu, wait_ab(&kv_empty[st], ((i / A2_STAGES) & 1) ^ 1, abort_flag))) {
+        // stages 1-3 hold the Q staging until the softmax warps have moved Q into TMEM
+        bool ok = (i == 0 || i >= A2_STAGES) || wait_ab(qt_full, 0, abort_flag);
+        ok = ok && wait_ab(&kv_empty[st], ((i / A2_STAGES) & 1) ^ 1, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) give_up(abort_flag);
           break;
         }
@@ -335,15 +344,14 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
     bool ok = true;
     if (ntiles > 0) {
       // Q row h, 64-dim block kb -> TMEM lane h, columns TM_Q + 32 kb + j hold dims 64 kb + 2j, 64 kb + 2j + 1,
-      // read from the TMA staging slot kb % 4 (chunk c of row h at ((c ^ h) & 7) * 16).  This loop always runs
-      // to the end (it has no break, so every Q load it waits for is issued and has landed before the CTA can
-      // exit, and the four warps meet at every named barrier); its waits are on TMA loads, which always complete,
-      // and are bounded all the same.  Every wait is decided warp-wide: the TMEM stores are warp-collective.
+      // read from its TMA staging slot (chunk c of row h at ((c ^ h) & 7) * 16).  This loop always runs to the end
+      // (no break: every Q load has landed before the CTA can exit); its waits are on TMA loads, which always
+      // complete, and are bounded all the same.  Every wait is decided warp-wide: the TMEM stores are
+      // warp-collective.
       #pragma unroll 1
       for (int kb = 0; kb < A2_KB; ++kb) {
-        const int slot = kb % A2_QSLOTS;
-        if (!__all_sync(0xffffffffu, mbar_spin(&q_slot[slot], (kb / A2_QSLOTS) & 1, WAIT_NS))) ok = false;
-        const unsigned char* src = p_s + slot * A2_QKB_BYTES + h * 128;
+        if (!__all_sync(0xffffffffu, mbar_spin(&q_slot[kb], 0, WAIT_NS))) ok = false;
+        const unsigned char* src = q_st + kb * A2_QKB_BYTES + h * 128;
         uint32_t v[32];
         #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -354,17 +362,12 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
           v[4 * c + 3] = x.w;
         }
         if (ok) tmem_st32(trow + TM_Q + 32 * kb, v);
-        named_bar_sync(1, 128);  // the four softmax warps have read the slot
-        if (warp == A2_SOFTMAX_WARP0 && lane == 0 && kb + A2_QSLOTS < A2_KB) {
-          mbar_expect_tx(&q_slot[slot], A2_QKB_BYTES);
-          tma_load_2d(p_s + slot * A2_QKB_BYTES, &tm_q, &q_slot[slot], 64 * (kb + A2_QSLOTS), b * A2_H);
-        }
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(qt_full);
-      // the P area doubles as Q staging: all four warps are past it before any P is written
+      // the P area and stages 1-3 double as Q staging: all four warps are past it before any P is written
       ok = ok && __all_sync(0xffffffffu, wait_ab(qt_full, 0, abort_flag));
     }
     for (int i = 0; ok && i < ntiles; ++i) {
@@ -442,58 +445,106 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
     fin_s[h] = l;
     fin_s[A2_H + h] = m_used;
     if (have && lane == 0) atomicAdd(have_s, 1);
-    const int64_t orow = static_cast<int64_t>(b) * A2_H + h;
-    if (a.S == 1) {
-      if (a.lse) a.lse[orow] = (have && l > 0.f) ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
-    } else {
-      const int64_t prow_i = (static_cast<int64_t>(b) * a.S + unit) * A2_H + h;
-      a.ws_ml[prow_i * 2 + 0] = have ? m_used : -INFINITY;
-      a.ws_ml[prow_i * 2 + 1] = have ? l : 0.f;
+    if (a.S == 1 && a.lse) {
+      a.lse[static_cast<int64_t>(b) * A2_H + h] = (have && l > 0.f) ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
   }
   // ------------------------------------------------------------------ output (gather and softmax warps)
-  // Five warps per TMEM lane quarter (four gather warps, one softmax warp) write O's 16 column chunks of 32
-  // (value dims 32c .. 32c + 31) straight from TMEM: the output row normalised to bf16 (one unit per query),
-  // else the fp32 partial.
+  // Five warps per TMEM lane quarter (four gather warps, one softmax warp) write O's eight 64-column chunks of
+  // each row: the output normalised to bf16 (one unit per query), else the unit's partial in fp16.  A partial row
+  // is scaled by a power of two 2^-e that brings its largest magnitude into [2^13, 2^14) (fp16 keeps 11
+  // significant bits over that whole range); e is folded into the row's softmax reference and sum, so the
+  // combine needs no other change.  A warp passes each chunk of its 32 rows through a private 4 KB staging tile
+  // (128-byte rows, 16-byte pieces swizzled by row) so that every store instruction writes four whole
+  // 128-byte lines.
   if (warp < A2_GATHER_WARPS || warp >= A2_SOFTMAX_WARP0) {
-    named_bar_sync(2, (A2_GATHER_WARPS + 4) * 32);  // fin_s, have_s
+    named_bar_sync(2, (A2_GATHER_WARPS + 4) * 32);  // fin_s, have_s; every gather copy has landed
+    if (ntiles == 0 && tid == 0) {
+      for (int kb = 0; kb < A2_QSLOTS; ++kb) (void)mbar_spin(&q_slot[kb], 0, WAIT_NS);  // Q loads of an empty unit
+    }
     const bool have = *reinterpret_cast<volatile int*>(have_s) == 4;
     const int rank = warp < A2_GATHER_WARPS ? warp / 4 : 4;  // this warp's place among its quarter's five
+    unsigned char* stg = st_s + (warp < A2_GATHER_WARPS ? warp : warp - 4) * 4096;
+    float* rmax_s = reinterpret_cast<float*>(p_s);  // [5][128]: each rank's largest |O| per row
     const float l = fin_s[h];
+    float mul = (have && l > 0.f) ? 1.f / l : 0.f;  // S == 1: normalise
+    int e = 0;
     tc_fence_after();
-    const int64_t orow = static_cast<int64_t>(b) * A2_H + h;
-    #pragma unroll 1
-    for (int c = rank; c < 16; c += 5) {
-      uint32_t o[32];
-      if (have) {
-        tmem_ld32(trow + 32 * c, o);  // chunks 0-7: O0 columns, 8-15: O1 columns (TM_O1 = TM_O0 + 256)
-        tmem_ld_wait();
-      } else {
+    if (a.S > 1) {
+      float mx = 0.f;
+      #pragma unroll 1
+      for (int c = rank; c < 8; c += 5) {
         #pragma unroll
-        for (int k = 0; k < 32; ++k) o[k] = 0u;
+        for (int part = 0; part < 2; ++part) {
+          uint32_t o[32];
+          if (have) {
+            tmem_ld32(trow + 64 * c + 32 * part, o);
+            tmem_ld_wait();
+            #pragma unroll
+            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, fabsf(__uint_as_float(o[k])));
+          }
+        }
       }
-      if (a.S == 1) {
-        const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
-        uint4* d4 = reinterpret_cast<uint4*>(a.out + orow * 512 + 32 * c);
+      rmax_s[rank * A2_H + h] = mx;
+      named_bar_sync(3, (A2_GATHER_WARPS + 4) * 32);
+      float rm = 0.f;
+      #pragma unroll
+      for (int k = 0; k < 5; ++k) rm = fmaxf(rm, rmax_s[k * A2_H + h]);
+      const int E = static_cast<int>((__float_as_uint(rm) >> 23) & 0xFFu) - 127;  // rm in [2^E, 2^(E+1))
+      e = min(max(E - 13, -64), 64);
+      mul = have ? __uint_as_float(static_cast<uint32_t>(127 - e) << 23) : 0.f;  // 2^-e, exact
+      if (rank == 4) {
+        const int64_t prow_i = (static_cast<int64_t>(b) * a.S + unit) * A2_H + h;
+        a.ws_ml[prow_i * 2 + 0] = have ? fin_s[A2_H + h] + static_cast<float>(e) : -INFINITY;
+        a.ws_ml[prow_i * 2 + 1] = have ? l * mul : 0.f;
+      }
+    }
+    #pragma unroll 1
+    for (int c = rank; c < 8; c += 5) {
+      // this row's 64 columns of chunk c as eight 16-byte pieces of 16-bit values (two loads of 32 columns)
+      #pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        uint32_t o[32];
+        if (have) {
+          tmem_ld32(trow + 64 * c + 32 * part, o);
+          tmem_ld_wait();
+        } else {
+          #pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
+        }
         #pragma unroll
         for (int k = 0; k < 4; ++k) {
           uint32_t pk[4];
           #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[8 * k + 2 * e]) * inv,
-                                                           __uint_as_float(o[8 * k + 2 * e + 1]) * inv);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&v);
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const float x0 = __uint_as_float(o[8 * k + 2 * q2]) * mul, x1 = __uint_as_float(o[8 * k + 2 * q2 + 1]) * mul;
+            if (a.S == 1) {
+              const __nv_bfloat162 bb = __floats2bfloat162_rn(x0, x1);
+              pk[q2] = *reinterpret_cast<const uint32_t*>(&bb);
+            } else {
+              const __half2 hh = __floats2half2_rn(x0, x1);
+              pk[q2] = *reinterpret_cast<const uint32_t*>(&hh);
+            }
           }
-          d4[k] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          const int piece = 4 * part + k;
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((piece ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-      } else {
-        const int64_t prow_i = (static_cast<int64_t>(b) * a.S + unit) * A2_H + h;
-        float4* d4 = reinterpret_cast<float4*>(a.ws_o + prow_i * 512 + 32 * c);
-        #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          d4[k] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]), __uint_as_float(o[4 * k + 2]),
-                              __uint_as_float(o[4 * k + 3]));
       }
+      __syncwarp();
+      // instruction i writes staging rows 4i .. 4i + 3: lane -> row 4i + lane / 8, 16-byte piece lane % 8
+      #pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = 4 * i + (lane >> 3), pc = lane & 7;
+        const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 128 + ((pc ^ (r & 7)) << 4));
+        const int hr = (warp & 3) * 32 + r;
+        if (a.S == 1) {
+          *reinterpret_cast<uint4*>(a.out + (static_cast<int64_t>(b) * A2_H + hr) * 512 + 64 * c + 8 * pc) = v;
+        } else {
+          const int64_t prow_r = (static_cast<int64_t>(b) * a.S + unit) * A2_H + hr;
+          *reinterpret_cast<uint4*>(a.ws_o + prow_r * 512 + 64 * c + 8 * pc) = v;
+        }
+      }
+      __syncwarp();  // the staging tile is read before the next chunk overwrites it
     }
   }
   tc_fence_before();
@@ -504,15 +555,80 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   }
 }
 
+// Merge of one (query, head)'s units: out = sum_u 2^(m_u - m*) O_u / sum_u 2^(m_u - m*) l_u (fp16 partials, their
+// scale already folded into m_u and l_u), lse = m* + log2(sum).  Each thread owns 4 columns.  One pass over the
+// units in batches of 8 whose loads (references, sums and values) are all issued before any is used; the running
+// reference m* moves batch by batch (online rescaling of the accumulators).
+constexpr int CB2_BATCH = 8;
+__global__ void __launch_bounds__(128) k_attn2_combine(const __half* __restrict__ ws_o, const float* __restrict__ ws_ml,
+                                                       int S, uint16_t* __restrict__ out, float* __restrict__ lse) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t bh = blockIdx.x;  // b * 128 + h
+  const int b = static_cast<int>(bh / A2_H), h = static_cast<int>(bh % A2_H);
+  const int64_t p0 = static_cast<int64_t>(b) * S * A2_H + h;  // row of unit u: p0 + u * 128
+  float mstar = -INFINITY, lsum = 0.f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int u0 = 0; u0 < S; u0 += CB2_BATCH) {
+    uint2 v[CB2_BATCH];
+    float2 ml[CB2_BATCH];
+    #pragma unroll
+    for (int k = 0; k < CB2_BATCH; ++k) {
+      if (u0 + k < S) {
+        ml[k] = reinterpret_cast<const float2*>(ws_ml)[p0 + (u0 + k) * A2_H];
+        v[k] = reinterpret_cast<const uint2*>(ws_o + (p0 + (u0 + k) * A2_H) * 512)[threadIdx.x];
+      }
+    }
+    float mb = -INFINITY;
+    #pragma unroll
+    for (int k = 0; k < CB2_BATCH; ++k)
+      if (u0 + k < S && ml[k].y > 0.f) mb = fmaxf(mb, ml[k].x);
+    if (mb == -INFINITY) continue;
+    if (mb > mstar) {
+      const float r = exp2f(mstar - mb);  // 0 while nothing has been accumulated
+      lsum *= r;
+      #pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j] *= r;
+      mstar = mb;
+    }
+    #pragma unroll
+    for (int k = 0; k < CB2_BATCH; ++k) {
+      if (u0 + k < S && ml[k].y > 0.f) {
+        const float wgt = exp2f(ml[k].x - mstar);
+        lsum += wgt * ml[k].y;
+        const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&v[k].x));
+        const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&v[k].y));
+        acc[0] += wgt * a0.x;
+        acc[1] += wgt * a0.y;
+        acc[2] += wgt * a1.x;
+        acc[3] += wgt * a1.y;
+      }
+    }
+  }
+  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+  uint2 pk;
+  pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+  pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+  reinterpret_cast<uint2*>(out + bh * 512)[threadIdx.x] = pk;
+  if (lse && threadIdx.x == 0) lse[bh] = lsum > 0.f ? (mstar + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
+}
+
 }  // namespace
 
 int make_map(CUtensorMap* m, const void* ptr, bool fp8, int64_t rows, int64_t cols, int box_cols, int box_rows);
-int launch_attn_combine(const float* ws_o, const float* ws_ml, int S, int64_t B, void* out, float* lse,
-                        cudaStream_t s);
 
 // Work units per query for the two-pass kernel, or 0 when the batch does not fit one wave of it (every unit at
 // most 8 tiles of 32 rows, at most 148 units).  Among the unit counts that keep the largest unit smallest, the
 // fewest (each unit writes a 256 KB partial that the combine reads back).
+// Workspace of the two-pass kernel with S units per query: fp16 partials [B, S, 128, 512] | (m, l) [B, S, 128, 2].
+size_t attn2_ml_offset(int64_t B, int S) { return align_up(static_cast<size_t>(B) * S * A2_H * 512 * 2, 256); }
+size_t attn2_ws_bytes(int64_t B, int S) {
+  if (S <= 1) return 0;
+  return attn2_ml_offset(B, S) + align_up(static_cast<size_t>(B) * S * A2_H * 2 * 4, 256);
+}
+
 int attn2_units(int64_t B, int64_t idx_ld) {
   if (B <= 0) return 0;
   const int64_t T = (idx_ld + A2_T - 1) / A2_T;
@@ -543,13 +659,15 @@ int launch_sparse_attn_2p(const void* q, const void* kv, int64_t L, const int32_
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
-  a.ws_o = S > 1 ? static_cast<float*>(ws) : nullptr;
-  a.ws_ml = S > 1 ? reinterpret_cast<float*>(static_cast<unsigned char*>(ws) +
-                                             align_up(static_cast<size_t>(B) * S * A2_H * 512 * 4, 256))
-                  : nullptr;
+  a.ws_o = S > 1 ? static_cast<__half*>(ws) : nullptr;
+  a.ws_ml = S > 1 ? reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + attn2_ml_offset(B, S)) : nullptr;
   LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_sparse_attn_2p), A2_SMEM));
   LSA_CUDA_TRY(launch_pdl(k_sparse_attn_2p, dim3(static_cast<unsigned>(B * S)), dim3(A2_THREADS), A2_SMEM, s, 0u, tq, a));
-  if (S > 1) return launch_attn_combine(a.ws_o, a.ws_ml, S, B, out, lse, s);
+  if (S > 1) {
+    LSA_CUDA_TRY(launch_pdl(k_attn2_combine, dim3(static_cast<unsigned>(B * A2_H)), dim3(128), 0, s, 0u,
+                            static_cast<const __half*>(a.ws_o), static_cast<const float*>(a.ws_ml), S,
+                            static_cast<uint16_t*>(out), lse));
+  }
   return LSA_OK;
 }
 

@@ -586,9 +586,13 @@ static int attn_slots(int64_t B, int64_t idx_ld) {
   return s2 > 0 ? s2 : splits_for(B);
 }
 
+size_t attn2_ws_bytes(int64_t B, int S);
+
 size_t sparse_attn_ws_bytes(int64_t B, int64_t idx_ld, int H) {
   if (H != AT_H) return 0;
-  const int S = attn_slots(B, idx_ld);
+  const int s2 = attn2_units(B, idx_ld);
+  if (s2 > 0) return attn2_ws_bytes(B, s2);
+  const int S = splits_for(B);
   if (S == 1) return 0;
   const size_t o = align_up(static_cast<size_t>(B) * S * AT_H * 512 * 4, 256);
   return o + align_up(static_cast<size_t>(B) * S * AT_H * 2 * 4, 256);
@@ -596,12 +600,6 @@ size_t sparse_attn_ws_bytes(int64_t B, int64_t idx_ld, int H) {
 
 int attn_launches_per_call(int64_t B, int64_t idx_ld, int H) { return (H == AT_H && attn_slots(B, idx_ld) > 1) ? 2 : 1; }
 
-int launch_attn_combine(const float* ws_o, const float* ws_ml, int S, int64_t B, void* out, float* lse,
-                        cudaStream_t s) {
-  LSA_CUDA_TRY(launch_pdl(k_attn_combine, dim3(static_cast<unsigned>(B * AT_H)), dim3(128), 0, s, 0u, ws_o, ws_ml, S,
-                          static_cast<uint16_t*>(out), lse));
-  return LSA_OK;
-}
 
 int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
                        const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, void* ws,
