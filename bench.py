@@ -634,9 +634,9 @@ def long_context_configs(device, l2_flush, iters: int = 10):
             t_idx, t_cnt = torch.empty_like(bstep.idx), torch.empty_like(bstep.cnt)
             ws_t = lsa_.workspace(lsa_.lsa_tree_workspace_size(B, NP, F, M2, wl.M), device)
 
-            def tree():
-                lsa_.lsa_tree_select(bstep.q_I, bstep.w, bstep.cen, par, F, bstep.members, M2, wl.M, wl.sink,
-                                     wl.window, wl.L, bstep.q_pos, t_idx, t_cnt, ws_t)
+            def tree():  # children from the cached split of the centres, on the tensor cores
+                lsa_.lsa_tree_select_split(bstep.q_I, bstep.w, bstep.split, par, F, bstep.members, M2, wl.M, wl.sink,
+                                           wl.window, wl.L, bstep.q_pos, t_idx, t_cnt, ws_t)
 
             st_t = _time_stages([tree], l2_flush, iters)
             bstep.select()
@@ -649,7 +649,8 @@ def long_context_configs(device, l2_flush, iters: int = 10):
             t_flops = 2.0 * B * wl.H_I * wl.d_I * (NP + M2 * F)
             res["flat10m_tree"] = {
                 "workload": "flat10m's buckets as a two-level tree: 2442 parents of 64 consecutive buckets (mean "
-                            "centres), top-64 parents, top-32 of their 4096 children, + sink 4 + window 512",
+                            "centres), top-64 parents, top-32 of their 4096 children (scored on the tensor cores "
+                            "from the centres' cached bf16 split), + sink 4 + window 512",
                 "stages": {"tree_select": _stage(st_t[0], t_bytes)}, "tree_select_flops": t_flops,
                 "flat_select_ms": round(float(st[0]), 5),
                 "share_of_flat_positions_kept": round(float(np.mean(kept)), 4)}

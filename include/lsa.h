@@ -7,7 +7,8 @@
  *                                      lsa_topk_refine   (FP8 scan's top-2K re-ranked exactly in bf16)
  *                                      lsa_bucket_select, lsa_bucket_select_split, lsa_bucket_select_noalloc
  *                                                        (Flat buckets / 4-token micro-blocks)
- *                                      lsa_tree_select   (two-level tree search over the Flat buckets)
+ *                                      lsa_tree_select, lsa_tree_select_split
+ *                                                        (two-level tree search over the Flat buckets)
  *                                      lsa_hi_select     (pages, then tokens: hierarchical index)
  *                                      lsa_msa_select    (group-wise 128-token blocks)
  *      precompute, cached once:        lsa_pool_keys, lsa_split_representatives, lsa_tree_parents
@@ -214,7 +215,21 @@ int lsa_tree_select(const void* q_idx, const float* w, int64_t B, int H_I, int d
                     int M, int sink, int window, int64_t L, const int64_t* q_pos, int32_t* idx, int64_t idx_ld,
                     int32_t* count, void* ws, size_t ws_bytes, void* stream);
 
-/* lsa_tree_workspace_size -- scratch bytes of lsa_tree_select; (size_t)-1 for invalid sizes. */
+/*
+ * lsa_tree_select_split -- lsa_tree_select with the children scored on the tensor cores.
+ *   Same search, arguments and result as lsa_tree_select, except that the bucket centres are given as their
+ *   exact three-part bf16 split (lsa_split_representatives of the fp32 centroids, split [3, NB, 128] bf16,
+ *   cached beside them) instead of the fp32 centres.  A kept parent's children are F consecutive centre rows,
+ *   so two kept parents form one 128-row tile against the query's 64 heads; each product is exact and the sums
+ *   are fp32, as in lsa_tree_select (results equal up to the order of the fp32 sums).
+ *   Requires F = 64, H_I = 64, d_I = 128 (LSA_ERR_UNSUPPORTED otherwise).  ws: lsa_tree_workspace_size.
+ */
+int lsa_tree_select_split(const void* q_idx, const float* w, int64_t B, int H_I, int d_I, const void* split,
+                          int64_t NB, const float* parents, int64_t NP, int F, const int32_t* members, int bsz,
+                          int M2, int M, int sink, int window, int64_t L, const int64_t* q_pos, int32_t* idx,
+                          int64_t idx_ld, int32_t* count, void* ws, size_t ws_bytes, void* stream);
+
+/* lsa_tree_workspace_size -- scratch bytes of lsa_tree_select(_split); (size_t)-1 for invalid sizes. */
 size_t lsa_tree_workspace_size(int64_t B, int64_t NP, int F, int M2, int M);
 
 /*
@@ -363,8 +378,15 @@ int lsa_bucket_select_noalloc(const void* q_idx, const float* q_scale, const flo
  *     z_s      = scale * q[b,h,:] . kv[s, 0:d_qk]
  *     out[b,h] = sum_s softmax(z)_s * kv[s, 0:d_v]          (bf16, fp32 accumulation)
  *     lse[b,h] = log sum_s exp(z_s)                          (natural log; -inf if S empty)
- *   An empty set gives out = 0.  Entries of idx must lie in [0, L); the call does not read
+ *   An empty set gives out = 0.  Entries of idx must lie in [0, L) (an entry outside is clamped, so the
+ *   access stays in bounds, and lsa_device_status reports LSA_ERR_DEVICE_CHECK); the call does not read
  *   idx past count[b].
+ *   Kernels: decode-sized batches (every query's rows in units of at most 256, at most 148 units) run one
+ *   unit per SM in two passes (logits and softmax, then P.V) and a merge of the units; larger batches run
+ *   the value-half kernel.  H < 128 runs the same kernels on zero-padded 128-head queries.  Programmatic
+ *   dependent launch: the decode kernel may start loading q while the kernel before it on `stream` is
+ *   still running, when that kernel signalled its dependents early (the library's own kernels do, and none
+ *   of them writes a query); every other input is read after that kernel has completed.
  *   q   [B, H, d_qk] bf16;  kv [L, d_qk] bf16 (row stride d_qk);  out [B, H, d_v] bf16;
  *   lse [B, H] fp32 or NULL.  Supported: d_qk = 576, d_v = 512, H in {16, 32, 64, 128},
  *   idx_ld >= max count, max count <= 65536.  q, kv, out 16-byte aligned.

@@ -48,6 +48,8 @@ SIGNATURES = {
     "lsa_tree_workspace_size": (_SZ, [_I64, _I64, _I32, _I32, _I32]),
     "lsa_tree_select": (_I32, [_P, _P, _I64, _I32, _I32, _P, _I64, _P, _I64, _I32, _P, _I32, _I32, _I32, _I32, _I32,
                                _I64, _P, _P, _I64, _P, _P, _SZ, _P]),
+    "lsa_tree_select_split": (_I32, [_P, _P, _I64, _I32, _I32, _P, _I64, _P, _I64, _I32, _P, _I32, _I32, _I32, _I32,
+                                     _I32, _I64, _P, _P, _I64, _P, _P, _SZ, _P]),
     "lsa_msa_select": (_I32, [_P, _P, _P, _I64, _I32, _I32, _I64, _I32, _I32, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "lsa_msa_workspace_size": (_SZ, [_I64, _I64, _I32, _I32]),
     "lsa_msa_attn_workspace_size": (_SZ, [_I64, _I64, _I32]),
@@ -208,6 +210,18 @@ def lsa_tree_select(q_idx, w, centroids, parents, F, members, M2, M, sink, windo
                                         _ptr(q_pos), _ptr(idx), idx.stride(0), _ptr(count), _ptr(ws),
                                         0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check("lsa_tree_select", st)
+
+
+def lsa_tree_select_split(q_idx, w, split, parents, F, members, M2, M, sink, window, L, q_pos, idx, count, ws,
+                          stream=None):
+    """lsa_tree_select with the children scored on the tensor cores from the centres' cached bf16 split."""
+    B, H_I, d_I = q_idx.shape
+    NB, bsz = members.shape
+    st = load_library().lsa_tree_select_split(_ptr(q_idx), _ptr(w), B, H_I, d_I, _ptr(split), NB, _ptr(parents),
+                                              parents.shape[0], F, _ptr(members), bsz, M2, M, sink, window, L,
+                                              _ptr(q_pos), _ptr(idx), idx.stride(0), _ptr(count), _ptr(ws),
+                                              0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("lsa_tree_select_split", st)
 
 
 def lsa_hi_workspace_size(B, L, P, Bsub, M, K, sink, window):

@@ -561,6 +561,33 @@ __global__ void __launch_bounds__(256) k_hfa_split(const int32_t* __restrict__ i
   }
 }
 
+// Head padding for the tensor-core kernels (128 heads = the MMA's M): qp[b, h] = q[b, h] for h < H, else 0 (576-dim
+// bf16 rows as 72 16-byte units); out[b, h] = outp[b, h] and lse[b, h] = lsep[b, h] for h < H.
+__global__ void k_pad_heads(const uint4* __restrict__ q, int H, int64_t B, uint4* __restrict__ qp) {
+  const int64_t total = B * AT_H * 72;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / 72;
+    const int c = static_cast<int>(i % 72);
+    const int64_t b = r / AT_H;
+    const int h = static_cast<int>(r % AT_H);
+    qp[i] = h < H ? q[(b * H + h) * 72 + c] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+__global__ void k_unpad_heads(const uint4* __restrict__ outp, const float* __restrict__ lsep, int H, int64_t B,
+                              uint4* __restrict__ out, float* __restrict__ lse) {
+  const int64_t total = B * H * 64;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / 64;
+    const int c = static_cast<int>(i % 64);
+    const int64_t b = r / H;
+    const int h = static_cast<int>(r % H);
+    out[i] = outp[(b * AT_H + h) * 64 + c];
+    if (lse != nullptr && c == 0) lse[r] = lsep[b * AT_H + h];
+  }
+}
+
 int splits_for(int64_t B) {
   int64_t s = 148 / (2 * (B > 0 ? B : 1));
   if (s < 1) s = 1;
@@ -571,6 +598,7 @@ int splits_for(int64_t B) {
 }  // namespace
 
 int make_map(CUtensorMap* m, const void* ptr, bool fp8, int64_t rows, int64_t cols, int box_cols, int box_rows);
+int sm_count();
 int launch_attn_simt(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
                      const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, cudaStream_t s);
 
@@ -588,7 +616,16 @@ static int attn_slots(int64_t B, int64_t idx_ld) {
 
 size_t attn2_ws_bytes(int64_t B, int S);
 
+// Head counts below 128 run on the 128-head tensor-core kernels with zero-padded queries: padded queries
+// [B, 128, 576] bf16 | padded outputs [B, 128, 512] bf16 | padded lse [B, 128] | the 128-head call's scratch.
+static bool padded_heads(int H) { return H == 16 || H == 32 || H == 64; }
+static size_t pad_bytes(int64_t B) {
+  return align_up(static_cast<size_t>(B) * AT_H * 576 * 2, 256) + align_up(static_cast<size_t>(B) * AT_H * 512 * 2, 256) +
+         align_up(static_cast<size_t>(B) * AT_H * 4, 256);
+}
+
 size_t sparse_attn_ws_bytes(int64_t B, int64_t idx_ld, int H) {
+  if (padded_heads(H)) return pad_bytes(B) + sparse_attn_ws_bytes(B, idx_ld, AT_H);
   if (H != AT_H) return 0;
   const int s2 = attn2_units(B, idx_ld);
   if (s2 > 0) return attn2_ws_bytes(B, s2);
@@ -598,13 +635,35 @@ size_t sparse_attn_ws_bytes(int64_t B, int64_t idx_ld, int H) {
   return o + align_up(static_cast<size_t>(B) * S * AT_H * 2 * 4, 256);
 }
 
-int attn_launches_per_call(int64_t B, int64_t idx_ld, int H) { return (H == AT_H && attn_slots(B, idx_ld) > 1) ? 2 : 1; }
+int attn_launches_per_call(int64_t B, int64_t idx_ld, int H) {
+  if (padded_heads(H)) return 2 + attn_launches_per_call(B, idx_ld, AT_H);
+  return (H == AT_H && attn_slots(B, idx_ld) > 1) ? 2 : 1;
+}
 
 
 int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
                        const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, void* ws,
                        size_t ws_bytes, cudaStream_t s) {
   if (B == 0) return LSA_OK;
+  if (padded_heads(H) && L < (int64_t(1) << 31)) {
+    // the query's heads in the first H rows of zero-padded 128-head queries, the 128-head kernels, then the
+    // real rows back
+    const size_t need = sparse_attn_ws_bytes(B, idx_ld, H);
+    if (ws == nullptr || !aligned256(ws) || ws_bytes < need) return LSA_ERR_WORKSPACE;
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    void* qp = base;
+    void* outp = base + align_up(static_cast<size_t>(B) * AT_H * 576 * 2, 256);
+    float* lsep = reinterpret_cast<float*>(static_cast<unsigned char*>(outp) +
+                                           align_up(static_cast<size_t>(B) * AT_H * 512 * 2, 256));
+    const int grid = sm_count() * 4;
+    k_pad_heads<<<grid, 256, 0, s>>>(static_cast<const uint4*>(q), H, B, static_cast<uint4*>(qp));
+    LSA_CUDA_TRY(cudaGetLastError());
+    const int st = launch_sparse_attn(qp, kv, L, idx, idx_ld, count, B, AT_H, scale, outp, lsep, base + pad_bytes(B),
+                                      ws_bytes - pad_bytes(B), s);
+    if (st != LSA_OK) return st;
+    k_unpad_heads<<<grid, 256, 0, s>>>(static_cast<const uint4*>(outp), lsep, H, B, static_cast<uint4*>(out), lse);
+    return cuda_status(cudaGetLastError());
+  }
   if (H != AT_H || L >= (int64_t(1) << 31)) return launch_attn_simt(q, kv, L, idx, idx_ld, count, B, H, scale, out, lse, s);
   const int S2 = attn2_units(B, idx_ld);
   const int S = S2 > 0 ? S2 : splits_for(B);

@@ -7,12 +7,14 @@
 // candidates are scattered over the bucket table, so there is no dense tile to put on the tensor cores), the
 // rest of the search is the cluster top-K and the Flat expansion.
 #include "lsa_common.cuh"
+#include "sm100.cuh"
 
 #include <algorithm>
 
 namespace lsa {
 
 int sm_count();
+int make_map(CUtensorMap* m, const void* ptr, bool fp8, int64_t rows, int64_t cols, int box_cols, int box_rows);
 
 namespace {
 
@@ -119,7 +121,173 @@ __global__ void k_tree_map(const int32_t* __restrict__ kpos, int64_t kpos_ld, co
   if (lane == 0) kcount[b] = static_cast<int32_t>(min(static_cast<int64_t>(base), kept_ld));
 }
 
+// ---------------------------------------------------------------------------------------------------------------
+// The kept parents' children on the tensor cores (F = 64, H_I = 64, d_I = 128).  A kept parent's 64 children are 64
+// consecutive rows of the bucket centres, so two kept parents of one query make an M = 128 tile of centre rows,
+// loaded by TMA boxes from the centres' exact three-part bf16 split (hi | mid | lo, NB rows apart); the query's 64
+// heads are N and d_I = 128 is K.  The three parts accumulate into one fp32 accumulator (every product is exact:
+// the query is bf16 and each part holds 8 significand bits of the fp32 centre), so the scores equal the CUDA-core
+// scorer's up to the order of the fp32 sums.  Epilogue: one child per thread (TMEM lane), sum_j w_j ReLU(acc_j).
+constexpr int TC_F = 64;        // children per parent (rows per TMA box)
+constexpr int TC_KB_BYTES = TC_F * 128;                 // 8 KB: one 64-dim block of one parent's children
+constexpr int TC_A_BYTES = 3 * 2 * 2 * TC_KB_BYTES;     // 96 KB: [part][64-dim block][parent of the pair]
+constexpr int TC_Q_BYTES = 2 * TC_KB_BYTES;             // 16 KB: the query's 64 heads
+constexpr int TC_SMEM = 1024 + TC_A_BYTES + TC_Q_BYTES + 512;
+constexpr uint32_t TC_IDESC = sm100::idesc_mma(128, 64, 1u, 0u);
+__device__ int g_tree_tc_timeout;
+
+struct TreeTcArgs {
+  const float* w;
+  int64_t NB;
+  const int32_t* kp;
+  int64_t kp_ld;
+  const int32_t* kpc;
+  int64_t n_cand;
+  float* cscore;
+  int32_t* cid;
+  int64_t ldc;
+};
+
+__global__ void __launch_bounds__(128, 1)
+    k_tree_child_tc(const __grid_constant__ CUtensorMap tm_split, const __grid_constant__ CUtensorMap tm_q,
+                    TreeTcArgs a) {
+  using namespace sm100;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* a_s = base;
+  unsigned char* q_s = a_s + TC_A_BYTES;
+  float* w_s = reinterpret_cast<float*>(q_s + TC_Q_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(w_s + 64);  // [0] loads landed, [1] MMAs complete
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int b = blockIdx.y;
+  const int64_t slot0 = 2 * static_cast<int64_t>(blockIdx.x);
+  const int64_t nkp = min(static_cast<int64_t>(max(a.kpc[b], 0)), a.kp_ld);
+  int par[2];
+  #pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int64_t sl = slot0 + i;
+    par[i] = (sl < nkp) ? a.kp[static_cast<int64_t>(b) * a.kp_ld + sl] : -1;
+    if (par[i] >= 0 && static_cast<int64_t>(par[i]) * TC_F >= a.NB) par[i] = -1;
+  }
+  if (tid < 64) w_s[tid] = a.w[static_cast<int64_t>(b) * 64 + tid];
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+    if (par[0] >= 0 || par[1] >= 0) {
+      const uint32_t bytes = TC_Q_BYTES + (par[0] >= 0 ? 6 : 0) * TC_KB_BYTES + (par[1] >= 0 ? 6 : 0) * TC_KB_BYTES;
+      mbar_expect_tx(&bars[0], bytes);
+      for (int kb = 0; kb < 2; ++kb) tma_load_2d(q_s + kb * TC_KB_BYTES, &tm_q, &bars[0], 64 * kb, b * 64);
+      for (int part = 0; part < 3; ++part)
+        for (int kb = 0; kb < 2; ++kb)
+          for (int i = 0; i < 2; ++i)
+            if (par[i] >= 0)
+              tma_load_2d(a_s + ((part * 2 + kb) * 2 + i) * TC_KB_BYTES, &tm_split, &bars[0], 64 * kb,
+                          static_cast<int>(part * a.NB + static_cast<int64_t>(par[i]) * TC_F));
+    }
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const bool any = par[0] >= 0 || par[1] >= 0;
+  bool ok = true;
+  if (any && tid == 0) {
+    ok = mbar_wait(&bars[0], 0);
+    if (ok) {
+      tc_fence_after();
+      const uint64_t ad = desc_sw128(smem_u32(a_s)), qd = desc_sw128(smem_u32(q_s));
+      #pragma unroll
+      for (int part = 0; part < 3; ++part) {
+        #pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem, ad + ((((part * 2 + kb) * 2) * TC_KB_BYTES + kk * 32) >> 4),
+                    qd + ((kb * TC_KB_BYTES + kk * 32) >> 4), TC_IDESC, (part | kb | kk) != 0);
+        }
+      }
+      mma_commit(&bars[1]);
+    } else {
+      atomicExch(&g_tree_tc_timeout, 1);
+      mbar_arrive(&bars[1]);  // nothing was issued: release the epilogue's wait
+    }
+  }
+  // epilogue: thread t = TMEM lane t = child (t & 63) of the kept parent in slot slot0 + (t >> 6)
+  const bool done = any && __all_sync(0xffffffffu, mbar_wait(&bars[1], 0));
+  tc_fence_after();
+  float score = -INFINITY;
+  if (done) {
+    uint32_t r0[32], r1[32];
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    tmem_ld32(taddr, r0);
+    tmem_ld32(taddr + 32, r1);
+    tmem_ld_wait();
+    float acc0 = 0.f, acc1 = 0.f;
+    #pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      acc0 = fmaf(w_s[c], fmaxf(__uint_as_float(r0[c]), 0.f), acc0);
+      acc1 = fmaf(w_s[32 + c], fmaxf(__uint_as_float(r1[c]), 0.f), acc1);
+    }
+    score = acc0 + acc1;
+  }
+  const int i = tid >> 6, r = tid & 63;
+  const int64_t c = (slot0 + i) * TC_F + r;
+  const int64_t child = par[i] >= 0 ? static_cast<int64_t>(par[i]) * TC_F + r : -1;
+  const bool valid = done && ok && child >= 0 && child < a.NB;
+  if (c < a.n_cand) {
+    a.cscore[static_cast<int64_t>(b) * a.ldc + c] = valid ? score : -INFINITY;
+    a.cid[static_cast<int64_t>(b) * a.ldc + c] = valid ? static_cast<int32_t>(child) : -1;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
 }  // namespace
+
+int launch_tree_child_score_tc(const void* q, const float* w, int64_t B, const void* split, int64_t NB,
+                               const int32_t* kp, int64_t kp_ld, const int32_t* kpc, int64_t n_cand, float* cscore,
+                               int32_t* cid, int64_t ldc, cudaStream_t s) {
+  if (B == 0 || n_cand == 0) return LSA_OK;
+  CUtensorMap tsplit, tq;
+  int st = make_map(&tsplit, split, false, 3 * NB, 128, 64, TC_F);
+  if (st) return st;
+  st = make_map(&tq, q, false, B * 64, 128, 64, 64);
+  if (st) return st;
+  TreeTcArgs a;
+  a.w = w;
+  a.NB = NB;
+  a.kp = kp;
+  a.kp_ld = kp_ld;
+  a.kpc = kpc;
+  a.n_cand = n_cand;
+  a.cscore = cscore;
+  a.cid = cid;
+  a.ldc = ldc;
+  LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_tree_child_tc), TC_SMEM));
+  const dim3 grid(static_cast<unsigned>(cdiv(cdiv(n_cand, TC_F), 2)), static_cast<unsigned>(B));
+  k_tree_child_tc<<<grid, 128, TC_SMEM, s>>>(tsplit, tq, a);
+  return cuda_status(cudaGetLastError());
+}
+
+int take_tree_tc_timeout() {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_tree_tc_timeout, sizeof(int)) != cudaSuccess) return -1;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_tree_tc_timeout, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
+}
 
 int launch_tree_parents(const float* reps, int64_t NB, int d_I, int F, float* parents, cudaStream_t s) {
   const int64_t NP = cdiv(NB, F);

@@ -183,12 +183,13 @@ int lsa_device_status(void* stream) {
   int a2_check = 0, at_check = 0;
   const int ix = take_index_timeout(), at = take_attn_timeout(&at_check), rs = take_rescore_timeout();
   const int a2 = take_attn2_flags(&a2_check), stw = take_selftest_timeout(), sm_check = take_attn_simt_check();
-  if (ix < 0 || at < 0 || rs < 0 || a2 < 0 || stw < 0 || sm_check < 0) return cuda_status(cudaGetLastError());
-  if (ix || at || rs || a2 || stw) {
-    char msg[192];
-    std::snprintf(msg, sizeof(msg), "bounded wait gave up in:%s%s%s%s%s", ix ? " k_index_score_tc" : "",
+  const int tt = take_tree_tc_timeout();
+  if (ix < 0 || at < 0 || rs < 0 || a2 < 0 || stw < 0 || sm_check < 0 || tt < 0) return cuda_status(cudaGetLastError());
+  if (ix || at || rs || a2 || stw || tt) {
+    char msg[224];
+    std::snprintf(msg, sizeof(msg), "bounded wait gave up in:%s%s%s%s%s%s", ix ? " k_index_score_tc" : "",
                   at ? " k_sparse_attn_tc" : "", rs ? " k_rescore_tc" : "", a2 ? " k_sparse_attn_2p" : "",
-                  stw ? " k_selftest_wait" : "");
+                  stw ? " k_selftest_wait" : "", tt ? " k_tree_child_tc" : "");
     set_last_error(msg);
     return LSA_ERR_TIMEOUT;
   }
@@ -445,20 +446,27 @@ size_t lsa_tree_workspace_size(int64_t B, int64_t NP, int F, int M2, int M) {
   return tree_ws_layout(B, NP, F, M2, M).total;
 }
 
-int lsa_tree_select(const void* q_idx, const float* w, int64_t B, int H_I, int d_I, const float* centroids,
-                    int64_t NB, const float* parents, int64_t NP, int F, const int32_t* members, int bsz, int M2,
-                    int M, int sink, int window, int64_t L, const int64_t* q_pos, int32_t* idx, int64_t idx_ld,
-                    int32_t* count, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace lsa {
+// The tree search of lsa_tree_select / lsa_tree_select_split: children scored from the fp32 centres on the CUDA
+// cores, or (split_given) from the centres' cached exact bf16 split on the tensor cores.
+static int tree_select_impl(const void* q_idx, const float* w, int64_t B, int H_I, int d_I, const float* centroids,
+                            const void* split_given, int64_t NB, const float* parents, int64_t NP, int F,
+                            const int32_t* members, int bsz, int M2, int M, int sink, int window, int64_t L,
+                            const int64_t* q_pos, int32_t* idx, int64_t idx_ld, int32_t* count, void* ws,
+                            size_t ws_bytes, void* stream) {
   LSA_CHECK_ARG(B >= 0 && NB >= 1 && NB < (int64_t(1) << 31) && F >= 1 && NP == cdiv(NB, F) && bsz >= 1);
   LSA_CHECK_ARG(M2 >= 1 && M2 <= 1024 && M >= 1 && M <= 1024 && static_cast<int64_t>(M2) * F < (int64_t(1) << 30));
   LSA_CHECK_ARG(sink >= 0 && window >= 0 && L >= 1 && H_I >= 1 && H_I <= 64);
   LSA_CHECK_ARG(static_cast<int64_t>(M) * bsz + sink + window <= 8192);
   LSA_CHECK_ARG(idx_ld >= static_cast<int64_t>(M) * bsz + sink + window);
   if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
+  if (split_given && (F != 64 || H_I != 64 || d_I != 128 || NB >= (int64_t(1) << 29))) return LSA_ERR_UNSUPPORTED;
   if (B == 0) return LSA_OK;
   LSA_CHECK_ARG(B <= 65535);
-  LSA_CHECK_ARG(q_idx && w && centroids && parents && members && q_pos && idx && count);
-  LSA_CHECK_ARG(aligned16(q_idx) && aligned16(centroids) && aligned16(parents));
+  LSA_CHECK_ARG(q_idx && w && (centroids || split_given) && parents && members && q_pos && idx && count);
+  LSA_CHECK_ARG(aligned16(q_idx) && aligned16(parents) && (split_given ? aligned16(split_given) : aligned16(centroids)));
   const TreeLayout t = tree_ws_layout(B, NP, F, M2, M);
   if (ws == nullptr || !aligned256(ws) || ws_bytes < t.total) return LSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -483,16 +491,42 @@ int lsa_tree_select(const void* q_idx, const float* w, int64_t B, int H_I, int d
     st = launch_centroid_score(q_idx, w, parents, B, H_I, d_I, NP, pscore, t.ldp, s);
   }
   if (st == LSA_OK) st = launch_topk_mode(pscore, t.ldp, B, NP, M2, 0, 0, q_pos, 1, 1, kp, M2, kpc, M2, s);
-  // level 1: the kept parents' children, scored by gather; the M best candidate slots
-  if (st == LSA_OK)
-    st = launch_tree_child_score(q_idx, w, B, H_I, d_I, centroids, NB, F, kp, M2, kpc, t.n_cand, cscore, cid, t.ldc,
-                                 s);
+  // level 1: the kept parents' children (64 consecutive centre rows per parent on the tensor cores, else a gather
+  // on the CUDA cores); the M best candidate slots
+  if (st == LSA_OK) {
+    if (split_given)
+      st = launch_tree_child_score_tc(q_idx, w, B, split_given, NB, kp, M2, kpc, t.n_cand, cscore, cid, t.ldc, s);
+    else
+      st = launch_tree_child_score(q_idx, w, B, H_I, d_I, centroids, NB, F, kp, M2, kpc, t.n_cand, cscore, cid,
+                                   t.ldc, s);
+  }
   if (st == LSA_OK) st = launch_topk_mode(cscore, t.ldc, B, t.n_cand, M, 0, 0, q_pos, 1, 1, kpos, M, kposc, M, s);
   if (st == LSA_OK) st = launch_tree_map(kpos, M, kposc, cid, t.ldc, t.n_cand, B, kb, M, kbc, s);
   // the kept buckets' members, sink and window (Flat expansion)
   if (st == LSA_OK)
     st = launch_bucket_expand(kb, M, kbc, members, bsz, sink, window, 0, q_pos, B, idx, idx_ld, count, idx_ld, s);
   return st;
+}
+}  // namespace lsa
+
+extern "C" {
+
+int lsa_tree_select(const void* q_idx, const float* w, int64_t B, int H_I, int d_I, const float* centroids,
+                    int64_t NB, const float* parents, int64_t NP, int F, const int32_t* members, int bsz, int M2,
+                    int M, int sink, int window, int64_t L, const int64_t* q_pos, int32_t* idx, int64_t idx_ld,
+                    int32_t* count, void* ws, size_t ws_bytes, void* stream) {
+  if (centroids == nullptr && B > 0) return LSA_ERR_INVALID_ARG;
+  return tree_select_impl(q_idx, w, B, H_I, d_I, centroids, nullptr, NB, parents, NP, F, members, bsz, M2, M, sink,
+                          window, L, q_pos, idx, idx_ld, count, ws, ws_bytes, stream);
+}
+
+int lsa_tree_select_split(const void* q_idx, const float* w, int64_t B, int H_I, int d_I, const void* split,
+                          int64_t NB, const float* parents, int64_t NP, int F, const int32_t* members, int bsz,
+                          int M2, int M, int sink, int window, int64_t L, const int64_t* q_pos, int32_t* idx,
+                          int64_t idx_ld, int32_t* count, void* ws, size_t ws_bytes, void* stream) {
+  if (split == nullptr && B > 0) return LSA_ERR_INVALID_ARG;
+  return tree_select_impl(q_idx, w, B, H_I, d_I, nullptr, split, NB, parents, NP, F, members, bsz, M2, M, sink,
+                          window, L, q_pos, idx, idx_ld, count, ws, ws_bytes, stream);
 }
 
 struct MsaAttnLayout {

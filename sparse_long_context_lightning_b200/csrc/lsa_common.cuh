@@ -174,6 +174,10 @@ int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* 
 int take_index_timeout();
 int take_attn_timeout(int* check);
 int take_attn_simt_check();
+int take_tree_tc_timeout();
+int launch_tree_child_score_tc(const void* q, const float* w, int64_t B, const void* split, int64_t NB,
+                               const int32_t* kp, int64_t kp_ld, const int32_t* kpc, int64_t n_cand, float* cscore,
+                               int32_t* cid, int64_t ldc, cudaStream_t s);
 int take_rescore_timeout();
 int launch_tree_parents(const float* reps, int64_t NB, int d_I, int F, float* parents, cudaStream_t s);
 int launch_tree_child_score(const void* q, const float* w, int64_t B, int H_I, int d_I, const float* reps, int64_t NB,

@@ -215,9 +215,11 @@ def flat10m_tables():
     return wl, q_I, w, members, cen, reps
 
 
-def test_flat10m_tree_full_size(flat10m_tables):
+@pytest.mark.parametrize("split", [False, True])
+def test_flat10m_tree_full_size(flat10m_tables, split):
     """The two-level tree search at the bench's sizes: 156,250 Flat buckets of 64, parents of 64 consecutive
-    buckets (2,442), top-64 parents, top-32 of their 4,096 children, + sink 4 + window 512, 8 queries.
+    buckets (2,442), top-64 parents, top-32 of their 4,096 children, + sink 4 + window 512, 8 queries; children
+    scored by the gather (CUDA cores) or from the centres' cached bf16 split (tensor cores, as in the bench).
     Differences from the oracle only where a bucket ties the M-th candidate or its parent the M2-th parent."""
     wl, q_I, w, members, cen, reps = flat10m_tables
     F, M2, M = 64, 64, wl.M
@@ -230,9 +232,16 @@ def test_flat10m_tree_full_size(flat10m_tables):
     idx = torch.full((wl.B, kmax), 777, dtype=torch.int32, device=DEV)
     cnt = torch.empty(wl.B, dtype=torch.int32, device=DEV)
     ws = lsa.workspace(lsa.lsa_tree_workspace_size(wl.B, NP, F, M2, M))
-    lsa.lsa_tree_select(q_I.to(DEV), w.to(DEV), cen, par, F, members, M2, M, wl.sink, wl.window, wl.L, qp.to(DEV),
-                        idx, cnt, ws)
+    if split:
+        sp = torch.empty(3, nb, 128, dtype=torch.bfloat16, device=DEV)
+        lsa.lsa_split_representatives(cen, sp)
+        lsa.lsa_tree_select_split(q_I.to(DEV), w.to(DEV), sp, par, F, members, M2, M, wl.sink, wl.window, wl.L,
+                                  qp.to(DEV), idx, cnt, ws)
+    else:
+        lsa.lsa_tree_select(q_I.to(DEV), w.to(DEV), cen, par, F, members, M2, M, wl.sink, wl.window, wl.L,
+                            qp.to(DEV), idx, cnt, ws)
     torch.cuda.synchronize()
+    lsa.lsa_device_status()
     np.testing.assert_allclose(f64(par), O.tree_parents(f64(cen), F), rtol=1e-5, atol=1e-5)
     mem_np = members.cpu().numpy()
     parents = O.tree_parents(reps, F)

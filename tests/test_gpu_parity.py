@@ -243,8 +243,9 @@ def test_microblock_select_paths(path):
     _bucket_case(L=4 * 16384 + 3, B=4, M=512, bsz=4, sink=4, window=128, flat=False, path=path)
 
 
-def _tree_run(L, B, bsz, F, M2, M, sink, window, q_pos=None):
-    """lsa_tree_select against the oracle's two-level search on the fp64 pooled keys.  Returns the GPU rows."""
+def _tree_run(L, B, bsz, F, M2, M, sink, window, q_pos=None, split=False):
+    """lsa_tree_select (split: lsa_tree_select_split, children on the tensor cores from the centres' cached bf16
+    split) against the oracle's two-level search on the fp64 pooled keys.  Returns the GPU rows."""
     wl = S.Workload("tr", L=L, B=B, H_I=64, d_I=128, K=M * bsz, H=16, sink=sink, window=window, mode="flat",
                     bsz=bsz, M=M)
     q_I, w = S.index_queries(wl)
@@ -261,9 +262,16 @@ def _tree_run(L, B, bsz, F, M2, M, sink, window, q_pos=None):
     idx = torch.full((B, kmax), 777, dtype=torch.int32, device=DEV)
     cnt = torch.empty(B, dtype=torch.int32, device=DEV)
     ws = lsa.workspace(lsa.lsa_tree_workspace_size(B, NP, F, M2, M))
-    lsa.lsa_tree_select(q_I.to(DEV), w.to(DEV), cen, par, F, members, M2, M, sink, window, L, qp.to(DEV), idx, cnt,
-                        ws)
+    if split:
+        sp = torch.empty(3, nb, 128, dtype=torch.bfloat16, device=DEV)
+        lsa.lsa_split_representatives(cen, sp)
+        lsa.lsa_tree_select_split(q_I.to(DEV), w.to(DEV), sp, par, F, members, M2, M, sink, window, L, qp.to(DEV),
+                                  idx, cnt, ws)
+    else:
+        lsa.lsa_tree_select(q_I.to(DEV), w.to(DEV), cen, par, F, members, M2, M, sink, window, L, qp.to(DEV), idx,
+                            cnt, ws)
     torch.cuda.synchronize()
+    lsa.lsa_device_status()
     # the parents themselves: fp32 means of the fp32 centres
     np.testing.assert_allclose(f64(par), O.tree_parents(f64(cen), F), rtol=1e-5, atol=1e-5)
     mem_np = members.cpu().numpy()
@@ -295,6 +303,24 @@ def test_tree_select(F, M2, M):
     the full beam; F = 1 ranks the buckets themselves; F = 100, M2 = 1 has exactly M candidates)."""
     L, B = 64 * 10000, 6
     _tree_run(L, B, 64, F, M2, M, 4, 512, q_pos=[L - 1, L - 1, L // 2, 70000, L - 1, 4000])
+
+
+@pytest.mark.parametrize("M2,M", [(16, 32), (7, 20), (156, 32)])
+def test_tree_select_split(M2, M):
+    """Children on the tensor cores (F = 64): 10000 buckets (a ragged last parent of 16), an odd number of kept
+    parents (the last pair half empty) and a full beam over all 157 parents but one."""
+    L, B = 64 * 10000, 6
+    _tree_run(L, B, 64, 64, M2, M, 4, 512, q_pos=[L - 1, L - 1, L // 2, 70000, L - 1, 4000], split=True)
+
+
+def test_tree_split_matches_gather_path():
+    """The tensor-core children scores equal the CUDA-core ones up to fp32 summation order: same rows, except ties."""
+    L, B = 64 * 6000 + 64 * 3, 4
+    a_idx, a_cnt = _tree_run(L, B, 64, 64, 24, 32, 4, 128)
+    b_idx, b_cnt = _tree_run(L, B, 64, 64, 24, 32, 4, 128, split=True)
+    for b in range(B):
+        d = np.setxor1d(a_idx[b, : a_cnt[b]], b_idx[b, : b_cnt[b]])
+        assert d.size <= 2 * 64, (b, d.size)  # at most one tied bucket swapped
 
 
 def test_tree_full_beam_matches_flat():
