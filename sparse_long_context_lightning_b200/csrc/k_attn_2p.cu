@@ -10,8 +10,8 @@
 //   pass 1  gathers whole rows (16-byte cp.async into the 128-byte-swizzled K-major tile), computes the logits
 //           S = Q C^T on the tensor cores with all of Q (576 dims = 288 columns) as the A operand in TMEM, and
 //           runs the online softmax; P (bf16) of every tile is kept in shared memory.  A stage is released as
-//           soon as its logits MMAs complete, and four warps issue the logits (one tile each, four S buffers),
-//           so four row tiles are in flight;
+//           soon as its logits MMAs complete; each tile's logits are split over two issuing warps (two K-half
+//           accumulators), two tiles at a time, and four row tiles are in flight;
 //   pass 2  gathers value dims [0, 512) of the same rows again (1 KB per row, mostly served by L2) and
 //           accumulates O = P V for both value halves (all 512 TMEM columns), replaying pass 1's (rare)
 //           rescales of the running softmax reference.
@@ -19,8 +19,9 @@
 // (L2) read per row instead of a second CTA that would gather the full rows and recompute the logits.  Units of
 // one query are merged by the combine kernel (log-sum-exp weights).
 //
-// Warp roles (768 threads): warps 0-15 gather (two rows of each tile per warp), 16-19 issue the logits MMAs of
-// tiles j = warp - 16 (mod 4) (16 owns TMEM; 19 also issues pass 2's P.V MMAs), 20-23 move Q into TMEM and run
+// Warp roles (768 threads): warps 0-15 gather (two rows of each tile per warp), 16-19 issue the logits MMAs
+// (16 and 17 for even tiles, 18 and 19 for odd ones, one K half each; 16 owns TMEM; 19 also issues pass 2's
+// P.V MMAs), 20-23 move Q into TMEM and run
 // the softmax (one head per thread = one TMEM lane).  The output is written by the twenty gather and softmax
 // warps (five per TMEM lane quarter).
 #include <cuda_fp16.h>
@@ -47,7 +48,7 @@ constexpr int A2_T = 32;          // rows per tile
 constexpr int A2_H = 128;         // heads (MMA M)
 constexpr int A2_KB = 9;          // 64-dim K-blocks of a 576-dim row
 constexpr int A2_MAXT = 8;        // tiles per work unit (P of every tile is kept)
-constexpr int A2_STAGES = 4;      // = the number of logits-issuing warps: tile j uses stage j % 4
+constexpr int A2_STAGES = 4;      // tile j uses stage j % 4
 constexpr int A2_QSLOTS = 9;      // Q's 64-dim blocks, all staged at once (stages 1-3 and the P area)
 constexpr int A2_KB_BYTES = A2_T * 128;                     // 4 KB: one 64-dim block of a tile
 constexpr int A2_STAGE_BYTES = A2_KB * A2_KB_BYTES;         // 36 KB
@@ -59,7 +60,7 @@ constexpr int A2_FIN_BYTES = A2_H * 4 * 2;                  // final sum and ref
 constexpr int A2_BAR_BYTES = 512;
 constexpr int A2_SMEM = 1024 + A2_STAGES * A2_STAGE_BYTES + A2_P_BYTES + A2_M_BYTES + A2_IDX_BYTES + A2_FIN_BYTES +
                         A2_BAR_BYTES;
-constexpr uint32_t TM_S = 0;     // pass 1: four S buffers of 32 columns [0, 128)
+constexpr uint32_t TM_S = 0;     // pass 1: two S buffers of two 32-column partials [0, 128)
 constexpr uint32_t TM_Q = 224;   // pass 1: Q dims [0, 576), two bf16 per column [224, 512)
 constexpr uint32_t TM_O0 = 0;    // pass 2: O value dims [0, 256)
 constexpr uint32_t TM_O1 = 256;  // pass 2: O value dims [256, 512)
@@ -162,8 +163,8 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   if (tid == 0) {
     for (int i = 0; i < A2_STAGES; ++i) {
       mbar_init(&kv_full[i], A2_GATHER_WARPS * 32);
-      mbar_init(&kv_empty[i], 1);
-      mbar_init(&s_full[i], 1);
+      mbar_init(&kv_empty[i], 2);
+      mbar_init(&s_full[i], 2);  // buffers 0, 1 used
       mbar_init(&s_empty[i], 4);
       mbar_init(&drain[i], 1);
     }
@@ -268,33 +269,36 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
     }
   } else if (warp < A2_SOFTMAX_WARP0) {
     // ------------------------------------------------------------------ logits MMAs (pass 1), P.V (pass 2)
-    // One thread issues about one tcgen05.mma per 30-50 ns, so tile j's 36 logits MMAs are issued by warp
-    // 16 + j % 4 into S buffer j % 4 from stage j % 4: four tiles' logits are in flight at once.
+    // One thread issues about one tcgen05.mma per 30-50 ns, so a tile's 36 logits MMAs (K = 576 in steps of 16)
+    // are split over a warp pair: warp 16 + 2 (j % 2) issues K steps 0-17 and the next warp steps 18-35 of tile j,
+    // each into its own partial S accumulator of buffer j % 2 (the softmax adds the two).  Two tiles' logits
+    // are in flight, each at about half the latency of one warp issuing all 36.
     const int lw = warp - A2_LOGIT_WARP0;
+    const int pair = lw >> 1, khalf = lw & 1;
     if (lane == 0 && ntiles > 0) {
       bool ok = true, issued = false;
-      if (ntiles > lw) {
+      if (ntiles > pair) {
         ok = wait_ab(qt_full, 0, abort_flag);
         tc_fence_after();
-        const uint32_t d = tmem + TM_S + lw * A2_T;
-        const uint64_t sdesc = desc_sw128(smem_u32(st_s + lw * A2_STAGE_BYTES));
-        for (int j = lw; ok && j < ntiles; j += A2_STAGES) {
-          const int use = j / A2_STAGES;
-          if (!wait_ab(&kv_full[lw], use & 1, abort_flag) || !wait_ab(&s_empty[lw], (use & 1) ^ 1, abort_flag)) {
+        const uint32_t d = tmem + TM_S + pair * 2 * A2_T + khalf * A2_T;
+        for (int j = pair; ok && j < ntiles; j += 2) {
+          const int st = j % A2_STAGES;
+          if (!wait_ab(&kv_full[st], (j / A2_STAGES) & 1, abort_flag) ||
+              !wait_ab(&s_empty[pair], ((j >> 1) & 1) ^ 1, abort_flag)) {
             ok = false;
             break;
           }
           fence_proxy_async_smem();  // the cp.async (generic proxy) writes are read by the tensor cores
           tc_fence_after();
+          const uint64_t sdesc = desc_sw128(smem_u32(st_s + st * A2_STAGE_BYTES));
           #pragma unroll
-          for (int kb = 0; kb < A2_KB; ++kb) {
-            #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_ta(d, tmem + TM_Q + kb * 32 + kk * 8, sdesc + ((kb * A2_KB_BYTES + kk * 32) >> 4), IDESC_S,
-                         (kb | kk) != 0);
+          for (int k = 0; k < 18; ++k) {
+            const int ks = khalf * 18 + k, kb = ks >> 2, kk = ks & 3;
+            mma_f16_ta(d, tmem + TM_Q + kb * 32 + kk * 8, sdesc + ((kb * A2_KB_BYTES + kk * 32) >> 4), IDESC_S,
+                       k != 0);
           }
-          mma_commit(&kv_empty[lw]);  // the stage is free once the logits have read it
-          mma_commit(&s_full[lw]);
+          mma_commit(&kv_empty[st]);  // the stage is free once both halves' logits have read it
+          mma_commit(&s_full[pair]);
           issued = true;
         }
       }
@@ -328,6 +332,7 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
                       desc_sw128_mn(v_addr + half * 4 * A2_KB_BYTES + kk * 16 * 128, A2_KB_BYTES, 1024), IDESC_PV,
                       (j > 0 || kk > 0) ? 1u : 0u);
           }
+          mma_commit(&kv_empty[st]);  // two arrivals: the stage barrier counts the two logits halves of pass 1
           mma_commit(&kv_empty[st]);
           mma_commit(&pv_done[j]);
           issued = true;
@@ -371,22 +376,24 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
       ok = ok && __all_sync(0xffffffffu, wait_ab(qt_full, 0, abort_flag));
     }
     for (int i = 0; ok && i < ntiles; ++i) {
-      const int sb = i % A2_STAGES;
+      const int sb = i & 1;
       const int nvalid = min(A2_T, nrows - i * A2_T);
-      if (!__all_sync(0xffffffffu, wait_ab(&s_full[sb], (i / A2_STAGES) & 1, abort_flag))) {
+      if (!__all_sync(0xffffffffu, wait_ab(&s_full[sb], (i >> 1) & 1, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[32];
-      tmem_ld32(trow + TM_S + sb * A2_T, sr);
+      uint32_t sr[32], sr2[32];
+      tmem_ld32(trow + TM_S + sb * 2 * A2_T, sr);  // the two K-half partial logits
+      tmem_ld32(trow + TM_S + sb * 2 * A2_T + A2_T, sr2);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[sb]);
       float z[A2_T];
       #pragma unroll
-      for (int c = 0; c < A2_T; ++c) z[c] = c < nvalid ? __uint_as_float(sr[c]) * a.scale_log2 : -INFINITY;
+      for (int c = 0; c < A2_T; ++c)
+        z[c] = c < nvalid ? (__uint_as_float(sr[c]) + __uint_as_float(sr2[c])) * a.scale_log2 : -INFINITY;
       float m8[8];
       #pragma unroll
       for (int j = 0; j < 8; ++j) m8[j] = z[j];
@@ -474,15 +481,13 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
       float mx = 0.f;
       #pragma unroll 1
       for (int c = rank; c < 8; c += 5) {
-        #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          uint32_t o[32];
-          if (have) {
-            tmem_ld32(trow + 64 * c + 32 * part, o);
-            tmem_ld_wait();
-            #pragma unroll
-            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, fabsf(__uint_as_float(o[k])));
-          }
+        if (have) {  // both 32-column halves of the chunk in flight before one wait
+          uint32_t o[32], o2[32];
+          tmem_ld32(trow + 64 * c, o);
+          tmem_ld32(trow + 64 * c + 32, o2);
+          tmem_ld_wait();
+          #pragma unroll
+          for (int k = 0; k < 32; ++k) mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(o[k])), fabsf(__uint_as_float(o2[k]))));
         }
       }
       rmax_s[rank * A2_H + h] = mx;
