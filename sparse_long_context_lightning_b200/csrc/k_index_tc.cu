@@ -98,25 +98,38 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 // later, which no warp reaches before every warp has finished this tile).
 template <int G>
 __device__ __forceinline__ void block_max_epilogue(const IxArgs& a, const float* w, const uint32_t (&r0)[32],
-                                                   const uint32_t (&r1)[32], int s, int b, int tile, int lane,
-                                                   uint32_t* mx, uint32_t* cnt) {
+                                                   const uint32_t (&r1)[32], int s, int b, int64_t qpb, int tile,
+                                                   int lane, uint32_t* mx, uint32_t* cnt) {
   constexpr int GW = 64 / G;  // heads per group
-  float acc[G];
+  constexpr int LG = G == 1 ? 0 : (G == 2 ? 1 : (G == 4 ? 2 : 3));
+  float v[G];
   #pragma unroll
-  for (int g = 0; g < G; ++g) acc[g] = 0.f;
+  for (int g = 0; g < G; ++g) v[g] = 0.f;
   #pragma unroll
-  for (int c = 0; c < 32; ++c) acc[c / GW] = fmaf(w[c], fmaxf(__uint_as_float(r0[c]), 0.f), acc[c / GW]);
+  for (int c = 0; c < 32; ++c) v[c / GW] = fmaf(w[c], fmaxf(__uint_as_float(r0[c]), 0.f), v[c / GW]);
   #pragma unroll
-  for (int c = 0; c < 32; ++c)
-    acc[(32 + c) / GW] = fmaf(w[32 + c], fmaxf(__uint_as_float(r1[c]), 0.f), acc[(32 + c) / GW]);
-  const bool valid = b < a.B && s < a.L && s <= a.q_pos[b];
+  for (int c = 0; c < 32; ++c) v[(32 + c) / GW] = fmaf(w[32 + c], fmaxf(__uint_as_float(r1[c]), 0.f), v[(32 + c) / GW]);
+  const bool valid = b < a.B && s < a.L && s <= qpb;
   #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float v = valid ? acc[g] : -INFINITY;
+  for (int g = 0; g < G; ++g) v[g] = valid ? v[g] : -INFINITY;
+  // max over the warp's 32 keys of each group sum, as a transposing reduction: each exchange over lane bit
+  // 4, 3, 2 halves the values a lane holds (it keeps the half its bit selects), then the remaining lane bits are
+  // reduced on one value; lane l ends with group l >> (5 - LG) (G - 1 + 5 - LG shuffles instead of 5 G)
+  #pragma unroll
+  for (int step = 0; step < LG; ++step) {
+    const int half = (G >> step) / 2, off = 16 >> step;
+    const bool upper = (lane & off) != 0;
     #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (lane == 0) atomicMax(&mx[g], float_key(v));
+    for (int i = 0; i < half; ++i) {
+      const float keep = upper ? v[i + half] : v[i];
+      const float send = upper ? v[i] : v[i + half];
+      v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, off));
+    }
   }
+  #pragma unroll
+  for (int off = 16 >> LG; off > 0; off >>= 1) v[0] = fmaxf(v[0], __shfl_xor_sync(0xffffffffu, v[0], off));
+  if ((lane & ((32 >> LG) - 1)) == 0) atomicMax(&mx[lane >> (5 - LG)], float_key(v[0]));
+  __syncwarp();  // every group's maximum is in before lane 0 counts this quarter
   if (lane == 0) {
     __threadfence_block();
     if (atomicAdd(cnt, 1u) == 3u) {
@@ -285,6 +298,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     const int quarter = warp & 3;
     const int col0 = (ew >> 2) * 64;
     const int nq = 64 / a.H_I;  // queries in this warp's 64 columns (1 or 2)
+    const int64_t qpb = (G > 0 && b0 + (col0 >> 6) < a.B) ? a.q_pos[b0 + (col0 >> 6)] : -1;  // grouped: one query
     for (int i = 0; i < n_my; ++i) {
       const int buf = i & 1;
       // decided warp-wide: the TMEM loads below are warp-collective
@@ -304,7 +318,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       if (lane == 0) mbar_arrive(&tempty[buf]);  // the accumulator columns are in registers now
       const int s = (t_begin + i) * IX_TILE_M + quarter * 32 + lane;
       if constexpr (G > 0) {
-        block_max_epilogue<G>(a, wsm + col0, r0, r1, s, b0 + (col0 >> 6), t_begin + i, lane,
+        block_max_epilogue<G>(a, wsm + col0, r0, r1, s, b0 + (col0 >> 6), qpb, t_begin + i, lane,
                               gmax + ((i & 3) * 4 + (ew >> 2)) * 8, gcnt + (i & 3) * 4 + (ew >> 2));
         continue;
       }
