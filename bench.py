@@ -263,7 +263,7 @@ def committed_traffic(kernel: str):
 
 STAGE_KERNEL = {"index": ("k_index_score_tc", ["k_index_tc.cu"]),
                 "topk": ("k_topk_cluster", ["k_topk.cu"]),
-                "attn": ("k_sparse_attn_tc", ["k_attn_tc.cu"])}
+                "attn": ("k_sparse_attn_2p", ["k_attn_2p.cu"])}
 # kernels each stage launches per step (the e2e leg adds none of ours)
 LAUNCHES = {"index": 1, "topk": 1, "attn": 1}
 

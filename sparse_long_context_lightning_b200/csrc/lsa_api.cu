@@ -180,24 +180,27 @@ int lsa_selftest_wait(uint64_t limit_ns, void* stream) {
 int lsa_device_status(void* stream) {
   const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_status(e);
-  int a2_check = 0, at_check = 0;
+  int a2_check = 0, at_check = 0, ma_check = 0;
   const int ix = take_index_timeout(), at = take_attn_timeout(&at_check), rs = take_rescore_timeout();
   const int a2 = take_attn2_flags(&a2_check), stw = take_selftest_timeout(), sm_check = take_attn_simt_check();
-  const int tt = take_tree_tc_timeout();
-  if (ix < 0 || at < 0 || rs < 0 || a2 < 0 || stw < 0 || sm_check < 0 || tt < 0) return cuda_status(cudaGetLastError());
-  if (ix || at || rs || a2 || stw || tt) {
-    char msg[224];
-    std::snprintf(msg, sizeof(msg), "bounded wait gave up in:%s%s%s%s%s%s", ix ? " k_index_score_tc" : "",
+  const int tt = take_tree_tc_timeout(), ma = take_msa_attn_flags(&ma_check);
+  if (ix < 0 || at < 0 || rs < 0 || a2 < 0 || stw < 0 || sm_check < 0 || tt < 0 || ma < 0)
+    return cuda_status(cudaGetLastError());
+  if (ix || at || rs || a2 || stw || tt || ma) {
+    char msg[256];
+    std::snprintf(msg, sizeof(msg), "bounded wait gave up in:%s%s%s%s%s%s%s", ix ? " k_index_score_tc" : "",
                   at ? " k_sparse_attn_tc" : "", rs ? " k_rescore_tc" : "", a2 ? " k_sparse_attn_2p" : "",
-                  stw ? " k_selftest_wait" : "", tt ? " k_tree_child_tc" : "");
+                  stw ? " k_selftest_wait" : "", tt ? " k_tree_child_tc" : "", ma ? " k_msa_attn_rows" : "");
     set_last_error(msg);
     return LSA_ERR_TIMEOUT;
   }
-  if (a2_check || at_check || sm_check) {
-    char msg[192];
-    std::snprintf(msg, sizeof(msg), "device check failed (a selected index outside [0, L); the row was clamped) in:%s%s%s",
+  if (a2_check || at_check || sm_check || ma_check) {
+    char msg[256];
+    std::snprintf(msg, sizeof(msg),
+                  "device check failed (a selected index outside [0, L), the row clamped; or MSA rows that are not whole "
+                  "blocks) in:%s%s%s%s",
                   a2_check ? " k_sparse_attn_2p" : "", at_check ? " k_sparse_attn_tc" : "",
-                  sm_check ? " k_attn_simt" : "");
+                  sm_check ? " k_attn_simt" : "", ma_check ? " k_msa_attn_rows" : "");
     set_last_error(msg);
     return LSA_ERR_DEVICE_CHECK;
   }
@@ -538,6 +541,11 @@ static MsaAttnLayout msa_attn_layout(int64_t B, int64_t idx_ld, int G) {
   m.o_cnt = align_up(bg * idx_ld * 4, 256);
   size_t o = m.o_cnt + align_up(bg * 4, 256);
   m.o_q = m.o_out = m.o_lse = o;
+  if (G == 8) {  // 16 heads per group: the rows-on-M kernel needs only the group rows and their counts
+    m.o_att = o;
+    m.total = o;
+    return m;
+  }
   if (G > 1) {  // the padded 128-head queries, their outputs and lse
     m.o_q = o;
     o += align_up(bg * 128 * 576 * 2, 256);
@@ -573,6 +581,11 @@ int lsa_msa_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, c
   // each group's rows; then one 128-head attention per (query, group) on the tensor cores, the group's heads in
   // the first 128 / G rows of a zero-padded query (G = 1: the query itself)
   int st = launch_msa_group_rows(idx, gmask, idx_ld, count, B, G, grows, gcnt, s);
+  if (G == 8) {
+    // 16 heads per group: one CTA per (query, group), each kept block's 128 rows on the MMA's M side
+    if (st == LSA_OK) st = launch_msa_attn_rows(q, kv, L, grows, idx_ld, gcnt, B, G, scale, out, lse, s);
+    return st;
+  }
   if (G == 1) {
     if (st == LSA_OK)
       st = launch_sparse_attn(q, kv, L, grows, idx_ld, gcnt, B, 128, scale, out, lse, base + m.o_att,

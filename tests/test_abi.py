@@ -96,10 +96,12 @@ def test_selection_workspace_sizes(lib):
     # MSA selection: block scores for every (query, group)
     m = lib.lsa_msa_workspace_size(16, 131072, 8, 16)
     assert m % 256 == 0 and m >= 16 * 8 * 1024 * 4
-    # MSA attention: per-group rows plus the padded 128-head queries and outputs when G > 1
+    # MSA attention: per-group rows and counts (G = 8: the rows-on-M kernel needs nothing more); the padded
+    # 128-head queries and outputs as well for G = 2 and 4
     a8 = lib.lsa_msa_attn_workspace_size(16, 129 * 128, 8)
-    a1 = lib.lsa_msa_attn_workspace_size(16, 129 * 128, 1)
-    assert a8 >= 16 * 8 * 129 * 128 * 4 + 16 * 8 * 128 * (576 + 512) * 2 and a1 < a8
+    a2 = lib.lsa_msa_attn_workspace_size(16, 129 * 128, 2)
+    assert a8 % 256 == 0 and a8 >= 16 * 8 * 129 * 128 * 4 + 16 * 8 * 4
+    assert a2 >= 16 * 2 * 129 * 128 * 4 + 16 * 2 * 128 * (576 + 512) * 2
     assert lib.lsa_msa_attn_workspace_size(16, 128, 0) == bad
     assert lib.lsa_hi_workspace_size(4, 1 << 20, 128, 8, 1024, 2048, 4, 128) > 0
 
