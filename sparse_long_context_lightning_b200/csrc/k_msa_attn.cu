@@ -38,11 +38,13 @@ constexpr int MA_QSLICE = MA_NH * 128;           // 2 KB: one slice of Q_g
 constexpr int MA_LR = 6;                         // logits ring slots (one slice each)
 constexpr int MA_VR = 2;                         // value ring slots (two slices each)
 constexpr int MA_P_BYTES = MA_NH * MA_ROWS * 2;  // 4 KB: P^T of a tile, bf16, K-major (16 head rows)
+constexpr int MA_MAXT = 512;                     // blocks per union row (idx_ld <= 65536)
 constexpr uint32_t TM_S = 0;                     // two S^T buffers, 16 columns each
 constexpr uint32_t TM_O = 32;                    // O^T: four 128-dim tiles of 16 columns
 constexpr float RESCALE_LOG2 = 8.f;
 constexpr uint64_t WAIT_NS = 2000000000ull;
-constexpr int MA_SMEM = 1024 + MA_KB * 1024 * 2 + MA_LR * MA_SLICE + MA_VR * 2 * MA_SLICE + 2 * MA_P_BYTES + 2048;
+constexpr int MA_SMEM =
+    1024 + MA_KB * 1024 * 2 + MA_LR * MA_SLICE + MA_VR * 2 * MA_SLICE + 2 * MA_P_BYTES + 2048 + MA_MAXT * 8;
 static_assert(MA_SMEM <= 232448, "shared memory");
 static_assert(MA_NH * MA_ROWS / 2 * 2 <= MA_LR * MA_SLICE, "epilogue staging fits the logits ring");
 
@@ -55,9 +57,11 @@ constexpr uint32_t IDESC_S = idesc_ab(MA_ROWS, MA_NH, 0u, 0u);   // A = C tile (
 constexpr uint32_t IDESC_PV = idesc_ab(128, MA_NH, 1u, 0u);      // A = V^T (dims contiguous), B = P^T (K-major)
 
 struct MaArgs {
-  const int32_t* rows;   // [B G, ld] each (query, group)'s rows, ascending (whole kept blocks, then the local block)
+  const int32_t* idx;     // [B, ld] the union of the groups' kept blocks, ascending (whole 128-token blocks, then
+                          // the partial local block)
+  const uint8_t* gmask;   // [B, ld] bit g: group g kept the entry's block
   int64_t ld;
-  const int32_t* count;  // [B G]
+  const int32_t* count;   // [B]
   int G;
   int L;
   float scale_log2;
@@ -148,10 +152,14 @@ __global__ void __launch_bounds__(MA_THREADS, 1)
   uint64_t* drain = o_done + 1;           // [2]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* ntiles_s = const_cast<int*>(abort_flag) + 1;
+  int* tfirst = reinterpret_cast<int*>(base + MA_SMEM - 1024 - MA_MAXT * 8);  // [512] this group's blocks: first entry
+  int* trows = tfirst + MA_MAXT;                                                // [512] and its number of rows
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bg = blockIdx.x;  // query b = bg / G, group g = bg % G
   const int b = bg / a.G, g = bg % a.G;
+  const int32_t* ridx = a.idx + static_cast<int64_t>(b) * a.ld;
   if (tid == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < MA_LR; ++i) {
@@ -185,13 +193,29 @@ __global__ void __launch_bounds__(MA_THREADS, 1)
   }
   pdl_wait();
   pdl_launch_dependents();
-  int n = a.count[bg];
-  n = n < 0 ? 0 : (static_cast<int64_t>(n) > a.ld ? static_cast<int>(a.ld) : n);
-  const int ntiles = (n + MA_ROWS - 1) / MA_ROWS;
-  const int32_t* rows = a.rows + static_cast<int64_t>(bg) * a.ld;
+  if (warp == 0) {
+    // this group's tiles: the union row's blocks (entries j * 128 ..) whose mask has bit g, in order
+    int n = a.count[b];
+    n = n < 0 ? 0 : (static_cast<int64_t>(n) > a.ld ? static_cast<int>(a.ld) : n);
+    const int nblk = min((n + MA_ROWS - 1) / MA_ROWS, MA_MAXT);
+    int kept = 0;
+    for (int j0 = 0; j0 < nblk; j0 += 32) {
+      const int j = j0 + lane;
+      const bool mine = j < nblk && ((a.gmask[static_cast<int64_t>(b) * a.ld + static_cast<int64_t>(j) * MA_ROWS] >> g) & 1u);
+      const uint32_t bal = __ballot_sync(0xffffffffu, mine);
+      if (mine) {
+        const int o = kept + __popc(bal & ((1u << lane) - 1u));
+        tfirst[o] = j * MA_ROWS;
+        trows[o] = min(MA_ROWS, n - j * MA_ROWS);
+      }
+      kept += __popc(bal);
+    }
+    if (lane == 0) *ntiles_s = kept;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const int ntiles = *ntiles_s;
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 0 || warp == 1) {
@@ -204,7 +228,7 @@ __global__ void __launch_bounds__(MA_THREADS, 1)
       int issued = 0;
       bool ok = true;
       for (int t = 0; ok && t < ntiles; ++t) {
-        int first = rows[t * MA_ROWS];
+        int first = ridx[tfirst[t]];
         first = first < 0 ? 0 : (first >= a.L ? a.L - 1 : first);
         const int nitems = logits ? MA_KB : 4;
         for (int k = 0; k < nitems; ++k) {
@@ -334,9 +358,8 @@ __global__ void __launch_bounds__(MA_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[x]);
-        const int rr = t * MA_ROWS + r;
-        const bool valid = rr < n;
-        if (valid && rows[rr] != rows[t * MA_ROWS] + r) atomicExch(&g_msa_attn_check, 1);  // not one block
+        const bool valid = r < trows[t];
+        if (valid && ridx[tfirst[t] + r] != ridx[tfirst[t]] + r) atomicExch(&g_msa_attn_check, 1);  // not one block
         #pragma unroll
         for (int h = 0; h < MA_NH; ++h) z[h] = valid ? __uint_as_float(sr[h]) * a.scale_log2 : -INFINITY;
       } else {
@@ -490,20 +513,21 @@ __global__ void __launch_bounds__(MA_THREADS, 1)
 
 int make_map(CUtensorMap* m, const void* ptr, bool fp8, int64_t rows, int64_t cols, int box_cols, int box_rows);
 
-// MSA attention with 16 heads per group (128 query heads in 8 groups): one CTA per (query, group) over the
-// group's compacted rows (whole kept blocks, then the local block).
-int launch_msa_attn_rows(const void* q, const void* kv, int64_t L, const int32_t* grows, int64_t ld,
-                         const int32_t* gcnt, int64_t B, int G, float scale, void* out, float* lse, cudaStream_t s) {
-  if (128 / G != MA_NH) return LSA_ERR_UNSUPPORTED;
+// MSA attention with 16 heads per group (128 query heads in 8 groups): one CTA per (query, group) over the union
+// row's blocks that the group kept.
+int launch_msa_attn_rows(const void* q, const void* kv, int64_t L, const int32_t* idx, const uint8_t* gmask, int64_t ld,
+                         const int32_t* count, int64_t B, int G, float scale, void* out, float* lse, cudaStream_t s) {
+  if (128 / G != MA_NH || ld > static_cast<int64_t>(MA_MAXT) * MA_ROWS) return LSA_ERR_UNSUPPORTED;
   CUtensorMap tkv, tq;
   int st = make_map(&tkv, kv, false, L, 576, 64, MA_ROWS);
   if (st) return st;
   st = make_map(&tq, q, false, B * 128, 576, 64, MA_NH);
   if (st) return st;
   MaArgs a;
-  a.rows = grows;
+  a.idx = idx;
+  a.gmask = gmask;
   a.ld = ld;
-  a.count = gcnt;
+  a.count = count;
   a.G = G;
   a.L = static_cast<int>(L);
   a.scale_log2 = scale * 1.4426950408889634f;

@@ -541,9 +541,8 @@ static MsaAttnLayout msa_attn_layout(int64_t B, int64_t idx_ld, int G) {
   m.o_cnt = align_up(bg * idx_ld * 4, 256);
   size_t o = m.o_cnt + align_up(bg * 4, 256);
   m.o_q = m.o_out = m.o_lse = o;
-  if (G == 8) {  // 16 heads per group: the rows-on-M kernel needs only the group rows and their counts
-    m.o_att = o;
-    m.total = o;
+  if (G == 8) {  // 16 heads per group: the rows-on-M kernel reads the union row and its masks directly
+    m.o_cnt = m.o_q = m.o_out = m.o_lse = m.o_att = m.total = 0;
     return m;
   }
   if (G > 1) {  // the padded 128-head queries, their outputs and lse
@@ -573,19 +572,19 @@ int lsa_msa_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, c
   LSA_CHECK_ARG(q && kv && idx && gmask && count && out);
   LSA_CHECK_ARG(aligned16(q) && aligned16(kv) && aligned16(out) && B * G <= 65535);
   const MsaAttnLayout m = msa_attn_layout(B, idx_ld, G);
-  if (ws == nullptr || !aligned256(ws) || ws_bytes < m.total) return LSA_ERR_WORKSPACE;
+  if (m.total > 0 && (ws == nullptr || !aligned256(ws) || ws_bytes < m.total)) return LSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (G == 8) {
+    // 16 heads per group: one CTA per (query, group), each kept 128-token block on the MMA's M side, the group's
+    // blocks read from the union row's masks
+    return launch_msa_attn_rows(q, kv, L, idx, gmask, idx_ld, count, B, G, scale, out, lse, s);
+  }
   unsigned char* base = static_cast<unsigned char*>(ws);
   int32_t* grows = reinterpret_cast<int32_t*>(base);
   int32_t* gcnt = reinterpret_cast<int32_t*>(base + m.o_cnt);
   // each group's rows; then one 128-head attention per (query, group) on the tensor cores, the group's heads in
   // the first 128 / G rows of a zero-padded query (G = 1: the query itself)
   int st = launch_msa_group_rows(idx, gmask, idx_ld, count, B, G, grows, gcnt, s);
-  if (G == 8) {
-    // 16 heads per group: one CTA per (query, group), each kept block's 128 rows on the MMA's M side
-    if (st == LSA_OK) st = launch_msa_attn_rows(q, kv, L, grows, idx_ld, gcnt, B, G, scale, out, lse, s);
-    return st;
-  }
   if (G == 1) {
     if (st == LSA_OK)
       st = launch_sparse_attn(q, kv, L, grows, idx_ld, gcnt, B, 128, scale, out, lse, base + m.o_att,

@@ -199,6 +199,6 @@ size_t sparse_attn_ws_bytes(int64_t B, int64_t kmax, int H);
 int attn_launches_per_call(int64_t B, int64_t idx_ld, int H);
 int take_attn2_flags(int* check);
 int take_msa_attn_flags(int* check);
-int launch_msa_attn_rows(const void* q, const void* kv, int64_t L, const int32_t* grows, int64_t ld,
-                         const int32_t* gcnt, int64_t B, int G, float scale, void* out, float* lse, cudaStream_t s);
+int launch_msa_attn_rows(const void* q, const void* kv, int64_t L, const int32_t* idx, const uint8_t* gmask, int64_t ld,
+                         const int32_t* count, int64_t B, int G, float scale, void* out, float* lse, cudaStream_t s);
 }  // namespace lsa
