@@ -74,3 +74,29 @@ def test_out_of_range_index_is_clamped_and_reported(B, H, kmax):
     pad[:, kmax - 10:] = -1
     lsa.lsa_sparse_attn(q, kv, pad.to(DEV), cnt2.to(DEV), scale, out, lse, ws)
     lsa.lsa_device_status()
+
+
+def test_msa_rows_that_are_not_whole_blocks_are_reported():
+    """The 8-group MSA attention runs each kept block as one tile of 128 consecutive tokens; a union row whose
+    block holds other tokens is computed all the same (every access stays in bounds) and flagged."""
+    B, G, KB, L = 1, 8, 2, 4096
+    ld = (G * KB + 1) * 128
+    idx = torch.full((B, ld), -1, dtype=torch.int32)
+    gm = torch.zeros((B, ld), dtype=torch.uint8)
+    # two whole blocks for every group, the second one with its tokens reversed (still in [0, L))
+    idx[0, :128] = torch.arange(256, 384, dtype=torch.int32)
+    idx[0, 128:256] = torch.arange(1023, 895, -1, dtype=torch.int32)
+    gm[0, :256] = 0xFF
+    cnt = torch.tensor([256], dtype=torch.int32)
+    kv = S.normal_bf16(S.ST_KV, (L, 576), DEV)
+    q = S.normal_bf16(S.ST_Q, (B, 128, 576), DEV)
+    out = torch.empty(B, 128, 512, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(B, 128, device=DEV)
+    lsa.lsa_device_status()  # clean start
+    lsa.lsa_msa_attn(q, kv, idx.to(DEV), gm.to(DEV), cnt.to(DEV), G, 1 / math.sqrt(576), out, lse,
+                     lsa.workspace(lsa.lsa_msa_attn_workspace_size(B, ld, G)))
+    with pytest.raises(lsa.LsaError) as e:
+        lsa.lsa_device_status()
+    assert e.value.status == LSA_ERR_DEVICE_CHECK
+    assert b"k_msa_attn_rows" in lsa.load_library().lsa_last_error()
+    lsa.lsa_device_status()  # the flag was cleared
