@@ -513,150 +513,161 @@ def _stage(ms, nbytes, flops=None, peak_tflops=None, pipe="tensor"):
     return d
 
 
-def long_context_configs(device, l2_flush, iters: int = 10):
+def long_context_configs(device, l2_flush, iters: int = 10, only=None):
     """Per-stage times of the long-context workloads (one GPU, inputs resident, L2 flushed before each pass):
     1M-token decode with the FP8 token path, 1M-token decode with micro-block selection, and the 10M-token
     Flat bucket workload.  Each stage's fraction is against the measured HBM copy peak (and, for the indexer,
     the FP8 tensor peak = measured bf16 x 2)."""
     res = {}
     bf16 = peaks()[0]["bf16_tflops"]
-    # 1M tokens, FP8 scan -> top-2K -> exact bf16 re-rank -> attention
-    wl = S.WORKLOADS["decode1m"]
-    step = DecodeStep(wl, "fp8", device)
-    st = _time_stages([step.index, step.topk, step.attn], l2_flush, iters)
-    rows = float(step.cnt.sum().item())
-    B, L = wl.B, wl.L
-    ix_bytes = L * wl.d_I + L * 4 + B * L * 4 + B * wl.H_I * wl.d_I + B * wl.H_I * 8
-    ix_flops = 2.0 * B * wl.H_I * wl.d_I * L
-    tk_bytes = B * L * 4 + B * 2 * wl.K * (wl.d_I * 2 + 4) + B * step.kmax * 4
-    at_bytes = rows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
-    res["decode1m_fp8"] = {
-        "workload": "B=4 decode queries, L=1048576, e4m3 indexer (H_I=64, d_I=128), top-4096 + exact bf16 re-rank "
-                    "to K=2048, sink 4 + window 128, H=128",
-        "stages": {"index": _stage(st[0], ix_bytes, ix_flops, fp8_peak()[0]), "topk_rerank": _stage(st[1], tk_bytes),
-                   "attn": _stage(st[2], at_bytes)},
-        "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
-    del step
-    torch.cuda.empty_cache()
-    # 1M tokens, hierarchical selection (bf16) against the flat bf16 indexer + top-K on the same keys
-    wl = S.WORKLOADS["decode1m"]
-    hstep = HiStep(wl, device)
-    st = _time_stages([hstep.hi, hstep.attn, hstep.flat], l2_flush, iters)
-    B, L = wl.B, wl.L
-    recalled = HiStep.M * HiStep.P
-    sub_flops = 3 * 2.0 * B * wl.H_I * wl.d_I * (L // HiStep.BSUB)
-    tok_flops = 2.0 * B * wl.H_I * wl.d_I * recalled
-    hi_bytes = (L // HiStep.BSUB) * wl.d_I * 6 + B * recalled * (wl.d_I * 2 + 8)
-    hrows = float(hstep.cnt.sum().item())
-    h_at_bytes = hrows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
-    res["decode1m_hi"] = {
-        "workload": "B=4 decode queries, L=1048576, bf16 indexer keys; pages of 128 tokens, 8-token sub-block means "
-                    "(cached bf16 split), top-1024 pages (131072 recalled tokens), exact token top-2048 on them, "
-                    "sink 4 + window 128, H=128",
-        "stages": {"hi_select": _stage(st[0], hi_bytes, sub_flops + tok_flops, bf16), "attn": _stage(st[1], h_at_bytes)},
-        "flat_select_ms": round(float(st[2]), 5),
-        "ms": round(float(st[0] + st[1]), 5), "queries_per_s": round(B / (float(st[0] + st[1]) * 1e-3), 1)}
-    del hstep
-    torch.cuda.empty_cache()
-    # the pages' fixed / dynamic split (sink 16 + window 1024 + 1024 sparse) at 128K: the attention as one
-    # gather pass over the row and as the hybrid operator (contiguous part on a second stream, LSE merge)
-    wl = S.Workload("decode128k_si", L=131072, B=16, H_I=64, d_I=128, K=1024, H=128, sink=16, window=1024,
-                    needles="cos06", n_needles=1310)
-    step = DecodeStep(wl, "bf16", device)
-    step.index()
-    step.topk()
-    ws_h = step.lsa.workspace(step.lsa.lsa_workspace_size(step.lsa.LSA_OP_HYBRID_ATTN, wl.B, wl.L, step.kmax, wl.H,
-                                                          wl.sink, wl.window), device)
 
-    def hybrid():
-        step.lsa.lsa_hybrid_attn(step.q, step.kv, step.idx, step.cnt, wl.sink, wl.window, step.q_pos, wl.scale,
-                                 step.out, step.lse, ws_h)
+    def want(name):  # --only: a comma-separated subset of the workloads (a short run, e.g. to profile one kernel)
+        return only is None or name in only
 
-    st = _time_stages([step.attn, hybrid], l2_flush, iters)
-    rows = float(step.cnt.sum().item())
-    at_bytes = rows * (wl.d_qk * 2 + 4) + wl.B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
-    res["decode128k_hfa"] = {
-        "workload": "B=16 decode queries, L=131072, sink 16 + window 1024 + top-1024 sparse (the pages' 1:1 fixed / "
-                    "dynamic budget), H=128",
-        "stages": {"attn_single_pass": _stage(st[0], at_bytes), "attn_hybrid": _stage(st[1], at_bytes)}}
-    del step, ws_h
-    torch.cuda.empty_cache()
-    # group-wise block selection at 128K: 8 groups, each its top-16 blocks of 128 (2048 tokens per group) + the
-    # local block; the attention stage reads each group's rows for its 16 query heads
-    wl = S.WORKLOADS["decode128k"]
-    mstep = MsaStep(wl, device, G=8, KB=16)
-    st = _time_stages([mstep.select, mstep.attn], l2_flush, iters)
-    B, L = wl.B, wl.L
-    nblk = L // 128
-    sel_bytes = L * wl.d_I * 2 + B * 8 * nblk * 4 + B * mstep.idx.shape[1] * 5
-    sel_flops = 2.0 * B * wl.H_I * wl.d_I * L
-    rows = float(mstep.cnt.sum().item())
-    gm = mstep.gmask.cpu().numpy()
-    grp_rows = float(sum(int(((gm[b, : int(c)] >> g) & 1).sum()) for b, c in enumerate(mstep.cnt.cpu().tolist())
-                         for g in range(8)))
-    at_bytes = rows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
-    res["decode128k_msa"] = {
-        "workload": "B=16 decode queries, L=131072, bf16 indexer (H_I=64 as 8 groups of 8 heads), top-16 blocks of "
-                    "128 per group + the local block, H=128 (8 groups of 16 query heads)",
-        "stages": {"msa_select": _stage(st[0], sel_bytes, sel_flops, bf16), "attn": _stage(st[1], at_bytes)},
-        "union_rows_per_query": round(rows / B, 1), "group_rows_per_query": round(grp_rows / B, 1),
-        "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
-    del mstep
-    torch.cuda.empty_cache()
-    for name in ("decode1m_mb", "flat10m"):
-        wl = S.WORKLOADS[name]
-        bstep = BucketStep(wl, device)
-        st = _time_stages([bstep.select, bstep.attn], l2_flush, iters)
-        B = wl.B
-        rows = float(bstep.cnt.sum().item())
-        sel_bytes = bstep.nb * wl.d_I * 6 + B * bstep.nb * 4 + B * wl.kmax * 4 + \
-            (B * wl.M * wl.bsz * 4 if wl.mode == "flat" else 0)
-        sel_flops = 2.0 * B * wl.H_I * wl.d_I * bstep.nb
+    if want("decode1m_fp8"):
+        # 1M tokens, FP8 scan -> top-2K -> exact bf16 re-rank -> attention
+        wl = S.WORKLOADS["decode1m"]
+        step = DecodeStep(wl, "fp8", device)
+        st = _time_stages([step.index, step.topk, step.attn], l2_flush, iters)
+        rows = float(step.cnt.sum().item())
+        B, L = wl.B, wl.L
+        ix_bytes = L * wl.d_I + L * 4 + B * L * 4 + B * wl.H_I * wl.d_I + B * wl.H_I * 8
+        ix_flops = 2.0 * B * wl.H_I * wl.d_I * L
+        tk_bytes = B * L * 4 + B * 2 * wl.K * (wl.d_I * 2 + 4) + B * step.kmax * 4
         at_bytes = rows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
-        desc = ("B=4 decode queries, L=1048576, 4-token mean-pooled blocks (fp32, scored from their cached exact "
-                "3 x bf16 split on tensor cores), top-512 blocks + tail + sink 4 + window 128, H=128"
-                if name == "decode1m_mb" else
-                "B=8 decode queries, L=10000000, 156250 Flat buckets of 64 (fp32 representatives scored from their "
-                "cached exact 3 x bf16 split on tensor cores), top-32 buckets + sink 4 + window 512, H=128, "
-                "11.5 GB latent cache")
-        res[name] = {"workload": desc,
-                     "stages": {"bucket_select": _stage(st[0], sel_bytes, 3 * sel_flops, bf16),
-                                "attn": _stage(st[1], at_bytes)},
-                     "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
-        if name == "flat10m":
-            # the Tree form over the same buckets: parents of 64 consecutive buckets, top-64 parents, then the
-            # top-32 of their 4096 children; timed beside Flat, with the share of Flat's positions it keeps
-            F, M2 = 64, 64
-            lsa_ = bstep.lsa
-            NP = -(-bstep.nb // F)
-            par = torch.empty(NP, wl.d_I, device=device)
-            lsa_.lsa_tree_parents(bstep.cen, F, par)
-            t_idx, t_cnt = torch.empty_like(bstep.idx), torch.empty_like(bstep.cnt)
-            ws_t = lsa_.workspace(lsa_.lsa_tree_workspace_size(B, NP, F, M2, wl.M), device)
-
-            def tree():  # children from the cached split of the centres, on the tensor cores
-                lsa_.lsa_tree_select_split(bstep.q_I, bstep.w, bstep.split, par, F, bstep.members, M2, wl.M, wl.sink,
-                                           wl.window, wl.L, bstep.q_pos, t_idx, t_cnt, ws_t)
-
-            st_t = _time_stages([tree], l2_flush, iters)
-            bstep.select()
-            tree()
-            torch.cuda.synchronize()
-            fi, fc, ti, tc = bstep.idx.cpu(), bstep.cnt.cpu(), t_idx.cpu(), t_cnt.cpu()
-            kept = [len(np.intersect1d(fi[b, : fc[b]].numpy(), ti[b, : tc[b]].numpy())) / max(int(fc[b]), 1)
-                    for b in range(B)]
-            t_bytes = NP * wl.d_I * 4 + B * M2 * F * (wl.d_I * 4 + 8) + B * wl.kmax * 4
-            t_flops = 2.0 * B * wl.H_I * wl.d_I * (NP + M2 * F)
-            res["flat10m_tree"] = {
-                "workload": "flat10m's buckets as a two-level tree: 2442 parents of 64 consecutive buckets (mean "
-                            "centres), top-64 parents, top-32 of their 4096 children (scored on the tensor cores "
-                            "from the centres' cached bf16 split), + sink 4 + window 512",
-                "stages": {"tree_select": _stage(st_t[0], t_bytes)}, "tree_select_flops": t_flops,
-                "flat_select_ms": round(float(st[0]), 5),
-                "share_of_flat_positions_kept": round(float(np.mean(kept)), 4)}
-            del par, t_idx, t_cnt, ws_t
-        del bstep
+        res["decode1m_fp8"] = {
+            "workload": "B=4 decode queries, L=1048576, e4m3 indexer (H_I=64, d_I=128), top-4096 + exact bf16 re-rank "
+                        "to K=2048, sink 4 + window 128, H=128",
+            "stages": {"index": _stage(st[0], ix_bytes, ix_flops, fp8_peak()[0]), "topk_rerank": _stage(st[1], tk_bytes),
+                       "attn": _stage(st[2], at_bytes)},
+            "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
+        del step
         torch.cuda.empty_cache()
+    if want("decode1m_hi"):
+        # 1M tokens, hierarchical selection (bf16) against the flat bf16 indexer + top-K on the same keys
+        wl = S.WORKLOADS["decode1m"]
+        hstep = HiStep(wl, device)
+        st = _time_stages([hstep.hi, hstep.attn, hstep.flat], l2_flush, iters)
+        B, L = wl.B, wl.L
+        recalled = HiStep.M * HiStep.P
+        sub_flops = 3 * 2.0 * B * wl.H_I * wl.d_I * (L // HiStep.BSUB)
+        tok_flops = 2.0 * B * wl.H_I * wl.d_I * recalled
+        hi_bytes = (L // HiStep.BSUB) * wl.d_I * 6 + B * recalled * (wl.d_I * 2 + 8)
+        hrows = float(hstep.cnt.sum().item())
+        h_at_bytes = hrows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
+        res["decode1m_hi"] = {
+            "workload": "B=4 decode queries, L=1048576, bf16 indexer keys; pages of 128 tokens, 8-token sub-block means "
+                        "(cached bf16 split), top-1024 pages (131072 recalled tokens), exact token top-2048 on them, "
+                        "sink 4 + window 128, H=128",
+            "stages": {"hi_select": _stage(st[0], hi_bytes, sub_flops + tok_flops, bf16), "attn": _stage(st[1], h_at_bytes)},
+            "flat_select_ms": round(float(st[2]), 5),
+            "ms": round(float(st[0] + st[1]), 5), "queries_per_s": round(B / (float(st[0] + st[1]) * 1e-3), 1)}
+        del hstep
+        torch.cuda.empty_cache()
+    if want("decode128k_hfa"):
+        # the pages' fixed / dynamic split (sink 16 + window 1024 + 1024 sparse) at 128K: the attention as one
+        # gather pass over the row and as the hybrid operator (contiguous part on a second stream, LSE merge)
+        wl = S.Workload("decode128k_si", L=131072, B=16, H_I=64, d_I=128, K=1024, H=128, sink=16, window=1024,
+                        needles="cos06", n_needles=1310)
+        step = DecodeStep(wl, "bf16", device)
+        step.index()
+        step.topk()
+        ws_h = step.lsa.workspace(step.lsa.lsa_workspace_size(step.lsa.LSA_OP_HYBRID_ATTN, wl.B, wl.L, step.kmax, wl.H,
+                                                              wl.sink, wl.window), device)
+
+        def hybrid():
+            step.lsa.lsa_hybrid_attn(step.q, step.kv, step.idx, step.cnt, wl.sink, wl.window, step.q_pos, wl.scale,
+                                     step.out, step.lse, ws_h)
+
+        st = _time_stages([step.attn, hybrid], l2_flush, iters)
+        rows = float(step.cnt.sum().item())
+        at_bytes = rows * (wl.d_qk * 2 + 4) + wl.B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
+        res["decode128k_hfa"] = {
+            "workload": "B=16 decode queries, L=131072, sink 16 + window 1024 + top-1024 sparse (the pages' 1:1 fixed / "
+                        "dynamic budget), H=128",
+            "stages": {"attn_single_pass": _stage(st[0], at_bytes), "attn_hybrid": _stage(st[1], at_bytes)}}
+        del step, ws_h
+        torch.cuda.empty_cache()
+    if want("decode128k_msa"):
+        # group-wise block selection at 128K: 8 groups, each its top-16 blocks of 128 (2048 tokens per group) + the
+        # local block; the attention stage reads each group's rows for its 16 query heads
+        wl = S.WORKLOADS["decode128k"]
+        mstep = MsaStep(wl, device, G=8, KB=16)
+        st = _time_stages([mstep.select, mstep.attn], l2_flush, iters)
+        B, L = wl.B, wl.L
+        nblk = L // 128
+        sel_bytes = L * wl.d_I * 2 + B * 8 * nblk * 4 + B * mstep.idx.shape[1] * 5
+        sel_flops = 2.0 * B * wl.H_I * wl.d_I * L
+        rows = float(mstep.cnt.sum().item())
+        gm = mstep.gmask.cpu().numpy()
+        grp_rows = float(sum(int(((gm[b, : int(c)] >> g) & 1).sum()) for b, c in enumerate(mstep.cnt.cpu().tolist())
+                             for g in range(8)))
+        at_bytes = rows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
+        res["decode128k_msa"] = {
+            "workload": "B=16 decode queries, L=131072, bf16 indexer (H_I=64 as 8 groups of 8 heads), top-16 blocks of "
+                        "128 per group + the local block, H=128 (8 groups of 16 query heads)",
+            "stages": {"msa_select": _stage(st[0], sel_bytes, sel_flops, bf16), "attn": _stage(st[1], at_bytes)},
+            "union_rows_per_query": round(rows / B, 1), "group_rows_per_query": round(grp_rows / B, 1),
+            "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
+        del mstep
+        torch.cuda.empty_cache()
+    if want("decode1m_mb") or want("flat10m") or want("flat10m_tree"):
+        for name in ("decode1m_mb", "flat10m"):
+            if not (want(name) or (name == "flat10m" and want("flat10m_tree"))):
+                continue
+            wl = S.WORKLOADS[name]
+            bstep = BucketStep(wl, device)
+            st = _time_stages([bstep.select, bstep.attn], l2_flush, iters)
+            B = wl.B
+            rows = float(bstep.cnt.sum().item())
+            sel_bytes = bstep.nb * wl.d_I * 6 + B * bstep.nb * 4 + B * wl.kmax * 4 + \
+                (B * wl.M * wl.bsz * 4 if wl.mode == "flat" else 0)
+            sel_flops = 2.0 * B * wl.H_I * wl.d_I * bstep.nb
+            at_bytes = rows * (wl.d_qk * 2 + 4) + B * wl.H * (wl.d_qk * 2 + wl.d_v * 2 + 4)
+            desc = ("B=4 decode queries, L=1048576, 4-token mean-pooled blocks (fp32, scored from their cached exact "
+                    "3 x bf16 split on tensor cores), top-512 blocks + tail + sink 4 + window 128, H=128"
+                    if name == "decode1m_mb" else
+                    "B=8 decode queries, L=10000000, 156250 Flat buckets of 64 (fp32 representatives scored from their "
+                    "cached exact 3 x bf16 split on tensor cores), top-32 buckets + sink 4 + window 512, H=128, "
+                    "11.5 GB latent cache")
+            res[name] = {"workload": desc,
+                         "stages": {"bucket_select": _stage(st[0], sel_bytes, 3 * sel_flops, bf16),
+                                    "attn": _stage(st[1], at_bytes)},
+                         "ms": round(float(st.sum()), 5), "queries_per_s": round(B / (float(st.sum()) * 1e-3), 1)}
+            if name == "flat10m":
+                # the Tree form over the same buckets: parents of 64 consecutive buckets, top-64 parents, then the
+                # top-32 of their 4096 children; timed beside Flat, with the share of Flat's positions it keeps
+                F, M2 = 64, 64
+                lsa_ = bstep.lsa
+                NP = -(-bstep.nb // F)
+                par = torch.empty(NP, wl.d_I, device=device)
+                lsa_.lsa_tree_parents(bstep.cen, F, par)
+                t_idx, t_cnt = torch.empty_like(bstep.idx), torch.empty_like(bstep.cnt)
+                ws_t = lsa_.workspace(lsa_.lsa_tree_workspace_size(B, NP, F, M2, wl.M), device)
+
+                def tree():  # children from the cached split of the centres, on the tensor cores
+                    lsa_.lsa_tree_select_split(bstep.q_I, bstep.w, bstep.split, par, F, bstep.members, M2, wl.M, wl.sink,
+                                               wl.window, wl.L, bstep.q_pos, t_idx, t_cnt, ws_t)
+
+                st_t = _time_stages([tree], l2_flush, iters)
+                bstep.select()
+                tree()
+                torch.cuda.synchronize()
+                fi, fc, ti, tc = bstep.idx.cpu(), bstep.cnt.cpu(), t_idx.cpu(), t_cnt.cpu()
+                kept = [len(np.intersect1d(fi[b, : fc[b]].numpy(), ti[b, : tc[b]].numpy())) / max(int(fc[b]), 1)
+                        for b in range(B)]
+                t_bytes = NP * wl.d_I * 4 + B * M2 * F * (wl.d_I * 4 + 8) + B * wl.kmax * 4
+                t_flops = 2.0 * B * wl.H_I * wl.d_I * (NP + M2 * F)
+                res["flat10m_tree"] = {
+                    "workload": "flat10m's buckets as a two-level tree: 2442 parents of 64 consecutive buckets (mean "
+                                "centres), top-64 parents, top-32 of their 4096 children (scored on the tensor cores "
+                                "from the centres' cached bf16 split), + sink 4 + window 512",
+                    "stages": {"tree_select": _stage(st_t[0], t_bytes)}, "tree_select_flops": t_flops,
+                    "flat_select_ms": round(float(st[0]), 5),
+                    "share_of_flat_positions_kept": round(float(np.mean(kept)), 4)}
+                del par, t_idx, t_cnt, ws_t
+            del bstep
+            torch.cuda.empty_cache()
     return res
 
 
@@ -808,7 +819,8 @@ def run_gpu(args, rank, world, local_rank):
         return None
     prefill = None if (args.no_prefill or world > 1) else prefill_chunk(device, l2_flush)
     fp8_line = None if (args.no_configs or world > 1 or step.fp8) else fp8_decode(device, l2_flush, step)
-    long_ctx = None if (args.no_configs or world > 1) else long_context_configs(device, l2_flush)
+    only = set(args.only.split(",")) if args.only else None
+    long_ctx = None if (args.no_configs or world > 1) else long_context_configs(device, l2_flush, only=only)
 
     pk, pk_src = peaks()
     work = algorithmic_work(wl, counts, step.fp8)
@@ -1041,6 +1053,9 @@ def main():
     ap.add_argument("--index", default="bf16", choices=["bf16", "fp8"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-chunk latency measurement")
+    ap.add_argument("--only", default=None,
+                    help="long-context workloads to run, comma-separated (decode1m_fp8, decode1m_hi, decode128k_hfa, "
+                         "decode128k_msa, decode1m_mb, flat10m, flat10m_tree); default all")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the long-context workloads (1M-token FP8 / micro-block decode, 10M-token Flat)")
     ap.add_argument("--measure-tensor-peaks", action="store_true",

@@ -140,10 +140,10 @@ __global__ void __launch_bounds__(MA_THREADS, 1)
   float* fin = red + 2 * 4 * MA_NH;                      // [16] final sums
   uint64_t* bars = reinterpret_cast<uint64_t*>(fin + MA_NH);
   uint64_t* q_full = bars;
-  uint64_t* lr_full = q_full + 1;         // [6]
-  uint64_t* lr_empty = lr_full + MA_LR;   // [6]
-  uint64_t* vr_full = lr_empty + MA_LR;   // [2]
-  uint64_t* vr_empty = vr_full + MA_VR;   // [2]
+  uint64_t* lr_full = q_full + 1;         // [MA_LR]
+  uint64_t* lr_empty = lr_full + MA_LR;   // [MA_LR]
+  uint64_t* vr_full = lr_empty + MA_LR;   // [MA_VR]
+  uint64_t* vr_empty = vr_full + MA_VR;   // [MA_VR]
   uint64_t* s_full = vr_empty + MA_VR;    // [2]
   uint64_t* s_empty = s_full + 2;         // [2] (4 softmax warps)
   uint64_t* p_full = s_empty + 2;         // [2] (4 softmax warps)
