@@ -319,17 +319,16 @@ size_t lsa_msa_workspace_size(int64_t B, int64_t L, int G, int KB);
  * lsa_msa_attn -- attention over a group-wise selection: each head attends to its own group's rows.
  *   Source: the same section (a group's query heads share its blocks).
  *   out[b,h] / lse[b,h] = lsa_sparse_attn's attention of head h (group g = h / (128 / G)) over the entries of
- *   idx[b, :count[b]] whose gmask has bit g.  G = 8 (16 heads per group): one CTA per (query, group) reads the
- *   union row's blocks whose mask has bit g and runs each 128-token block with its rows on the MMA's M side (the
- *   16 heads on N), no scratch; this needs idx / gmask as lsa_msa_select writes them (whole 128-token blocks, then
- *   the partial local block) and reports LSA_ERR_DEVICE_CHECK (lsa_device_status) for a block whose entries are not
- *   consecutive tokens.  G = 1, 2, 4: each group's rows are compacted (k_msa_group_rows) and each (query, group)
- *   pair runs the tensor-core attention as one 128-head query whose first 128 / G rows are the group's heads and
- *   whose other rows are zero (outputs dropped).
+ *   idx[b, :count[b]] whose gmask has bit g.  G = 2, 4, 8: one CTA per (query, 16-head slice of one group) reads
+ *   the union row's blocks whose mask has bit g and runs each 128-token block with its rows on the MMA's M side (the
+ *   slice's 16 heads on N), no scratch; this needs idx / gmask as lsa_msa_select writes them (whole 128-token
+ *   blocks, then the partial local block) and reports LSA_ERR_DEVICE_CHECK (lsa_device_status) for a block whose
+ *   entries are not consecutive tokens.  G = 1 (every head shares the union): the rows are compacted
+ *   (k_msa_group_rows) and run through the 128-head tensor-core attention.
  *   q [B, 128, 576] bf16, kv [L, 576] bf16 (value = first 512 dims), idx / gmask / count as lsa_msa_select
  *   writes them (idx_ld <= 65536), out [B, 128, 512] bf16, lse [B, 128] fp32 or NULL; all 16-byte aligned.
  *   H = 128, d_qk = 576, d_v = 512, G in {1, 2, 4, 8}, B*G <= 65535.
- *   ws: lsa_msa_attn_workspace_size(B, idx_ld, G) bytes (0 for G = 8: ws may be NULL).
+ *   ws: lsa_msa_attn_workspace_size(B, idx_ld, G) bytes (0 for G = 2, 4, 8: ws may be NULL).
  */
 int lsa_msa_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, const uint8_t* gmask,
                  int64_t idx_ld, const int32_t* count, int64_t B, int H, int d_qk, int d_v, int G,

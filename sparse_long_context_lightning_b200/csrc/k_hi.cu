@@ -227,41 +227,6 @@ __global__ void __launch_bounds__(GR_THREADS) k_msa_group_rows(const int32_t* __
   if (tid == 0) gcount[bg] = static_cast<int32_t>(base);
 }
 
-// Per-group attention queries: qg[b G + g] is a 128-head query whose rows h < 128 / G are head g 128 / G + h
-// of q[b] and whose other rows are 0 (their outputs are dropped).  16-byte units: a 576-wide bf16 row is 72.
-__global__ void k_msa_pad_q(const uint4* __restrict__ q, int G, int64_t n_bg, uint4* __restrict__ qg) {
-  const int64_t total = n_bg * 128 * 72;
-  const int hg = 128 / G;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / 72;
-    const int c = static_cast<int>(i % 72);
-    const int64_t bg = r / 128;
-    const int h = static_cast<int>(r % 128);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (h < hg) v = q[((bg / G) * 128 + (bg % G) * hg + h) * 72 + c];
-    qg[i] = v;
-  }
-}
-
-// The real rows back: out[b, h] = outg[b G + h / (128 / G), h mod (128 / G)] (512-wide bf16 rows: 64 units),
-// lse likewise when given.
-__global__ void k_msa_unpad(const uint4* __restrict__ outg, const float* __restrict__ lseg, int G, int64_t B,
-                            uint4* __restrict__ out, float* __restrict__ lse) {
-  const int64_t total = B * 128 * 64;
-  const int hg = 128 / G;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / 64;
-    const int c = static_cast<int>(i % 64);
-    const int64_t b = r / 128;
-    const int h = static_cast<int>(r % 128);
-    const int64_t src = (b * G + h / hg) * 128 + h % hg;
-    out[i] = outg[src * 64 + c];
-    if (lse != nullptr && c == 0) lse[r] = lseg[src];
-  }
-}
-
 }  // namespace
 
 int launch_page_sum(const float* sub, int64_t sub_ld, int64_t nsub, int P, int Bsub, int64_t npages, int64_t B,
@@ -303,20 +268,6 @@ int launch_msa_group_rows(const int32_t* idx, const uint8_t* gmask, int64_t idx_
                           int G, int32_t* grows, int32_t* gcount, cudaStream_t s) {
   if (B == 0) return LSA_OK;
   k_msa_group_rows<<<static_cast<unsigned>(B * G), GR_THREADS, 0, s>>>(idx, gmask, idx_ld, count, G, grows, gcount);
-  return cuda_status(cudaGetLastError());
-}
-
-int launch_msa_pad_q(const void* q, int G, int64_t B, void* qg, cudaStream_t s) {
-  if (B == 0) return LSA_OK;
-  k_msa_pad_q<<<static_cast<unsigned>(sm_count() * 4), 256, 0, s>>>(static_cast<const uint4*>(q), G, B * G,
-                                                                    static_cast<uint4*>(qg));
-  return cuda_status(cudaGetLastError());
-}
-
-int launch_msa_unpad(const void* outg, const float* lseg, int G, int64_t B, void* out, float* lse, cudaStream_t s) {
-  if (B == 0) return LSA_OK;
-  k_msa_unpad<<<static_cast<unsigned>(sm_count() * 4), 256, 0, s>>>(static_cast<const uint4*>(outg), lseg, G, B,
-                                                                    static_cast<uint4*>(out), lse);
   return cuda_status(cudaGetLastError());
 }
 

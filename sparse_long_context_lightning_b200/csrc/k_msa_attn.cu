@@ -4,13 +4,13 @@
 // the 128-token blocks their group kept (plus the local block); "LongCat Sparse Attention（LSA）完全拆解",
 // section "DSA 基线": the attention itself is absorbed MQA over 576-dim bf16 latent rows, value = the first 512.
 //
-// B200 design.  A group has 16 query heads (8 groups of the 128), so heads are too few for the MMA's M side; the
-// rows are: S^T = C Q_g^T takes 128 consecutive rows (one kept block) on M, the 16 heads on N and the 576 dims
-// in 36 K steps; O^T += V^T P^T takes 128 value dims on M (two 64-dim blocks), the heads on N and the block's 128
-// rows in 8 K steps.  Both run at the MMA's fixed cost per instruction for N = 16, and a block is one TMA box per
+// B200 design.  A CTA serves 16 query heads of one query (a group of 8, or a 16-head slice of a group of 2 or 4),
+// too few for the MMA's M side; the rows are: S^T = C Q_g^T takes 128 consecutive rows (one kept block) on M, the
+// 16 heads on N and the 576 dims in 36 K steps; O^T += V^T P^T takes 128 value dims on M (two 64-dim blocks),
+// the heads on N and the block's 128 rows in 8 K steps.  Both run at the MMA's fixed cost per instruction for N = 16, and a block is one TMA box per
 // 64-dim slice (its rows are consecutive tokens), so there is no per-row gather.  The value slices are loaded a
 // second time for O^T (from L2, a few microseconds after the first read): shared memory holds a ring of slices,
-// not whole blocks.  One CTA per (query, group); no partials, no combine.
+// not whole blocks.  One CTA per (query, 16-head slice), over the blocks its group kept; no partials, no combine.
 //
 // Warp roles (256 threads): warp 0 loads the logits slices (and Q_g), warp 1 the value-slice pairs, warp 2 owns
 // TMEM and issues S^T, warp 3 issues O^T, warps 4-7 run the softmax (thread = row = TMEM lane) and write the
@@ -157,8 +157,8 @@ __global__ void __launch_bounds__(MA_THREADS, 1)
   int* trows = tfirst + MA_MAXT;                                                // [512] and its number of rows
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bg = blockIdx.x;  // query b = bg / G, group g = bg % G
-  const int b = bg / a.G, g = bg % a.G;
+  const int bg = blockIdx.x;  // query b = bg / 8, heads 16 hs .. 16 hs + 15 (hs = bg % 8) of group hs G / 8
+  const int b = bg / 8, hs = bg % 8, g = hs * a.G / 8;
   const int32_t* ridx = a.idx + static_cast<int64_t>(b) * a.ld;
   if (tid == 0) {
     mbar_init(q_full, 1);
@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(MA_THREADS, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_kv);
     mbar_expect_tx(q_full, MA_KB * MA_QSLICE);
-    for (int kb = 0; kb < MA_KB; ++kb) tma_load_2d(qs + kb * 2048, &tm_q, q_full, 64 * kb, b * 128 + g * MA_NH);
+    for (int kb = 0; kb < MA_KB; ++kb) tma_load_2d(qs + kb * 2048, &tm_q, q_full, 64 * kb, b * 128 + hs * MA_NH);
   }
   if (warp == 2) {
     tmem_alloc(tmem_holder, 128);
@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(MA_THREADS, 1)
       const float l = rd2[h] + rd2[MA_NH + h] + rd2[2 * MA_NH + h] + rd2[3 * MA_NH + h];
       inv[h] = (have && l > 0.f) ? 1.f / l : 0.f;
       if (a.lse && r == h) {
-        a.lse[static_cast<int64_t>(b) * 128 + g * MA_NH + h] =
+        a.lse[static_cast<int64_t>(b) * 128 + hs * MA_NH + h] =
             (have && l > 0.f) ? (m_used[h] + log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
     }
@@ -497,7 +497,7 @@ __global__ void __launch_bounds__(MA_THREADS, 1)
     for (int i = 0; i < (MA_NH * 512 * 2 / 16) / 128; ++i) {
       const int e = i * 128 + r;  // 16-byte piece e of the 16 KB
       const int h = e / 64, c = e % 64;
-      *reinterpret_cast<uint4*>(a.out + (static_cast<int64_t>(b) * 128 + g * MA_NH + h) * 512 + 8 * c) =
+      *reinterpret_cast<uint4*>(a.out + (static_cast<int64_t>(b) * 128 + hs * MA_NH + h) * 512 + 8 * c) =
           reinterpret_cast<const uint4*>(stage)[e];
     }
   }
@@ -513,11 +513,11 @@ __global__ void __launch_bounds__(MA_THREADS, 1)
 
 int make_map(CUtensorMap* m, const void* ptr, bool fp8, int64_t rows, int64_t cols, int box_cols, int box_rows);
 
-// MSA attention with 16 heads per group (128 query heads in 8 groups): one CTA per (query, group) over the union
-// row's blocks that the group kept.
+// MSA attention, 128 query heads in G = 2, 4 or 8 groups: one CTA per (query, 16-head slice) over the union row's
+// blocks that the slice's group kept.
 int launch_msa_attn_rows(const void* q, const void* kv, int64_t L, const int32_t* idx, const uint8_t* gmask, int64_t ld,
                          const int32_t* count, int64_t B, int G, float scale, void* out, float* lse, cudaStream_t s) {
-  if (128 / G != MA_NH || ld > static_cast<int64_t>(MA_MAXT) * MA_ROWS) return LSA_ERR_UNSUPPORTED;
+  if ((G != 2 && G != 4 && G != 8) || ld > static_cast<int64_t>(MA_MAXT) * MA_ROWS) return LSA_ERR_UNSUPPORTED;
   CUtensorMap tkv, tq;
   int st = make_map(&tkv, kv, false, L, 576, 64, MA_ROWS);
   if (st) return st;
@@ -534,7 +534,7 @@ int launch_msa_attn_rows(const void* q, const void* kv, int64_t L, const int32_t
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
   LSA_CUDA_TRY(func_smem_once(reinterpret_cast<const void*>(k_msa_attn_rows), MA_SMEM));
-  LSA_CUDA_TRY(launch_pdl(k_msa_attn_rows, dim3(static_cast<unsigned>(B * G)), dim3(MA_THREADS), MA_SMEM, s, 0u, tkv,
+  LSA_CUDA_TRY(launch_pdl(k_msa_attn_rows, dim3(static_cast<unsigned>(B * 8)), dim3(MA_THREADS), MA_SMEM, s, 0u, tkv,
                           tq, a));
   return LSA_OK;
 }

@@ -532,29 +532,20 @@ int lsa_tree_select_split(const void* q_idx, const float* w, int64_t B, int H_I,
                           window, L, q_pos, idx, idx_ld, count, ws, ws_bytes, stream);
 }
 
+// Scratch of lsa_msa_attn: G = 1 compacts the rows (all of the union, the one group's) and runs the 128-head
+// attention on them: rows [B, idx_ld] | counts [B] | the attention's scratch.  G = 2, 4, 8 need none.
 struct MsaAttnLayout {
-  size_t o_cnt, o_q, o_out, o_lse, o_att, total;
+  size_t o_cnt, o_att, total;
 };
 static MsaAttnLayout msa_attn_layout(int64_t B, int64_t idx_ld, int G) {
   MsaAttnLayout m;
-  const size_t bg = static_cast<size_t>(B) * G;
-  m.o_cnt = align_up(bg * idx_ld * 4, 256);
-  size_t o = m.o_cnt + align_up(bg * 4, 256);
-  m.o_q = m.o_out = m.o_lse = o;
-  if (G == 8) {  // 16 heads per group: the rows-on-M kernel reads the union row and its masks directly
-    m.o_cnt = m.o_q = m.o_out = m.o_lse = m.o_att = m.total = 0;
+  if (G > 1) {
+    m.o_cnt = m.o_att = m.total = 0;
     return m;
   }
-  if (G > 1) {  // the padded 128-head queries, their outputs and lse
-    m.o_q = o;
-    o += align_up(bg * 128 * 576 * 2, 256);
-    m.o_out = o;
-    o += align_up(bg * 128 * 512 * 2, 256);
-    m.o_lse = o;
-    o += align_up(bg * 128 * 4, 256);
-  }
-  m.o_att = o;
-  m.total = o + sparse_attn_ws_bytes(static_cast<int64_t>(bg), idx_ld, 128);
+  m.o_cnt = align_up(static_cast<size_t>(B) * idx_ld * 4, 256);
+  m.o_att = m.o_cnt + align_up(static_cast<size_t>(B) * 4, 256);
+  m.total = m.o_att + sparse_attn_ws_bytes(B, idx_ld, 128);
   return m;
 }
 
@@ -574,31 +565,18 @@ int lsa_msa_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, c
   const MsaAttnLayout m = msa_attn_layout(B, idx_ld, G);
   if (m.total > 0 && (ws == nullptr || !aligned256(ws) || ws_bytes < m.total)) return LSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (G == 8) {
-    // 16 heads per group: one CTA per (query, group), each kept 128-token block on the MMA's M side, the group's
-    // blocks read from the union row's masks
+  if (G > 1) {
+    // one CTA per (query, 16-head slice), each block its group kept on the MMA's M side, the group's blocks read
+    // from the union row's masks
     return launch_msa_attn_rows(q, kv, L, idx, gmask, idx_ld, count, B, G, scale, out, lse, s);
   }
+  // G = 1: the rows compacted, then the 128-head tensor-core attention
   unsigned char* base = static_cast<unsigned char*>(ws);
   int32_t* grows = reinterpret_cast<int32_t*>(base);
   int32_t* gcnt = reinterpret_cast<int32_t*>(base + m.o_cnt);
-  // each group's rows; then one 128-head attention per (query, group) on the tensor cores, the group's heads in
-  // the first 128 / G rows of a zero-padded query (G = 1: the query itself)
   int st = launch_msa_group_rows(idx, gmask, idx_ld, count, B, G, grows, gcnt, s);
-  if (G == 1) {
-    if (st == LSA_OK)
-      st = launch_sparse_attn(q, kv, L, grows, idx_ld, gcnt, B, 128, scale, out, lse, base + m.o_att,
-                              ws_bytes - m.o_att, s);
-    return st;
-  }
-  void* qg = base + m.o_q;
-  void* outg = base + m.o_out;
-  float* lseg = reinterpret_cast<float*>(base + m.o_lse);
-  if (st == LSA_OK) st = launch_msa_pad_q(q, G, B, qg, s);
   if (st == LSA_OK)
-    st = launch_sparse_attn(qg, kv, L, grows, idx_ld, gcnt, B * G, 128, scale, outg, lseg, base + m.o_att,
-                            ws_bytes - m.o_att, s);
-  if (st == LSA_OK) st = launch_msa_unpad(outg, lseg, G, B, out, lse, s);
+    st = launch_sparse_attn(q, kv, L, grows, idx_ld, gcnt, B, 128, scale, out, lse, base + m.o_att, ws_bytes - m.o_att, s);
   return st;
 }
 

@@ -185,8 +185,6 @@ int launch_tree_child_score(const void* q, const float* w, int64_t B, int H_I, i
                             float* cscore, int32_t* cid, int64_t ldc, cudaStream_t s);
 int launch_tree_map(const int32_t* kpos, int64_t kpos_ld, const int32_t* kposc, const int32_t* cid, int64_t ldc,
                     int64_t n_cand, int64_t B, int32_t* kept, int64_t kept_ld, int32_t* kcount, cudaStream_t s);
-int launch_msa_pad_q(const void* q, int G, int64_t B, void* qg, cudaStream_t s);
-int launch_msa_unpad(const void* outg, const float* lseg, int G, int64_t B, void* out, float* lse, cudaStream_t s);
 int launch_msa_group_rows(const int32_t* idx, const uint8_t* gmask, int64_t idx_ld, const int32_t* count, int64_t B,
                           int G, int32_t* grows, int32_t* gcount, cudaStream_t s);
 int launch_block_max_tc(const void* q, const float* w, const void* k, int64_t B, int64_t L, int G,

@@ -96,12 +96,12 @@ def test_selection_workspace_sizes(lib):
     # MSA selection: block scores for every (query, group)
     m = lib.lsa_msa_workspace_size(16, 131072, 8, 16)
     assert m % 256 == 0 and m >= 16 * 8 * 1024 * 4
-    # MSA attention: G = 8 reads the union row directly (no scratch); G = 2 and 4 compact per-group rows and pad
-    # the groups' heads into 128-head queries
-    a8 = lib.lsa_msa_attn_workspace_size(16, 129 * 128, 8)
-    a2 = lib.lsa_msa_attn_workspace_size(16, 129 * 128, 2)
-    assert a8 == 0
-    assert a2 >= 16 * 2 * 129 * 128 * 4 + 16 * 2 * 128 * (576 + 512) * 2
+    # MSA attention: G = 2, 4, 8 read the union row directly (no scratch); G = 1 compacts the rows for the
+    # 128-head attention
+    for G in (2, 4, 8):
+        assert lib.lsa_msa_attn_workspace_size(16, 129 * 128, G) == 0
+    a1 = lib.lsa_msa_attn_workspace_size(16, 129 * 128, 1)
+    assert a1 % 256 == 0 and a1 >= 16 * 129 * 128 * 4
     assert lib.lsa_msa_attn_workspace_size(16, 128, 0) == bad
     assert lib.lsa_hi_workspace_size(4, 1 << 20, 128, 8, 1024, 2048, 4, 128) > 0
 
@@ -131,8 +131,8 @@ def test_selection_argument_checks_launch_nothing(lib):
     # MSA attention: G = 3; workspace missing
     assert lib.lsa_msa_attn(fake, fake, 4096, fake, fake, 1024, fake, 1, 128, 576, 512, 3, 1.0, fake, None, fake,
                             1 << 20, None) == -2
-    assert lib.lsa_msa_attn(fake, fake, 4096, fake, fake, 1024, fake, 1, 128, 576, 512, 2, 1.0, fake, None, None, 0,
-                            None) == -3  # G = 2 compacts and pads through the workspace (G = 8 needs none)
+    assert lib.lsa_msa_attn(fake, fake, 4096, fake, fake, 1024, fake, 1, 128, 576, 512, 1, 1.0, fake, None, None, 0,
+                            None) == -3  # G = 1 compacts the rows through the workspace (G = 2, 4, 8 need none)
     # empty batches are a no-op
     assert lib.lsa_tree_select(fake, fake, 0, 64, 128, fake, 1000, fake, 100, 10, fake, 64, 8, 4, 0, 0, 64000, fake,
                                fake, 256, fake, None, 0, None) == 0

@@ -769,11 +769,14 @@ def test_msa_select(G, KB):
                 assert abs(sc - kth) <= 1e-5 * abs(kth), (b, g, blk)
 
 
-@pytest.mark.parametrize("G,KB", [(8, 16), (2, 8), (1, 8)])
-def test_msa_attn(G, KB):
-    """Head h attends to its group's rows only: against the oracle attention per head over those rows."""
-    L, B = 40000 + 77, 3
-    q_pos = [L - 1, 20000, 5000]
+@pytest.mark.parametrize("G,KB,q_pos", [(8, 16, [40076, 20000, 5000]), (2, 8, [40076, 20000, 5000]),
+                                         (4, 5, [40076, 20000, 5000]), (1, 8, [40076, 20000, 5000]),
+                                         (8, 4, [50, 127, 300, 40076]), (2, 3, [50, 127, 300, 40076])])
+def test_msa_attn(G, KB, q_pos):
+    """Head h attends to its group's rows only: against the oracle attention per head over those rows.  The last
+    case has queries whose only block is the partial local one (q_pos 50, 127) and one with fewer kept blocks than
+    KB (q_pos 300)."""
+    L, B = 40000 + 77, len(q_pos)
     _, _, _, _, idx, gm, cnt = _msa_case(L, B, G, KB, q_pos)
     kv = S.normal_bf16(S.ST_KV, (L, 576), DEV)
     q = S.normal_bf16(S.ST_Q, (B, 128, 576), DEV)
