@@ -57,29 +57,17 @@ struct IxArgs {
   int split_rows;  // SPLITS > 1: rows between the key matrices that are summed (the exact bf16 split parts)
 };
 
-// acc0 = sum_c w[c] ReLU(r0[c]), acc1 = sum_c w[32 + c] ReLU(r1[c]).  The 64 weights are the same for every
-// lane (a broadcast): read as 16 float4 so that the epilogue's shared-memory reads (one wavefront per load
-// instruction) stay small next to the tensor cores' operand reads from the same shared memory.
-__device__ __forceinline__ void relu_weighted_sum64(const float* w, const uint32_t (&r0)[32], const uint32_t (&r1)[32],
-                                                    float& acc0, float& acc1) {
-  const float4* w4 = reinterpret_cast<const float4*>(w);
-  acc0 = 0.f;
-  acc1 = 0.f;
+// NP partial sums of w[c] ReLU(D[c]) over the 64 columns of an epilogue thread, partial j over columns
+// [64 j / NP, 64 (j + 1) / NP); r holds columns [16 q, 16 q + 16).  The 64 weights stay in registers for the whole
+// kernel: re-reading them from shared memory every tile (a broadcast load still returns 4 bytes per lane through
+// the shared-memory crossbar) costs about as many shared-memory cycles as the tensor cores' operand reads.
+template <int NP>
+__device__ __forceinline__ void relu_weighted_quarter(const float (&w)[64], const uint32_t (&r)[16], int q,
+                                                      float (&p)[NP]) {
   #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const float4 v = w4[c];
-    acc0 = fmaf(v.x, fmaxf(__uint_as_float(r0[4 * c]), 0.f), acc0);
-    acc0 = fmaf(v.y, fmaxf(__uint_as_float(r0[4 * c + 1]), 0.f), acc0);
-    acc0 = fmaf(v.z, fmaxf(__uint_as_float(r0[4 * c + 2]), 0.f), acc0);
-    acc0 = fmaf(v.w, fmaxf(__uint_as_float(r0[4 * c + 3]), 0.f), acc0);
-  }
-  #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const float4 v = w4[8 + c];
-    acc1 = fmaf(v.x, fmaxf(__uint_as_float(r1[4 * c]), 0.f), acc1);
-    acc1 = fmaf(v.y, fmaxf(__uint_as_float(r1[4 * c + 1]), 0.f), acc1);
-    acc1 = fmaf(v.z, fmaxf(__uint_as_float(r1[4 * c + 2]), 0.f), acc1);
-    acc1 = fmaf(v.w, fmaxf(__uint_as_float(r1[4 * c + 3]), 0.f), acc1);
+  for (int c = 0; c < 16; ++c) {
+    const int col = 16 * q + c;
+    p[col / (64 / NP)] = fmaf(w[col], fmaxf(__uint_as_float(r[c]), 0.f), p[col / (64 / NP)]);
   }
 }
 
@@ -92,23 +80,14 @@ __device__ __forceinline__ float key_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// Grouped block maxima of one tile for one warp (32 keys x the 64 heads of query b): the G group sums of each
-// key, their max over the warp's keys, then over the tile's four lane quarters through shared memory -- the
+// Grouped block maxima of one tile for one warp (32 keys x the 64 heads of query b): given the G group sums v of
+// each key, their max over the warp's keys, then over the tile's four lane quarters through shared memory -- the
 // quarter that contributes last writes the G block scores and clears the slot (its next user is four tiles
 // later, which no warp reaches before every warp has finished this tile).
 template <int G>
-__device__ __forceinline__ void block_max_epilogue(const IxArgs& a, const float* w, const uint32_t (&r0)[32],
-                                                   const uint32_t (&r1)[32], int s, int b, int64_t qpb, int tile,
-                                                   int lane, uint32_t* mx, uint32_t* cnt) {
-  constexpr int GW = 64 / G;  // heads per group
+__device__ __forceinline__ void block_max_epilogue(const IxArgs& a, float (&v)[G], int s, int b, int64_t qpb,
+                                                   int tile, int lane, uint32_t* mx, uint32_t* cnt) {
   constexpr int LG = G == 1 ? 0 : (G == 2 ? 1 : (G == 4 ? 2 : 3));
-  float v[G];
-  #pragma unroll
-  for (int g = 0; g < G; ++g) v[g] = 0.f;
-  #pragma unroll
-  for (int c = 0; c < 32; ++c) v[c / GW] = fmaf(w[c], fmaxf(__uint_as_float(r0[c]), 0.f), v[c / GW]);
-  #pragma unroll
-  for (int c = 0; c < 32; ++c) v[(32 + c) / GW] = fmaf(w[32 + c], fmaxf(__uint_as_float(r1[c]), 0.f), v[(32 + c) / GW]);
   const bool valid = b < a.B && s < a.L && s <= qpb;
   #pragma unroll
   for (int g = 0; g < G; ++g) v[g] = valid ? v[g] : -INFINITY;
@@ -299,6 +278,16 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     const int col0 = (ew >> 2) * 64;
     const int nq = 64 / a.H_I;  // queries in this warp's 64 columns (1 or 2)
     const int64_t qpb = (G > 0 && b0 + (col0 >> 6) < a.B) ? a.q_pos[b0 + (col0 >> 6)] : -1;  // grouped: one query
+    constexpr int NP = G > 2 ? G : 2;  // partial sums per key: one per group, or one per 32 columns
+    float wr[64];
+    #pragma unroll
+    for (int c = 0; c < 64; c += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(wsm + col0 + c);
+      wr[c] = v.x;
+      wr[c + 1] = v.y;
+      wr[c + 2] = v.z;
+      wr[c + 3] = v.w;
+    }
     for (int i = 0; i < n_my; ++i) {
       const int buf = i & 1;
       // decided warp-wide: the TMEM loads below are warp-collective
@@ -309,22 +298,38 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       }
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * IX_CHUNK_N + col0;
-      uint32_t r0[32], r1[32];
-      tmem_ld32(taddr, r0);
-      tmem_ld32(taddr + 32, r1);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);  // the accumulator columns are in registers now
+      // 16 columns at a time (64 weights + 16 columns live; 18 warps leave 96 registers a thread), four or G
+      // partial sums
+      float p[NP];
+      #pragma unroll
+      for (int j = 0; j < NP; ++j) p[j] = 0.f;
+      #pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t r[16];
+        tmem_ld16(taddr + 16 * q, r);
+        tmem_ld_wait();
+        if (q == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);  // the accumulator columns are in registers now
+        }
+        relu_weighted_quarter<NP>(wr, r, q, p);
+      }
       const int s = (t_begin + i) * IX_TILE_M + quarter * 32 + lane;
       if constexpr (G > 0) {
-        block_max_epilogue<G>(a, wsm + col0, r0, r1, s, b0 + (col0 >> 6), qpb, t_begin + i, lane,
+        float v[G > 0 ? G : 1];
+        #pragma unroll
+        for (int g = 0; g < G; ++g) {
+          v[g] = 0.f;
+          #pragma unroll
+          for (int j = g * (NP / G); j < (g + 1) * (NP / G); ++j) v[g] += p[j];
+        }
+        block_max_epilogue<G>(a, v, s, b0 + (col0 >> 6), qpb, t_begin + i, lane,
                               gmax + ((i & 3) * 4 + (ew >> 2)) * 8, gcnt + (i & 3) * 4 + (ew >> 2));
         continue;
       }
       const float ks = (FP8 && s < a.L) ? a.k_scale[s] : 1.f;
-      float acc0, acc1;
-      relu_weighted_sum64(wsm + col0, r0, r1, acc0, acc1);
+      const float acc0 = p[0], acc1 = p[1];
       if (s < a.L) {
         if (nq == 1) {
           const int b = b0 + col0 / a.H_I;

@@ -97,16 +97,6 @@ __device__ __forceinline__ void drain_mmas(uint64_t* bar) {
   (void)mbar_spin(bar, 0, WAIT_NS);
 }
 
-// 32 lanes x 16 consecutive 32-bit TMEM columns (lane = thread of the warp)
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-
 // Per-head reduction over the warp's 32 rows of 16 values (head h in v[h]) by transposing exchanges: over lane
 // bits 4, 3, 2, 1 each lane keeps the half of its values its bit selects, then lane bit 0 on one value.  Lane l
 // ends with head l >> 1 (both lanes of a pair hold it).
