@@ -58,15 +58,15 @@ struct IxArgs {
 };
 
 // NP partial sums of w[c] ReLU(D[c]) over the 64 columns of an epilogue thread, partial j over columns
-// [64 j / NP, 64 (j + 1) / NP); r holds columns [16 q, 16 q + 16).  The 64 weights stay in registers for the whole
+// [64 j / NP, 64 (j + 1) / NP); r holds columns [PW q, PW q + PW).  The 64 weights stay in registers for the whole
 // kernel: re-reading them from shared memory every tile (a broadcast load still returns 4 bytes per lane through
 // the shared-memory crossbar) costs about as many shared-memory cycles as the tensor cores' operand reads.
-template <int NP>
-__device__ __forceinline__ void relu_weighted_quarter(const float (&w)[64], const uint32_t (&r)[16], int q,
-                                                      float (&p)[NP]) {
+template <int NP, int PW>
+__device__ __forceinline__ void relu_weighted_piece(const float (&w)[64], const uint32_t (&r)[PW], int q,
+                                                    float (&p)[NP]) {
   #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const int col = 16 * q + c;
+  for (int c = 0; c < PW; ++c) {
+    const int col = PW * q + c;
     p[col / (64 / NP)] = fmaf(w[col], fmaxf(__uint_as_float(r[c]), 0.f), p[col / (64 / NP)]);
   }
 }
@@ -279,6 +279,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     const int nq = 64 / a.H_I;  // queries in this warp's 64 columns (1 or 2)
     const int64_t qpb = (G > 0 && b0 + (col0 >> 6) < a.B) ? a.q_pos[b0 + (col0 >> 6)] : -1;  // grouped: one query
     constexpr int NP = G > 2 ? G : 2;  // partial sums per key: one per group, or one per 32 columns
+    constexpr int PW = 16;               // TMEM columns per load
     float wr[64];
     #pragma unroll
     for (int c = 0; c < 64; c += 4) {
@@ -288,8 +289,22 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       wr[c + 2] = v.z;
       wr[c + 3] = v.w;
     }
+    // FP8: the key scales two tiles ahead (a scale read in the tile that uses it would put a global load's latency
+    // in every tile); the queries' positions once
+    const int s_lane = t_begin * IX_TILE_M + quarter * 32 + lane;
+    auto key_scale = [&](int t) -> float {
+      const int sk = s_lane + t * IX_TILE_M;
+      return (FP8 && t < n_my && sk < a.L) ? a.k_scale[sk] : 1.f;
+    };
+    float ks0 = key_scale(0), ks1 = key_scale(1);
+    const int bA = b0 + col0 / a.H_I, bB = bA + 1;
+    const int64_t posA = (a.q_pos && bA < a.B) ? a.q_pos[bA] : INT64_MAX;
+    const int64_t posB = (a.q_pos && nq == 2 && bB < a.B) ? a.q_pos[bB] : INT64_MAX;
     for (int i = 0; i < n_my; ++i) {
       const int buf = i & 1;
+      const float ks = ks0;
+      ks0 = ks1;
+      ks1 = key_scale(i + 2);
       // decided warp-wide: the TMEM loads below are warp-collective
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (i >> 1) & 1))) {
         atomicExch(&g_index_tc_timeout, 1);
@@ -298,22 +313,22 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       }
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * IX_CHUNK_N + col0;
-      // 16 columns at a time (64 weights + 16 columns live; 18 warps leave 96 registers a thread), four or G
+      // PW columns at a time (64 weights + PW columns live; 18 warps leave 96 registers a thread), two or G
       // partial sums
       float p[NP];
       #pragma unroll
       for (int j = 0; j < NP; ++j) p[j] = 0.f;
       #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t r[16];
-        tmem_ld16(taddr + 16 * q, r);
+      for (int q = 0; q < 64 / PW; ++q) {
+        uint32_t r[PW];
+        tmem_ld16(taddr + PW * q, r);
         tmem_ld_wait();
-        if (q == 3) {
+        if (q == 64 / PW - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[buf]);  // the accumulator columns are in registers now
         }
-        relu_weighted_quarter<NP>(wr, r, q, p);
+        relu_weighted_piece<NP, PW>(wr, r, q, p);
       }
       const int s = (t_begin + i) * IX_TILE_M + quarter * 32 + lane;
       if constexpr (G > 0) {
@@ -328,16 +343,13 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                               gmax + ((i & 3) * 4 + (ew >> 2)) * 8, gcnt + (i & 3) * 4 + (ew >> 2));
         continue;
       }
-      const float ks = (FP8 && s < a.L) ? a.k_scale[s] : 1.f;
       const float acc0 = p[0], acc1 = p[1];
       if (s < a.L) {
         if (nq == 1) {
-          const int b = b0 + col0 / a.H_I;
-          if (b < a.B) a.scores[static_cast<int64_t>(b) * a.ld + s] = (a.q_pos && s > a.q_pos[b]) ? -INFINITY : (acc0 + acc1) * ks;
+          if (bA < a.B) a.scores[static_cast<int64_t>(bA) * a.ld + s] = s > posA ? -INFINITY : (acc0 + acc1) * ks;
         } else {
-          const int bA = b0 + col0 / a.H_I, bB = bA + 1;
-          if (bA < a.B) a.scores[static_cast<int64_t>(bA) * a.ld + s] = (a.q_pos && s > a.q_pos[bA]) ? -INFINITY : acc0 * ks;
-          if (bB < a.B) a.scores[static_cast<int64_t>(bB) * a.ld + s] = (a.q_pos && s > a.q_pos[bB]) ? -INFINITY : acc1 * ks;
+          if (bA < a.B) a.scores[static_cast<int64_t>(bA) * a.ld + s] = s > posA ? -INFINITY : acc0 * ks;
+          if (bB < a.B) a.scores[static_cast<int64_t>(bB) * a.ld + s] = s > posB ? -INFINITY : acc1 * ks;
         }
       }
     }
