@@ -7,12 +7,13 @@
 // Design (B200): one thread-block cluster of C CTAs (C <= 16) per score row, two CTAs per SM.  Each CTA
 // owns a contiguous chunk of the row and, when it fits (<= 16384 scores), keeps it in shared memory (one
 // bulk asynchronous copy), so HBM is read once.  The threshold is found by refining the order-preserving
-// uint32 key: level 0 histograms 256 bins over the candidates' key range, each further level one 8-bit
+// uint32 key: level 0 histograms 256 bins over a key range that every CTA takes from the same fixed sample of
+// the row (keys outside it are clamped into the end bins), each further level one 8-bit
 // digit inside the boundary bin.  Per-CTA histograms are all-gathered through distributed shared memory
 // (DSMEM), so every CTA finds the boundary bin itself (one cluster barrier per level).  When the
 // boundary bin holds <= 1024 elements, its keys are all-gathered too and every CTA finishes the
 // refinement locally; the tie shares and every CTA's output offset follow from the gathered counts, so
-// the ordered write pass needs no further communication.  Common case: three cluster barriers.  Each
+// the ordered write pass needs no further communication.  Common case: two cluster barriers.  Each
 // CTA runs this code once, so the passes are short rolled loops (a small instruction footprint) rather
 // than unrolled code.  All synchronisation is the hardware cluster barrier: no spin-waits on memory, no
 // global atomics, no scratch memory.
@@ -61,7 +62,6 @@ struct TopkSmem {
   uint32_t tot[TK_BINS];   // cluster-wide histogram of a level
   uint32_t cand[TK_CAP];   // boundary-bin keys; CTA c's at [segoff[c], segoff[c] + segcnt[c])
   uint8_t cand_w[TK_CAP];  // warp of each of this CTA's own boundary-bin elements (local slot order)
-  uint32_t kmin[TK_MAXC], kmax[TK_MAXC];
   uint32_t above[TK_MAXC];  // CTA c's elements above the boundary bins of all levels
   uint32_t segoff[TK_MAXC], segcnt[TK_MAXC];
   uint32_t gtb[TK_MAXC], eqb[TK_MAXC];  // CTA c's boundary elements with key > T / key == T
@@ -298,6 +298,9 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     cluster_wait();
     return;
   }
+  // this thread's sample of the row for level 0's key range (below), loaded before the chunk is staged
+  const uint32_t ksample =
+      valid_key(__ldg(a.scores + static_cast<int64_t>(b) * a.ld + rs.clo + static_cast<int64_t>(tid) * rs.ncand / TK_THREADS));
   if (tid < TK_MAXC) sm.above[tid] = 0;
   if (tid < TK_WARPS) {
     sm.wgt[tid] = 0;
@@ -352,78 +355,36 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     }
   }
 
-  // ---- order keys (in place, when cached) and the finite key range of the candidates ----
+  // ---- level 0's key range, from a fixed sample of the candidates that every CTA of the cluster reads alike:
+  // all CTAs use the same bins without exchanging anything, and keys outside the sampled range are clamped into
+  // the end bins (the counts stay exact; only the bins' widths depend on the sample) ----
+  uint32_t klo = 0xFFFFFFFFu, khi = 0u;
   {
-    uint32_t lo1 = 0xFFFFFFFFu, hi = 0u;  // lo1 = min(key) - 1 over valid keys (invalid: 0 - 1 = max)
-    if (a.cached) {
-      for (int g = gw0 + lane; g < gw1; g += 32) {
-        const uint4 k = ch.from_scores(g, g < nvec ? cache[g] : ch.gload(g));
-        reinterpret_cast<uint4*>(cache)[g] = k;
-        lo1 = min(min(lo1, k.x - 1u), min(k.y - 1u, min(k.z - 1u, k.w - 1u)));
-        hi = max(max(hi, k.x), max(k.y, max(k.z, k.w)));
-      }
-    } else {
-      for_groups<STREAMED>(ch, gw0, gw1, lane, [&](const uint4 k) {
-        lo1 = min(min(lo1, k.x - 1u), min(k.y - 1u, min(k.z - 1u, k.w - 1u)));
-        hi = max(max(hi, k.x), max(k.y, max(k.z, k.w)));
-      });
+    // sample tid is candidate clo + tid ncand / TK_THREADS (ncand > K >= 1 here)
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    if (key_finite(ksample)) {
+      lo = ksample;
+      hi = ksample;
     }
-    if (a.cached) ch.keys = reinterpret_cast<const uint4*>(cache);  // each thread reads back only its own groups
-    uint32_t lo = lo1 + 1u;  // 0 when this thread saw no valid key
     #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      lo1 = min(lo1, __shfl_xor_sync(0xffffffffu, lo1, o));
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
       hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-    }
-    lo = lo1 + 1u;
-    if (hi != 0u && (!key_finite(lo) || !key_finite(hi))) {
-      // non-finite scores in this warp's range (rare): redo the warp's range over finite keys only
-      lo = 0xFFFFFFFFu;
-      hi = 0u;
-      for (int g = gw0 + lane; g < gw1; g += 32) {
-        const uint4 k4 = ch.load(g);
-        const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
-        #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (key_finite(k[e])) {
-            lo = min(lo, k[e]);
-            hi = max(hi, k[e]);
-          }
-        }
-      }
-      #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-      }
-    } else if (hi == 0u) {
-      lo = 0xFFFFFFFFu;  // no valid key in this warp's range
     }
     if (lane == 0) {
       sm.wa[warp] = lo;
       sm.wb[warp] = hi;
     }
     __syncthreads();
-    if (warp == 0) {
-      lo = lane < TK_WARPS ? sm.wa[lane] : 0xFFFFFFFFu;
-      hi = lane < TK_WARPS ? sm.wb[lane] : 0u;
-      #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-      }
+    lo = lane < TK_WARPS ? sm.wa[lane] : 0xFFFFFFFFu;
+    hi = lane < TK_WARPS ? sm.wb[lane] : 0u;
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
-    cluster_wait();  // every CTA of the cluster has started: DSMEM is addressable
-    if (warp == 0 && lane < C) {
-      *cluster.map_shared_rank(&sm.kmin[r], lane) = lo;
-      *cluster.map_shared_rank(&sm.kmax[r], lane) = hi;
-    }
-    cluster.sync();
-  }
-  uint32_t klo = 0xFFFFFFFFu, khi = 0u;
-  for (int c = 0; c < C; ++c) {
-    klo = min(klo, sm.kmin[c]);
-    khi = max(khi, sm.kmax[c]);
+    klo = lo;
+    khi = hi;
   }
   if (klo > khi) klo = khi = 0x80000000u;  // no finite candidate: every key is clamped into one bin
 
@@ -439,7 +400,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     uint32_t* hl = hall + (level & 1) * C * TK_BINS;
     if (tid < TK_BINS) sm.h[tid] = 0;
     __syncthreads();
-    for_groups<STREAMED>(ch, gw0, gw1, lane, [&](const uint4 k4) {
+    auto count_keys = [&](const uint4 k4) {
       const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
       #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -449,8 +410,20 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
           atomicAdd(&sm.h[(k[e] - klo) >> shift], 1u);
         }
       }
-    });
+    };
+    if (level == 0 && a.cached) {
+      // the scores of my groups become order keys in place (each thread reads back only its own groups)
+      for (int g = gw0 + lane; g < gw1; g += 32) {
+        const uint4 k = ch.from_scores(g, g < nvec ? cache[g] : ch.gload(g));
+        reinterpret_cast<uint4*>(cache)[g] = k;
+        count_keys(k);
+      }
+      ch.keys = reinterpret_cast<const uint4*>(cache);
+    } else {
+      for_groups<STREAMED>(ch, gw0, gw1, lane, count_keys);
+    }
     __syncthreads();
+    if (level == 0) cluster_wait();  // every CTA of the cluster has started: DSMEM is addressable
     for (int i = tid; i < TK_BINS * C; i += TK_THREADS) {
       const int c = i / TK_BINS, bin = i - c * TK_BINS;
       *cluster.map_shared_rank(hl + r * TK_BINS + bin, c) = sm.h[bin];
