@@ -129,6 +129,29 @@ def test_topk_exact_heavy_ties(L):
         _topk_case(scores, [L - 1] * B, K, sink, window)
 
 
+@pytest.mark.parametrize("L", [131072, 200003, 600000])
+@pytest.mark.parametrize("K", [64, 2048])
+def test_topk_exact_stride_blind_spots(L, K):
+    """Rows whose values at a regular stride (L / 1024 apart, the spacing of a fixed sample of the row) look nothing
+    like the rest: the largest scores all off that stride; that stride holding a single value; holding only -inf;
+    holding the largest values.  The kernel's level-0 bins come from such a sample, so its selection must not
+    depend on the sample being representative."""
+    rng = np.random.default_rng(L + K)
+    on = (np.arange(1024, dtype=np.int64) * L) // 1024  # the stride positions
+    off = np.setdiff1d(np.arange(L), on)
+    scores = np.empty((4, L))
+    scores[0] = rng.standard_normal(L)
+    top = rng.choice(off, K + 100, replace=False)
+    scores[0, top] = 10.0 ** rng.uniform(3, 6, top.size)  # the top K and more, none on the stride
+    scores[1] = rng.standard_normal(L) * 30
+    scores[1, on] = 5.0
+    scores[2] = rng.standard_normal(L)
+    scores[2, on] = -np.inf
+    scores[3] = rng.standard_normal(L)
+    scores[3, on] = 1e4 + rng.standard_normal(on.size)
+    _topk_case(scores, [L - 1] * 4, K, 0, 0)
+
+
 def test_topk_many_rows_prefill_like():
     rng = np.random.default_rng(5)
     B, L = 300, 20000
