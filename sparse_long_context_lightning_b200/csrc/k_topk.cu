@@ -68,7 +68,7 @@ struct TopkSmem {
   uint32_t wa[TK_WARPS], wb[TK_WARPS];
   uint32_t wgt[TK_WARPS], weq[TK_WARPS];  // this CTA's elements with key > T / key == T, per warp
   uint32_t ccount;
-  uint32_t sel_bin, sel_above, sel_count;
+  uint32_t sel_bin, sel_above, sel_count, sel_total;
   uint64_t load_bar[TK_PIECES];  // one per piece of the chunk's bulk copy
 };
 
@@ -218,7 +218,8 @@ __device__ __forceinline__ void for_groups(const Chunk& ch, int gw0, int gw1, in
 }
 
 // Boundary bin of hist[] (bins ascend with the key): the bin holding the need-th largest element.
-// Warp 0 only; lane l scans bins [8l, 8l + 8).  Writes sel_bin / sel_above / sel_count.
+// Warp 0 only; lane l scans bins [8l, 8l + 8).  Writes sel_total, and sel_bin / sel_above / sel_count when the
+// bins hold at least `need` elements.
 __device__ __forceinline__ void find_boundary(TopkSmem& sm, const uint32_t* hist, uint32_t need, int lane) {
   const uint4 v0 = reinterpret_cast<const uint4*>(hist)[2 * lane];
   const uint4 v1 = reinterpret_cast<const uint4*>(hist)[2 * lane + 1];
@@ -232,6 +233,7 @@ __device__ __forceinline__ void find_boundary(TopkSmem& sm, const uint32_t* hist
     const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
     if (lane + o < 32) suf += v;
   }
+  if (lane == 0) sm.sel_total = suf;  // every bin
   uint32_t acc = suf - lsum;  // elements in bins above this lane's range
   if (acc < need && acc + lsum >= need) {
     for (int j = 7; j >= 0; --j) {
@@ -358,7 +360,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
   // ---- level 0's key range, from a fixed sample of the candidates that every CTA of the cluster reads alike:
   // all CTAs use the same bins without exchanging anything, and keys outside the sampled range are clamped into
   // the end bins (the counts stay exact; only the bins' widths depend on the sample) ----
-  uint32_t klo = 0xFFFFFFFFu, khi = 0u;
+  uint32_t klo = 0xFFFFFFFFu, khi = 0u, tau = 0u;
   {
     // sample tid is candidate clo + tid ncand / TK_THREADS (ncand > K >= 1 here)
     uint32_t lo = 0xFFFFFFFFu, hi = 0u;
@@ -378,15 +380,20 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     __syncthreads();
     lo = lane < TK_WARPS ? sm.wa[lane] : 0xFFFFFFFFu;
     hi = lane < TK_WARPS ? sm.wb[lane] : 0u;
+    // the smallest of the warps' sample maxima (each the largest of 32 samples: about the 97th percentile, so
+    // their minimum sits near the 90th): level 0 counts only the keys at or above it
+    uint32_t cut = (lane < TK_WARPS && hi != 0u) ? hi : 0xFFFFFFFFu;
     #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
       hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      cut = min(cut, __shfl_xor_sync(0xffffffffu, cut, o));
     }
     klo = lo;
     khi = hi;
+    tau = cut;
   }
-  if (klo > khi) klo = khi = 0x80000000u;  // no finite candidate: every key is clamped into one bin
+  if (klo > khi) klo = khi = tau = 0x80000000u;  // no finite sample: every key is clamped into one bin
 
   // ---- cluster-level refinement: each level histograms one 8-bit digit of (key - klo) in [klo, khi] ----
   // Level 0 covers every valid key: keys outside the finite range are clamped to it, so the first bin's
@@ -394,6 +401,12 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
   uint32_t need = static_cast<uint32_t>(K);
   uint32_t T = 0, need_eq = 0;
   bool gathered = false;
+  // mode 0 (the first level): bins over [tau, khi], keys below tau not counted, keys above khi in the top bin;
+  // mode 1 (only when fewer than `need` keys reach tau): bins over [klo, khi] with keys outside clamped into the end
+  // bins, on the next level's buffers; mode 2: bins over the previous boundary bin, exactly
+  const uint32_t klo_all = klo;
+  int mode = 0;
+  klo = tau;
   for (int level = 0; level < 8; ++level) {
     const int shift = level_shift(klo, khi);
     const uint32_t bmax = (khi - klo) >> shift;  // last occupied bin, <= 255
@@ -404,7 +417,9 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
       const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
       #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        if (level == 0) {
+        if (mode == 0) {
+          if (k[e] >= klo) atomicAdd(&sm.h[(min(k[e], khi) - klo) >> shift], 1u);
+        } else if (mode == 1) {
           if (k[e]) atomicAdd(&sm.h[(min(max(k[e], klo), khi) - klo) >> shift], 1u);
         } else if (k[e] >= klo && k[e] <= khi) {
           atomicAdd(&sm.h[(k[e] - klo) >> shift], 1u);
@@ -437,6 +452,11 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     __syncthreads();
     if (warp == 0) find_boundary(sm, sm.tot, need, lane);
     __syncthreads();
+    if (mode == 0 && sm.sel_total < need) {  // fewer than `need` keys reach tau (row-uniform): all keys, clamped
+      mode = 1;
+      klo = klo_all;
+      continue;
+    }
     const uint32_t bstar = sm.sel_bin, bcount = sm.sel_count;
     need -= sm.sel_above;
     if (warp < C) {  // CTA `warp`'s elements above the boundary bin
@@ -450,8 +470,9 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     }
     uint32_t nlo, nhi;
     bin_range(klo, khi, shift, bstar, nlo, nhi);
-    if (level == 0 && bstar == 0) nlo = 1u;  // valid keys are >= 1
-    if (level == 0 && bstar == bmax) nhi = 0xFFFFFFFFu;
+    if (mode == 1 && bstar == 0) nlo = 1u;  // valid keys are >= 1
+    if (mode != 2 && bstar == bmax) nhi = 0xFFFFFFFFu;
+    mode = 2;
     const bool tie = nlo == nhi;  // the boundary bin is one key value
     const bool gather = !tie && bcount <= static_cast<uint32_t>(TK_CAP);
     if (!tie && !gather) {
