@@ -635,11 +635,6 @@ size_t sparse_attn_ws_bytes(int64_t B, int64_t idx_ld, int H) {
   return o + align_up(static_cast<size_t>(B) * S * AT_H * 2 * 4, 256);
 }
 
-int attn_launches_per_call(int64_t B, int64_t idx_ld, int H) {
-  if (padded_heads(H)) return 2 + attn_launches_per_call(B, idx_ld, AT_H);
-  return (H == AT_H && attn_slots(B, idx_ld) > 1) ? 2 : 1;
-}
-
 
 int launch_sparse_attn(const void* q, const void* kv, int64_t L, const int32_t* idx, int64_t idx_ld,
                        const int32_t* count, int64_t B, int H, float scale, void* out, float* lse, void* ws,

@@ -766,10 +766,4 @@ int launch_topk_mode(const float* scores, int64_t ld, int64_t B, int64_t L, int 
   return LSA_OK;
 }
 
-int launch_topk(const float* scores, int64_t ld, int64_t B, int64_t L, int K, int sink, int window,
-                const int64_t* q_pos, int64_t, int32_t* idx, int64_t idx_ld, int32_t* count, int64_t kmax,
-                cudaStream_t s) {
-  return launch_topk_mode(scores, ld, B, L, K, sink, window, q_pos, MODE_TOKEN, 1, idx, idx_ld, count, kmax, s);
-}
-
 }  // namespace lsa

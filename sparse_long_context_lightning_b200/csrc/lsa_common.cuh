@@ -155,9 +155,6 @@ int launch_page_sum(const float* sub, int64_t sub_ld, int64_t nsub, int P, int B
 int launch_page_expand(const int32_t* kept, int64_t kept_ld, const int32_t* kcnt, int P, int Bsub, int sink,
                        int window, const int64_t* q_pos, int64_t B, int32_t* cand, int64_t cand_ld,
                        int32_t* ccount, cudaStream_t s);
-int launch_topk(const float* scores, int64_t ld, int64_t B, int64_t L, int K, int sink, int window,
-                const int64_t* q_pos, int64_t rank_limit_div, int32_t* idx, int64_t idx_ld, int32_t* count,
-                int64_t kmax, cudaStream_t s);
 int launch_pool_keys(const void* k, int dtype, const float* k_scale, int64_t L, int d_I,
                      const int32_t* members, int bsz, int64_t NB, float* centroids, cudaStream_t s);
 int launch_bucket_expand(const int32_t* kept, int64_t kept_ld, const int32_t* kept_count,
@@ -194,7 +191,6 @@ int launch_msa_expand(const int32_t* kept, int64_t kept_ld, const int32_t* kcnt,
                       cudaStream_t s);
 int launch_shift_qpos(const int64_t* q_pos, int64_t B, int G, int64_t delta, int64_t* out, cudaStream_t s);
 size_t sparse_attn_ws_bytes(int64_t B, int64_t kmax, int H);
-int attn_launches_per_call(int64_t B, int64_t idx_ld, int H);
 int take_attn2_flags(int* check);
 int take_msa_attn_flags(int* check);
 int launch_msa_attn_rows(const void* q, const void* kv, int64_t L, const int32_t* idx, const uint8_t* gmask, int64_t ld,
