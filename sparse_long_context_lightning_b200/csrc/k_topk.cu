@@ -13,7 +13,8 @@
 // (DSMEM), so every CTA finds the boundary bin itself (one cluster barrier per level).  When the
 // boundary bin holds <= 1024 elements, its keys are all-gathered too and every CTA finishes the
 // refinement locally; the tie shares and every CTA's output offset follow from the gathered counts, so
-// the ordered write pass needs no further communication.  Common case: two cluster barriers.  Each
+// the ordered write needs no further communication (it walks per-warp lists of the keys at or above the final
+// boundary bin, built by the gather pass, when they fit).  Common case: two cluster barriers.  Each
 // CTA runs this code once, so the passes are short rolled loops (a small instruction footprint) rather
 // than unrolled code.  All synchronisation is the hardware cluster barrier: no spin-waits on memory, no
 // global atomics, no scratch memory.
@@ -34,6 +35,7 @@ constexpr int TK_MAXC = 16;    // cluster size limit (non-portable above 8)
 constexpr int TK_CACHE = 24576;  // scores per CTA kept in shared memory (96 KB)
 constexpr int TK_PIECES = 4;     // the chunk arrives in this many bulk copies; each warp waits for its own
 constexpr int TK_UNROLL = 4;     // groups per lane whose loads are in flight together in a pass
+constexpr int TK_WLIST = 64;     // per-warp list of the final pass's keys at or above the boundary bin (cached rows)
 
 enum { MODE_TOKEN = 0, MODE_ALL = 1, MODE_BLOCKS = 2 };
 
@@ -62,6 +64,9 @@ struct TopkSmem {
   uint32_t tot[TK_BINS];   // cluster-wide histogram of a level
   uint32_t cand[TK_CAP];   // boundary-bin keys; CTA c's at [segoff[c], segoff[c] + segcnt[c])
   uint8_t cand_w[TK_CAP];  // warp of each of this CTA's own boundary-bin elements (local slot order)
+  uint32_t wl_key[TK_WARPS][TK_WLIST];  // cached rows: each warp's keys >= the final boundary bin's low end and
+  int32_t wl_pos[TK_WARPS][TK_WLIST];   // their positions, in ascending position order
+  uint32_t wl_over;                     // some warp's list overflowed: the ordered write walks the whole chunk
   uint32_t above[TK_MAXC];  // CTA c's elements above the boundary bins of all levels
   uint32_t segoff[TK_MAXC], segcnt[TK_MAXC];
   uint32_t gtb[TK_MAXC], eqb[TK_MAXC];  // CTA c's boundary elements with key > T / key == T
@@ -304,6 +309,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
   const uint32_t ksample =
       valid_key(__ldg(a.scores + static_cast<int64_t>(b) * a.ld + rs.clo + static_cast<int64_t>(tid) * rs.ncand / TK_THREADS));
   if (tid < TK_MAXC) sm.above[tid] = 0;
+  if (tid == 0) sm.wl_over = 0;
   if (tid < TK_WARPS) {
     sm.wgt[tid] = 0;
     sm.weq[tid] = 0;
@@ -494,7 +500,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     }
     const uint32_t off = gather ? sm.segoff[r] : 0u;
     uint32_t nab = 0, nin = 0;
-    for_groups<STREAMED>(ch, gw0, gw1, lane, [&](const uint4 k4) {
+    auto final_keys = [&](const uint4 k4) {
       const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
       #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -509,7 +515,39 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
           }
         }
       }
-    });
+    };
+    if (!STREAMED) {
+      // warp-uniform steps of 32 groups; the keys >= nlo (every key the write can select: T >= nlo) also go to
+      // the warp's list, ordered by a ballot prefix, so that the ordered write needs only the lists
+      const uint32_t lt = lanemask_lt();
+      uint32_t wn = 0;
+      for (int g0 = gw0; g0 < gw1; g0 += 32) {
+        const int g = g0 + lane;
+        const uint4 k4 = g < gw1 ? ch.keys[g] : make_uint4(0u, 0u, 0u, 0u);
+        final_keys(k4);
+        const uint32_t k[4] = {k4.x, k4.y, k4.z, k4.w};
+        uint32_t c = 0;
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) c += k[e] >= nlo;  // nlo >= 1: invalid slots (key 0) never count
+        uint32_t tot;
+        uint32_t o = wn + ballot_prefix(c, lt, tot);
+        if (wn + tot <= static_cast<uint32_t>(TK_WLIST)) {
+          #pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (k[e] >= nlo) {
+              sm.wl_key[warp][o] = k[e];
+              sm.wl_pos[warp][o] = c0 + 4 * g + e;
+              ++o;
+            }
+          }
+        }
+        wn += tot;
+      }
+      if (wn > static_cast<uint32_t>(TK_WLIST) && lane == 0) sm.wl_over = 1u;
+      if (lane == 0) sm.wa[warp] = wn;  // this warp's list length (sm.wa is free after the sampled range)
+    } else {
+      for_groups<STREAMED>(ch, gw0, gw1, lane, final_keys);
+    }
     nab = warp_sum_u32(nab);
     nin = warp_sum_u32(nin);
     if (lane == 0) {
@@ -656,7 +694,23 @@ __global__ void __launch_bounds__(TK_THREADS, 1) k_topk_cluster(TopkArgs a) {
     gt_run += gtot;
     eq_run += etot;
   };
-  if (!STREAMED) {
+  if (!STREAMED && sm.wl_over == 0u) {
+    // the warp's list holds every key it can select, in position order: one key per lane per step
+    const int n = static_cast<int>(sm.wa[warp]);
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t k = i < n ? sm.wl_key[warp][i] : 0u;
+      const bool gt = k > T, eq = k == T;
+      const uint32_t bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+      const uint32_t gb = gt_run + __popc(bg & lt), eb = eq_run + __popc(be & lt);
+      if (gt || (eq && eb < take)) {
+        const uint32_t o = base + gb + min(eb, take);
+        if (o < lim) rs.out[o] = sm.wl_pos[warp][i];  // bounded even if the counts were inconsistent
+      }
+      gt_run += __popc(bg);
+      eq_run += __popc(be);
+    }
+  } else if (!STREAMED) {
     for (int g0 = gw0; g0 < gw1; g0 += 32) {
       const int g = g0 + lane;
       step(g, g < gw1 ? ch.keys[g] : make_uint4(0u, 0u, 0u, 0u));
