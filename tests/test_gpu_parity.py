@@ -152,6 +152,22 @@ def test_topk_exact_stride_blind_spots(L, K):
     _topk_case(scores, [L - 1] * 4, K, 0, 0)
 
 
+@pytest.mark.parametrize("K", [300, 2048])
+def test_topk_exact_clustered_top(K):
+    """The largest scores packed into contiguous runs (one run of K, runs of 70 every 5000 positions, runs of 60):
+    a stretch of the row then holds more selected keys than a warp's list of them can hold, and the write must
+    fall back to walking the chunk; the run lengths straddle that list size."""
+    L = 131072
+    rng = np.random.default_rng(K)
+    scores = rng.standard_normal((4, L))
+    scores[0, 1000:1000 + K] = 100.0 + rng.standard_normal(K)
+    for start in range(7, L - 70, 5000):
+        scores[1, start:start + 70] = 50.0 + rng.standard_normal(70)
+        scores[2, start:start + 60] = 50.0 + rng.standard_normal(60)
+    scores[3] = np.repeat(rng.standard_normal(L // 512), 512)  # runs of 512 equal values
+    _topk_case(scores, [L - 1] * 4, K, 4, 128)
+
+
 def test_topk_many_rows_prefill_like():
     rng = np.random.default_rng(5)
     B, L = 300, 20000
