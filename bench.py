@@ -839,6 +839,11 @@ def run_gpu(args, rank, world, local_rank):
         stages[name] = st
     dom = max(stages, key=lambda k: stages[k]["ms"])
     kname, _ = STAGE_KERNEL[dom]
+    tkey = kname  # the committed DRAM traffic of this kernel in this mode, if any
+    if step.fp8 and dom == "index":
+        tkey = "k_index_score_tc<fp8>"
+    elif step.fp8 and dom == "topk":  # the FP8 mode's selection stage is four launches
+        kname, tkey = "k_topk_cluster (top-2K) + k_rescore_tc + k_refine_assemble + k_topk_cluster", None
     if dom == "index":
         roof = {"bound": "tensor", "achieved": stages[dom]["achieved_tflops"], "peak": tensor_peak, "unit": "TFLOP/s",
                 "frac": stages[dom]["tensor_frac"]}
@@ -846,7 +851,7 @@ def run_gpu(args, rank, world, local_rank):
         roof = {"bound": "hbm", "achieved": stages[dom]["achieved_gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": stages[dom]["hbm_frac"]}
     roof.update({"kernel": kname, "peak_source": fp8_peak()[2] if (dom == "index" and step.fp8) else pk_src,
-                 "traffic": committed_traffic(kname)})
+                 "traffic": committed_traffic(tkey) if tkey else None})
     qps = job_rate(wl.B, world, step_ms)
     n_launch = sum(launches.values()) * args.steps
     return {
